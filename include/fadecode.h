@@ -1,0 +1,218 @@
+/*
+ * fadecode.h -- C ABI of the split-KV GQA decode-attention library for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (one new query token per request, attending over that
+ * request's KV cache):
+ *
+ *   for request b, query head h, kv head g = h / (qo_heads / kv_heads),
+ *   visible keys J_b = [max(0, L_b - window), L_b)   (all keys if window <= 0)
+ *     s_j   = sm_scale * <q[b,h,:], K_b[j,g,:]>
+ *     out   = sum_j softmax(s)_j * V_b[j,g,:]          (bf16, round-to-nearest)
+ *     lse   = ln sum_j exp(s_j)                         (fp32, natural log)
+ *
+ * Sources: "Forcing Flash Attention onto a TPU" (LLM internals part 5),
+ * sections "Standard causal attention" (the definition) and "Flash Attention
+ * in JAX" (tiles with a running max, running sum and accumulator);
+ * "FlashInfer x JAX via jax-tvm-ffi", section on single_decode (GQA decode of
+ * one request over its KV cache, a caller-provided scratch buffer, sentinel
+ * values for optional arguments) and section "Applying it to Gemma 3"
+ * (local sliding-window layers); "Beyond the Memory Wall", section
+ * "2. FlashInfer" (paged KV, FP8 KV); "FlashDecoding++" explainer, sections
+ * "Asynchronous softmax and unified max value" (partial softmax per KV tile,
+ * merged afterwards) and "Hardware-aware heuristic dataflow" (the path is
+ * chosen from the shape and the GPU).
+ *
+ * Conventions shared by every entry point:
+ *  - Every buffer is owned by the caller.  The library never allocates or
+ *    frees device memory.  A plan is a small host object owned by the
+ *    caller and released with fa_plan_destroy.
+ *  - Device pointers are plain CUDA device addresses on the current device.
+ *    `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream); work is enqueued on it and the call returns without waiting,
+ *    except where a function says it synchronises.
+ *  - Errors are returned as fa_status; nothing aborts or traps.  Argument
+ *    errors are detected on the host before any work is enqueued.
+ *  - bf16 tensors are raw IEEE bfloat16 bit patterns (uint16); fp8 tensors
+ *    are e4m3 "fn" codes (uint8: bias 7, no infinities).
+ */
+#ifndef FADECODE_H_
+#define FADECODE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,         /* null pointer, bad shape, bad sentinel   */
+  FA_ERR_UNSUPPORTED = 2,         /* valid, but no kernel for this shape    */
+  FA_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes below the plan's need  */
+  FA_ERR_MISALIGNED = 4,          /* a pointer below its required alignment */
+  FA_ERR_CUDA = 5,                /* a CUDA runtime/driver call failed      */
+  FA_ERR_DEVICE_CHECK = 6         /* a kernel recorded a device-side check  */
+} fa_status;
+
+typedef enum { FA_KV_BF16 = 0, FA_KV_FP8_E4M3 = 1 } fa_kv_dtype;
+
+/* Dataflow for the KV-tile math.  SIMT computes q.k with per-lane fp32 FMAs
+ * and warp-shuffle reductions (a GEMV per head); MMA runs the two skinny
+ * products (scores and probabilities times V) on the warp-level tensor-core
+ * instruction with fp32 accumulation, which keeps the instruction count per
+ * KV byte low when several query heads share a kv head.  AUTO lets the
+ * planner choose from the shape (see fa_plan_info). */
+typedef enum { FA_PATH_AUTO = 0, FA_PATH_SIMT = 1, FA_PATH_MMA = 2 } fa_path;
+
+/* Device-side check bits, reported by fa_decode_status. */
+enum {
+  FA_DEVICE_BAD_PAGE = 1u,   /* a page_table entry outside [0, num_pages)     */
+  FA_DEVICE_TIMEOUT = 2u,    /* a pipeline wait exceeded its time limit       */
+  FA_DEVICE_BAD_INDPTR = 4u  /* kv_indptr decreasing or past the K/V extent   */
+};
+
+typedef struct {
+  int32_t batch;      /* requests, >= 1                                       */
+  int32_t qo_heads;   /* query heads per request                              */
+  int32_t kv_heads;   /* kv heads; qo_heads % kv_heads == 0                   */
+  int32_t head_dim;   /* 64, 128 or 256 (fp8: 128 or 256)                     */
+  int32_t kv_dtype;   /* fa_kv_dtype                                          */
+  int32_t paged;      /* 0: contiguous (ragged) rows, 1: paged pool           */
+  int32_t page_size;  /* paged only: tokens per page, a power of two <= 256  */
+  int32_t window;     /* sentinel -1 (or any value <= 0): attend to all keys; */
+                      /* w > 0: attend to the last w keys only               */
+  float sm_scale;     /* multiplies q.k before the softmax; must be finite   */
+  int32_t path;       /* fa_path                                             */
+  int32_t num_ctas;   /* 0: planner's choice.  n > 0 forces n thread blocks, */
+                      /* i.e. the KV split granularity (used to test that    */
+                      /* split-then-merge equals the unsplit result)         */
+} fa_decode_desc;
+
+typedef struct fa_plan fa_plan;
+
+/* What the planner chose (read-only view of a plan). */
+typedef struct {
+  int32_t path;             /* FA_PATH_SIMT or FA_PATH_MMA                    */
+  int32_t num_ctas;         /* thread blocks launched by fa_decode_run        */
+  int32_t tile_tokens;      /* tokens per KV tile moved by one TMA transaction */
+  int32_t stages;           /* depth of the shared-memory tile ring           */
+  int32_t total_tiles;      /* KV tiles over all (request, kv head) segments  */
+  int32_t max_partials;     /* partial-state slots reserved in the workspace  */
+  size_t workspace_bytes;   /* minimum workspace size for fa_decode_run       */
+  size_t smem_bytes;        /* dynamic shared memory per thread block         */
+} fa_plan_info_t;
+
+/*
+ * fa_decode_plan -- host only; touches no device memory and enqueues nothing.
+ *
+ * Decides the split of the KV sequence into tiles and of the tiles over
+ * thread blocks ("FlashDecoding++", section "Hardware-aware heuristic
+ * dataflow": the dataflow is chosen from batch, lengths and the GPU).
+ * Every (request, kv head) is a segment of KV tiles; the segments are laid
+ * end to end and cut into num_ctas equal runs, so every SM streams the same
+ * number of bytes whatever the length mix.  A segment cut into several runs
+ * yields partial softmax states that fa_decode_run merges exactly.
+ *
+ *  desc            shapes and options (copied into the plan).
+ *  kv_indptr_host  int32[batch + 1], host memory: cumulative token counts;
+ *                  kv_indptr_host[0] == 0, non-decreasing.  Only used to size
+ *                  the split; fa_decode_run reads the device copy.
+ *  num_sms         SM count of the target device (0: query the current
+ *                  device; on a host without a GPU pass it explicitly).
+ *  plan            receives the new plan (caller frees: fa_plan_destroy).
+ *  workspace_bytes receives the minimum workspace size.
+ * Errors: FA_ERR_INVALID_ARG (null pointer, non-positive shape, qo_heads not
+ * a multiple of kv_heads, bad indptr, non-finite sm_scale, bad page_size),
+ * FA_ERR_UNSUPPORTED (head_dim / group / dtype / path combination without a
+ * kernel), FA_ERR_CUDA (num_sms == 0 and no device could be queried).
+ */
+fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* kv_indptr_host,
+                         int32_t num_sms, fa_plan** plan, size_t* workspace_bytes);
+
+/* Fills *info from a plan.  FA_ERR_INVALID_ARG on null pointers. */
+fa_status fa_plan_get_info(const fa_plan* plan, fa_plan_info_t* info);
+
+/* Releases a plan (NULL is a no-op). */
+void fa_plan_destroy(fa_plan* plan);
+
+/*
+ * fa_decode_run -- enqueue one decode-attention pass on `stream`.
+ *
+ * Layouts (row-major, all device memory):
+ *  q           bf16 [batch, qo_heads, head_dim], 16-byte aligned.
+ *  k, v        contiguous: [kv_rows, kv_heads, head_dim]; request b owns rows
+ *              [kv_indptr[b], kv_indptr[b+1]) (batch 1: rows 0..kv_len-1).
+ *              paged: pools [kv_rows, page_size, kv_heads, head_dim] where
+ *              kv_rows is the number of pages.  Element type per desc
+ *              (bf16 or e4m3), 16-byte aligned.
+ *  kv_rows     contiguous: number of rows of k and v; paged: number of pages
+ *              in each pool.  Reads never leave [0, kv_rows).
+ *  page_table  paged only (else NULL): int32 [batch, page_table_stride];
+ *              token t of request b lives in page page_table[b][t/page_size],
+ *              slot t % page_size.  Only entries of pages holding visible
+ *              tokens are read.  An entry outside [0, kv_rows) reads zeros
+ *              and sets FA_DEVICE_BAD_PAGE.
+ *  kv_indptr   int32 [batch + 1], device copy of the plan's indptr.
+ *  k_scale,    fp8 only (else NULL): fp32 [kv_heads]; a stored code c of kv
+ *  v_scale     head g means e4m3(c) * scale[g].
+ *  out         bf16 [batch, qo_heads, head_dim], 16-byte aligned.
+ *  lse         fp32 [batch, qo_heads], natural log; NULL = do not write.
+ *              A request with no visible key gets out = 0, lse = -inf.
+ *  workspace   device scratch of >= the plan's workspace_bytes, 256-byte
+ *              aligned, zero-filled once before its first use (and again
+ *              after FA_ERR_DEVICE_CHECK).  The library leaves its ticket
+ *              counters at zero after every completed call, so one workspace
+ *              serves any number of calls in stream order.  Two calls that
+ *              share a workspace must not overlap on the GPU.
+ * No allocation, no synchronisation, no host<->device copies.  Errors:
+ * FA_ERR_INVALID_ARG, FA_ERR_MISALIGNED, FA_ERR_WORKSPACE_TOO_SMALL,
+ * FA_ERR_CUDA (launch failure).  Device-side checks are reported later by
+ * fa_decode_status.
+ */
+fa_status fa_decode_run(const fa_plan* plan, const void* q, const void* k, const void* v,
+                        int64_t kv_rows, const int32_t* page_table, int32_t page_table_stride,
+                        const int32_t* kv_indptr, const float* k_scale, const float* v_scale,
+                        void* out, float* lse, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/*
+ * fa_decode_status -- SYNCHRONISES `stream`, then reads the device-side check
+ * word of `workspace` into *flags (FA_DEVICE_* bits, 0 = clean) and clears
+ * it.  Returns FA_ERR_DEVICE_CHECK when any bit was set, FA_ERR_CUDA when the
+ * copy failed, else FA_OK.
+ */
+fa_status fa_decode_status(void* workspace, size_t workspace_bytes, uint32_t* flags,
+                           void* stream);
+
+/*
+ * fa_merge_states -- exact merge of n partial attention states per
+ * (row, head) ("FlashDecoding++" explainer, partial softmax per tile combined
+ * afterwards; "Flashlight", section "Method": exp(x - y) = exp(x) / exp(y)
+ * makes the combination exact):
+ *   lse = M + ln sum_c exp(lse_c - M),  M = max_c lse_c
+ *   out = sum_c exp(lse_c - lse) * o_c
+ * States with lse_c = -inf carry no weight; all -inf gives out = 0,
+ * lse = -inf.
+ *  o_parts   fp32 [n, rows, heads, head_dim] (each o_c already normalised)
+ *  lse_parts fp32 [n, rows, heads], natural log
+ *  out       bf16 [rows, heads, head_dim]; lse_out fp32 [rows, heads] or NULL
+ * head_dim must be a multiple of 4 and <= 1024; o_parts, out 16-byte aligned.
+ * Errors: FA_ERR_INVALID_ARG, FA_ERR_MISALIGNED, FA_ERR_CUDA.
+ */
+fa_status fa_merge_states(const float* o_parts, const float* lse_parts, int32_t n, int32_t rows,
+                          int32_t heads, int32_t head_dim, void* out, float* lse_out,
+                          void* stream);
+
+/* Static description of a status code (never NULL). */
+const char* fa_status_string(fa_status status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int32_t fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FADECODE_H_ */
