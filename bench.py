@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Decode-attention benchmark (one JSON line on rank 0).
+
+A step is one whole decode pass over one batch: plan (host split of the KV
+tiles over thread blocks) + the fused split-KV kernel (TMA tile loads,
+scores, online softmax, partial states, in-kernel log-sum-exp merge).
+Default workload: batched paged decode, batch 64, 32 query / 8 kv heads,
+head_dim 128, per-request kv_len uniform in [512, 16384] (seed 4), 16-token
+pages in a random permutation of the pool, bf16 K/V ~ N(0,1).  Its K/V
+(about 2.2 GB) are larger than L2, so no flush is needed between steps.
+
+value       = KV bytes read by all ranks / device time (CUDA events, max over
+              ranks), in GB/s; tokens/s = requests decoded per second.
+e2e         = the same metric through the C ABI with host buffers: every step
+              copies q, K, V, kv_indptr and page_table host->device from pinned
+              memory and reads out and lse back.
+roofline    = algorithmic bytes per launch / mean launch time (events on the
+              launching stream), against the measured HBM copy bandwidth.
+cpu_baseline= the fp64 oracle on the host cores on a bounded sample.
+
+--impl reference times the oracle (this tier's reference arm) on the same
+workload and metric.  Multi-GPU: one process per GPU (torchrun); every rank
+decodes its own copy of the batch (weak scaling, no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import glob
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode attention achieved HBM GB/s (% of B200 peak) and tokens/sec at 1 GPU"
+HEADLINE = "paged_b64_gqa4_L512-16384"
+SWEEP = ["gqa4_d64_L512", "gemma3_1b_global_L8192", "gemma3_1b_local_w512_L8192",
+         "llama2_7b_mha_L1024", "llama2_7b_mha_L4096", "llama2_7b_mha_L16384",
+         "llama2_7b_mha_L32768", "fp8_gqa8_L131072"]
+FALLBACK_HBM_GBS = 6650.0
+
+
+def hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "gqa_decode_attention_split_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on
+    the current kernel sources."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+        e = t.get(workload)
+        if e and e.get("source_hash") == source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_index(local_rank):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return local_rank
+
+
+# ------------------------------------------------------------ device side
+class Runner:
+    """Holds the device copies of one workload and the raw C-ABI arguments so
+    a step is two C calls (plan, run) with no Python allocation."""
+
+    def __init__(self, x, path="auto", device="cuda"):
+        import torch
+        from gqa_decode_attention_split_b200 import binding
+        self.torch = torch
+        self.binding = binding
+        self.lib = binding.load_library()
+        self.x = x
+        bits = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device)
+        fp8 = x.kv_dtype == "fp8_e4m3"
+        self.q = bits(x.q)
+        if fp8:
+            self.k = torch.from_numpy(np.ascontiguousarray(x.k)).to(device)
+            self.v = torch.from_numpy(np.ascontiguousarray(x.v)).to(device)
+            self.ks = torch.from_numpy(x.k_scale).to(device)
+            self.vs = torch.from_numpy(x.v_scale).to(device)
+        else:
+            self.k, self.v = bits(x.k), bits(x.v)
+            self.ks = self.vs = None
+        self.ind = torch.from_numpy(x.kv_indptr).to(device)
+        self.pt = torch.from_numpy(x.page_table).to(device) if x.paged else None
+        self.ind_host = np.ascontiguousarray(x.kv_indptr, dtype=np.int32)
+        self.desc = binding.DecodeDesc(
+            batch=x.batch, qo_heads=x.qo_heads, kv_heads=x.kv_heads, head_dim=x.head_dim,
+            kv_dtype=1 if fp8 else 0, paged=int(x.paged), page_size=int(x.page_size),
+            window=int(x.window), sm_scale=float(x.sm_scale),
+            path={"auto": 0, "simt": 1, "mma": 2}[path], num_ctas=0)
+        p = binding.plan(x.batch, x.qo_heads, x.kv_heads, x.head_dim, x.kv_indptr,
+                         kv_dtype=x.kv_dtype, paged=x.paged, page_size=x.page_size,
+                         window=x.window, sm_scale=x.sm_scale, path=path)
+        self.info = p.info()
+        self.ws = p.new_workspace(device)
+        self.out = torch.empty((x.batch, x.qo_heads, x.head_dim), dtype=torch.bfloat16,
+                               device=device)
+        self.lse = torch.empty((x.batch, x.qo_heads), dtype=torch.float32, device=device)
+        ptr = lambda t: None if t is None else t.data_ptr()
+        self.stream = torch.cuda.current_stream()
+        self.args = (ptr(self.q), ptr(self.k), ptr(self.v), int(self.k.shape[0]), ptr(self.pt),
+                     int(self.pt.stride(0)) if self.pt is not None else 0, ptr(self.ind),
+                     ptr(self.ks), ptr(self.vs), ptr(self.out), ptr(self.lse), ptr(self.ws),
+                     int(self.ws.numel()), self.stream.cuda_stream or None)
+        self._handle = ctypes.c_void_p()
+        self._wsb = ctypes.c_size_t()
+
+    def step(self):
+        """plan + run (the whole hot path for one batch)."""
+        lib = self.lib
+        st = lib.fa_decode_plan(ctypes.byref(self.desc), self.ind_host.ctypes.data, 0,
+                                ctypes.byref(self._handle), ctypes.byref(self._wsb))
+        if st != 0:
+            raise RuntimeError(f"fa_decode_plan failed: {st}")
+        st = lib.fa_decode_run(self._handle, *self.args)
+        lib.fa_plan_destroy(self._handle)
+        if st != 0:
+            raise RuntimeError(f"fa_decode_run failed: {st}")
+
+    def check_status(self):
+        flags = self.binding.decode_status(self.ws)
+        if flags:
+            raise RuntimeError(f"device check flags {flags}")
+
+
+def time_steps(fn, steps, stream):
+    import torch
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def per_launch_ms(fn, reps, stream, flush=None):
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(reps)]
+    for a, b in evs:
+        if flush is not None:
+            flush()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def l2_flusher(device="cuda"):
+    import torch
+    buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    return lambda: buf.fill_(1)
+
+
+def e2e_measure(x, runner, steps):
+    """Same metric through the C ABI with host buffers (pinned), copies in the
+    timed region."""
+    import torch
+    hq = torch.from_numpy(np.ascontiguousarray(x.q).view(np.int16)).pin_memory()
+    fp8 = x.kv_dtype == "fp8_e4m3"
+    conv = (lambda a: torch.from_numpy(np.ascontiguousarray(a))) if fp8 else \
+        (lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)))
+    hk, hv = conv(x.k).pin_memory(), conv(x.v).pin_memory()
+    hind = torch.from_numpy(x.kv_indptr).pin_memory()
+    hpt = torch.from_numpy(x.page_table).pin_memory() if x.paged else None
+    hks = torch.from_numpy(x.k_scale).pin_memory() if fp8 else None
+    hvs = torch.from_numpy(x.v_scale).pin_memory() if fp8 else None
+    out_h = torch.empty(runner.out.shape, dtype=runner.out.dtype).pin_memory()
+    lse_h = torch.empty(runner.lse.shape, dtype=runner.lse.dtype).pin_memory()
+    pairs = [(runner.q, hq), (runner.k, hk), (runner.v, hv), (runner.ind, hind)]
+    if hpt is not None:
+        pairs.append((runner.pt, hpt))
+    if fp8:
+        pairs += [(runner.ks, hks), (runner.vs, hvs)]
+    h2d = sum(h.numel() * h.element_size() for _, h in pairs)
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+
+    def step():
+        for d, h in pairs:
+            d.copy_(h, non_blocking=True)
+        runner.step()
+        out_h.copy_(runner.out, non_blocking=True)
+        lse_h.copy_(runner.lse, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    ms = time_steps(step, steps, runner.stream) / steps
+    return ms, h2d, d2h
+
+
+# --------------------------------------------------------------- CPU side
+def oracle_sample(x, budget_s, max_requests=None):
+    """Time the fp64 oracle on whole requests of x (all their heads) for about
+    budget_s seconds.  Returns (seconds, kv bytes, requests, threads)."""
+    from oracle import oracle
+    threads = int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
+    order = list(range(x.batch))
+    done_b, t_total, nbytes = 0, 0.0, 0
+    vis = x.visible_lens()
+    per_tok = x.kv_heads * x.head_dim * x.elem_bytes * 2
+    for b in order:
+        rows = np.arange(b * x.qo_heads, (b + 1) * x.qo_heads)
+        t0 = time.perf_counter()
+        oracle.decode_rows(x, rows, nthreads=threads)
+        t_total += time.perf_counter() - t0
+        nbytes += int(vis[b]) * per_tok
+        done_b += 1
+        if t_total >= budget_s or (max_requests and done_b >= max_requests):
+            break
+    return t_total, nbytes, done_b, threads
+
+
+def cpu_baseline(x, budget_s=12.0):
+    t, nbytes, nreq, threads = oracle_sample(x, budget_s)
+    return {"value": round(nbytes / t / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": "oracle", "tokens_per_s": round(nreq / t, 3),
+            "sample": f"fp64 oracle over {nreq} whole request(s) of {x.name} "
+                      f"({nbytes / 1e9:.3f} GB of K/V) in {t:.2f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    from gqa_decode_attention_split_b200 import synth
+    x = synth.workload(args.workload)
+    total_budget = 150.0
+    per_step = max(0.5, total_budget / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(x, per_step)
+    times, byts, reqs = [], [], []
+    threads = 0
+    for _ in range(args.steps):
+        t, nbytes, nreq, threads = oracle_sample(x, per_step)
+        times.append(t)
+        byts.append(nbytes)
+        reqs.append(nreq)
+    t, nbytes, nreq = sum(times), sum(byts), sum(reqs)
+    value = nbytes / t / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * t / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(x, world),
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+                             "kind": "oracle",
+                             "sample": f"each step: fp64 oracle over whole requests of {x.name} "
+                                       f"for about {per_step:.1f} s ({nreq} requests in total)"},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "tokens_per_s": round(nreq / t, 3)}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(x, world):
+    lens = x.kv_lens
+    return {"workload": x.name, "batch": x.batch, "qo_heads": x.qo_heads,
+            "kv_heads": x.kv_heads, "head_dim": x.head_dim, "kv_dtype": x.kv_dtype,
+            "paged": bool(x.paged), "page_size": x.page_size, "window": x.window,
+            "kv_len_min": int(lens.min()), "kv_len_max": int(lens.max()),
+            "kv_tokens": int(lens.sum()), "kv_bytes_per_step_per_gpu": x.kv_bytes(),
+            "l2": "inputs larger than L2 (no flush)" if x.kv_bytes() > 256e6
+            else "L2 flushed (256 MB write) before every timed launch",
+            "parallelism": f"replicas x{world} (independent batches, no collective)"}
+
+
+# ------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=HEADLINE)
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "mma"])
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    from gqa_decode_attention_split_b200 import synth
+
+    x = synth.workload(args.workload)
+    runner = Runner(x, path=args.path)
+    stream = runner.stream
+    for _ in range(args.warmup):
+        runner.step()
+    torch.cuda.synchronize()
+    runner.check_status()
+    sampler = ClockSampler(gpu_index(local_rank))
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ms_total = time_steps(runner.step, args.steps, stream)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    t = torch.tensor([ms_total], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    kv_bytes = x.kv_bytes()
+    value = world * kv_bytes / (ms_step * 1e-3) / 1e9
+    tokens = world * x.batch / (ms_step * 1e-3)
+
+    # dominant kernel: per-launch device time on the launching stream
+    launch_ms = per_launch_ms(runner.step, min(args.steps, 100), stream,
+                              flush=None if kv_bytes > 256e6 else l2_flusher())
+    mean_launch = statistics.mean(launch_ms)
+    peak, peak_kind = hbm_peak()
+    achieved = kv_bytes / (mean_launch * 1e-3) / 1e9
+    traffic = ncu_traffic(x.name)
+    runner.check_status()
+
+    e2e = None
+    if not args.no_e2e:
+        ms_e2e, h2d, d2h = e2e_measure(x, runner, args.e2e_steps)
+        e2e = {"value": round(world * kv_bytes / (ms_e2e * 1e-3) / 1e9, 3), "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(ms_e2e, 3), "steps": args.e2e_steps,
+               "tokens_per_s": round(world * x.batch / (ms_e2e * 1e-3), 1)}
+
+    sweep = None
+    if rank == 0 and world == 1 and not args.no_sweep:
+        sweep = {}
+        flush = l2_flusher()
+        for name in SWEEP:
+            y = synth.workload(name)
+            r = Runner(y)
+            for _ in range(5):
+                r.step()
+            ms = per_launch_ms(r.step, 30, r.stream, flush=flush if y.kv_bytes() <= 256e6 else None)
+            med = statistics.median(ms)
+            r.check_status()
+            sweep[name] = {"us": round(med * 1e3, 2), "gbps": round(y.kv_bytes() / (med * 1e-3) / 1e9, 1),
+                           "frac": round(y.kv_bytes() / (med * 1e-3) / 1e9 / peak, 4),
+                           "tokens_per_s": round(y.batch / (med * 1e-3), 1),
+                           "path": "mma" if r.info["path"] == 2 else "simt",
+                           "ctas": r.info["num_ctas"], "kv_bytes": y.kv_bytes()}
+            del r
+            torch.cuda.empty_cache()
+        for path in ("simt", "mma"):
+            try:
+                r = Runner(x, path=path)
+            except Exception:
+                continue
+            for _ in range(5):
+                r.step()
+            med = statistics.median(per_launch_ms(r.step, 30, r.stream))
+            sweep[f"{x.name}[{path}]"] = {"us": round(med * 1e3, 2),
+                                          "gbps": round(kv_bytes / (med * 1e-3) / 1e9, 1),
+                                          "frac": round(kv_bytes / (med * 1e-3) / 1e9 / peak, 4)}
+            del r
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(x)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16" if x.kv_dtype == "bf16" else "fp8_e4m3",
+                "data": "synthetic", "config": workload_config(x, world),
+                "tokens_per_s": round(tokens, 1), "frac_of_peak": round(value / world / peak, 4),
+                "path": "mma" if runner.info["path"] == 2 else "simt",
+                "num_ctas": runner.info["num_ctas"],
+                "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                             "unit": "GB/s", "frac": round(achieved / peak, 4),
+                             "traffic": traffic, "peak_source": peak_kind,
+                             "launch_us": round(mean_launch * 1e3, 2),
+                             "algorithmic_bytes_per_launch": kv_bytes},
+                "gpu_launches": args.steps, "clocks": clocks, "e2e": e2e,
+                "cpu_baseline": cpu, "sweep": sweep}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

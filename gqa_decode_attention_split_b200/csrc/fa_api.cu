@@ -1,0 +1,426 @@
+// fa_api.cu -- host side of the C ABI declared in include/fadecode.h:
+// planner, argument validation, tensor-map construction, launches, and the
+// standalone merge-states kernel.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+#include <new>
+
+#include "../../include/fadecode.h"
+#include "fa_kernel.cuh"
+#include "fa_registry.h"
+
+using fa::KernelEntry;
+
+// ------------------------------------------------------------ registry
+namespace {
+
+constexpr int kMaxEntries = 64;
+KernelEntry g_entries[kMaxEntries];
+int g_num_entries = 0;
+std::once_flag g_registry_once;
+
+void build_registry() {
+  int n = 0;
+  n += fa::register_d64(g_entries + n, kMaxEntries - n);
+  n += fa::register_d128(g_entries + n, kMaxEntries - n);
+  n += fa::register_d256(g_entries + n, kMaxEntries - n);
+  g_num_entries = n;
+}
+
+const KernelEntry* find_entry(int head_dim, int group, int fp8, int path) {
+  std::call_once(g_registry_once, build_registry);
+  for (int i = 0; i < g_num_entries; ++i) {
+    const KernelEntry& e = g_entries[i];
+    if (e.head_dim != head_dim || e.fp8 != fp8 || e.path != path) continue;
+    if (e.group != 0 ? e.group == group : group <= e.max_group) return &e;
+  }
+  return nullptr;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// dependency on libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------- the plan
+struct fa_plan {
+  fa_decode_desc desc;
+  const KernelEntry* kernel;
+  int32_t group;
+  int32_t num_ctas;
+  int32_t box_t;
+  int32_t swz;
+  int32_t page_shift;
+  int64_t total_tiles;
+  int64_t max_partials;
+  size_t ws_bytes;
+  size_t off_counters, off_part_o, off_part_lse;
+  size_t smem;
+};
+
+namespace {
+
+int ilog2_exact(int x) {
+  int s = 0;
+  while ((1 << s) < x) ++s;
+  return (1 << s) == x ? s : -1;
+}
+
+int64_t host_num_tiles(int32_t L, int32_t window, int32_t T) {
+  if (L <= 0) return 0;
+  const int32_t lo = (window > 0 && L > window) ? L - window : 0;
+  return (L + T - 1) / T - lo / T;
+}
+
+fa_status validate_desc(const fa_decode_desc* d) {
+  if (d->batch < 1 || d->qo_heads < 1 || d->kv_heads < 1 || d->head_dim < 1)
+    return FA_ERR_INVALID_ARG;
+  if (d->qo_heads % d->kv_heads != 0) return FA_ERR_INVALID_ARG;
+  if (d->kv_dtype != FA_KV_BF16 && d->kv_dtype != FA_KV_FP8_E4M3) return FA_ERR_INVALID_ARG;
+  if (d->paged != 0 && d->paged != 1) return FA_ERR_INVALID_ARG;
+  if (d->paged && (d->page_size < 1 || d->page_size > 256 || ilog2_exact(d->page_size) < 0))
+    return FA_ERR_INVALID_ARG;
+  if (!isfinite(d->sm_scale)) return FA_ERR_INVALID_ARG;
+  if (d->path < FA_PATH_AUTO || d->path > FA_PATH_MMA) return FA_ERR_INVALID_ARG;
+  if (d->num_ctas < 0) return FA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(d->batch) * d->kv_heads > (1 << 30)) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* kv_indptr_host,
+                                    int32_t num_sms, fa_plan** plan, size_t* workspace_bytes) {
+  if (desc == nullptr || kv_indptr_host == nullptr || plan == nullptr) return FA_ERR_INVALID_ARG;
+  *plan = nullptr;
+  fa_status st = validate_desc(desc);
+  if (st != FA_OK) return st;
+  if (kv_indptr_host[0] != 0) return FA_ERR_INVALID_ARG;
+  for (int b = 0; b < desc->batch; ++b)
+    if (kv_indptr_host[b + 1] < kv_indptr_host[b]) return FA_ERR_INVALID_ARG;
+  if (num_sms < 0) return FA_ERR_INVALID_ARG;
+  if (num_sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+  }
+  const int group = desc->qo_heads / desc->kv_heads;
+  const int fp8 = desc->kv_dtype == FA_KV_FP8_E4M3 ? 1 : 0;
+
+  // Dataflow choice: the tensor-core (MMA) path whenever a kernel exists for
+  // the shape; the SIMT path when asked for, or when the group exceeds 8.
+  const KernelEntry* k = nullptr;
+  if (desc->path == FA_PATH_SIMT) {
+    k = find_entry(desc->head_dim, group, fp8, fa::kPathSimt);
+  } else if (desc->path == FA_PATH_MMA) {
+    k = find_entry(desc->head_dim, group, fp8, fa::kPathMma);
+  } else {
+    k = find_entry(desc->head_dim, group, fp8, fa::kPathMma);
+    if (k == nullptr) k = find_entry(desc->head_dim, group, fp8, fa::kPathSimt);
+  }
+  if (k == nullptr) return FA_ERR_UNSUPPORTED;
+
+  const int T = k->tile_tokens;
+  int64_t tiles = 0;
+  for (int b = 0; b < desc->batch; ++b)
+    tiles += host_num_tiles(kv_indptr_host[b + 1] - kv_indptr_host[b], desc->window, T);
+  tiles *= desc->kv_heads;
+
+  int64_t P;
+  if (desc->num_ctas > 0) {
+    P = desc->num_ctas;
+  } else {
+    // one block per SM (each holds a 128 KB tile ring); small problems use
+    // fewer blocks so that each streams at least half a ring of tiles.
+    const int64_t min_tiles = k->stages / 2 > 0 ? k->stages / 2 : 1;
+    const int64_t want = (tiles + min_tiles - 1) / min_tiles;
+    P = want < num_sms ? want : num_sms;
+    if (P < 1) P = 1;
+  }
+  if (P > (1 << 20)) return FA_ERR_UNSUPPORTED;
+
+  fa_plan* p = new (std::nothrow) fa_plan();
+  if (p == nullptr) return FA_ERR_INVALID_ARG;
+  p->desc = *desc;
+  p->kernel = k;
+  p->group = group;
+  p->num_ctas = static_cast<int32_t>(P);
+  p->total_tiles = tiles;
+  const int segs = desc->batch * desc->kv_heads;
+  p->max_partials = P + segs;
+  p->page_shift = desc->paged ? ilog2_exact(desc->page_size) : 0;
+  p->box_t = desc->paged ? (desc->page_size < T ? desc->page_size : T) : T;
+  p->swz = (k->plane_bytes == 128 && p->box_t >= 8) ? 1 : 0;
+  size_t off = 256;  // header: device-check word
+  p->off_counters = off;
+  off = align_up(off + sizeof(uint32_t) * static_cast<size_t>(segs), 256);
+  p->off_part_o = off;
+  off = align_up(off + sizeof(float) * static_cast<size_t>(p->max_partials) * group * desc->head_dim,
+                 256);
+  p->off_part_lse = off;
+  off = align_up(off + sizeof(float) * static_cast<size_t>(p->max_partials) * group, 256);
+  p->ws_bytes = off;
+  p->smem = k->smem_bytes(desc->batch);
+  if (p->smem > 232448) {
+    delete p;
+    return FA_ERR_UNSUPPORTED;  // batch too large for the per-block schedule arrays
+  }
+  *plan = p;
+  if (workspace_bytes != nullptr) *workspace_bytes = p->ws_bytes;
+  return FA_OK;
+}
+
+extern "C" fa_status fa_plan_get_info(const fa_plan* plan, fa_plan_info_t* info) {
+  if (plan == nullptr || info == nullptr) return FA_ERR_INVALID_ARG;
+  info->path = plan->kernel->path == fa::kPathMma ? FA_PATH_MMA : FA_PATH_SIMT;
+  info->num_ctas = plan->num_ctas;
+  info->tile_tokens = plan->kernel->tile_tokens;
+  info->stages = plan->kernel->stages;
+  info->total_tiles = static_cast<int32_t>(plan->total_tiles > INT32_MAX ? INT32_MAX : plan->total_tiles);
+  info->max_partials = static_cast<int32_t>(plan->max_partials);
+  info->workspace_bytes = plan->ws_bytes;
+  info->smem_bytes = plan->smem;
+  return FA_OK;
+}
+
+extern "C" void fa_plan_destroy(fa_plan* plan) { delete plan; }
+
+namespace {
+
+fa_status make_kv_map(const fa_plan* p, const void* base, int64_t kv_rows, CUtensorMap* map) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return FA_ERR_CUDA;
+  const fa_decode_desc& d = p->desc;
+  const KernelEntry* k = p->kernel;
+  const int es = d.kv_dtype == FA_KV_FP8_E4M3 ? 1 : 2;
+  const cuuint64_t row = static_cast<cuuint64_t>(d.head_dim) * es;
+  const CUtensorMapDataType dt = es == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
+  const CUtensorMapSwizzle sw = p->swz ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
+  const cuuint32_t inner = static_cast<cuuint32_t>(k->plane_bytes / es);
+  CUresult r;
+  if (!d.paged) {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d.head_dim),
+                                static_cast<cuuint64_t>(d.kv_heads),
+                                static_cast<cuuint64_t>(kv_rows)};
+    const cuuint64_t strides[2] = {row, row * d.kv_heads};
+    const cuuint32_t box[3] = {inner, 1, static_cast<cuuint32_t>(k->tile_tokens)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else {
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d.head_dim),
+                                static_cast<cuuint64_t>(d.kv_heads),
+                                static_cast<cuuint64_t>(d.page_size),
+                                static_cast<cuuint64_t>(kv_rows)};
+    const cuuint64_t strides[3] = {row, row * d.kv_heads, row * d.kv_heads * d.page_size};
+    const cuuint32_t box[4] = {inner, 1, static_cast<cuuint32_t>(p->box_t), 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    r = enc(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  }
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" fa_status fa_decode_run(const fa_plan* plan, const void* q, const void* k,
+                                   const void* v, int64_t kv_rows, const int32_t* page_table,
+                                   int32_t page_table_stride, const int32_t* kv_indptr,
+                                   const float* k_scale, const float* v_scale, void* out,
+                                   float* lse, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  if (plan == nullptr || q == nullptr || k == nullptr || v == nullptr || kv_indptr == nullptr ||
+      out == nullptr || workspace == nullptr)
+    return FA_ERR_INVALID_ARG;
+  const fa_decode_desc& d = plan->desc;
+  const bool fp8 = d.kv_dtype == FA_KV_FP8_E4M3;
+  if (d.paged && (page_table == nullptr || page_table_stride < 1)) return FA_ERR_INVALID_ARG;
+  if (fp8 && (k_scale == nullptr || v_scale == nullptr)) return FA_ERR_INVALID_ARG;
+  if (kv_rows < 1 || kv_rows > INT32_MAX) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      !aligned(workspace, 256) || !aligned(kv_indptr, 4) || (lse && !aligned(lse, 4)) ||
+      (page_table && !aligned(page_table, 4)) || (k_scale && !aligned(k_scale, 4)) ||
+      (v_scale && !aligned(v_scale, 4)))
+    return FA_ERR_MISALIGNED;
+  if (workspace_bytes < plan->ws_bytes) return FA_ERR_WORKSPACE_TOO_SMALL;
+
+  fa::KernelArgs a;
+  memset(&a, 0, sizeof(a));
+  fa_status st = make_kv_map(plan, k, kv_rows, &a.kmap);
+  if (st == FA_OK) st = make_kv_map(plan, v, kv_rows, &a.vmap);
+  if (st != FA_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.q = static_cast<const uint16_t*>(q);
+  a.kv_indptr = kv_indptr;
+  a.page_table = d.paged ? page_table : nullptr;
+  a.k_scale = fp8 ? k_scale : nullptr;
+  a.v_scale = fp8 ? v_scale : nullptr;
+  a.out = static_cast<uint16_t*>(out);
+  a.lse = lse;
+  a.status = reinterpret_cast<uint32_t*>(ws);
+  a.counters = reinterpret_cast<uint32_t*>(ws + plan->off_counters);
+  a.part_o = reinterpret_cast<float*>(ws + plan->off_part_o);
+  a.part_lse = reinterpret_cast<float*>(ws + plan->off_part_lse);
+  a.kv_rows = kv_rows;
+  a.batch = d.batch;
+  a.qo_heads = d.qo_heads;
+  a.kv_heads = d.kv_heads;
+  a.group = plan->group;
+  a.window = d.window > 0 ? d.window : -1;
+  a.paged = d.paged;
+  a.page_shift = plan->page_shift;
+  a.pt_stride = d.paged ? page_table_stride : 0;
+  a.box_t = plan->box_t;
+  a.swz = plan->swz;
+  a.score_scale = d.sm_scale * 1.4426950408889634f;
+
+  cudaError_t e = plan->kernel->launch(a, plan->num_ctas, plan->smem,
+                                       static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+extern "C" fa_status fa_decode_status(void* workspace, size_t workspace_bytes, uint32_t* flags,
+                                      void* stream) {
+  if (workspace == nullptr || flags == nullptr || workspace_bytes < 256) return FA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t h = 0;
+  if (cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  *flags = h;
+  if (h != 0) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    return FA_ERR_DEVICE_CHECK;
+  }
+  return FA_OK;
+}
+
+// ------------------------------------------------------------ merge states
+namespace {
+
+// One warp per (row, head): lse = M + ln sum exp(lse_c - M); out = sum
+// exp(lse_c - lse) o_c.  States with lse = -inf carry no weight.
+__global__ void fa_merge_states_kernel(const float* __restrict__ o_parts,
+                                       const float* __restrict__ lse_parts, int n, long long rh_count,
+                                       int d, uint16_t* __restrict__ out, float* __restrict__ lse_out) {
+  const long long rh = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (rh >= rh_count) return;
+  float M = -CUDART_INF_F;
+  for (int c = lane; c < n; c += 32) M = fmaxf(M, lse_parts[c * rh_count + rh]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  if (M == -CUDART_INF_F) {
+    for (int x = lane * 4; x < d; x += 128)
+      *reinterpret_cast<uint2*>(out + rh * d + x) = make_uint2(0u, 0u);
+    if (lane == 0 && lse_out != nullptr) lse_out[rh] = -CUDART_INF_F;
+    return;
+  }
+  float Z = 0.f;
+  for (int c = lane; c < n; c += 32) {
+    const float l = lse_parts[c * rh_count + rh];
+    if (l != -CUDART_INF_F) Z += exp2f((l - M) * fa::kLog2e);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, off);
+  const float L = M + logf(Z);
+  for (int x = lane * 4; x < d; x += 128) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = 0; c < n; ++c) {
+      const float l = lse_parts[c * rh_count + rh];
+      if (l == -CUDART_INF_F) continue;
+      const float w = exp2f((l - L) * fa::kLog2e);
+      const float4 v = *reinterpret_cast<const float4*>(o_parts + (c * rh_count + rh) * d + x);
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+    }
+    const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(acc.x)) |
+                        (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc.y))) << 16);
+    const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(acc.z)) |
+                        (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc.w))) << 16);
+    *reinterpret_cast<uint2*>(out + rh * d + x) = make_uint2(lo, hi);
+  }
+  if (lane == 0 && lse_out != nullptr) lse_out[rh] = L;
+}
+
+}  // namespace
+
+extern "C" fa_status fa_merge_states(const float* o_parts, const float* lse_parts, int32_t n,
+                                     int32_t rows, int32_t heads, int32_t head_dim, void* out,
+                                     float* lse_out, void* stream) {
+  if (o_parts == nullptr || lse_parts == nullptr || out == nullptr) return FA_ERR_INVALID_ARG;
+  if (n < 1 || rows < 1 || heads < 1 || head_dim < 4 || head_dim % 4 != 0 || head_dim > 1024)
+    return FA_ERR_INVALID_ARG;
+  if (!aligned(o_parts, 16) || !aligned(out, 16) || !aligned(lse_parts, 4) ||
+      (lse_out && !aligned(lse_out, 4)))
+    return FA_ERR_MISALIGNED;
+  const long long rh = static_cast<long long>(rows) * heads;
+  const int threads = 256;
+  const long long blocks = (rh * 32 + threads - 1) / threads;
+  if (blocks > INT32_MAX) return FA_ERR_INVALID_ARG;
+  fa_merge_states_kernel<<<static_cast<unsigned>(blocks), threads, 0,
+                           static_cast<cudaStream_t>(stream)>>>(
+      o_parts, lse_parts, n, rh, head_dim, static_cast<uint16_t*>(out), lse_out);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  return FA_OK;
+}
+
+extern "C" const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case FA_ERR_WORKSPACE_TOO_SMALL: return "workspace smaller than the plan requires";
+    case FA_ERR_MISALIGNED: return "pointer below its required alignment";
+    case FA_ERR_CUDA: return "CUDA call failed";
+    case FA_ERR_DEVICE_CHECK: return "device-side check recorded an error";
+  }
+  return "unknown status";
+}
+
+extern "C" int32_t fa_version(void) { return 100; }

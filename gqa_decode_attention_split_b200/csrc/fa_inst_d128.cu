@@ -1,0 +1,6 @@
+// Decode-kernel variants for head_dim 128.
+#include "fa_instantiate.cuh"
+
+namespace fa {
+int register_d128(KernelEntry* out, int cap) { return register_bf16_and_fp8<128>(out, cap, true); }
+}  // namespace fa

@@ -1,0 +1,6 @@
+// Decode-kernel variants for head_dim 64.
+#include "fa_instantiate.cuh"
+
+namespace fa {
+int register_d64(KernelEntry* out, int cap) { return register_bf16_and_fp8<64>(out, cap, true); }
+}  // namespace fa

@@ -1,0 +1,77 @@
+// fa_instantiate.cuh -- helpers that turn a consumer type into a registry
+// entry (included by the per-head_dim instantiation units only).
+#pragma once
+
+#include <atomic>
+
+#include "fa_kernel.cuh"
+#include "fa_registry.h"
+
+namespace fa {
+
+constexpr int kMaxDynamicSmem = 232448;  // 227 KB per block on sm_100
+
+template <class Cons>
+cudaError_t launch_decode(const KernelArgs& args, int grid, size_t smem, cudaStream_t stream) {
+  static std::atomic<unsigned long long> configured{0};  // one bit per device ordinal
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(configured.load() & bit)) {
+    e = cudaFuncSetAttribute(fa_decode_kernel<Cons>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kMaxDynamicSmem);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit);
+  }
+  fa_decode_kernel<Cons><<<grid, Cons::C::THREADS, smem, stream>>>(args);
+  return cudaGetLastError();
+}
+
+template <class Cons>
+size_t smem_bytes_for(int batch) {
+  return SmemLayout<Cons>::bytes(batch);
+}
+
+template <class Cons>
+KernelEntry make_entry(int path, int group, int max_group, int fp8) {
+  using C = typename Cons::C;
+  KernelEntry e;
+  e.head_dim = C::ROWB / C::ES;
+  e.group = group;
+  e.max_group = max_group;
+  e.fp8 = fp8;
+  e.path = path;
+  e.tile_tokens = C::T;
+  e.stages = C::STAGES;
+  e.threads = C::THREADS;
+  e.row_bytes = C::ROWB;
+  e.plane_bytes = C::CB;
+  e.smem_bytes = &smem_bytes_for<Cons>;
+  e.launch = &launch_decode<Cons>;
+  return e;
+}
+
+template <int D>
+int register_bf16_and_fp8(KernelEntry* out, int cap, bool with_fp8) {
+  int n = 0;
+  auto add = [&](const KernelEntry& e) {
+    if (n < cap) out[n++] = e;
+  };
+  add(make_entry<MmaConsumer<D, false>>(kPathMma, 0, 8, 0));
+  add(make_entry<SimtConsumer<D, 1, false>>(kPathSimt, 1, 1, 0));
+  add(make_entry<SimtConsumer<D, 2, false>>(kPathSimt, 2, 2, 0));
+  add(make_entry<SimtConsumer<D, 4, false>>(kPathSimt, 4, 4, 0));
+  add(make_entry<SimtConsumer<D, 8, false>>(kPathSimt, 8, 8, 0));
+  if constexpr (D >= 128) {
+    if (with_fp8) {
+      add(make_entry<MmaConsumer<D, true>>(kPathMma, 0, 8, 1));
+      add(make_entry<SimtConsumer<D, 1, true>>(kPathSimt, 1, 1, 1));
+      add(make_entry<SimtConsumer<D, 2, true>>(kPathSimt, 2, 2, 1));
+      add(make_entry<SimtConsumer<D, 4, true>>(kPathSimt, 4, 4, 1));
+    }
+  }
+  return n;
+}
+
+}  // namespace fa

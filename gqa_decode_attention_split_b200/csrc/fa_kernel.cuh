@@ -1,0 +1,908 @@
+// fa_kernel.cuh -- split-KV GQA decode attention for sm_100a.
+//
+// One launch does the whole pass:
+//  1. schedule: every (request, kv head) is a segment of KV tiles; segments
+//     are laid end to end and cut into gridDim.x equal runs, one per thread
+//     block, so every SM streams the same number of bytes whatever the
+//     length mix ("FlashDecoding++" explainer, section "Hardware-aware
+//     heuristic dataflow": the split is chosen from batch, lengths and GPU).
+//     Each block derives its runs from kv_indptr in shared memory; nothing
+//     is uploaded from the host.
+//  2. load: a producer warp streams K and V tiles HBM -> shared memory with
+//     bulk tensor copies (TMA) into a ring of mbarrier-guarded stages, so the
+//     next tiles are in flight while the current ones are consumed ("Beyond
+//     the Memory Wall", section on FlashAttention-3: the next tile is
+//     prefetched while the current one is computed).
+//  3. math: consumer warps take whole tiles round-robin.  Each keeps a
+//     running (max, sum, acc) per query head and rescales when the max grows
+//     ("Forcing Flash Attention onto a TPU", section "Flash Attention in
+//     JAX").  Two dataflows: SIMT (per-lane fp32 FMAs, warp-shuffle
+//     reductions) and MMA (the two skinny products on mma.sync with fp32
+//     accumulation).
+//  4. merge: warps of a block merge their states in shared memory; a
+//     segment cut across blocks writes (o, lse) partials and the last block
+//     to finish it (atomic ticket, no waiting) merges them exactly through
+//     log-sum-exp ("FlashDecoding++" explainer, section "Asynchronous softmax
+//     and unified max value": partial softmax per tile, combined afterwards;
+//     "Flashlight", section "Method": exp(x - y) = exp(x) / exp(y)).
+#pragma once
+
+#include <math_constants.h>
+
+#include "fa_device.cuh"
+
+namespace fa {
+
+constexpr int kConsumerWarps = 8;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait, then give up
+constexpr float kRescaleSlack = 8.0f;               // log2 units
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// Device-check bits (same values as the public FA_DEVICE_* constants).
+constexpr uint32_t kFlagBadPage = 1u;
+constexpr uint32_t kFlagTimeout = 2u;
+constexpr uint32_t kFlagBadIndptr = 4u;
+
+struct KernelArgs {
+  CUtensorMap kmap;
+  CUtensorMap vmap;
+  const uint16_t* q;
+  const int32_t* kv_indptr;
+  const int32_t* page_table;
+  const float* k_scale;
+  const float* v_scale;
+  uint16_t* out;
+  float* lse;
+  uint32_t* status;
+  uint32_t* counters;
+  float* part_o;
+  float* part_lse;
+  long long kv_rows;
+  int batch, qo_heads, kv_heads, group;
+  int window;
+  int paged, page_shift, pt_stride, box_t, swz;
+  float score_scale;  // sm_scale * log2(e)
+};
+
+// Shared-memory tile geometry for one head_dim / element type.  A K (or V)
+// tile of T tokens is stored plane-major: [NP][T][CB] where a plane holds
+// CB = min(128, row bytes) bytes of every token row; with 128-byte rows the
+// 16-byte chunks of row r are XOR-swizzled by (r & 7) (TMA 128B swizzle).
+template <int D, bool FP8>
+struct TileCfg {
+  static constexpr int ES = FP8 ? 1 : 2;
+  static constexpr int ROWB = D * ES;
+  static constexpr int CB = ROWB < 128 ? ROWB : 128;
+  static constexpr int NP = ROWB / CB;
+  static constexpr int T = (4096 / ROWB) > 16 ? (4096 / ROWB) : 16;
+  static constexpr int TILE_BYTES = T * ROWB;
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  static constexpr int NW = kConsumerWarps;
+  static constexpr int STAGES_RAW = (128 * 1024) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW < NW ? NW : (STAGES_RAW / NW) * NW;
+  static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
+  static constexpr int THREADS = (NW + 1) * 32;
+  static_assert(ROWB % 16 == 0, "rows must be whole 16-byte chunks");
+};
+
+__device__ __forceinline__ uint32_t swz_off(int row, int chunk, int swz) {
+  return static_cast<uint32_t>(((chunk ^ (swz ? (row & 7) : 0)) << 4));
+}
+
+// ------------------------------------------------------------ schedule
+struct Piece {
+  int b, h;          // request, kv head
+  int t0, t1;        // request-local tile indices [t0, t1)
+  int seg;           // b * kv_heads + h
+  int n_pieces;      // blocks sharing this segment
+  int c_first;       // first block of the segment
+  long long seg_start;
+};
+
+struct PieceIter {
+  long long u, u1, per;
+};
+
+__device__ __forceinline__ int first_tile(int L, int window, int T) {
+  int lo = (window > 0 && L > window) ? L - window : 0;
+  return lo / T;
+}
+__device__ __forceinline__ int num_tiles(int L, int window, int T) {
+  if (L <= 0) return 0;
+  return (L + T - 1) / T - first_tile(L, window, T);
+}
+
+__device__ __forceinline__ bool next_piece(PieceIter& it, Piece& pc, const int* s_pre,
+                                           const int* s_len, int B, int H, int window, int T) {
+  if (it.u >= it.u1) return false;
+  int lo = 0, hi = B;  // H*pre[lo] <= u < H*pre[hi]
+  while (hi - lo > 1) {
+    int mid = (lo + hi) >> 1;
+    if (static_cast<long long>(H) * s_pre[mid] <= it.u)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  const int b = lo;
+  const int n = s_pre[b + 1] - s_pre[b];
+  const long long base = static_cast<long long>(H) * s_pre[b];
+  const long long off = it.u - base;
+  const int h = static_cast<int>(off / n);
+  const int tin = static_cast<int>(off % n);
+  long long len = n - tin;
+  if (it.u1 - it.u < len) len = it.u1 - it.u;
+  const int ft = first_tile(s_len[b], window, T);
+  pc.b = b;
+  pc.h = h;
+  pc.t0 = ft + tin;
+  pc.t1 = pc.t0 + static_cast<int>(len);
+  pc.seg = b * H + h;
+  pc.seg_start = base + static_cast<long long>(h) * n;
+  const long long seg_end = pc.seg_start + n;
+  pc.c_first = static_cast<int>(pc.seg_start / it.per);
+  pc.n_pieces = static_cast<int>((seg_end - 1) / it.per) - pc.c_first + 1;
+  it.u += len;
+  return true;
+}
+
+// ------------------------------------------------------ SIMT dataflow
+// Lanes are grouped LPT per token; a lane owns CPL 16-byte chunks of every
+// row (E elements), holds q for those elements for all G heads and an fp32
+// accumulator for the same.  q.k partial sums are all-reduced over the LPT
+// lanes with xor shuffles; each group of lanes ("slot") keeps its own
+// running softmax state, merged across slots at the end of a segment piece.
+template <int D, int G, bool FP8>
+struct SimtConsumer {
+  using C = TileCfg<D, FP8>;
+  static constexpr int GM = G;  // merge-area heads
+  static constexpr int EPC = 16 / C::ES;
+  static constexpr int NCH = C::ROWB / 16;
+  static constexpr int E_TARGET = 64 / G;
+  static constexpr int CPL_RAW = E_TARGET / EPC;
+  static constexpr int CPL = CPL_RAW < 1 ? 1 : (CPL_RAW > NCH ? NCH : CPL_RAW);
+  static constexpr int E = CPL * EPC;
+  static constexpr int LPT = NCH / CPL;
+  static constexpr int SLOTS = 32 / LPT;
+  static constexpr int TPS = C::T / SLOTS;
+  static constexpr int NCP = C::CB / 16;
+  static_assert(LPT >= 1 && LPT <= 32 && (NCH % CPL) == 0, "lane mapping");
+  static_assert(TPS >= 1 && (C::T % SLOTS) == 0, "tokens per slot");
+
+  float q[G][E];
+  float acc[G][E];
+  float m[G], l[G];
+  int slot, j;
+
+  __device__ __forceinline__ int chunk_plane(int k) const { return (j + LPT * k) / NCP; }
+  __device__ __forceinline__ int chunk_in_plane(int k) const { return (j + LPT * k) % NCP; }
+  __device__ __forceinline__ int dim_of(int k, int e) const {
+    return chunk_plane(k) * (C::CB / C::ES) + chunk_in_plane(k) * EPC + e;
+  }
+
+  __device__ __forceinline__ void convert(const uint4& w, float (&x)[EPC]) const {
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+    if constexpr (!FP8) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        x[2 * i] = bf16lo(u[i]);
+        x[2 * i + 1] = bf16hi(u[i]);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float2 a = f16x2_to_float2(e4m3x2_to_f16x2(static_cast<uint16_t>(u[i] & 0xFFFFu)));
+        float2 b = f16x2_to_float2(e4m3x2_to_f16x2(static_cast<uint16_t>(u[i] >> 16)));
+        x[4 * i] = a.x;
+        x[4 * i + 1] = a.y;
+        x[4 * i + 2] = b.x;
+        x[4 * i + 3] = b.y;
+      }
+    }
+  }
+
+  __device__ __forceinline__ uint32_t addr(uint32_t tile, int r, int k, int swz) const {
+    return tile + chunk_plane(k) * (C::T * C::CB) + r * C::CB +
+           swz_off(r, chunk_in_plane(k), swz);
+  }
+
+  __device__ __forceinline__ void begin_piece(const KernelArgs& a, int b, int hkv, int lane) {
+    slot = lane / LPT;
+    j = lane % LPT;
+    float scale = a.score_scale;
+    if constexpr (FP8) scale *= __ldg(a.k_scale + hkv);
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const uint16_t* qrow =
+          a.q + (static_cast<size_t>(b) * a.qo_heads + static_cast<size_t>(hkv) * G + h) * D;
+#pragma unroll
+      for (int k = 0; k < CPL; ++k) {
+#pragma unroll
+        for (int e = 0; e < EPC; e += 8) {
+          const uint4 w = __ldg(reinterpret_cast<const uint4*>(qrow + dim_of(k, e)));
+          const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            q[h][k * EPC + e + 2 * i] = bf16lo(u[i]) * scale;
+            q[h][k * EPC + e + 2 * i + 1] = bf16hi(u[i]) * scale;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) acc[h][k * EPC + e] = 0.f;
+      }
+      m[h] = -CUDART_INF_F;
+      l[h] = 0.f;
+    }
+  }
+
+  __device__ __forceinline__ void tile(const KernelArgs& a, uint32_t kt, uint32_t vt, int pos0,
+                                       int lo, int hi, int lane) {
+    float s[TPS][G];
+#pragma unroll
+    for (int tt = 0; tt < TPS; ++tt) {
+      const int r = tt * SLOTS + slot;
+      float part[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) part[h] = 0.f;
+#pragma unroll
+      for (int k = 0; k < CPL; ++k) {
+        float x[EPC];
+        convert(lds128(addr(kt, r, k, a.swz)), x);
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+          for (int e = 0; e < EPC; ++e) part[h] = fmaf(q[h][k * EPC + e], x[e], part[h]);
+      }
+#pragma unroll
+      for (int off = 1; off < LPT; off <<= 1)
+#pragma unroll
+        for (int h = 0; h < G; ++h) part[h] += __shfl_xor_sync(0xffffffffu, part[h], off);
+      const int pos = pos0 + r;
+      const bool valid = pos >= lo && pos < hi;
+#pragma unroll
+      for (int h = 0; h < G; ++h) s[tt][h] = valid ? part[h] : -CUDART_INF_F;
+    }
+    // running max with slack: rescale only when the tile max exceeds it by kRescaleSlack
+    bool need = false;
+    float tmax[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      tmax[h] = s[0][h];
+#pragma unroll
+      for (int tt = 1; tt < TPS; ++tt) tmax[h] = fmaxf(tmax[h], s[tt][h]);
+      need |= tmax[h] > m[h] + kRescaleSlack;
+    }
+    if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        if (tmax[h] > m[h] + kRescaleSlack) {
+          const float alpha = exp2_approx(m[h] - tmax[h]);  // m = -inf -> 0
+          l[h] *= alpha;
+#pragma unroll
+          for (int e = 0; e < E; ++e) acc[h][e] *= alpha;
+          m[h] = tmax[h];
+        }
+      }
+    }
+    float p[TPS][G];
+#pragma unroll
+    for (int tt = 0; tt < TPS; ++tt)
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        p[tt][h] = (m[h] == -CUDART_INF_F) ? 0.f : exp2_approx(s[tt][h] - m[h]);
+        l[h] += p[tt][h];
+      }
+#pragma unroll
+    for (int tt = 0; tt < TPS; ++tt) {
+      const int r = tt * SLOTS + slot;
+      const int pos = pos0 + r;
+      if (pos >= lo && pos < hi) {  // masked rows may hold anything: never read them as values
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) {
+          float x[EPC];
+          convert(lds128(addr(vt, r, k, a.swz)), x);
+#pragma unroll
+          for (int h = 0; h < G; ++h)
+#pragma unroll
+            for (int e = 0; e < EPC; ++e)
+              acc[h][k * EPC + e] = fmaf(p[tt][h], x[e], acc[h][k * EPC + e]);
+        }
+      }
+    }
+  }
+
+  // Merge the slots' states and publish the warp's state.
+  __device__ __forceinline__ void end_piece(float* m_area, float* l_area, float* acc_area, int w,
+                                            int lane) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float M = m[h];
+#pragma unroll
+      for (int off = LPT; off < 32; off <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+      const float sc = (m[h] == -CUDART_INF_F) ? 0.f : exp2_approx(m[h] - M);
+      float lh = l[h] * sc;
+#pragma unroll
+      for (int off = LPT; off < 32; off <<= 1) lh += __shfl_xor_sync(0xffffffffu, lh, off);
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        float v = acc[h][e] * sc;
+#pragma unroll
+        for (int off = LPT; off < 32; off <<= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        acc[h][e] = v;
+      }
+      if (lane == 0) {
+        m_area[w * GM + h] = M;
+        l_area[w * GM + h] = lh;
+      }
+      if (slot == 0) {
+#pragma unroll
+        for (int k = 0; k < CPL; ++k)
+#pragma unroll
+          for (int e = 0; e < EPC; ++e) acc_area[(w * GM + h) * D + dim_of(k, e)] = acc[h][k * EPC + e];
+      }
+    }
+  }
+};
+
+// ------------------------------------------------------- MMA dataflow
+// Scores S^T = K . Q^T on mma.m16n8k16 (16 tokens x 8 query heads x 16 dims
+// per instruction, fp32 accumulate); probabilities are transposed in
+// registers (movmatrix) into the B operand of O^T += V^T . P^T, with O^T
+// (dims x heads) accumulated in fp32 registers.  Up to 8 query heads per kv
+// head; missing heads are zero columns.  bf16 K/V use bf16 operands; e4m3
+// K/V are widened exactly to f16 and q is scaled by a power of two per head
+// into f16 range (the scale is undone on the fp32 scores).
+template <int D, bool FP8>
+struct MmaConsumer {
+  using C = TileCfg<D, FP8>;
+  static constexpr int GM = 8;
+  static constexpr int KS = D / 16;     // k-steps of the score product = m-tiles of O^T
+  static constexpr int SUB = C::T / 16;  // 16-token subtiles per tile
+  static constexpr int BPT = D / 4;      // fp8 K: bytes of a row owned by one lane
+  static constexpr int VBT = D / 8;      // fp8 V: bytes of a row owned by one lane
+  static_assert(D % 16 == 0 && C::T % 16 == 0, "mma tiling");
+  static_assert(!FP8 || C::CB == 128, "fp8 mma path needs 128-byte planes");
+
+  uint32_t qb[KS][2];
+  float o[KS][4];
+  float m[2], l[2];
+  float sscale[2];
+  int g, t;
+
+  __device__ __forceinline__ void begin_piece(const KernelArgs& a, int b, int hkv, int lane) {
+    g = lane >> 2;
+    t = lane & 3;
+    const int G = a.group;
+    const bool real = g < G;
+    const uint16_t* qrow =
+        a.q + (static_cast<size_t>(b) * a.qo_heads + static_cast<size_t>(hkv) * G + (real ? g : 0)) * D;
+    if constexpr (!FP8) {
+#pragma unroll
+      for (int kk = 0; kk < KS; ++kk) {
+        qb[kk][0] = real ? __ldg(reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * t)) : 0u;
+        qb[kk][1] = real ? __ldg(reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * t + 8)) : 0u;
+      }
+      sscale[0] = sscale[1] = a.score_scale;
+    } else {
+      // this lane's q elements: [BPT*t, BPT*t + BPT)
+      float mx = 0.f;
+      uint32_t qw[BPT / 2];
+#pragma unroll
+      for (int i = 0; i < BPT / 8; ++i) {
+        const uint4 w = real ? __ldg(reinterpret_cast<const uint4*>(qrow + BPT * t + 8 * i))
+                             : make_uint4(0, 0, 0, 0);
+        qw[4 * i] = w.x;
+        qw[4 * i + 1] = w.y;
+        qw[4 * i + 2] = w.z;
+        qw[4 * i + 3] = w.w;
+      }
+#pragma unroll
+      for (int i = 0; i < BPT / 2; ++i)
+        mx = fmaxf(mx, fmaxf(fabsf(bf16lo(qw[i])), fabsf(bf16hi(qw[i]))));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      int ex = 0;
+      frexpf(mx, &ex);
+      const int sh = (mx > 0.f && isfinite(mx)) ? 15 - ex : 0;  // |q| * 2^sh < 2^15
+      const float mul = ldexpf(1.f, sh);
+#pragma unroll
+      for (int kk = 0; kk < KS; ++kk) {
+        // logical k-columns 2t,2t+1 / 2t+8,2t+9 of step kk <-> bytes BPT*t + 4kk + {0,1} / {2,3}
+        const uint32_t w0 = qw[2 * kk], w1 = qw[2 * kk + 1];
+        qb[kk][0] = pack_f16x2(bf16lo(w0) * mul, bf16hi(w0) * mul);
+        qb[kk][1] = pack_f16x2(bf16lo(w1) * mul, bf16hi(w1) * mul);
+      }
+      const int sh0 = __shfl_sync(0xffffffffu, sh, (2 * t) * 4);
+      const int sh1 = __shfl_sync(0xffffffffu, sh, (2 * t + 1) * 4);
+      const float base = a.score_scale * __ldg(a.k_scale + hkv);
+      sscale[0] = base * ldexpf(1.f, -sh0);
+      sscale[1] = base * ldexpf(1.f, -sh1);
+    }
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[mt][i] = 0.f;
+    m[0] = m[1] = -CUDART_INF_F;
+    l[0] = l[1] = 0.f;
+  }
+
+  __device__ __forceinline__ uint32_t chunk_addr(uint32_t tile, int row, int chunk, int swz) const {
+    return tile + (chunk >> 3) * (C::T * 128) + row * 128 + swz_off(row, chunk & 7, swz);
+  }
+
+  __device__ __forceinline__ void scores(uint32_t kt, int sub, int lane, int swz, float (&c)[4]) const {
+    c[0] = c[1] = c[2] = c[3] = 0.f;
+    if constexpr (!FP8) {
+      const int row = sub * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int kk = 0; kk < KS; ++kk) {
+        uint32_t af[4];
+        const int ch = kk * 2 + (lane >> 4);
+        if constexpr (C::CB == 128)
+          ldsm_x4(chunk_addr(kt, row, ch, swz), af);
+        else  // 64-element rows: one plane of CB bytes, no swizzle
+          ldsm_x4(kt + row * C::CB + ch * 16, af);
+        mma_bf16(c, af, qb[kk][0], qb[kk][1]);
+      }
+    } else {
+      const int r0 = sub * 16 + g, r1 = r0 + 8;
+      uint32_t w0[BPT / 4], w1[BPT / 4];
+#pragma unroll
+      for (int i = 0; i < BPT / 16; ++i) {
+        const int ch = (BPT * t) / 16 + i;
+        const uint4 x0 = lds128(chunk_addr(kt, r0, ch, swz));
+        const uint4 x1 = lds128(chunk_addr(kt, r1, ch, swz));
+        w0[4 * i] = x0.x; w0[4 * i + 1] = x0.y; w0[4 * i + 2] = x0.z; w0[4 * i + 3] = x0.w;
+        w1[4 * i] = x1.x; w1[4 * i + 1] = x1.y; w1[4 * i + 2] = x1.z; w1[4 * i + 3] = x1.w;
+      }
+#pragma unroll
+      for (int kk = 0; kk < KS; ++kk) {
+        uint32_t af[4];
+        af[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(w0[kk] & 0xFFFFu));
+        af[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[kk] & 0xFFFFu));
+        af[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(w0[kk] >> 16));
+        af[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[kk] >> 16));
+        mma_f16(c, af, qb[kk][0], qb[kk][1]);
+      }
+    }
+  }
+
+  __device__ __forceinline__ void tile(const KernelArgs& a, uint32_t kt, uint32_t vt, int pos0,
+                                       int lo, int hi, int lane) {
+#pragma unroll
+    for (int sub = 0; sub < SUB; ++sub) {
+      float c[4];
+      scores(kt, sub, lane, a.swz, c);
+      const int pr = pos0 + sub * 16 + g;
+      const bool v0 = pr >= lo && pr < hi, v1 = pr + 8 >= lo && pr + 8 < hi;
+      const float s0 = v0 ? c[0] * sscale[0] : -CUDART_INF_F;
+      const float s1 = v0 ? c[1] * sscale[1] : -CUDART_INF_F;
+      const float s2 = v1 ? c[2] * sscale[0] : -CUDART_INF_F;
+      const float s3 = v1 ? c[3] * sscale[1] : -CUDART_INF_F;
+      float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+      }
+      const bool up0 = mx0 > m[0] + kRescaleSlack, up1 = mx1 > m[1] + kRescaleSlack;
+      if (__any_sync(0xffffffffu, up0 || up1)) {
+        const float a0 = up0 ? exp2_approx(m[0] - mx0) : 1.f;
+        const float a1 = up1 ? exp2_approx(m[1] - mx1) : 1.f;
+        if (up0) m[0] = mx0;
+        if (up1) m[1] = mx1;
+        l[0] *= a0;
+        l[1] *= a1;
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+          o[mt][0] *= a0;
+          o[mt][1] *= a1;
+          o[mt][2] *= a0;
+          o[mt][3] *= a1;
+        }
+      }
+      const bool dead0 = m[0] == -CUDART_INF_F, dead1 = m[1] == -CUDART_INF_F;
+      const float p0 = dead0 ? 0.f : exp2_approx(s0 - m[0]);
+      const float p1 = dead1 ? 0.f : exp2_approx(s1 - m[1]);
+      const float p2 = dead0 ? 0.f : exp2_approx(s2 - m[0]);
+      const float p3 = dead1 ? 0.f : exp2_approx(s3 - m[1]);
+      l[0] += p0 + p2;
+      l[1] += p1 + p3;
+      uint32_t x0, x1;
+      if constexpr (FP8) {
+        x0 = pack_f16x2(p0, p1);
+        x1 = pack_f16x2(p2, p3);
+      } else {
+        x0 = pack_bf16x2(p0, p1);
+        x1 = pack_bf16x2(p2, p3);
+      }
+      const uint32_t pb0 = movmatrix_trans(x0);  // P[head g][tokens 2t, 2t+1]
+      const uint32_t pb1 = movmatrix_trans(x1);  // P[head g][tokens 2t+8, 2t+9]
+      // rows that are not visible may hold anything (NaN included): zero them in V
+      const int pt = pos0 + sub * 16 + 2 * t;
+      const bool e0 = pt >= lo && pt < hi, e1 = pt + 1 >= lo && pt + 1 < hi;
+      const bool e8 = pt + 8 >= lo && pt + 8 < hi, e9 = pt + 9 >= lo && pt + 9 < hi;
+      const bool edge = __any_sync(0xffffffffu, !(e0 && e1 && e8 && e9));
+      const uint32_t mk01 = (e0 ? 0x0000FFFFu : 0u) | (e1 ? 0xFFFF0000u : 0u);
+      const uint32_t mk89 = (e8 ? 0x0000FFFFu : 0u) | (e9 ? 0xFFFF0000u : 0u);
+      if constexpr (!FP8) {
+        const int vrow = sub * 16 + (lane & 7) + (lane >> 4) * 8;
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+          uint32_t af[4];
+          const int ch = mt * 2 + ((lane >> 3) & 1);
+          if constexpr (C::CB == 128)
+            ldsm_x4_trans(chunk_addr(vt, vrow, ch, a.swz), af);
+          else
+            ldsm_x4_trans(vt + vrow * C::CB + ch * 16, af);
+          if (edge) {
+            af[0] &= mk01;
+            af[1] &= mk01;
+            af[2] &= mk89;
+            af[3] &= mk89;
+          }
+          mma_bf16(o[mt], af, pb0, pb1);
+        }
+      } else {
+        // lane owns dims [VBT*g, VBT*g + VBT) of tokens 2t, 2t+1, 2t+8, 2t+9
+        const int rb = sub * 16 + 2 * t;
+        const int rows[4] = {rb, rb + 1, rb + 8, rb + 9};
+        uint32_t vw[4][VBT / 4];
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+          for (int i = 0; i < VBT / 16; ++i) {
+            const uint4 x = lds128(chunk_addr(vt, rows[rr], (VBT * g) / 16 + i, a.swz));
+            vw[rr][4 * i] = x.x;
+            vw[rr][4 * i + 1] = x.y;
+            vw[rr][4 * i + 2] = x.z;
+            vw[rr][4 * i + 3] = x.w;
+          }
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+          const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
+          const uint32_t x01 = prmt(vw[0][mt >> 1], vw[1][mt >> 1], sel);
+          const uint32_t x89 = prmt(vw[2][mt >> 1], vw[3][mt >> 1], sel);
+          uint32_t af[4];
+          af[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(x01 & 0xFFFFu));
+          af[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(x01 >> 16));
+          af[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(x89 & 0xFFFFu));
+          af[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(x89 >> 16));
+          if (edge) {
+            af[0] &= mk01;
+            af[1] &= mk01;
+            af[2] &= mk89;
+            af[3] &= mk89;
+          }
+          mma_f16(o[mt], af, pb0, pb1);
+        }
+      }
+    }
+  }
+
+  __device__ __forceinline__ int out_dim(int mt, int half) const {
+    if constexpr (FP8)
+      return VBT * g + 2 * mt + half;
+    else
+      return mt * 16 + g + 8 * half;
+  }
+
+  __device__ __forceinline__ void end_piece(float* m_area, float* l_area, float* acc_area, int w,
+                                            int lane) {
+    float l0 = l[0], l1 = l[1];
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+    }
+    const int h0 = 2 * t, h1 = 2 * t + 1;
+    if (g == 0) {
+      m_area[w * GM + h0] = m[0];
+      m_area[w * GM + h1] = m[1];
+      l_area[w * GM + h0] = l0;
+      l_area[w * GM + h1] = l1;
+    }
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt) {
+      acc_area[(w * GM + h0) * D + out_dim(mt, 0)] = o[mt][0];
+      acc_area[(w * GM + h1) * D + out_dim(mt, 0)] = o[mt][1];
+      acc_area[(w * GM + h0) * D + out_dim(mt, 1)] = o[mt][2];
+      acc_area[(w * GM + h1) * D + out_dim(mt, 1)] = o[mt][3];
+    }
+  }
+};
+
+// ------------------------------------------------------------- kernel
+template <class Cons>
+struct SmemLayout {
+  using C = typename Cons::C;
+  static constexpr int D = C::ROWB / C::ES;
+  static constexpr int kBars = C::RING_BYTES;                        // full[S], empty[S]
+  static constexpr int kMerge = kBars + 2 * C::STAGES * 8;           // m[NW][GM], l[NW][GM]
+  static constexpr int kAccOff = kMerge + C::NW * Cons::GM * 2 * 4;  // acc[NW][GM][D]
+  static constexpr int kMisc = kAccOff + C::NW * Cons::GM * D * 4;   // ticket flag
+  static constexpr int kSched = kMisc + 16;                          // start[B] len[B] pre[B+1]
+  static constexpr size_t bytes(int batch) {
+    return 1024 + static_cast<size_t>(kSched) + static_cast<size_t>(3 * batch + 1) * 4;
+  }
+};
+
+template <class Cons>
+__global__ void __maxnreg__(224)
+    fa_decode_kernel(const __grid_constant__ KernelArgs a) {
+  using C = typename Cons::C;
+  using S = SmemLayout<Cons>;
+  constexpr int D = C::ROWB / C::ES;
+  constexpr int T = C::T;
+  constexpr int NW = C::NW;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (sbase - raw);
+  const uint32_t ring = sbase;
+  const uint32_t full0 = sbase + S::kBars;
+  const uint32_t empty0 = full0 + C::STAGES * 8;
+  float* m_area = reinterpret_cast<float*>(base + S::kMerge);
+  float* l_area = m_area + NW * Cons::GM;
+  float* acc_area = reinterpret_cast<float*>(base + S::kAccOff);
+  int* s_flag = reinterpret_cast<int*>(base + S::kMisc);
+  int* s_start = reinterpret_cast<int*>(base + S::kSched);
+  const int B = a.batch, H = a.kv_heads;
+  int* s_len = s_start + B;
+  int* s_pre = s_len + B;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int ps = a.paged ? (1 << a.page_shift) : 0;
+
+  // ---- setup: request lengths (validated), barriers, tile prefix sums
+  for (int b = tid; b < B; b += blockDim.x) {
+    const int st = __ldg(a.kv_indptr + b), en = __ldg(a.kv_indptr + b + 1);
+    int L = en - st;
+    bool bad = false;
+    if (st < 0 || L < 0) {
+      L = 0;
+      bad = true;
+    } else if (!a.paged && static_cast<long long>(en) > a.kv_rows) {
+      bad = true;  // rows past the extent read as zeros
+    } else if (a.paged && L > 0 && ((L + ps - 1) >> a.page_shift) > a.pt_stride) {
+      L = a.pt_stride << a.page_shift;
+      bad = true;
+    }
+    s_start[b] = st;
+    s_len[b] = L;
+    if (bad) atomicOr(a.status, kFlagBadIndptr);
+  }
+  if (tid == 32) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int carry = 0;
+    for (int b0 = 0; b0 < B; b0 += 32) {
+      const int b = b0 + lane;
+      const int n = b < B ? num_tiles(s_len[b], a.window, T) : 0;
+      int incl = n;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      if (b < B) s_pre[b] = carry + incl - n;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_pre[B] = carry;
+  }
+  __syncthreads();
+
+  const long long N = static_cast<long long>(H) * s_pre[B];
+  const int P = gridDim.x, c = blockIdx.x;
+  PieceIter it;
+  it.per = N > 0 ? (N + P - 1) / P : 1;
+  it.u = static_cast<long long>(c) * it.per;
+  it.u1 = it.u + it.per < N ? it.u + it.per : N;
+
+  if (warp == 0) {
+    // ================= producer: one elected lane issues the copies
+    const uint64_t pol = l2_evict_first_policy();
+    if (lane == 0) {
+      prefetch_tensormap(&a.kmap);
+      prefetch_tensormap(&a.vmap);
+    }
+    const int NB = T / a.box_t;  // copies per plane per tile (paged: one per page)
+    long long i = 0;
+    bool ok = true;
+    Piece pc;
+    while (ok && next_piece(it, pc, s_pre, s_len, B, H, a.window, T)) {
+      const int L = s_len[pc.b];
+      const int npages = a.paged ? (L + ps - 1) >> a.page_shift : 0;
+      int cache_base = -(1 << 30), cache_val = -1;
+      for (int tt = pc.t0; tt < pc.t1 && ok; ++tt, ++i) {
+        const int stage = static_cast<int>(i % C::STAGES);
+        const uint32_t parity = static_cast<uint32_t>((i / C::STAGES) & 1) ^ 1u;
+        const uint32_t fb = full0 + 8 * stage;
+        const uint32_t kdst = ring + stage * C::STAGE_BYTES;
+        const uint32_t vdst = kdst + C::TILE_BYTES;
+        if (lane == 0) {
+          if (!mbar_wait(empty0 + 8 * stage, parity, kWaitLimitNs)) {
+            atomicOr(a.status, kFlagTimeout);
+            ok = false;
+          } else {
+            mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        if (!a.paged) {
+          if (lane == 0) {
+            const int row = s_start[pc.b] + tt * T;
+#pragma unroll
+            for (int p = 0; p < C::NP; ++p) {
+              tma_load_3d(kdst + p * (T * C::CB), &a.kmap, fb, p * (C::CB / C::ES), pc.h, row, pol);
+              tma_load_3d(vdst + p * (T * C::CB), &a.vmap, fb, p * (C::CB / C::ES), pc.h, row, pol);
+            }
+          }
+        } else {
+          for (int jb = 0; jb < NB; ++jb) {
+            const int tok = tt * T + jb * a.box_t;
+            const int pidx = tok >> a.page_shift;
+            if (pidx < cache_base || pidx - cache_base >= 32) {
+              cache_base = pidx;
+              const int e = cache_base + lane;
+              cache_val = -1;
+              if (e < npages) {
+                cache_val = __ldg(a.page_table + static_cast<long long>(pc.b) * a.pt_stride + e);
+                if (cache_val < 0 || static_cast<long long>(cache_val) >= a.kv_rows)
+                  atomicOr(a.status, kFlagBadPage);
+              }
+            }
+            int page = __shfl_sync(0xffffffffu, cache_val, pidx - cache_base);
+            if (pidx >= npages || page < 0) page = -1;  // out of range: the copy fills zeros
+            if (lane == 0) {
+              const int slot0 = tok & (ps - 1);
+#pragma unroll
+              for (int p = 0; p < C::NP; ++p) {
+                const uint32_t off = p * (T * C::CB) + jb * a.box_t * C::CB;
+                tma_load_4d(kdst + off, &a.kmap, fb, p * (C::CB / C::ES), pc.h, slot0, page, pol);
+                tma_load_4d(vdst + off, &a.vmap, fb, p * (C::CB / C::ES), pc.h, slot0, page, pol);
+              }
+            }
+          }
+        }
+      }
+    }
+    // drain: every issued copy has landed before the block may exit
+    if (lane == 0) {
+      const long long first = i > C::STAGES ? i - C::STAGES : 0;
+      for (long long k = first; k < i; ++k) {
+        const int stage = static_cast<int>(k % C::STAGES);
+        if (!mbar_wait(full0 + 8 * stage, static_cast<uint32_t>((k / C::STAGES) & 1),
+                       kWaitLimitNs)) {
+          atomicOr(a.status, kFlagTimeout);
+          break;
+        }
+      }
+    }
+    return;
+  }
+
+  // ================= consumers
+  const int w = warp - 1;
+  const int ctid = tid - 32;
+  constexpr int NCT = NW * 32;
+  const int G = a.group;
+
+  // requests without keys: out = 0, lse = -inf (spread over blocks)
+  for (int b = c; b < B; b += P) {
+    if (s_len[b] != 0) continue;
+    const int nq = a.qo_heads * D;
+    for (int x = ctid; x < nq; x += NCT) {
+      a.out[static_cast<size_t>(b) * nq + x] = 0;
+      if (a.lse != nullptr && (x % D) == 0) a.lse[static_cast<size_t>(b) * a.qo_heads + x / D] = -CUDART_INF_F;
+    }
+  }
+
+  Cons cons;
+  long long i = 0;
+  bool alive = true;
+  Piece pc;
+  while (next_piece(it, pc, s_pre, s_len, B, H, a.window, T)) {
+    const int L = s_len[pc.b];
+    const int lo = (a.window > 0 && L > a.window) ? L - a.window : 0;
+    cons.begin_piece(a, pc.b, pc.h, lane);
+    for (int tt = pc.t0; tt < pc.t1; ++tt, ++i) {
+      if (static_cast<int>(i % NW) != w) continue;
+      const int stage = static_cast<int>(i % C::STAGES);
+      const uint32_t parity = static_cast<uint32_t>((i / C::STAGES) & 1);
+      if (alive) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(full0 + 8 * stage, parity, kWaitLimitNs);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) {
+          if (lane == 0) atomicOr(a.status, kFlagTimeout);
+          alive = false;
+        }
+      }
+      if (alive) {
+        const uint32_t kt = ring + stage * C::STAGE_BYTES;
+        cons.tile(a, kt, kt + C::TILE_BYTES, tt * T, lo, L, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8 * stage);
+      }
+    }
+    // ---- merge the warps' states of this piece
+    cons.end_piece(m_area, l_area, acc_area, w, lane);
+    named_barrier_sync(1, NCT);
+    const bool whole = pc.n_pieces == 1;
+    const int slot_idx = c + pc.seg;
+    const float vs = Cons::C::ES == 1 ? __ldg(a.v_scale + pc.h) : 1.f;
+    for (int x = ctid; x < G * D; x += NCT) {
+      const int h = x / D, dim = x - h * D;
+      float M = -CUDART_INF_F;
+#pragma unroll
+      for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, m_area[ww * Cons::GM + h]);
+      float Ls = 0.f, O = 0.f;
+      if (M != -CUDART_INF_F) {
+#pragma unroll
+        for (int ww = 0; ww < NW; ++ww) {
+          const float mw = m_area[ww * Cons::GM + h];
+          if (mw == -CUDART_INF_F) continue;
+          const float sc = exp2_approx(mw - M);
+          Ls = fmaf(l_area[ww * Cons::GM + h], sc, Ls);
+          O = fmaf(acc_area[(ww * Cons::GM + h) * D + dim], sc, O);
+        }
+      }
+      const bool empty = !(Ls > 0.f);
+      const float ov = empty ? 0.f : O / Ls * vs;
+      const float lv = empty ? -CUDART_INF_F : (M + __log2f(Ls)) * kLn2;
+      const size_t row = static_cast<size_t>(pc.b) * a.qo_heads + static_cast<size_t>(pc.h) * G + h;
+      if (whole) {
+        a.out[row * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(ov));
+        if (dim == 0 && a.lse != nullptr) a.lse[row] = lv;
+      } else {
+        a.part_o[(static_cast<size_t>(slot_idx) * G + h) * D + dim] = ov;
+        if (dim == 0) a.part_lse[static_cast<size_t>(slot_idx) * G + h] = lv;
+      }
+    }
+    if (!whole) {
+      __threadfence();
+      named_barrier_sync(1, NCT);
+      if (ctid == 0) {
+        const unsigned ticket = atomicInc(a.counters + pc.seg, static_cast<unsigned>(pc.n_pieces - 1));
+        *s_flag = (ticket == static_cast<unsigned>(pc.n_pieces - 1)) ? 1 : 0;
+      }
+      named_barrier_sync(1, NCT);
+      if (*s_flag) {
+        // last block of this segment: merge every block's (o, lse) exactly
+        __threadfence();
+        for (int x = ctid; x < G * D; x += NCT) {
+          const int h = x / D, dim = x - h * D;
+          float M = -CUDART_INF_F;
+          for (int k = 0; k < pc.n_pieces; ++k)
+            M = fmaxf(M, __ldcg(a.part_lse + static_cast<size_t>(pc.c_first + k + pc.seg) * G + h));
+          float Z = 0.f, O = 0.f;
+          if (M != -CUDART_INF_F) {
+            for (int k = 0; k < pc.n_pieces; ++k) {
+              const size_t sl = static_cast<size_t>(pc.c_first + k + pc.seg);
+              const float lk = __ldcg(a.part_lse + sl * G + h);
+              if (lk == -CUDART_INF_F) continue;
+              const float wgt = exp2_approx((lk - M) * kLog2e);
+              Z += wgt;
+              O = fmaf(wgt, __ldcg(a.part_o + (sl * G + h) * D + dim), O);
+            }
+          }
+          const bool empty = !(Z > 0.f);
+          const size_t row = static_cast<size_t>(pc.b) * a.qo_heads + static_cast<size_t>(pc.h) * G + h;
+          a.out[row * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(empty ? 0.f : O / Z));
+          if (dim == 0 && a.lse != nullptr) a.lse[row] = empty ? -CUDART_INF_F : M + __logf(Z);
+        }
+      }
+    }
+    named_barrier_sync(1, NCT);  // merge area is reused by the next piece
+  }
+}
+
+}  // namespace fa

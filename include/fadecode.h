@@ -42,6 +42,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -128,14 +134,14 @@ typedef struct {
  * FA_ERR_UNSUPPORTED (head_dim / group / dtype / path combination without a
  * kernel), FA_ERR_CUDA (num_sms == 0 and no device could be queried).
  */
-fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* kv_indptr_host,
+FA_API fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* kv_indptr_host,
                          int32_t num_sms, fa_plan** plan, size_t* workspace_bytes);
 
 /* Fills *info from a plan.  FA_ERR_INVALID_ARG on null pointers. */
-fa_status fa_plan_get_info(const fa_plan* plan, fa_plan_info_t* info);
+FA_API fa_status fa_plan_get_info(const fa_plan* plan, fa_plan_info_t* info);
 
 /* Releases a plan (NULL is a no-op). */
-void fa_plan_destroy(fa_plan* plan);
+FA_API void fa_plan_destroy(fa_plan* plan);
 
 /*
  * fa_decode_run -- enqueue one decode-attention pass on `stream`.
@@ -171,7 +177,7 @@ void fa_plan_destroy(fa_plan* plan);
  * FA_ERR_CUDA (launch failure).  Device-side checks are reported later by
  * fa_decode_status.
  */
-fa_status fa_decode_run(const fa_plan* plan, const void* q, const void* k, const void* v,
+FA_API fa_status fa_decode_run(const fa_plan* plan, const void* q, const void* k, const void* v,
                         int64_t kv_rows, const int32_t* page_table, int32_t page_table_stride,
                         const int32_t* kv_indptr, const float* k_scale, const float* v_scale,
                         void* out, float* lse, void* workspace, size_t workspace_bytes,
@@ -183,7 +189,7 @@ fa_status fa_decode_run(const fa_plan* plan, const void* q, const void* k, const
  * it.  Returns FA_ERR_DEVICE_CHECK when any bit was set, FA_ERR_CUDA when the
  * copy failed, else FA_OK.
  */
-fa_status fa_decode_status(void* workspace, size_t workspace_bytes, uint32_t* flags,
+FA_API fa_status fa_decode_status(void* workspace, size_t workspace_bytes, uint32_t* flags,
                            void* stream);
 
 /*
@@ -201,15 +207,15 @@ fa_status fa_decode_status(void* workspace, size_t workspace_bytes, uint32_t* fl
  * head_dim must be a multiple of 4 and <= 1024; o_parts, out 16-byte aligned.
  * Errors: FA_ERR_INVALID_ARG, FA_ERR_MISALIGNED, FA_ERR_CUDA.
  */
-fa_status fa_merge_states(const float* o_parts, const float* lse_parts, int32_t n, int32_t rows,
+FA_API fa_status fa_merge_states(const float* o_parts, const float* lse_parts, int32_t n, int32_t rows,
                           int32_t heads, int32_t head_dim, void* out, float* lse_out,
                           void* stream);
 
 /* Static description of a status code (never NULL). */
-const char* fa_status_string(fa_status status);
+FA_API const char* fa_status_string(fa_status status);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
-int32_t fa_version(void);
+FA_API int32_t fa_version(void);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,210 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+declared in include/fadecode.h, plans the workloads, and rejects bad
+arguments with the documented status codes before touching the device."""
+import ctypes
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+from gqa_decode_attention_split_b200 import binding, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fadecode.h")
+B200_SMS = 148
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gqa_decode_attention_split_b200 import build_lib
+    build_lib.build()
+    return binding.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(", text)
+
+
+def test_header_declares_the_entry_points():
+    names = set(declared_functions())
+    assert {"fa_decode_plan", "fa_decode_run", "fa_merge_states", "fa_plan_destroy",
+            "fa_plan_get_info", "fa_decode_status", "fa_status_string", "fa_version"} <= names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.fa_version() >= 100
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        s = lib.fa_status_string(code)
+        assert s and isinstance(s, bytes)
+    assert lib.fa_status_string(99) == b"unknown status"
+
+
+def _desc(**kw):
+    base = dict(batch=1, qo_heads=8, kv_heads=2, head_dim=128, kv_dtype=0, paged=0, page_size=0,
+                window=-1, sm_scale=1.0 / math.sqrt(128), path=0, num_ctas=0)
+    base.update(kw)
+    return binding.DecodeDesc(**base)
+
+
+def _plan(lib, desc, indptr, num_sms=B200_SMS):
+    ind = np.ascontiguousarray(indptr, dtype=np.int32)
+    h = ctypes.c_void_p()
+    ws = ctypes.c_size_t()
+    st = lib.fa_decode_plan(ctypes.byref(desc), ind.ctypes.data, num_sms, ctypes.byref(h),
+                            ctypes.byref(ws))
+    return st, h, ws.value
+
+
+def _info(lib, h):
+    inf = binding.PlanInfo()
+    assert lib.fa_plan_get_info(h, ctypes.byref(inf)) == 0
+    return inf
+
+
+@pytest.mark.parametrize("name", ["gqa4_d64_L512", "gemma3_1b_global_L8192",
+                                  "gemma3_1b_local_w512_L8192", "llama2_7b_mha_L32768"])
+def test_plans_for_named_workloads(lib, name):
+    spec = {"gqa4_d64_L512": (1, 8, 2, 64, [512], -1),
+            "gemma3_1b_global_L8192": (1, 4, 1, 256, [8192], -1),
+            "gemma3_1b_local_w512_L8192": (1, 4, 1, 256, [8192], 512),
+            "llama2_7b_mha_L32768": (1, 32, 32, 128, [32768], -1)}[name]
+    B, Hq, Hk, d, lens, w = spec
+    ind = np.concatenate([[0], np.cumsum(lens)])
+    st, h, ws = _plan(lib, _desc(batch=B, qo_heads=Hq, kv_heads=Hk, head_dim=d, window=w), ind)
+    assert st == 0
+    inf = _info(lib, h)
+    assert 1 <= inf.num_ctas <= B200_SMS
+    assert ws == inf.workspace_bytes and ws >= 256 and ws % 256 == 0
+    assert inf.smem_bytes <= 232448
+    T = inf.tile_tokens
+    L = lens[0]
+    lo = max(0, L - w) if w > 0 else 0
+    assert inf.total_tiles == Hk * ((L + T - 1) // T - lo // T)
+    lib.fa_plan_destroy(h)
+
+
+def test_plan_paged_and_fp8(lib):
+    lens = synth.c4_lengths()
+    ind = np.concatenate([[0], np.cumsum(lens)])
+    st, h, ws = _plan(lib, _desc(batch=64, qo_heads=32, kv_heads=8, paged=1, page_size=16), ind)
+    assert st == 0
+    inf = _info(lib, h)
+    assert inf.num_ctas == B200_SMS and inf.path == binding.PATH_MMA
+    assert inf.max_partials == B200_SMS + 64 * 8
+    lib.fa_plan_destroy(h)
+    st, h, ws = _plan(lib, _desc(qo_heads=64, kv_heads=8, kv_dtype=1), [0, 131072])
+    assert st == 0 and _info(lib, h).path == binding.PATH_MMA
+    lib.fa_plan_destroy(h)
+
+
+def test_forced_split_and_paths(lib):
+    for path in (binding.PATH_SIMT, binding.PATH_MMA):
+        for n in (1, 2, 7, 64):
+            st, h, _ = _plan(lib, _desc(path=path, num_ctas=n), [0, 1000])
+            assert st == 0
+            inf = _info(lib, h)
+            assert inf.num_ctas == n and inf.path == path
+            lib.fa_plan_destroy(h)
+
+
+@pytest.mark.parametrize("kw,indptr,code", [
+    (dict(qo_heads=6, kv_heads=4), [0, 10], 1),          # group not integral
+    (dict(batch=0), [0], 1),
+    (dict(head_dim=96), [0, 10], 2),                     # no kernel
+    (dict(kv_dtype=1, head_dim=64), [0, 10], 2),         # fp8 needs 128-byte rows
+    (dict(qo_heads=32, kv_heads=2, path=1), [0, 10], 2),  # SIMT group 16
+    (dict(qo_heads=32, kv_heads=2, path=2), [0, 10], 2),  # MMA group 16
+    (dict(paged=1, page_size=12), [0, 10], 1),           # not a power of two
+    (dict(paged=1, page_size=512), [0, 10], 1),
+    (dict(sm_scale=float("nan")), [0, 10], 1),
+    (dict(kv_dtype=3), [0, 10], 1),
+    (dict(path=7), [0, 10], 1),
+    (dict(num_ctas=-1), [0, 10], 1),
+    (dict(batch=2), [0, 10, 5], 1),                      # decreasing indptr
+    (dict(), [3, 10], 1),                                # indptr[0] != 0
+])
+def test_plan_rejects_bad_descriptions(lib, kw, indptr, code):
+    st, h, _ = _plan(lib, _desc(**kw), indptr)
+    assert st == code
+    assert not h.value
+
+
+def test_plan_null_arguments(lib):
+    d = _desc()
+    ind = np.array([0, 10], np.int32)
+    h = ctypes.c_void_p()
+    assert lib.fa_decode_plan(None, ind.ctypes.data, 148, ctypes.byref(h), None) == 1
+    assert lib.fa_decode_plan(ctypes.byref(d), None, 148, ctypes.byref(h), None) == 1
+    assert lib.fa_decode_plan(ctypes.byref(d), ind.ctypes.data, 148, None, None) == 1
+    assert lib.fa_plan_get_info(None, None) == 1
+    lib.fa_plan_destroy(None)
+
+
+def test_plan_without_device_needs_sm_count(lib):
+    st, h, _ = _plan(lib, _desc(), [0, 10], num_sms=0)
+    if st == 0:  # a device is present
+        lib.fa_plan_destroy(h)
+    else:
+        assert st == 5
+
+
+def test_run_validates_before_touching_the_device(lib):
+    st, h, ws = _plan(lib, _desc(batch=1, qo_heads=8, kv_heads=2, paged=1, page_size=16), [0, 100])
+    assert st == 0
+    good = 0x10000  # never dereferenced: every call below fails validation first
+    args = dict(q=good, k=good, v=good, rows=8, pt=good, pts=7, ind=good, ks=None, vs=None,
+                out=good, lse=good, ws=good, wsb=ws)
+
+    def run(**kw):
+        a = dict(args, **kw)
+        return lib.fa_decode_run(h, a["q"], a["k"], a["v"], a["rows"], a["pt"], a["pts"],
+                                 a["ind"], a["ks"], a["vs"], a["out"], a["lse"], a["ws"], a["wsb"],
+                                 None)
+
+    assert run(q=None) == 1
+    assert run(out=None) == 1
+    assert run(ind=None) == 1
+    assert run(pt=None) == 1
+    assert run(pts=0) == 1
+    assert run(rows=0) == 1
+    assert run(q=good + 8) == 4
+    assert run(out=good + 2) == 4
+    assert run(ws=good + 128) == 4
+    assert run(wsb=ws - 1) == 3
+    assert lib.fa_decode_run(None, good, good, good, 8, good, 7, good, None, None, good, good,
+                             good, ws, None) == 1
+    lib.fa_plan_destroy(h)
+    # fp8 needs both scales
+    st, h, ws = _plan(lib, _desc(kv_dtype=1), [0, 100])
+    assert st == 0
+    assert lib.fa_decode_run(h, good, good, good, 100, None, 0, good, None, good, good, good, good,
+                             ws, None) == 1
+    lib.fa_plan_destroy(h)
+
+
+def test_merge_states_validation(lib):
+    g = 0x10000
+    assert lib.fa_merge_states(None, g, 2, 1, 1, 128, g, g, None) == 1
+    assert lib.fa_merge_states(g, g, 0, 1, 1, 128, g, g, None) == 1
+    assert lib.fa_merge_states(g, g, 2, 1, 1, 126, g, g, None) == 1
+    assert lib.fa_merge_states(g + 4, g, 2, 1, 1, 128, g, g, None) == 4
+    assert lib.fa_merge_states(g, g, 2, 1, 1, 128, g + 8, g, None) == 4
+
+
+def test_binding_raises_without_library(monkeypatch, tmp_path):
+    monkeypatch.setenv("FADECODE_LIBRARY", str(tmp_path / "missing.so"))
+    saved = binding._lib
+    binding._lib = None
+    try:
+        with pytest.raises(binding.FadecodeError):
+            binding.load_library()
+    finally:
+        binding._lib = saved

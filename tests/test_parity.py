@@ -1,0 +1,220 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle,
+element by element, on seeded inputs.  Small cases span several KV tiles and
+a ragged tail; the full-size workloads run in the launch configuration the
+benchmark times and are checked on sampled (request, head) rows."""
+import zlib
+
+import numpy as np
+import pytest
+
+from gqa_decode_attention_split_b200 import binding, synth
+from gpu_util import DeviceInputs, assert_matches, run_gpu, to_numpy
+from oracle import oracle
+
+pytestmark = pytest.mark.gpu
+
+PATHS = ["simt", "mma"]
+
+
+def _has_path(x, path):
+    g = x.group
+    if path == "simt":
+        return g in (1, 2, 4, 8) and not (x.kv_dtype == "fp8_e4m3" and g == 8)
+    return g <= 8
+
+
+def _check(x, path="auto", num_ctas=0, what=""):
+    ref_out, ref_lse = oracle.decode_all(x)
+    out, lse, flags, info = run_gpu(x, path=path, num_ctas=num_ctas)
+    assert flags == 0, f"{what}: device flags {flags}"
+    assert_matches(out, lse, ref_out, ref_lse, what=f"{x.name} {path} ctas={num_ctas} {what}")
+    return out, lse, info
+
+
+SMALL = [
+    # (name, batch, qo, kv, d, lens, kw)
+    ("gqa4_d64", 1, 8, 2, 64, [517], {}),
+    ("mha_d128", 2, 4, 4, 128, [301, 77], {}),
+    ("gqa8_d128", 2, 16, 2, 128, [1000, 33], {}),
+    ("gqa4_d256", 1, 4, 1, 256, [777], {}),
+    ("gqa2_d128_win", 3, 4, 2, 128, [500, 37, 1], {"window": 45}),
+    ("gqa3_d128", 2, 6, 2, 128, [129, 300], {}),
+    ("gqa5_d64", 1, 5, 1, 64, [250], {}),
+    ("fp8_gqa8", 1, 16, 2, 128, [1111], {"kv_dtype": "fp8_e4m3"}),
+    ("fp8_gqa4_d256", 2, 8, 2, 256, [333, 64], {"kv_dtype": "fp8_e4m3"}),
+    ("fp8_mha", 1, 4, 4, 128, [257], {"kv_dtype": "fp8_e4m3", "window": 100}),
+    ("paged16_gqa4", 4, 8, 2, 128, [40, 16, 1, 300], {"paged": True, "page_size": 16}),
+    ("paged1_gqa4", 2, 8, 2, 128, [70, 9], {"paged": True, "page_size": 1}),
+    ("paged4_d64", 2, 8, 2, 64, [70, 33], {"paged": True, "page_size": 4}),
+    ("paged64_d256", 2, 4, 1, 256, [200, 65], {"paged": True, "page_size": 64}),
+    ("paged256_fp8", 2, 16, 2, 128, [600, 20], {"paged": True, "page_size": 256,
+                                                 "kv_dtype": "fp8_e4m3"}),
+    ("paged8_fp8_win", 3, 8, 8, 128, [90, 8, 150], {"paged": True, "page_size": 8,
+                                                     "kv_dtype": "fp8_e4m3", "window": 17}),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+@pytest.mark.parametrize("path", PATHS)
+def test_small_cases(case, path):
+    name, B, Hq, Hk, d, lens, kw = case
+    kw = dict(kw)
+    x = synth.generate(B, Hq, Hk, d, lens, seed=zlib.crc32(name.encode()) % 1000, name=name,
+                       unused_slot_fill="nan" if kw.get("paged") else None,
+                       extra_rows=0 if kw.get("paged") else 40, **kw)
+    if not _has_path(x, path):
+        pytest.skip("no kernel for this group on this path")
+    _check(x, path=path)
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_empty_and_degenerate_requests(path):
+    x = synth.generate(5, 8, 2, 128, [0, 1, 0, 17, 16], seed=21, extra_rows=16)
+    _check(x, path=path)
+    y = x.with_window(1)
+    _check(y, path=path, what="window 1")
+    z = synth.generate(2, 8, 2, 128, [0, 0], seed=22, extra_rows=8)
+    out, lse, flags, _ = run_gpu(z, path=path)
+    assert flags == 0 and (out == 0).all() and np.isneginf(lse).all()
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_forced_splits_agree(path):
+    """Splitting the KV sequence over more blocks, then merging, gives the
+    oracle's result at every granularity (one block up to one tile per block)."""
+    x = synth.generate(2, 8, 2, 128, [1500, 203], seed=23)
+    results = []
+    total = None
+    for n in (1, 2, 7, 64, 0):
+        out, lse, info = _check(x, path=path, num_ctas=n)
+        total = info["total_tiles"]
+        results.append((out, lse))
+    out, lse, info = _check(x, path=path, num_ctas=total)
+    results.append((out, lse))
+    for o, l in results[1:]:
+        assert np.abs(l - results[0][1]).max() <= 2e-5
+        assert np.abs(o - results[0][0]).max() <= 4e-3
+
+
+def test_paged_equals_contiguous_on_gpu():
+    x = synth.generate(3, 16, 2, 128, [250, 31, 1024], seed=24)
+    ps = 16
+    npg = [(int(L) + ps - 1) // ps for L in x.kv_lens]
+    perm = np.random.default_rng(5).permutation(sum(npg))
+    kp = np.full((sum(npg), ps, 2, 128), 0x7FC0, np.uint16)
+    vp = kp.copy()
+    pt = np.full((3, max(npg)), -1, np.int32)
+    off = 0
+    for b in range(3):
+        a = int(x.kv_indptr[b])
+        for t in range(int(x.kv_lens[b])):
+            kp[perm[off + t // ps], t % ps] = x.k[a + t]
+            vp[perm[off + t // ps], t % ps] = x.v[a + t]
+        pt[b, :npg[b]] = perm[off:off + npg[b]]
+        off += npg[b]
+    y = synth.DecodeInputs(**{**x.__dict__, "paged": True, "page_size": ps, "k": kp, "v": vp,
+                              "page_table": pt})
+    for path in PATHS:
+        o1, l1, f1, _ = run_gpu(x, path=path, num_ctas=5)
+        o2, l2, f2, _ = run_gpu(y, path=path, num_ctas=5)
+        assert f1 == 0 and f2 == 0
+        np.testing.assert_array_equal(o1, o2)
+        np.testing.assert_array_equal(l1, l2)
+
+
+def test_bad_page_id_is_flagged_not_read():
+    x = synth.generate(2, 8, 2, 128, [64, 64], paged=True, page_size=16, seed=25)
+    x.page_table[1, 2] = x.k.shape[0] + 5  # outside the pool
+    out, lse, flags, _ = run_gpu(x, path="mma")
+    assert flags & 1
+    ref_out, ref_lse = oracle.decode_all(synth.DecodeInputs(**{**x.__dict__, "batch": 1,
+                                                               "q": x.q[:1],
+                                                               "kv_indptr": x.kv_indptr[:2],
+                                                               "page_table": x.page_table[:1]}))
+    assert_matches(out[:1], lse[:1], ref_out, ref_lse, what="unaffected request")
+
+
+def test_lse_optional_and_workspace_reuse():
+    x = synth.generate(2, 8, 2, 128, [700, 900], seed=26)
+    dev = DeviceInputs(x)
+    p = dev.plan(num_ctas=16)
+    ws = p.new_workspace()
+    ref_out, ref_lse = oracle.decode_all(x)
+    for _ in range(3):  # counters return to zero after every call
+        out, lse = dev.run(p, workspace=ws)
+        o, l = to_numpy(out, lse)
+        assert_matches(o, l, ref_out, ref_lse, what="reuse")
+    out, lse = dev.run(p, workspace=ws, want_lse=False)
+    assert lse is None
+    o, _ = to_numpy(out, None)
+    assert_matches(o, None, ref_out, None, what="no lse")
+    assert binding.decode_status(ws) == 0
+
+
+def test_merge_states_kernel():
+    import torch
+    rng = np.random.default_rng(27)
+    n, rows, heads, d = 5, 3, 4, 128
+    o = rng.standard_normal((n, rows, heads, d)).astype(np.float32)
+    l = (3 * rng.standard_normal((n, rows, heads))).astype(np.float32)
+    l[1, 0, 0] = -np.inf
+    l[:, 2, 3] = -np.inf
+    ref_o, ref_l = oracle.merge(o.astype(np.float64), l.astype(np.float64))
+    out, lse = binding.merge_states(torch.from_numpy(o).cuda(), torch.from_numpy(l).cuda())
+    go, gl = to_numpy(out, lse)
+    assert_matches(go, gl, ref_o, ref_l, what="merge_states")
+    assert (go[2, 3] == 0).all() and np.isneginf(gl[2, 3])
+
+
+# ---------------------------------------------------------------- full size
+def _sample_rows(x, n, rng):
+    rows = rng.choice(x.batch * x.qo_heads, size=min(n, x.batch * x.qo_heads), replace=False)
+    return np.sort(rows)
+
+
+def _check_full(x, path="auto", nrows=48, seed=0):
+    dev = DeviceInputs(x)
+    p = dev.plan(path=path)
+    ws = p.new_workspace()
+    out, lse = dev.run(p, workspace=ws)
+    o, l = to_numpy(out, lse)
+    assert binding.decode_status(ws) == 0
+    rows = _sample_rows(x, nrows, np.random.default_rng(seed))
+    ref_o, ref_l = oracle.decode_rows(x, rows)
+    b, h = rows // x.qo_heads, rows % x.qo_heads
+    assert_matches(o[b, h], l[b, h], ref_o, ref_l, what=f"{x.name} {path} sampled")
+    return p.info()
+
+
+@pytest.mark.parametrize("name", ["gqa4_d64_L512", "gemma3_1b_global_L8192",
+                                  "gemma3_1b_local_w512_L8192", "llama2_7b_mha_L1024",
+                                  "llama2_7b_mha_L4096"])
+@pytest.mark.parametrize("path", PATHS)
+def test_full_size_small_workloads(name, path):
+    x = synth.workload(name)
+    ref_o, ref_l = oracle.decode_all(x)
+    out, lse, flags, _ = run_gpu(x, path=path)
+    assert flags == 0
+    assert_matches(out, lse, ref_o, ref_l, what=f"{name} {path}")
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_full_size_llama2_32k(path):
+    _check_full(synth.workload("llama2_7b_mha_L32768"), path=path, nrows=32)
+
+
+@pytest.fixture(scope="module")
+def paged_workload():
+    return synth.workload("paged_b64_gqa4_L512-16384")
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_full_size_batched_paged(paged_workload, path):
+    x = paged_workload
+    info = _check_full(x, path=path, nrows=96, seed=1)
+    assert info["num_ctas"] > 1
+
+
+@pytest.mark.parametrize("path", ["mma"])
+def test_full_size_fp8_long_context(path):
+    _check_full(synth.workload("fp8_gqa8_L131072"), path=path, nrows=24, seed=2)
