@@ -360,6 +360,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--profile", type=int, default=0,
+                    help="profiler driver: run --warmup steps, then N steps, print nothing")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -383,6 +385,12 @@ def main():
     x = synth.workload(args.workload)
     runner = Runner(x, path=args.path)
     stream = runner.stream
+    if args.profile:
+        for _ in range(args.warmup + args.profile):
+            runner.step()
+        torch.cuda.synchronize()
+        runner.check_status()
+        return
     for _ in range(args.warmup):
         runner.step()
     torch.cuda.synchronize()
@@ -427,33 +435,32 @@ def main():
     if rank == 0 and world == 1 and not args.no_sweep:
         sweep = {}
         flush = l2_flusher()
-        for name in SWEEP:
-            y = synth.workload(name)
-            r = Runner(y)
-            for _ in range(5):
-                r.step()
-            ms = per_launch_ms(r.step, 30, r.stream, flush=flush if y.kv_bytes() <= 256e6 else None)
-            med = statistics.median(ms)
-            r.check_status()
-            sweep[name] = {"us": round(med * 1e3, 2), "gbps": round(y.kv_bytes() / (med * 1e-3) / 1e9, 1),
-                           "frac": round(y.kv_bytes() / (med * 1e-3) / 1e9 / peak, 4),
-                           "tokens_per_s": round(y.batch / (med * 1e-3), 1),
-                           "path": "mma" if r.info["path"] == 2 else "simt",
-                           "ctas": r.info["num_ctas"], "kv_bytes": y.kv_bytes()}
-            del r
-            torch.cuda.empty_cache()
-        for path in ("simt", "mma"):
+        jobs = [(name, "auto") for name in SWEEP]
+        jobs += [(x.name, "simt"), (x.name, "mma"), ("fp8_gqa8_L131072", "mma"),
+                 ("llama2_7b_mha_L32768", "simt"), ("llama2_7b_mha_L32768", "mma")]
+        cache = {x.name: x}
+        for name, path in jobs:
+            key = name if path == "auto" else f"{name}[{path}]"
             try:
-                r = Runner(x, path=path)
-            except Exception:
-                continue
-            for _ in range(5):
-                r.step()
-            med = statistics.median(per_launch_ms(r.step, 30, r.stream))
-            sweep[f"{x.name}[{path}]"] = {"us": round(med * 1e3, 2),
-                                          "gbps": round(kv_bytes / (med * 1e-3) / 1e9, 1),
-                                          "frac": round(kv_bytes / (med * 1e-3) / 1e9 / peak, 4)}
-            del r
+                y = cache.get(name) or synth.workload(name)
+                cache = {x.name: x, name: y}
+                r = Runner(y, path=path)
+                for _ in range(5):
+                    r.step()
+                ms = per_launch_ms(r.step, 30, r.stream,
+                                   flush=flush if y.kv_bytes() <= 256e6 else None)
+                med = statistics.median(ms)
+                r.check_status()
+                gbps = y.kv_bytes() / (med * 1e-3) / 1e9
+                sweep[key] = {"us": round(med * 1e3, 2), "gbps": round(gbps, 1),
+                              "frac": round(gbps / peak, 4),
+                              "tokens_per_s": round(y.batch / (med * 1e-3), 1),
+                              "path": "mma" if r.info["path"] == 2 else "simt",
+                              "ctas": r.info["num_ctas"], "kv_bytes": y.kv_bytes()}
+                del r
+            except Exception as e:  # keep the headline line even if a sweep entry fails
+                sweep[key] = {"error": str(e)[:300]}
+            torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

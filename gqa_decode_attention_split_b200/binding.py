@@ -84,6 +84,8 @@ def load_library():
     lib.fa_merge_states.restype = ctypes.c_int
     lib.fa_status_string.argtypes = [ctypes.c_int]
     lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_last_error.argtypes = []
+    lib.fa_last_error.restype = ctypes.c_char_p
     lib.fa_version.argtypes = []
     lib.fa_version.restype = i32
     _lib = lib
@@ -93,7 +95,10 @@ def load_library():
 def _check(status: int, where: str):
     if status != FA_OK:
         lib = load_library()
-        raise FadecodeError(status, where, lib.fa_status_string(status).decode())
+        detail = lib.fa_status_string(status).decode()
+        if status == 5:
+            detail += f" [{lib.fa_last_error().decode()}]"
+        raise FadecodeError(status, where, detail)
 
 
 def _ptr(t) -> Optional[int]:

@@ -51,16 +51,23 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False,
+          checks: bool = False, out: str = None) -> str:
+    """Compile and link.  checks=True builds the self-checking variant
+    (-DFA_CHECKS: range/alignment checks on every shared-memory read, bulk
+    copy destination and global write, reported through the status word)."""
+    lib = out or LIB
+    if not force and out is None and not checks and up_to_date():
         return LIB
-    os.makedirs(BUILD, exist_ok=True)
-    os.makedirs(os.path.dirname(LIB), exist_ok=True)
+    build_dir = BUILD + ("_checks" if checks else "")
+    os.makedirs(build_dir, exist_ok=True)
+    os.makedirs(os.path.dirname(lib), exist_ok=True)
     nvcc = _nvcc()
+    extra = ["-DFA_CHECKS"] if checks else []
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
-        cmd = [nvcc, *NVCC_FLAGS, "-c", src, "-o", obj]
+        obj = os.path.join(build_dir, os.path.basename(src) + ".o")
+        cmd = [nvcc, *NVCC_FLAGS, *extra, "-c", src, "-o", obj]
         if ptxas_info:
             cmd += ["-Xptxas", "-v"]
         r = subprocess.run(cmd, capture_output=True, text=True)
@@ -73,14 +80,14 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     srcs = _sources()
     with ThreadPoolExecutor(max_workers=min(len(srcs), os.cpu_count() or 4)) as ex:
         objs = list(ex.map(compile_one, srcs))
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [nvcc, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp, *objs,
            "-Xcompiler", "-fPIC"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 def main():
@@ -88,8 +95,11 @@ def main():
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-v", "--verbose", action="store_true")
     ap.add_argument("--ptxas-info", action="store_true")
+    ap.add_argument("--checks", action="store_true", help="self-checking build (-DFA_CHECKS)")
+    ap.add_argument("--out", default=None, help="output path (default: lib/libfadecode.so)")
     args = ap.parse_args()
-    print(build(force=args.force, verbose=args.verbose, ptxas_info=args.ptxas_info))
+    print(build(force=args.force, verbose=args.verbose, ptxas_info=args.ptxas_info,
+                checks=args.checks, out=args.out))
 
 
 if __name__ == "__main__":

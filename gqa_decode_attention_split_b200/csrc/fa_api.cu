@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdio.h>
 #include <string.h>
 
 #include <mutex>
@@ -46,6 +47,16 @@ const KernelEntry* find_entry(int head_dim, int group, int fp8, int path) {
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Text of the last CUDA failure seen by a call on this thread.
+thread_local char g_last_error[256] = "";
+
+fa_status cuda_failure(const char* where, cudaError_t e) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", where, cudaGetErrorString(e),
+           static_cast<int>(e));
+  cudaGetLastError();  // clear a non-sticky error so the caller can continue
+  return FA_ERR_CUDA;
+}
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
 // dependency on libcuda).
@@ -129,11 +140,9 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   if (num_sms < 0) return FA_ERR_INVALID_ARG;
   if (num_sms == 0) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
-      cudaGetLastError();
-      return FA_ERR_CUDA;
-    }
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_failure("fa_decode_plan: SM count", e);
   }
   const int group = desc->qo_heads / desc->kv_heads;
   const int fp8 = desc->kv_dtype == FA_KV_FP8_E4M3 ? 1 : 0;
@@ -161,10 +170,15 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   if (desc->num_ctas > 0) {
     P = desc->num_ctas;
   } else {
-    // one block per SM (each holds a 128 KB tile ring); small problems use
-    // fewer blocks so that each streams at least half a ring of tiles.
-    const int64_t min_tiles = k->stages / 2 > 0 ? k->stages / 2 : 1;
-    const int64_t want = (tiles + min_tiles - 1) / min_tiles;
+    // One block per SM (each holds a ~170 KB tile ring).  Small problems use
+    // fewer blocks so that every consumer warp streams at least two tiles,
+    // and a segment is cut into at most kMaxPiecesPerSegment runs on average
+    // so that the last block's merge of the partial states stays short.
+    constexpr int64_t kMaxPiecesPerSegment = 32;
+    const int64_t min_tiles = 2 * (k->threads / 32 - 1);
+    int64_t want = (tiles + min_tiles - 1) / min_tiles;
+    const int64_t seg_cap = kMaxPiecesPerSegment * desc->batch * desc->kv_heads;
+    if (want > seg_cap) want = seg_cap;
     P = want < num_sms ? want : num_sms;
     if (P < 1) P = 1;
   }
@@ -191,7 +205,7 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   p->off_part_lse = off;
   off = align_up(off + sizeof(float) * static_cast<size_t>(p->max_partials) * group, 256);
   p->ws_bytes = off;
-  p->smem = k->smem_bytes(desc->batch);
+  p->smem = k->smem_bytes(desc->batch, group);
   if (p->smem > 232448) {
     delete p;
     return FA_ERR_UNSUPPORTED;  // batch too large for the per-block schedule arrays
@@ -220,7 +234,10 @@ namespace {
 
 fa_status make_kv_map(const fa_plan* p, const void* base, int64_t kv_rows, CUtensorMap* map) {
   EncodeTiledFn enc = encode_fn();
-  if (enc == nullptr) return FA_ERR_CUDA;
+  if (enc == nullptr) {
+    snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled unavailable");
+    return FA_ERR_CUDA;
+  }
   const fa_decode_desc& d = p->desc;
   const KernelEntry* k = p->kernel;
   const int es = d.kv_dtype == FA_KV_FP8_E4M3 ? 1 : 2;
@@ -251,7 +268,12 @@ fa_status make_kv_map(const fa_plan* p, const void* base, int64_t kv_rows, CUten
             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   }
-  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+  if (r != CUDA_SUCCESS) {
+    snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed (%d)",
+             static_cast<int>(r));
+    return FA_ERR_CUDA;
+  }
+  return FA_OK;
 }
 
 }  // namespace
@@ -295,6 +317,7 @@ extern "C" fa_status fa_decode_run(const fa_plan* plan, const void* q, const voi
   a.part_o = reinterpret_cast<float*>(ws + plan->off_part_o);
   a.part_lse = reinterpret_cast<float*>(ws + plan->off_part_lse);
   a.kv_rows = kv_rows;
+  a.max_partials = static_cast<int>(plan->max_partials);
   a.batch = d.batch;
   a.qo_heads = d.qo_heads;
   a.kv_heads = d.kv_heads;
@@ -309,10 +332,7 @@ extern "C" fa_status fa_decode_run(const fa_plan* plan, const void* q, const voi
 
   cudaError_t e = plan->kernel->launch(a, plan->num_ctas, plan->smem,
                                        static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return FA_ERR_CUDA;
-  }
+  if (e != cudaSuccess) return cuda_failure("fa_decode_run: launch", e);
   return FA_OK;
 }
 
@@ -321,18 +341,14 @@ extern "C" fa_status fa_decode_status(void* workspace, size_t workspace_bytes, u
   if (workspace == nullptr || flags == nullptr || workspace_bytes < 256) return FA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t h = 0;
-  if (cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-      cudaStreamSynchronize(s) != cudaSuccess) {
-    cudaGetLastError();
-    return FA_ERR_CUDA;
-  }
+  cudaError_t e = cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_failure("fa_decode_status: read", e);
   *flags = h;
   if (h != 0) {
-    if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), s) != cudaSuccess ||
-        cudaStreamSynchronize(s) != cudaSuccess) {
-      cudaGetLastError();
-      return FA_ERR_CUDA;
-    }
+    e = cudaMemsetAsync(workspace, 0, sizeof(uint32_t), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_failure("fa_decode_status: clear", e);
     return FA_ERR_DEVICE_CHECK;
   }
   return FA_OK;
@@ -406,7 +422,8 @@ extern "C" fa_status fa_merge_states(const float* o_parts, const float* lse_part
   fa_merge_states_kernel<<<static_cast<unsigned>(blocks), threads, 0,
                            static_cast<cudaStream_t>(stream)>>>(
       o_parts, lse_parts, n, rh, head_dim, static_cast<uint16_t*>(out), lse_out);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_failure("fa_merge_states: launch", e);
   return FA_OK;
 }
 
@@ -424,3 +441,5 @@ extern "C" const char* fa_status_string(fa_status s) {
 }
 
 extern "C" int32_t fa_version(void) { return 100; }
+
+extern "C" const char* fa_last_error(void) { return g_last_error; }

@@ -29,14 +29,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+// Tests the phase of `parity`; if it is not complete the thread is suspended
+// in hardware until it completes or about `hint_ns` pass (no busy polling).
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
@@ -48,14 +50,21 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 // Waits for the phase of `parity` to complete; gives up after limit_ns of
 // wall time and returns false (the caller records the timeout and unwinds).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  constexpr uint32_t kHintNs = 1000000;  // re-check the wall clock about every millisecond
+  if (mbar_try_wait(bar, parity, kHintNs)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity, kHintNs)) return true;
     if (global_timer_ns() - t0 > limit_ns) return false;
   }
+}
+
+// Raw 64-bit state of an mbarrier (phase, pending arrivals, pending bytes);
+// read only to describe a wait that gave up.
+__device__ __forceinline__ uint64_t mbar_raw_state(uint32_t bar) {
+  uint64_t v;
+  asm volatile("ld.shared.b64 %0, [%1];" : "=l"(v) : "r"(bar) : "memory");
+  return v;
 }
 
 // ------------------------------------------------------------ bulk tensor
@@ -166,8 +175,13 @@ __device__ __forceinline__ float exp2_approx(float x) {
   return y;
 }
 
+// Barrier over `nthreads` threads (a multiple of 32) of the block.  The
+// non-aligned form is used, and the warp is reconverged first, because
+// callers reach it after per-lane branches (the .aligned form, which
+// "bar.sync" denotes, is undefined for a diverged warp).
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+  __syncwarp();
+  asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 }  // namespace fa

@@ -29,8 +29,8 @@ cudaError_t launch_decode(const KernelArgs& args, int grid, size_t smem, cudaStr
 }
 
 template <class Cons>
-size_t smem_bytes_for(int batch) {
-  return SmemLayout<Cons>::bytes(batch);
+size_t smem_bytes_for(int batch, int group) {
+  return SmemLayout<Cons>::bytes(batch, group);
 }
 
 template <class Cons>

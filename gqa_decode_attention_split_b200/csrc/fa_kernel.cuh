@@ -33,7 +33,7 @@
 
 namespace fa {
 
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = 7;  // + 1 producer warp = 2 warps per SM sub-partition
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait, then give up
 constexpr float kRescaleSlack = 8.0f;               // log2 units
 constexpr float kLog2e = 1.4426950408889634f;
@@ -59,28 +59,47 @@ struct KernelArgs {
   float* part_o;
   float* part_lse;
   long long kv_rows;
+  int max_partials;
   int batch, qo_heads, kv_heads, group;
   int window;
   int paged, page_shift, pt_stride, box_t, swz;
   float score_scale;  // sm_scale * log2(e)
 };
 
+constexpr int kSmemPerBlock = 232448;  // 227 KB of shared memory per block (sm_100)
+constexpr int kSchedReserve = 8192;    // schedule arrays for up to 682 requests
+
 // Shared-memory tile geometry for one head_dim / element type.  A K (or V)
 // tile of T tokens is stored plane-major: [NP][T][CB] where a plane holds
 // CB = min(128, row bytes) bytes of every token row; with 128-byte rows the
 // 16-byte chunks of row r are XOR-swizzled by (r & 7) (TMA 128B swizzle).
-template <int D, bool FP8>
+// A tile is 4 KB of K (and 4 KB of V) for rows up to 256 bytes: T = 4096 /
+// row bytes tokens, at least 16.  The ring takes what is left of the block's
+// shared memory after the merge area for GMAX query heads, in a multiple of
+// the consumer-warp count: tile i uses stage i % STAGES and warp i % NW, so
+// every stage belongs to exactly one warp, which waits on it round after
+// round.  (A stage shared by two warps would let one warp wait for round r+1
+// while round r is still pending; an mbarrier parity wait cannot tell the two
+// apart and would pass early.)
+template <int D, bool FP8, int GMAX>
 struct TileCfg {
   static constexpr int ES = FP8 ? 1 : 2;
   static constexpr int ROWB = D * ES;
   static constexpr int CB = ROWB < 128 ? ROWB : 128;
   static constexpr int NP = ROWB / CB;
-  static constexpr int T = (4096 / ROWB) > 16 ? (4096 / ROWB) : 16;
+  static constexpr int T_RAW = 4096 / ROWB;
+  static constexpr int T = T_RAW < 16 ? 16 : (T_RAW > 64 ? 64 : T_RAW);
   static constexpr int TILE_BYTES = T * ROWB;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   static constexpr int NW = kConsumerWarps;
-  static constexpr int STAGES_RAW = (128 * 1024) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_RAW < NW ? NW : (STAGES_RAW / NW) * NW;
+  static constexpr int MERGE_BYTES = NW * GMAX * (D + 2) * 4;
+  static constexpr int RING_BUDGET = kSmemPerBlock - 1024 - kSchedReserve - 512 - MERGE_BYTES;
+  static constexpr int STAGES_RAW = RING_BUDGET / STAGE_BYTES;
+  static constexpr int STAGES_PER_WARP_RAW = STAGES_RAW / NW;
+  static constexpr int STAGES_PER_WARP = STAGES_PER_WARP_RAW > 3 ? 3 : STAGES_PER_WARP_RAW;
+  static constexpr int STAGES = NW * STAGES_PER_WARP;
+  static_assert(STAGES_PER_WARP >= 1, "every consumer warp needs a stage");
+  static_assert(STAGES % NW == 0, "a stage must belong to one consumer warp");
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
   static constexpr int THREADS = (NW + 1) * 32;
   static_assert(ROWB % 16 == 0, "rows must be whole 16-byte chunks");
@@ -88,6 +107,65 @@ struct TileCfg {
 
 __device__ __forceinline__ uint32_t swz_off(int row, int chunk, int swz) {
   return static_cast<uint32_t>(((chunk ^ (swz ? (row & 7) : 0)) << 4));
+}
+
+// A wait that gives up records where (first one wins) in words 8..15 of the
+// workspace header: site (1 producer/empty, 2 producer drain/full,
+// 3 consumer/full), block, warp, block-sequence tile index, stage, parity and
+// the barrier's raw 64-bit state.
+__device__ __noinline__ static void record_timeout(uint32_t* status, uint32_t site, int tile, int stage,
+                                                   uint32_t parity, uint32_t bar) {
+  atomicOr(status, kFlagTimeout);
+  if (atomicCAS(status + 8, 0u, site) == 0u) {
+    const uint64_t raw = mbar_raw_state(bar);
+    status[9] = blockIdx.x;
+    status[10] = threadIdx.x >> 5;
+    status[11] = static_cast<uint32_t>(tile);
+    status[12] = static_cast<uint32_t>(stage);
+    status[13] = parity;
+    status[14] = static_cast<uint32_t>(raw);
+    status[15] = static_cast<uint32_t>(raw >> 32);
+  }
+}
+
+// ------------------------------------------------------- debug checks
+// Built with -DFA_CHECKS, every shared-memory read, bulk-copy destination and
+// global write is range- and alignment-checked; a violation sets
+// kFlagCheck in the status word, records (code, block, thread, value) in the
+// next four words of the workspace header (first violation wins) and the
+// access is skipped.  Without FA_CHECKS the checks compile to nothing.
+constexpr uint32_t kFlagCheck = 8u;
+#ifdef FA_CHECKS
+static __device__ __noinline__ void check_fail(uint32_t* status, uint32_t code, long long value) {
+  atomicOr(status, kFlagCheck);
+  if (atomicCAS(status + 1, 0u, code) == 0u) {
+    status[2] = blockIdx.x;
+    status[3] = threadIdx.x;
+    status[4] = static_cast<uint32_t>(value);
+    status[5] = static_cast<uint32_t>(value >> 32);
+  }
+}
+#define FA_CHECK(status, cond, code, value) \
+  ((cond) ? true : (::fa::check_fail((status), (code), static_cast<long long>(value)), false))
+#else
+#define FA_CHECK(status, cond, code, value) true
+#endif
+// Shared-memory 16-byte load that stays inside [tile, tile + bytes).
+// Row address for a warp-collective ldmatrix: a bad address is replaced by
+// the tile base (the instruction must still be executed by every lane).
+__device__ __forceinline__ uint32_t ldsm_addr_in(uint32_t* status, uint32_t addr, uint32_t tile,
+                                                 uint32_t bytes, uint32_t code) {
+  return FA_CHECK(status, addr >= tile && addr + 16 <= tile + bytes && (addr & 15u) == 0, code,
+                  static_cast<long long>(addr) - tile)
+             ? addr
+             : tile;
+}
+__device__ __forceinline__ uint4 lds128_in(uint32_t* status, uint32_t addr, uint32_t tile,
+                                           uint32_t bytes, uint32_t code) {
+  if (!FA_CHECK(status, addr >= tile && addr + 16 <= tile + bytes && (addr & 15u) == 0, code,
+                static_cast<long long>(addr) - tile))
+    return make_uint4(0, 0, 0, 0);
+  return lds128(addr);
 }
 
 // ------------------------------------------------------------ schedule
@@ -154,8 +232,7 @@ __device__ __forceinline__ bool next_piece(PieceIter& it, Piece& pc, const int* 
 // running softmax state, merged across slots at the end of a segment piece.
 template <int D, int G, bool FP8>
 struct SimtConsumer {
-  using C = TileCfg<D, FP8>;
-  static constexpr int GM = G;  // merge-area heads
+  using C = TileCfg<D, FP8, G>;
   static constexpr int EPC = 16 / C::ES;
   static constexpr int NCH = C::ROWB / 16;
   static constexpr int E_TARGET = 64 / G;
@@ -235,77 +312,85 @@ struct SimtConsumer {
     }
   }
 
+  // A tile is processed in sub-steps of TPSC tokens per slot (bounded
+  // register use); each sub-step updates the slot's running softmax once.
+  static constexpr int TPSC = TPS < 4 ? TPS : 4;
+  static constexpr int NSUB = TPS / TPSC;
+  static_assert(TPS % TPSC == 0, "sub-steps");
+
   __device__ __forceinline__ void tile(const KernelArgs& a, uint32_t kt, uint32_t vt, int pos0,
                                        int lo, int hi, int lane) {
-    float s[TPS][G];
+#pragma unroll 1
+    for (int si = 0; si < NSUB; ++si) {
+      float s[TPSC][G];
 #pragma unroll
-    for (int tt = 0; tt < TPS; ++tt) {
-      const int r = tt * SLOTS + slot;
-      float part[G];
+      for (int tt = 0; tt < TPSC; ++tt) {
+        const int r = (si * TPSC + tt) * SLOTS + slot;
+        float part[G];
 #pragma unroll
-      for (int h = 0; h < G; ++h) part[h] = 0.f;
-#pragma unroll
-      for (int k = 0; k < CPL; ++k) {
-        float x[EPC];
-        convert(lds128(addr(kt, r, k, a.swz)), x);
-#pragma unroll
-        for (int h = 0; h < G; ++h)
-#pragma unroll
-          for (int e = 0; e < EPC; ++e) part[h] = fmaf(q[h][k * EPC + e], x[e], part[h]);
-      }
-#pragma unroll
-      for (int off = 1; off < LPT; off <<= 1)
-#pragma unroll
-        for (int h = 0; h < G; ++h) part[h] += __shfl_xor_sync(0xffffffffu, part[h], off);
-      const int pos = pos0 + r;
-      const bool valid = pos >= lo && pos < hi;
-#pragma unroll
-      for (int h = 0; h < G; ++h) s[tt][h] = valid ? part[h] : -CUDART_INF_F;
-    }
-    // running max with slack: rescale only when the tile max exceeds it by kRescaleSlack
-    bool need = false;
-    float tmax[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      tmax[h] = s[0][h];
-#pragma unroll
-      for (int tt = 1; tt < TPS; ++tt) tmax[h] = fmaxf(tmax[h], s[tt][h]);
-      need |= tmax[h] > m[h] + kRescaleSlack;
-    }
-    if (__any_sync(0xffffffffu, need)) {
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        if (tmax[h] > m[h] + kRescaleSlack) {
-          const float alpha = exp2_approx(m[h] - tmax[h]);  // m = -inf -> 0
-          l[h] *= alpha;
-#pragma unroll
-          for (int e = 0; e < E; ++e) acc[h][e] *= alpha;
-          m[h] = tmax[h];
-        }
-      }
-    }
-    float p[TPS][G];
-#pragma unroll
-    for (int tt = 0; tt < TPS; ++tt)
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        p[tt][h] = (m[h] == -CUDART_INF_F) ? 0.f : exp2_approx(s[tt][h] - m[h]);
-        l[h] += p[tt][h];
-      }
-#pragma unroll
-    for (int tt = 0; tt < TPS; ++tt) {
-      const int r = tt * SLOTS + slot;
-      const int pos = pos0 + r;
-      if (pos >= lo && pos < hi) {  // masked rows may hold anything: never read them as values
+        for (int h = 0; h < G; ++h) part[h] = 0.f;
 #pragma unroll
         for (int k = 0; k < CPL; ++k) {
           float x[EPC];
-          convert(lds128(addr(vt, r, k, a.swz)), x);
+          convert(lds128_in(a.status, addr(kt, r, k, a.swz), kt, C::TILE_BYTES, 101), x);
 #pragma unroll
           for (int h = 0; h < G; ++h)
 #pragma unroll
-            for (int e = 0; e < EPC; ++e)
-              acc[h][k * EPC + e] = fmaf(p[tt][h], x[e], acc[h][k * EPC + e]);
+            for (int e = 0; e < EPC; ++e) part[h] = fmaf(q[h][k * EPC + e], x[e], part[h]);
+        }
+#pragma unroll
+        for (int off = 1; off < LPT; off <<= 1)
+#pragma unroll
+          for (int h = 0; h < G; ++h) part[h] += __shfl_xor_sync(0xffffffffu, part[h], off);
+        const int pos = pos0 + r;
+        const bool valid = pos >= lo && pos < hi;
+#pragma unroll
+        for (int h = 0; h < G; ++h) s[tt][h] = valid ? part[h] : -CUDART_INF_F;
+      }
+      // running max with slack: rescale only when the max grows by more than kRescaleSlack
+      bool need = false;
+      float tmax[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        tmax[h] = s[0][h];
+#pragma unroll
+        for (int tt = 1; tt < TPSC; ++tt) tmax[h] = fmaxf(tmax[h], s[tt][h]);
+        need |= tmax[h] > m[h] + kRescaleSlack;
+      }
+      if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          if (tmax[h] > m[h] + kRescaleSlack) {
+            const float alpha = exp2_approx(m[h] - tmax[h]);  // m = -inf -> 0
+            l[h] *= alpha;
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc[h][e] *= alpha;
+            m[h] = tmax[h];
+          }
+        }
+      }
+#pragma unroll
+      for (int tt = 0; tt < TPSC; ++tt)
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          s[tt][h] = (m[h] == -CUDART_INF_F) ? 0.f : exp2_approx(s[tt][h] - m[h]);
+          l[h] += s[tt][h];
+        }
+#pragma unroll
+      for (int tt = 0; tt < TPSC; ++tt) {
+        const int r = (si * TPSC + tt) * SLOTS + slot;
+        const int pos = pos0 + r;
+        if (pos >= lo && pos < hi) {  // masked rows may hold anything: never read them as values
+#pragma unroll
+          for (int k = 0; k < CPL; ++k) {
+            float x[EPC];
+            convert(lds128_in(a.status, addr(vt, r, k, a.swz), vt, C::TILE_BYTES, 102), x);
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+#pragma unroll
+              for (int e = 0; e < EPC; ++e)
+                acc[h][k * EPC + e] = fmaf(s[tt][h], x[e], acc[h][k * EPC + e]);
+          }
         }
       }
     }
@@ -313,7 +398,7 @@ struct SimtConsumer {
 
   // Merge the slots' states and publish the warp's state.
   __device__ __forceinline__ void end_piece(float* m_area, float* l_area, float* acc_area, int w,
-                                            int lane) {
+                                            int lane, int /*group*/) {
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       float M = m[h];
@@ -331,14 +416,14 @@ struct SimtConsumer {
         acc[h][e] = v;
       }
       if (lane == 0) {
-        m_area[w * GM + h] = M;
-        l_area[w * GM + h] = lh;
+        m_area[w * G + h] = M;
+        l_area[w * G + h] = lh;
       }
       if (slot == 0) {
 #pragma unroll
         for (int k = 0; k < CPL; ++k)
 #pragma unroll
-          for (int e = 0; e < EPC; ++e) acc_area[(w * GM + h) * D + dim_of(k, e)] = acc[h][k * EPC + e];
+          for (int e = 0; e < EPC; ++e) acc_area[(w * G + h) * D + dim_of(k, e)] = acc[h][k * EPC + e];
       }
     }
   }
@@ -354,8 +439,7 @@ struct SimtConsumer {
 // into f16 range (the scale is undone on the fp32 scores).
 template <int D, bool FP8>
 struct MmaConsumer {
-  using C = TileCfg<D, FP8>;
-  static constexpr int GM = 8;
+  using C = TileCfg<D, FP8, 8>;
   static constexpr int KS = D / 16;     // k-steps of the score product = m-tiles of O^T
   static constexpr int SUB = C::T / 16;  // 16-token subtiles per tile
   static constexpr int BPT = D / 4;      // fp8 K: bytes of a row owned by one lane
@@ -430,7 +514,11 @@ struct MmaConsumer {
     return tile + (chunk >> 3) * (C::T * 128) + row * 128 + swz_off(row, chunk & 7, swz);
   }
 
-  __device__ __forceinline__ void scores(uint32_t kt, int sub, int lane, int swz, float (&c)[4]) const {
+  // Two accumulators (even / odd k-steps) halve the dependent chain of mma.
+  __device__ __forceinline__ void scores(const KernelArgs& a, uint32_t kt, int sub, int lane,
+                                         float (&c)[4]) const {
+    const int swz = a.swz;
+    float c2[4] = {0.f, 0.f, 0.f, 0.f};
     c[0] = c[1] = c[2] = c[3] = 0.f;
     if constexpr (!FP8) {
       const int row = sub * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
@@ -439,10 +527,13 @@ struct MmaConsumer {
         uint32_t af[4];
         const int ch = kk * 2 + (lane >> 4);
         if constexpr (C::CB == 128)
-          ldsm_x4(chunk_addr(kt, row, ch, swz), af);
+          ldsm_x4(ldsm_addr_in(a.status, chunk_addr(kt, row, ch, swz), kt, C::TILE_BYTES, 201), af);
         else  // 64-element rows: one plane of CB bytes, no swizzle
-          ldsm_x4(kt + row * C::CB + ch * 16, af);
-        mma_bf16(c, af, qb[kk][0], qb[kk][1]);
+          ldsm_x4(ldsm_addr_in(a.status, kt + row * C::CB + ch * 16, kt, C::TILE_BYTES, 202), af);
+        if (kk & 1)
+          mma_bf16(c2, af, qb[kk][0], qb[kk][1]);
+        else
+          mma_bf16(c, af, qb[kk][0], qb[kk][1]);
       }
     } else {
       const int r0 = sub * 16 + g, r1 = r0 + 8;
@@ -450,8 +541,8 @@ struct MmaConsumer {
 #pragma unroll
       for (int i = 0; i < BPT / 16; ++i) {
         const int ch = (BPT * t) / 16 + i;
-        const uint4 x0 = lds128(chunk_addr(kt, r0, ch, swz));
-        const uint4 x1 = lds128(chunk_addr(kt, r1, ch, swz));
+        const uint4 x0 = lds128_in(a.status, chunk_addr(kt, r0, ch, swz), kt, C::TILE_BYTES, 203);
+        const uint4 x1 = lds128_in(a.status, chunk_addr(kt, r1, ch, swz), kt, C::TILE_BYTES, 204);
         w0[4 * i] = x0.x; w0[4 * i + 1] = x0.y; w0[4 * i + 2] = x0.z; w0[4 * i + 3] = x0.w;
         w1[4 * i] = x1.x; w1[4 * i + 1] = x1.y; w1[4 * i + 2] = x1.z; w1[4 * i + 3] = x1.w;
       }
@@ -462,62 +553,88 @@ struct MmaConsumer {
         af[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[kk] & 0xFFFFu));
         af[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(w0[kk] >> 16));
         af[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[kk] >> 16));
-        mma_f16(c, af, qb[kk][0], qb[kk][1]);
+        if (kk & 1)
+          mma_f16(c2, af, qb[kk][0], qb[kk][1]);
+        else
+          mma_f16(c, af, qb[kk][0], qb[kk][1]);
       }
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) c[i] += c2[i];
   }
 
+  // One tile: the scores of all SUB subtiles first (independent mma chains),
+  // one softmax update for the whole tile, then O^T += V^T P^T per subtile.
   __device__ __forceinline__ void tile(const KernelArgs& a, uint32_t kt, uint32_t vt, int pos0,
                                        int lo, int hi, int lane) {
+    float sc[SUB][4];
+#pragma unroll
+    for (int sub = 0; sub < SUB; ++sub) scores(a, kt, sub, lane, sc[sub]);
+    float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F;
 #pragma unroll
     for (int sub = 0; sub < SUB; ++sub) {
-      float c[4];
-      scores(kt, sub, lane, a.swz, c);
       const int pr = pos0 + sub * 16 + g;
       const bool v0 = pr >= lo && pr < hi, v1 = pr + 8 >= lo && pr + 8 < hi;
-      const float s0 = v0 ? c[0] * sscale[0] : -CUDART_INF_F;
-      const float s1 = v0 ? c[1] * sscale[1] : -CUDART_INF_F;
-      const float s2 = v1 ? c[2] * sscale[0] : -CUDART_INF_F;
-      const float s3 = v1 ? c[3] * sscale[1] : -CUDART_INF_F;
-      float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+      sc[sub][0] = v0 ? sc[sub][0] * sscale[0] : -CUDART_INF_F;
+      sc[sub][1] = v0 ? sc[sub][1] * sscale[1] : -CUDART_INF_F;
+      sc[sub][2] = v1 ? sc[sub][2] * sscale[0] : -CUDART_INF_F;
+      sc[sub][3] = v1 ? sc[sub][3] * sscale[1] : -CUDART_INF_F;
+      mx0 = fmaxf(mx0, fmaxf(sc[sub][0], sc[sub][2]));
+      mx1 = fmaxf(mx1, fmaxf(sc[sub][1], sc[sub][3]));
+    }
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-      }
-      const bool up0 = mx0 > m[0] + kRescaleSlack, up1 = mx1 > m[1] + kRescaleSlack;
-      if (__any_sync(0xffffffffu, up0 || up1)) {
-        const float a0 = up0 ? exp2_approx(m[0] - mx0) : 1.f;
-        const float a1 = up1 ? exp2_approx(m[1] - mx1) : 1.f;
-        if (up0) m[0] = mx0;
-        if (up1) m[1] = mx1;
-        l[0] *= a0;
-        l[1] *= a1;
+    for (int off = 4; off < 32; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    const bool up0 = mx0 > m[0] + kRescaleSlack, up1 = mx1 > m[1] + kRescaleSlack;
+    if (__any_sync(0xffffffffu, up0 || up1)) {
+      const float a0 = up0 ? exp2_approx(m[0] - mx0) : 1.f;
+      const float a1 = up1 ? exp2_approx(m[1] - mx1) : 1.f;
+      if (up0) m[0] = mx0;
+      if (up1) m[1] = mx1;
+      l[0] *= a0;
+      l[1] *= a1;
 #pragma unroll
-        for (int mt = 0; mt < KS; ++mt) {
-          o[mt][0] *= a0;
-          o[mt][1] *= a1;
-          o[mt][2] *= a0;
-          o[mt][3] *= a1;
-        }
+      for (int mt = 0; mt < KS; ++mt) {
+        o[mt][0] *= a0;
+        o[mt][1] *= a1;
+        o[mt][2] *= a0;
+        o[mt][3] *= a1;
       }
-      const bool dead0 = m[0] == -CUDART_INF_F, dead1 = m[1] == -CUDART_INF_F;
-      const float p0 = dead0 ? 0.f : exp2_approx(s0 - m[0]);
-      const float p1 = dead1 ? 0.f : exp2_approx(s1 - m[1]);
-      const float p2 = dead0 ? 0.f : exp2_approx(s2 - m[0]);
-      const float p3 = dead1 ? 0.f : exp2_approx(s3 - m[1]);
+    }
+    const bool dead0 = m[0] == -CUDART_INF_F, dead1 = m[1] == -CUDART_INF_F;
+    // P enters the tensor core as hi + lo 16-bit parts (two products), so the
+    // weights keep ~16 significant bits instead of 8 (bf16) or 11 (f16).
+    uint32_t pb[SUB][4];
+#pragma unroll
+    for (int sub = 0; sub < SUB; ++sub) {
+      const float p0 = dead0 ? 0.f : exp2_approx(sc[sub][0] - m[0]);
+      const float p1 = dead1 ? 0.f : exp2_approx(sc[sub][1] - m[1]);
+      const float p2 = dead0 ? 0.f : exp2_approx(sc[sub][2] - m[0]);
+      const float p3 = dead1 ? 0.f : exp2_approx(sc[sub][3] - m[1]);
       l[0] += p0 + p2;
       l[1] += p1 + p3;
-      uint32_t x0, x1;
+      uint32_t x0, x1, y0, y1;
       if constexpr (FP8) {
         x0 = pack_f16x2(p0, p1);
         x1 = pack_f16x2(p2, p3);
+        const float2 h0 = f16x2_to_float2(x0), h1 = f16x2_to_float2(x1);
+        y0 = pack_f16x2(p0 - h0.x, p1 - h0.y);
+        y1 = pack_f16x2(p2 - h1.x, p3 - h1.y);
       } else {
         x0 = pack_bf16x2(p0, p1);
         x1 = pack_bf16x2(p2, p3);
+        y0 = pack_bf16x2(p0 - bf16lo(x0), p1 - bf16hi(x0));
+        y1 = pack_bf16x2(p2 - bf16lo(x1), p3 - bf16hi(x1));
       }
-      const uint32_t pb0 = movmatrix_trans(x0);  // P[head g][tokens 2t, 2t+1]
-      const uint32_t pb1 = movmatrix_trans(x1);  // P[head g][tokens 2t+8, 2t+9]
+      pb[sub][0] = movmatrix_trans(x0);  // P[head g][tokens 2t, 2t+1]
+      pb[sub][1] = movmatrix_trans(x1);  // P[head g][tokens 2t+8, 2t+9]
+      pb[sub][2] = movmatrix_trans(y0);
+      pb[sub][3] = movmatrix_trans(y1);
+    }
+#pragma unroll
+    for (int sub = 0; sub < SUB; ++sub) {
       // rows that are not visible may hold anything (NaN included): zero them in V
       const int pt = pos0 + sub * 16 + 2 * t;
       const bool e0 = pt >= lo && pt < hi, e1 = pt + 1 >= lo && pt + 1 < hi;
@@ -532,16 +649,17 @@ struct MmaConsumer {
           uint32_t af[4];
           const int ch = mt * 2 + ((lane >> 3) & 1);
           if constexpr (C::CB == 128)
-            ldsm_x4_trans(chunk_addr(vt, vrow, ch, a.swz), af);
+            ldsm_x4_trans(ldsm_addr_in(a.status, chunk_addr(vt, vrow, ch, a.swz), vt, C::TILE_BYTES, 205), af);
           else
-            ldsm_x4_trans(vt + vrow * C::CB + ch * 16, af);
+            ldsm_x4_trans(ldsm_addr_in(a.status, vt + vrow * C::CB + ch * 16, vt, C::TILE_BYTES, 206), af);
           if (edge) {
             af[0] &= mk01;
             af[1] &= mk01;
             af[2] &= mk89;
             af[3] &= mk89;
           }
-          mma_bf16(o[mt], af, pb0, pb1);
+          mma_bf16(o[mt], af, pb[sub][0], pb[sub][1]);
+          mma_bf16(o[mt], af, pb[sub][2], pb[sub][3]);
         }
       } else {
         // lane owns dims [VBT*g, VBT*g + VBT) of tokens 2t, 2t+1, 2t+8, 2t+9
@@ -552,7 +670,8 @@ struct MmaConsumer {
         for (int rr = 0; rr < 4; ++rr)
 #pragma unroll
           for (int i = 0; i < VBT / 16; ++i) {
-            const uint4 x = lds128(chunk_addr(vt, rows[rr], (VBT * g) / 16 + i, a.swz));
+            const uint4 x = lds128_in(a.status, chunk_addr(vt, rows[rr], (VBT * g) / 16 + i, a.swz), vt,
+                                      C::TILE_BYTES, 207);
             vw[rr][4 * i] = x.x;
             vw[rr][4 * i + 1] = x.y;
             vw[rr][4 * i + 2] = x.z;
@@ -574,7 +693,8 @@ struct MmaConsumer {
             af[2] &= mk89;
             af[3] &= mk89;
           }
-          mma_f16(o[mt], af, pb0, pb1);
+          mma_f16(o[mt], af, pb[sub][0], pb[sub][1]);
+          mma_f16(o[mt], af, pb[sub][2], pb[sub][3]);
         }
       }
     }
@@ -588,7 +708,7 @@ struct MmaConsumer {
   }
 
   __device__ __forceinline__ void end_piece(float* m_area, float* l_area, float* acc_area, int w,
-                                            int lane) {
+                                            int lane, int G) {
     float l0 = l[0], l1 = l[1];
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
@@ -596,34 +716,45 @@ struct MmaConsumer {
       l1 += __shfl_xor_sync(0xffffffffu, l1, off);
     }
     const int h0 = 2 * t, h1 = 2 * t + 1;
+    const bool r0 = h0 < G, r1 = h1 < G;
     if (g == 0) {
-      m_area[w * GM + h0] = m[0];
-      m_area[w * GM + h1] = m[1];
-      l_area[w * GM + h0] = l0;
-      l_area[w * GM + h1] = l1;
+      if (r0) m_area[w * G + h0] = m[0];
+      if (r1) m_area[w * G + h1] = m[1];
+      if (r0) l_area[w * G + h0] = l0;
+      if (r1) l_area[w * G + h1] = l1;
     }
 #pragma unroll
     for (int mt = 0; mt < KS; ++mt) {
-      acc_area[(w * GM + h0) * D + out_dim(mt, 0)] = o[mt][0];
-      acc_area[(w * GM + h1) * D + out_dim(mt, 0)] = o[mt][1];
-      acc_area[(w * GM + h0) * D + out_dim(mt, 1)] = o[mt][2];
-      acc_area[(w * GM + h1) * D + out_dim(mt, 1)] = o[mt][3];
+      if (r0) {
+        acc_area[(w * G + h0) * D + out_dim(mt, 0)] = o[mt][0];
+        acc_area[(w * G + h0) * D + out_dim(mt, 1)] = o[mt][2];
+      }
+      if (r1) {
+        acc_area[(w * G + h1) * D + out_dim(mt, 0)] = o[mt][1];
+        acc_area[(w * G + h1) * D + out_dim(mt, 1)] = o[mt][3];
+      }
     }
   }
 };
 
 // ------------------------------------------------------------- kernel
+// Block shared memory, from a 1024-aligned base:
+//   ring [STAGES][K tile, V tile] | full[STAGES], empty[STAGES] mbarriers |
+//   m[NW][G], l[NW][G] | acc[NW][G][D] | flag | pages[64] | start[B], len[B], pre[B+1]
 template <class Cons>
 struct SmemLayout {
   using C = typename Cons::C;
   static constexpr int D = C::ROWB / C::ES;
-  static constexpr int kBars = C::RING_BYTES;                        // full[S], empty[S]
-  static constexpr int kMerge = kBars + 2 * C::STAGES * 8;           // m[NW][GM], l[NW][GM]
-  static constexpr int kAccOff = kMerge + C::NW * Cons::GM * 2 * 4;  // acc[NW][GM][D]
-  static constexpr int kMisc = kAccOff + C::NW * Cons::GM * D * 4;   // ticket flag
-  static constexpr int kSched = kMisc + 16;                          // start[B] len[B] pre[B+1]
-  static constexpr size_t bytes(int batch) {
-    return 1024 + static_cast<size_t>(kSched) + static_cast<size_t>(3 * batch + 1) * 4;
+  static constexpr int kBars = C::RING_BYTES;
+  static constexpr int kMerge = kBars + 2 * C::STAGES * 8;
+  __host__ __device__ static constexpr int acc_off(int G) {
+    return kMerge + ((C::NW * G * 2 * 4 + 15) / 16) * 16;
+  }
+  __host__ __device__ static constexpr int misc_off(int G) { return acc_off(G) + C::NW * G * D * 4; }
+  // misc: ticket flag (16 B), then 64 staged page ids (256 B)
+  __host__ __device__ static constexpr int sched_off(int G) { return misc_off(G) + 16 + 256; }
+  static constexpr size_t bytes(int batch, int G) {
+    return 1024 + static_cast<size_t>(sched_off(G)) + static_cast<size_t>(3 * batch + 1) * 4;
   }
 };
 
@@ -642,11 +773,13 @@ __global__ void __maxnreg__(224)
   const uint32_t ring = sbase;
   const uint32_t full0 = sbase + S::kBars;
   const uint32_t empty0 = full0 + C::STAGES * 8;
+  const int G = a.group;
   float* m_area = reinterpret_cast<float*>(base + S::kMerge);
-  float* l_area = m_area + NW * Cons::GM;
-  float* acc_area = reinterpret_cast<float*>(base + S::kAccOff);
-  int* s_flag = reinterpret_cast<int*>(base + S::kMisc);
-  int* s_start = reinterpret_cast<int*>(base + S::kSched);
+  float* l_area = m_area + NW * G;
+  float* acc_area = reinterpret_cast<float*>(base + S::acc_off(G));
+  int* s_flag = reinterpret_cast<int*>(base + S::misc_off(G));
+  int* s_pages = s_flag + 4;
+  int* s_start = reinterpret_cast<int*>(base + S::sched_off(G));
   const int B = a.batch, H = a.kv_heads;
   int* s_len = s_start + B;
   int* s_pre = s_len + B;
@@ -706,82 +839,112 @@ __global__ void __maxnreg__(224)
   it.u1 = it.u + it.per < N ? it.u + it.per : N;
 
   if (warp == 0) {
-    // ================= producer: one elected lane issues the copies
+    // ================= producer
+    // Lane 0 walks the block's tiles in order and, per tile, waits for its
+    // ring stage to be free, arms the stage's barrier with the tile's bytes
+    // and issues the bulk tensor copies.  For paged KV the whole warp first
+    // stages the page ids of the next window of tiles in shared memory
+    // (coalesced reads of the page table), so lane 0's loop has no global
+    // loads and no warp-wide operations.
     const uint64_t pol = l2_evict_first_policy();
     if (lane == 0) {
       prefetch_tensormap(&a.kmap);
       prefetch_tensormap(&a.vmap);
     }
-    const int NB = T / a.box_t;  // copies per plane per tile (paged: one per page)
-    long long i = 0;
+    const int NB = T / a.box_t;  // boxes per tile (paged: one page each, contiguous: 1)
+    int stage = 0;
+    uint32_t ph = 0;             // lane 0's ring position (stage, wrap parity)
+    int issued = 0;
     bool ok = true;
     Piece pc;
     while (ok && next_piece(it, pc, s_pre, s_len, B, H, a.window, T)) {
       const int L = s_len[pc.b];
-      const int npages = a.paged ? (L + ps - 1) >> a.page_shift : 0;
-      int cache_base = -(1 << 30), cache_val = -1;
-      for (int tt = pc.t0; tt < pc.t1 && ok; ++tt, ++i) {
-        const int stage = static_cast<int>(i % C::STAGES);
-        const uint32_t parity = static_cast<uint32_t>((i / C::STAGES) & 1) ^ 1u;
-        const uint32_t fb = full0 + 8 * stage;
-        const uint32_t kdst = ring + stage * C::STAGE_BYTES;
-        const uint32_t vdst = kdst + C::TILE_BYTES;
+      // tiles per window of 64 staged page ids (a window that starts inside a
+      // page may touch one page more than its token count suggests)
+      const int tiles_per_win = a.paged ? (ps >= T ? 63 * (ps / T) : (64 * ps) / T) : (pc.t1 - pc.t0);
+      for (int w0 = pc.t0; w0 < pc.t1 && ok; w0 += tiles_per_win) {
+        const int w1 = w0 + tiles_per_win < pc.t1 ? w0 + tiles_per_win : pc.t1;
+        int pbase = 0, npages = 0;
+        if (a.paged) {
+          npages = (L + ps - 1) >> a.page_shift;
+          pbase = (w0 * T) >> a.page_shift;
+          __syncwarp();
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int e = pbase + half * 32 + lane;
+            int v = -1;
+            if (e < npages) {
+              v = __ldg(a.page_table + static_cast<long long>(pc.b) * a.pt_stride + e);
+              if (v < 0 || static_cast<long long>(v) >= a.kv_rows) {
+                atomicOr(a.status, kFlagBadPage);
+                v = -1;  // the copy reads out of range: zeros, no memory access
+              }
+            }
+            s_pages[half * 32 + lane] = v;
+          }
+          __syncwarp();
+        }
         if (lane == 0) {
-          if (!mbar_wait(empty0 + 8 * stage, parity, kWaitLimitNs)) {
-            atomicOr(a.status, kFlagTimeout);
-            ok = false;
-          } else {
+          for (int tt = w0; tt < w1; ++tt) {
+            if (!mbar_wait(empty0 + 8 * stage, ph ^ 1u, kWaitLimitNs)) {
+              record_timeout(a.status, 1, issued, stage, ph ^ 1u, empty0 + 8 * stage);
+              ok = false;
+              break;
+            }
+            const uint32_t fb = full0 + 8 * stage;
+            const uint32_t kdst = ring + stage * C::STAGE_BYTES;
+            const uint32_t vdst = kdst + C::TILE_BYTES;
             mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+            if (!a.paged) {
+              const int row = s_start[pc.b] + tt * T;
+#pragma unroll
+              for (int p = 0; p < C::NP; ++p) {
+                const uint32_t off = p * (T * C::CB);
+                if (FA_CHECK(a.status, off + T * C::CB <= C::TILE_BYTES && (off & 127u) == 0, 301, off)) {
+                  tma_load_3d(kdst + off, &a.kmap, fb, p * (C::CB / C::ES), pc.h, row, pol);
+                  tma_load_3d(vdst + off, &a.vmap, fb, p * (C::CB / C::ES), pc.h, row, pol);
+                }
+              }
+            } else {
+              for (int jb = 0; jb < NB; ++jb) {
+                const int tok = tt * T + jb * a.box_t;
+                const int pidx = tok >> a.page_shift;
+                const int page = (pidx < npages && pidx - pbase < 64) ? s_pages[pidx - pbase] : -1;
+                const int slot0 = tok & (ps - 1);
+#pragma unroll
+                for (int p = 0; p < C::NP; ++p) {
+                  const uint32_t off = p * (T * C::CB) + jb * a.box_t * C::CB;
+                  if (FA_CHECK(a.status, off + a.box_t * C::CB <= C::TILE_BYTES && (off & 127u) == 0 &&
+                                             pidx - pbase >= 0 && pidx - pbase < 64,
+                               302, off)) {
+                    tma_load_4d(kdst + off, &a.kmap, fb, p * (C::CB / C::ES), pc.h, slot0, page, pol);
+                    tma_load_4d(vdst + off, &a.vmap, fb, p * (C::CB / C::ES), pc.h, slot0, page, pol);
+                  }
+                }
+              }
+            }
+            ++issued;
+            if (++stage == C::STAGES) {
+              stage = 0;
+              ph ^= 1u;
+            }
           }
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        if (!ok) break;
-        if (!a.paged) {
-          if (lane == 0) {
-            const int row = s_start[pc.b] + tt * T;
-#pragma unroll
-            for (int p = 0; p < C::NP; ++p) {
-              tma_load_3d(kdst + p * (T * C::CB), &a.kmap, fb, p * (C::CB / C::ES), pc.h, row, pol);
-              tma_load_3d(vdst + p * (T * C::CB), &a.vmap, fb, p * (C::CB / C::ES), pc.h, row, pol);
-            }
-          }
-        } else {
-          for (int jb = 0; jb < NB; ++jb) {
-            const int tok = tt * T + jb * a.box_t;
-            const int pidx = tok >> a.page_shift;
-            if (pidx < cache_base || pidx - cache_base >= 32) {
-              cache_base = pidx;
-              const int e = cache_base + lane;
-              cache_val = -1;
-              if (e < npages) {
-                cache_val = __ldg(a.page_table + static_cast<long long>(pc.b) * a.pt_stride + e);
-                if (cache_val < 0 || static_cast<long long>(cache_val) >= a.kv_rows)
-                  atomicOr(a.status, kFlagBadPage);
-              }
-            }
-            int page = __shfl_sync(0xffffffffu, cache_val, pidx - cache_base);
-            if (pidx >= npages || page < 0) page = -1;  // out of range: the copy fills zeros
-            if (lane == 0) {
-              const int slot0 = tok & (ps - 1);
-#pragma unroll
-              for (int p = 0; p < C::NP; ++p) {
-                const uint32_t off = p * (T * C::CB) + jb * a.box_t * C::CB;
-                tma_load_4d(kdst + off, &a.kmap, fb, p * (C::CB / C::ES), pc.h, slot0, page, pol);
-                tma_load_4d(vdst + off, &a.vmap, fb, p * (C::CB / C::ES), pc.h, slot0, page, pol);
-              }
-            }
-          }
-        }
       }
     }
     // drain: every issued copy has landed before the block may exit
     if (lane == 0) {
-      const long long first = i > C::STAGES ? i - C::STAGES : 0;
-      for (long long k = first; k < i; ++k) {
-        const int stage = static_cast<int>(k % C::STAGES);
-        if (!mbar_wait(full0 + 8 * stage, static_cast<uint32_t>((k / C::STAGES) & 1),
-                       kWaitLimitNs)) {
-          atomicOr(a.status, kFlagTimeout);
+      const int n = issued < C::STAGES ? issued : C::STAGES;
+      for (int k = 1; k <= n; ++k) {
+        int st = stage - k;
+        uint32_t par = ph;
+        if (st < 0) {
+          st += C::STAGES;
+          par ^= 1u;
+        }
+        if (!mbar_wait(full0 + 8 * st, par, kWaitLimitNs)) {
+          record_timeout(a.status, 2, issued - k, st, par, full0 + 8 * st);
           break;
         }
       }
@@ -793,7 +956,6 @@ __global__ void __maxnreg__(224)
   const int w = warp - 1;
   const int ctid = tid - 32;
   constexpr int NCT = NW * 32;
-  const int G = a.group;
 
   // requests without keys: out = 0, lse = -inf (spread over blocks)
   for (int b = c; b < B; b += P) {
@@ -805,36 +967,45 @@ __global__ void __maxnreg__(224)
     }
   }
 
+  // Tile i of the block's sequence lives in stage i % STAGES and is consumed
+  // by warp i % NW (STAGES is a multiple of NW, so each stage has one owner
+  // warp that waits on it in order); each warp tracks its next tile and that
+  // tile's stage.
   Cons cons;
-  long long i = 0;
+  int next = w;          // next tile index (block sequence) of this warp
+  int stage = w;         // its stage (STAGES >= NW)
+  uint32_t ph = 0;       // wrap parity of that stage
+  int base_i = 0;        // block-sequence index of the current piece's first tile
   bool alive = true;
   Piece pc;
   while (next_piece(it, pc, s_pre, s_len, B, H, a.window, T)) {
     const int L = s_len[pc.b];
     const int lo = (a.window > 0 && L > a.window) ? L - a.window : 0;
+    const int n = pc.t1 - pc.t0;
     cons.begin_piece(a, pc.b, pc.h, lane);
-    for (int tt = pc.t0; tt < pc.t1; ++tt, ++i) {
-      if (static_cast<int>(i % NW) != w) continue;
-      const int stage = static_cast<int>(i % C::STAGES);
-      const uint32_t parity = static_cast<uint32_t>((i / C::STAGES) & 1);
+    for (; next < base_i + n; next += NW) {
       if (alive) {
-        bool ok = true;
-        if (lane == 0) ok = mbar_wait(full0 + 8 * stage, parity, kWaitLimitNs);
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(full0 + 8 * stage, ph, kWaitLimitNs));
         if (!ok) {
-          if (lane == 0) atomicOr(a.status, kFlagTimeout);
+          if (lane == 0) record_timeout(a.status, 3, next, stage, ph, full0 + 8 * stage);
           alive = false;
         }
       }
       if (alive) {
         const uint32_t kt = ring + stage * C::STAGE_BYTES;
-        cons.tile(a, kt, kt + C::TILE_BYTES, tt * T, lo, L, lane);
+        cons.tile(a, kt, kt + C::TILE_BYTES, (pc.t0 + next - base_i) * T, lo, L, lane);
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * stage);
       }
+      stage += NW;
+      if (stage >= C::STAGES) {
+        stage -= C::STAGES;
+        ph ^= 1u;
+      }
     }
+    base_i += n;
     // ---- merge the warps' states of this piece
-    cons.end_piece(m_area, l_area, acc_area, w, lane);
+    cons.end_piece(m_area, l_area, acc_area, w, lane, G);
     named_barrier_sync(1, NCT);
     const bool whole = pc.n_pieces == 1;
     const int slot_idx = c + pc.seg;
@@ -843,16 +1014,16 @@ __global__ void __maxnreg__(224)
       const int h = x / D, dim = x - h * D;
       float M = -CUDART_INF_F;
 #pragma unroll
-      for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, m_area[ww * Cons::GM + h]);
+      for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, m_area[ww * G + h]);
       float Ls = 0.f, O = 0.f;
       if (M != -CUDART_INF_F) {
 #pragma unroll
         for (int ww = 0; ww < NW; ++ww) {
-          const float mw = m_area[ww * Cons::GM + h];
+          const float mw = m_area[ww * G + h];
           if (mw == -CUDART_INF_F) continue;
           const float sc = exp2_approx(mw - M);
-          Ls = fmaf(l_area[ww * Cons::GM + h], sc, Ls);
-          O = fmaf(acc_area[(ww * Cons::GM + h) * D + dim], sc, O);
+          Ls = fmaf(l_area[ww * G + h], sc, Ls);
+          O = fmaf(acc_area[(ww * G + h) * D + dim], sc, O);
         }
       }
       const bool empty = !(Ls > 0.f);
@@ -860,9 +1031,11 @@ __global__ void __maxnreg__(224)
       const float lv = empty ? -CUDART_INF_F : (M + __log2f(Ls)) * kLn2;
       const size_t row = static_cast<size_t>(pc.b) * a.qo_heads + static_cast<size_t>(pc.h) * G + h;
       if (whole) {
-        a.out[row * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(ov));
-        if (dim == 0 && a.lse != nullptr) a.lse[row] = lv;
-      } else {
+        if (FA_CHECK(a.status, row < static_cast<size_t>(B) * a.qo_heads, 401, row)) {
+          a.out[row * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(ov));
+          if (dim == 0 && a.lse != nullptr) a.lse[row] = lv;
+        }
+      } else if (FA_CHECK(a.status, slot_idx < a.max_partials, 402, slot_idx)) {
         a.part_o[(static_cast<size_t>(slot_idx) * G + h) * D + dim] = ov;
         if (dim == 0) a.part_lse[static_cast<size_t>(slot_idx) * G + h] = lv;
       }
@@ -871,33 +1044,86 @@ __global__ void __maxnreg__(224)
       __threadfence();
       named_barrier_sync(1, NCT);
       if (ctid == 0) {
-        const unsigned ticket = atomicInc(a.counters + pc.seg, static_cast<unsigned>(pc.n_pieces - 1));
+        unsigned ticket = 0;
+        if (FA_CHECK(a.status, pc.seg < B * H && pc.n_pieces >= 1 &&
+                                   pc.c_first + pc.n_pieces - 1 + pc.seg < a.max_partials,
+                     403, pc.seg))
+          ticket = atomicInc(a.counters + pc.seg, static_cast<unsigned>(pc.n_pieces - 1));
         *s_flag = (ticket == static_cast<unsigned>(pc.n_pieces - 1)) ? 1 : 0;
       }
       named_barrier_sync(1, NCT);
       if (*s_flag) {
-        // last block of this segment: merge every block's (o, lse) exactly
+        // last block of this segment: merge every block's (o, lse) exactly.
+        // 1) per head, lse = M + ln sum_k exp(lse_k - M) (one warp per head);
+        // 2) weights w_k = exp(lse_k - lse) into shared memory (the merge
+        //    area is free now); 3) out = sum_k w_k o_k with independent loads.
         __threadfence();
-        for (int x = ctid; x < G * D; x += NCT) {
-          const int h = x / D, dim = x - h * D;
+        float* s_w = acc_area;                 // [chunk][G] weights
+        float* s_lse = m_area;                 // [G] merged lse
+        const int cap = (NW * D) > 1 ? NW * D : 1;  // pieces per chunk (acc area holds NW*G*D)
+        for (int h = w; h < G; h += NW) {
           float M = -CUDART_INF_F;
-          for (int k = 0; k < pc.n_pieces; ++k)
+          for (int k = lane; k < pc.n_pieces; k += 32)
             M = fmaxf(M, __ldcg(a.part_lse + static_cast<size_t>(pc.c_first + k + pc.seg) * G + h));
-          float Z = 0.f, O = 0.f;
-          if (M != -CUDART_INF_F) {
-            for (int k = 0; k < pc.n_pieces; ++k) {
-              const size_t sl = static_cast<size_t>(pc.c_first + k + pc.seg);
-              const float lk = __ldcg(a.part_lse + sl * G + h);
-              if (lk == -CUDART_INF_F) continue;
-              const float wgt = exp2_approx((lk - M) * kLog2e);
-              Z += wgt;
-              O = fmaf(wgt, __ldcg(a.part_o + (sl * G + h) * D + dim), O);
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+          float Z = 0.f;
+          if (M != -CUDART_INF_F)
+            for (int k = lane; k < pc.n_pieces; k += 32) {
+              const float lk = __ldcg(a.part_lse + static_cast<size_t>(pc.c_first + k + pc.seg) * G + h);
+              if (lk != -CUDART_INF_F) Z += exp2_approx((lk - M) * kLog2e);
+            }
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, off);
+          if (lane == 0) s_lse[h] = (Z > 0.f) ? M + __logf(Z) : -CUDART_INF_F;
+        }
+        named_barrier_sync(1, NCT);
+        float accv[(D * 8 + NCT - 1) / NCT];
+        constexpr int PER = (D * 8 + NCT - 1) / NCT;  // outputs per thread at G = 8
+#pragma unroll
+        for (int r = 0; r < PER; ++r) accv[r] = 0.f;
+        for (int k0 = 0; k0 < pc.n_pieces; k0 += cap) {
+          const int kn = pc.n_pieces - k0 < cap ? pc.n_pieces - k0 : cap;
+          for (int x = ctid; x < kn * G; x += NCT) {
+            const int k = x / G, h = x - k * G;
+            const float lk = __ldcg(a.part_lse + static_cast<size_t>(pc.c_first + k0 + k + pc.seg) * G + h);
+            const float L = s_lse[h];
+            s_w[x] = (lk == -CUDART_INF_F || L == -CUDART_INF_F) ? 0.f : exp2_approx((lk - L) * kLog2e);
+          }
+          named_barrier_sync(1, NCT);
+#pragma unroll
+          for (int r = 0; r < PER; ++r) {
+            const int x = ctid + r * NCT;
+            if (x < G * D) {
+              const int h = x / D, dim = x - h * D;
+              const float* src = a.part_o + (static_cast<size_t>(pc.c_first + k0 + pc.seg) * G + h) * D + dim;
+              const size_t step = static_cast<size_t>(G) * D;
+              float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+              int k = 0;
+              for (; k + 4 <= kn; k += 4) {
+                const float o0 = __ldcg(src + (k + 0) * step), o1 = __ldcg(src + (k + 1) * step);
+                const float o2 = __ldcg(src + (k + 2) * step), o3 = __ldcg(src + (k + 3) * step);
+                s0 = fmaf(s_w[(k + 0) * G + h], o0, s0);
+                s1 = fmaf(s_w[(k + 1) * G + h], o1, s1);
+                s2 = fmaf(s_w[(k + 2) * G + h], o2, s2);
+                s3 = fmaf(s_w[(k + 3) * G + h], o3, s3);
+              }
+              for (; k < kn; ++k) s0 = fmaf(s_w[k * G + h], __ldcg(src + k * step), s0);
+              accv[r] += (s0 + s1) + (s2 + s3);
             }
           }
-          const bool empty = !(Z > 0.f);
-          const size_t row = static_cast<size_t>(pc.b) * a.qo_heads + static_cast<size_t>(pc.h) * G + h;
-          a.out[row * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(empty ? 0.f : O / Z));
-          if (dim == 0 && a.lse != nullptr) a.lse[row] = empty ? -CUDART_INF_F : M + __logf(Z);
+          named_barrier_sync(1, NCT);
+        }
+#pragma unroll
+        for (int r = 0; r < PER; ++r) {
+          const int x = ctid + r * NCT;
+          if (x < G * D) {
+            const int h = x / D, dim = x - h * D;
+            const size_t row = static_cast<size_t>(pc.b) * a.qo_heads + static_cast<size_t>(pc.h) * G + h;
+            const float L = s_lse[h];
+            a.out[row * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(L == -CUDART_INF_F ? 0.f : accv[r]));
+            if (dim == 0 && a.lse != nullptr) a.lse[row] = L;
+          }
         }
       }
     }

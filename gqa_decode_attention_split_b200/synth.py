@@ -238,6 +238,13 @@ def _c4():
                     name="paged_b64_gqa4_L512-16384")
 
 
+def _c4_small():
+    """Same recipe as the batch-64 paged workload, first 16 requests (~0.56 GB
+    of K/V: larger than L2, small enough for a many-pass profiler capture)."""
+    return generate(16, 32, 8, 128, c4_lengths()[:16], paged=True, page_size=16, seed=4,
+                    name="paged_b16_gqa4_L512-16384")
+
+
 def _c5():
     return generate(1, 64, 8, 128, [131072], kv_dtype="fp8_e4m3", seed=5,
                     name="fp8_gqa8_L131072")
@@ -252,6 +259,7 @@ WORKLOADS = {
     "llama2_7b_mha_L16384": _c3(16384),
     "llama2_7b_mha_L32768": _c3(32768),
     "paged_b64_gqa4_L512-16384": _c4,
+    "paged_b16_gqa4_L512-16384": _c4_small,
     "fp8_gqa8_L131072": _c5,
 }
 

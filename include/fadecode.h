@@ -214,6 +214,11 @@ FA_API fa_status fa_merge_states(const float* o_parts, const float* lse_parts, i
 /* Static description of a status code (never NULL). */
 FA_API const char* fa_status_string(fa_status status);
 
+/* Text of the most recent CUDA failure (FA_ERR_CUDA) returned to the calling
+ * thread, or "" if there was none.  The buffer is thread-local and is
+ * overwritten by the next failure. */
+FA_API const char* fa_last_error(void);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 FA_API int32_t fa_version(void);
 
