@@ -78,6 +78,8 @@ def load_library():
     lib.fa_plan_destroy.restype = None
     lib.fa_decode_run.argtypes = [vp, vp, vp, vp, i64, vp, i32, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.fa_decode_run.restype = ctypes.c_int
+    lib.fa_decode_run_static.argtypes = [vp, vp, vp, vp, i64, vp, i32, vp, vp, vp, vp, vp, vp]
+    lib.fa_decode_run_static.restype = ctypes.c_int
     lib.fa_decode_status.argtypes = [vp, sz, ctypes.POINTER(ctypes.c_uint32), vp]
     lib.fa_decode_status.restype = ctypes.c_int
     lib.fa_merge_states.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp]
@@ -183,6 +185,29 @@ def run(p: DecodePlan, q, k, v, kv_indptr, *, page_table=None, k_scale=None, v_s
                              _ptr(v_scale), _ptr(out), _ptr(lse), _ptr(workspace),
                              int(workspace.numel() * workspace.element_size()),
                              _stream_handle(stream)), "fa_decode_run")
+    return out, lse
+
+
+def run_static(p: DecodePlan, q, k, v, kv_indptr, *, page_table=None, k_scale=None,
+               v_scale=None, out=None, lse=None, stream=None, want_lse: bool = True):
+    """Like run(), through fa_decode_run_static: no workspace, the library's
+    fixed device scratch is used (for callers that cannot allocate; the
+    output tensors here are allocated only when not passed in)."""
+    import torch
+    lib = load_library()
+    d = p.desc
+    if out is None:
+        out = torch.empty((d.batch, d.qo_heads, d.head_dim), dtype=torch.bfloat16,
+                          device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((d.batch, d.qo_heads), dtype=torch.float32, device=q.device)
+    pt_stride = int(page_table.stride(0)) if page_table is not None else 0
+    st = lib.fa_decode_run_static(p._handle, _ptr(q), _ptr(k), _ptr(v), int(k.shape[0]),
+                                  _ptr(page_table), pt_stride, _ptr(kv_indptr), _ptr(k_scale),
+                                  _ptr(v_scale), _ptr(out), _ptr(lse), _stream_handle(stream))
+    if st != FA_OK:
+        raise FadecodeError(st, "fa_decode_run_static",
+                            f"{lib.fa_status_string(st).decode()} [{lib.fa_last_error().decode()}]")
     return out, lse
 
 

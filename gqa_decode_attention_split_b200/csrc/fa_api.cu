@@ -230,6 +230,15 @@ extern "C" fa_status fa_plan_get_info(const fa_plan* plan, fa_plan_info_t* info)
 
 extern "C" void fa_plan_destroy(fa_plan* plan) { delete plan; }
 
+namespace fa {
+// Bytes at the start of a plan's workspace that must be zero before a run
+// (device-check word and ticket counters); the partial states after them
+// are always written before they are read.
+size_t plan_zero_prefix_bytes(const fa_plan* plan) { return plan->off_part_o; }
+// Sets the text returned by fa_last_error on this thread.
+void set_last_error(const char* text) { snprintf(g_last_error, sizeof(g_last_error), "%s", text); }
+}  // namespace fa
+
 namespace {
 
 fa_status make_kv_map(const fa_plan* p, const void* base, int64_t kv_rows, CUtensorMap* map) {

@@ -183,6 +183,39 @@ FA_API fa_status fa_decode_run(const fa_plan* plan, const void* q, const void* k
                         void* out, float* lse, void* workspace, size_t workspace_bytes,
                         void* stream);
 
+/* Size of the fixed scratch behind fa_decode_run_static: 4 MiB. */
+#define FA_STATIC_WORKSPACE_BYTES (4u << 20)
+
+/*
+ * fa_decode_run_static -- fa_decode_run for callers that cannot allocate.
+ * (An addition of this library; the pages have no counterpart.)
+ *
+ * Some callers cannot call cudaMalloc or any other allocating routine where
+ * they run attention: a runtime that hands out all device memory itself, a
+ * plugin that receives only input and output buffers, or a path that must
+ * not synchronise the device (cudaMalloc and cudaFree may).  This entry point
+ * takes the same arguments as fa_decode_run minus the workspace, and
+ * allocates nothing: its scratch is a fixed array of
+ * FA_STATIC_WORKSPACE_BYTES in the library's device memory, which every GPU
+ * that loads the library holds until the process exits.
+ *  - The first call on a device looks up that array's device address (once
+ *    per device, on the current device); make that first call before any
+ *    stream capture.
+ *  - Every call on a device shares the one array, which keeps what the
+ *    previous call left.  Each call clears the part that must start at zero
+ *    (check word, ticket counters) in stream order before its kernel.  Calls
+ *    that overlap on the GPU (other streams, other host threads) race on the
+ *    array and must be avoided.
+ *  - A plan whose workspace_bytes exceeds FA_STATIC_WORKSPACE_BYTES is
+ *    rejected with FA_ERR_WORKSPACE_TOO_SMALL (fa_last_error says how much
+ *    it needed).  Other errors as fa_decode_run.
+ */
+FA_API fa_status fa_decode_run_static(const fa_plan* plan, const void* q, const void* k,
+                                      const void* v, int64_t kv_rows, const int32_t* page_table,
+                                      int32_t page_table_stride, const int32_t* kv_indptr,
+                                      const float* k_scale, const float* v_scale, void* out,
+                                      float* lse, void* stream);
+
 /*
  * fa_decode_status -- SYNCHRONISES `stream`, then reads the device-side check
  * word of `workspace` into *flags (FA_DEVICE_* bits, 0 = clean) and clears
