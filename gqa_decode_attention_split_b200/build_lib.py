@@ -52,18 +52,19 @@ def up_to_date() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False,
-          checks: bool = False, out: str = None) -> str:
+          checks: bool = False, out: str = None, defines=()) -> str:
     """Compile and link.  checks=True builds the self-checking variant
     (-DFA_CHECKS: range/alignment checks on every shared-memory read, bulk
     copy destination and global write, reported through the status word)."""
     lib = out or LIB
-    if not force and out is None and not checks and up_to_date():
+    if not force and out is None and not checks and not defines and up_to_date():
         return LIB
-    build_dir = BUILD + ("_checks" if checks else "")
+    tag = ("_checks" if checks else "") + "".join("_" + d.replace("=", "") for d in defines)
+    build_dir = BUILD + tag
     os.makedirs(build_dir, exist_ok=True)
     os.makedirs(os.path.dirname(lib), exist_ok=True)
     nvcc = _nvcc()
-    extra = ["-DFA_CHECKS"] if checks else []
+    extra = (["-DFA_CHECKS"] if checks else []) + ["-D" + d for d in defines]
 
     def compile_one(src):
         obj = os.path.join(build_dir, os.path.basename(src) + ".o")
@@ -97,9 +98,11 @@ def main():
     ap.add_argument("--ptxas-info", action="store_true")
     ap.add_argument("--checks", action="store_true", help="self-checking build (-DFA_CHECKS)")
     ap.add_argument("--out", default=None, help="output path (default: lib/libfadecode.so)")
+    ap.add_argument("-D", dest="defines", action="append", default=[],
+                    help="extra preprocessor definition, e.g. -D FA_TILE_BYTES=8192")
     args = ap.parse_args()
     print(build(force=args.force, verbose=args.verbose, ptxas_info=args.ptxas_info,
-                checks=args.checks, out=args.out))
+                checks=args.checks, out=args.out, defines=tuple(args.defines)))
 
 
 if __name__ == "__main__":

@@ -195,7 +195,12 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   p->max_partials = P + segs;
   p->page_shift = desc->paged ? ilog2_exact(desc->page_size) : 0;
   p->box_t = desc->paged ? (desc->page_size < T ? desc->page_size : T) : T;
-  p->swz = (k->plane_bytes == 128 && p->box_t >= 8) ? 1 : 0;
+  // 128B swizzle needs every copy to start on a 1024-byte boundary of the
+  // tile: whole 8-line groups of 128-byte lines per copy.
+  {
+    const int lines_per_copy = k->token_major ? p->box_t * (k->row_bytes / k->plane_bytes) : p->box_t;
+    p->swz = (k->plane_bytes == 128 && lines_per_copy % 8 == 0) ? 1 : 0;
+  }
   size_t off = 256;  // header: device-check word
   p->off_counters = off;
   off = align_up(off + sizeof(uint32_t) * static_cast<size_t>(segs), 256);
@@ -251,17 +256,41 @@ fa_status make_kv_map(const fa_plan* p, const void* base, int64_t kv_rows, CUten
   const KernelEntry* k = p->kernel;
   const int es = d.kv_dtype == FA_KV_FP8_E4M3 ? 1 : 2;
   const cuuint64_t row = static_cast<cuuint64_t>(d.head_dim) * es;
+  const cuuint64_t cb = static_cast<cuuint64_t>(k->plane_bytes);
+  const cuuint64_t np = row / cb;
   const CUtensorMapDataType dt = es == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
   const CUtensorMapSwizzle sw = p->swz ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
-  const cuuint32_t inner = static_cast<cuuint32_t>(k->plane_bytes / es);
+  const cuuint32_t inner = static_cast<cuuint32_t>(cb / es);
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r;
-  if (!d.paged) {
+  if (k->token_major) {
+    // [.. rows][kv_heads][planes][plane elements]: one copy carries whole rows
+    if (!d.paged) {
+      const cuuint64_t dims[4] = {inner, np, static_cast<cuuint64_t>(d.kv_heads),
+                                  static_cast<cuuint64_t>(kv_rows)};
+      const cuuint64_t strides[3] = {cb, row, row * d.kv_heads};
+      const cuuint32_t box[4] = {inner, static_cast<cuuint32_t>(np), 1,
+                                 static_cast<cuuint32_t>(k->tile_tokens)};
+      r = enc(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    } else {
+      const cuuint64_t dims[5] = {inner, np, static_cast<cuuint64_t>(d.kv_heads),
+                                  static_cast<cuuint64_t>(d.page_size),
+                                  static_cast<cuuint64_t>(kv_rows)};
+      const cuuint64_t strides[4] = {cb, row, row * d.kv_heads, row * d.kv_heads * d.page_size};
+      const cuuint32_t box[5] = {inner, static_cast<cuuint32_t>(np), 1,
+                                 static_cast<cuuint32_t>(p->box_t), 1};
+      r = enc(map, dt, 5, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    }
+  } else if (!d.paged) {
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d.head_dim),
                                 static_cast<cuuint64_t>(d.kv_heads),
                                 static_cast<cuuint64_t>(kv_rows)};
     const cuuint64_t strides[2] = {row, row * d.kv_heads};
     const cuuint32_t box[3] = {inner, 1, static_cast<cuuint32_t>(k->tile_tokens)};
-    const cuuint32_t estr[3] = {1, 1, 1};
     r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -272,7 +301,6 @@ fa_status make_kv_map(const fa_plan* p, const void* base, int64_t kv_rows, CUten
                                 static_cast<cuuint64_t>(kv_rows)};
     const cuuint64_t strides[3] = {row, row * d.kv_heads, row * d.kv_heads * d.page_size};
     const cuuint32_t box[4] = {inner, 1, static_cast<cuuint32_t>(p->box_t), 1};
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
     r = enc(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

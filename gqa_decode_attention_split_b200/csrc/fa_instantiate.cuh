@@ -47,6 +47,7 @@ KernelEntry make_entry(int path, int group, int max_group, int fp8) {
   e.threads = C::THREADS;
   e.row_bytes = C::ROWB;
   e.plane_bytes = C::CB;
+  e.token_major = C::TOKEN_MAJOR ? 1 : 0;
   e.smem_bytes = &smem_bytes_for<Cons>;
   e.launch = &launch_decode<Cons>;
   return e;

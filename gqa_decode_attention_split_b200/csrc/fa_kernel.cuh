@@ -33,7 +33,35 @@
 
 namespace fa {
 
-constexpr int kConsumerWarps = 7;  // + 1 producer warp = 2 warps per SM sub-partition
+// Tuning knobs (compile-time).  Defaults are the settings measured best on
+// B200 for each dataflow: the tensor-core path wants large tiles (few bulk
+// copies and barrier round trips per byte) and five consumer warps; the
+// instruction-heavier SIMT and fp8 paths want more warps.  Every knob can be
+// overridden with -D for tuning sweeps.
+#ifndef FA_MMA_TILE_BYTES
+#define FA_MMA_TILE_BYTES 16384      // bytes of K (and of V) per stage, bf16 MMA path
+#endif
+#ifndef FA_MMA_CONSUMER_WARPS
+#define FA_MMA_CONSUMER_WARPS 5
+#endif
+#ifndef FA_FP8_MMA_TILE_BYTES
+#define FA_FP8_MMA_TILE_BYTES 8192
+#endif
+#ifndef FA_FP8_MMA_CONSUMER_WARPS
+#define FA_FP8_MMA_CONSUMER_WARPS 7
+#endif
+#ifndef FA_SIMT_TILE_BYTES
+#define FA_SIMT_TILE_BYTES 8192
+#endif
+#ifndef FA_SIMT_CONSUMER_WARPS
+#define FA_SIMT_CONSUMER_WARPS 6
+#endif
+#ifndef FA_MAX_STAGES_PER_WARP
+#define FA_MAX_STAGES_PER_WARP 3
+#endif
+#ifndef FA_PLANE_COPIES
+#define FA_PLANE_COPIES 0    // 0: one bulk copy per box, planes a tensor-map dimension
+#endif
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait, then give up
 constexpr float kRescaleSlack = 8.0f;               // log2 units
 constexpr float kLog2e = 1.4426950408889634f;
@@ -69,44 +97,60 @@ struct KernelArgs {
 constexpr int kSmemPerBlock = 232448;  // 227 KB of shared memory per block (sm_100)
 constexpr int kSchedReserve = 8192;    // schedule arrays for up to 682 requests
 
-// Shared-memory tile geometry for one head_dim / element type.  A K (or V)
-// tile of T tokens is stored plane-major: [NP][T][CB] where a plane holds
-// CB = min(128, row bytes) bytes of every token row; with 128-byte rows the
-// 16-byte chunks of row r are XOR-swizzled by (r & 7) (TMA 128B swizzle).
-// A tile is 4 KB of K (and 4 KB of V) for rows up to 256 bytes: T = 4096 /
-// row bytes tokens, at least 16.  The ring takes what is left of the block's
+// Shared-memory tile geometry for one head_dim / element type.  A token row
+// is cut into NP planes of CB = min(128, row bytes) bytes (the widest box row
+// the 128-byte swizzle allows).  Default (token-major) layout of a K or V
+// tile: [T][NP][CB], written by ONE bulk copy per box whose tensor map has
+// the plane as a dimension; the 16-byte chunks of 128-byte line l of the tile
+// are XOR-swizzled by (l & 7) (TMA 128B swizzle).  With FA_PLANE_COPIES the
+// layout is plane-major, [NP][T][CB], one copy per plane.
+// A tile holds TILE_BYTES_TARGET / row bytes tokens (16 to 128).  The ring takes what is left of the block's
 // shared memory after the merge area for GMAX query heads, in a multiple of
 // the consumer-warp count: tile i uses stage i % STAGES and warp i % NW, so
 // every stage belongs to exactly one warp, which waits on it round after
 // round.  (A stage shared by two warps would let one warp wait for round r+1
 // while round r is still pending; an mbarrier parity wait cannot tell the two
 // apart and would pass early.)
-template <int D, bool FP8, int GMAX>
+template <int D, bool FP8, int GMAX, int TILE_BYTES_TARGET, int NWARPS>
 struct TileCfg {
   static constexpr int ES = FP8 ? 1 : 2;
   static constexpr int ROWB = D * ES;
   static constexpr int CB = ROWB < 128 ? ROWB : 128;
   static constexpr int NP = ROWB / CB;
-  static constexpr int T_RAW = 4096 / ROWB;
-  static constexpr int T = T_RAW < 16 ? 16 : (T_RAW > 64 ? 64 : T_RAW);
+  static constexpr int T_RAW = TILE_BYTES_TARGET / ROWB;
+  static constexpr int T = T_RAW < 16 ? 16 : (T_RAW > 128 ? 128 : T_RAW);
   static constexpr int TILE_BYTES = T * ROWB;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-  static constexpr int NW = kConsumerWarps;
+  static constexpr int NW = NWARPS;
   static constexpr int MERGE_BYTES = NW * GMAX * (D + 2) * 4;
   static constexpr int RING_BUDGET = kSmemPerBlock - 1024 - kSchedReserve - 512 - MERGE_BYTES;
   static constexpr int STAGES_RAW = RING_BUDGET / STAGE_BYTES;
   static constexpr int STAGES_PER_WARP_RAW = STAGES_RAW / NW;
-  static constexpr int STAGES_PER_WARP = STAGES_PER_WARP_RAW > 3 ? 3 : STAGES_PER_WARP_RAW;
+  static constexpr int STAGES_PER_WARP =
+      STAGES_PER_WARP_RAW > FA_MAX_STAGES_PER_WARP ? FA_MAX_STAGES_PER_WARP : STAGES_PER_WARP_RAW;
   static constexpr int STAGES = NW * STAGES_PER_WARP;
   static_assert(STAGES_PER_WARP >= 1, "every consumer warp needs a stage");
   static_assert(STAGES % NW == 0, "a stage must belong to one consumer warp");
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
   static constexpr int THREADS = (NW + 1) * 32;
+  static constexpr bool TOKEN_MAJOR = FA_PLANE_COPIES == 0;
   static_assert(ROWB % 16 == 0, "rows must be whole 16-byte chunks");
 };
 
 __device__ __forceinline__ uint32_t swz_off(int row, int chunk, int swz) {
   return static_cast<uint32_t>(((chunk ^ (swz ? (row & 7) : 0)) << 4));
+}
+
+// Shared-memory address of 16-byte chunk `chunk` of plane `plane` of token
+// row `row` in a tile.
+template <class C>
+__device__ __forceinline__ uint32_t tile_addr(uint32_t tile, int row, int plane, int chunk, int swz) {
+  if constexpr (C::TOKEN_MAJOR) {
+    const int line = row * C::NP + plane;
+    return tile + line * C::CB + swz_off(line, chunk, swz);
+  } else {
+    return tile + plane * (C::T * C::CB) + row * C::CB + swz_off(row, chunk, swz);
+  }
 }
 
 // A wait that gives up records where (first one wins) in words 8..15 of the
@@ -232,7 +276,7 @@ __device__ __forceinline__ bool next_piece(PieceIter& it, Piece& pc, const int* 
 // running softmax state, merged across slots at the end of a segment piece.
 template <int D, int G, bool FP8>
 struct SimtConsumer {
-  using C = TileCfg<D, FP8, G>;
+  using C = TileCfg<D, FP8, G, FA_SIMT_TILE_BYTES, FA_SIMT_CONSUMER_WARPS>;
   static constexpr int EPC = 16 / C::ES;
   static constexpr int NCH = C::ROWB / 16;
   static constexpr int E_TARGET = 64 / G;
@@ -279,8 +323,7 @@ struct SimtConsumer {
   }
 
   __device__ __forceinline__ uint32_t addr(uint32_t tile, int r, int k, int swz) const {
-    return tile + chunk_plane(k) * (C::T * C::CB) + r * C::CB +
-           swz_off(r, chunk_in_plane(k), swz);
+    return tile_addr<C>(tile, r, chunk_plane(k), chunk_in_plane(k), swz);
   }
 
   __device__ __forceinline__ void begin_piece(const KernelArgs& a, int b, int hkv, int lane) {
@@ -439,7 +482,8 @@ struct SimtConsumer {
 // into f16 range (the scale is undone on the fp32 scores).
 template <int D, bool FP8>
 struct MmaConsumer {
-  using C = TileCfg<D, FP8, 8>;
+  using C = TileCfg<D, FP8, 8, FP8 ? FA_FP8_MMA_TILE_BYTES : FA_MMA_TILE_BYTES,
+                    FP8 ? FA_FP8_MMA_CONSUMER_WARPS : FA_MMA_CONSUMER_WARPS>;
   static constexpr int KS = D / 16;     // k-steps of the score product = m-tiles of O^T
   static constexpr int SUB = C::T / 16;  // 16-token subtiles per tile
   static constexpr int BPT = D / 4;      // fp8 K: bytes of a row owned by one lane
@@ -511,7 +555,7 @@ struct MmaConsumer {
   }
 
   __device__ __forceinline__ uint32_t chunk_addr(uint32_t tile, int row, int chunk, int swz) const {
-    return tile + (chunk >> 3) * (C::T * 128) + row * 128 + swz_off(row, chunk & 7, swz);
+    return tile_addr<C>(tile, row, chunk >> 3, chunk & 7, swz);
   }
 
   // Two accumulators (even / odd k-steps) halve the dependent chain of mma.
@@ -897,12 +941,31 @@ __global__ void __maxnreg__(224)
             mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
             if (!a.paged) {
               const int row = s_start[pc.b] + tt * T;
+              if constexpr (C::TOKEN_MAJOR) {
+                tma_load_4d(kdst, &a.kmap, fb, 0, 0, pc.h, row, pol);
+                tma_load_4d(vdst, &a.vmap, fb, 0, 0, pc.h, row, pol);
+              } else {
 #pragma unroll
-              for (int p = 0; p < C::NP; ++p) {
-                const uint32_t off = p * (T * C::CB);
-                if (FA_CHECK(a.status, off + T * C::CB <= C::TILE_BYTES && (off & 127u) == 0, 301, off)) {
-                  tma_load_3d(kdst + off, &a.kmap, fb, p * (C::CB / C::ES), pc.h, row, pol);
-                  tma_load_3d(vdst + off, &a.vmap, fb, p * (C::CB / C::ES), pc.h, row, pol);
+                for (int p = 0; p < C::NP; ++p) {
+                  const uint32_t off = p * (T * C::CB);
+                  if (FA_CHECK(a.status, off + T * C::CB <= C::TILE_BYTES && (off & 127u) == 0, 301, off)) {
+                    tma_load_3d(kdst + off, &a.kmap, fb, p * (C::CB / C::ES), pc.h, row, pol);
+                    tma_load_3d(vdst + off, &a.vmap, fb, p * (C::CB / C::ES), pc.h, row, pol);
+                  }
+                }
+              }
+            } else if constexpr (C::TOKEN_MAJOR) {
+              for (int jb = 0; jb < NB; ++jb) {
+                const int tok = tt * T + jb * a.box_t;
+                const int pidx = tok >> a.page_shift;
+                const int page = (pidx < npages && pidx - pbase < 64) ? s_pages[pidx - pbase] : -1;
+                const int slot0 = tok & (ps - 1);
+                const uint32_t off = jb * a.box_t * C::ROWB;
+                if (FA_CHECK(a.status, off + a.box_t * C::ROWB <= C::TILE_BYTES && (off & 127u) == 0 &&
+                                           pidx - pbase >= 0 && pidx - pbase < 64,
+                             303, off)) {
+                  tma_load_5d(kdst + off, &a.kmap, fb, 0, 0, pc.h, slot0, page, pol);
+                  tma_load_5d(vdst + off, &a.vmap, fb, 0, 0, pc.h, slot0, page, pol);
                 }
               }
             } else {
