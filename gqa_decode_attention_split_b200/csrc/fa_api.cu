@@ -170,13 +170,14 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   if (desc->num_ctas > 0) {
     P = desc->num_ctas;
   } else {
-    // One block per SM (each holds a ~170 KB tile ring).  Small problems use
-    // fewer blocks so that every consumer warp streams at least two tiles,
-    // and a segment is cut into at most kMaxPiecesPerSegment runs on average
-    // so that the last block's merge of the partial states stays short.
+    // One block per SM (each holds a ~170 KB tile ring).  A problem with
+    // fewer tiles than SMs gets one tile per block (the fixed cost of a
+    // block is small next to a KV tile's load latency, and the tiles load in
+    // parallel); a segment is cut into at most kMaxPiecesPerSegment runs on
+    // average so that the last block's merge of the partial states stays
+    // short.
     constexpr int64_t kMaxPiecesPerSegment = 32;
-    const int64_t min_tiles = 2 * (k->threads / 32 - 1);
-    int64_t want = (tiles + min_tiles - 1) / min_tiles;
+    int64_t want = tiles;
     const int64_t seg_cap = kMaxPiecesPerSegment * desc->batch * desc->kv_heads;
     if (want > seg_cap) want = seg_cap;
     P = want < num_sms ? want : num_sms;
@@ -262,6 +263,11 @@ fa_status make_kv_map(const fa_plan* p, const void* base, int64_t kv_rows, CUten
   const CUtensorMapSwizzle sw = p->swz ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
   const cuuint32_t inner = static_cast<cuuint32_t>(cb / es);
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  // L2 fills no wider than a token row: a 256-byte fill of a 128-byte row
+  // would pull in the next kv head's row, which another block reads much
+  // later (measured 1.48x DRAM traffic on 128-byte fp8 rows).
+  const CUtensorMapL2promotion promo =
+      row >= 256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_L2_128B;
   CUresult r;
   if (k->token_major) {
     // [.. rows][kv_heads][planes][plane elements]: one copy carries whole rows
@@ -272,7 +278,7 @@ fa_status make_kv_map(const fa_plan* p, const void* base, int64_t kv_rows, CUten
       const cuuint32_t box[4] = {inner, static_cast<cuuint32_t>(np), 1,
                                  static_cast<cuuint32_t>(k->tile_tokens)};
       r = enc(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, promo,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     } else {
       const cuuint64_t dims[5] = {inner, np, static_cast<cuuint64_t>(d.kv_heads),
@@ -282,7 +288,7 @@ fa_status make_kv_map(const fa_plan* p, const void* base, int64_t kv_rows, CUten
       const cuuint32_t box[5] = {inner, static_cast<cuuint32_t>(np), 1,
                                  static_cast<cuuint32_t>(p->box_t), 1};
       r = enc(map, dt, 5, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, promo,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     }
   } else if (!d.paged) {
@@ -292,7 +298,7 @@ fa_status make_kv_map(const fa_plan* p, const void* base, int64_t kv_rows, CUten
     const cuuint64_t strides[2] = {row, row * d.kv_heads};
     const cuuint32_t box[3] = {inner, 1, static_cast<cuuint32_t>(k->tile_tokens)};
     r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, promo,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   } else {
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d.head_dim),
@@ -302,7 +308,7 @@ fa_status make_kv_map(const fa_plan* p, const void* base, int64_t kv_rows, CUten
     const cuuint64_t strides[3] = {row, row * d.kv_heads, row * d.kv_heads * d.page_size};
     const cuuint32_t box[4] = {inner, 1, static_cast<cuuint32_t>(p->box_t), 1};
     r = enc(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, promo,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   }
   if (r != CUDA_SUCCESS) {

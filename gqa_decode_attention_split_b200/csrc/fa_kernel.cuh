@@ -50,6 +50,9 @@ namespace fa {
 #ifndef FA_FP8_MMA_CONSUMER_WARPS
 #define FA_FP8_MMA_CONSUMER_WARPS 7
 #endif
+#ifndef FA_FP8_QSPLIT
+#define FA_FP8_QSPLIT 0              // 1: fp8 scores on the e4m3 product (measured slower)
+#endif
 #ifndef FA_SIMT_TILE_BYTES
 #define FA_SIMT_TILE_BYTES 8192
 #endif
@@ -477,9 +480,13 @@ struct SimtConsumer {
 // per instruction, fp32 accumulate); probabilities are transposed in
 // registers (movmatrix) into the B operand of O^T += V^T . P^T, with O^T
 // (dims x heads) accumulated in fp32 registers.  Up to 8 query heads per kv
-// head; missing heads are zero columns.  bf16 K/V use bf16 operands; e4m3
-// K/V are widened exactly to f16 and q is scaled by a power of two per head
-// into f16 range (the scale is undone on the fp32 scores).
+// head; missing heads are zero columns.  bf16 K/V use bf16 operands.  For
+// e4m3 K the scores run on the e4m3 product (m16n8k32) straight from the
+// stored codes: q, scaled by a power of two per head, is split into three
+// e4m3 parts hi + mid + lo (about 12 significant bits, the part sum is within
+// 2^-12 of the bf16 value) and the three products are summed in fp32.  e4m3
+// V is widened exactly to f16 for the P.V product.  The q scale is undone on
+// the fp32 scores.
 template <int D, bool FP8>
 struct MmaConsumer {
   using C = TileCfg<D, FP8, 8, FP8 ? FA_FP8_MMA_TILE_BYTES : FA_MMA_TILE_BYTES,
@@ -487,11 +494,14 @@ struct MmaConsumer {
   static constexpr int KS = D / 16;     // k-steps of the score product = m-tiles of O^T
   static constexpr int SUB = C::T / 16;  // 16-token subtiles per tile
   static constexpr int BPT = D / 4;      // fp8 K: bytes of a row owned by one lane
+  static constexpr bool kQSplit = FP8 && FA_FP8_QSPLIT;
+  static constexpr int KS32 = D / 32;    // k-steps of the e4m3 score product
   static constexpr int VBT = D / 8;      // fp8 V: bytes of a row owned by one lane
   static_assert(D % 16 == 0 && C::T % 16 == 0, "mma tiling");
   static_assert(!FP8 || C::CB == 128, "fp8 mma path needs 128-byte planes");
 
   uint32_t qb[KS][2];
+  uint32_t qb8[KS32][3][2];  // e4m3 q parts (hi, mid, lo) per k-step
   float o[KS][4];
   float m[2], l[2];
   float sscale[2];
@@ -531,14 +541,44 @@ struct MmaConsumer {
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
       int ex = 0;
       frexpf(mx, &ex);
-      const int sh = (mx > 0.f && isfinite(mx)) ? 15 - ex : 0;  // |q| * 2^sh < 2^15
-      const float mul = ldexpf(1.f, sh);
+      int sh = 0;
+      if constexpr (kQSplit) {
+        sh = (mx > 0.f && isfinite(mx)) ? 8 - ex : 0;  // max |q| * 2^sh in [128, 256)
+        const float mul = ldexpf(1.f, sh);
 #pragma unroll
-      for (int kk = 0; kk < KS; ++kk) {
-        // logical k-columns 2t,2t+1 / 2t+8,2t+9 of step kk <-> bytes BPT*t + 4kk + {0,1} / {2,3}
-        const uint32_t w0 = qw[2 * kk], w1 = qw[2 * kk + 1];
-        qb[kk][0] = pack_f16x2(bf16lo(w0) * mul, bf16hi(w0) * mul);
-        qb[kk][1] = pack_f16x2(bf16lo(w1) * mul, bf16hi(w1) * mul);
+        for (int kk = 0; kk < KS32; ++kk) {
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            // logical k-columns 4t..4t+3 (half 0) / 16+4t..16+4t+3 (half 1) of
+            // step kk <-> dims BPT*t + 8kk + 4*half + 0..3
+            const uint32_t wa = qw[4 * kk + 2 * half], wb = qw[4 * kk + 2 * half + 1];
+            float x0 = bf16lo(wa) * mul, x1 = bf16hi(wa) * mul;
+            float x2 = bf16lo(wb) * mul, x3 = bf16hi(wb) * mul;
+#pragma unroll
+            for (int part = 0; part < 3; ++part) {
+              const uint16_t e01 = float2_to_e4m3x2(x0, x1), e23 = float2_to_e4m3x2(x2, x3);
+              qb8[kk][part][half] = static_cast<uint32_t>(e01) | (static_cast<uint32_t>(e23) << 16);
+              if (part < 2) {  // the next part carries what this one missed
+                const float2 d01 = f16x2_to_float2(e4m3x2_to_f16x2(e01));
+                const float2 d23 = f16x2_to_float2(e4m3x2_to_f16x2(e23));
+                x0 -= d01.x;
+                x1 -= d01.y;
+                x2 -= d23.x;
+                x3 -= d23.y;
+              }
+            }
+          }
+        }
+      } else {
+        sh = (mx > 0.f && isfinite(mx)) ? 15 - ex : 0;  // |q| * 2^sh < 2^15
+        const float mul = ldexpf(1.f, sh);
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+          // logical k-columns 2t,2t+1 / 2t+8,2t+9 of step kk <-> bytes BPT*t + 4kk + {0,1} / {2,3}
+          const uint32_t w0 = qw[2 * kk], w1 = qw[2 * kk + 1];
+          qb[kk][0] = pack_f16x2(bf16lo(w0) * mul, bf16hi(w0) * mul);
+          qb[kk][1] = pack_f16x2(bf16lo(w1) * mul, bf16hi(w1) * mul);
+        }
       }
       const int sh0 = __shfl_sync(0xffffffffu, sh, (2 * t) * 4);
       const int sh1 = __shfl_sync(0xffffffffu, sh, (2 * t + 1) * 4);
@@ -590,17 +630,32 @@ struct MmaConsumer {
         w0[4 * i] = x0.x; w0[4 * i + 1] = x0.y; w0[4 * i + 2] = x0.z; w0[4 * i + 3] = x0.w;
         w1[4 * i] = x1.x; w1[4 * i + 1] = x1.y; w1[4 * i + 2] = x1.z; w1[4 * i + 3] = x1.w;
       }
+      if constexpr (kQSplit) {
+        float c3[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int kk = 0; kk < KS; ++kk) {
-        uint32_t af[4];
-        af[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(w0[kk] & 0xFFFFu));
-        af[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[kk] & 0xFFFFu));
-        af[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(w0[kk] >> 16));
-        af[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[kk] >> 16));
-        if (kk & 1)
-          mma_f16(c2, af, qb[kk][0], qb[kk][1]);
-        else
-          mma_f16(c, af, qb[kk][0], qb[kk][1]);
+        for (int kk = 0; kk < KS32; ++kk) {
+          // A (16 tokens x 32 dims, e4m3): rows g / g+8, logical k 4t..4t+3
+          // and 16+4t..16+4t+3 <-> words 2kk and 2kk+1 of the lane's bytes
+          const uint32_t af[4] = {w0[2 * kk], w1[2 * kk], w0[2 * kk + 1], w1[2 * kk + 1]};
+          mma_e4m3(c, af, qb8[kk][0][0], qb8[kk][0][1]);
+          mma_e4m3(c2, af, qb8[kk][1][0], qb8[kk][1][1]);
+          mma_e4m3(c3, af, qb8[kk][2][0], qb8[kk][2][1]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) c2[i] += c3[i];
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+          uint32_t af[4];
+          af[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(w0[kk] & 0xFFFFu));
+          af[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[kk] & 0xFFFFu));
+          af[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(w0[kk] >> 16));
+          af[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[kk] >> 16));
+          if (kk & 1)
+            mma_f16(c2, af, qb[kk][0], qb[kk][1]);
+          else
+            mma_f16(c, af, qb[kk][0], qb[kk][1]);
+        }
       }
     }
 #pragma unroll
