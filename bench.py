@@ -480,7 +480,10 @@ def main():
                              "traffic": traffic, "peak_source": peak_kind,
                              "launch_us": round(mean_launch * 1e3, 2),
                              "algorithmic_bytes_per_launch": kv_bytes},
-                "gpu_launches": args.steps, "clocks": clocks, "e2e": e2e,
+                # per step: the decode kernel, plus the split-merge kernel when
+                # the pass runs on more than one block
+                "gpu_launches": args.steps * (2 if runner.info["num_ctas"] > 1 else 1),
+                "clocks": clocks, "e2e": e2e,
                 "cpu_baseline": cpu, "sweep": sweep}
         print(json.dumps(line), flush=True)
     if world > 1:

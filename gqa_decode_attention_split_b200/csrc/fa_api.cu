@@ -93,7 +93,7 @@ struct fa_plan {
   int64_t total_tiles;
   int64_t max_partials;
   size_t ws_bytes;
-  size_t off_counters, off_part_o, off_part_lse;
+  size_t off_records, off_part_o, off_part_lse;
   size_t smem;
 };
 
@@ -202,9 +202,9 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
     const int lines_per_copy = k->token_major ? p->box_t * (k->row_bytes / k->plane_bytes) : p->box_t;
     p->swz = (k->plane_bytes == 128 && lines_per_copy % 8 == 0) ? 1 : 0;
   }
-  size_t off = 256;  // header: device-check word
-  p->off_counters = off;
-  off = align_up(off + sizeof(uint32_t) * static_cast<size_t>(segs), 256);
+  size_t off = 256;  // header: device-check word, timeout record
+  p->off_records = off;
+  off = align_up(off + sizeof(int32_t) * 4 * static_cast<size_t>(P), 256);
   p->off_part_o = off;
   off = align_up(off + sizeof(float) * static_cast<size_t>(p->max_partials) * group * desc->head_dim,
                  256);
@@ -238,9 +238,9 @@ extern "C" void fa_plan_destroy(fa_plan* plan) { delete plan; }
 
 namespace fa {
 // Bytes at the start of a plan's workspace that must be zero before a run
-// (device-check word and ticket counters); the partial states after them
-// are always written before they are read.
-size_t plan_zero_prefix_bytes(const fa_plan* plan) { return plan->off_part_o; }
+// (the device-check header); the boundary records and partial states after
+// it are always written by a pass before that pass reads them.
+size_t plan_zero_prefix_bytes(const fa_plan* plan) { return plan->off_records; }
 // Sets the text returned by fa_last_error on this thread.
 void set_last_error(const char* text) { snprintf(g_last_error, sizeof(g_last_error), "%s", text); }
 }  // namespace fa
@@ -356,7 +356,7 @@ extern "C" fa_status fa_decode_run(const fa_plan* plan, const void* q, const voi
   a.out = static_cast<uint16_t*>(out);
   a.lse = lse;
   a.status = reinterpret_cast<uint32_t*>(ws);
-  a.counters = reinterpret_cast<uint32_t*>(ws + plan->off_counters);
+  a.records = reinterpret_cast<int4*>(ws + plan->off_records);
   a.part_o = reinterpret_cast<float*>(ws + plan->off_part_o);
   a.part_lse = reinterpret_cast<float*>(ws + plan->off_part_lse);
   a.kv_rows = kv_rows;
@@ -376,6 +376,20 @@ extern "C" fa_status fa_decode_run(const fa_plan* plan, const void* q, const voi
   cudaError_t e = plan->kernel->launch(a, plan->num_ctas, plan->smem,
                                        static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_failure("fa_decode_run: launch", e);
+  fa::SplitMergeArgs m;
+  m.records = a.records;
+  m.part_o = a.part_o;
+  m.part_lse = a.part_lse;
+  m.out = a.out;
+  m.lse = a.lse;
+  m.num_records = plan->num_ctas;
+  m.group = plan->group;
+  m.kv_heads = d.kv_heads;
+  m.qo_heads = d.qo_heads;
+  m.batch = d.batch;
+  m.max_partials = plan->max_partials;
+  e = fa::launch_split_merge(m, d.head_dim, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_failure("fa_decode_run: merge launch", e);
   return FA_OK;
 }
 

@@ -1,6 +1,7 @@
 // fa_kernel.cuh -- split-KV GQA decode attention for sm_100a.
 //
-// One launch does the whole pass:
+// A pass is one launch of fa_decode_kernel plus, when a segment is split
+// across blocks, one launch of fa_split_merge_kernel:
 //  1. schedule: every (request, kv head) is a segment of KV tiles; segments
 //     are laid end to end and cut into gridDim.x equal runs, one per thread
 //     block, so every SM streams the same number of bytes whatever the
@@ -20,11 +21,16 @@
 //     reductions) and MMA (the two skinny products on mma.sync with fp32
 //     accumulation).
 //  4. merge: warps of a block merge their states in shared memory; a
-//     segment cut across blocks writes (o, lse) partials and the last block
-//     to finish it (atomic ticket, no waiting) merges them exactly through
+//     segment that lies whole in one block is written out directly.  A
+//     segment cut across blocks writes one (o, lse) partial per block, and
+//     a second, small kernel (fa_split_merge_kernel, launched as a
+//     programmatic dependent of this one) merges them exactly through
 //     log-sum-exp ("FlashDecoding++" explainer, section "Asynchronous softmax
 //     and unified max value": partial softmax per tile, combined afterwards;
-//     "Flashlight", section "Method": exp(x - y) = exp(x) / exp(y)).
+//     "Flashlight", section "Method": exp(x - y) = exp(x) / exp(y)).  The
+//     merge runs on every SM at once: a single block merging a segment's
+//     partials is bound by L2 round trips (one block keeps too few bytes in
+//     flight), which on B200 cost about a microsecond each.
 #pragma once
 
 #include <math_constants.h>
@@ -86,7 +92,7 @@ struct KernelArgs {
   uint16_t* out;
   float* lse;
   uint32_t* status;
-  uint32_t* counters;
+  int4* records;     // [gridDim.x]: split segment whose first cut is at block c
   float* part_o;
   float* part_lse;
   long long kv_rows;
@@ -850,7 +856,7 @@ struct SmemLayout {
     return kMerge + ((C::NW * G * 2 * 4 + 15) / 16) * 16;
   }
   __host__ __device__ static constexpr int misc_off(int G) { return acc_off(G) + C::NW * G * D * 4; }
-  // misc: ticket flag (16 B), then 64 staged page ids (256 B)
+  // misc: 16 spare bytes, then 64 staged page ids (256 B)
   __host__ __device__ static constexpr int sched_off(int G) { return misc_off(G) + 16 + 256; }
   static constexpr size_t bytes(int batch, int G) {
     return 1024 + static_cast<size_t>(sched_off(G)) + static_cast<size_t>(3 * batch + 1) * 4;
@@ -876,8 +882,7 @@ __global__ void __maxnreg__(224)
   float* m_area = reinterpret_cast<float*>(base + S::kMerge);
   float* l_area = m_area + NW * G;
   float* acc_area = reinterpret_cast<float*>(base + S::acc_off(G));
-  int* s_flag = reinterpret_cast<int*>(base + S::misc_off(G));
-  int* s_pages = s_flag + 4;
+  int* s_pages = reinterpret_cast<int*>(base + S::misc_off(G)) + 4;
   int* s_start = reinterpret_cast<int*>(base + S::sched_off(G));
   const int B = a.batch, H = a.kv_heads;
   int* s_len = s_start + B;
@@ -936,6 +941,22 @@ __global__ void __maxnreg__(224)
   it.per = N > 0 ? (N + P - 1) / P : 1;
   it.u = static_cast<long long>(c) * it.per;
   it.u1 = it.u + it.per < N ? it.u + it.per : N;
+
+  // The merge kernel may be scheduled now (it waits for this grid to finish
+  // before it reads anything this grid writes).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // Boundary record: block c's run starts at tile c * per.  If that cut lies
+  // inside a segment that began in block c - 1's run, it is the segment's
+  // first cut and block c names the segment for the merge kernel; every
+  // other block writes "none", so no record survives from an earlier pass.
+  if (tid == 0 && c > 0) {
+    PieceIter i0 = it;
+    Piece p0;
+    int4 rec = make_int4(-1, 0, 0, 0);
+    if (next_piece(i0, p0, s_pre, s_len, B, H, a.window, T) && p0.c_first == c - 1)
+      rec = make_int4(p0.seg, p0.c_first, p0.n_pieces, 0);
+    a.records[c] = rec;
+  }
 
   if (warp == 0) {
     // ================= producer
@@ -1156,93 +1177,6 @@ __global__ void __maxnreg__(224)
       } else if (FA_CHECK(a.status, slot_idx < a.max_partials, 402, slot_idx)) {
         a.part_o[(static_cast<size_t>(slot_idx) * G + h) * D + dim] = ov;
         if (dim == 0) a.part_lse[static_cast<size_t>(slot_idx) * G + h] = lv;
-      }
-    }
-    if (!whole) {
-      __threadfence();
-      named_barrier_sync(1, NCT);
-      if (ctid == 0) {
-        unsigned ticket = 0;
-        if (FA_CHECK(a.status, pc.seg < B * H && pc.n_pieces >= 1 &&
-                                   pc.c_first + pc.n_pieces - 1 + pc.seg < a.max_partials,
-                     403, pc.seg))
-          ticket = atomicInc(a.counters + pc.seg, static_cast<unsigned>(pc.n_pieces - 1));
-        *s_flag = (ticket == static_cast<unsigned>(pc.n_pieces - 1)) ? 1 : 0;
-      }
-      named_barrier_sync(1, NCT);
-      if (*s_flag) {
-        // last block of this segment: merge every block's (o, lse) exactly.
-        // 1) per head, lse = M + ln sum_k exp(lse_k - M) (one warp per head);
-        // 2) weights w_k = exp(lse_k - lse) into shared memory (the merge
-        //    area is free now); 3) out = sum_k w_k o_k with independent loads.
-        __threadfence();
-        float* s_w = acc_area;                 // [chunk][G] weights
-        float* s_lse = m_area;                 // [G] merged lse
-        const int cap = (NW * D) > 1 ? NW * D : 1;  // pieces per chunk (acc area holds NW*G*D)
-        for (int h = w; h < G; h += NW) {
-          float M = -CUDART_INF_F;
-          for (int k = lane; k < pc.n_pieces; k += 32)
-            M = fmaxf(M, __ldcg(a.part_lse + static_cast<size_t>(pc.c_first + k + pc.seg) * G + h));
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-          float Z = 0.f;
-          if (M != -CUDART_INF_F)
-            for (int k = lane; k < pc.n_pieces; k += 32) {
-              const float lk = __ldcg(a.part_lse + static_cast<size_t>(pc.c_first + k + pc.seg) * G + h);
-              if (lk != -CUDART_INF_F) Z += exp2_approx((lk - M) * kLog2e);
-            }
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, off);
-          if (lane == 0) s_lse[h] = (Z > 0.f) ? M + __logf(Z) : -CUDART_INF_F;
-        }
-        named_barrier_sync(1, NCT);
-        float accv[(D * 8 + NCT - 1) / NCT];
-        constexpr int PER = (D * 8 + NCT - 1) / NCT;  // outputs per thread at G = 8
-#pragma unroll
-        for (int r = 0; r < PER; ++r) accv[r] = 0.f;
-        for (int k0 = 0; k0 < pc.n_pieces; k0 += cap) {
-          const int kn = pc.n_pieces - k0 < cap ? pc.n_pieces - k0 : cap;
-          for (int x = ctid; x < kn * G; x += NCT) {
-            const int k = x / G, h = x - k * G;
-            const float lk = __ldcg(a.part_lse + static_cast<size_t>(pc.c_first + k0 + k + pc.seg) * G + h);
-            const float L = s_lse[h];
-            s_w[x] = (lk == -CUDART_INF_F || L == -CUDART_INF_F) ? 0.f : exp2_approx((lk - L) * kLog2e);
-          }
-          named_barrier_sync(1, NCT);
-#pragma unroll
-          for (int r = 0; r < PER; ++r) {
-            const int x = ctid + r * NCT;
-            if (x < G * D) {
-              const int h = x / D, dim = x - h * D;
-              const float* src = a.part_o + (static_cast<size_t>(pc.c_first + k0 + pc.seg) * G + h) * D + dim;
-              const size_t step = static_cast<size_t>(G) * D;
-              float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-              int k = 0;
-              for (; k + 4 <= kn; k += 4) {
-                const float o0 = __ldcg(src + (k + 0) * step), o1 = __ldcg(src + (k + 1) * step);
-                const float o2 = __ldcg(src + (k + 2) * step), o3 = __ldcg(src + (k + 3) * step);
-                s0 = fmaf(s_w[(k + 0) * G + h], o0, s0);
-                s1 = fmaf(s_w[(k + 1) * G + h], o1, s1);
-                s2 = fmaf(s_w[(k + 2) * G + h], o2, s2);
-                s3 = fmaf(s_w[(k + 3) * G + h], o3, s3);
-              }
-              for (; k < kn; ++k) s0 = fmaf(s_w[k * G + h], __ldcg(src + k * step), s0);
-              accv[r] += (s0 + s1) + (s2 + s3);
-            }
-          }
-          named_barrier_sync(1, NCT);
-        }
-#pragma unroll
-        for (int r = 0; r < PER; ++r) {
-          const int x = ctid + r * NCT;
-          if (x < G * D) {
-            const int h = x / D, dim = x - h * D;
-            const size_t row = static_cast<size_t>(pc.b) * a.qo_heads + static_cast<size_t>(pc.h) * G + h;
-            const float L = s_lse[h];
-            a.out[row * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(L == -CUDART_INF_F ? 0.f : accv[r]));
-            if (dim == 0 && a.lse != nullptr) a.lse[row] = L;
-          }
-        }
       }
     }
     named_barrier_sync(1, NCT);  // merge area is reused by the next piece

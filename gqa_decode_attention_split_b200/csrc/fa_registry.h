@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 #include <stddef.h>
+#include <stdint.h>
 
 namespace fa {
 
@@ -25,6 +26,22 @@ struct KernelEntry {
   size_t (*smem_bytes)(int batch, int group);
   cudaError_t (*launch)(const KernelArgs& args, int grid, size_t smem, cudaStream_t stream);
 };
+
+// Arguments of the split-segment merge kernel (fa_split_merge.cu).
+struct SplitMergeArgs {
+  const int4* records;    // [num_records]: (segment, first block, pieces) or segment -1
+  const float* part_o;    // [max_partials][group][head_dim], each o_k normalised
+  const float* part_lse;  // [max_partials][group], natural log
+  uint16_t* out;          // bf16 [batch][qo_heads][head_dim]
+  float* lse;             // [batch][qo_heads] or null
+  int num_records;        // blocks of the main launch
+  int group, kv_heads, qo_heads, batch;
+  long long max_partials;
+};
+
+// Enqueues the merge behind the main kernel on `stream` as a programmatic
+// dependent launch; nothing is launched for a single-block pass.
+cudaError_t launch_split_merge(const SplitMergeArgs& args, int head_dim, cudaStream_t stream);
 
 // Each instantiation unit appends its variants; returns how many it wrote.
 int register_d64(KernelEntry* out, int cap);

@@ -6,8 +6,8 @@
 // the allocator (an allocator-free inference runtime, a plugin host that owns
 // all device memory, a path that must not synchronise the device, which
 // cudaMalloc/cudaFree may do).  For them this entry point takes no workspace
-// argument: the scratch the kernel needs (device-check word, per-segment
-// ticket counters, partial softmax states) lives in a file-scope
+// argument: the scratch the kernels need (device-check word, boundary
+// records, partial softmax states) lives in a file-scope
 // __device__ array of fixed size, which every GPU that loads this library
 // holds until the process exits.
 #include <cuda_runtime.h>
@@ -87,8 +87,8 @@ extern "C" fa_status fa_decode_run_static(const fa_plan* plan, const void* q, co
   void* scratch = nullptr;
   st = scratch_address(&scratch);
   if (st != FA_OK) return st;
-  // The device-check word and the ticket counters must start at zero; the
-  // array keeps whatever the previous call (or an aborted one) left there.
+  // The device-check word must start at zero; the array keeps whatever the
+  // previous call (or an aborted one) left there.
   cudaError_t e = cudaMemsetAsync(scratch, 0, fa::plan_zero_prefix_bytes(plan),
                                   static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_error("clearing the static scratch", e);

@@ -168,10 +168,14 @@ FA_API void fa_plan_destroy(fa_plan* plan);
  *              A request with no visible key gets out = 0, lse = -inf.
  *  workspace   device scratch of >= the plan's workspace_bytes, 256-byte
  *              aligned, zero-filled once before its first use (and again
- *              after FA_ERR_DEVICE_CHECK).  The library leaves its ticket
- *              counters at zero after every completed call, so one workspace
- *              serves any number of calls in stream order.  Two calls that
- *              share a workspace must not overlap on the GPU.
+ *              after FA_ERR_DEVICE_CHECK).  Apart from its check word every
+ *              byte is written by a pass before that pass reads it, so one
+ *              workspace serves any number of calls in stream order.  Two
+ *              calls that share a workspace must not overlap on the GPU.
+ * A pass is one kernel launch, plus a second small one when some segment is
+ * cut across thread blocks: it merges those segments' partial states and is
+ * enqueued as a programmatic dependent launch of the first (it is scheduled
+ * early and waits on the device for the first to finish).
  * No allocation, no synchronisation, no host<->device copies.  Errors:
  * FA_ERR_INVALID_ARG, FA_ERR_MISALIGNED, FA_ERR_WORKSPACE_TOO_SMALL,
  * FA_ERR_CUDA (launch failure).  Device-side checks are reported later by
@@ -203,7 +207,7 @@ FA_API fa_status fa_decode_run(const fa_plan* plan, const void* q, const void* k
  *    stream capture.
  *  - Every call on a device shares the one array, which keeps what the
  *    previous call left.  Each call clears the part that must start at zero
- *    (check word, ticket counters) in stream order before its kernel.  Calls
+ *    (the check word) in stream order before its kernel.  Calls
  *    that overlap on the GPU (other streams, other host threads) race on the
  *    array and must be avoided.
  *  - A plan whose workspace_bytes exceeds FA_STATIC_WORKSPACE_BYTES is

@@ -140,7 +140,7 @@ def test_lse_optional_and_workspace_reuse():
     p = dev.plan(num_ctas=16)
     ws = p.new_workspace()
     ref_out, ref_lse = oracle.decode_all(x)
-    for _ in range(3):  # counters return to zero after every call
+    for _ in range(3):  # the workspace keeps the previous call's records and partials
         out, lse = dev.run(p, workspace=ws)
         o, l = to_numpy(out, lse)
         assert_matches(o, l, ref_out, ref_lse, what="reuse")
