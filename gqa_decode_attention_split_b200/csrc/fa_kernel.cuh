@@ -1144,17 +1144,21 @@ __global__ void __maxnreg__(224)
     }
     base_i += n;
     // ---- merge the warps' states of this piece
+    const float vs = Cons::C::ES == 1 ? __ldg(a.v_scale + pc.h) : 1.f;  // in flight across the barrier
     cons.end_piece(m_area, l_area, acc_area, w, lane, G);
     named_barrier_sync(1, NCT);
     const bool whole = pc.n_pieces == 1;
     const int slot_idx = c + pc.seg;
-    const float vs = Cons::C::ES == 1 ? __ldg(a.v_scale + pc.h) : 1.f;
-    for (int x = ctid; x < G * D; x += NCT) {
-      const int h = x / D, dim = x - h * D;
+    // four dims per thread: float4 reads of the warps' accumulators, one
+    // 16-byte partial store (or 8-byte bf16x4 output store) per thread
+    constexpr int D4 = D / 4;
+    for (int x4 = ctid; x4 < G * D4; x4 += NCT) {
+      const int h = x4 / D4, dim = (x4 - h * D4) * 4;
       float M = -CUDART_INF_F;
 #pragma unroll
       for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, m_area[ww * G + h]);
-      float Ls = 0.f, O = 0.f;
+      float Ls = 0.f;
+      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
       if (M != -CUDART_INF_F) {
 #pragma unroll
         for (int ww = 0; ww < NW; ++ww) {
@@ -1162,20 +1166,31 @@ __global__ void __maxnreg__(224)
           if (mw == -CUDART_INF_F) continue;
           const float sc = exp2_approx(mw - M);
           Ls = fmaf(l_area[ww * G + h], sc, Ls);
-          O = fmaf(acc_area[(ww * G + h) * D + dim], sc, O);
+          const float4 av = *reinterpret_cast<const float4*>(acc_area + (ww * G + h) * D + dim);
+          O.x = fmaf(av.x, sc, O.x);
+          O.y = fmaf(av.y, sc, O.y);
+          O.z = fmaf(av.z, sc, O.z);
+          O.w = fmaf(av.w, sc, O.w);
         }
       }
       const bool empty = !(Ls > 0.f);
-      const float ov = empty ? 0.f : O / Ls * vs;
+      const float f = empty ? 0.f : vs / Ls;
+      O.x *= f;
+      O.y *= f;
+      O.z *= f;
+      O.w *= f;
       const float lv = empty ? -CUDART_INF_F : (M + __log2f(Ls)) * kLn2;
       const size_t row = static_cast<size_t>(pc.b) * a.qo_heads + static_cast<size_t>(pc.h) * G + h;
       if (whole) {
         if (FA_CHECK(a.status, row < static_cast<size_t>(B) * a.qo_heads, 401, row)) {
-          a.out[row * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(ov));
+          uint2 packed;
+          packed.x = pack_bf16x2(O.x, O.y);
+          packed.y = pack_bf16x2(O.z, O.w);
+          *reinterpret_cast<uint2*>(a.out + row * D + dim) = packed;
           if (dim == 0 && a.lse != nullptr) a.lse[row] = lv;
         }
       } else if (FA_CHECK(a.status, slot_idx < a.max_partials, 402, slot_idx)) {
-        a.part_o[(static_cast<size_t>(slot_idx) * G + h) * D + dim] = ov;
+        *reinterpret_cast<float4*>(a.part_o + (static_cast<size_t>(slot_idx) * G + h) * D + dim) = O;
         if (dim == 0) a.part_lse[static_cast<size_t>(slot_idx) * G + h] = lv;
       }
     }
