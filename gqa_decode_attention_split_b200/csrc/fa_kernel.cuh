@@ -856,7 +856,8 @@ struct SmemLayout {
     return kMerge + ((C::NW * G * 2 * 4 + 15) / 16) * 16;
   }
   __host__ __device__ static constexpr int misc_off(int G) { return acc_off(G) + C::NW * G * D * 4; }
-  // misc: 16 spare bytes, then 64 staged page ids (256 B)
+  // misc: merge counter (4 B), pad, merge-free mbarrier (8 B), then 64
+  // staged page ids (256 B)
   __host__ __device__ static constexpr int sched_off(int G) { return misc_off(G) + 16 + 256; }
   static constexpr size_t bytes(int batch, int G) {
     return 1024 + static_cast<size_t>(sched_off(G)) + static_cast<size_t>(3 * batch + 1) * 4;
@@ -882,6 +883,8 @@ __global__ void __maxnreg__(224)
   float* m_area = reinterpret_cast<float*>(base + S::kMerge);
   float* l_area = m_area + NW * G;
   float* acc_area = reinterpret_cast<float*>(base + S::acc_off(G));
+  int* s_mcnt = reinterpret_cast<int*>(base + S::misc_off(G));  // warps done with the open piece
+  const uint32_t mfree = sbase + S::misc_off(G) + 8;              // completes when a piece is merged
   int* s_pages = reinterpret_cast<int*>(base + S::misc_off(G)) + 4;
   int* s_start = reinterpret_cast<int*>(base + S::sched_off(G));
   const int B = a.batch, H = a.kv_heads;
@@ -914,6 +917,8 @@ __global__ void __maxnreg__(224)
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
+    mbar_init(mfree, 1);
+    *s_mcnt = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -1116,6 +1121,7 @@ __global__ void __maxnreg__(224)
   uint32_t ph = 0;       // wrap parity of that stage
   int base_i = 0;        // block-sequence index of the current piece's first tile
   bool alive = true;
+  int piece = 0;         // pieces this block has finished (merge-area uses)
   Piece pc;
   while (next_piece(it, pc, s_pre, s_len, B, H, a.window, T)) {
     const int L = s_len[pc.b];
@@ -1143,58 +1149,97 @@ __global__ void __maxnreg__(224)
       }
     }
     base_i += n;
-    // ---- merge the warps' states of this piece
-    const float vs = Cons::C::ES == 1 ? __ldg(a.v_scale + pc.h) : 1.f;  // in flight across the barrier
+    // ---- merge the warps' states of this piece, without a block barrier:
+    // each warp parks its state in the merge area and goes on to its tiles
+    // of the next piece; the last warp to park merges the NW states, writes
+    // the result (or the partial) and frees the area.  A warp waits only if
+    // it finishes its share of the next piece before that merge is done.
+    const float vs = Cons::C::ES == 1 ? __ldg(a.v_scale + pc.h) : 1.f;
+    if (piece > 0 && alive) {
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(mfree, (piece - 1) & 1, kWaitLimitNs));
+      if (!ok) {
+        if (lane == 0) record_timeout(a.status, 4, piece, 0, (piece - 1) & 1, mfree);
+        alive = false;
+      }
+    }
     cons.end_piece(m_area, l_area, acc_area, w, lane, G);
-    named_barrier_sync(1, NCT);
-    const bool whole = pc.n_pieces == 1;
-    const int slot_idx = c + pc.seg;
-    // four dims per thread: float4 reads of the warps' accumulators, one
-    // 16-byte partial store (or 8-byte bf16x4 output store) per thread
-    constexpr int D4 = D / 4;
-    for (int x4 = ctid; x4 < G * D4; x4 += NCT) {
-      const int h = x4 / D4, dim = (x4 - h * D4) * 4;
-      float M = -CUDART_INF_F;
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+      __threadfence_block();  // this warp's state is visible before it is counted
+      last = atomicAdd(s_mcnt, 1) == NW - 1;
+      __threadfence_block();  // and the other warps' states before they are read
+    }
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last) {
+      __syncwarp();
+      const bool whole = pc.n_pieces == 1;
+      const int slot_idx = c + pc.seg;
+      // 1) lane h < G: the head's max over the warps' states, each warp's
+      //    weight exp(m_w - M) / L (times the fp8 V scale) written over m_w,
+      //    and the head's lse.  end_piece writes every warp's accumulator
+      //    (zeros for a warp without tiles), so a zero weight is exact.
+      if (lane < G) {
+        const int h = lane;
+        float M = -CUDART_INF_F;
 #pragma unroll
-      for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, m_area[ww * G + h]);
-      float Ls = 0.f;
-      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (M != -CUDART_INF_F) {
+        for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, m_area[ww * G + h]);
+        float scw[NW];
+        float Ls = 0.f;
 #pragma unroll
         for (int ww = 0; ww < NW; ++ww) {
           const float mw = m_area[ww * G + h];
-          if (mw == -CUDART_INF_F) continue;
-          const float sc = exp2_approx(mw - M);
-          Ls = fmaf(l_area[ww * G + h], sc, Ls);
-          const float4 av = *reinterpret_cast<const float4*>(acc_area + (ww * G + h) * D + dim);
-          O.x = fmaf(av.x, sc, O.x);
-          O.y = fmaf(av.y, sc, O.y);
-          O.z = fmaf(av.z, sc, O.z);
-          O.w = fmaf(av.w, sc, O.w);
+          scw[ww] = (M == -CUDART_INF_F || mw == -CUDART_INF_F) ? 0.f : exp2_approx(mw - M);
+          Ls = fmaf(l_area[ww * G + h], scw[ww], Ls);
+        }
+        const bool empty = !(Ls > 0.f);
+        const float f = empty ? 0.f : vs / Ls;
+#pragma unroll
+        for (int ww = 0; ww < NW; ++ww) m_area[ww * G + h] = scw[ww] * f;
+        const float lv = empty ? -CUDART_INF_F : (M + __log2f(Ls)) * kLn2;
+        const size_t row = static_cast<size_t>(pc.b) * a.qo_heads + static_cast<size_t>(pc.h) * G + h;
+        if (whole) {
+          if (a.lse != nullptr && FA_CHECK(a.status, row < static_cast<size_t>(B) * a.qo_heads, 401, row))
+            a.lse[row] = lv;
+        } else if (FA_CHECK(a.status, slot_idx < a.max_partials, 402, slot_idx)) {
+          a.part_lse[static_cast<size_t>(slot_idx) * G + h] = lv;
         }
       }
-      const bool empty = !(Ls > 0.f);
-      const float f = empty ? 0.f : vs / Ls;
-      O.x *= f;
-      O.y *= f;
-      O.z *= f;
-      O.w *= f;
-      const float lv = empty ? -CUDART_INF_F : (M + __log2f(Ls)) * kLn2;
-      const size_t row = static_cast<size_t>(pc.b) * a.qo_heads + static_cast<size_t>(pc.h) * G + h;
-      if (whole) {
-        if (FA_CHECK(a.status, row < static_cast<size_t>(B) * a.qo_heads, 401, row)) {
-          uint2 packed;
-          packed.x = pack_bf16x2(O.x, O.y);
-          packed.y = pack_bf16x2(O.z, O.w);
-          *reinterpret_cast<uint2*>(a.out + row * D + dim) = packed;
-          if (dim == 0 && a.lse != nullptr) a.lse[row] = lv;
+      __syncwarp();
+      // 2) four dims per lane: out = sum_w weight_w * acc_w, branch-free
+      //    float4 reads, one 16-byte partial store (or bf16x4 output store)
+      constexpr int D4 = D / 4;
+      for (int x4 = lane; x4 < G * D4; x4 += 32) {
+        const int h = x4 / D4, dim = (x4 - h * D4) * 4;
+        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int ww = 0; ww < NW; ++ww) {
+          const float f = m_area[ww * G + h];
+          const float4 av = *reinterpret_cast<const float4*>(acc_area + (ww * G + h) * D + dim);
+          O.x = fmaf(av.x, f, O.x);
+          O.y = fmaf(av.y, f, O.y);
+          O.z = fmaf(av.z, f, O.z);
+          O.w = fmaf(av.w, f, O.w);
         }
-      } else if (FA_CHECK(a.status, slot_idx < a.max_partials, 402, slot_idx)) {
-        *reinterpret_cast<float4*>(a.part_o + (static_cast<size_t>(slot_idx) * G + h) * D + dim) = O;
-        if (dim == 0) a.part_lse[static_cast<size_t>(slot_idx) * G + h] = lv;
+        const size_t row = static_cast<size_t>(pc.b) * a.qo_heads + static_cast<size_t>(pc.h) * G + h;
+        if (whole) {
+          if (FA_CHECK(a.status, row < static_cast<size_t>(B) * a.qo_heads, 401, row)) {
+            uint2 packed;
+            packed.x = pack_bf16x2(O.x, O.y);
+            packed.y = pack_bf16x2(O.z, O.w);
+            *reinterpret_cast<uint2*>(a.out + row * D + dim) = packed;
+          }
+        } else if (FA_CHECK(a.status, slot_idx < a.max_partials, 402, slot_idx)) {
+          *reinterpret_cast<float4*>(a.part_o + (static_cast<size_t>(slot_idx) * G + h) * D + dim) = O;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
+        *s_mcnt = 0;
+        mbar_arrive(mfree);
       }
     }
-    named_barrier_sync(1, NCT);  // merge area is reused by the next piece
+    ++piece;
   }
 }
 
