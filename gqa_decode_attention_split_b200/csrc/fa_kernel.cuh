@@ -105,6 +105,7 @@ struct KernelArgs {
 
 constexpr int kSmemPerBlock = 232448;  // 227 KB of shared memory per block (sm_100)
 constexpr int kSchedReserve = 8192;    // schedule arrays for up to 682 requests
+constexpr int kScaleCap = 128;         // fp8 per-kv-head scales kept in shared memory
 
 // Shared-memory tile geometry for one head_dim / element type.  A token row
 // is cut into NP planes of CB = min(128, row bytes) bytes (the widest box row
@@ -132,11 +133,21 @@ struct TileCfg {
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   static constexpr int NW = NWARPS;
   static constexpr int MERGE_BYTES = NW * GMAX * (D + 2) * 4;
-  static constexpr int RING_BUDGET = kSmemPerBlock - 1024 - kSchedReserve - 512 - MERGE_BYTES;
-  static constexpr int STAGES_RAW = RING_BUDGET / STAGE_BYTES;
-  static constexpr int STAGES_PER_WARP_RAW = STAGES_RAW / NW;
-  static constexpr int STAGES_PER_WARP =
-      STAGES_PER_WARP_RAW > FA_MAX_STAGES_PER_WARP ? FA_MAX_STAGES_PER_WARP : STAGES_PER_WARP_RAW;
+  // q area: four mbarriers, then (STAGE_Q) two slots of a piece's GMAX query
+  // rows (bf16) that the producer stages, then (fp8) the k / v scale tables.
+  // Query rows are staged only where the slots cost no ring stage; otherwise
+  // consumers read them from global memory.
+  static constexpr int QSLOT_BYTES = GMAX * D * 2;
+  static constexpr int SCALE_BYTES = FP8 ? 2 * kScaleCap * 4 : 0;
+  static constexpr int BASE_BUDGET = kSmemPerBlock - 1024 - kSchedReserve - 512 - MERGE_BYTES - 32 - SCALE_BYTES;
+  static constexpr int stages_per_warp(int budget) {
+    return budget / STAGE_BYTES / NW > FA_MAX_STAGES_PER_WARP ? FA_MAX_STAGES_PER_WARP
+                                                               : budget / STAGE_BYTES / NW;
+  }
+  static constexpr bool STAGE_Q = stages_per_warp(BASE_BUDGET - 2 * QSLOT_BYTES) == stages_per_warp(BASE_BUDGET);
+  static constexpr int QAREA_BYTES = 32 + (STAGE_Q ? 2 * QSLOT_BYTES : 0) + SCALE_BYTES;
+  static constexpr int RING_BUDGET = BASE_BUDGET + 32 + SCALE_BYTES - QAREA_BYTES;
+  static constexpr int STAGES_PER_WARP = stages_per_warp(RING_BUDGET);
   static constexpr int STAGES = NW * STAGES_PER_WARP;
   static_assert(STAGES_PER_WARP >= 1, "every consumer warp needs a stage");
   static_assert(STAGES % NW == 0, "a stage must belong to one consumer warp");
@@ -335,20 +346,23 @@ struct SimtConsumer {
     return tile_addr<C>(tile, r, chunk_plane(k), chunk_in_plane(k), swz);
   }
 
-  __device__ __forceinline__ void begin_piece(const KernelArgs& a, int b, int hkv, int lane) {
+  // qs: the piece's G query rows (staged in shared memory, or in global
+  // memory where the tile geometry leaves no room); kscale: the fp8
+  // K scale of the piece's kv head (1 for bf16).
+  __device__ __forceinline__ void begin_piece(const KernelArgs& a, const uint16_t* qs, float kscale,
+                                              int lane) {
     slot = lane / LPT;
     j = lane % LPT;
     float scale = a.score_scale;
-    if constexpr (FP8) scale *= __ldg(a.k_scale + hkv);
+    if constexpr (FP8) scale *= kscale;
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      const uint16_t* qrow =
-          a.q + (static_cast<size_t>(b) * a.qo_heads + static_cast<size_t>(hkv) * G + h) * D;
+      const uint16_t* qrow = qs + h * D;
 #pragma unroll
       for (int k = 0; k < CPL; ++k) {
 #pragma unroll
         for (int e = 0; e < EPC; e += 8) {
-          const uint4 w = __ldg(reinterpret_cast<const uint4*>(qrow + dim_of(k, e)));
+          const uint4 w = *reinterpret_cast<const uint4*>(qrow + dim_of(k, e));
           const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -513,18 +527,21 @@ struct MmaConsumer {
   float sscale[2];
   int g, t;
 
-  __device__ __forceinline__ void begin_piece(const KernelArgs& a, int b, int hkv, int lane) {
+  // qs: the piece's G query rows (staged in shared memory, or in global
+  // memory where the tile geometry leaves no room); kscale: the fp8
+  // K scale of the piece's kv head (1 for bf16).
+  __device__ __forceinline__ void begin_piece(const KernelArgs& a, const uint16_t* qs, float kscale,
+                                              int lane) {
     g = lane >> 2;
     t = lane & 3;
     const int G = a.group;
     const bool real = g < G;
-    const uint16_t* qrow =
-        a.q + (static_cast<size_t>(b) * a.qo_heads + static_cast<size_t>(hkv) * G + (real ? g : 0)) * D;
+    const uint16_t* qrow = qs + (real ? g : 0) * D;
     if constexpr (!FP8) {
 #pragma unroll
       for (int kk = 0; kk < KS; ++kk) {
-        qb[kk][0] = real ? __ldg(reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * t)) : 0u;
-        qb[kk][1] = real ? __ldg(reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * t + 8)) : 0u;
+        qb[kk][0] = real ? *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * t) : 0u;
+        qb[kk][1] = real ? *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * t + 8) : 0u;
       }
       sscale[0] = sscale[1] = a.score_scale;
     } else {
@@ -533,7 +550,7 @@ struct MmaConsumer {
       uint32_t qw[BPT / 2];
 #pragma unroll
       for (int i = 0; i < BPT / 8; ++i) {
-        const uint4 w = real ? __ldg(reinterpret_cast<const uint4*>(qrow + BPT * t + 8 * i))
+        const uint4 w = real ? *reinterpret_cast<const uint4*>(qrow + BPT * t + 8 * i)
                              : make_uint4(0, 0, 0, 0);
         qw[4 * i] = w.x;
         qw[4 * i + 1] = w.y;
@@ -588,7 +605,7 @@ struct MmaConsumer {
       }
       const int sh0 = __shfl_sync(0xffffffffu, sh, (2 * t) * 4);
       const int sh1 = __shfl_sync(0xffffffffu, sh, (2 * t + 1) * 4);
-      const float base = a.score_scale * __ldg(a.k_scale + hkv);
+      const float base = a.score_scale * kscale;
       sscale[0] = base * ldexpf(1.f, -sh0);
       sscale[1] = base * ldexpf(1.f, -sh1);
     }
@@ -845,7 +862,8 @@ struct MmaConsumer {
 // ------------------------------------------------------------- kernel
 // Block shared memory, from a 1024-aligned base:
 //   ring [STAGES][K tile, V tile] | full[STAGES], empty[STAGES] mbarriers |
-//   m[NW][G], l[NW][G] | acc[NW][G][D] | flag | pages[64] | start[B], len[B], pre[B+1]
+//   m[NW][G], l[NW][G] | acc[NW][G][D] | merge counter, merge mbarrier |
+//   pages[64] | q mbarriers, q slots, scales | start[B], len[B], pre[B+1]
 template <class Cons>
 struct SmemLayout {
   using C = typename Cons::C;
@@ -858,7 +876,10 @@ struct SmemLayout {
   __host__ __device__ static constexpr int misc_off(int G) { return acc_off(G) + C::NW * G * D * 4; }
   // misc: merge counter (4 B), pad, merge-free mbarrier (8 B), then 64
   // staged page ids (256 B)
-  __host__ __device__ static constexpr int sched_off(int G) { return misc_off(G) + 16 + 256; }
+  // q area: qfull[2], qempty[2] mbarriers (32 B) | q slots [2][QSLOT_BYTES]
+  // (if STAGE_Q) | fp8: k scales [kScaleCap], v scales [kScaleCap]
+  __host__ __device__ static constexpr int q_off(int G) { return misc_off(G) + 16 + 256; }
+  __host__ __device__ static constexpr int sched_off(int G) { return q_off(G) + C::QAREA_BYTES; }
   static constexpr size_t bytes(int batch, int G) {
     return 1024 + static_cast<size_t>(sched_off(G)) + static_cast<size_t>(3 * batch + 1) * 4;
   }
@@ -886,6 +907,10 @@ __global__ void __maxnreg__(224)
   int* s_mcnt = reinterpret_cast<int*>(base + S::misc_off(G));  // warps done with the open piece
   const uint32_t mfree = sbase + S::misc_off(G) + 8;              // completes when a piece is merged
   int* s_pages = reinterpret_cast<int*>(base + S::misc_off(G)) + 4;
+  const uint32_t qfull0 = sbase + S::q_off(G), qempty0 = qfull0 + 16;  // [2] each
+  uint16_t* q_slots = reinterpret_cast<uint16_t*>(base + S::q_off(G) + 32);
+  float* s_kscale = reinterpret_cast<float*>(base + S::q_off(G) + 32 + (C::STAGE_Q ? 2 * C::QSLOT_BYTES : 0));
+  float* s_vscale = s_kscale + kScaleCap;
   int* s_start = reinterpret_cast<int*>(base + S::sched_off(G));
   const int B = a.batch, H = a.kv_heads;
   int* s_len = s_start + B;
@@ -912,6 +937,13 @@ __global__ void __maxnreg__(224)
     s_len[b] = L;
     if (bad) atomicOr(a.status, kFlagBadIndptr);
   }
+  const bool scales_in_smem = H <= kScaleCap;
+  if (C::ES == 1 && scales_in_smem) {
+    for (int i = tid; i < H; i += blockDim.x) {
+      s_kscale[i] = __ldg(a.k_scale + i);
+      s_vscale[i] = __ldg(a.v_scale + i);
+    }
+  }
   if (tid == 32) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(full0 + 8 * s, 1);
@@ -919,6 +951,10 @@ __global__ void __maxnreg__(224)
     }
     mbar_init(mfree, 1);
     *s_mcnt = 0;
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(qfull0 + 8 * s, 1);
+      mbar_init(qempty0 + 8 * s, NW);
+    }
     fence_mbar_init();
   }
   __syncthreads();
@@ -967,114 +1003,174 @@ __global__ void __maxnreg__(224)
     // ================= producer
     // Lane 0 walks the block's tiles in order and, per tile, waits for its
     // ring stage to be free, arms the stage's barrier with the tile's bytes
-    // and issues the bulk tensor copies.  For paged KV the whole warp first
-    // stages the page ids of the next window of tiles in shared memory
-    // (coalesced reads of the page table), so lane 0's loop has no global
-    // loads and no warp-wide operations.
+    // and issues the bulk tensor copies.  Tiles go out in windows.  For paged
+    // KV the page ids of the current window sit in shared memory (read from
+    // the page table by the whole warp, coalesced), so lane 0's loop has no
+    // global loads and no warp-wide operations; the next window's ids are
+    // loaded into registers before lane 0 issues the current window and
+    // stored after it, so the page-table round trip overlaps the copies.
     const uint64_t pol = l2_evict_first_policy();
     if (lane == 0) {
       prefetch_tensormap(&a.kmap);
       prefetch_tensormap(&a.vmap);
     }
     const int NB = T / a.box_t;  // boxes per tile (paged: one page each, contiguous: 1)
+    // tiles per window of 64 page ids (a window that starts inside a page may
+    // touch one page more than its token count suggests)
+    const int win_paged = !a.paged ? 1 : (ps >= T ? 63 * (ps / T) : (64 * ps) / T);
     int stage = 0;
     uint32_t ph = 0;             // lane 0's ring position (stage, wrap parity)
     int issued = 0;
+    int pq = 0;                  // pieces whose query rows were staged
     bool ok = true;
+    // this lane's two page ids of the window starting at tile w of piece p
+    auto load_ids = [&](const Piece& p, int w, int (&v)[2], bool (&in)[2]) {
+      const int np = (s_len[p.b] + ps - 1) >> a.page_shift;
+      const int pb = (w * T) >> a.page_shift;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int e = pb + half * 32 + lane;
+        in[half] = e < np;
+        v[half] = in[half] ? __ldg(a.page_table + static_cast<long long>(p.b) * a.pt_stride + e) : -1;
+      }
+    };
+    auto store_ids = [&](const int (&v)[2], const bool (&in)[2]) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        int x = v[half];
+        if (in[half] && (x < 0 || static_cast<long long>(x) >= a.kv_rows)) {
+          atomicOr(a.status, kFlagBadPage);
+          x = -1;  // the copy reads out of range: zeros, no memory access
+        }
+        s_pages[half * 32 + lane] = in[half] ? x : -1;
+      }
+    };
     Piece pc;
-    while (ok && next_piece(it, pc, s_pre, s_len, B, H, a.window, T)) {
+    bool have = next_piece(it, pc, s_pre, s_len, B, H, a.window, T);
+    int w0 = have ? pc.t0 : 0;
+    if (have && a.paged) {
+      int v[2];
+      bool in[2];
+      load_ids(pc, w0, v, in);
+      store_ids(v, in);
+      __syncwarp();
+    }
+    while (ok && have) {
       const int L = s_len[pc.b];
-      // tiles per window of 64 staged page ids (a window that starts inside a
-      // page may touch one page more than its token count suggests)
-      const int tiles_per_win = a.paged ? (ps >= T ? 63 * (ps / T) : (64 * ps) / T) : (pc.t1 - pc.t0);
-      for (int w0 = pc.t0; w0 < pc.t1 && ok; w0 += tiles_per_win) {
-        const int w1 = w0 + tiles_per_win < pc.t1 ? w0 + tiles_per_win : pc.t1;
-        int pbase = 0, npages = 0;
-        if (a.paged) {
-          npages = (L + ps - 1) >> a.page_shift;
-          pbase = (w0 * T) >> a.page_shift;
-          __syncwarp();
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const int e = pbase + half * 32 + lane;
-            int v = -1;
-            if (e < npages) {
-              v = __ldg(a.page_table + static_cast<long long>(pc.b) * a.pt_stride + e);
-              if (v < 0 || static_cast<long long>(v) >= a.kv_rows) {
-                atomicOr(a.status, kFlagBadPage);
-                v = -1;  // the copy reads out of range: zeros, no memory access
-              }
-            }
-            s_pages[half * 32 + lane] = v;
-          }
-          __syncwarp();
-        }
-        if (lane == 0) {
-          for (int tt = w0; tt < w1; ++tt) {
-            if (!mbar_wait(empty0 + 8 * stage, ph ^ 1u, kWaitLimitNs)) {
-              record_timeout(a.status, 1, issued, stage, ph ^ 1u, empty0 + 8 * stage);
-              ok = false;
-              break;
-            }
-            const uint32_t fb = full0 + 8 * stage;
-            const uint32_t kdst = ring + stage * C::STAGE_BYTES;
-            const uint32_t vdst = kdst + C::TILE_BYTES;
-            mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
-            if (!a.paged) {
-              const int row = s_start[pc.b] + tt * T;
-              if constexpr (C::TOKEN_MAJOR) {
-                tma_load_4d(kdst, &a.kmap, fb, 0, 0, pc.h, row, pol);
-                tma_load_4d(vdst, &a.vmap, fb, 0, 0, pc.h, row, pol);
-              } else {
-#pragma unroll
-                for (int p = 0; p < C::NP; ++p) {
-                  const uint32_t off = p * (T * C::CB);
-                  if (FA_CHECK(a.status, off + T * C::CB <= C::TILE_BYTES && (off & 127u) == 0, 301, off)) {
-                    tma_load_3d(kdst + off, &a.kmap, fb, p * (C::CB / C::ES), pc.h, row, pol);
-                    tma_load_3d(vdst + off, &a.vmap, fb, p * (C::CB / C::ES), pc.h, row, pol);
-                  }
-                }
-              }
-            } else if constexpr (C::TOKEN_MAJOR) {
-              for (int jb = 0; jb < NB; ++jb) {
-                const int tok = tt * T + jb * a.box_t;
-                const int pidx = tok >> a.page_shift;
-                const int page = (pidx < npages && pidx - pbase < 64) ? s_pages[pidx - pbase] : -1;
-                const int slot0 = tok & (ps - 1);
-                const uint32_t off = jb * a.box_t * C::ROWB;
-                if (FA_CHECK(a.status, off + a.box_t * C::ROWB <= C::TILE_BYTES && (off & 127u) == 0 &&
-                                           pidx - pbase >= 0 && pidx - pbase < 64,
-                             303, off)) {
-                  tma_load_5d(kdst + off, &a.kmap, fb, 0, 0, pc.h, slot0, page, pol);
-                  tma_load_5d(vdst + off, &a.vmap, fb, 0, 0, pc.h, slot0, page, pol);
-                }
-              }
-            } else {
-              for (int jb = 0; jb < NB; ++jb) {
-                const int tok = tt * T + jb * a.box_t;
-                const int pidx = tok >> a.page_shift;
-                const int page = (pidx < npages && pidx - pbase < 64) ? s_pages[pidx - pbase] : -1;
-                const int slot0 = tok & (ps - 1);
-#pragma unroll
-                for (int p = 0; p < C::NP; ++p) {
-                  const uint32_t off = p * (T * C::CB) + jb * a.box_t * C::CB;
-                  if (FA_CHECK(a.status, off + a.box_t * C::CB <= C::TILE_BYTES && (off & 127u) == 0 &&
-                                             pidx - pbase >= 0 && pidx - pbase < 64,
-                               302, off)) {
-                    tma_load_4d(kdst + off, &a.kmap, fb, p * (C::CB / C::ES), pc.h, slot0, page, pol);
-                    tma_load_4d(vdst + off, &a.vmap, fb, p * (C::CB / C::ES), pc.h, slot0, page, pol);
-                  }
-                }
-              }
-            }
-            ++issued;
-            if (++stage == C::STAGES) {
-              stage = 0;
-              ph ^= 1u;
+      if (w0 == pc.t0) {
+        // stage the piece's G query rows (contiguous in q) in q slot pq % 2
+        // once the consumers have read what the slot held two pieces ago
+        if (C::STAGE_Q && lane == 0) {
+          const int qs = pq & 1;
+          const uint32_t qpar = ((pq >> 1) & 1) ^ 1u;
+          if (!mbar_wait(qempty0 + 8 * qs, qpar, kWaitLimitNs)) {
+            record_timeout(a.status, 5, pq, qs, qpar, qempty0 + 8 * qs);
+            ok = false;
+          } else {
+            const uint32_t qbytes = static_cast<uint32_t>(G * D * 2);
+            if (FA_CHECK(a.status, qbytes <= static_cast<uint32_t>(C::QSLOT_BYTES), 304, qbytes)) {
+              mbar_arrive_expect_tx(qfull0 + 8 * qs, qbytes);
+              bulk_load(smem_addr(q_slots) + qs * C::QSLOT_BYTES,
+                        a.q + (static_cast<size_t>(pc.b) * a.qo_heads + static_cast<size_t>(pc.h) * G) * D,
+                        qbytes, qfull0 + 8 * qs);
             }
           }
         }
+        ++pq;
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+      }
+      const int w1 = a.paged && w0 + win_paged < pc.t1 ? w0 + win_paged : pc.t1;
+      // the window after this one: the rest of this piece, else the next piece
+      PieceIter itn = it;
+      Piece pn = pc;
+      int nw0 = w1;
+      bool nhave = true;
+      if (w1 >= pc.t1) {
+        nhave = next_piece(itn, pn, s_pre, s_len, B, H, a.window, T);
+        nw0 = nhave ? pn.t0 : 0;
+      }
+      int nv[2] = {-1, -1};
+      bool nin[2] = {false, false};
+      if (a.paged && nhave) load_ids(pn, nw0, nv, nin);  // in flight during the issue loop
+      const int npages = a.paged ? (L + ps - 1) >> a.page_shift : 0;
+      const int pbase = a.paged ? (w0 * T) >> a.page_shift : 0;
+      if (lane == 0) {
+        for (int tt = w0; tt < w1; ++tt) {
+          if (!mbar_wait(empty0 + 8 * stage, ph ^ 1u, kWaitLimitNs)) {
+            record_timeout(a.status, 1, issued, stage, ph ^ 1u, empty0 + 8 * stage);
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full0 + 8 * stage;
+          const uint32_t kdst = ring + stage * C::STAGE_BYTES;
+          const uint32_t vdst = kdst + C::TILE_BYTES;
+          mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+          if (!a.paged) {
+            const int row = s_start[pc.b] + tt * T;
+            if constexpr (C::TOKEN_MAJOR) {
+              tma_load_4d(kdst, &a.kmap, fb, 0, 0, pc.h, row, pol);
+              tma_load_4d(vdst, &a.vmap, fb, 0, 0, pc.h, row, pol);
+            } else {
+#pragma unroll
+              for (int p = 0; p < C::NP; ++p) {
+                const uint32_t off = p * (T * C::CB);
+                if (FA_CHECK(a.status, off + T * C::CB <= C::TILE_BYTES && (off & 127u) == 0, 301, off)) {
+                  tma_load_3d(kdst + off, &a.kmap, fb, p * (C::CB / C::ES), pc.h, row, pol);
+                  tma_load_3d(vdst + off, &a.vmap, fb, p * (C::CB / C::ES), pc.h, row, pol);
+                }
+              }
+            }
+          } else if constexpr (C::TOKEN_MAJOR) {
+            for (int jb = 0; jb < NB; ++jb) {
+              const int tok = tt * T + jb * a.box_t;
+              const int pidx = tok >> a.page_shift;
+              const int page = (pidx < npages && pidx - pbase < 64) ? s_pages[pidx - pbase] : -1;
+              const int slot0 = tok & (ps - 1);
+              const uint32_t off = jb * a.box_t * C::ROWB;
+              if (FA_CHECK(a.status, off + a.box_t * C::ROWB <= C::TILE_BYTES && (off & 127u) == 0 &&
+                                         pidx - pbase >= 0 && pidx - pbase < 64,
+                           303, off)) {
+                tma_load_5d(kdst + off, &a.kmap, fb, 0, 0, pc.h, slot0, page, pol);
+                tma_load_5d(vdst + off, &a.vmap, fb, 0, 0, pc.h, slot0, page, pol);
+              }
+            }
+          } else {
+            for (int jb = 0; jb < NB; ++jb) {
+              const int tok = tt * T + jb * a.box_t;
+              const int pidx = tok >> a.page_shift;
+              const int page = (pidx < npages && pidx - pbase < 64) ? s_pages[pidx - pbase] : -1;
+              const int slot0 = tok & (ps - 1);
+#pragma unroll
+              for (int p = 0; p < C::NP; ++p) {
+                const uint32_t off = p * (T * C::CB) + jb * a.box_t * C::CB;
+                if (FA_CHECK(a.status, off + a.box_t * C::CB <= C::TILE_BYTES && (off & 127u) == 0 &&
+                                           pidx - pbase >= 0 && pidx - pbase < 64,
+                             302, off)) {
+                  tma_load_4d(kdst + off, &a.kmap, fb, p * (C::CB / C::ES), pc.h, slot0, page, pol);
+                  tma_load_4d(vdst + off, &a.vmap, fb, p * (C::CB / C::ES), pc.h, slot0, page, pol);
+                }
+              }
+            }
+          }
+          ++issued;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      __syncwarp();
+      if (a.paged && nhave) store_ids(nv, nin);
+      __syncwarp();
+      if (w1 >= pc.t1) {
+        have = nhave;
+        pc = pn;
+        it = itn;
+        w0 = nw0;
+      } else {
+        w0 = w1;
       }
     }
     // drain: every issued copy has landed before the block may exit
@@ -1089,6 +1185,13 @@ __global__ void __maxnreg__(224)
         }
         if (!mbar_wait(full0 + 8 * st, par, kWaitLimitNs)) {
           record_timeout(a.status, 2, issued - k, st, par, full0 + 8 * st);
+          break;
+        }
+      }
+      // and the last staged query rows (each slot's latest copy)
+      for (int k = !C::STAGE_Q ? pq : (pq - 2 < 0 ? 0 : pq - 2); k < pq; ++k) {
+        if (!mbar_wait(qfull0 + 8 * (k & 1), (k >> 1) & 1, kWaitLimitNs)) {
+          record_timeout(a.status, 7, k, k & 1, (k >> 1) & 1, qfull0 + 8 * (k & 1));
           break;
         }
       }
@@ -1127,7 +1230,24 @@ __global__ void __maxnreg__(224)
     const int L = s_len[pc.b];
     const int lo = (a.window > 0 && L > a.window) ? L - a.window : 0;
     const int n = pc.t1 - pc.t0;
-    cons.begin_piece(a, pc.b, pc.h, lane);
+    if constexpr (C::STAGE_Q) {
+      const int qs = piece & 1;
+      if (alive) {
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(qfull0 + 8 * qs, (piece >> 1) & 1, kWaitLimitNs));
+        if (!ok) {
+          if (lane == 0) record_timeout(a.status, 6, piece, qs, (piece >> 1) & 1, qfull0 + 8 * qs);
+          alive = false;
+        }
+      }
+      const float ks = C::ES == 1 ? (scales_in_smem ? s_kscale[pc.h] : __ldg(a.k_scale + pc.h)) : 1.f;
+      cons.begin_piece(a, q_slots + qs * (C::QSLOT_BYTES / 2), ks, lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(qempty0 + 8 * qs);
+    } else {
+      const float ks = C::ES == 1 ? (scales_in_smem ? s_kscale[pc.h] : __ldg(a.k_scale + pc.h)) : 1.f;
+      cons.begin_piece(a, a.q + (static_cast<size_t>(pc.b) * a.qo_heads + static_cast<size_t>(pc.h) * G) * D,
+                       ks, lane);
+    }
     for (; next < base_i + n; next += NW) {
       if (alive) {
         const bool ok = __all_sync(0xffffffffu, mbar_wait(full0 + 8 * stage, ph, kWaitLimitNs));
@@ -1154,7 +1274,7 @@ __global__ void __maxnreg__(224)
     // of the next piece; the last warp to park merges the NW states, writes
     // the result (or the partial) and frees the area.  A warp waits only if
     // it finishes its share of the next piece before that merge is done.
-    const float vs = Cons::C::ES == 1 ? __ldg(a.v_scale + pc.h) : 1.f;
+    const float vs = C::ES == 1 ? (scales_in_smem ? s_vscale[pc.h] : __ldg(a.v_scale + pc.h)) : 1.f;
     if (piece > 0 && alive) {
       const bool ok = __all_sync(0xffffffffu, mbar_wait(mfree, (piece - 1) & 1, kWaitLimitNs));
       if (!ok) {
