@@ -2,8 +2,9 @@
 """Decode-attention benchmark (one JSON line on rank 0).
 
 A step is one whole decode pass over one batch: plan (host split of the KV
-tiles over thread blocks) + the fused split-KV kernel (TMA tile loads,
-scores, online softmax, partial states, in-kernel log-sum-exp merge).
+tiles over thread blocks) + the split-KV kernel (TMA tile loads, scores,
+online softmax, partial states) + the split-segment merge kernel (exact
+log-sum-exp merge, launched as a programmatic dependent of the first).
 Default workload: batched paged decode, batch 64, 32 query / 8 kv heads,
 head_dim 128, per-request kv_len uniform in [512, 16384] (seed 4), 16-token
 pages in a random permutation of the pool, bf16 K/V ~ N(0,1).  Its K/V
@@ -272,6 +273,28 @@ def e2e_measure(x, runner, steps):
     return ms, h2d, d2h
 
 
+# ------------------------------------------------------------ multi-rank
+def max_over_ranks(value, world, device):
+    """The largest of one float per rank (every rank gets it); the identity on
+    one rank.  Every rank must call it at the same point."""
+    if world == 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(kv_bytes, batch, ms_total, steps, world):
+    """Whole-job figures for `steps` steps that took ms_total (the slowest
+    rank's device time) with every rank decoding its own batch."""
+    ms_step = ms_total / steps
+    return {"ms_per_step": ms_step,
+            "value": world * kv_bytes / (ms_step * 1e-3) / 1e9,
+            "tokens_per_s": world * batch / (ms_step * 1e-3)}
+
+
 # --------------------------------------------------------------- CPU side
 def oracle_sample(x, budget_s, max_requests=None):
     """Time the fp64 oracle on whole requests of x (all their heads) for about
@@ -405,19 +428,15 @@ def main():
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    t = torch.tensor([ms_total], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total = float(t.item())
-    ms_step = ms_total / args.steps
+    ms_total = max_over_ranks(ms_total, world, "cuda")
     kv_bytes = x.kv_bytes()
-    value = world * kv_bytes / (ms_step * 1e-3) / 1e9
-    tokens = world * x.batch / (ms_step * 1e-3)
+    agg = aggregate(kv_bytes, x.batch, ms_total, args.steps, world)
+    ms_step, value, tokens = agg["ms_per_step"], agg["value"], agg["tokens_per_s"]
 
     # dominant kernel: per-launch device time on the launching stream
     launch_ms = per_launch_ms(runner.step, min(args.steps, 100), stream,
                               flush=None if kv_bytes > 256e6 else l2_flusher())
-    mean_launch = statistics.mean(launch_ms)
+    mean_launch = max_over_ranks(statistics.mean(launch_ms), world, "cuda")
     peak, peak_kind = hbm_peak()
     achieved = kv_bytes / (mean_launch * 1e-3) / 1e9
     traffic = ncu_traffic(x.name)
@@ -426,6 +445,7 @@ def main():
     e2e = None
     if not args.no_e2e:
         ms_e2e, h2d, d2h = e2e_measure(x, runner, args.e2e_steps)
+        ms_e2e = max_over_ranks(ms_e2e, world, "cuda")
         e2e = {"value": round(world * kv_bytes / (ms_e2e * 1e-3) / 1e9, 3), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(ms_e2e, 3), "steps": args.e2e_steps,

@@ -134,6 +134,28 @@ def test_bad_page_id_is_flagged_not_read():
     assert_matches(out[:1], lse[:1], ref_out, ref_lse, what="unaffected request")
 
 
+def test_status_word_is_reported_and_cleared():
+    """fa_decode_status returns the check bits found in the workspace header
+    and clears them, and a pass into that workspace still computes the right
+    result.  The bits (a timeout and its record) are written by the test:
+    no fault or timeout is provoked on the device."""
+    import torch
+    x = synth.generate(1, 8, 2, 128, [300], seed=27)
+    dev = DeviceInputs(x)
+    p = dev.plan(num_ctas=4)
+    ws = p.new_workspace()
+    hdr = ws[:64].view(torch.int32)
+    hdr[0] = 2       # FA_DEVICE_TIMEOUT
+    hdr[8] = 3       # timeout site: a consumer's wait on a full stage
+    assert binding.decode_status(ws) == 2
+    assert binding.decode_status(ws) == 0   # cleared by the first read
+    out, lse = dev.run(p, workspace=ws)
+    o, l = to_numpy(out, lse)
+    ref_out, ref_lse = oracle.decode_all(x)
+    assert_matches(o, l, ref_out, ref_lse, what="after a reported status")
+    assert binding.decode_status(ws) == 0
+
+
 def test_lse_optional_and_workspace_reuse():
     x = synth.generate(2, 8, 2, 128, [700, 900], seed=26)
     dev = DeviceInputs(x)
