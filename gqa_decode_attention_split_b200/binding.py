@@ -48,7 +48,8 @@ class PlanInfo(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int32), ("num_ctas", ctypes.c_int32),
                 ("tile_tokens", ctypes.c_int32), ("stages", ctypes.c_int32),
                 ("total_tiles", ctypes.c_int32), ("max_partials", ctypes.c_int32),
-                ("workspace_bytes", ctypes.c_size_t), ("smem_bytes", ctypes.c_size_t)]
+                ("workspace_bytes", ctypes.c_size_t), ("smem_bytes", ctypes.c_size_t),
+                ("v_stages", ctypes.c_int32)]
 
 
 _lib = None

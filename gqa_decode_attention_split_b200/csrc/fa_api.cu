@@ -227,6 +227,7 @@ extern "C" fa_status fa_plan_get_info(const fa_plan* plan, fa_plan_info_t* info)
   info->num_ctas = plan->num_ctas;
   info->tile_tokens = plan->kernel->tile_tokens;
   info->stages = plan->kernel->stages;
+  info->v_stages = plan->kernel->v_stages;
   info->total_tiles = static_cast<int32_t>(plan->total_tiles > INT32_MAX ? INT32_MAX : plan->total_tiles);
   info->max_partials = static_cast<int32_t>(plan->max_partials);
   info->workspace_bytes = plan->ws_bytes;

@@ -43,7 +43,8 @@ KernelEntry make_entry(int path, int group, int max_group, int fp8) {
   e.fp8 = fp8;
   e.path = path;
   e.tile_tokens = C::T;
-  e.stages = C::STAGES;
+  e.stages = C::KSTAGES;
+  e.v_stages = C::VSTAGES;
   e.threads = C::THREADS;
   e.row_bytes = C::ROWB;
   e.plane_bytes = C::CB;

@@ -114,14 +114,19 @@ constexpr int kScaleCap = 128;         // fp8 per-kv-head scales kept in shared 
 // the plane as a dimension; the 16-byte chunks of 128-byte line l of the tile
 // are XOR-swizzled by (l & 7) (TMA 128B swizzle).  With FA_PLANE_COPIES the
 // layout is plane-major, [NP][T][CB], one copy per plane.
-// A tile holds TILE_BYTES_TARGET / row bytes tokens (16 to 128).  The ring takes what is left of the block's
-// shared memory after the merge area for GMAX query heads, in a multiple of
-// the consumer-warp count: tile i uses stage i % STAGES and warp i % NW, so
-// every stage belongs to exactly one warp, which waits on it round after
-// round.  (A stage shared by two warps would let one warp wait for round r+1
-// while round r is still pending; an mbarrier parity wait cannot tell the two
-// apart and would pass early.)
-template <int D, bool FP8, int GMAX, int TILE_BYTES_TARGET, int NWARPS>
+// A tile holds TILE_BYTES_TARGET / row bytes tokens (16 to 128).  K and V
+// tiles live in two rings that take what is left of the block's shared
+// memory after the merge area for GMAX query heads: KSTAGES K slots and
+// VSTAGES V slots, each a multiple of the consumer-warp count.  Tile i uses K
+// slot i % KSTAGES, V slot i % VSTAGES and warp i % NW, so every slot belongs
+// to exactly one warp, which waits on it round after round.  (A slot shared
+// by two warps would let one warp wait for round r+1 while round r is still
+// pending; an mbarrier parity wait cannot tell the two apart and would pass
+// early.)  A consumer that frees its K slot as soon as the scores are taken
+// (EARLY_K) holds V longer than K, so the V ring gets the extra slots: a
+// slot is refilled only after its warp releases it, and a slot held through
+// the tile's math is a slot with no copy in flight.
+template <int D, bool FP8, int GMAX, int TILE_BYTES_TARGET, int NWARPS, bool EARLY_K>
 struct TileCfg {
   static constexpr int ES = FP8 ? 1 : 2;
   static constexpr int ROWB = D * ES;
@@ -130,7 +135,6 @@ struct TileCfg {
   static constexpr int T_RAW = TILE_BYTES_TARGET / ROWB;
   static constexpr int T = T_RAW < 16 ? 16 : (T_RAW > 128 ? 128 : T_RAW);
   static constexpr int TILE_BYTES = T * ROWB;
-  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   static constexpr int NW = NWARPS;
   static constexpr int MERGE_BYTES = NW * GMAX * (D + 2) * 4;
   // q area: four mbarriers, then (STAGE_Q) two slots of a piece's GMAX query
@@ -139,19 +143,24 @@ struct TileCfg {
   // consumers read them from global memory.
   static constexpr int QSLOT_BYTES = GMAX * D * 2;
   static constexpr int SCALE_BYTES = FP8 ? 2 * kScaleCap * 4 : 0;
-  static constexpr int BASE_BUDGET = kSmemPerBlock - 1024 - kSchedReserve - 512 - MERGE_BYTES - 32 - SCALE_BYTES;
-  static constexpr int stages_per_warp(int budget) {
-    return budget / STAGE_BYTES / NW > FA_MAX_STAGES_PER_WARP ? FA_MAX_STAGES_PER_WARP
-                                                               : budget / STAGE_BYTES / NW;
+  // (1024: base alignment; 272: merge counter, merge mbarrier, 64 page ids)
+  static constexpr int BASE_BUDGET = kSmemPerBlock - 1024 - kSchedReserve - 272 - MERGE_BYTES - 32 - SCALE_BYTES;
+  // K + V tiles per consumer warp that fit (a tile slot costs its bytes
+  // plus two 8-byte mbarriers)
+  static constexpr int tiles_per_warp(int budget) {
+    return budget / (TILE_BYTES + 16) / NW > 2 * FA_MAX_STAGES_PER_WARP ? 2 * FA_MAX_STAGES_PER_WARP
+                                                                       : budget / (TILE_BYTES + 16) / NW;
   }
-  static constexpr bool STAGE_Q = stages_per_warp(BASE_BUDGET - 2 * QSLOT_BYTES) == stages_per_warp(BASE_BUDGET);
+  static constexpr bool STAGE_Q = tiles_per_warp(BASE_BUDGET - 2 * QSLOT_BYTES) == tiles_per_warp(BASE_BUDGET);
   static constexpr int QAREA_BYTES = 32 + (STAGE_Q ? 2 * QSLOT_BYTES : 0) + SCALE_BYTES;
   static constexpr int RING_BUDGET = BASE_BUDGET + 32 + SCALE_BYTES - QAREA_BYTES;
-  static constexpr int STAGES_PER_WARP = stages_per_warp(RING_BUDGET);
-  static constexpr int STAGES = NW * STAGES_PER_WARP;
-  static_assert(STAGES_PER_WARP >= 1, "every consumer warp needs a stage");
-  static_assert(STAGES % NW == 0, "a stage must belong to one consumer warp");
-  static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
+  static constexpr int TPW = tiles_per_warp(RING_BUDGET);
+  static constexpr int KPW = EARLY_K ? (TPW / 3 > 1 ? TPW / 3 : 1) : TPW / 2;
+  static constexpr int VPW = TPW - KPW;
+  static_assert(KPW >= 1 && VPW >= 1, "every consumer warp needs a K and a V slot");
+  static constexpr int KSTAGES = NW * KPW;
+  static constexpr int VSTAGES = NW * VPW;
+  static constexpr int RING_BYTES = (KSTAGES + VSTAGES) * TILE_BYTES;
   static constexpr int THREADS = (NW + 1) * 32;
   static constexpr bool TOKEN_MAJOR = FA_PLANE_COPIES == 0;
   static_assert(ROWB % 16 == 0, "rows must be whole 16-byte chunks");
@@ -296,7 +305,7 @@ __device__ __forceinline__ bool next_piece(PieceIter& it, Piece& pc, const int* 
 // running softmax state, merged across slots at the end of a segment piece.
 template <int D, int G, bool FP8>
 struct SimtConsumer {
-  using C = TileCfg<D, FP8, G, FA_SIMT_TILE_BYTES, FA_SIMT_CONSUMER_WARPS>;
+  using C = TileCfg<D, FP8, G, FA_SIMT_TILE_BYTES, FA_SIMT_CONSUMER_WARPS, false>;
   static constexpr int EPC = 16 / C::ES;
   static constexpr int NCH = C::ROWB / 16;
   static constexpr int E_TARGET = 64 / G;
@@ -384,8 +393,11 @@ struct SimtConsumer {
   static constexpr int NSUB = TPS / TPSC;
   static_assert(TPS % TPSC == 0, "sub-steps");
 
+  // K and V rows are read together sub-step by sub-step, so K is released
+  // at the end (release_k as for the MMA dataflow).
+  template <class ReleaseK>
   __device__ __forceinline__ void tile(const KernelArgs& a, uint32_t kt, uint32_t vt, int pos0,
-                                       int lo, int hi, int lane) {
+                                       int lo, int hi, int lane, ReleaseK&& release_k) {
 #pragma unroll 1
     for (int si = 0; si < NSUB; ++si) {
       float s[TPSC][G];
@@ -460,6 +472,7 @@ struct SimtConsumer {
         }
       }
     }
+    release_k();
   }
 
   // Merge the slots' states and publish the warp's state.
@@ -510,7 +523,7 @@ struct SimtConsumer {
 template <int D, bool FP8>
 struct MmaConsumer {
   using C = TileCfg<D, FP8, 8, FP8 ? FA_FP8_MMA_TILE_BYTES : FA_MMA_TILE_BYTES,
-                    FP8 ? FA_FP8_MMA_CONSUMER_WARPS : FA_MMA_CONSUMER_WARPS>;
+                    FP8 ? FA_FP8_MMA_CONSUMER_WARPS : FA_MMA_CONSUMER_WARPS, true>;
   static constexpr int KS = D / 16;     // k-steps of the score product = m-tiles of O^T
   static constexpr int SUB = C::T / 16;  // 16-token subtiles per tile
   static constexpr int BPT = D / 4;      // fp8 K: bytes of a row owned by one lane
@@ -687,11 +700,14 @@ struct MmaConsumer {
 
   // One tile: the scores of all SUB subtiles first (independent mma chains),
   // one softmax update for the whole tile, then O^T += V^T P^T per subtile.
+  // release_k() is called as soon as the K tile is no longer read.
+  template <class ReleaseK>
   __device__ __forceinline__ void tile(const KernelArgs& a, uint32_t kt, uint32_t vt, int pos0,
-                                       int lo, int hi, int lane) {
+                                       int lo, int hi, int lane, ReleaseK&& release_k) {
     float sc[SUB][4];
 #pragma unroll
     for (int sub = 0; sub < SUB; ++sub) scores(a, kt, sub, lane, sc[sub]);
+    release_k();
     float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F;
 #pragma unroll
     for (int sub = 0; sub < SUB; ++sub) {
@@ -861,7 +877,8 @@ struct MmaConsumer {
 
 // ------------------------------------------------------------- kernel
 // Block shared memory, from a 1024-aligned base:
-//   ring [STAGES][K tile, V tile] | full[STAGES], empty[STAGES] mbarriers |
+//   K ring [KSTAGES][tile] | V ring [VSTAGES][tile] |
+//   fullK[KSTAGES], emptyK[KSTAGES], fullV[VSTAGES], emptyV[VSTAGES] mbarriers |
 //   m[NW][G], l[NW][G] | acc[NW][G][D] | merge counter, merge mbarrier |
 //   pages[64] | q mbarriers, q slots, scales | start[B], len[B], pre[B+1]
 template <class Cons>
@@ -869,7 +886,7 @@ struct SmemLayout {
   using C = typename Cons::C;
   static constexpr int D = C::ROWB / C::ES;
   static constexpr int kBars = C::RING_BYTES;
-  static constexpr int kMerge = kBars + 2 * C::STAGES * 8;
+  static constexpr int kMerge = kBars + 2 * (C::KSTAGES + C::VSTAGES) * 8;
   __host__ __device__ static constexpr int acc_off(int G) {
     return kMerge + ((C::NW * G * 2 * 4 + 15) / 16) * 16;
   }
@@ -899,7 +916,16 @@ __global__ void __maxnreg__(224)
   uint8_t* base = smem_raw + (sbase - raw);
   const uint32_t ring = sbase;
   const uint32_t full0 = sbase + S::kBars;
-  const uint32_t empty0 = full0 + C::STAGES * 8;
+  const uint32_t empty0 = full0 + C::KSTAGES * 8;    // K slots: full0[s], empty0[s]
+  const uint32_t vfull0 = empty0 + C::KSTAGES * 8;   // V slots: vfull0[s], vempty0[s]
+  const uint32_t vempty0 = vfull0 + C::VSTAGES * 8;
+  const uint32_t vring = ring + C::KSTAGES * C::TILE_BYTES;
+  // Separate K and V barriers only where the rings differ in depth.  With
+  // equal depths a tile's K and V copies complete on its K slot's barriers
+  // and are released together: a second wait and a second release per tile
+  // measured slower in the paged producer loop (one copy per page, so the
+  // loop's length bounds how fast copies go out), for no gain.
+  constexpr bool kSplitKV = C::KSTAGES != C::VSTAGES;
   const int G = a.group;
   float* m_area = reinterpret_cast<float*>(base + S::kMerge);
   float* l_area = m_area + NW * G;
@@ -945,9 +971,13 @@ __global__ void __maxnreg__(224)
     }
   }
   if (tid == 32) {
-    for (int s = 0; s < C::STAGES; ++s) {
+    for (int s = 0; s < C::KSTAGES; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int s = 0; s < C::VSTAGES; ++s) {
+      mbar_init(vfull0 + 8 * s, 1);
+      mbar_init(vempty0 + 8 * s, 1);
     }
     mbar_init(mfree, 1);
     *s_mcnt = 0;
@@ -1018,9 +1048,9 @@ __global__ void __maxnreg__(224)
     // tiles per window of 64 page ids (a window that starts inside a page may
     // touch one page more than its token count suggests)
     const int win_paged = !a.paged ? 1 : (ps >= T ? 63 * (ps / T) : (64 * ps) / T);
-    int stage = 0;
-    uint32_t ph = 0;             // lane 0's ring position (stage, wrap parity)
-    int issued = 0;
+    int ks = 0, vs = 0;          // lane 0's ring positions (K slot, V slot)
+    uint32_t kph = 0, vph = 0;   // and their wrap parities
+    int issued = 0;              // tiles whose K and V copies were issued
     int pq = 0;                  // pieces whose query rows were staged
     bool ok = true;
     // this lane's two page ids of the window starting at tile w of piece p
@@ -1097,27 +1127,42 @@ __global__ void __maxnreg__(224)
       const int pbase = a.paged ? (w0 * T) >> a.page_shift : 0;
       if (lane == 0) {
         for (int tt = w0; tt < w1; ++tt) {
-          if (!mbar_wait(empty0 + 8 * stage, ph ^ 1u, kWaitLimitNs)) {
-            record_timeout(a.status, 1, issued, stage, ph ^ 1u, empty0 + 8 * stage);
+          // both slots first, then the K and V copies of each box back to back
+          // (one pass over the boxes keeps lane 0's issue loop as short as a
+          // single ring's: paged tiles take one copy per page and the loop's
+          // length bounds how fast copies go out).  V is waited for first: a
+          // warp frees its V slot after its K slot, so the K wait then passes
+          // without a second suspension.
+          if (kSplitKV && !mbar_wait(vempty0 + 8 * vs, vph ^ 1u, kWaitLimitNs)) {
+            record_timeout(a.status, 8, issued, vs, vph ^ 1u, vempty0 + 8 * vs);
             ok = false;
             break;
           }
-          const uint32_t fb = full0 + 8 * stage;
-          const uint32_t kdst = ring + stage * C::STAGE_BYTES;
-          const uint32_t vdst = kdst + C::TILE_BYTES;
-          mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+          if (!mbar_wait(empty0 + 8 * ks, kph ^ 1u, kWaitLimitNs)) {
+            record_timeout(a.status, 1, issued, ks, kph ^ 1u, empty0 + 8 * ks);
+            ok = false;
+            break;
+          }
+          const uint32_t kfb = full0 + 8 * ks, vfb = kSplitKV ? vfull0 + 8 * vs : kfb;
+          const uint32_t kdst = ring + ks * C::TILE_BYTES, vdst = vring + vs * C::TILE_BYTES;
+          if constexpr (kSplitKV) {
+            mbar_arrive_expect_tx(kfb, C::TILE_BYTES);
+            mbar_arrive_expect_tx(vfb, C::TILE_BYTES);
+          } else {
+            mbar_arrive_expect_tx(kfb, 2 * C::TILE_BYTES);
+          }
           if (!a.paged) {
             const int row = s_start[pc.b] + tt * T;
             if constexpr (C::TOKEN_MAJOR) {
-              tma_load_4d(kdst, &a.kmap, fb, 0, 0, pc.h, row, pol);
-              tma_load_4d(vdst, &a.vmap, fb, 0, 0, pc.h, row, pol);
+              tma_load_4d(kdst, &a.kmap, kfb, 0, 0, pc.h, row, pol);
+              tma_load_4d(vdst, &a.vmap, vfb, 0, 0, pc.h, row, pol);
             } else {
 #pragma unroll
               for (int p = 0; p < C::NP; ++p) {
                 const uint32_t off = p * (T * C::CB);
                 if (FA_CHECK(a.status, off + T * C::CB <= C::TILE_BYTES && (off & 127u) == 0, 301, off)) {
-                  tma_load_3d(kdst + off, &a.kmap, fb, p * (C::CB / C::ES), pc.h, row, pol);
-                  tma_load_3d(vdst + off, &a.vmap, fb, p * (C::CB / C::ES), pc.h, row, pol);
+                  tma_load_3d(kdst + off, &a.kmap, kfb, p * (C::CB / C::ES), pc.h, row, pol);
+                  tma_load_3d(vdst + off, &a.vmap, vfb, p * (C::CB / C::ES), pc.h, row, pol);
                 }
               }
             }
@@ -1131,8 +1176,8 @@ __global__ void __maxnreg__(224)
               if (FA_CHECK(a.status, off + a.box_t * C::ROWB <= C::TILE_BYTES && (off & 127u) == 0 &&
                                          pidx - pbase >= 0 && pidx - pbase < 64,
                            303, off)) {
-                tma_load_5d(kdst + off, &a.kmap, fb, 0, 0, pc.h, slot0, page, pol);
-                tma_load_5d(vdst + off, &a.vmap, fb, 0, 0, pc.h, slot0, page, pol);
+                tma_load_5d(kdst + off, &a.kmap, kfb, 0, 0, pc.h, slot0, page, pol);
+                tma_load_5d(vdst + off, &a.vmap, vfb, 0, 0, pc.h, slot0, page, pol);
               }
             }
           } else {
@@ -1147,16 +1192,20 @@ __global__ void __maxnreg__(224)
                 if (FA_CHECK(a.status, off + a.box_t * C::CB <= C::TILE_BYTES && (off & 127u) == 0 &&
                                            pidx - pbase >= 0 && pidx - pbase < 64,
                              302, off)) {
-                  tma_load_4d(kdst + off, &a.kmap, fb, p * (C::CB / C::ES), pc.h, slot0, page, pol);
-                  tma_load_4d(vdst + off, &a.vmap, fb, p * (C::CB / C::ES), pc.h, slot0, page, pol);
+                  tma_load_4d(kdst + off, &a.kmap, kfb, p * (C::CB / C::ES), pc.h, slot0, page, pol);
+                  tma_load_4d(vdst + off, &a.vmap, vfb, p * (C::CB / C::ES), pc.h, slot0, page, pol);
                 }
               }
             }
           }
           ++issued;
-          if (++stage == C::STAGES) {
-            stage = 0;
-            ph ^= 1u;
+          if (++ks == C::KSTAGES) {
+            ks = 0;
+            kph ^= 1u;
+          }
+          if (++vs == C::VSTAGES) {
+            vs = 0;
+            vph ^= 1u;
           }
         }
       }
@@ -1175,16 +1224,19 @@ __global__ void __maxnreg__(224)
     }
     // drain: every issued copy has landed before the block may exit
     if (lane == 0) {
-      const int n = issued < C::STAGES ? issued : C::STAGES;
-      for (int k = 1; k <= n; ++k) {
-        int st = stage - k;
-        uint32_t par = ph;
-        if (st < 0) {
-          st += C::STAGES;
-          par ^= 1u;
-        }
+      for (int j = issued - C::KSTAGES < 0 ? 0 : issued - C::KSTAGES; j < issued; ++j) {
+        const int st = j % C::KSTAGES;
+        const uint32_t par = (j / C::KSTAGES) & 1;
         if (!mbar_wait(full0 + 8 * st, par, kWaitLimitNs)) {
-          record_timeout(a.status, 2, issued - k, st, par, full0 + 8 * st);
+          record_timeout(a.status, 2, j, st, par, full0 + 8 * st);
+          break;
+        }
+      }
+      for (int j = !kSplitKV ? issued : (issued - C::VSTAGES < 0 ? 0 : issued - C::VSTAGES); j < issued; ++j) {
+        const int st = j % C::VSTAGES;
+        const uint32_t par = (j / C::VSTAGES) & 1;
+        if (!mbar_wait(vfull0 + 8 * st, par, kWaitLimitNs)) {
+          record_timeout(a.status, 9, j, st, par, vfull0 + 8 * st);
           break;
         }
       }
@@ -1214,14 +1266,16 @@ __global__ void __maxnreg__(224)
     }
   }
 
-  // Tile i of the block's sequence lives in stage i % STAGES and is consumed
-  // by warp i % NW (STAGES is a multiple of NW, so each stage has one owner
-  // warp that waits on it in order); each warp tracks its next tile and that
-  // tile's stage.
+  // Tile i of the block's sequence lives in K slot i % KSTAGES and V slot
+  // i % VSTAGES and is consumed by warp i % NW (both slot counts are
+  // multiples of NW, so each slot has one owner warp that waits on it in
+  // order); each warp tracks its next tile and that tile's slots.
   Cons cons;
   int next = w;          // next tile index (block sequence) of this warp
-  int stage = w;         // its stage (STAGES >= NW)
-  uint32_t ph = 0;       // wrap parity of that stage
+  int kslot = w;         // its K slot (KSTAGES >= NW)
+  int vslot = w;         // its V slot (VSTAGES >= NW)
+  uint32_t kph = 0;      // wrap parities of those slots
+  uint32_t vph = 0;
   int base_i = 0;        // block-sequence index of the current piece's first tile
   bool alive = true;
   int piece = 0;         // pieces this block has finished (merge-area uses)
@@ -1249,23 +1303,44 @@ __global__ void __maxnreg__(224)
                        ks, lane);
     }
     for (; next < base_i + n; next += NW) {
-      if (alive) {
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(full0 + 8 * stage, ph, kWaitLimitNs));
+      // both halves of the tile are waited for up front (a second wait in
+      // the middle of the tile's math measured slower than it saves); V
+      // first, as its last copy is issued after K's
+      if (kSplitKV && alive) {
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(vfull0 + 8 * vslot, vph, kWaitLimitNs));
         if (!ok) {
-          if (lane == 0) record_timeout(a.status, 3, next, stage, ph, full0 + 8 * stage);
+          if (lane == 0) record_timeout(a.status, 10, next, vslot, vph, vfull0 + 8 * vslot);
           alive = false;
         }
       }
       if (alive) {
-        const uint32_t kt = ring + stage * C::STAGE_BYTES;
-        cons.tile(a, kt, kt + C::TILE_BYTES, (pc.t0 + next - base_i) * T, lo, L, lane);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty0 + 8 * stage);
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(full0 + 8 * kslot, kph, kWaitLimitNs));
+        if (!ok) {
+          if (lane == 0) record_timeout(a.status, 3, next, kslot, kph, full0 + 8 * kslot);
+          alive = false;
+        }
       }
-      stage += NW;
-      if (stage >= C::STAGES) {
-        stage -= C::STAGES;
-        ph ^= 1u;
+      if (alive) {
+        const uint32_t kempty = empty0 + 8 * kslot;
+        cons.tile(a, ring + kslot * C::TILE_BYTES, vring + vslot * C::TILE_BYTES,
+                  (pc.t0 + next - base_i) * T, lo, L, lane, [&] {
+                    if constexpr (kSplitKV) {  // K slot free: the scores are taken
+                      __syncwarp();
+                      if (lane == 0) mbar_arrive(kempty);
+                    }
+                  });
+        __syncwarp();
+        if (lane == 0) mbar_arrive(kSplitKV ? vempty0 + 8 * vslot : kempty);
+      }
+      kslot += NW;
+      if (kslot >= C::KSTAGES) {
+        kslot -= C::KSTAGES;
+        kph ^= 1u;
+      }
+      vslot += NW;
+      if (vslot >= C::VSTAGES) {
+        vslot -= C::VSTAGES;
+        vph ^= 1u;
       }
     }
     base_i += n;

@@ -18,7 +18,8 @@ struct KernelEntry {
   int fp8;
   int path;
   int tile_tokens;  // T
-  int stages;
+  int stages;       // K tile slots
+  int v_stages;     // V tile slots
   int threads;
   int row_bytes;    // head_dim * element size
   int plane_bytes;  // min(128, row_bytes)

@@ -103,11 +103,12 @@ typedef struct {
   int32_t path;             /* FA_PATH_SIMT or FA_PATH_MMA                    */
   int32_t num_ctas;         /* thread blocks launched by fa_decode_run        */
   int32_t tile_tokens;      /* tokens per KV tile moved by one TMA transaction */
-  int32_t stages;           /* depth of the shared-memory tile ring           */
+  int32_t stages;           /* K tile slots of the shared-memory ring         */
   int32_t total_tiles;      /* KV tiles over all (request, kv head) segments  */
   int32_t max_partials;     /* partial-state slots reserved in the workspace  */
   size_t workspace_bytes;   /* minimum workspace size for fa_decode_run       */
   size_t smem_bytes;        /* dynamic shared memory per thread block         */
+  int32_t v_stages;         /* V tile slots (at least stages: V is held longer) */
 } fa_plan_info_t;
 
 /*
