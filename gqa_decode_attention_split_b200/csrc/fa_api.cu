@@ -162,8 +162,12 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
 
   const int T = k->tile_tokens;
   int64_t tiles = 0;
-  for (int b = 0; b < desc->batch; ++b)
-    tiles += host_num_tiles(kv_indptr_host[b + 1] - kv_indptr_host[b], desc->window, T);
+  int64_t seg_tiles = -1;  // tiles of every segment when all are equal, else -1
+  for (int b = 0; b < desc->batch; ++b) {
+    const int64_t n = host_num_tiles(kv_indptr_host[b + 1] - kv_indptr_host[b], desc->window, T);
+    tiles += n;
+    seg_tiles = b == 0 ? n : (seg_tiles == n ? n : -1);
+  }
   tiles *= desc->kv_heads;
 
   int64_t P;
@@ -182,6 +186,25 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
     if (want > seg_cap) want = seg_cap;
     P = want < num_sms ? want : num_sms;
     if (P < 1) P = 1;
+    // Segments of equal length and rows of at most 128 bytes: prefer a grid
+    // that gives every segment the same whole number of blocks, each run
+    // starting on a segment boundary, even at the cost of up to a fifth of
+    // the SMs.  The blocks that read the kv heads of the same tokens then
+    // advance in step, so a DRAM row holding one token's heads is read while
+    // it is open, instead of once per head at different times.  Measured on
+    // fp8 head_dim 128: 7-12% faster than using every SM; with 256-byte rows
+    // it made no difference.
+    const int64_t segs = static_cast<int64_t>(desc->batch) * desc->kv_heads;
+    if (seg_tiles > 0 && k->row_bytes <= 128 && P == num_sms && segs <= num_sms) {
+      const int64_t kmax = num_sms / segs;
+      const int64_t kmin = (4 * static_cast<int64_t>(num_sms) + 5 * segs - 1) / (5 * segs);
+      for (int64_t kk = kmax; kk >= (kmin > 1 ? kmin : 1); --kk) {
+        if (seg_tiles % kk == 0) {
+          P = kk * segs;
+          break;
+        }
+      }
+    }
   }
   if (P > (1 << 20)) return FA_ERR_UNSUPPORTED;
 
