@@ -100,6 +100,7 @@ struct KernelArgs {
   int batch, qo_heads, kv_heads, group;
   int window;
   int paged, page_shift, pt_stride, box_t, swz;
+  int seg_parts;      // 0: equal runs of all tiles; k > 0: k runs per segment
   float score_scale;  // sm_scale * log2(e)
 };
 
@@ -251,8 +252,12 @@ struct Piece {
   long long seg_start;
 };
 
+// The block's run is tiles [u, u1) of the segments laid end to end.  Either
+// all runs have `per` tiles (parts == 0), or every segment is cut into
+// `parts` runs, block c taking run c % parts of segment c / parts.
 struct PieceIter {
   long long u, u1, per;
+  int parts;
 };
 
 __device__ __forceinline__ int first_tile(int L, int window, int T) {
@@ -291,8 +296,13 @@ __device__ __forceinline__ bool next_piece(PieceIter& it, Piece& pc, const int* 
   pc.seg = b * H + h;
   pc.seg_start = base + static_cast<long long>(h) * n;
   const long long seg_end = pc.seg_start + n;
-  pc.c_first = static_cast<int>(pc.seg_start / it.per);
-  pc.n_pieces = static_cast<int>((seg_end - 1) / it.per) - pc.c_first + 1;
+  if (it.parts > 0) {
+    pc.c_first = pc.seg * it.parts;
+    pc.n_pieces = it.parts;
+  } else {
+    pc.c_first = static_cast<int>(pc.seg_start / it.per);
+    pc.n_pieces = static_cast<int>((seg_end - 1) / it.per) - pc.c_first + 1;
+  }
   it.u += len;
   return true;
 }
@@ -1010,8 +1020,24 @@ __global__ void __maxnreg__(224)
   const int P = gridDim.x, c = blockIdx.x;
   PieceIter it;
   it.per = N > 0 ? (N + P - 1) / P : 1;
+  it.parts = 0;
   it.u = static_cast<long long>(c) * it.per;
   it.u1 = it.u + it.per < N ? it.u + it.per : N;
+  if (a.seg_parts > 0) {
+    // run c % k of segment c / k (runs differ by at most one tile; the
+    // planner gives every run at least one tile)
+    const int k = a.seg_parts;
+    const int seg = c / k, part = c - seg * k;
+    it.parts = k;
+    it.u = it.u1 = 0;
+    if (seg < B * H) {
+      const int b = seg / H, h = seg - b * H;
+      const long long n = s_pre[b + 1] - s_pre[b];
+      const long long base = static_cast<long long>(H) * s_pre[b] + static_cast<long long>(h) * n;
+      it.u = base + part * n / k;
+      it.u1 = base + (part + 1) * n / k;
+    }
+  }
 
   // The merge kernel may be scheduled now (it waits for this grid to finish
   // before it reads anything this grid writes).
@@ -1255,6 +1281,17 @@ __global__ void __maxnreg__(224)
   const int w = warp - 1;
   const int ctid = tid - 32;
   constexpr int NCT = NW * 32;
+
+  // a run of a split segment that holds no tile (only if the device indptr
+  // is not the plan's): an empty partial state, so the merge gives it no
+  // weight
+  if (it.parts > 1 && it.u >= it.u1 && c / it.parts < B * H) {
+    const size_t slot = static_cast<size_t>(c) + c / it.parts;
+    for (int x = ctid; x < G * D; x += NCT) {
+      a.part_o[slot * G * D + x] = 0.f;
+      if (x < G) a.part_lse[slot * G + x] = -CUDART_INF_F;
+    }
+  }
 
   // requests without keys: out = 0, lse = -inf (spread over blocks)
   for (int b = c; b < B; b += P) {

@@ -102,6 +102,13 @@ def test_plan_paged_and_fp8(lib):
     lib.fa_plan_destroy(h)
     st, h, ws = _plan(lib, _desc(qo_heads=64, kv_heads=8, kv_dtype=1), [0, 131072])
     assert st == 0 and _info(lib, h).path == binding.PATH_MMA
+    # 8 equal segments of 128-byte rows: 18 whole runs per segment, so no run
+    # crosses a segment boundary (144 of the 148 SMs)
+    assert _info(lib, h).num_ctas == 144
+    lib.fa_plan_destroy(h)
+    # the same shape in bf16 (256-byte rows) keeps equal runs over every SM
+    st, h, ws = _plan(lib, _desc(qo_heads=64, kv_heads=8), [0, 131072])
+    assert st == 0 and _info(lib, h).num_ctas == B200_SMS
     lib.fa_plan_destroy(h)
 
 

@@ -96,6 +96,16 @@ def test_forced_splits_agree(path):
         assert np.abs(o - results[0][0]).max() <= 4e-3
 
 
+@pytest.mark.parametrize("window", [-1, 1500])
+def test_segment_aligned_split(window):
+    """Equal segments of 128-byte rows are cut into whole runs per segment
+    (here 41 tiles into 18 runs of 2 or 3 tiles, with a ragged last tile)."""
+    x = synth.generate(1, 64, 8, 128, [2597], kv_dtype="fp8_e4m3", window=window, seed=28)
+    out, lse, info = _check(x, path="mma")
+    if window < 0:
+        assert info["num_ctas"] == 8 * 18
+
+
 def test_paged_equals_contiguous_on_gpu():
     x = synth.generate(3, 16, 2, 128, [250, 31, 1024], seed=24)
     ps = 16
