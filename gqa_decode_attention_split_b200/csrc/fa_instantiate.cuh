@@ -24,8 +24,23 @@ cudaError_t launch_decode(const KernelArgs& args, int grid, size_t smem, cudaStr
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
-  fa_decode_kernel<Cons><<<grid, Cons::C::THREADS, smem, stream>>>(args);
-  return cudaGetLastError();
+  // Launched as a programmatic dependent of whatever precedes it on the
+  // stream: its blocks may be placed while that work drains (they wait in
+  // griddepcontrol.wait before touching global memory), which hides the
+  // launch between back-to-back passes.  The split-merge kernel that ends a
+  // pass does not signal early, so the next pass's blocks are placed only
+  // once it has finished.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(Cons::C::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fa_decode_kernel<Cons>, args);
 }
 
 template <class Cons>

@@ -954,6 +954,14 @@ __global__ void __maxnreg__(224)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ps = a.paged ? (1 << a.page_shift) : 0;
+  if (tid == 0) {  // kernel parameters: safe to touch before the wait below
+    prefetch_tensormap(&a.kmap);
+    prefetch_tensormap(&a.vmap);
+  }
+  // Nothing in global memory is read or written before the work that
+  // precedes this launch on the stream has finished (this kernel may be
+  // placed early as a programmatic dependent of it).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // ---- setup: request lengths (validated), barriers, tile prefix sums
   for (int b = tid; b < B; b += blockDim.x) {
@@ -1066,10 +1074,6 @@ __global__ void __maxnreg__(224)
     // loaded into registers before lane 0 issues the current window and
     // stored after it, so the page-table round trip overlaps the copies.
     const uint64_t pol = l2_evict_first_policy();
-    if (lane == 0) {
-      prefetch_tensormap(&a.kmap);
-      prefetch_tensormap(&a.vmap);
-    }
     const int NB = T / a.box_t;  // boxes per tile (paged: one page each, contiguous: 1)
     // tiles per window of 64 page ids (a window that starts inside a page may
     // touch one page more than its token count suggests)
