@@ -84,13 +84,14 @@ class DecodeInputs:
     page_size: int
     window: int            # <= 0: all keys
     sm_scale: float
-    q: np.ndarray          # uint16 [batch, qo_heads, head_dim]
+    q: np.ndarray          # uint16 [batch, qo_heads, head_dim] ([batch, q_len, ...] if q_len > 1)
     k: np.ndarray          # contiguous [rows, kv_heads, d]; paged [pages, page_size, kv_heads, d]
     v: np.ndarray
     kv_indptr: np.ndarray  # int32 [batch + 1]
     page_table: Optional[np.ndarray] = None  # int32 [batch, stride]
     k_scale: Optional[np.ndarray] = None     # float32 [kv_heads]
     v_scale: Optional[np.ndarray] = None
+    q_len: int = 1         # query tokens per request: the request's newest keys
 
     @property
     def group(self) -> int:
@@ -110,9 +111,12 @@ class DecodeInputs:
         return 1 if self.kv_dtype == "fp8_e4m3" else 2
 
     def visible_lens(self) -> np.ndarray:
+        """Keys some query token of the request sees (the union of the
+        tokens' windows: the last query token's window plus the q_len - 1
+        keys before it)."""
         L = self.kv_lens
         if self.window > 0:
-            return np.minimum(L, self.window)
+            return np.minimum(L, self.window + self.q_len - 1)
         return L
 
     def kv_bytes(self) -> int:
@@ -131,7 +135,8 @@ def generate(batch: int, qo_heads: int, kv_heads: int, head_dim: int,
              kv_lens: Sequence[int], *, kv_dtype: str = "bf16", paged: bool = False,
              page_size: int = 16, window: int = -1, sm_scale: Optional[float] = None,
              seed: int = 0, name: str = "custom", page_order: str = "random",
-             unused_slot_fill: Optional[str] = None, extra_rows: int = 0) -> DecodeInputs:
+             unused_slot_fill: Optional[str] = None, extra_rows: int = 0,
+             q_len: int = 1) -> DecodeInputs:
     """Draw one decode problem.
 
     kv_lens: per-request key counts.  paged: pool of sum(ceil(L/page_size))
@@ -140,6 +145,8 @@ def generate(batch: int, qo_heads: int, kv_heads: int, head_dim: int,
     past each request's last key (they must never be read as values).
     extra_rows: contiguous layout only, rows of random data appended after
     the last request (tiles that run past a request read them).
+    q_len: query tokens per request (q is [batch, q_len, qo_heads, head_dim]
+    when q_len > 1); they are the request's q_len newest keys.
     """
     if kv_dtype not in ("bf16", "fp8_e4m3"):
         raise ValueError(kv_dtype)
@@ -154,7 +161,10 @@ def generate(batch: int, qo_heads: int, kv_heads: int, head_dim: int,
         sm_scale = 1.0 / math.sqrt(head_dim)
     d = head_dim
 
-    q = _to_bf16_bits(_normals(seed, _S_Q, batch * qo_heads * d)).reshape(batch, qo_heads, d)
+    if q_len < 1:
+        raise ValueError("q_len must be >= 1")
+    qshape = (batch, qo_heads, d) if q_len == 1 else (batch, q_len, qo_heads, d)
+    q = _to_bf16_bits(_normals(seed, _S_Q, batch * q_len * qo_heads * d)).reshape(qshape)
 
     page_table = None
     if paged:
@@ -207,7 +217,7 @@ def generate(batch: int, qo_heads: int, kv_heads: int, head_dim: int,
                         page_size=page_size if paged else 0, window=window,
                         sm_scale=float(sm_scale), q=q, k=k, v=v,
                         kv_indptr=indptr.astype(np.int32), page_table=page_table,
-                        k_scale=k_scale, v_scale=v_scale)
+                        k_scale=k_scale, v_scale=v_scale, q_len=q_len)
 
 
 def c4_lengths(seed: int = 4, batch: int = 64, lo: int = 512, hi: int = 16384) -> np.ndarray:

@@ -31,6 +31,12 @@
  *    combine exactly through exp(x - y) = exp(x) / exp(y).  oracle_merge is
  *    that combination written out.
  *
+ * Several query tokens per request (speculative or chunked decode, the small-M
+ * regime of the "FlashDecoding++" explainer, section "Flat GEMM
+ * optimization"): the request's q_len newest cached keys are its query
+ * tokens, and token i (position L - q_len + i) sees keys [0, L - q_len + i],
+ * the causal mask of "Standard causal attention" restricted to the new rows.
+ *
  * Readings where the pages are silent (each also listed in the design notes):
  *  - GQA grouping: query head h reads kv head h / (qo_heads / kv_heads).
  *  - window w > 0 keeps exactly the last w keys [L - w, L); w <= 0 keeps all.
@@ -65,6 +71,8 @@ typedef struct {
     const float *v_scale;    /* [kv_heads], fp8 only                          */
     const int32_t *kv_indptr;  /* [batch + 1] token counts, cumulative        */
     const int32_t *page_table; /* [batch, page_table_stride], paged only      */
+    int32_t q_len;           /* query tokens per request (0 means 1); q is
+                                [batch, q_len, qo_heads, head_dim]            */
 } oracle_problem;
 
 /* bf16 is the upper half of an IEEE binary32; widening is exact. */
@@ -110,31 +118,45 @@ static double kv_element(const oracle_problem *p, const void *base,
     return oracle_bf16_to_double(((const uint16_t *)base)[idx]);
 }
 
-/* Visible key range [*lo, *hi) of request b. */
-void oracle_visible_range(const oracle_problem *p, int b, int32_t *lo, int32_t *hi) {
+static int32_t q_len_of(const oracle_problem *p) { return p->q_len > 1 ? p->q_len : 1; }
+
+/* Visible key range [*lo, *hi) of query token i of request b.  The request's
+ * q_len newest keys are its query tokens, so token i sits at position
+ * L - q_len + i and sees every key up to and including itself (causal), or
+ * the last `window` of them.  A token whose position would be negative
+ * (L < q_len) sees nothing. */
+void oracle_visible_range_q(const oracle_problem *p, int b, int i, int32_t *lo, int32_t *hi) {
     int32_t L = p->kv_indptr[b + 1] - p->kv_indptr[b];
+    int32_t end = L - q_len_of(p) + i + 1;
+    if (end < 0) end = 0;
     int32_t start = 0;
-    if (p->window > 0 && L > p->window) start = L - p->window;
+    if (p->window > 0 && end > p->window) start = end - p->window;
     *lo = start;
-    *hi = L;
+    *hi = end;
 }
 
-/* One (request b, query head h): writes head_dim outputs and the lse.
- * Scratch `s` must hold the request's visible key count.  Returns 0. */
-static int decode_one(const oracle_problem *p, int b, int h, double *s,
+/* Visible key range [*lo, *hi) of request b's last query token (the only
+ * one when q_len is 1). */
+void oracle_visible_range(const oracle_problem *p, int b, int32_t *lo, int32_t *hi) {
+    oracle_visible_range_q(p, b, q_len_of(p) - 1, lo, hi);
+}
+
+/* One (request b, query token qi, query head h): writes head_dim outputs and
+ * the lse.  Scratch `s` must hold the request's visible key count.  Returns 0. */
+static int decode_one(const oracle_problem *p, int b, int qi, int h, double *s,
                       double *out, double *lse) {
     const int d = p->head_dim;
     const int group = p->qo_heads / p->kv_heads;
     const int g = h / group;
     int32_t lo, hi;
-    oracle_visible_range(p, b, &lo, &hi);
+    oracle_visible_range_q(p, b, qi, &lo, &hi);
     const int n = hi - lo;
     for (int i = 0; i < d; ++i) out[i] = 0.0;
     if (n <= 0) {
         *lse = -INFINITY;
         return 0;
     }
-    const uint16_t *qrow = p->q + ((int64_t)b * p->qo_heads + h) * d;
+    const uint16_t *qrow = p->q + (((int64_t)b * q_len_of(p) + qi) * p->qo_heads + h) * d;
 
     /* scores */
     for (int j = 0; j < n; ++j) {
@@ -171,7 +193,8 @@ static int32_t max_visible(const oracle_problem *p) {
     return m;
 }
 
-/* Selected (request, head) pairs: rows[k] = b * qo_heads + h.
+/* Selected (request, query token, head) rows:
+ * rows[k] = (b * q_len + qi) * qo_heads + h.
  * out: [count, head_dim]; lse: [count].  Returns 0, or -1 on allocation
  * failure. */
 int oracle_decode_rows(const oracle_problem *p, const int64_t *rows, int64_t count,
@@ -192,9 +215,11 @@ int oracle_decode_rows(const oracle_problem *p, const int64_t *rows, int64_t cou
         } else {
 #pragma omp for schedule(dynamic, 1)
             for (int64_t r = 0; r < count; ++r) {
-                int b = (int)(rows[r] / p->qo_heads);
+                int64_t bq = rows[r] / p->qo_heads;
                 int h = (int)(rows[r] % p->qo_heads);
-                decode_one(p, b, h, s, out + r * p->head_dim, lse + r);
+                int b = (int)(bq / q_len_of(p));
+                int qi = (int)(bq % q_len_of(p));
+                decode_one(p, b, qi, h, s, out + r * p->head_dim, lse + r);
             }
             free(s);
         }
@@ -202,9 +227,10 @@ int oracle_decode_rows(const oracle_problem *p, const int64_t *rows, int64_t cou
     return failed ? -1 : 0;
 }
 
-/* Every (request, head): out [batch, qo_heads, head_dim]; lse [batch, qo_heads]. */
+/* Every (request, query token, head): out [batch, q_len, qo_heads, head_dim];
+ * lse [batch, q_len, qo_heads]. */
 int oracle_decode_all(const oracle_problem *p, double *out, double *lse, int nthreads) {
-    int64_t count = (int64_t)p->batch * p->qo_heads;
+    int64_t count = (int64_t)p->batch * q_len_of(p) * p->qo_heads;
     int64_t *rows = (int64_t *)malloc(sizeof(int64_t) * (size_t)(count > 0 ? count : 1));
     if (!rows) return -1;
     for (int64_t r = 0; r < count; ++r) rows[r] = r;

@@ -48,6 +48,7 @@ class _Problem(ctypes.Structure):
         ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
         ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
         ("kv_indptr", ctypes.c_void_p), ("page_table", ctypes.c_void_p),
+        ("q_len", ctypes.c_int32),
     ]
 
 
@@ -102,19 +103,32 @@ def _problem(x) -> Tuple[_Problem, list]:
                  page_table_stride=int(pt.shape[1]) if pt is not None else 0,
                  window=int(x.window), sm_scale=float(x.sm_scale),
                  q=_ptr(q), k=_ptr(k), v=_ptr(v), k_scale=_ptr(ks), v_scale=_ptr(vs),
-                 kv_indptr=_ptr(ind), page_table=_ptr(pt))
+                 kv_indptr=_ptr(ind), page_table=_ptr(pt), q_len=_q_len(x))
     return p, keep
 
 
+def _q_len(x) -> int:
+    return int(getattr(x, "q_len", 1) or 1)
+
+
+def _row_shape(x):
+    """Leading dims of out / lse: [batch, qo_heads], or [batch, q_len,
+    qo_heads] when a request has several query tokens."""
+    Q = _q_len(x)
+    return (x.batch, x.qo_heads) if Q == 1 else (x.batch, Q, x.qo_heads)
+
+
 def decode_all(x, nthreads: int = 0) -> Tuple[np.ndarray, np.ndarray]:
-    """Exact attention for every (request, query head).
+    """Exact attention for every (request, query token, query head).
 
     Returns out float64 [batch, qo_heads, head_dim] and lse float64
-    [batch, qo_heads] (natural log; -inf for an empty key set)."""
+    [batch, qo_heads] (natural log; -inf for an empty key set); with several
+    query tokens per request, [batch, q_len, qo_heads, head_dim] and
+    [batch, q_len, qo_heads]."""
     lib = _load()
     p, keep = _problem(x)
-    out = np.empty((x.batch, x.qo_heads, x.head_dim), dtype=np.float64)
-    lse = np.empty((x.batch, x.qo_heads), dtype=np.float64)
+    out = np.empty(_row_shape(x) + (x.head_dim,), dtype=np.float64)
+    lse = np.empty(_row_shape(x), dtype=np.float64)
     dp = ctypes.POINTER(ctypes.c_double)
     rc = lib.oracle_decode_all(ctypes.byref(p), out.ctypes.data_as(dp), lse.ctypes.data_as(dp),
                                int(nthreads))
@@ -125,13 +139,14 @@ def decode_all(x, nthreads: int = 0) -> Tuple[np.ndarray, np.ndarray]:
 
 
 def decode_rows(x, rows, nthreads: int = 0) -> Tuple[np.ndarray, np.ndarray]:
-    """Exact attention for selected rows r = b * qo_heads + h.
+    """Exact attention for selected rows r = (b * q_len + i) * qo_heads + h
+    (r = b * qo_heads + h for one query token per request).
 
     Returns out float64 [len(rows), head_dim] and lse float64 [len(rows)]."""
     lib = _load()
     p, keep = _problem(x)
     rows = np.ascontiguousarray(rows, dtype=np.int64)
-    if rows.size and (rows.min() < 0 or rows.max() >= x.batch * x.qo_heads):
+    if rows.size and (rows.min() < 0 or rows.max() >= x.batch * _q_len(x) * x.qo_heads):
         raise IndexError("row out of range")
     out = np.empty((rows.size, x.head_dim), dtype=np.float64)
     lse = np.empty((rows.size,), dtype=np.float64)

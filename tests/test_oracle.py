@@ -348,3 +348,99 @@ def test_merge_closed_forms_and_algebra():
     np.testing.assert_allclose(lm, l[0], atol=1e-15)
     om, lm = oracle.merge(o[:2], np.stack([ninf, ninf]))
     assert (om == 0).all() and np.isneginf(lm).all()
+
+
+# ------------------------------------------------------ several query tokens
+# A request's q_len newest keys are its query tokens; token i sits at position
+# L - q_len + i and sees keys up to and including itself (the causal mask of
+# "Standard causal attention" restricted to the new rows), or the last
+# `window` of those.
+
+def _brute_multi(x):
+    """Plain numpy two-pass softmax with an explicit causal mask, written
+    apart from the oracle: out [B, Q, Hq, d], lse [B, Q, Hq]."""
+    B, Q, Hq, d = x.batch, x.q_len, x.qo_heads, x.head_dim
+    G = Hq // x.kv_heads
+    qf = bf16_values(x.q).reshape(B, Q, Hq, d)
+    out = np.zeros((B, Q, Hq, d))
+    lse = np.full((B, Q, Hq), -np.inf)
+    for b in range(B):
+        kf, vf = dense_kv(x, b)
+        L = kf.shape[0]
+        pos = np.arange(L)
+        for i in range(Q):
+            me = L - Q + i
+            mask = pos <= me
+            if x.window > 0:
+                mask &= pos > me - x.window
+            if not mask.any():
+                continue
+            for h in range(Hq):
+                s = x.sm_scale * (kf[mask, h // G] @ qf[b, i, h])
+                m = s.max()
+                z = np.exp(s - m).sum()
+                out[b, i, h] = (np.exp(s - m) / z) @ vf[mask, h // G]
+                lse[b, i, h] = m + math.log(z)
+    return out, lse
+
+
+@pytest.mark.parametrize("window", [-1, 1, 4, 6])
+def test_multi_token_matches_brute_force(window):
+    x = synth.generate(3, 4, 2, 8, [9, 3, 17], q_len=3, paged=True, page_size=4, seed=40,
+                       window=window)
+    out, lse = oracle.decode_all(x)
+    assert out.shape == (3, 3, 4, 8) and lse.shape == (3, 3, 4)
+    ref_out, ref_lse = _brute_multi(x)
+    np.testing.assert_allclose(out, ref_out, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("window", [-1, 5])
+def test_multi_token_rows_are_single_token_decodes(window):
+    """Row (b, i, h) of a q_len problem is the one-token decode of request b
+    truncated to L - q_len + i + 1 keys, with token i's query: the same pool,
+    only the token counts change."""
+    Q = 4
+    lens = [33, 4, 18]
+    x = synth.generate(3, 8, 2, 16, lens, q_len=Q, paged=True, page_size=8, seed=41,
+                       window=window)
+    out, lse = oracle.decode_all(x)
+    for i in range(Q):
+        short = np.array([L - Q + i + 1 for L in lens])
+        ind = np.concatenate([[0], np.cumsum(short)]).astype(np.int32)
+        y = DecodeInputs(**{**x.__dict__, "q": np.ascontiguousarray(x.q[:, i]), "kv_indptr": ind,
+                            "q_len": 1})
+        o1, l1 = oracle.decode_all(y)
+        np.testing.assert_allclose(out[:, i], o1, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[:, i], l1, rtol=0, atol=1e-12)
+
+
+def test_multi_token_causal_boundary_with_a_spike_key():
+    """A spike key at position p is seen by the query tokens at or after p
+    (they return its value row) and by none before it."""
+    d, L, Q = 8, 40, 5
+    x = synth.generate(1, 2, 1, d, [L], q_len=Q, seed=42)
+    q = np.zeros((1, Q, 2, d), np.float32)
+    q[..., 0] = 8.0
+    k = np.zeros_like(x.k)
+    p = L - 3  # the position of query token Q - 3
+    k[p, 0, 0] = bf16_bits(np.float32(5.0))
+    y = DecodeInputs(**{**x.__dict__, "q": bf16_bits(q), "k": k, "sm_scale": 1.0})
+    out, lse = oracle.decode_all(y)
+    _, vf = dense_kv(y, 0)
+    for i in range(Q):
+        me = L - Q + i
+        if me >= p:
+            np.testing.assert_allclose(out[0, i, 0], vf[p, 0], atol=1e-12)
+        else:
+            np.testing.assert_allclose(out[0, i, 0], vf[:me + 1, 0].mean(axis=0), atol=1e-12)
+            assert abs(lse[0, i, 0] - math.log(me + 1)) < 1e-12
+
+
+def test_multi_token_shorter_request_than_query_block():
+    """A query token whose position would be negative (L < q_len) sees no key:
+    out = 0, lse = -inf; the others behave as usual."""
+    x = synth.generate(1, 2, 1, 8, [2], q_len=4, seed=43)
+    out, lse = oracle.decode_all(x)
+    assert np.isneginf(lse[0, :2]).all() and (out[0, :2] == 0).all()
+    assert np.isfinite(lse[0, 2:]).all()
