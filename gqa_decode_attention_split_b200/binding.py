@@ -41,7 +41,7 @@ class DecodeDesc(ctypes.Structure):
                 ("kv_dtype", ctypes.c_int32), ("paged", ctypes.c_int32),
                 ("page_size", ctypes.c_int32), ("window", ctypes.c_int32),
                 ("sm_scale", ctypes.c_float), ("path", ctypes.c_int32),
-                ("num_ctas", ctypes.c_int32)]
+                ("num_ctas", ctypes.c_int32), ("q_len", ctypes.c_int32)]
 
 
 class PlanInfo(ctypes.Structure):
@@ -149,7 +149,7 @@ class DecodePlan:
 def plan(batch: int, qo_heads: int, kv_heads: int, head_dim: int, kv_indptr_host, *,
          kv_dtype: str = "bf16", paged: bool = False, page_size: int = 0, window: int = -1,
          sm_scale: Optional[float] = None, path: str = "auto", num_ctas: int = 0,
-         num_sms: int = 0) -> DecodePlan:
+         num_sms: int = 0, q_len: int = 1) -> DecodePlan:
     lib = load_library()
     ind = np.ascontiguousarray(np.asarray(
         kv_indptr_host.cpu().numpy() if hasattr(kv_indptr_host, "cpu") else kv_indptr_host,
@@ -159,12 +159,19 @@ def plan(batch: int, qo_heads: int, kv_heads: int, head_dim: int, kv_indptr_host
     desc = DecodeDesc(batch=batch, qo_heads=qo_heads, kv_heads=kv_heads, head_dim=head_dim,
                       kv_dtype=KV_FP8_E4M3 if kv_dtype == "fp8_e4m3" else KV_BF16,
                       paged=int(bool(paged)), page_size=int(page_size), window=int(window),
-                      sm_scale=float(sm_scale), path=_PATH_NAMES[path], num_ctas=int(num_ctas))
+                      sm_scale=float(sm_scale), path=_PATH_NAMES[path], num_ctas=int(num_ctas),
+                      q_len=int(q_len))
     handle = ctypes.c_void_p()
     ws = ctypes.c_size_t()
     _check(lib.fa_decode_plan(ctypes.byref(desc), ind.ctypes.data, int(num_sms),
                               ctypes.byref(handle), ctypes.byref(ws)), "fa_decode_plan")
     return DecodePlan(handle.value, desc, ws.value)
+
+
+def _rows(d) -> tuple:
+    """Leading dims of out / lse: [batch, qo_heads], or [batch, q_len,
+    qo_heads] with several query tokens per request."""
+    return (d.batch, d.qo_heads) if d.q_len <= 1 else (d.batch, d.q_len, d.qo_heads)
 
 
 def run(p: DecodePlan, q, k, v, kv_indptr, *, page_table=None, k_scale=None, v_scale=None,
@@ -174,10 +181,9 @@ def run(p: DecodePlan, q, k, v, kv_indptr, *, page_table=None, k_scale=None, v_s
     lib = load_library()
     d = p.desc
     if out is None:
-        out = torch.empty((d.batch, d.qo_heads, d.head_dim), dtype=torch.bfloat16,
-                          device=q.device)
+        out = torch.empty(_rows(d) + (d.head_dim,), dtype=torch.bfloat16, device=q.device)
     if lse is None and want_lse:
-        lse = torch.empty((d.batch, d.qo_heads), dtype=torch.float32, device=q.device)
+        lse = torch.empty(_rows(d), dtype=torch.float32, device=q.device)
     if workspace is None:
         workspace = p.new_workspace(q.device)
     pt_stride = int(page_table.stride(0)) if page_table is not None else 0
@@ -198,10 +204,9 @@ def run_static(p: DecodePlan, q, k, v, kv_indptr, *, page_table=None, k_scale=No
     lib = load_library()
     d = p.desc
     if out is None:
-        out = torch.empty((d.batch, d.qo_heads, d.head_dim), dtype=torch.bfloat16,
-                          device=q.device)
+        out = torch.empty(_rows(d) + (d.head_dim,), dtype=torch.bfloat16, device=q.device)
     if lse is None and want_lse:
-        lse = torch.empty((d.batch, d.qo_heads), dtype=torch.float32, device=q.device)
+        lse = torch.empty(_rows(d), dtype=torch.float32, device=q.device)
     pt_stride = int(page_table.stride(0)) if page_table is not None else 0
     st = lib.fa_decode_run_static(p._handle, _ptr(q), _ptr(k), _ptr(v), int(k.shape[0]),
                                   _ptr(page_table), pt_stride, _ptr(kv_indptr), _ptr(k_scale),

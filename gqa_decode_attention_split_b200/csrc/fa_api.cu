@@ -123,8 +123,17 @@ fa_status validate_desc(const fa_decode_desc* d) {
   if (!isfinite(d->sm_scale)) return FA_ERR_INVALID_ARG;
   if (d->path < FA_PATH_AUTO || d->path > FA_PATH_MMA) return FA_ERR_INVALID_ARG;
   if (d->num_ctas < 0) return FA_ERR_INVALID_ARG;
+  if (d->q_len < 0 || d->q_len > 64) return FA_ERR_INVALID_ARG;
   if (static_cast<int64_t>(d->batch) * d->kv_heads > (1 << 30)) return FA_ERR_UNSUPPORTED;
   return FA_OK;
+}
+
+int32_t q_len_of(const fa_decode_desc* d) { return d->q_len > 1 ? d->q_len : 1; }
+
+// Keys that some query token of a request sees: the last token's window and
+// the q_len - 1 keys before it (<= 0: all keys).
+int32_t union_window(const fa_decode_desc* d) {
+  return d->window > 0 ? d->window + q_len_of(d) - 1 : d->window;
 }
 
 }  // namespace
@@ -145,7 +154,8 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_failure("fa_decode_plan: SM count", e);
   }
-  const int group = desc->qo_heads / desc->kv_heads;
+  // rows of a segment: the group's query heads for every query token
+  const int group = desc->qo_heads / desc->kv_heads * q_len_of(desc);
   const int fp8 = desc->kv_dtype == FA_KV_FP8_E4M3 ? 1 : 0;
 
   // Dataflow choice: the tensor-core (MMA) path whenever a kernel exists for
@@ -165,7 +175,7 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   int64_t tiles = 0;
   int64_t seg_tiles = -1;  // tiles of every segment when all are equal, else -1
   for (int b = 0; b < desc->batch; ++b) {
-    const int64_t n = host_num_tiles(kv_indptr_host[b + 1] - kv_indptr_host[b], desc->window, T);
+    const int64_t n = host_num_tiles(kv_indptr_host[b + 1] - kv_indptr_host[b], union_window(desc), T);
     tiles += n;
     seg_tiles = b == 0 ? n : (seg_tiles == n ? n : -1);
   }
@@ -389,7 +399,9 @@ extern "C" fa_status fa_decode_run(const fa_plan* plan, const void* q, const voi
   a.batch = d.batch;
   a.qo_heads = d.qo_heads;
   a.kv_heads = d.kv_heads;
-  a.group = plan->group;
+  a.group = d.qo_heads / d.kv_heads;
+  a.q_len = q_len_of(&d);
+  a.window_u = d.window > 0 ? union_window(&d) : -1;
   a.window = d.window > 0 ? d.window : -1;
   a.paged = d.paged;
   a.page_shift = plan->page_shift;
@@ -410,6 +422,8 @@ extern "C" fa_status fa_decode_run(const fa_plan* plan, const void* q, const voi
   m.lse = a.lse;
   m.num_records = plan->num_ctas;
   m.group = plan->group;
+  m.kv_group = d.qo_heads / d.kv_heads;
+  m.q_len = q_len_of(&d);
   m.kv_heads = d.kv_heads;
   m.qo_heads = d.qo_heads;
   m.batch = d.batch;

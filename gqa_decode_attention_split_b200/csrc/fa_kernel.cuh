@@ -97,7 +97,9 @@ struct KernelArgs {
   float* part_lse;
   long long kv_rows;
   int max_partials;
-  int batch, qo_heads, kv_heads, group;
+  int batch, qo_heads, kv_heads, group;   // group: query heads per kv head
+  int q_len;          // query tokens per request (rows of a segment: group * q_len)
+  int window_u;       // keys any query token of a request sees: window + q_len - 1 (<= 0: all)
   int window;
   int paged, page_shift, pt_stride, box_t, swz;
   int seg_parts;      // 0: equal runs of all tiles; k > 0: k runs per segment
@@ -365,18 +367,19 @@ struct SimtConsumer {
     return tile_addr<C>(tile, r, chunk_plane(k), chunk_in_plane(k), swz);
   }
 
-  // qs: the piece's G query rows (staged in shared memory, or in global
-  // memory where the tile geometry leaves no room); kscale: the fp8
-  // K scale of the piece's kv head (1 for bf16).
-  __device__ __forceinline__ void begin_piece(const KernelArgs& a, const uint16_t* qs, float kscale,
-                                              int lane) {
+  // qs: the piece's query rows (staged in shared memory, or in global
+  // memory where the tile geometry leaves no room): row r (token r / group,
+  // head r % group) at qs + (r / group) * qstride + (r % group) * D; kscale:
+  // the fp8 K scale of the piece's kv head (1 for bf16).
+  __device__ __forceinline__ void begin_piece(const KernelArgs& a, const uint16_t* qs, int qstride,
+                                              float kscale, int lane) {
     slot = lane / LPT;
     j = lane % LPT;
     float scale = a.score_scale;
     if constexpr (FP8) scale *= kscale;
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      const uint16_t* qrow = qs + h * D;
+      const uint16_t* qrow = qs + (h / a.group) * qstride + (h % a.group) * D;
 #pragma unroll
       for (int k = 0; k < CPL; ++k) {
 #pragma unroll
@@ -404,10 +407,19 @@ struct SimtConsumer {
   static_assert(TPS % TPSC == 0, "sub-steps");
 
   // K and V rows are read together sub-step by sub-step, so K is released
-  // at the end (release_k as for the MMA dataflow).
+  // at the end (release_k as for the MMA dataflow).  [lo, hi) is the union
+  // of the rows' key ranges (hi: the request's length); with several query
+  // tokens, row h (token h / group) sees one key fewer per token before the
+  // last, within its own window.
+  __device__ __forceinline__ bool row_sees(const KernelArgs& a, int h, int pos, int hi) const {
+    const int rhi = hi - (a.q_len - 1 - h / a.group);
+    const int rlo = (a.window > 0 && rhi > a.window) ? rhi - a.window : 0;
+    return pos >= rlo && pos < rhi;
+  }
   template <class ReleaseK>
   __device__ __forceinline__ void tile(const KernelArgs& a, uint32_t kt, uint32_t vt, int pos0,
                                        int lo, int hi, int lane, ReleaseK&& release_k) {
+    const bool multi = a.q_len > 1;
 #pragma unroll 1
     for (int si = 0; si < NSUB; ++si) {
       float s[TPSC][G];
@@ -433,7 +445,8 @@ struct SimtConsumer {
         const int pos = pos0 + r;
         const bool valid = pos >= lo && pos < hi;
 #pragma unroll
-        for (int h = 0; h < G; ++h) s[tt][h] = valid ? part[h] : -CUDART_INF_F;
+        for (int h = 0; h < G; ++h)
+          s[tt][h] = (multi ? row_sees(a, h, pos, hi) : valid) ? part[h] : -CUDART_INF_F;
       }
       // running max with slack: rescale only when the max grows by more than kRescaleSlack
       bool need = false;
@@ -550,16 +563,18 @@ struct MmaConsumer {
   float sscale[2];
   int g, t;
 
-  // qs: the piece's G query rows (staged in shared memory, or in global
-  // memory where the tile geometry leaves no room); kscale: the fp8
-  // K scale of the piece's kv head (1 for bf16).
-  __device__ __forceinline__ void begin_piece(const KernelArgs& a, const uint16_t* qs, float kscale,
-                                              int lane) {
+  // qs: the piece's query rows (staged in shared memory, or in global
+  // memory where the tile geometry leaves no room): row r (token r / group,
+  // head r % group) at qs + (r / group) * qstride + (r % group) * D; kscale:
+  // the fp8 K scale of the piece's kv head (1 for bf16).
+  __device__ __forceinline__ void begin_piece(const KernelArgs& a, const uint16_t* qs, int qstride,
+                                              float kscale, int lane) {
     g = lane >> 2;
     t = lane & 3;
-    const int G = a.group;
+    const int G = a.group * a.q_len;
     const bool real = g < G;
-    const uint16_t* qrow = qs + (real ? g : 0) * D;
+    const int r = real ? g : 0;
+    const uint16_t* qrow = qs + (r / a.group) * qstride + (r % a.group) * D;
     if constexpr (!FP8) {
 #pragma unroll
       for (int kk = 0; kk < KS; ++kk) {
@@ -718,15 +733,25 @@ struct MmaConsumer {
 #pragma unroll
     for (int sub = 0; sub < SUB; ++sub) scores(a, kt, sub, lane, sc[sub]);
     release_k();
+    // key range of this lane's two columns (rows 2t, 2t + 1: query token
+    // row / group sees one key fewer per token before the last, within its
+    // own window); [lo, hi) is the union, and padding columns keep it
+    int chi0 = hi - (a.q_len - 1 - (2 * t) / a.group);
+    int chi1 = hi - (a.q_len - 1 - (2 * t + 1) / a.group);
+    chi0 = chi0 < hi ? chi0 : hi;
+    chi1 = chi1 < hi ? chi1 : hi;
+    const int clo0 = (a.window > 0 && chi0 > a.window) ? chi0 - a.window : 0;
+    const int clo1 = (a.window > 0 && chi1 > a.window) ? chi1 - a.window : 0;
     float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F;
 #pragma unroll
     for (int sub = 0; sub < SUB; ++sub) {
       const int pr = pos0 + sub * 16 + g;
-      const bool v0 = pr >= lo && pr < hi, v1 = pr + 8 >= lo && pr + 8 < hi;
-      sc[sub][0] = v0 ? sc[sub][0] * sscale[0] : -CUDART_INF_F;
-      sc[sub][1] = v0 ? sc[sub][1] * sscale[1] : -CUDART_INF_F;
-      sc[sub][2] = v1 ? sc[sub][2] * sscale[0] : -CUDART_INF_F;
-      sc[sub][3] = v1 ? sc[sub][3] * sscale[1] : -CUDART_INF_F;
+      const bool v00 = pr >= clo0 && pr < chi0, v01 = pr >= clo1 && pr < chi1;
+      const bool v80 = pr + 8 >= clo0 && pr + 8 < chi0, v81 = pr + 8 >= clo1 && pr + 8 < chi1;
+      sc[sub][0] = v00 ? sc[sub][0] * sscale[0] : -CUDART_INF_F;
+      sc[sub][1] = v01 ? sc[sub][1] * sscale[1] : -CUDART_INF_F;
+      sc[sub][2] = v80 ? sc[sub][2] * sscale[0] : -CUDART_INF_F;
+      sc[sub][3] = v81 ? sc[sub][3] * sscale[1] : -CUDART_INF_F;
       mx0 = fmaxf(mx0, fmaxf(sc[sub][0], sc[sub][2]));
       mx1 = fmaxf(mx1, fmaxf(sc[sub][1], sc[sub][3]));
     }
@@ -936,7 +961,10 @@ __global__ void __maxnreg__(224)
   // measured slower in the paged producer loop (one copy per page, so the
   // loop's length bounds how fast copies go out), for no gain.
   constexpr bool kSplitKV = C::KSTAGES != C::VSTAGES;
-  const int G = a.group;
+  // A segment's rows are its group's query heads for each of the request's
+  // query tokens: row r is token r / GK, head r % GK of the group.
+  const int GK = a.group, Q = a.q_len;
+  const int G = GK * Q;
   float* m_area = reinterpret_cast<float*>(base + S::kMerge);
   float* l_area = m_area + NW * G;
   float* acc_area = reinterpret_cast<float*>(base + S::acc_off(G));
@@ -1010,7 +1038,7 @@ __global__ void __maxnreg__(224)
     int carry = 0;
     for (int b0 = 0; b0 < B; b0 += 32) {
       const int b = b0 + lane;
-      const int n = b < B ? num_tiles(s_len[b], a.window, T) : 0;
+      const int n = b < B ? num_tiles(s_len[b], a.window_u, T) : 0;
       int incl = n;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -1058,7 +1086,7 @@ __global__ void __maxnreg__(224)
     PieceIter i0 = it;
     Piece p0;
     int4 rec = make_int4(-1, 0, 0, 0);
-    if (next_piece(i0, p0, s_pre, s_len, B, H, a.window, T) && p0.c_first == c - 1)
+    if (next_piece(i0, p0, s_pre, s_len, B, H, a.window_u, T) && p0.c_first == c - 1)
       rec = make_int4(p0.seg, p0.c_first, p0.n_pieces, 0);
     a.records[c] = rec;
   }
@@ -1106,7 +1134,7 @@ __global__ void __maxnreg__(224)
       }
     };
     Piece pc;
-    bool have = next_piece(it, pc, s_pre, s_len, B, H, a.window, T);
+    bool have = next_piece(it, pc, s_pre, s_len, B, H, a.window_u, T);
     int w0 = have ? pc.t0 : 0;
     if (have && a.paged) {
       int v[2];
@@ -1127,12 +1155,16 @@ __global__ void __maxnreg__(224)
             record_timeout(a.status, 5, pq, qs, qpar, qempty0 + 8 * qs);
             ok = false;
           } else {
-            const uint32_t qbytes = static_cast<uint32_t>(G * D * 2);
+            // one copy per query token: its GK rows are contiguous in q
+            const uint32_t tbytes = static_cast<uint32_t>(GK * D * 2);
+            const uint32_t qbytes = tbytes * static_cast<uint32_t>(Q);
             if (FA_CHECK(a.status, qbytes <= static_cast<uint32_t>(C::QSLOT_BYTES), 304, qbytes)) {
               mbar_arrive_expect_tx(qfull0 + 8 * qs, qbytes);
-              bulk_load(smem_addr(q_slots) + qs * C::QSLOT_BYTES,
-                        a.q + (static_cast<size_t>(pc.b) * a.qo_heads + static_cast<size_t>(pc.h) * G) * D,
-                        qbytes, qfull0 + 8 * qs);
+              for (int i = 0; i < Q; ++i)
+                bulk_load(smem_addr(q_slots) + qs * C::QSLOT_BYTES + i * tbytes,
+                          a.q + ((static_cast<size_t>(pc.b) * Q + i) * a.qo_heads +
+                                 static_cast<size_t>(pc.h) * GK) * D,
+                          tbytes, qfull0 + 8 * qs);
             }
           }
         }
@@ -1147,7 +1179,7 @@ __global__ void __maxnreg__(224)
       int nw0 = w1;
       bool nhave = true;
       if (w1 >= pc.t1) {
-        nhave = next_piece(itn, pn, s_pre, s_len, B, H, a.window, T);
+        nhave = next_piece(itn, pn, s_pre, s_len, B, H, a.window_u, T);
         nw0 = nhave ? pn.t0 : 0;
       }
       int nv[2] = {-1, -1};
@@ -1300,10 +1332,11 @@ __global__ void __maxnreg__(224)
   // requests without keys: out = 0, lse = -inf (spread over blocks)
   for (int b = c; b < B; b += P) {
     if (s_len[b] != 0) continue;
-    const int nq = a.qo_heads * D;
+    const int nq = Q * a.qo_heads * D;  // every query token's rows
     for (int x = ctid; x < nq; x += NCT) {
       a.out[static_cast<size_t>(b) * nq + x] = 0;
-      if (a.lse != nullptr && (x % D) == 0) a.lse[static_cast<size_t>(b) * a.qo_heads + x / D] = -CUDART_INF_F;
+      if (a.lse != nullptr && (x % D) == 0)
+        a.lse[static_cast<size_t>(b) * Q * a.qo_heads + x / D] = -CUDART_INF_F;
     }
   }
 
@@ -1321,9 +1354,9 @@ __global__ void __maxnreg__(224)
   bool alive = true;
   int piece = 0;         // pieces this block has finished (merge-area uses)
   Piece pc;
-  while (next_piece(it, pc, s_pre, s_len, B, H, a.window, T)) {
+  while (next_piece(it, pc, s_pre, s_len, B, H, a.window_u, T)) {
     const int L = s_len[pc.b];
-    const int lo = (a.window > 0 && L > a.window) ? L - a.window : 0;
+    const int lo = (a.window_u > 0 && L > a.window_u) ? L - a.window_u : 0;  // union of the rows' ranges
     const int n = pc.t1 - pc.t0;
     if constexpr (C::STAGE_Q) {
       const int qs = piece & 1;
@@ -1335,13 +1368,14 @@ __global__ void __maxnreg__(224)
         }
       }
       const float ks = C::ES == 1 ? (scales_in_smem ? s_kscale[pc.h] : __ldg(a.k_scale + pc.h)) : 1.f;
-      cons.begin_piece(a, q_slots + qs * (C::QSLOT_BYTES / 2), ks, lane);
+      cons.begin_piece(a, q_slots + qs * (C::QSLOT_BYTES / 2), GK * D, ks, lane);
       __syncwarp();
       if (lane == 0) mbar_arrive(qempty0 + 8 * qs);
     } else {
       const float ks = C::ES == 1 ? (scales_in_smem ? s_kscale[pc.h] : __ldg(a.k_scale + pc.h)) : 1.f;
-      cons.begin_piece(a, a.q + (static_cast<size_t>(pc.b) * a.qo_heads + static_cast<size_t>(pc.h) * G) * D,
-                       ks, lane);
+      cons.begin_piece(a,
+                       a.q + (static_cast<size_t>(pc.b) * Q * a.qo_heads + static_cast<size_t>(pc.h) * GK) * D,
+                       a.qo_heads * D, ks, lane);
     }
     for (; next < base_i + n; next += NW) {
       // both halves of the tile are waited for up front (a second wait in
@@ -1433,9 +1467,10 @@ __global__ void __maxnreg__(224)
 #pragma unroll
         for (int ww = 0; ww < NW; ++ww) m_area[ww * G + h] = scw[ww] * f;
         const float lv = empty ? -CUDART_INF_F : (M + __log2f(Ls)) * kLn2;
-        const size_t row = static_cast<size_t>(pc.b) * a.qo_heads + static_cast<size_t>(pc.h) * G + h;
+        const size_t row = (static_cast<size_t>(pc.b) * Q + h / GK) * a.qo_heads +
+                           static_cast<size_t>(pc.h) * GK + h % GK;
         if (whole) {
-          if (a.lse != nullptr && FA_CHECK(a.status, row < static_cast<size_t>(B) * a.qo_heads, 401, row))
+          if (a.lse != nullptr && FA_CHECK(a.status, row < static_cast<size_t>(B) * Q * a.qo_heads, 401, row))
             a.lse[row] = lv;
         } else if (FA_CHECK(a.status, slot_idx < a.max_partials, 402, slot_idx)) {
           a.part_lse[static_cast<size_t>(slot_idx) * G + h] = lv;
@@ -1457,9 +1492,10 @@ __global__ void __maxnreg__(224)
           O.z = fmaf(av.z, f, O.z);
           O.w = fmaf(av.w, f, O.w);
         }
-        const size_t row = static_cast<size_t>(pc.b) * a.qo_heads + static_cast<size_t>(pc.h) * G + h;
+        const size_t row = (static_cast<size_t>(pc.b) * Q + h / GK) * a.qo_heads +
+                           static_cast<size_t>(pc.h) * GK + h % GK;
         if (whole) {
-          if (FA_CHECK(a.status, row < static_cast<size_t>(B) * a.qo_heads, 401, row)) {
+          if (FA_CHECK(a.status, row < static_cast<size_t>(B) * Q * a.qo_heads, 401, row)) {
             uint2 packed;
             packed.x = pack_bf16x2(O.x, O.y);
             packed.y = pack_bf16x2(O.z, O.w);

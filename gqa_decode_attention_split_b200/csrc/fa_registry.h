@@ -36,7 +36,9 @@ struct SplitMergeArgs {
   uint16_t* out;          // bf16 [batch][qo_heads][head_dim]
   float* lse;             // [batch][qo_heads] or null
   int num_records;        // blocks of the main launch
-  int group, kv_heads, qo_heads, batch;
+  int group;              // rows of a segment: kv_group * q_len
+  int kv_group, q_len;    // query heads per kv head, query tokens per request
+  int kv_heads, qo_heads, batch;
   long long max_partials;
 };
 

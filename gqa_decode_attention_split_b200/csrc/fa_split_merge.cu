@@ -129,7 +129,9 @@ __global__ void __launch_bounds__(kMergeThreads)
   }
   const bool none = !(Z > 0.f);
   const float inv = none ? 0.f : 1.f / Z;
-  const size_t row = static_cast<size_t>(b) * a.qo_heads + static_cast<size_t>(hk) * G + h;
+  // row h of the segment: query token h / kv_group, head h % kv_group
+  const size_t row = (static_cast<size_t>(b) * a.q_len + h / a.kv_group) * a.qo_heads +
+                     static_cast<size_t>(hk) * a.kv_group + h % a.kv_group;
   for (int col = threadIdx.x; col < D4; col += kMergeThreads) {
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll

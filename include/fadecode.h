@@ -94,6 +94,14 @@ typedef struct {
   int32_t num_ctas;   /* 0: planner's choice.  n > 0 forces n thread blocks, */
                       /* i.e. the KV split granularity (used to test that    */
                       /* split-then-merge equals the unsplit result)         */
+  int32_t q_len;      /* query tokens per request, 0 or 1: one.  q_len > 1   */
+                      /* (speculative or chunked decode, the small-M case of */
+                      /* the "FlashDecoding++" explainer, section "Flat GEMM */
+                      /* optimization"): the request's q_len newest keys are */
+                      /* its query tokens, and token i (position            */
+                      /* L - q_len + i) sees the keys up to and including    */
+                      /* itself, or the last `window` of them.  Needs        */
+                      /* (qo_heads / kv_heads) * q_len <= 8.                 */
 } fa_decode_desc;
 
 typedef struct fa_plan fa_plan;
@@ -131,9 +139,10 @@ typedef struct {
  *  plan            receives the new plan (caller frees: fa_plan_destroy).
  *  workspace_bytes receives the minimum workspace size.
  * Errors: FA_ERR_INVALID_ARG (null pointer, non-positive shape, qo_heads not
- * a multiple of kv_heads, bad indptr, non-finite sm_scale, bad page_size),
- * FA_ERR_UNSUPPORTED (head_dim / group / dtype / path combination without a
- * kernel), FA_ERR_CUDA (num_sms == 0 and no device could be queried).
+ * a multiple of kv_heads, bad indptr, non-finite sm_scale, bad page_size,
+ * q_len < 0 or > 64), FA_ERR_UNSUPPORTED (head_dim / group * q_len / dtype /
+ * path combination without a kernel), FA_ERR_CUDA (num_sms == 0 and no
+ * device could be queried).
  */
 FA_API fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* kv_indptr_host,
                          int32_t num_sms, fa_plan** plan, size_t* workspace_bytes);
@@ -148,7 +157,8 @@ FA_API void fa_plan_destroy(fa_plan* plan);
  * fa_decode_run -- enqueue one decode-attention pass on `stream`.
  *
  * Layouts (row-major, all device memory):
- *  q           bf16 [batch, qo_heads, head_dim], 16-byte aligned.
+ *  q           bf16 [batch, q_len, qo_heads, head_dim] (q_len = 1:
+ *              [batch, qo_heads, head_dim]), 16-byte aligned.
  *  k, v        contiguous: [kv_rows, kv_heads, head_dim]; request b owns rows
  *              [kv_indptr[b], kv_indptr[b+1]) (batch 1: rows 0..kv_len-1).
  *              paged: pools [kv_rows, page_size, kv_heads, head_dim] where
@@ -164,8 +174,10 @@ FA_API void fa_plan_destroy(fa_plan* plan);
  *  kv_indptr   int32 [batch + 1], device copy of the plan's indptr.
  *  k_scale,    fp8 only (else NULL): fp32 [kv_heads]; a stored code c of kv
  *  v_scale     head g means e4m3(c) * scale[g].
- *  out         bf16 [batch, qo_heads, head_dim], 16-byte aligned.
- *  lse         fp32 [batch, qo_heads], natural log; NULL = do not write.
+ *  out         bf16 [batch, q_len, qo_heads, head_dim], 16-byte aligned.
+ *  lse         fp32 [batch, q_len, qo_heads], natural log; NULL = do not
+ *              write.  A query token with no visible key (a request shorter
+ *              than q_len) gets out = 0, lse = -inf.
  *              A request with no visible key gets out = 0, lse = -inf.
  *  workspace   device scratch of >= the plan's workspace_bytes, 256-byte
  *              aligned, zero-filled once before its first use (and again

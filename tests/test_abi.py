@@ -215,3 +215,26 @@ def test_binding_raises_without_library(monkeypatch, tmp_path):
             binding.load_library()
     finally:
         binding._lib = saved
+
+
+def test_plan_with_several_query_tokens(lib):
+    """q_len multiplies the rows of a segment (group * q_len <= 8 on the MMA
+    dataflow) and widens the tile range by q_len - 1 keys under a window."""
+    st, h, ws = _plan(lib, _desc(qo_heads=8, kv_heads=2, q_len=2), [0, 1000])
+    assert st == 0
+    inf = _info(lib, h)
+    assert inf.path == binding.PATH_MMA
+    lib.fa_plan_destroy(h)
+    # rows 4 * 4 = 16 exceed every kernel
+    st, h, ws = _plan(lib, _desc(qo_heads=8, kv_heads=2, q_len=4), [0, 1000])
+    assert st == 2 and not h  # FA_ERR_UNSUPPORTED
+    # window 128 with 8 query tokens: the union spans 135 keys
+    st, h, ws = _plan(lib, _desc(qo_heads=1, kv_heads=1, q_len=8, window=128), [0, 4096])
+    assert st == 0
+    inf = _info(lib, h)
+    T = inf.tile_tokens
+    assert inf.total_tiles == (4096 + T - 1) // T - (4096 - 135) // T
+    lib.fa_plan_destroy(h)
+    for bad in (-1, 65):
+        st, h, ws = _plan(lib, _desc(q_len=bad), [0, 100])
+        assert st == 1  # FA_ERR_INVALID_ARG

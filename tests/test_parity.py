@@ -250,3 +250,54 @@ def test_full_size_batched_paged(paged_workload, path):
 @pytest.mark.parametrize("path", ["mma"])
 def test_full_size_fp8_long_context(path):
     _check_full(synth.workload("fp8_gqa8_L131072"), path=path, nrows=24, seed=2)
+
+
+# ------------------------------------------------------ several query tokens
+MULTI = [
+    # (name, batch, qo, kv, d, lens, kw)
+    ("q2_gqa4_paged", 3, 8, 2, 128, [300, 2, 65], {"q_len": 2, "paged": True, "page_size": 16}),
+    ("q8_mha_d64_win", 2, 4, 4, 64, [500, 9], {"q_len": 8, "window": 100}),
+    ("q4_gqa2_d256", 2, 8, 4, 256, [700, 40], {"q_len": 4}),
+    ("q4_gqa2_fp8_paged", 2, 16, 8, 128, [333, 70], {"q_len": 4, "kv_dtype": "fp8_e4m3",
+                                                     "paged": True, "page_size": 32}),
+    ("q4_short_request", 2, 2, 1, 128, [2, 90], {"q_len": 4}),
+]
+
+
+@pytest.mark.parametrize("case", MULTI, ids=[c[0] for c in MULTI])
+@pytest.mark.parametrize("path", PATHS)
+def test_several_query_tokens(case, path):
+    name, B, Hq, Hk, d, lens, kw = case
+    x = synth.generate(B, Hq, Hk, d, lens, seed=zlib.crc32(name.encode()) & 0xFFFF, name=name, **kw)
+    rows = x.group * x.q_len
+    if path == "simt" and (rows not in (1, 2, 4, 8) or (x.kv_dtype == "fp8_e4m3" and rows > 4)):
+        pytest.skip("no SIMT kernel for this many rows")
+    _check(x, path=path)
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_several_query_tokens_forced_splits_agree(path):
+    x = synth.generate(2, 4, 2, 128, [1500, 203], q_len=4, seed=29, window=700)
+    results = []
+    for n in (1, 7, 64, 0):
+        out, lse, info = _check(x, path=path, num_ctas=n)
+        results.append((out, lse))
+    for o, l in results[1:]:
+        assert np.abs(l - results[0][1]).max() <= 2e-5
+        assert np.abs(o - results[0][0]).max() <= 4e-3
+
+
+def test_several_query_tokens_full_size_batched_paged():
+    """The batch-64 paged workload with two query tokens per request (one
+    draft token being verified), sampled rows against the oracle."""
+    lens = synth.c4_lengths()
+    x = synth.generate(64, 32, 8, 128, lens, paged=True, page_size=16, seed=4, q_len=2,
+                       name="paged_b64_gqa4_q2")
+    out, lse, flags, info = run_gpu(x)
+    assert flags == 0 and info["path"] == binding.PATH_MMA
+    rng = np.random.default_rng(5)
+    rows = np.sort(rng.choice(64 * 2 * 32, 48, replace=False))
+    ro, rl = oracle.decode_rows(x, rows)
+    b, rem = rows // 64, rows % 64
+    i, h = rem // 32, rem % 32
+    assert_matches(out[b, i, h], lse[b, i, h], ro, rl, what="paged b64 q2 sampled")
