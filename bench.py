@@ -48,7 +48,9 @@ METRIC = "decode attention achieved HBM GB/s (% of B200 peak) and tokens/sec at 
 HEADLINE = "paged_b64_gqa4_L512-16384"
 SWEEP = ["gqa4_d64_L512", "gemma3_1b_global_L8192", "gemma3_1b_local_w512_L8192",
          "llama2_7b_mha_L1024", "llama2_7b_mha_L4096", "llama2_7b_mha_L16384",
-         "llama2_7b_mha_L32768", "fp8_gqa8_L131072"]
+         "llama2_7b_mha_L32768", "fp8_gqa8_L131072",
+         # several query tokens per request
+         "paged_b64_gqa4_q2_L512-16384", "llama2_7b_mha_q8_L32768"]
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -171,15 +173,15 @@ class Runner:
             batch=x.batch, qo_heads=x.qo_heads, kv_heads=x.kv_heads, head_dim=x.head_dim,
             kv_dtype=1 if fp8 else 0, paged=int(x.paged), page_size=int(x.page_size),
             window=int(x.window), sm_scale=float(x.sm_scale),
-            path={"auto": 0, "simt": 1, "mma": 2}[path], num_ctas=0)
+            path={"auto": 0, "simt": 1, "mma": 2}[path], num_ctas=0, q_len=int(x.q_len))
         p = binding.plan(x.batch, x.qo_heads, x.kv_heads, x.head_dim, x.kv_indptr,
                          kv_dtype=x.kv_dtype, paged=x.paged, page_size=x.page_size,
-                         window=x.window, sm_scale=x.sm_scale, path=path)
+                         window=x.window, sm_scale=x.sm_scale, path=path, q_len=x.q_len)
         self.info = p.info()
         self.ws = p.new_workspace(device)
-        self.out = torch.empty((x.batch, x.qo_heads, x.head_dim), dtype=torch.bfloat16,
-                               device=device)
-        self.lse = torch.empty((x.batch, x.qo_heads), dtype=torch.float32, device=device)
+        rows = (x.batch, x.qo_heads) if x.q_len == 1 else (x.batch, x.q_len, x.qo_heads)
+        self.out = torch.empty(rows + (x.head_dim,), dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty(rows, dtype=torch.float32, device=device)
         ptr = lambda t: None if t is None else t.data_ptr()
         self.stream = torch.cuda.current_stream()
         self.args = (ptr(self.q), ptr(self.k), ptr(self.v), int(self.k.shape[0]), ptr(self.pt),
@@ -308,7 +310,8 @@ def oracle_sample(x, budget_s, max_requests=None):
     vis = x.visible_lens()
     per_tok = x.kv_heads * x.head_dim * x.elem_bytes * 2
     for b in order:
-        rows = np.arange(b * x.qo_heads, (b + 1) * x.qo_heads)
+        per = x.q_len * x.qo_heads  # rows of one request
+        rows = np.arange(b * per, (b + 1) * per)
         t0 = time.perf_counter()
         oracle.decode_rows(x, rows, nthreads=threads)
         t_total += time.perf_counter() - t0
@@ -365,6 +368,7 @@ def workload_config(x, world):
     return {"workload": x.name, "batch": x.batch, "qo_heads": x.qo_heads,
             "kv_heads": x.kv_heads, "head_dim": x.head_dim, "kv_dtype": x.kv_dtype,
             "paged": bool(x.paged), "page_size": x.page_size, "window": x.window,
+            "q_len": x.q_len,
             "kv_len_min": int(lens.min()), "kv_len_max": int(lens.max()),
             "kv_tokens": int(lens.sum()), "kv_bytes_per_step_per_gpu": x.kv_bytes(),
             "l2": "inputs larger than L2 (no flush)" if x.kv_bytes() > 256e6
@@ -432,7 +436,7 @@ def main():
     clocks = sampler.stop()
     ms_total = max_over_ranks(ms_total, world, "cuda")
     kv_bytes = x.kv_bytes()
-    agg = aggregate(kv_bytes, x.batch, ms_total, args.steps, world)
+    agg = aggregate(kv_bytes, x.batch * x.q_len, ms_total, args.steps, world)  # query tokens
     ms_step, value, tokens = agg["ms_per_step"], agg["value"], agg["tokens_per_s"]
 
     # dominant kernel: its average duration in the timed region (CUDA events on
@@ -455,7 +459,7 @@ def main():
         e2e = {"value": round(world * kv_bytes / (ms_e2e * 1e-3) / 1e9, 3), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(ms_e2e, 3), "steps": args.e2e_steps,
-               "tokens_per_s": round(world * x.batch / (ms_e2e * 1e-3), 1)}
+               "tokens_per_s": round(world * x.batch * x.q_len / (ms_e2e * 1e-3), 1)}
 
     sweep = None
     if rank == 0 and world == 1 and not args.no_sweep:
@@ -486,7 +490,7 @@ def main():
                               "back_to_back_us": None if loop_us is None else round(loop_us, 2),
                               "back_to_back_frac": None if loop_us is None else
                               round(y.kv_bytes() / (loop_us * 1e-6) / 1e9 / peak, 4),
-                              "tokens_per_s": round(y.batch / (med * 1e-3), 1),
+                              "tokens_per_s": round(y.batch * y.q_len / (med * 1e-3), 1),
                               "path": "mma" if r.info["path"] == 2 else "simt",
                               "ctas": r.info["num_ctas"], "kv_bytes": y.kv_bytes()}
                 del r

@@ -255,6 +255,19 @@ def _c4_small():
                     name="paged_b16_gqa4_L512-16384")
 
 
+def _c4_q2():
+    """The batch-64 paged workload with two query tokens per request (a draft
+    token verified next to the regular decode token)."""
+    return generate(64, 32, 8, 128, c4_lengths(), paged=True, page_size=16, seed=4, q_len=2,
+                    name="paged_b64_gqa4_q2_L512-16384")
+
+
+def _c3_q8():
+    """Llama-2-7B-shaped MHA layer at 32k keys with eight query tokens per
+    request (seven draft tokens)."""
+    return generate(1, 32, 32, 128, [32768], seed=3, q_len=8, name="llama2_7b_mha_q8_L32768")
+
+
 def _c5():
     return generate(1, 64, 8, 128, [131072], kv_dtype="fp8_e4m3", seed=5,
                     name="fp8_gqa8_L131072")
@@ -271,6 +284,8 @@ WORKLOADS = {
     "paged_b64_gqa4_L512-16384": _c4,
     "paged_b16_gqa4_L512-16384": _c4_small,
     "fp8_gqa8_L131072": _c5,
+    "paged_b64_gqa4_q2_L512-16384": _c4_q2,
+    "llama2_7b_mha_q8_L32768": _c3_q8,
 }
 
 
