@@ -92,6 +92,7 @@ class DecodeInputs:
     k_scale: Optional[np.ndarray] = None     # float32 [kv_heads]
     v_scale: Optional[np.ndarray] = None
     q_len: int = 1         # query tokens per request: the request's newest keys
+    logit_cap: float = 0.0  # > 0: scores s become cap * tanh(s / cap)
 
     @property
     def group(self) -> int:
@@ -136,7 +137,7 @@ def generate(batch: int, qo_heads: int, kv_heads: int, head_dim: int,
              page_size: int = 16, window: int = -1, sm_scale: Optional[float] = None,
              seed: int = 0, name: str = "custom", page_order: str = "random",
              unused_slot_fill: Optional[str] = None, extra_rows: int = 0,
-             q_len: int = 1) -> DecodeInputs:
+             q_len: int = 1, logit_cap: float = 0.0) -> DecodeInputs:
     """Draw one decode problem.
 
     kv_lens: per-request key counts.  paged: pool of sum(ceil(L/page_size))
@@ -217,7 +218,8 @@ def generate(batch: int, qo_heads: int, kv_heads: int, head_dim: int,
                         page_size=page_size if paged else 0, window=window,
                         sm_scale=float(sm_scale), q=q, k=k, v=v,
                         kv_indptr=indptr.astype(np.int32), page_table=page_table,
-                        k_scale=k_scale, v_scale=v_scale, q_len=q_len)
+                        k_scale=k_scale, v_scale=v_scale, q_len=q_len,
+                        logit_cap=float(logit_cap))
 
 
 def c4_lengths(seed: int = 4, batch: int = 64, lo: int = 512, hi: int = 16384) -> np.ndarray:

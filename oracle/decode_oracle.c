@@ -37,6 +37,11 @@
  * tokens, and token i (position L - q_len + i) sees keys [0, L - q_len + i],
  * the causal mask of "Standard causal attention" restricted to the new rows.
  *
+ * Logit soft-capping (named on "FlashInfer x JAX via jax-tvm-ffi", section
+ * "Applying it to Gemma 3", as Gemma 2's, and on "Flashlight", section
+ * "Results", as the Softcap variant; neither gives the formula): each
+ * scaled score s becomes cap * tanh(s / cap), Gemma 2's published form.
+ *
  * Readings where the pages are silent (each also listed in the design notes):
  *  - GQA grouping: query head h reads kv head h / (qo_heads / kv_heads).
  *  - window w > 0 keeps exactly the last w keys [L - w, L); w <= 0 keeps all.
@@ -73,6 +78,8 @@ typedef struct {
     const int32_t *page_table; /* [batch, page_table_stride], paged only      */
     int32_t q_len;           /* query tokens per request (0 means 1); q is
                                 [batch, q_len, qo_heads, head_dim]            */
+    double logit_cap;        /* > 0: each scaled score s becomes
+                                cap * tanh(s / cap) before the softmax       */
 } oracle_problem;
 
 /* bf16 is the upper half of an IEEE binary32; widening is exact. */
@@ -165,6 +172,7 @@ static int decode_one(const oracle_problem *p, int b, int qi, int h, double *s,
             acc += oracle_bf16_to_double(qrow[i]) *
                    kv_element(p, p->k, p->k_scale, b, lo + j, g, i);
         s[j] = p->sm_scale * acc;
+        if (p->logit_cap > 0.0) s[j] = p->logit_cap * tanh(s[j] / p->logit_cap);
     }
     /* stable softmax: max, then normaliser */
     double M = -INFINITY;

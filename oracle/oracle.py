@@ -48,7 +48,7 @@ class _Problem(ctypes.Structure):
         ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
         ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
         ("kv_indptr", ctypes.c_void_p), ("page_table", ctypes.c_void_p),
-        ("q_len", ctypes.c_int32),
+        ("q_len", ctypes.c_int32), ("logit_cap", ctypes.c_double),
     ]
 
 
@@ -103,7 +103,8 @@ def _problem(x) -> Tuple[_Problem, list]:
                  page_table_stride=int(pt.shape[1]) if pt is not None else 0,
                  window=int(x.window), sm_scale=float(x.sm_scale),
                  q=_ptr(q), k=_ptr(k), v=_ptr(v), k_scale=_ptr(ks), v_scale=_ptr(vs),
-                 kv_indptr=_ptr(ind), page_table=_ptr(pt), q_len=_q_len(x))
+                 kv_indptr=_ptr(ind), page_table=_ptr(pt), q_len=_q_len(x),
+                 logit_cap=float(getattr(x, "logit_cap", 0.0) or 0.0))
     return p, keep
 
 

@@ -444,3 +444,45 @@ def test_multi_token_shorter_request_than_query_block():
     out, lse = oracle.decode_all(x)
     assert np.isneginf(lse[0, :2]).all() and (out[0, :2] == 0).all()
     assert np.isfinite(lse[0, 2:]).all()
+
+
+# ------------------------------------------------------------ logit soft-cap
+# Each scaled score s becomes cap * tanh(s / cap) before the softmax (Gemma
+# 2's soft-capping; the pages name the variant without the formula).
+
+def test_softcap_two_keys_closed_form():
+    """Two keys with scaled scores a, b: weights follow the capped scores."""
+    a_, b_, cap = 3.0, -1.5, 2.0
+    q = [[[1.0, 0.0]]]
+    k = [[[a_, 0.0]], [[b_, 0.0]]]
+    v = [[[1.0, 2.0]], [[-3.0, 0.5]]]
+    x = contiguous_inputs(q, k, v, [2], sm_scale=1.0)
+    x = DecodeInputs(**{**x.__dict__, "logit_cap": cap})
+    out, lse = oracle.decode_all(x)
+    ca, cb = cap * math.tanh(a_ / cap), cap * math.tanh(b_ / cap)
+    wa = math.exp(ca) / (math.exp(ca) + math.exp(cb))
+    np.testing.assert_allclose(out[0, 0], [wa * 1.0 + (1 - wa) * -3.0, wa * 2.0 + (1 - wa) * 0.5],
+                               rtol=0, atol=1e-14)
+    assert abs(lse[0, 0] - math.log(math.exp(ca) + math.exp(cb))) < 1e-14
+
+
+def test_softcap_limits_and_brute_force():
+    x = synth.generate(2, 4, 2, 16, [40, 7], seed=44, sm_scale=0.9)
+    plain_out, plain_lse = oracle.decode_all(x)
+    # a cap far above every score changes nothing (tanh(s/c)*c = s - s^3/(3c^2) ...)
+    big = DecodeInputs(**{**x.__dict__, "logit_cap": 1e7})
+    o, l = oracle.decode_all(big)
+    np.testing.assert_allclose(o, plain_out, rtol=0, atol=1e-10)
+    np.testing.assert_allclose(l, plain_lse, rtol=0, atol=1e-10)
+    # a small cap: numpy restatement of the capped softmax
+    cap = 1.5
+    y = DecodeInputs(**{**x.__dict__, "logit_cap": cap})
+    o, l = oracle.decode_all(y)
+    qf = bf16_values(x.q)
+    for b in range(2):
+        kf, vf = dense_kv(x, b)
+        for h in range(4):
+            s = cap * np.tanh(x.sm_scale * (kf[:, h // 2] @ qf[b, h]) / cap)
+            w = np.exp(s - s.max())
+            np.testing.assert_allclose(o[b, h], (w / w.sum()) @ vf[:, h // 2], rtol=0, atol=1e-12)
+            assert abs(l[b, h] - (s.max() + math.log(w.sum()))) < 1e-12
