@@ -50,7 +50,9 @@ SWEEP = ["gqa4_d64_L512", "gemma3_1b_global_L8192", "gemma3_1b_local_w512_L8192"
          "llama2_7b_mha_L1024", "llama2_7b_mha_L4096", "llama2_7b_mha_L16384",
          "llama2_7b_mha_L32768", "fp8_gqa8_L131072",
          # several query tokens per request
-         "paged_b64_gqa4_q2_L512-16384", "llama2_7b_mha_q8_L32768"]
+         "paged_b64_gqa4_q2_L512-16384", "llama2_7b_mha_q8_L32768",
+         # logit soft-capping
+         "gemma2_2b_softcap50_L8192"]
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -173,10 +175,12 @@ class Runner:
             batch=x.batch, qo_heads=x.qo_heads, kv_heads=x.kv_heads, head_dim=x.head_dim,
             kv_dtype=1 if fp8 else 0, paged=int(x.paged), page_size=int(x.page_size),
             window=int(x.window), sm_scale=float(x.sm_scale),
-            path={"auto": 0, "simt": 1, "mma": 2}[path], num_ctas=0, q_len=int(x.q_len))
+            path={"auto": 0, "simt": 1, "mma": 2}[path], num_ctas=0, q_len=int(x.q_len),
+            logit_cap=float(x.logit_cap))
         p = binding.plan(x.batch, x.qo_heads, x.kv_heads, x.head_dim, x.kv_indptr,
                          kv_dtype=x.kv_dtype, paged=x.paged, page_size=x.page_size,
-                         window=x.window, sm_scale=x.sm_scale, path=path, q_len=x.q_len)
+                         window=x.window, sm_scale=x.sm_scale, path=path, q_len=x.q_len,
+                         logit_cap=x.logit_cap)
         self.info = p.info()
         self.ws = p.new_workspace(device)
         rows = (x.batch, x.qo_heads) if x.q_len == 1 else (x.batch, x.q_len, x.qo_heads)
@@ -368,7 +372,7 @@ def workload_config(x, world):
     return {"workload": x.name, "batch": x.batch, "qo_heads": x.qo_heads,
             "kv_heads": x.kv_heads, "head_dim": x.head_dim, "kv_dtype": x.kv_dtype,
             "paged": bool(x.paged), "page_size": x.page_size, "window": x.window,
-            "q_len": x.q_len,
+            "q_len": x.q_len, "logit_cap": x.logit_cap,
             "kv_len_min": int(lens.min()), "kv_len_max": int(lens.max()),
             "kv_tokens": int(lens.sum()), "kv_bytes_per_step_per_gpu": x.kv_bytes(),
             "l2": "inputs larger than L2 (no flush)" if x.kv_bytes() > 256e6

@@ -41,7 +41,8 @@ class DecodeDesc(ctypes.Structure):
                 ("kv_dtype", ctypes.c_int32), ("paged", ctypes.c_int32),
                 ("page_size", ctypes.c_int32), ("window", ctypes.c_int32),
                 ("sm_scale", ctypes.c_float), ("path", ctypes.c_int32),
-                ("num_ctas", ctypes.c_int32), ("q_len", ctypes.c_int32)]
+                ("num_ctas", ctypes.c_int32), ("q_len", ctypes.c_int32),
+                ("logit_cap", ctypes.c_float)]
 
 
 class PlanInfo(ctypes.Structure):
@@ -149,7 +150,7 @@ class DecodePlan:
 def plan(batch: int, qo_heads: int, kv_heads: int, head_dim: int, kv_indptr_host, *,
          kv_dtype: str = "bf16", paged: bool = False, page_size: int = 0, window: int = -1,
          sm_scale: Optional[float] = None, path: str = "auto", num_ctas: int = 0,
-         num_sms: int = 0, q_len: int = 1) -> DecodePlan:
+         num_sms: int = 0, q_len: int = 1, logit_cap: float = 0.0) -> DecodePlan:
     lib = load_library()
     ind = np.ascontiguousarray(np.asarray(
         kv_indptr_host.cpu().numpy() if hasattr(kv_indptr_host, "cpu") else kv_indptr_host,
@@ -160,7 +161,7 @@ def plan(batch: int, qo_heads: int, kv_heads: int, head_dim: int, kv_indptr_host
                       kv_dtype=KV_FP8_E4M3 if kv_dtype == "fp8_e4m3" else KV_BF16,
                       paged=int(bool(paged)), page_size=int(page_size), window=int(window),
                       sm_scale=float(sm_scale), path=_PATH_NAMES[path], num_ctas=int(num_ctas),
-                      q_len=int(q_len))
+                      q_len=int(q_len), logit_cap=float(logit_cap))
     handle = ctypes.c_void_p()
     ws = ctypes.c_size_t()
     _check(lib.fa_decode_plan(ctypes.byref(desc), ind.ctypes.data, int(num_sms),

@@ -104,6 +104,7 @@ struct KernelArgs {
   int paged, page_shift, pt_stride, box_t, swz;
   int seg_parts;      // 0: equal runs of all tiles; k > 0: k runs per segment
   float score_scale;  // sm_scale * log2(e)
+  float cap_l2;       // > 0: logit soft-cap in log2 units (cap * log2(e)); 0: none
 };
 
 constexpr int kSmemPerBlock = 232448;  // 227 KB of shared memory per block (sm_100)
@@ -445,8 +446,11 @@ struct SimtConsumer {
         const int pos = pos0 + r;
         const bool valid = pos >= lo && pos < hi;
 #pragma unroll
-        for (int h = 0; h < G; ++h)
-          s[tt][h] = (multi ? row_sees(a, h, pos, hi) : valid) ? part[h] : -CUDART_INF_F;
+        for (int h = 0; h < G; ++h) {
+          float x = part[h];
+          if (a.cap_l2 > 0.f) x = a.cap_l2 * tanhf(x / a.cap_l2);  // soft-cap, log2 units
+          s[tt][h] = (multi ? row_sees(a, h, pos, hi) : valid) ? x : -CUDART_INF_F;
+        }
       }
       // running max with slack: rescale only when the max grows by more than kRescaleSlack
       bool need = false;
@@ -752,6 +756,10 @@ struct MmaConsumer {
       sc[sub][1] = v01 ? sc[sub][1] * sscale[1] : -CUDART_INF_F;
       sc[sub][2] = v80 ? sc[sub][2] * sscale[0] : -CUDART_INF_F;
       sc[sub][3] = v81 ? sc[sub][3] * sscale[1] : -CUDART_INF_F;
+      if (a.cap_l2 > 0.f) {  // soft-cap: c tanh(s / c) (log2 units; -inf stays -inf)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[sub][e] = a.cap_l2 * tanhf(sc[sub][e] / a.cap_l2);
+      }
       mx0 = fmaxf(mx0, fmaxf(sc[sub][0], sc[sub][2]));
       mx1 = fmaxf(mx1, fmaxf(sc[sub][1], sc[sub][3]));
     }

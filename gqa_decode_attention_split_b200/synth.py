@@ -270,6 +270,13 @@ def _c3_q8():
     return generate(1, 32, 32, 128, [32768], seed=3, q_len=8, name="llama2_7b_mha_q8_L32768")
 
 
+def _gemma2_softcap():
+    """A Gemma-2-2B-shaped global layer (8 query / 4 kv heads, head_dim 256,
+    scores scaled by 1/16) with its logit soft-cap of 50."""
+    return generate(1, 8, 4, 256, [8192], seed=6, sm_scale=1.0 / 16.0, logit_cap=50.0,
+                    name="gemma2_2b_softcap50_L8192")
+
+
 def _c5():
     return generate(1, 64, 8, 128, [131072], kv_dtype="fp8_e4m3", seed=5,
                     name="fp8_gqa8_L131072")
@@ -288,6 +295,7 @@ WORKLOADS = {
     "fp8_gqa8_L131072": _c5,
     "paged_b64_gqa4_q2_L512-16384": _c4_q2,
     "llama2_7b_mha_q8_L32768": _c3_q8,
+    "gemma2_2b_softcap50_L8192": _gemma2_softcap,
 }
 
 

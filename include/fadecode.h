@@ -102,6 +102,11 @@ typedef struct {
                       /* L - q_len + i) sees the keys up to and including    */
                       /* itself, or the last `window` of them.  Needs        */
                       /* (qo_heads / kv_heads) * q_len <= 8.                 */
+  float logit_cap;    /* 0: none.  c > 0: logit soft-capping, each scaled    */
+                      /* score s becomes c * tanh(s / c) before the softmax  */
+                      /* (Gemma 2's soft-cap, named on "FlashInfer x JAX via */
+                      /* jax-tvm-ffi", section "Applying it to Gemma 3").    */
+                      /* Must be finite and >= 0.                            */
 } fa_decode_desc;
 
 typedef struct fa_plan fa_plan;
@@ -140,7 +145,7 @@ typedef struct {
  *  workspace_bytes receives the minimum workspace size.
  * Errors: FA_ERR_INVALID_ARG (null pointer, non-positive shape, qo_heads not
  * a multiple of kv_heads, bad indptr, non-finite sm_scale, bad page_size,
- * q_len < 0 or > 64), FA_ERR_UNSUPPORTED (head_dim / group * q_len / dtype /
+ * q_len < 0 or > 64, negative or non-finite logit_cap), FA_ERR_UNSUPPORTED (head_dim / group * q_len / dtype /
  * path combination without a kernel), FA_ERR_CUDA (num_sms == 0 and no
  * device could be queried).
  */

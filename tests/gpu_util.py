@@ -38,7 +38,7 @@ class DeviceInputs:
         return binding.plan(x.batch, x.qo_heads, x.kv_heads, x.head_dim, x.kv_indptr,
                             kv_dtype=x.kv_dtype, paged=x.paged, page_size=x.page_size,
                             window=x.window, sm_scale=x.sm_scale, path=path, num_ctas=num_ctas,
-                            q_len=getattr(x, "q_len", 1))
+                            q_len=getattr(x, "q_len", 1), logit_cap=getattr(x, "logit_cap", 0.0))
 
     def run(self, p, workspace=None, out=None, lse=None, want_lse=True):
         return binding.run(p, self.q, self.k, self.v, self.kv_indptr, page_table=self.page_table,

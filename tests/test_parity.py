@@ -301,3 +301,35 @@ def test_several_query_tokens_full_size_batched_paged():
     b, rem = rows // 64, rows % 64
     i, h = rem // 32, rem % 32
     assert_matches(out[b, i, h], lse[b, i, h], ro, rl, what="paged b64 q2 sampled")
+
+
+# ------------------------------------------------------------ logit soft-cap
+CAPPED = [
+    # (name, batch, qo, kv, d, lens, kw); sm_scale raised so the cap bends the scores
+    ("cap20_gqa4", 2, 8, 2, 128, [700, 33], {"logit_cap": 20.0, "sm_scale": 0.5}),
+    ("cap50_d256", 1, 8, 4, 256, [3000], {"logit_cap": 50.0, "sm_scale": 0.25}),
+    ("cap10_fp8_paged_q2", 2, 8, 4, 128, [500, 77], {"logit_cap": 10.0, "sm_scale": 0.4,
+                                                     "kv_dtype": "fp8_e4m3", "paged": True,
+                                                     "page_size": 16, "q_len": 2}),
+]
+
+
+@pytest.mark.parametrize("case", CAPPED, ids=[c[0] for c in CAPPED])
+@pytest.mark.parametrize("path", PATHS)
+def test_logit_softcap(case, path):
+    name, B, Hq, Hk, d, lens, kw = case
+    x = synth.generate(B, Hq, Hk, d, lens, seed=zlib.crc32(name.encode()) & 0xFFFF, name=name, **kw)
+    rows = x.group * x.q_len
+    if path == "simt" and (rows not in (1, 2, 4, 8) or (x.kv_dtype == "fp8_e4m3" and rows > 4)):
+        pytest.skip("no SIMT kernel for this many rows")
+    out, lse, _ = _check(x, path=path)
+    # the cap must matter here: the uncapped result is different
+    plain = synth.DecodeInputs(**{**x.__dict__, "logit_cap": 0.0})
+    po, pl = oracle.decode_all(plain)
+    assert np.abs(pl - lse).max() > 0.1
+
+
+def test_logit_softcap_forced_splits():
+    x = synth.generate(1, 8, 2, 128, [2500], seed=30, logit_cap=15.0, sm_scale=0.5)
+    for n in (1, 9, 0):
+        _check(x, path="mma", num_ctas=n)
