@@ -443,13 +443,33 @@ struct SimtConsumer {
         for (int off = 1; off < LPT; off <<= 1)
 #pragma unroll
           for (int h = 0; h < G; ++h) part[h] += __shfl_xor_sync(0xffffffffu, part[h], off);
-        const int pos = pos0 + r;
-        const bool valid = pos >= lo && pos < hi;
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float x = part[h];
-          if (a.cap_l2 > 0.f) x = a.cap_l2 * tanhf(x / a.cap_l2);  // soft-cap, log2 units
-          s[tt][h] = (multi ? row_sees(a, h, pos, hi) : valid) ? x : -CUDART_INF_F;
+        for (int h = 0; h < G; ++h) s[tt][h] = part[h];
+      }
+      // soft-cap and masking once per sub-step, behind uniform branches, so
+      // the score products above schedule as one straight block
+      if (a.cap_l2 > 0.f) {  // c tanh(s / c), log2 units
+#pragma unroll
+        for (int tt = 0; tt < TPSC; ++tt)
+#pragma unroll
+          for (int h = 0; h < G; ++h) s[tt][h] = a.cap_l2 * tanhf(s[tt][h] / a.cap_l2);
+      }
+      if (multi) {
+#pragma unroll
+        for (int tt = 0; tt < TPSC; ++tt) {
+          const int pos = pos0 + (si * TPSC + tt) * SLOTS + slot;
+#pragma unroll
+          for (int h = 0; h < G; ++h)
+            if (!row_sees(a, h, pos, hi)) s[tt][h] = -CUDART_INF_F;
+        }
+      } else {
+#pragma unroll
+        for (int tt = 0; tt < TPSC; ++tt) {
+          const int pos = pos0 + (si * TPSC + tt) * SLOTS + slot;
+          if (pos < lo || pos >= hi) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) s[tt][h] = -CUDART_INF_F;
+          }
         }
       }
       // running max with slack: rescale only when the max grows by more than kRescaleSlack
