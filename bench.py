@@ -50,7 +50,10 @@ SWEEP = ["gqa4_d64_L512", "gemma3_1b_global_L8192", "gemma3_1b_local_w512_L8192"
          "llama2_7b_mha_L1024", "llama2_7b_mha_L4096", "llama2_7b_mha_L16384",
          "llama2_7b_mha_L32768", "fp8_gqa8_L131072",
          # several query tokens per request
-         "paged_b64_gqa4_q2_L512-16384", "llama2_7b_mha_q8_L32768",
+         "paged_b64_gqa4_q2_L512-16384", "paged_b64_gqa4_q4_L512-16384",
+         "paged_b64_gqa4_q8_L512-16384", "llama2_7b_mha_q8_L32768",
+         # query groups wider than 8 (row teams)
+         "llama3_405b_tp8_gqa16_paged_b64_L512-16384",
          # logit soft-capping
          "gemma2_2b_softcap50_L8192"]
 FALLBACK_HBM_GBS = 6650.0

@@ -75,14 +75,20 @@ int register_bf16_and_fp8(KernelEntry* out, int cap, bool with_fp8) {
   auto add = [&](const KernelEntry& e) {
     if (n < cap) out[n++] = e;
   };
-  add(make_entry<MmaConsumer<D, false>>(kPathMma, 0, 8, 0));
+  // tensor-core variants in order of rows (the planner takes the first that
+  // holds a segment's rows): one, two and four row teams of 8
+  add(make_entry<MmaConsumer<D, false, 1>>(kPathMma, 0, 8, 0));
+  add(make_entry<MmaConsumer<D, false, 2>>(kPathMma, 0, 16, 0));
+  add(make_entry<MmaConsumer<D, false, 4>>(kPathMma, 0, 32, 0));
   add(make_entry<SimtConsumer<D, 1, false>>(kPathSimt, 1, 1, 0));
   add(make_entry<SimtConsumer<D, 2, false>>(kPathSimt, 2, 2, 0));
   add(make_entry<SimtConsumer<D, 4, false>>(kPathSimt, 4, 4, 0));
   add(make_entry<SimtConsumer<D, 8, false>>(kPathSimt, 8, 8, 0));
   if constexpr (D >= 128) {
     if (with_fp8) {
-      add(make_entry<MmaConsumer<D, true>>(kPathMma, 0, 8, 1));
+      add(make_entry<MmaConsumer<D, true, 1>>(kPathMma, 0, 8, 1));
+      add(make_entry<MmaConsumer<D, true, 2>>(kPathMma, 0, 16, 1));
+      add(make_entry<MmaConsumer<D, true, 4>>(kPathMma, 0, 32, 1));
       add(make_entry<SimtConsumer<D, 1, true>>(kPathSimt, 1, 1, 1));
       add(make_entry<SimtConsumer<D, 2, true>>(kPathSimt, 2, 2, 1));
       add(make_entry<SimtConsumer<D, 4, true>>(kPathSimt, 4, 4, 1));

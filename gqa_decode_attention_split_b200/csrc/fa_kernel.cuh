@@ -120,17 +120,20 @@ constexpr int kScaleCap = 128;         // fp8 per-kv-head scales kept in shared 
 // layout is plane-major, [NP][T][CB], one copy per plane.
 // A tile holds TILE_BYTES_TARGET / row bytes tokens (16 to 128).  K and V
 // tiles live in two rings that take what is left of the block's shared
-// memory after the merge area for GMAX query heads: KSTAGES K slots and
-// VSTAGES V slots, each a multiple of the consumer-warp count.  Tile i uses K
-// slot i % KSTAGES, V slot i % VSTAGES and warp i % NW, so every slot belongs
-// to exactly one warp, which waits on it round after round.  (A slot shared
-// by two warps would let one warp wait for round r+1 while round r is still
-// pending; an mbarrier parity wait cannot tell the two apart and would pass
-// early.)  A consumer that frees its K slot as soon as the scores are taken
-// (EARLY_K) holds V longer than K, so the V ring gets the extra slots: a
-// slot is refilled only after its warp releases it, and a slot held through
-// the tile's math is a slot with no copy in flight.
-template <int D, bool FP8, int GMAX, int TILE_BYTES_TARGET, int NWARPS, bool EARLY_K>
+// memory after the merge area: KSTAGES K slots and VSTAGES V slots.  The NW
+// consumer warps form R row teams of NT = NW / R warps: a tile is consumed
+// by one warp of every team (warp u of each team takes tiles i with
+// i % NT == u, the team's own GW query rows of the segment), so a tile
+// carries up to GW * R rows.  Both slot counts are multiples of NT and tile
+// i uses K slot i % KSTAGES and V slot i % VSTAGES: every slot belongs to
+// exactly one tile lane u, whose R warps wait on it round after round.  (A
+// slot shared by two tile lanes would let one wait for round r+1 while round
+// r is still pending; an mbarrier parity wait cannot tell the two apart and
+// would pass early.)  A consumer that frees its K slot as soon as the scores
+// are taken (EARLY_K) holds V longer than K, so the V ring gets the extra
+// slots: a slot is refilled only after its warps release it, and a slot
+// held through the tile's math is a slot with no copy in flight.
+template <int D, bool FP8, int GW, int R, int TILE_BYTES_TARGET, int NWARPS, bool EARLY_K>
 struct TileCfg {
   static constexpr int ES = FP8 ? 1 : 2;
   static constexpr int ROWB = D * ES;
@@ -140,7 +143,12 @@ struct TileCfg {
   static constexpr int T = T_RAW < 16 ? 16 : (T_RAW > 128 ? 128 : T_RAW);
   static constexpr int TILE_BYTES = T * ROWB;
   static constexpr int NW = NWARPS;
-  static constexpr int MERGE_BYTES = NW * GMAX * (D + 2) * 4;
+  static constexpr int TEAMS = R;       // row teams
+  static constexpr int NT = NW / R;     // tile lanes (warps per team)
+  static_assert(NW % R == 0, "every row team has the same warps");
+  static constexpr int GMAX = GW * R;   // rows of a segment
+  // merge area: one (m, l, acc[D]) state per tile lane and row
+  static constexpr int MERGE_BYTES = NT * GMAX * (D + 2) * 4;
   // q area: four mbarriers, then (STAGE_Q) two slots of a piece's GMAX query
   // rows (bf16) that the producer stages, then (fp8) the k / v scale tables.
   // Query rows are staged only where the slots cost no ring stage; otherwise
@@ -149,21 +157,21 @@ struct TileCfg {
   static constexpr int SCALE_BYTES = FP8 ? 2 * kScaleCap * 4 : 0;
   // (1024: base alignment; 272: merge counter, merge mbarrier, 64 page ids)
   static constexpr int BASE_BUDGET = kSmemPerBlock - 1024 - kSchedReserve - 272 - MERGE_BYTES - 32 - SCALE_BYTES;
-  // K + V tiles per consumer warp that fit (a tile slot costs its bytes
-  // plus two 8-byte mbarriers)
+  // K + V tiles per tile lane that fit (a tile slot costs its bytes plus two
+  // 8-byte mbarriers)
+  static constexpr int kLaneCap = 2 * FA_MAX_STAGES_PER_WARP * R;
   static constexpr int tiles_per_warp(int budget) {
-    return budget / (TILE_BYTES + 16) / NW > 2 * FA_MAX_STAGES_PER_WARP ? 2 * FA_MAX_STAGES_PER_WARP
-                                                                       : budget / (TILE_BYTES + 16) / NW;
+    return budget / (TILE_BYTES + 16) / NT > kLaneCap ? kLaneCap : budget / (TILE_BYTES + 16) / NT;
   }
   static constexpr bool STAGE_Q = tiles_per_warp(BASE_BUDGET - 2 * QSLOT_BYTES) == tiles_per_warp(BASE_BUDGET);
   static constexpr int QAREA_BYTES = 32 + (STAGE_Q ? 2 * QSLOT_BYTES : 0) + SCALE_BYTES;
   static constexpr int RING_BUDGET = BASE_BUDGET + 32 + SCALE_BYTES - QAREA_BYTES;
   static constexpr int TPW = tiles_per_warp(RING_BUDGET);
   static constexpr int KPW = EARLY_K ? (TPW / 3 > 1 ? TPW / 3 : 1) : TPW / 2;
-  static constexpr int VPW = TPW - KPW;
-  static_assert(KPW >= 1 && VPW >= 1, "every consumer warp needs a K and a V slot");
-  static constexpr int KSTAGES = NW * KPW;
-  static constexpr int VSTAGES = NW * VPW;
+  static constexpr int VPW = EARLY_K ? TPW - KPW : KPW;
+  static_assert(KPW >= 1 && VPW >= 1, "every tile lane needs a K and a V slot");
+  static constexpr int KSTAGES = NT * KPW;
+  static constexpr int VSTAGES = NT * VPW;
   static constexpr int RING_BYTES = (KSTAGES + VSTAGES) * TILE_BYTES;
   static constexpr int THREADS = (NW + 1) * 32;
   static constexpr bool TOKEN_MAJOR = FA_PLANE_COPIES == 0;
@@ -318,7 +326,7 @@ __device__ __forceinline__ bool next_piece(PieceIter& it, Piece& pc, const int* 
 // running softmax state, merged across slots at the end of a segment piece.
 template <int D, int G, bool FP8>
 struct SimtConsumer {
-  using C = TileCfg<D, FP8, G, FA_SIMT_TILE_BYTES, FA_SIMT_CONSUMER_WARPS, false>;
+  using C = TileCfg<D, FP8, G, 1, FA_SIMT_TILE_BYTES, FA_SIMT_CONSUMER_WARPS, false>;
   static constexpr int EPC = 16 / C::ES;
   static constexpr int NCH = C::ROWB / 16;
   static constexpr int E_TARGET = 64 / G;
@@ -373,7 +381,7 @@ struct SimtConsumer {
   // head r % group) at qs + (r / group) * qstride + (r % group) * D; kscale:
   // the fp8 K scale of the piece's kv head (1 for bf16).
   __device__ __forceinline__ void begin_piece(const KernelArgs& a, const uint16_t* qs, int qstride,
-                                              float kscale, int lane) {
+                                              float kscale, int lane, int /*team: one team*/) {
     slot = lane / LPT;
     j = lane % LPT;
     float scale = a.score_scale;
@@ -567,10 +575,24 @@ struct SimtConsumer {
 // 2^-12 of the bf16 value) and the three products are summed in fp32.  e4m3
 // V is widened exactly to f16 for the P.V product.  The q scale is undone on
 // the fp32 scores.
-template <int D, bool FP8>
+// R row teams of 8 query rows each (a segment of up to 8R rows: the query
+// heads of a kv head times the query tokens).  A team's warp computes its 8
+// rows of every tile it takes; with more than one team the bf16 tiles are
+// 32 tokens, so that the fewer tile lanes still keep a deep ring.
+template <int D, bool FP8, int R = 1>
 struct MmaConsumer {
-  using C = TileCfg<D, FP8, 8, FP8 ? FA_FP8_MMA_TILE_BYTES : FA_MMA_TILE_BYTES,
-                    FP8 ? FA_FP8_MMA_CONSUMER_WARPS : FA_MMA_CONSUMER_WARPS, true>;
+  static constexpr int kTileBytes =
+      FP8 ? FA_FP8_MMA_TILE_BYTES : (R == 1 ? FA_MMA_TILE_BYTES : FA_MMA_TILE_BYTES / 2);
+  // Consumer warps: two teams of 3, or four of 2 (a 9-warp block, whose
+  // registers are capped at 168 per thread); fp8 rows of 256 dims need more
+  // registers than that and take four teams of one warp.
+  static constexpr int kWarps = R == 1   ? (FP8 ? FA_FP8_MMA_CONSUMER_WARPS : FA_MMA_CONSUMER_WARPS)
+                                : R == 2 ? 6
+                                         : (FP8 && D >= 256 ? 4 : 8);
+  // V held longer than K (EARLY_K: one K slot per two V slots) pays where
+  // the V half of a tile is the longer one, fp8 with one team; elsewhere
+  // equal rings keep the most tiles in flight.
+  using C = TileCfg<D, FP8, 8, R, kTileBytes, kWarps, FP8 && R == 1>;
   static constexpr int KS = D / 16;     // k-steps of the score product = m-tiles of O^T
   static constexpr int SUB = C::T / 16;  // 16-token subtiles per tile
   static constexpr int BPT = D / 4;      // fp8 K: bytes of a row owned by one lane
@@ -586,18 +608,21 @@ struct MmaConsumer {
   float m[2], l[2];
   float sscale[2];
   int g, t;
+  int rbase;  // first segment row of this warp's team
 
   // qs: the piece's query rows (staged in shared memory, or in global
   // memory where the tile geometry leaves no room): row r (token r / group,
   // head r % group) at qs + (r / group) * qstride + (r % group) * D; kscale:
-  // the fp8 K scale of the piece's kv head (1 for bf16).
+  // the fp8 K scale of the piece's kv head (1 for bf16); team: this warp's
+  // row team (rows 8 * team .. 8 * team + 7).
   __device__ __forceinline__ void begin_piece(const KernelArgs& a, const uint16_t* qs, int qstride,
-                                              float kscale, int lane) {
+                                              float kscale, int lane, int team) {
     g = lane >> 2;
     t = lane & 3;
+    rbase = 8 * team;
     const int G = a.group * a.q_len;
-    const bool real = g < G;
-    const int r = real ? g : 0;
+    const bool real = rbase + g < G;
+    const int r = real ? rbase + g : 0;
     const uint16_t* qrow = qs + (r / a.group) * qstride + (r % a.group) * D;
     if constexpr (!FP8) {
 #pragma unroll
@@ -760,8 +785,8 @@ struct MmaConsumer {
     // key range of this lane's two columns (rows 2t, 2t + 1: query token
     // row / group sees one key fewer per token before the last, within its
     // own window); [lo, hi) is the union, and padding columns keep it
-    int chi0 = hi - (a.q_len - 1 - (2 * t) / a.group);
-    int chi1 = hi - (a.q_len - 1 - (2 * t + 1) / a.group);
+    int chi0 = hi - (a.q_len - 1 - (rbase + 2 * t) / a.group);
+    int chi1 = hi - (a.q_len - 1 - (rbase + 2 * t + 1) / a.group);
     chi0 = chi0 < hi ? chi0 : hi;
     chi1 = chi1 < hi ? chi1 : hi;
     const int clo0 = (a.window > 0 && chi0 > a.window) ? chi0 - a.window : 0;
@@ -908,6 +933,7 @@ struct MmaConsumer {
       return mt * 16 + g + 8 * half;
   }
 
+  // Park this warp's state for its team's rows as tile lane w's state.
   __device__ __forceinline__ void end_piece(float* m_area, float* l_area, float* acc_area, int w,
                                             int lane, int G) {
     float l0 = l[0], l1 = l[1];
@@ -916,7 +942,7 @@ struct MmaConsumer {
       l0 += __shfl_xor_sync(0xffffffffu, l0, off);
       l1 += __shfl_xor_sync(0xffffffffu, l1, off);
     }
-    const int h0 = 2 * t, h1 = 2 * t + 1;
+    const int h0 = rbase + 2 * t, h1 = h0 + 1;
     const bool r0 = h0 < G, r1 = h1 < G;
     if (g == 0) {
       if (r0) m_area[w * G + h0] = m[0];
@@ -942,7 +968,7 @@ struct MmaConsumer {
 // Block shared memory, from a 1024-aligned base:
 //   K ring [KSTAGES][tile] | V ring [VSTAGES][tile] |
 //   fullK[KSTAGES], emptyK[KSTAGES], fullV[VSTAGES], emptyV[VSTAGES] mbarriers |
-//   m[NW][G], l[NW][G] | acc[NW][G][D] | merge counter, merge mbarrier |
+//   m[NT][G], l[NT][G] | acc[NT][G][D] | merge counter, merge mbarrier |
 //   pages[64] | q mbarriers, q slots, scales | start[B], len[B], pre[B+1]
 template <class Cons>
 struct SmemLayout {
@@ -951,9 +977,9 @@ struct SmemLayout {
   static constexpr int kBars = C::RING_BYTES;
   static constexpr int kMerge = kBars + 2 * (C::KSTAGES + C::VSTAGES) * 8;
   __host__ __device__ static constexpr int acc_off(int G) {
-    return kMerge + ((C::NW * G * 2 * 4 + 15) / 16) * 16;
+    return kMerge + ((C::NT * G * 2 * 4 + 15) / 16) * 16;
   }
-  __host__ __device__ static constexpr int misc_off(int G) { return acc_off(G) + C::NW * G * D * 4; }
+  __host__ __device__ static constexpr int misc_off(int G) { return acc_off(G) + C::NT * G * D * 4; }
   // misc: merge counter (4 B), pad, merge-free mbarrier (8 B), then 64
   // staged page ids (256 B)
   // q area: qfull[2], qempty[2] mbarriers (32 B) | q slots [2][QSLOT_BYTES]
@@ -965,14 +991,23 @@ struct SmemLayout {
   }
 };
 
+// Registers per thread: each of an SM's four sub-partitions holds 16384, and
+// a block's warps are spread over them, so a block of 9 to 12 warps (3 on
+// some sub-partition) may use at most 168 per thread; up to 8 warps, 224.
 template <class Cons>
-__global__ void __maxnreg__(224)
+__host__ __device__ constexpr int max_regs() {
+  return Cons::C::THREADS > 8 * 32 ? 168 : 224;
+}
+
+template <class Cons>
+__global__ void __maxnreg__(max_regs<Cons>())
     fa_decode_kernel(const __grid_constant__ KernelArgs a) {
   using C = typename Cons::C;
   using S = SmemLayout<Cons>;
   constexpr int D = C::ROWB / C::ES;
   constexpr int T = C::T;
   constexpr int NW = C::NW;
+  constexpr int NT = C::NT;  // tile lanes (NW / row teams)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -994,7 +1029,7 @@ __global__ void __maxnreg__(224)
   const int GK = a.group, Q = a.q_len;
   const int G = GK * Q;
   float* m_area = reinterpret_cast<float*>(base + S::kMerge);
-  float* l_area = m_area + NW * G;
+  float* l_area = m_area + NT * G;
   float* acc_area = reinterpret_cast<float*>(base + S::acc_off(G));
   int* s_mcnt = reinterpret_cast<int*>(base + S::misc_off(G));  // warps done with the open piece
   const uint32_t mfree = sbase + S::misc_off(G) + 8;              // completes when a piece is merged
@@ -1045,13 +1080,14 @@ __global__ void __maxnreg__(224)
     }
   }
   if (tid == 32) {
+    // a slot is free again once every row team's warp has released it
     for (int s = 0; s < C::KSTAGES; ++s) {
       mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, C::TEAMS);
     }
     for (int s = 0; s < C::VSTAGES; ++s) {
       mbar_init(vfull0 + 8 * s, 1);
-      mbar_init(vempty0 + 8 * s, 1);
+      mbar_init(vempty0 + 8 * s, C::TEAMS);
     }
     mbar_init(mfree, 1);
     *s_mcnt = 0;
@@ -1369,13 +1405,16 @@ __global__ void __maxnreg__(224)
   }
 
   // Tile i of the block's sequence lives in K slot i % KSTAGES and V slot
-  // i % VSTAGES and is consumed by warp i % NW (both slot counts are
-  // multiples of NW, so each slot has one owner warp that waits on it in
-  // order); each warp tracks its next tile and that tile's slots.
+  // i % VSTAGES and is consumed by tile lane i % NT, one warp per row team
+  // (both slot counts are multiples of NT, so each slot has one owner lane
+  // whose warps wait on it in order); each warp tracks its next tile and
+  // that tile's slots.
+  const int u = w % NT;     // this warp's tile lane
+  const int team = w / NT;  // and row team
   Cons cons;
-  int next = w;          // next tile index (block sequence) of this warp
-  int kslot = w;         // its K slot (KSTAGES >= NW)
-  int vslot = w;         // its V slot (VSTAGES >= NW)
+  int next = u;          // next tile index (block sequence) of this warp
+  int kslot = u;         // its K slot (KSTAGES >= NT)
+  int vslot = u;         // its V slot (VSTAGES >= NT)
   uint32_t kph = 0;      // wrap parities of those slots
   uint32_t vph = 0;
   int base_i = 0;        // block-sequence index of the current piece's first tile
@@ -1396,16 +1435,16 @@ __global__ void __maxnreg__(224)
         }
       }
       const float ks = C::ES == 1 ? (scales_in_smem ? s_kscale[pc.h] : __ldg(a.k_scale + pc.h)) : 1.f;
-      cons.begin_piece(a, q_slots + qs * (C::QSLOT_BYTES / 2), GK * D, ks, lane);
+      cons.begin_piece(a, q_slots + qs * (C::QSLOT_BYTES / 2), GK * D, ks, lane, team);
       __syncwarp();
       if (lane == 0) mbar_arrive(qempty0 + 8 * qs);
     } else {
       const float ks = C::ES == 1 ? (scales_in_smem ? s_kscale[pc.h] : __ldg(a.k_scale + pc.h)) : 1.f;
       cons.begin_piece(a,
                        a.q + (static_cast<size_t>(pc.b) * Q * a.qo_heads + static_cast<size_t>(pc.h) * GK) * D,
-                       a.qo_heads * D, ks, lane);
+                       a.qo_heads * D, ks, lane, team);
     }
-    for (; next < base_i + n; next += NW) {
+    for (; next < base_i + n; next += NT) {
       // both halves of the tile are waited for up front (a second wait in
       // the middle of the tile's math measured slower than it saves); V
       // first, as its last copy is issued after K's
@@ -1435,12 +1474,12 @@ __global__ void __maxnreg__(224)
         __syncwarp();
         if (lane == 0) mbar_arrive(kSplitKV ? vempty0 + 8 * vslot : kempty);
       }
-      kslot += NW;
+      kslot += NT;
       if (kslot >= C::KSTAGES) {
         kslot -= C::KSTAGES;
         kph ^= 1u;
       }
-      vslot += NW;
+      vslot += NT;
       if (vslot >= C::VSTAGES) {
         vslot -= C::VSTAGES;
         vph ^= 1u;
@@ -1460,7 +1499,7 @@ __global__ void __maxnreg__(224)
         alive = false;
       }
     }
-    cons.end_piece(m_area, l_area, acc_area, w, lane, G);
+    cons.end_piece(m_area, l_area, acc_area, u, lane, G);
     __syncwarp();
     int last = 0;
     if (lane == 0) {
@@ -1473,19 +1512,20 @@ __global__ void __maxnreg__(224)
       __syncwarp();
       const bool whole = pc.n_pieces == 1;
       const int slot_idx = c + pc.seg;
-      // 1) lane h < G: the head's max over the warps' states, each warp's
-      //    weight exp(m_w - M) / L (times the fp8 V scale) written over m_w,
-      //    and the head's lse.  end_piece writes every warp's accumulator
-      //    (zeros for a warp without tiles), so a zero weight is exact.
+      // 1) lane h < G: the row's max over the tile lanes' states, each
+      //    lane's weight exp(m_u - M) / L (times the fp8 V scale) written
+      //    over m_u, and the row's lse.  end_piece writes every lane's
+      //    accumulator (zeros for a lane without tiles), so a zero weight is
+      //    exact.
       if (lane < G) {
         const int h = lane;
         float M = -CUDART_INF_F;
 #pragma unroll
-        for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, m_area[ww * G + h]);
-        float scw[NW];
+        for (int ww = 0; ww < NT; ++ww) M = fmaxf(M, m_area[ww * G + h]);
+        float scw[NT];
         float Ls = 0.f;
 #pragma unroll
-        for (int ww = 0; ww < NW; ++ww) {
+        for (int ww = 0; ww < NT; ++ww) {
           const float mw = m_area[ww * G + h];
           scw[ww] = (M == -CUDART_INF_F || mw == -CUDART_INF_F) ? 0.f : exp2_approx(mw - M);
           Ls = fmaf(l_area[ww * G + h], scw[ww], Ls);
@@ -1493,7 +1533,7 @@ __global__ void __maxnreg__(224)
         const bool empty = !(Ls > 0.f);
         const float f = empty ? 0.f : vs / Ls;
 #pragma unroll
-        for (int ww = 0; ww < NW; ++ww) m_area[ww * G + h] = scw[ww] * f;
+        for (int ww = 0; ww < NT; ++ww) m_area[ww * G + h] = scw[ww] * f;
         const float lv = empty ? -CUDART_INF_F : (M + __log2f(Ls)) * kLn2;
         const size_t row = (static_cast<size_t>(pc.b) * Q + h / GK) * a.qo_heads +
                            static_cast<size_t>(pc.h) * GK + h % GK;
@@ -1505,14 +1545,14 @@ __global__ void __maxnreg__(224)
         }
       }
       __syncwarp();
-      // 2) four dims per lane: out = sum_w weight_w * acc_w, branch-free
+      // 2) four dims per lane: out = sum_u weight_u * acc_u, branch-free
       //    float4 reads, one 16-byte partial store (or bf16x4 output store)
       constexpr int D4 = D / 4;
       for (int x4 = lane; x4 < G * D4; x4 += 32) {
         const int h = x4 / D4, dim = (x4 - h * D4) * 4;
         float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int ww = 0; ww < NW; ++ww) {
+        for (int ww = 0; ww < NT; ++ww) {
           const float f = m_area[ww * G + h];
           const float4 av = *reinterpret_cast<const float4*>(acc_area + (ww * G + h) * D + dim);
           O.x = fmaf(av.x, f, O.x);

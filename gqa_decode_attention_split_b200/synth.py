@@ -264,6 +264,24 @@ def _c4_q2():
                     name="paged_b64_gqa4_q2_L512-16384")
 
 
+def _c4_q(q_len):
+    def f():
+        """The batch-64 paged workload with q_len query tokens per request
+        (q_len - 1 draft tokens verified next to the decode token): 4 x q_len
+        rows per segment."""
+        return generate(64, 32, 8, 128, c4_lengths(), paged=True, page_size=16, seed=4, q_len=q_len,
+                        name=f"paged_b64_gqa4_q{q_len}_L512-16384")
+    return f
+
+
+def _gqa16():
+    """A Llama-3.1-405B-shaped layer on one of eight tensor-parallel GPUs
+    (128 query / 8 kv heads in all: 16 query heads on one kv head per GPU),
+    batch-64 paged decode with the same length mix."""
+    return generate(64, 16, 1, 128, c4_lengths(), paged=True, page_size=16, seed=7,
+                    name="llama3_405b_tp8_gqa16_paged_b64_L512-16384")
+
+
 def _c3_q8():
     """Llama-2-7B-shaped MHA layer at 32k keys with eight query tokens per
     request (seven draft tokens)."""
@@ -294,6 +312,9 @@ WORKLOADS = {
     "paged_b16_gqa4_L512-16384": _c4_small,
     "fp8_gqa8_L131072": _c5,
     "paged_b64_gqa4_q2_L512-16384": _c4_q2,
+    "paged_b64_gqa4_q4_L512-16384": _c4_q(4),
+    "paged_b64_gqa4_q8_L512-16384": _c4_q(8),
+    "llama3_405b_tp8_gqa16_paged_b64_L512-16384": _gqa16,
     "llama2_7b_mha_q8_L32768": _c3_q8,
     "gemma2_2b_softcap50_L8192": _gemma2_softcap,
 }

@@ -128,7 +128,7 @@ def test_forced_split_and_paths(lib):
     (dict(head_dim=96), [0, 10], 2),                     # no kernel
     (dict(kv_dtype=1, head_dim=64), [0, 10], 2),         # fp8 needs 128-byte rows
     (dict(qo_heads=32, kv_heads=2, path=1), [0, 10], 2),  # SIMT group 16
-    (dict(qo_heads=32, kv_heads=2, path=2), [0, 10], 2),  # MMA group 16
+    (dict(qo_heads=64, kv_heads=1, path=2), [0, 10], 2),  # MMA group 64 (rows > 32)
     (dict(paged=1, page_size=12), [0, 10], 1),           # not a power of two
     (dict(paged=1, page_size=512), [0, 10], 1),
     (dict(sm_scale=float("nan")), [0, 10], 1),
@@ -218,15 +218,21 @@ def test_binding_raises_without_library(monkeypatch, tmp_path):
 
 
 def test_plan_with_several_query_tokens(lib):
-    """q_len multiplies the rows of a segment (group * q_len <= 8 on the MMA
+    """q_len multiplies the rows of a segment (group * q_len <= 32 on the MMA
     dataflow) and widens the tile range by q_len - 1 keys under a window."""
     st, h, ws = _plan(lib, _desc(qo_heads=8, kv_heads=2, q_len=2), [0, 1000])
     assert st == 0
     inf = _info(lib, h)
     assert inf.path == binding.PATH_MMA
     lib.fa_plan_destroy(h)
-    # rows 4 * 4 = 16 exceed every kernel
-    st, h, ws = _plan(lib, _desc(qo_heads=8, kv_heads=2, q_len=4), [0, 1000])
+    # rows 4 * 4 = 16 and 4 * 8 = 32: row teams on the MMA dataflow
+    for q_len in (4, 8):
+        st, h, ws = _plan(lib, _desc(qo_heads=8, kv_heads=2, q_len=q_len), [0, 1000])
+        assert st == 0
+        assert _info(lib, h).path == binding.PATH_MMA
+        lib.fa_plan_destroy(h)
+    # rows 8 * 8 = 64 exceed every kernel
+    st, h, ws = _plan(lib, _desc(qo_heads=16, kv_heads=2, q_len=8), [0, 1000])
     assert st == 2 and not h  # FA_ERR_UNSUPPORTED
     # window 128 with 8 query tokens: the union spans 135 keys
     st, h, ws = _plan(lib, _desc(qo_heads=1, kv_heads=1, q_len=8, window=128), [0, 4096])
@@ -238,3 +244,24 @@ def test_plan_with_several_query_tokens(lib):
     for bad in (-1, 65):
         st, h, ws = _plan(lib, _desc(q_len=bad), [0, 100])
         assert st == 1  # FA_ERR_INVALID_ARG
+
+
+def test_row_team_variants(lib):
+    """Segments of 9..32 rows take the MMA variants with two or four row
+    teams: bf16 tiles of 32 tokens, equal K and V rings, a larger grid of
+    threads; 8 rows or fewer keep the single-team variant."""
+    cases = [(dict(qo_heads=8, kv_heads=8), 1, 64), (dict(qo_heads=16, kv_heads=1), 2, 32),
+             (dict(qo_heads=32, kv_heads=8, q_len=3), 2, 32),
+             (dict(qo_heads=32, kv_heads=8, q_len=8), 4, 32),
+             (dict(qo_heads=32, kv_heads=1), 4, 32)]
+    for kw, teams, T in cases:
+        st, h, ws = _plan(lib, _desc(path=2, **kw), [0, 5000])
+        assert st == 0, kw
+        inf = _info(lib, h)
+        assert inf.path == binding.PATH_MMA and inf.tile_tokens == T, (kw, inf.tile_tokens)
+        if teams > 1:
+            assert inf.stages == inf.v_stages  # equal rings
+        lib.fa_plan_destroy(h)
+    # SIMT keeps exact groups of at most 8 rows
+    st, h, _ = _plan(lib, _desc(path=1, qo_heads=16, kv_heads=1), [0, 100])
+    assert st == 2 and not h.value

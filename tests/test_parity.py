@@ -261,6 +261,18 @@ MULTI = [
     ("q4_gqa2_fp8_paged", 2, 16, 8, 128, [333, 70], {"q_len": 4, "kv_dtype": "fp8_e4m3",
                                                      "paged": True, "page_size": 32}),
     ("q4_short_request", 2, 2, 1, 128, [2, 90], {"q_len": 4}),
+    # more than 8 rows: two or four row teams on the MMA dataflow
+    ("q3_gqa4_d64_rows12", 2, 8, 2, 64, [260, 31], {"q_len": 3}),
+    ("q4_gqa4_paged_rows16", 3, 8, 2, 128, [300, 2, 65], {"q_len": 4, "paged": True, "page_size": 16}),
+    ("q8_gqa4_paged_rows32", 3, 8, 2, 128, [411, 17, 96], {"q_len": 8, "paged": True,
+                                                           "page_size": 16}),
+    ("q8_gqa4_fp8_win_rows32", 2, 8, 2, 128, [700, 50], {"q_len": 8, "kv_dtype": "fp8_e4m3",
+                                                         "window": 200}),
+    ("q2_gqa8_fp8_paged_rows16", 2, 16, 2, 128, [333, 70], {"q_len": 2, "kv_dtype": "fp8_e4m3",
+                                                            "paged": True, "page_size": 32}),
+    ("gqa16_d128_rows16", 1, 16, 1, 128, [2000], {}),
+    ("gqa32_d256_rows32", 1, 32, 1, 256, [900], {}),
+    ("q4_gqa8_d256_fp8_rows32", 1, 16, 2, 256, [530], {"q_len": 4, "kv_dtype": "fp8_e4m3"}),
 ]
 
 
@@ -278,6 +290,18 @@ def test_several_query_tokens(case, path):
 @pytest.mark.parametrize("path", PATHS)
 def test_several_query_tokens_forced_splits_agree(path):
     x = synth.generate(2, 4, 2, 128, [1500, 203], q_len=4, seed=29, window=700)
+    _forced_splits_agree(x, path)
+
+
+@pytest.mark.parametrize("q_len", [3, 8])
+def test_row_teams_forced_splits_agree(q_len):
+    """12 and 32 rows (two and four row teams): any split of the tiles over
+    blocks merges to the same result."""
+    x = synth.generate(2, 16, 4, 128, [1500, 203], q_len=q_len, seed=31, paged=True, page_size=16)
+    _forced_splits_agree(x, "mma")
+
+
+def _forced_splits_agree(x, path):
     results = []
     for n in (1, 7, 64, 0):
         out, lse, info = _check(x, path=path, num_ctas=n)
@@ -287,20 +311,23 @@ def test_several_query_tokens_forced_splits_agree(path):
         assert np.abs(o - results[0][0]).max() <= 4e-3
 
 
-def test_several_query_tokens_full_size_batched_paged():
-    """The batch-64 paged workload with two query tokens per request (one
-    draft token being verified), sampled rows against the oracle."""
+@pytest.mark.parametrize("q_len", [2, 8])
+def test_several_query_tokens_full_size_batched_paged(q_len):
+    """The batch-64 paged workload with 2 query tokens per request (one draft
+    token being verified; 8 rows per segment) and with 8 (32 rows, four row
+    teams), sampled rows against the oracle."""
     lens = synth.c4_lengths()
-    x = synth.generate(64, 32, 8, 128, lens, paged=True, page_size=16, seed=4, q_len=2,
-                       name="paged_b64_gqa4_q2")
+    x = synth.generate(64, 32, 8, 128, lens, paged=True, page_size=16, seed=4, q_len=q_len,
+                       name=f"paged_b64_gqa4_q{q_len}")
     out, lse, flags, info = run_gpu(x)
     assert flags == 0 and info["path"] == binding.PATH_MMA
     rng = np.random.default_rng(5)
-    rows = np.sort(rng.choice(64 * 2 * 32, 48, replace=False))
+    per = q_len * 32
+    rows = np.sort(rng.choice(64 * per, 48, replace=False))
     ro, rl = oracle.decode_rows(x, rows)
-    b, rem = rows // 64, rows % 64
+    b, rem = rows // per, rows % per
     i, h = rem // 32, rem % 32
-    assert_matches(out[b, i, h], lse[b, i, h], ro, rl, what="paged b64 q2 sampled")
+    assert_matches(out[b, i, h], lse[b, i, h], ro, rl, what=f"paged b64 q{q_len} sampled")
 
 
 # ------------------------------------------------------------ logit soft-cap
@@ -311,6 +338,8 @@ CAPPED = [
     ("cap10_fp8_paged_q2", 2, 8, 4, 128, [500, 77], {"logit_cap": 10.0, "sm_scale": 0.4,
                                                      "kv_dtype": "fp8_e4m3", "paged": True,
                                                      "page_size": 16, "q_len": 2}),
+    ("cap30_gqa16_q2_rows32", 1, 32, 2, 128, [1200], {"logit_cap": 30.0, "sm_scale": 0.5,
+                                                       "q_len": 2}),
 ]
 
 
