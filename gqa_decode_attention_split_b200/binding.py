@@ -53,6 +53,14 @@ class PlanInfo(ctypes.Structure):
                 ("v_stages", ctypes.c_int32)]
 
 
+class TuningEntry(ctypes.Structure):
+    """One row of the measured dataflow-choice table (fa_tuning_entry)."""
+    _fields_ = [("head_dim", ctypes.c_int32), ("kv_dtype", ctypes.c_int32),
+                ("rows_min", ctypes.c_int32), ("rows_max", ctypes.c_int32),
+                ("bytes_min", ctypes.c_int64), ("bytes_max", ctypes.c_int64),
+                ("path", ctypes.c_int32), ("max_pieces", ctypes.c_int32)]
+
+
 _lib = None
 
 
@@ -90,6 +98,10 @@ def load_library():
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_last_error.argtypes = []
     lib.fa_last_error.restype = ctypes.c_char_p
+    lib.fa_set_tuning.argtypes = [ctypes.POINTER(TuningEntry), i32]
+    lib.fa_set_tuning.restype = ctypes.c_int
+    lib.fa_get_tuning.argtypes = [ctypes.POINTER(TuningEntry), i32, ctypes.POINTER(i32)]
+    lib.fa_get_tuning.restype = ctypes.c_int
     lib.fa_version.argtypes = []
     lib.fa_version.restype = i32
     _lib = lib
@@ -242,3 +254,32 @@ def merge_states(o_parts, lse_parts, *, out=None, lse=None, stream=None) -> Tupl
     _check(lib.fa_merge_states(_ptr(o_parts), _ptr(lse_parts), n, rows, heads, d, _ptr(out),
                                _ptr(lse), _stream_handle(stream)), "fa_merge_states")
     return out, lse
+
+
+_TUNING_FIELDS = [f for f, _ in TuningEntry._fields_]
+
+
+def get_tuning() -> list:
+    """The active dataflow-choice table as a list of dicts."""
+    lib = load_library()
+    n = ctypes.c_int32(0)
+    _check(lib.fa_get_tuning(None, 0, ctypes.byref(n)), "fa_get_tuning")
+    arr = (TuningEntry * max(n.value, 1))()
+    _check(lib.fa_get_tuning(arr, n.value, ctypes.byref(n)), "fa_get_tuning")
+    return [{f: getattr(arr[i], f) for f in _TUNING_FIELDS} for i in range(n.value)]
+
+
+def set_tuning(rows) -> None:
+    """Install a dataflow-choice table (list of dicts with the fields of
+    TuningEntry; path and kv_dtype as the C enum values); None restores the
+    built-in table."""
+    lib = load_library()
+    if rows is None:
+        _check(lib.fa_set_tuning(None, 0), "fa_set_tuning")
+        return
+    arr = (TuningEntry * max(len(rows), 1))()
+    for i, r in enumerate(rows):
+        for f in _TUNING_FIELDS:
+            setattr(arr[i], f, int(r[f]))
+    _check(lib.fa_set_tuning(arr, len(rows)), "fa_set_tuning")
+

@@ -11,6 +11,7 @@
 
 #include <mutex>
 #include <new>
+#include <vector>
 
 #include "../../include/fadecode.h"
 #include "fa_kernel.cuh"
@@ -137,7 +138,69 @@ int32_t union_window(const fa_decode_desc* d) {
   return d->window > 0 ? d->window + q_len_of(d) - 1 : d->window;
 }
 
+// ------------------------------------------------------------ measured choice
+// The dataflow-choice table ("FlashDecoding++" explainer, section
+// "Hardware-aware heuristic dataflow"): rows measured on the GPU, first match
+// wins.  Starts as the built-in table; fa_set_tuning replaces it.
+#define FA_TUNING_ROW(d, dt, r0, r1, b0, b1, path, pieces) {d, dt, r0, r1, b0, b1, path, pieces},
+const fa_tuning_entry kBuiltinTuning[] = {
+#include "fa_tuning_b200.inc"
+    {0, 0, 0, 0, 0, 0, 0, 0}};  // end mark
+#undef FA_TUNING_ROW
+
+std::vector<fa_tuning_entry> builtin_tuning() {
+  std::vector<fa_tuning_entry> t;
+  for (const fa_tuning_entry& e : kBuiltinTuning)
+    if (e.head_dim != 0) t.push_back(e);
+  return t;
+}
+
+std::vector<fa_tuning_entry>& tuning_table() {
+  static std::vector<fa_tuning_entry> t = builtin_tuning();
+  return t;
+}
+
+bool valid_tuning_row(const fa_tuning_entry& e) {
+  return e.head_dim > 0 && (e.kv_dtype == FA_KV_BF16 || e.kv_dtype == FA_KV_FP8_E4M3) &&
+         e.rows_min >= 1 && e.rows_min <= e.rows_max && e.bytes_min >= 0 &&
+         e.bytes_min <= e.bytes_max && (e.path == FA_PATH_SIMT || e.path == FA_PATH_MMA) &&
+         e.max_pieces >= 0 && e.max_pieces <= 1024;
+}
+
+// Visible K/V bytes of a decode: the keys some query token of each request
+// sees, times kv heads, K and V, and the row size.
+int64_t visible_kv_bytes(const fa_decode_desc* d, const int32_t* indptr) {
+  const int32_t wu = union_window(d);
+  int64_t toks = 0;
+  for (int b = 0; b < d->batch; ++b) {
+    const int64_t L = indptr[b + 1] - indptr[b];
+    toks += (wu > 0 && L > wu) ? wu : L;
+  }
+  const int64_t row = static_cast<int64_t>(d->head_dim) * (d->kv_dtype == FA_KV_FP8_E4M3 ? 1 : 2);
+  return toks * d->kv_heads * 2 * row;
+}
+
 }  // namespace
+
+extern "C" fa_status fa_set_tuning(const fa_tuning_entry* entries, int32_t n) {
+  if (n < 0 || n > 4096 || (entries == nullptr && n > 0)) return FA_ERR_INVALID_ARG;
+  if (entries == nullptr) {
+    tuning_table() = builtin_tuning();
+    return FA_OK;
+  }
+  for (int32_t i = 0; i < n; ++i)
+    if (!valid_tuning_row(entries[i])) return FA_ERR_INVALID_ARG;
+  tuning_table().assign(entries, entries + n);
+  return FA_OK;
+}
+
+extern "C" fa_status fa_get_tuning(fa_tuning_entry* out, int32_t cap, int32_t* n) {
+  if (n == nullptr || cap < 0 || (out == nullptr && cap > 0)) return FA_ERR_INVALID_ARG;
+  const std::vector<fa_tuning_entry>& t = tuning_table();
+  *n = static_cast<int32_t>(t.size());
+  for (int32_t i = 0; i < cap && i < *n; ++i) out[i] = t[static_cast<size_t>(i)];
+  return FA_OK;
+}
 
 extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* kv_indptr_host,
                                     int32_t num_sms, fa_plan** plan, size_t* workspace_bytes) {
@@ -159,15 +222,30 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   const int group = desc->qo_heads / desc->kv_heads * q_len_of(desc);
   const int fp8 = desc->kv_dtype == FA_KV_FP8_E4M3 ? 1 : 0;
 
-  // Dataflow choice: the tensor-core (MMA) path whenever a kernel exists for
-  // the shape; the SIMT path when asked for, or when the group exceeds 8.
+  // Dataflow choice.  Asked for: that dataflow.  Otherwise the first row of
+  // the measured table that covers the shape (when the grid is not forced),
+  // else the fixed rule: the tensor-core (MMA) path whenever a kernel exists
+  // for the shape, the SIMT path otherwise.
   const KernelEntry* k = nullptr;
+  int64_t max_pieces = 32;  // average blocks per segment, at most
   if (desc->path == FA_PATH_SIMT) {
     k = find_entry(desc->head_dim, group, fp8, fa::kPathSimt);
   } else if (desc->path == FA_PATH_MMA) {
     k = find_entry(desc->head_dim, group, fp8, fa::kPathMma);
   } else {
-    k = find_entry(desc->head_dim, group, fp8, fa::kPathMma);
+    if (desc->num_ctas == 0) {
+      const int64_t bytes = visible_kv_bytes(desc, kv_indptr_host);
+      for (const fa_tuning_entry& e : tuning_table()) {
+        if (e.head_dim != desc->head_dim || e.kv_dtype != desc->kv_dtype || group < e.rows_min ||
+            group > e.rows_max || bytes < e.bytes_min || bytes > e.bytes_max)
+          continue;
+        k = find_entry(desc->head_dim, group, fp8, e.path == FA_PATH_SIMT ? fa::kPathSimt : fa::kPathMma);
+        if (k == nullptr) continue;
+        if (e.max_pieces > 0) max_pieces = e.max_pieces;
+        break;
+      }
+    }
+    if (k == nullptr) k = find_entry(desc->head_dim, group, fp8, fa::kPathMma);
     if (k == nullptr) k = find_entry(desc->head_dim, group, fp8, fa::kPathSimt);
   }
   if (k == nullptr) return FA_ERR_UNSUPPORTED;
@@ -190,12 +268,11 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
     // One block per SM (each holds a ~170 KB tile ring).  A problem with
     // fewer tiles than SMs gets one tile per block (the fixed cost of a
     // block is small next to a KV tile's load latency, and the tiles load in
-    // parallel); a segment is cut into at most kMaxPiecesPerSegment runs on
+    // parallel); a segment is cut into at most max_pieces runs on
     // average so that the last block's merge of the partial states stays
-    // short.
-    constexpr int64_t kMaxPiecesPerSegment = 32;
+    // short (32 unless the measured table says otherwise).
     int64_t want = tiles;
-    const int64_t seg_cap = kMaxPiecesPerSegment * desc->batch * desc->kv_heads;
+    const int64_t seg_cap = max_pieces * desc->batch * desc->kv_heads;
     if (want > seg_cap) want = seg_cap;
     P = want < num_sms ? want : num_sms;
     if (P < 1) P = 1;

@@ -100,8 +100,10 @@ typedef struct {
                       /* optimization"): the request's q_len newest keys are */
                       /* its query tokens, and token i (position            */
                       /* L - q_len + i) sees the keys up to and including    */
-                      /* itself, or the last `window` of them.  Needs        */
-                      /* (qo_heads / kv_heads) * q_len <= 8.                 */
+                      /* itself, or the last `window` of them.  The rows of  */
+                      /* a (request, kv head) segment, (qo_heads / kv_heads) */
+                      /* * q_len, must be <= 32 on the MMA dataflow (SIMT:   */
+                      /* exactly 1, 2, 4 or 8; 1, 2 or 4 for fp8).           */
   float logit_cap;    /* 0: none.  c > 0: logit soft-capping, each scaled    */
                       /* score s becomes c * tanh(s / c) before the softmax  */
                       /* (Gemma 2's soft-cap, named on "FlashInfer x JAX via */
@@ -157,6 +159,51 @@ FA_API fa_status fa_plan_get_info(const fa_plan* plan, fa_plan_info_t* info);
 
 /* Releases a plan (NULL is a no-op). */
 FA_API void fa_plan_destroy(fa_plan* plan);
+
+/*
+ * Measured dataflow choice ("FlashDecoding++" explainer, section
+ * "Hardware-aware heuristic dataflow": which implementation runs a shape is
+ * decided from measurements of the shapes on the GPU, not from a fixed
+ * rule).  A table row covers decodes with the given head_dim and kv dtype
+ * whose rows per (request, kv head) segment, (qo_heads / kv_heads) * q_len,
+ * lie in [rows_min, rows_max] and whose visible K/V bytes (keys each query
+ * token sees, at most window + q_len - 1 per request, x kv_heads x 2 x
+ * head_dim x element size) lie in [bytes_min, bytes_max].  It names the
+ * dataflow and the largest average number of thread blocks per segment
+ * (max_pieces; 0: the planner's default of 32), which bounds the split of
+ * short problems.
+ */
+typedef struct {
+  int32_t head_dim;
+  int32_t kv_dtype;      /* fa_kv_dtype                                     */
+  int32_t rows_min, rows_max;
+  int64_t bytes_min, bytes_max;
+  int32_t path;          /* FA_PATH_SIMT or FA_PATH_MMA                     */
+  int32_t max_pieces;    /* 0, or 1 .. 1024                                 */
+} fa_tuning_entry;
+
+/*
+ * fa_set_tuning -- install the table fa_decode_plan consults when
+ * desc->path is FA_PATH_AUTO and desc->num_ctas is 0.  The first matching
+ * row wins; a row whose dataflow has no kernel for the shape is passed
+ * over; a decode no row matches gets the fixed rule (MMA where a kernel
+ * exists, else SIMT; up to 32 blocks per segment).  The rows are copied.
+ * entries == NULL (with n == 0) restores the built-in table, which was
+ * measured on a B200 by the package's tuning script; n == 0 with a non-NULL
+ * pointer installs an empty table (fixed rule only).  Not safe to call while
+ * another thread is planning.
+ * Errors: FA_ERR_INVALID_ARG (n < 0 or > 4096, NULL with n > 0, a row with
+ * rows_min > rows_max, bytes_min > bytes_max, rows_min < 1, an unknown path
+ * or dtype, max_pieces outside 0 .. 1024).
+ */
+FA_API fa_status fa_set_tuning(const fa_tuning_entry* entries, int32_t n);
+
+/*
+ * fa_get_tuning -- copy the active table: *n receives its row count and the
+ * first min(cap, *n) rows go to out (out may be NULL when cap == 0).
+ * Errors: FA_ERR_INVALID_ARG (n NULL, cap < 0, out NULL with cap > 0).
+ */
+FA_API fa_status fa_get_tuning(fa_tuning_entry* out, int32_t cap, int32_t* n);
 
 /*
  * fa_decode_run -- enqueue one decode-attention pass on `stream`.

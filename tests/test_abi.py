@@ -265,3 +265,96 @@ def test_row_team_variants(lib):
     # SIMT keeps exact groups of at most 8 rows
     st, h, _ = _plan(lib, _desc(path=1, qo_heads=16, kv_heads=1), [0, 100])
     assert st == 2 and not h.value
+
+
+def _row(**kw):
+    r = dict(head_dim=128, kv_dtype=0, rows_min=1, rows_max=8, bytes_min=0, bytes_max=1 << 40,
+             path=binding.PATH_SIMT, max_pieces=0)
+    r.update(kw)
+    return r
+
+
+def test_tuning_table_drives_the_auto_choice(lib):
+    """The planner takes the first table row that covers a decode (head_dim,
+    dtype, rows, visible K/V bytes) when the path is AUTO and the grid is not
+    forced; rows that do not cover it, or name a dataflow without a kernel,
+    are passed over and the fixed rule applies."""
+    builtin = binding.get_tuning()
+    try:
+        # 1000 keys x 2 kv heads x 2 x 256 B = 1,024,000 visible bytes
+        binding.set_tuning([_row(rows_min=4, rows_max=4, bytes_max=1_024_000, max_pieces=2)])
+        assert binding.get_tuning()[0]["max_pieces"] == 2
+        st, h, _ = _plan(lib, _desc(), [0, 1000])
+        inf = _info(lib, h)
+        assert st == 0 and inf.path == binding.PATH_SIMT
+        assert inf.num_ctas <= 2 * 2  # at most 2 blocks per segment on average
+        lib.fa_plan_destroy(h)
+        # one key more: outside the row -> fixed rule (MMA, up to 32 per segment)
+        st, h, _ = _plan(lib, _desc(), [0, 1001])
+        inf = _info(lib, h)
+        assert inf.path == binding.PATH_MMA and inf.num_ctas > 4
+        lib.fa_plan_destroy(h)
+        # a window bounds the visible bytes: 1001 keys, window 1000 -> covered
+        st, h, _ = _plan(lib, _desc(window=1000), [0, 1001])
+        assert _info(lib, h).path == binding.PATH_SIMT
+        lib.fa_plan_destroy(h)
+        # forced path or forced grid: the table is not consulted
+        for kw in (dict(path=binding.PATH_MMA), dict(num_ctas=7)):
+            st, h, _ = _plan(lib, _desc(**kw), [0, 1000])
+            assert _info(lib, h).path == binding.PATH_MMA
+            lib.fa_plan_destroy(h)
+        # a SIMT row for 16 rows has no kernel: passed over, MMA row teams run it
+        binding.set_tuning([_row(rows_min=16, rows_max=16)])
+        st, h, _ = _plan(lib, _desc(qo_heads=16, kv_heads=1), [0, 1000])
+        assert st == 0 and _info(lib, h).path == binding.PATH_MMA
+        lib.fa_plan_destroy(h)
+        # an empty table: fixed rule only
+        binding.set_tuning([])
+        assert binding.get_tuning() == []
+    finally:
+        binding.set_tuning(None)
+    assert binding.get_tuning() == builtin
+
+
+@pytest.mark.parametrize("bad", [dict(rows_min=0), dict(rows_min=5, rows_max=4),
+                                 dict(bytes_min=10, bytes_max=9), dict(bytes_min=-1),
+                                 dict(path=0), dict(path=3), dict(kv_dtype=2),
+                                 dict(max_pieces=-1), dict(max_pieces=1025), dict(head_dim=0)])
+def test_tuning_table_rejects_bad_rows(lib, bad):
+    before = binding.get_tuning()
+    with pytest.raises(binding.FadecodeError):
+        binding.set_tuning([_row(), _row(**bad)])
+    assert binding.get_tuning() == before  # nothing installed
+    n = ctypes.c_int32(0)
+    assert lib.fa_set_tuning(None, 3) == 1
+    assert lib.fa_get_tuning(None, 0, None) == 1
+    assert lib.fa_get_tuning(None, 2, ctypes.byref(n)) == 1
+
+
+def test_builtin_tuning_table_is_well_formed(lib):
+    for r in binding.get_tuning():
+        assert r["rows_min"] <= r["rows_max"] and r["bytes_min"] <= r["bytes_max"]
+        assert r["path"] in (binding.PATH_SIMT, binding.PATH_MMA)
+        assert r["head_dim"] in (64, 128, 256) and r["kv_dtype"] in (0, 1)
+
+
+def test_builtin_tuning_rows_take_effect(lib):
+    """Every row of the built-in (measured) table decides the plan of a
+    decode inside its range: batch 1, 8 kv heads, as many keys as put the
+    visible K/V bytes at the row's lower bound (or 1 MiB above zero)."""
+    rows = binding.get_tuning()
+    for r in rows:
+        es = 1 if r["kv_dtype"] == 1 else 2
+        per_key = 8 * 2 * r["head_dim"] * es
+        target = max(r["bytes_min"], 1 << 20)
+        L = -(-target // per_key)
+        assert L * per_key <= r["bytes_max"]
+        st, h, _ = _plan(lib, _desc(head_dim=r["head_dim"], kv_dtype=r["kv_dtype"], kv_heads=8,
+                                    qo_heads=8 * r["rows_min"],
+                                    sm_scale=1.0 / math.sqrt(r["head_dim"])), [0, L])
+        assert st == 0, r
+        inf = _info(lib, h)
+        assert inf.path == r["path"], r
+        if r["max_pieces"]:
+            assert inf.num_ctas <= r["max_pieces"] * 8, r
+        lib.fa_plan_destroy(h)

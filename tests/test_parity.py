@@ -362,3 +362,23 @@ def test_logit_softcap_forced_splits():
     x = synth.generate(1, 8, 2, 128, [2500], seed=30, logit_cap=15.0, sm_scale=0.5)
     for n in (1, 9, 0):
         _check(x, path="mma", num_ctas=n)
+
+
+# ------------------------------------------------- measured dataflow choice
+def test_tuned_choices_match_the_oracle():
+    """Decodes that fall in a row of the built-in measured table (those of at
+    most 48 MB of visible K/V) run on the chosen dataflow and piece cap and
+    still match the oracle."""
+    rows = [r for r in binding.get_tuning() if r["bytes_min"] <= 48 << 20]
+    assert rows, "the built-in table has small-problem rows"
+    for r in rows:
+        d, rows_per = r["head_dim"], r["rows_min"]
+        es = 1 if r["kv_dtype"] == 1 else 2
+        per_key = 8 * 2 * d * es
+        L = -(-max(r["bytes_min"], 1 << 20) // per_key) + 3
+        assert L * per_key <= r["bytes_max"]
+        x = synth.generate(1, 8 * rows_per, 8, d, [L], seed=L % 1000,
+                           kv_dtype="fp8_e4m3" if r["kv_dtype"] == 1 else "bf16",
+                           name=f"tuned_d{d}_r{rows_per}_L{L}")
+        out, lse, info = _check(x, path="auto")
+        assert info["path"] == r["path"]
