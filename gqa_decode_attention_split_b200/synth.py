@@ -8,7 +8,10 @@ scales, int32 index arrays), so the two sides see bit-identical inputs.
 Value recipe: i.i.d. standard normal draws from numpy's PCG64, rounded to
 bf16 with round-to-nearest-even.  FP8 KV: the same normal draws, divided by a
 per-kv-head scale amax/448 and rounded to e4m3 "fn" (round-to-nearest-even,
-clamped to +-448); the scales are returned with the codes.  Random streams are
+clamped to +-448); the scales are returned with the codes.  INT4 KV: the same
+draws divided by a per-kv-head scale amax/7, rounded to the nearest integer
+(ties to even) and clamped to [-7, 7], stored as two's-complement nibbles,
+two per byte with the even element in the low nibble.  Random streams are
 keyed by (seed, stream id) and generated in fixed-size chunks, so the values
 do not depend on the number of threads used to draw them.
 
@@ -35,6 +38,8 @@ _CHUNK = 1 << 22  # elements per independently seeded chunk
 _S_Q, _S_K, _S_V, _S_LEN, _S_PERM = 0, 1, 2, 3, 4
 
 FP8_MAX = 448.0
+INT4_MAX = 7.0
+KV_DTYPES = ("bf16", "fp8_e4m3", "int4")
 
 
 def _normals(seed: int, stream: int, n: int) -> np.ndarray:
@@ -79,7 +84,7 @@ class DecodeInputs:
     qo_heads: int
     kv_heads: int
     head_dim: int
-    kv_dtype: str          # "bf16" or "fp8_e4m3"
+    kv_dtype: str          # "bf16", "fp8_e4m3" or "int4" (k, v: packed bytes [..., d / 2])
     paged: bool
     page_size: int
     window: int            # <= 0: all keys
@@ -109,7 +114,14 @@ class DecodeInputs:
 
     @property
     def elem_bytes(self) -> int:
-        return 1 if self.kv_dtype == "fp8_e4m3" else 2
+        """Bytes per element (int4: 1, the packed byte unit; see row_bytes)."""
+        return 2 if self.kv_dtype == "bf16" else 1
+
+    @property
+    def row_bytes(self) -> int:
+        """Bytes of one token's row of one kv head (K or V)."""
+        return {"bf16": 2 * self.head_dim, "fp8_e4m3": self.head_dim,
+                "int4": self.head_dim // 2}[self.kv_dtype]
 
     def visible_lens(self) -> np.ndarray:
         """Keys some query token of the request sees (the union of the
@@ -122,7 +134,7 @@ class DecodeInputs:
 
     def kv_bytes(self) -> int:
         """Algorithmic bytes: K and V of every visible key, read once."""
-        return int(self.visible_lens().sum()) * self.kv_heads * self.head_dim * self.elem_bytes * 2
+        return int(self.visible_lens().sum()) * self.kv_heads * self.row_bytes * 2
 
     def with_window(self, window: int, name: Optional[str] = None) -> "DecodeInputs":
         """Same arrays, different window."""
@@ -149,8 +161,10 @@ def generate(batch: int, qo_heads: int, kv_heads: int, head_dim: int,
     q_len: query tokens per request (q is [batch, q_len, qo_heads, head_dim]
     when q_len > 1); they are the request's q_len newest keys.
     """
-    if kv_dtype not in ("bf16", "fp8_e4m3"):
+    if kv_dtype not in KV_DTYPES:
         raise ValueError(kv_dtype)
+    if kv_dtype == "int4" and head_dim % 2:
+        raise ValueError("int4 rows hold whole bytes: head_dim must be even")
     lens = np.asarray(list(kv_lens), dtype=np.int64)
     if lens.shape != (batch,):
         raise ValueError("kv_lens must have one entry per request")
@@ -191,6 +205,17 @@ def generate(batch: int, qo_heads: int, kv_heads: int, head_dim: int,
     if kv_dtype == "bf16":
         k = _to_bf16_bits(_normals(seed, _S_K, n_el)).reshape(shape)
         v = _to_bf16_bits(_normals(seed, _S_V, n_el)).reshape(shape)
+    elif kv_dtype == "int4":
+        arrs, scales = [], []
+        for stream in (_S_K, _S_V):
+            x = _normals(seed, stream, n_el).reshape(shape)
+            amax = np.abs(x).reshape(-1, kv_heads, d).max(axis=(0, 2)).astype(np.float32)
+            scale = np.where(amax > 0, amax / np.float32(INT4_MAX), np.float32(1.0)).astype(np.float32)
+            x /= scale.reshape((1,) * (len(shape) - 2) + (kv_heads, 1))
+            arrs.append(_pack_int4(np.clip(np.rint(x), -INT4_MAX, INT4_MAX).astype(np.int8)))
+            scales.append(scale)
+        k, v = arrs
+        k_scale, v_scale = scales
     else:
         arrs, scales = [], []
         for stream in (_S_K, _S_V):
@@ -204,7 +229,9 @@ def generate(batch: int, qo_heads: int, kv_heads: int, head_dim: int,
         k_scale, v_scale = scales
 
     if paged and unused_slot_fill == "nan":
-        nan_code = np.uint16(0x7FC0) if kv_dtype == "bf16" else np.uint8(0x7F)
+        # int4 has no NaN: the extreme code -8 in every nibble instead
+        nan_code = {"bf16": np.uint16(0x7FC0), "fp8_e4m3": np.uint8(0x7F),
+                    "int4": np.uint8(0x88)}[kv_dtype]
         for b in range(batch):
             L = int(lens[b])
             n = (L + page_size - 1) // page_size
@@ -220,6 +247,13 @@ def generate(batch: int, qo_heads: int, kv_heads: int, head_dim: int,
                         kv_indptr=indptr.astype(np.int32), page_table=page_table,
                         k_scale=k_scale, v_scale=v_scale, q_len=q_len,
                         logit_cap=float(logit_cap))
+
+
+def _pack_int4(codes: np.ndarray) -> np.ndarray:
+    """Signed codes [..., d] (int8 in [-8, 7]) -> bytes [..., d / 2], element
+    2i in the low nibble of byte i (two's complement nibbles)."""
+    u = codes.astype(np.uint8) & np.uint8(0xF)
+    return (u[..., 0::2] | (u[..., 1::2] << np.uint8(4))).astype(np.uint8)
 
 
 def c4_lengths(seed: int = 4, batch: int = 64, lo: int = 512, hi: int = 16384) -> np.ndarray:

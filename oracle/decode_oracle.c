@@ -48,6 +48,11 @@
  *  - an empty key set gives out = 0 and lse = -inf.
  *  - FP8 is e4m3 "fn" (bias 7, no infinities, S.1111.111 is NaN); a stored
  *    code c of kv head g means decode(c) * scale[g], product taken in fp64.
+ *  - INT4 ("Beyond the Memory Wall", section "2. FlashInfer", names INT4
+ *    KV quantization without a format): two's-complement 4-bit codes in
+ *    [-8, 7], two per byte, the even element of a row in the low nibble; a
+ *    code c of kv head g means c * scale[g] (one scale per kv head for K and
+ *    one for V, as for FP8).
  *  - paged pool layout [num_pages, page_size, kv_heads, head_dim]; token t of
  *    request b sits in page page_table[b*stride + t/page_size], slot
  *    t % page_size.  Contiguous layout [total_tokens, kv_heads, head_dim];
@@ -64,16 +69,18 @@
 /* Problem description.  All pointers are host memory owned by the caller. */
 typedef struct {
     int32_t batch, qo_heads, kv_heads, head_dim;
-    int32_t kv_fp8;          /* 0: K/V are bf16 bit patterns; 1: e4m3 codes  */
+    int32_t kv_kind;         /* 0: K/V are bf16 bit patterns; 1: e4m3 codes;
+                                2: int4 codes, two per byte                  */
     int32_t paged;           /* 0: contiguous rows; 1: paged pool            */
     int32_t page_size;       /* paged only                                    */
     int32_t page_table_stride;
     int32_t window;          /* <= 0: all keys; > 0: last `window` keys       */
     double sm_scale;
     const uint16_t *q;       /* bf16 bits [batch, qo_heads, head_dim]         */
-    const void *k, *v;       /* uint16 (bf16) or uint8 (e4m3), layout above   */
-    const float *k_scale;    /* [kv_heads], fp8 only                          */
-    const float *v_scale;    /* [kv_heads], fp8 only                          */
+    const void *k, *v;       /* uint16 (bf16), uint8 (e4m3) or packed int4
+                                bytes (head_dim / 2 per row), layout above   */
+    const float *k_scale;    /* [kv_heads], fp8 and int4 only                 */
+    const float *v_scale;    /* [kv_heads], fp8 and int4 only                 */
     const int32_t *kv_indptr;  /* [batch + 1] token counts, cumulative        */
     const int32_t *page_table; /* [batch, page_table_stride], paged only      */
     int32_t q_len;           /* query tokens per request (0 means 1); q is
@@ -107,6 +114,13 @@ double oracle_e4m3_to_double(uint8_t code) {
     return sign ? -mag : mag;
 }
 
+/* Signed value of the int4 code in the low (high = 0) or high nibble of a
+ * byte: two's complement, so 0x8 .. 0xF stand for -8 .. -1. */
+int oracle_int4_code(uint8_t byte, int high) {
+    int c = high ? (byte >> 4) & 0xF : byte & 0xF;
+    return c >= 8 ? c - 16 : c;
+}
+
 /* Value of K or V element (token t of request b, kv head g, dim i), as a
  * real number. */
 static double kv_element(const oracle_problem *p, const void *base,
@@ -120,8 +134,11 @@ static double kv_element(const oracle_problem *p, const void *base,
         row = (int64_t)p->kv_indptr[b] + t;
     }
     int64_t idx = (row * p->kv_heads + g) * p->head_dim + i;
-    if (p->kv_fp8)
+    if (p->kv_kind == 1)
         return oracle_e4m3_to_double(((const uint8_t *)base)[idx]) * (double)scale[g];
+    if (p->kv_kind == 2)  /* head_dim is even: element idx is nibble idx & 1 of byte idx / 2 */
+        return (double)oracle_int4_code(((const uint8_t *)base)[idx >> 1], (int)(idx & 1)) *
+               (double)scale[g];
     return oracle_bf16_to_double(((const uint16_t *)base)[idx]);
 }
 

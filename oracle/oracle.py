@@ -42,7 +42,7 @@ class _Problem(ctypes.Structure):
     _fields_ = [
         ("batch", ctypes.c_int32), ("qo_heads", ctypes.c_int32),
         ("kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
-        ("kv_fp8", ctypes.c_int32), ("paged", ctypes.c_int32),
+        ("kv_kind", ctypes.c_int32), ("paged", ctypes.c_int32),
         ("page_size", ctypes.c_int32), ("page_table_stride", ctypes.c_int32),
         ("window", ctypes.c_int32), ("sm_scale", ctypes.c_double),
         ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
@@ -70,6 +70,8 @@ def _load():
         lib.oracle_bf16_to_double.restype = ctypes.c_double
         lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
         lib.oracle_e4m3_to_double.restype = ctypes.c_double
+        lib.oracle_int4_code.argtypes = [ctypes.c_uint8, ctypes.c_int]
+        lib.oracle_int4_code.restype = ctypes.c_int
         lib.oracle_max_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -89,16 +91,17 @@ def _problem(x) -> Tuple[_Problem, list]:
         keep.append(a)
         return a
 
-    fp8 = x.kv_dtype == "fp8_e4m3"
+    kind = {"bf16": 0, "fp8_e4m3": 1, "int4": 2}[x.kv_dtype]
+    quant = kind != 0
     q = c(x.q, np.uint16)
-    k = c(x.k, np.uint8 if fp8 else np.uint16)
-    v = c(x.v, np.uint8 if fp8 else np.uint16)
-    ks = c(x.k_scale, np.float32) if fp8 else None
-    vs = c(x.v_scale, np.float32) if fp8 else None
+    k = c(x.k, np.uint8 if quant else np.uint16)
+    v = c(x.v, np.uint8 if quant else np.uint16)
+    ks = c(x.k_scale, np.float32) if quant else None
+    vs = c(x.v_scale, np.float32) if quant else None
     ind = c(x.kv_indptr, np.int32)
     pt = c(x.page_table, np.int32) if x.paged else None
     p = _Problem(batch=x.batch, qo_heads=x.qo_heads, kv_heads=x.kv_heads,
-                 head_dim=x.head_dim, kv_fp8=int(fp8), paged=int(bool(x.paged)),
+                 head_dim=x.head_dim, kv_kind=kind, paged=int(bool(x.paged)),
                  page_size=int(x.page_size) if x.paged else 1,
                  page_table_stride=int(pt.shape[1]) if pt is not None else 0,
                  window=int(x.window), sm_scale=float(x.sm_scale),
@@ -188,6 +191,20 @@ def e4m3_to_double(codes) -> np.ndarray:
     lib = _load()
     c = np.asarray(codes, dtype=np.uint8)
     return np.array([lib.oracle_e4m3_to_double(int(v)) for v in c.ravel()]).reshape(c.shape)
+
+
+def int4_codes(packed) -> np.ndarray:
+    """Signed int4 codes of packed bytes [..., n] -> [..., 2n] (element 2i
+    from the low nibble of byte i)."""
+    lib = _load()
+    b = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), dtype=np.int64)
+    flat_b, flat_o = b.reshape(-1, b.shape[-1]), out.reshape(-1, out.shape[-1])
+    for r in range(flat_b.shape[0]):
+        for i in range(flat_b.shape[1]):
+            flat_o[r, 2 * i] = lib.oracle_int4_code(int(flat_b[r, i]), 0)
+            flat_o[r, 2 * i + 1] = lib.oracle_int4_code(int(flat_b[r, i]), 1)
+    return out
 
 
 def max_threads() -> int:

@@ -31,6 +31,21 @@ def e4m3_values(codes) -> np.ndarray:
     return torch.from_numpy(c).view(torch.float8_e4m3fn).to(torch.float64).numpy()
 
 
+def int4_values(packed) -> np.ndarray:
+    """Signed int4 codes of packed bytes [..., n] as float64 [..., 2n]: the
+    low nibble of byte i is element 2i, the high nibble element 2i + 1, each
+    a two's-complement 4-bit number (decoded here with numpy shifts, apart
+    from the oracle's decoder)."""
+    b = np.asarray(packed, dtype=np.uint8).astype(np.int64)
+    lo, hi = b & 15, b >> 4
+    lo = np.where(lo >= 8, lo - 16, lo)
+    hi = np.where(hi >= 8, hi - 16, hi)
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), dtype=np.float64)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return out
+
+
 def contiguous_inputs(q, k, v, kv_lens, *, sm_scale=1.0, window=-1, name="hand") -> DecodeInputs:
     """q [B, Hq, d], k/v [rows, Hkv, d] as float values exactly representable in bf16."""
     q = np.asarray(q, dtype=np.float32)
@@ -56,14 +71,17 @@ def dense_kv(x: DecodeInputs, b: int):
             pg = int(x.page_table[b, t // x.page_size])
             rows_k.append(x.k[pg, t % x.page_size])
             rows_v.append(x.v[pg, t % x.page_size])
-        kk = np.stack(rows_k) if L else np.zeros((0, x.kv_heads, x.head_dim), x.k.dtype)
-        vv = np.stack(rows_v) if L else np.zeros((0, x.kv_heads, x.head_dim), x.v.dtype)
+        kk = np.stack(rows_k) if L else np.zeros((0, x.kv_heads, x.k.shape[-1]), x.k.dtype)
+        vv = np.stack(rows_v) if L else np.zeros((0, x.kv_heads, x.v.shape[-1]), x.v.dtype)
     else:
         a = int(x.kv_indptr[b])
         kk, vv = x.k[a:a + L], x.v[a:a + L]
     if x.kv_dtype == "fp8_e4m3":
         kf = e4m3_values(kk) * x.k_scale.astype(np.float64)[None, :, None]
         vf = e4m3_values(vv) * x.v_scale.astype(np.float64)[None, :, None]
+    elif x.kv_dtype == "int4":
+        kf = int4_values(kk) * x.k_scale.astype(np.float64)[None, :, None]
+        vf = int4_values(vv) * x.v_scale.astype(np.float64)[None, :, None]
     else:
         kf, vf = bf16_values(kk), bf16_values(vv)
     return kf, vf

@@ -20,7 +20,8 @@ import torch
 
 from gqa_decode_attention_split_b200 import synth
 from gqa_decode_attention_split_b200.synth import DecodeInputs
-from helpers import bf16_bits, bf16_values, contiguous_inputs, dense_kv, e4m3_values, visible
+from helpers import (bf16_bits, bf16_values, contiguous_inputs, dense_kv, e4m3_values, int4_values,
+                     visible)
 from oracle import oracle
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
@@ -129,10 +130,12 @@ def _sdpa_reference(x: DecodeInputs, b: int):
     dict(batch=2, qo=4, kv=2, d=16, lens=[33, 7], paged=True, page_size=4),
     dict(batch=2, qo=8, kv=2, d=32, lens=[45, 12], fp8=True),
     dict(batch=2, qo=4, kv=2, d=16, lens=[19, 50], fp8=True, paged=True, page_size=8, window=9),
+    dict(batch=2, qo=8, kv=2, d=32, lens=[45, 12], dtype="int4"),
+    dict(batch=2, qo=4, kv=2, d=16, lens=[19, 50], dtype="int4", paged=True, page_size=8, window=9),
 ])
 def test_matches_textbook_sdpa(case):
     x = synth.generate(case["batch"], case["qo"], case["kv"], case["d"], case["lens"],
-                       kv_dtype="fp8_e4m3" if case.get("fp8") else "bf16",
+                       kv_dtype=case.get("dtype", "fp8_e4m3" if case.get("fp8") else "bf16"),
                        paged=case.get("paged", False), page_size=case.get("page_size", 16),
                        window=case.get("window", -1), seed=11, unused_slot_fill="nan")
     out, lse = oracle.decode_all(x)
@@ -486,3 +489,86 @@ def test_softcap_limits_and_brute_force():
             w = np.exp(s - s.max())
             np.testing.assert_allclose(o[b, h], (w / w.sum()) @ vf[:, h // 2], rtol=0, atol=1e-12)
             assert abs(l[b, h] - (s.max() + math.log(w.sum()))) < 1e-12
+
+
+# ---------------------------------------------------------------- int4 KV
+def test_int4_nibble_decoding_by_hand():
+    """Two's-complement nibbles, the even element in the low nibble (the
+    reading of INT4 KV on "Beyond the Memory Wall", section "2. FlashInfer",
+    which names the format without its layout)."""
+    table = {0x00: (0, 0), 0x7F: (-1, 7), 0x80: (0, -8), 0x19: (-7, 1), 0xF8: (-8, -1),
+             0x07: (7, 0), 0x88: (-8, -8), 0x21: (1, 2)}
+    got = oracle.int4_codes(np.array([list(table)], np.uint8))[0]
+    assert list(got) == [c for pair in table.values() for c in pair]
+    assert np.array_equal(int4_values(np.array(list(table), np.uint8)), got.astype(np.float64))
+
+
+def _int4_pack_by_hand(codes):
+    """[..., d] ints in [-8, 7] -> bytes, element 2i low nibble of byte i."""
+    c = np.asarray(codes, np.int64) % 16
+    return (c[..., 0::2] + 16 * c[..., 1::2]).astype(np.uint8)
+
+
+def _int4_inputs(qv, kc, vc, lens, k_scale, v_scale, sm_scale=1.0, window=-1):
+    x = contiguous_inputs(qv, np.zeros(kc.shape, np.float32), np.zeros(vc.shape, np.float32), lens,
+                          sm_scale=sm_scale, window=window)
+    return DecodeInputs(**{**x.__dict__, "kv_dtype": "int4", "k": _int4_pack_by_hand(kc),
+                           "v": _int4_pack_by_hand(vc),
+                           "k_scale": np.asarray(k_scale, np.float32),
+                           "v_scale": np.asarray(v_scale, np.float32)})
+
+
+def test_int4_constant_keys_and_scales():
+    """All K codes equal: every score equal, out = mean of the dequantised V
+    rows (codes x the head's V scale), lse = score + ln |J|; the scales are
+    per kv head and separate for K and V."""
+    rng = np.random.default_rng(4)
+    L, d = 77, 8
+    qv = rng.integers(-4, 5, size=(1, 4, d)).astype(np.float32)
+    kc = np.empty((L, 2, d), np.int64)
+    kc[:, 0], kc[:, 1] = 3, -5
+    vc = rng.integers(-8, 8, size=(L, 2, d))
+    ks, vs = [0.5, 0.25], [0.125, 2.0]
+    for window in (-1, 9):
+        out, lse = oracle.decode_all(_int4_inputs(qv, kc, vc, [L], ks, vs, 0.5, window))
+        lo = L - window if window > 0 else 0
+        for h in range(4):
+            g = h // 2
+            np.testing.assert_allclose(out[0, h], vc[lo:, g].mean(axis=0) * vs[g], atol=1e-12)
+            s = 0.5 * float(qv[0, h] @ np.full(d, kc[0, g, 0])) * ks[g]
+            assert abs(lse[0, h] - (s + math.log(L - lo))) < 1e-12
+
+
+def test_int4_spike_pins_the_nibble_and_head():
+    """One key holds code 7 at an odd dimension (a high nibble) of kv head 1;
+    q is one-hot there, the K scale makes that score 40 and every other 0:
+    out = that key's V row to within n e^-40.  The same code placed at the
+    neighbouring even dimension (the low nibble of the same byte) scores 0."""
+    L, d = 64, 8
+    q = np.zeros((1, 4, d), np.float32)
+    q[0, :, 3] = 1.0
+    vc = np.random.default_rng(5).integers(-8, 8, size=(L, 2, d))
+    for dim, hit in ((3, True), (2, False)):
+        kc = np.zeros((L, 2, d), np.int64)
+        kc[41, 1, dim] = 7
+        out, lse = oracle.decode_all(_int4_inputs(q, kc, vc, [L], [1.0, 40.0 / 7.0], [1.0, 0.5]))
+        if hit:
+            np.testing.assert_allclose(out[0, 2], vc[41, 1] * 0.5, atol=1e-12)
+            s = 7.0 * float(np.float32(40.0 / 7.0))  # the stored fp32 scale
+            assert abs(lse[0, 3] - (s + math.log1p((L - 1) * math.exp(-s)))) < 1e-12
+        else:
+            np.testing.assert_allclose(out[0, 2], vc[:, 1].mean(axis=0) * 0.5, atol=1e-12)
+            assert abs(lse[0, 3] - math.log(L)) < 1e-12
+        np.testing.assert_allclose(out[0, 0], vc[:, 0].mean(axis=0), atol=1e-12)  # kv head 0
+
+
+def test_int4_quantised_inputs_follow_the_recipe():
+    """synth's INT4 inputs decode (by the independent numpy decoder) to
+    integers in [-7, 7] times a per-head scale of amax / 7: the largest code
+    of every head has magnitude 7."""
+    x = synth.generate(1, 4, 2, 16, [300], kv_dtype="int4", seed=12)
+    for arr in (x.k, x.v):
+        codes = int4_values(arr)
+        assert codes.min() >= -7 and codes.max() <= 7
+        assert (np.abs(codes).max(axis=(0, 2)) == 7).all()
+
