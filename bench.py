@@ -54,6 +54,8 @@ SWEEP = ["gqa4_d64_L512", "gemma3_1b_global_L8192", "gemma3_1b_local_w512_L8192"
          "paged_b64_gqa4_q8_L512-16384", "llama2_7b_mha_q8_L32768",
          # query groups wider than 8 (row teams)
          "llama3_405b_tp8_gqa16_paged_b64_L512-16384",
+         # INT4 KV cache
+         "int4_gqa8_L131072", "int4_paged_b64_gqa4_L512-16384",
          # logit soft-capping
          "gemma2_2b_softcap50_L8192"]
 FALLBACK_HBM_GBS = 6650.0
@@ -161,9 +163,9 @@ class Runner:
         self.lib = binding.load_library()
         self.x = x
         bits = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device)
-        fp8 = x.kv_dtype == "fp8_e4m3"
+        quant = x.kv_dtype != "bf16"  # fp8 / int4 codes (bytes) with per-head scales
         self.q = bits(x.q)
-        if fp8:
+        if quant:
             self.k = torch.from_numpy(np.ascontiguousarray(x.k)).to(device)
             self.v = torch.from_numpy(np.ascontiguousarray(x.v)).to(device)
             self.ks = torch.from_numpy(x.k_scale).to(device)
@@ -176,7 +178,8 @@ class Runner:
         self.ind_host = np.ascontiguousarray(x.kv_indptr, dtype=np.int32)
         self.desc = binding.DecodeDesc(
             batch=x.batch, qo_heads=x.qo_heads, kv_heads=x.kv_heads, head_dim=x.head_dim,
-            kv_dtype=1 if fp8 else 0, paged=int(x.paged), page_size=int(x.page_size),
+            kv_dtype={"bf16": 0, "fp8_e4m3": 1, "int4": 2}[x.kv_dtype], paged=int(x.paged),
+            page_size=int(x.page_size),
             window=int(x.window), sm_scale=float(x.sm_scale),
             path={"auto": 0, "simt": 1, "mma": 2}[path], num_ctas=0, q_len=int(x.q_len),
             logit_cap=float(x.logit_cap))
@@ -253,20 +256,20 @@ def e2e_measure(x, runner, steps):
     timed region."""
     import torch
     hq = torch.from_numpy(np.ascontiguousarray(x.q).view(np.int16)).pin_memory()
-    fp8 = x.kv_dtype == "fp8_e4m3"
-    conv = (lambda a: torch.from_numpy(np.ascontiguousarray(a))) if fp8 else \
+    quant = x.kv_dtype != "bf16"
+    conv = (lambda a: torch.from_numpy(np.ascontiguousarray(a))) if quant else \
         (lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)))
     hk, hv = conv(x.k).pin_memory(), conv(x.v).pin_memory()
     hind = torch.from_numpy(x.kv_indptr).pin_memory()
     hpt = torch.from_numpy(x.page_table).pin_memory() if x.paged else None
-    hks = torch.from_numpy(x.k_scale).pin_memory() if fp8 else None
-    hvs = torch.from_numpy(x.v_scale).pin_memory() if fp8 else None
+    hks = torch.from_numpy(x.k_scale).pin_memory() if quant else None
+    hvs = torch.from_numpy(x.v_scale).pin_memory() if quant else None
     out_h = torch.empty(runner.out.shape, dtype=runner.out.dtype).pin_memory()
     lse_h = torch.empty(runner.lse.shape, dtype=runner.lse.dtype).pin_memory()
     pairs = [(runner.q, hq), (runner.k, hk), (runner.v, hv), (runner.ind, hind)]
     if hpt is not None:
         pairs.append((runner.pt, hpt))
-    if fp8:
+    if quant:
         pairs += [(runner.ks, hks), (runner.vs, hvs)]
     h2d = sum(h.numel() * h.element_size() for _, h in pairs)
     d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
@@ -513,7 +516,7 @@ def main():
         line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "bf16" if x.kv_dtype == "bf16" else "fp8_e4m3",
+                "dtype": x.kv_dtype,
                 "data": "synthetic", "config": workload_config(x, world),
                 "tokens_per_s": round(tokens, 1), "frac_of_peak": round(value / world / peak, 4),
                 "path": "mma" if runner.info["path"] == 2 else "simt",

@@ -18,7 +18,8 @@ import numpy as np
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_NAME = "libfadecode.so"
 
-KV_BF16, KV_FP8_E4M3 = 0, 1
+KV_BF16, KV_FP8_E4M3, KV_INT4 = 0, 1, 2
+_KV_DTYPES = {"bf16": KV_BF16, "fp8_e4m3": KV_FP8_E4M3, "int4": KV_INT4}
 PATH_AUTO, PATH_SIMT, PATH_MMA = 0, 1, 2
 _PATH_NAMES = {"auto": PATH_AUTO, "simt": PATH_SIMT, "mma": PATH_MMA}
 
@@ -170,7 +171,7 @@ def plan(batch: int, qo_heads: int, kv_heads: int, head_dim: int, kv_indptr_host
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(head_dim)
     desc = DecodeDesc(batch=batch, qo_heads=qo_heads, kv_heads=kv_heads, head_dim=head_dim,
-                      kv_dtype=KV_FP8_E4M3 if kv_dtype == "fp8_e4m3" else KV_BF16,
+                      kv_dtype=_KV_DTYPES[kv_dtype],
                       paged=int(bool(paged)), page_size=int(page_size), window=int(window),
                       sm_scale=float(sm_scale), path=_PATH_NAMES[path], num_ctas=int(num_ctas),
                       q_len=int(q_len), logit_cap=float(logit_cap))

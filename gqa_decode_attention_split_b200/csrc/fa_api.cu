@@ -35,11 +35,11 @@ void build_registry() {
   g_num_entries = n;
 }
 
-const KernelEntry* find_entry(int head_dim, int group, int fp8, int path) {
+const KernelEntry* find_entry(int head_dim, int group, int kv_kind, int path) {
   std::call_once(g_registry_once, build_registry);
   for (int i = 0; i < g_num_entries; ++i) {
     const KernelEntry& e = g_entries[i];
-    if (e.head_dim != head_dim || e.fp8 != fp8 || e.path != path) continue;
+    if (e.head_dim != head_dim || e.kv_kind != kv_kind || e.path != path) continue;
     if (e.group != 0 ? e.group == group : group <= e.max_group) return &e;
   }
   return nullptr;
@@ -117,7 +117,9 @@ fa_status validate_desc(const fa_decode_desc* d) {
   if (d->batch < 1 || d->qo_heads < 1 || d->kv_heads < 1 || d->head_dim < 1)
     return FA_ERR_INVALID_ARG;
   if (d->qo_heads % d->kv_heads != 0) return FA_ERR_INVALID_ARG;
-  if (d->kv_dtype != FA_KV_BF16 && d->kv_dtype != FA_KV_FP8_E4M3) return FA_ERR_INVALID_ARG;
+  if (d->kv_dtype != FA_KV_BF16 && d->kv_dtype != FA_KV_FP8_E4M3 && d->kv_dtype != FA_KV_INT4)
+    return FA_ERR_INVALID_ARG;
+  if (d->kv_dtype == FA_KV_INT4 && d->head_dim % 2 != 0) return FA_ERR_INVALID_ARG;
   if (d->paged != 0 && d->paged != 1) return FA_ERR_INVALID_ARG;
   if (d->paged && (d->page_size < 1 || d->page_size > 256 || ilog2_exact(d->page_size) < 0))
     return FA_ERR_INVALID_ARG;
@@ -131,6 +133,12 @@ fa_status validate_desc(const fa_decode_desc* d) {
 }
 
 int32_t q_len_of(const fa_decode_desc* d) { return d->q_len > 1 ? d->q_len : 1; }
+
+// Bytes of one token's K (or V) row of one kv head.
+int64_t row_bytes_of(const fa_decode_desc* d) {
+  const int64_t D = d->head_dim;
+  return d->kv_dtype == FA_KV_BF16 ? 2 * D : (d->kv_dtype == FA_KV_FP8_E4M3 ? D : D / 2);
+}
 
 // Keys that some query token of a request sees: the last token's window and
 // the q_len - 1 keys before it (<= 0: all keys).
@@ -161,7 +169,8 @@ std::vector<fa_tuning_entry>& tuning_table() {
 }
 
 bool valid_tuning_row(const fa_tuning_entry& e) {
-  return e.head_dim > 0 && (e.kv_dtype == FA_KV_BF16 || e.kv_dtype == FA_KV_FP8_E4M3) &&
+  return e.head_dim > 0 &&
+         (e.kv_dtype == FA_KV_BF16 || e.kv_dtype == FA_KV_FP8_E4M3 || e.kv_dtype == FA_KV_INT4) &&
          e.rows_min >= 1 && e.rows_min <= e.rows_max && e.bytes_min >= 0 &&
          e.bytes_min <= e.bytes_max && (e.path == FA_PATH_SIMT || e.path == FA_PATH_MMA) &&
          e.max_pieces >= 0 && e.max_pieces <= 1024;
@@ -176,8 +185,7 @@ int64_t visible_kv_bytes(const fa_decode_desc* d, const int32_t* indptr) {
     const int64_t L = indptr[b + 1] - indptr[b];
     toks += (wu > 0 && L > wu) ? wu : L;
   }
-  const int64_t row = static_cast<int64_t>(d->head_dim) * (d->kv_dtype == FA_KV_FP8_E4M3 ? 1 : 2);
-  return toks * d->kv_heads * 2 * row;
+  return toks * d->kv_heads * 2 * row_bytes_of(d);
 }
 
 }  // namespace
@@ -220,7 +228,7 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   }
   // rows of a segment: the group's query heads for every query token
   const int group = desc->qo_heads / desc->kv_heads * q_len_of(desc);
-  const int fp8 = desc->kv_dtype == FA_KV_FP8_E4M3 ? 1 : 0;
+  const int kind = desc->kv_dtype;  // registry kinds follow fa_kv_dtype
 
   // Dataflow choice.  Asked for: that dataflow.  Otherwise the first row of
   // the measured table that covers the shape (when the grid is not forced),
@@ -229,9 +237,9 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   const KernelEntry* k = nullptr;
   int64_t max_pieces = 32;  // average blocks per segment, at most
   if (desc->path == FA_PATH_SIMT) {
-    k = find_entry(desc->head_dim, group, fp8, fa::kPathSimt);
+    k = find_entry(desc->head_dim, group, kind, fa::kPathSimt);
   } else if (desc->path == FA_PATH_MMA) {
-    k = find_entry(desc->head_dim, group, fp8, fa::kPathMma);
+    k = find_entry(desc->head_dim, group, kind, fa::kPathMma);
   } else {
     if (desc->num_ctas == 0) {
       const int64_t bytes = visible_kv_bytes(desc, kv_indptr_host);
@@ -239,14 +247,14 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
         if (e.head_dim != desc->head_dim || e.kv_dtype != desc->kv_dtype || group < e.rows_min ||
             group > e.rows_max || bytes < e.bytes_min || bytes > e.bytes_max)
           continue;
-        k = find_entry(desc->head_dim, group, fp8, e.path == FA_PATH_SIMT ? fa::kPathSimt : fa::kPathMma);
+        k = find_entry(desc->head_dim, group, kind, e.path == FA_PATH_SIMT ? fa::kPathSimt : fa::kPathMma);
         if (k == nullptr) continue;
         if (e.max_pieces > 0) max_pieces = e.max_pieces;
         break;
       }
     }
-    if (k == nullptr) k = find_entry(desc->head_dim, group, fp8, fa::kPathMma);
-    if (k == nullptr) k = find_entry(desc->head_dim, group, fp8, fa::kPathSimt);
+    if (k == nullptr) k = find_entry(desc->head_dim, group, kind, fa::kPathMma);
+    if (k == nullptr) k = find_entry(desc->head_dim, group, kind, fa::kPathSimt);
   }
   if (k == nullptr) return FA_ERR_UNSUPPORTED;
 
@@ -308,6 +316,14 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   p->max_partials = P + segs;
   p->page_shift = desc->paged ? ilog2_exact(desc->page_size) : 0;
   p->box_t = desc->paged ? (desc->page_size < T ? desc->page_size : T) : T;
+  // A tile is filled box by box (one box per page when pages are shorter
+  // than a tile) and a bulk tensor copy must land on a 128-byte boundary of
+  // shared memory: rows narrower than 128 bytes (int4 at head_dim 128) need
+  // pages of at least 128 / row-bytes tokens.
+  if ((static_cast<int64_t>(p->box_t) * k->row_bytes) % 128 != 0) {
+    delete p;
+    return FA_ERR_UNSUPPORTED;
+  }
   // 128B swizzle needs every copy to start on a 1024-byte boundary of the
   // tile: whole 8-line groups of 128-byte lines per copy.
   {
@@ -368,8 +384,8 @@ fa_status make_kv_map(const fa_plan* p, const void* base, int64_t kv_rows, CUten
   }
   const fa_decode_desc& d = p->desc;
   const KernelEntry* k = p->kernel;
-  const int es = d.kv_dtype == FA_KV_FP8_E4M3 ? 1 : 2;
-  const cuuint64_t row = static_cast<cuuint64_t>(d.head_dim) * es;
+  const int es = d.kv_dtype == FA_KV_BF16 ? 2 : 1;  // int4: bytes of two codes
+  const cuuint64_t row = static_cast<cuuint64_t>(row_bytes_of(&d));
   const cuuint64_t cb = static_cast<cuuint64_t>(k->plane_bytes);
   const cuuint64_t np = row / cb;
   const CUtensorMapDataType dt = es == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
@@ -379,8 +395,9 @@ fa_status make_kv_map(const fa_plan* p, const void* base, int64_t kv_rows, CUten
   // L2 fills no wider than a token row: a 256-byte fill of a 128-byte row
   // would pull in the next kv head's row, which another block reads much
   // later (measured 1.48x DRAM traffic on 128-byte fp8 rows).
-  const CUtensorMapL2promotion promo =
-      row >= 256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_L2_128B;
+  const CUtensorMapL2promotion promo = row >= 256   ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+                                      : row >= 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
+                                                   : CU_TENSOR_MAP_L2_PROMOTION_NONE;
   CUresult r;
   if (k->token_major) {
     // [.. rows][kv_heads][planes][plane elements]: one copy carries whole rows
@@ -444,9 +461,9 @@ extern "C" fa_status fa_decode_run(const fa_plan* plan, const void* q, const voi
       out == nullptr || workspace == nullptr)
     return FA_ERR_INVALID_ARG;
   const fa_decode_desc& d = plan->desc;
-  const bool fp8 = d.kv_dtype == FA_KV_FP8_E4M3;
+  const bool quant = d.kv_dtype != FA_KV_BF16;  // fp8 / int4 codes with per-head scales
   if (d.paged && (page_table == nullptr || page_table_stride < 1)) return FA_ERR_INVALID_ARG;
-  if (fp8 && (k_scale == nullptr || v_scale == nullptr)) return FA_ERR_INVALID_ARG;
+  if (quant && (k_scale == nullptr || v_scale == nullptr)) return FA_ERR_INVALID_ARG;
   if (kv_rows < 1 || kv_rows > INT32_MAX) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
       !aligned(workspace, 256) || !aligned(kv_indptr, 4) || (lse && !aligned(lse, 4)) ||
@@ -464,8 +481,8 @@ extern "C" fa_status fa_decode_run(const fa_plan* plan, const void* q, const voi
   a.q = static_cast<const uint16_t*>(q);
   a.kv_indptr = kv_indptr;
   a.page_table = d.paged ? page_table : nullptr;
-  a.k_scale = fp8 ? k_scale : nullptr;
-  a.v_scale = fp8 ? v_scale : nullptr;
+  a.k_scale = quant ? k_scale : nullptr;
+  a.v_scale = quant ? v_scale : nullptr;
   a.out = static_cast<uint16_t*>(out);
   a.lse = lse;
   a.status = reinterpret_cast<uint32_t*>(ws);

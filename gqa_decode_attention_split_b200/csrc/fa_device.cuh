@@ -121,6 +121,11 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
                : "r"(addr));
   return v;
 }
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -196,6 +201,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+// Two int4 codes -> f16x2, exact: bits 0-3 of x give the low half, bits
+// 16-19 the high half, each a two's-complement nibble c.  The f16 with bit
+// pattern 0x6400 | u is 1024 + u for u < 1024 (the unit in the last place
+// of 1024 is 1), so (nibble ^ 8) = c + 8 placed under 0x6400 reads 1032 + c;
+// one f16x2 subtraction of 1032 leaves c.
+__device__ __forceinline__ uint32_t int4x2_to_f16x2(uint32_t x) {
+  const uint32_t biased = (x & 0x000F000Fu) ^ 0x64086408u;
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(biased), "r"(0x64086408u));
+  return r;
 }
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t r;

@@ -2,5 +2,5 @@
 #include "fa_instantiate.cuh"
 
 namespace fa {
-int register_d128(KernelEntry* out, int cap) { return register_bf16_and_fp8<128>(out, cap, true); }
+int register_d128(KernelEntry* out, int cap) { return register_variants<128>(out, cap, true); }
 }  // namespace fa

@@ -2,5 +2,5 @@
 #include "fa_instantiate.cuh"
 
 namespace fa {
-int register_d256(KernelEntry* out, int cap) { return register_bf16_and_fp8<256>(out, cap, true); }
+int register_d256(KernelEntry* out, int cap) { return register_variants<256>(out, cap, true); }
 }  // namespace fa

@@ -2,5 +2,5 @@
 #include "fa_instantiate.cuh"
 
 namespace fa {
-int register_d64(KernelEntry* out, int cap) { return register_bf16_and_fp8<64>(out, cap, true); }
+int register_d64(KernelEntry* out, int cap) { return register_variants<64>(out, cap, true); }
 }  // namespace fa

@@ -49,13 +49,13 @@ size_t smem_bytes_for(int batch, int group) {
 }
 
 template <class Cons>
-KernelEntry make_entry(int path, int group, int max_group, int fp8) {
+KernelEntry make_entry(int path, int group, int max_group, int kv_kind) {
   using C = typename Cons::C;
   KernelEntry e;
-  e.head_dim = C::ROWB / C::ES;
+  e.head_dim = C::DIM;
   e.group = group;
   e.max_group = max_group;
-  e.fp8 = fp8;
+  e.kv_kind = kv_kind;
   e.path = path;
   e.tile_tokens = C::T;
   e.stages = C::KSTAGES;
@@ -70,28 +70,32 @@ KernelEntry make_entry(int path, int group, int max_group, int fp8) {
 }
 
 template <int D>
-int register_bf16_and_fp8(KernelEntry* out, int cap, bool with_fp8) {
+int register_variants(KernelEntry* out, int cap, bool with_quant) {
   int n = 0;
   auto add = [&](const KernelEntry& e) {
     if (n < cap) out[n++] = e;
   };
   // tensor-core variants in order of rows (the planner takes the first that
   // holds a segment's rows): one, two and four row teams of 8
-  add(make_entry<MmaConsumer<D, false, 1>>(kPathMma, 0, 8, 0));
-  add(make_entry<MmaConsumer<D, false, 2>>(kPathMma, 0, 16, 0));
-  add(make_entry<MmaConsumer<D, false, 4>>(kPathMma, 0, 32, 0));
-  add(make_entry<SimtConsumer<D, 1, false>>(kPathSimt, 1, 1, 0));
-  add(make_entry<SimtConsumer<D, 2, false>>(kPathSimt, 2, 2, 0));
-  add(make_entry<SimtConsumer<D, 4, false>>(kPathSimt, 4, 4, 0));
-  add(make_entry<SimtConsumer<D, 8, false>>(kPathSimt, 8, 8, 0));
+  add(make_entry<MmaConsumer<D, kKvBf16, 1>>(kPathMma, 0, 8, kKvBf16));
+  add(make_entry<MmaConsumer<D, kKvBf16, 2>>(kPathMma, 0, 16, kKvBf16));
+  add(make_entry<MmaConsumer<D, kKvBf16, 4>>(kPathMma, 0, 32, kKvBf16));
+  add(make_entry<SimtConsumer<D, 1, false>>(kPathSimt, 1, 1, kKvBf16));
+  add(make_entry<SimtConsumer<D, 2, false>>(kPathSimt, 2, 2, kKvBf16));
+  add(make_entry<SimtConsumer<D, 4, false>>(kPathSimt, 4, 4, kKvBf16));
+  add(make_entry<SimtConsumer<D, 8, false>>(kPathSimt, 8, 8, kKvBf16));
   if constexpr (D >= 128) {
-    if (with_fp8) {
-      add(make_entry<MmaConsumer<D, true, 1>>(kPathMma, 0, 8, 1));
-      add(make_entry<MmaConsumer<D, true, 2>>(kPathMma, 0, 16, 1));
-      add(make_entry<MmaConsumer<D, true, 4>>(kPathMma, 0, 32, 1));
-      add(make_entry<SimtConsumer<D, 1, true>>(kPathSimt, 1, 1, 1));
-      add(make_entry<SimtConsumer<D, 2, true>>(kPathSimt, 2, 2, 1));
-      add(make_entry<SimtConsumer<D, 4, true>>(kPathSimt, 4, 4, 1));
+    if (with_quant) {
+      add(make_entry<MmaConsumer<D, kKvFp8, 1>>(kPathMma, 0, 8, kKvFp8));
+      add(make_entry<MmaConsumer<D, kKvFp8, 2>>(kPathMma, 0, 16, kKvFp8));
+      add(make_entry<MmaConsumer<D, kKvFp8, 4>>(kPathMma, 0, 32, kKvFp8));
+      add(make_entry<SimtConsumer<D, 1, true>>(kPathSimt, 1, 1, kKvFp8));
+      add(make_entry<SimtConsumer<D, 2, true>>(kPathSimt, 2, 2, kKvFp8));
+      add(make_entry<SimtConsumer<D, 4, true>>(kPathSimt, 4, 4, kKvFp8));
+      // int4 KV: tensor-core dataflow only
+      add(make_entry<MmaConsumer<D, kKvInt4, 1>>(kPathMma, 0, 8, kKvInt4));
+      add(make_entry<MmaConsumer<D, kKvInt4, 2>>(kPathMma, 0, 16, kKvInt4));
+      add(make_entry<MmaConsumer<D, kKvInt4, 4>>(kPathMma, 0, 32, kKvInt4));
     }
   }
   return n;

@@ -133,10 +133,15 @@ constexpr int kScaleCap = 128;         // fp8 per-kv-head scales kept in shared 
 // are taken (EARLY_K) holds V longer than K, so the V ring gets the extra
 // slots: a slot is refilled only after its warps release it, and a slot
 // held through the tile's math is a slot with no copy in flight.
-template <int D, bool FP8, int GW, int R, int TILE_BYTES_TARGET, int NWARPS, bool EARLY_K>
+// KV element kinds: bf16, fp8 e4m3, int4 (two codes per byte).
+enum : int { kKvBf16 = 0, kKvFp8 = 1, kKvInt4 = 2 };
+
+template <int D, int KIND, int GW, int R, int TILE_BYTES_TARGET, int NWARPS, bool EARLY_K>
 struct TileCfg {
-  static constexpr int ES = FP8 ? 1 : 2;
-  static constexpr int ROWB = D * ES;
+  static constexpr int DIM = D;
+  static constexpr bool QUANT = KIND != kKvBf16;  // codes with per-kv-head scales
+  static constexpr int ES = KIND == kKvBf16 ? 2 : 1;  // bytes per tensor-map element
+  static constexpr int ROWB = KIND == kKvBf16 ? 2 * D : (KIND == kKvFp8 ? D : D / 2);
   static constexpr int CB = ROWB < 128 ? ROWB : 128;
   static constexpr int NP = ROWB / CB;
   static constexpr int T_RAW = TILE_BYTES_TARGET / ROWB;
@@ -154,7 +159,7 @@ struct TileCfg {
   // Query rows are staged only where the slots cost no ring stage; otherwise
   // consumers read them from global memory.
   static constexpr int QSLOT_BYTES = GMAX * D * 2;
-  static constexpr int SCALE_BYTES = FP8 ? 2 * kScaleCap * 4 : 0;
+  static constexpr int SCALE_BYTES = QUANT ? 2 * kScaleCap * 4 : 0;
   // (1024: base alignment; 272: merge counter, merge mbarrier, 64 page ids)
   static constexpr int BASE_BUDGET = kSmemPerBlock - 1024 - kSchedReserve - 272 - MERGE_BYTES - 32 - SCALE_BYTES;
   // K + V tiles per tile lane that fit (a tile slot costs its bytes plus two
@@ -253,6 +258,15 @@ __device__ __forceinline__ uint4 lds128_in(uint32_t* status, uint32_t addr, uint
   return lds128(addr);
 }
 
+// Shared-memory 8-byte load that stays inside [tile, tile + bytes).
+__device__ __forceinline__ uint2 lds64_in(uint32_t* status, uint32_t addr, uint32_t tile,
+                                          uint32_t bytes, uint32_t code) {
+  if (!FA_CHECK(status, addr >= tile && addr + 8 <= tile + bytes && (addr & 7u) == 0, code,
+                static_cast<long long>(addr) - tile))
+    return make_uint2(0, 0);
+  return lds64(addr);
+}
+
 // ------------------------------------------------------------ schedule
 struct Piece {
   int b, h;          // request, kv head
@@ -326,7 +340,7 @@ __device__ __forceinline__ bool next_piece(PieceIter& it, Piece& pc, const int* 
 // running softmax state, merged across slots at the end of a segment piece.
 template <int D, int G, bool FP8>
 struct SimtConsumer {
-  using C = TileCfg<D, FP8, G, 1, FA_SIMT_TILE_BYTES, FA_SIMT_CONSUMER_WARPS, false>;
+  using C = TileCfg<D, FP8 ? kKvFp8 : kKvBf16, G, 1, FA_SIMT_TILE_BYTES, FA_SIMT_CONSUMER_WARPS, false>;
   static constexpr int EPC = 16 / C::ES;
   static constexpr int NCH = C::ROWB / 16;
   static constexpr int E_TARGET = 64 / G;
@@ -579,31 +593,41 @@ struct SimtConsumer {
 // heads of a kv head times the query tokens).  A team's warp computes its 8
 // rows of every tile it takes; with more than one team the bf16 tiles are
 // 32 tokens, so that the fewer tile lanes still keep a deep ring.
-template <int D, bool FP8, int R = 1>
+// KIND: bf16 (tiles through ldmatrix), fp8 e4m3 or int4 (bytes loaded per
+// lane and widened to f16; the query is held as f16 times a power of two).
+template <int D, int KIND, int R = 1>
 struct MmaConsumer {
-  static constexpr int kTileBytes =
-      FP8 ? FA_FP8_MMA_TILE_BYTES : (R == 1 ? FA_MMA_TILE_BYTES : FA_MMA_TILE_BYTES / 2);
+  static constexpr bool FP8 = KIND == kKvFp8;
+  static constexpr bool I4 = KIND == kKvInt4;
+  static constexpr bool BF16 = KIND == kKvBf16;
+  static constexpr int kTileBytes = FP8 ? FA_FP8_MMA_TILE_BYTES
+                                    : I4  ? FA_FP8_MMA_TILE_BYTES / 2
+                                          : (R == 1 ? FA_MMA_TILE_BYTES : FA_MMA_TILE_BYTES / 2);
   // Consumer warps: two teams of 3, or four of 2 (a 9-warp block, whose
   // registers are capped at 168 per thread); fp8 rows of 256 dims need more
   // registers than that and take four teams of one warp.
-  static constexpr int kWarps = R == 1   ? (FP8 ? FA_FP8_MMA_CONSUMER_WARPS : FA_MMA_CONSUMER_WARPS)
+  static constexpr int kWarps = R == 1   ? (!BF16 ? FA_FP8_MMA_CONSUMER_WARPS : FA_MMA_CONSUMER_WARPS)
                                 : R == 2 ? 6
-                                         : (FP8 && D >= 256 ? 4 : 8);
+                                         : (!BF16 && D >= 256 ? 4 : 8);
   // V held longer than K (EARLY_K: one K slot per two V slots) pays where
   // the V half of a tile is the longer one, fp8 with one team; elsewhere
   // equal rings keep the most tiles in flight.
-  using C = TileCfg<D, FP8, 8, R, kTileBytes, kWarps, FP8 && R == 1>;
+  using C = TileCfg<D, KIND, 8, R, kTileBytes, kWarps, !BF16 && R == 1>;
   static constexpr int KS = D / 16;     // k-steps of the score product = m-tiles of O^T
   static constexpr int SUB = C::T / 16;  // 16-token subtiles per tile
-  static constexpr int BPT = D / 4;      // fp8 K: bytes of a row owned by one lane
+  static constexpr int BPT = D / 4;      // fp8 / int4 K: elements of a row owned by one lane
   static constexpr bool kQSplit = FP8 && FA_FP8_QSPLIT;
   static constexpr int KS32 = D / 32;    // k-steps of the e4m3 score product
-  static constexpr int VBT = D / 8;      // fp8 V: bytes of a row owned by one lane
+  static constexpr int VBT = D / 8;      // fp8 / int4 V: elements of a row owned by one lane
+  static constexpr int KB = I4 ? BPT / 2 : BPT;  // their bytes
+  static constexpr int VB = I4 ? VBT / 2 : VBT;
   static_assert(D % 16 == 0 && C::T % 16 == 0, "mma tiling");
   static_assert(!FP8 || C::CB == 128, "fp8 mma path needs 128-byte planes");
+  static_assert(!I4 || ((D == 128 || D == 256) && KB % 16 == 0 && (VB == 8 || VB == 16)),
+                "int4 mma path: 64- or 128-byte rows");
 
   uint32_t qb[KS][2];
-  uint32_t qb8[KS32][3][2];  // e4m3 q parts (hi, mid, lo) per k-step
+  uint32_t qb8[kQSplit ? KS32 : 1][3][2];  // e4m3 q parts (hi, mid, lo) per k-step
   float o[KS][4];
   float m[2], l[2];
   float sscale[2];
@@ -624,7 +648,7 @@ struct MmaConsumer {
     const bool real = rbase + g < G;
     const int r = real ? rbase + g : 0;
     const uint16_t* qrow = qs + (r / a.group) * qstride + (r % a.group) * D;
-    if constexpr (!FP8) {
+    if constexpr (BF16) {
 #pragma unroll
       for (int kk = 0; kk < KS; ++kk) {
         qb[kk][0] = real ? *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * t) : 0u;
@@ -684,10 +708,21 @@ struct MmaConsumer {
         const float mul = ldexpf(1.f, sh);
 #pragma unroll
         for (int kk = 0; kk < KS; ++kk) {
-          // logical k-columns 2t,2t+1 / 2t+8,2t+9 of step kk <-> bytes BPT*t + 4kk + {0,1} / {2,3}
-          const uint32_t w0 = qw[2 * kk], w1 = qw[2 * kk + 1];
-          qb[kk][0] = pack_f16x2(bf16lo(w0) * mul, bf16hi(w0) * mul);
-          qb[kk][1] = pack_f16x2(bf16lo(w1) * mul, bf16hi(w1) * mul);
+          if constexpr (FP8) {
+            // logical k-columns 2t,2t+1 / 2t+8,2t+9 of step kk <-> bytes BPT*t + 4kk + {0,1} / {2,3}
+            const uint32_t w0 = qw[2 * kk], w1 = qw[2 * kk + 1];
+            qb[kk][0] = pack_f16x2(bf16lo(w0) * mul, bf16hi(w0) * mul);
+            qb[kk][1] = pack_f16x2(bf16lo(w1) * mul, bf16hi(w1) * mul);
+          } else {
+            // int4: logical k-columns 2t,2t+1 / 2t+8,2t+9 of step kk <-> the
+            // lane's elements (8j + 2c, 8j + 2c + 4) / (8j + 2c + 1, 8j + 2c + 5),
+            // j = kk / 2, c = kk % 2: the nibble pairs one shift and one mask
+            // take out of K's 32-bit word j
+            const int e = 8 * (kk >> 1) + 2 * (kk & 1);
+            auto qe = [&](int i) { return (i & 1) ? bf16hi(qw[i >> 1]) : bf16lo(qw[i >> 1]); };
+            qb[kk][0] = pack_f16x2(qe(e) * mul, qe(e + 4) * mul);
+            qb[kk][1] = pack_f16x2(qe(e + 1) * mul, qe(e + 5) * mul);
+          }
         }
       }
       const int sh0 = __shfl_sync(0xffffffffu, sh, (2 * t) * 4);
@@ -707,6 +742,14 @@ struct MmaConsumer {
   __device__ __forceinline__ uint32_t chunk_addr(uint32_t tile, int row, int chunk, int swz) const {
     return tile_addr<C>(tile, row, chunk >> 3, chunk & 7, swz);
   }
+  // Shared address of byte `off` of a tile row: swizzled 128-byte planes, or
+  // one unswizzled plane for rows narrower than 128 bytes.
+  __device__ __forceinline__ uint32_t byte_addr(uint32_t tile, int row, int off, int swz) const {
+    if constexpr (C::CB == 128)
+      return chunk_addr(tile, row, off >> 4, swz) + (off & 15);
+    else
+      return tile + row * C::ROWB + off;
+  }
 
   // Two accumulators (even / odd k-steps) halve the dependent chain of mma.
   __device__ __forceinline__ void scores(const KernelArgs& a, uint32_t kt, int sub, int lane,
@@ -714,7 +757,7 @@ struct MmaConsumer {
     const int swz = a.swz;
     float c2[4] = {0.f, 0.f, 0.f, 0.f};
     c[0] = c[1] = c[2] = c[3] = 0.f;
-    if constexpr (!FP8) {
+    if constexpr (BF16) {
       const int row = sub * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
       for (int kk = 0; kk < KS; ++kk) {
@@ -731,12 +774,12 @@ struct MmaConsumer {
       }
     } else {
       const int r0 = sub * 16 + g, r1 = r0 + 8;
-      uint32_t w0[BPT / 4], w1[BPT / 4];
+      uint32_t w0[KB / 4], w1[KB / 4];
 #pragma unroll
-      for (int i = 0; i < BPT / 16; ++i) {
-        const int ch = (BPT * t) / 16 + i;
-        const uint4 x0 = lds128_in(a.status, chunk_addr(kt, r0, ch, swz), kt, C::TILE_BYTES, 203);
-        const uint4 x1 = lds128_in(a.status, chunk_addr(kt, r1, ch, swz), kt, C::TILE_BYTES, 204);
+      for (int i = 0; i < KB / 16; ++i) {
+        const int off = KB * t + 16 * i;
+        const uint4 x0 = lds128_in(a.status, byte_addr(kt, r0, off, swz), kt, C::TILE_BYTES, 203);
+        const uint4 x1 = lds128_in(a.status, byte_addr(kt, r1, off, swz), kt, C::TILE_BYTES, 204);
         w0[4 * i] = x0.x; w0[4 * i + 1] = x0.y; w0[4 * i + 2] = x0.z; w0[4 * i + 3] = x0.w;
         w1[4 * i] = x1.x; w1[4 * i + 1] = x1.y; w1[4 * i + 2] = x1.z; w1[4 * i + 3] = x1.w;
       }
@@ -753,6 +796,22 @@ struct MmaConsumer {
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) c2[i] += c3[i];
+      } else if constexpr (I4) {
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+          // word kk / 2 of each row; pairs (8c, 8c + 4) bits up: the nibble
+          // pairs of the lane's elements listed in begin_piece
+          const int sh = 8 * (kk & 1);
+          uint32_t af[4];
+          af[0] = int4x2_to_f16x2(w0[kk >> 1] >> sh);
+          af[1] = int4x2_to_f16x2(w1[kk >> 1] >> sh);
+          af[2] = int4x2_to_f16x2(w0[kk >> 1] >> (sh + 4));
+          af[3] = int4x2_to_f16x2(w1[kk >> 1] >> (sh + 4));
+          if (kk & 1)
+            mma_f16(c2, af, qb[kk][0], qb[kk][1]);
+          else
+            mma_f16(c, af, qb[kk][0], qb[kk][1]);
+        }
       } else {
 #pragma unroll
         for (int kk = 0; kk < KS; ++kk) {
@@ -842,7 +901,7 @@ struct MmaConsumer {
       l[0] += p0 + p2;
       l[1] += p1 + p3;
       uint32_t x0, x1, y0, y1;
-      if constexpr (FP8) {
+      if constexpr (!BF16) {  // the f16 product of the fp8 / int4 dataflow
         x0 = pack_f16x2(p0, p1);
         x1 = pack_f16x2(p2, p3);
         const float2 h0 = f16x2_to_float2(x0), h1 = f16x2_to_float2(x1);
@@ -868,7 +927,7 @@ struct MmaConsumer {
       const bool edge = __any_sync(0xffffffffu, !(e0 && e1 && e8 && e9));
       const uint32_t mk01 = (e0 ? 0x0000FFFFu : 0u) | (e1 ? 0xFFFF0000u : 0u);
       const uint32_t mk89 = (e8 ? 0x0000FFFFu : 0u) | (e9 ? 0xFFFF0000u : 0u);
-      if constexpr (!FP8) {
+      if constexpr (BF16) {
         const int vrow = sub * 16 + (lane & 7) + (lane >> 4) * 8;
 #pragma unroll
         for (int mt = 0; mt < KS; ++mt) {
@@ -886,6 +945,50 @@ struct MmaConsumer {
           }
           mma_bf16(o[mt], af, pb[sub][0], pb[sub][1]);
           mma_bf16(o[mt], af, pb[sub][2], pb[sub][3]);
+        }
+      } else if constexpr (I4) {
+        // lane owns dims [VBT*g, VBT*g + VBT) (VB bytes) of tokens 2t, 2t+1,
+        // 2t+8, 2t+9.  Bytes 2u, 2u+1 of two tokens' chunks, permuted into
+        // one word [tok0 byte 2u, tok0 byte 2u+1, tok1 byte 2u, tok1 byte
+        // 2u+1], give per shift of 0, 4, 8, 12 bits the f16 pair (tok0, tok1)
+        // of dims 4u, 4u+1, 4u+2, 4u+3: m-tile 2u + s takes dims 4u + 2s
+        // (row g) and 4u + 2s + 1 (row g + 8), as out_dim states.
+        const int rb = sub * 16 + 2 * t;
+        const int rows[4] = {rb, rb + 1, rb + 8, rb + 9};
+        uint32_t vw[4][VB / 4];
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+          if constexpr (VB == 8) {
+            const uint2 x = lds64_in(a.status, byte_addr(vt, rows[rr], VB * g, a.swz), vt, C::TILE_BYTES, 208);
+            vw[rr][0] = x.x;
+            vw[rr][1] = x.y;
+          } else {
+            const uint4 x = lds128_in(a.status, byte_addr(vt, rows[rr], VB * g, a.swz), vt, C::TILE_BYTES, 209);
+            vw[rr][0] = x.x;
+            vw[rr][1] = x.y;
+            vw[rr][2] = x.z;
+            vw[rr][3] = x.w;
+          }
+        }
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+          const int u = mt >> 1, sh = 8 * (mt & 1);
+          const uint32_t sel = (u & 1) ? 0x7632u : 0x5410u;
+          const uint32_t z01 = prmt(vw[0][u >> 1], vw[1][u >> 1], sel);
+          const uint32_t z89 = prmt(vw[2][u >> 1], vw[3][u >> 1], sel);
+          uint32_t af[4];
+          af[0] = int4x2_to_f16x2(z01 >> sh);
+          af[1] = int4x2_to_f16x2(z01 >> (sh + 4));
+          af[2] = int4x2_to_f16x2(z89 >> sh);
+          af[3] = int4x2_to_f16x2(z89 >> (sh + 4));
+          if (edge) {
+            af[0] &= mk01;
+            af[1] &= mk01;
+            af[2] &= mk89;
+            af[3] &= mk89;
+          }
+          mma_f16(o[mt], af, pb[sub][0], pb[sub][1]);
+          mma_f16(o[mt], af, pb[sub][2], pb[sub][3]);
         }
       } else {
         // lane owns dims [VBT*g, VBT*g + VBT) of tokens 2t, 2t+1, 2t+8, 2t+9
@@ -927,7 +1030,7 @@ struct MmaConsumer {
   }
 
   __device__ __forceinline__ int out_dim(int mt, int half) const {
-    if constexpr (FP8)
+    if constexpr (!BF16)
       return VBT * g + 2 * mt + half;
     else
       return mt * 16 + g + 8 * half;
@@ -973,7 +1076,7 @@ struct MmaConsumer {
 template <class Cons>
 struct SmemLayout {
   using C = typename Cons::C;
-  static constexpr int D = C::ROWB / C::ES;
+  static constexpr int D = C::DIM;
   static constexpr int kBars = C::RING_BYTES;
   static constexpr int kMerge = kBars + 2 * (C::KSTAGES + C::VSTAGES) * 8;
   __host__ __device__ static constexpr int acc_off(int G) {
@@ -1004,7 +1107,7 @@ __global__ void __maxnreg__(max_regs<Cons>())
     fa_decode_kernel(const __grid_constant__ KernelArgs a) {
   using C = typename Cons::C;
   using S = SmemLayout<Cons>;
-  constexpr int D = C::ROWB / C::ES;
+  constexpr int D = C::DIM;
   constexpr int T = C::T;
   constexpr int NW = C::NW;
   constexpr int NT = C::NT;  // tile lanes (NW / row teams)
@@ -1073,7 +1176,7 @@ __global__ void __maxnreg__(max_regs<Cons>())
     if (bad) atomicOr(a.status, kFlagBadIndptr);
   }
   const bool scales_in_smem = H <= kScaleCap;
-  if (C::ES == 1 && scales_in_smem) {
+  if (C::QUANT && scales_in_smem) {
     for (int i = tid; i < H; i += blockDim.x) {
       s_kscale[i] = __ldg(a.k_scale + i);
       s_vscale[i] = __ldg(a.v_scale + i);
@@ -1434,12 +1537,12 @@ __global__ void __maxnreg__(max_regs<Cons>())
           alive = false;
         }
       }
-      const float ks = C::ES == 1 ? (scales_in_smem ? s_kscale[pc.h] : __ldg(a.k_scale + pc.h)) : 1.f;
+      const float ks = C::QUANT ? (scales_in_smem ? s_kscale[pc.h] : __ldg(a.k_scale + pc.h)) : 1.f;
       cons.begin_piece(a, q_slots + qs * (C::QSLOT_BYTES / 2), GK * D, ks, lane, team);
       __syncwarp();
       if (lane == 0) mbar_arrive(qempty0 + 8 * qs);
     } else {
-      const float ks = C::ES == 1 ? (scales_in_smem ? s_kscale[pc.h] : __ldg(a.k_scale + pc.h)) : 1.f;
+      const float ks = C::QUANT ? (scales_in_smem ? s_kscale[pc.h] : __ldg(a.k_scale + pc.h)) : 1.f;
       cons.begin_piece(a,
                        a.q + (static_cast<size_t>(pc.b) * Q * a.qo_heads + static_cast<size_t>(pc.h) * GK) * D,
                        a.qo_heads * D, ks, lane, team);
@@ -1491,7 +1594,7 @@ __global__ void __maxnreg__(max_regs<Cons>())
     // of the next piece; the last warp to park merges the NW states, writes
     // the result (or the partial) and frees the area.  A warp waits only if
     // it finishes its share of the next piece before that merge is done.
-    const float vs = C::ES == 1 ? (scales_in_smem ? s_vscale[pc.h] : __ldg(a.v_scale + pc.h)) : 1.f;
+    const float vs = C::QUANT ? (scales_in_smem ? s_vscale[pc.h] : __ldg(a.v_scale + pc.h)) : 1.f;
     if (piece > 0 && alive) {
       const bool ok = __all_sync(0xffffffffu, mbar_wait(mfree, (piece - 1) & 1, kWaitLimitNs));
       if (!ok) {

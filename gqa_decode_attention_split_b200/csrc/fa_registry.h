@@ -15,7 +15,7 @@ struct KernelEntry {
   int head_dim;
   int group;        // SIMT: exact group size; MMA: 0 (any group <= max_group)
   int max_group;
-  int fp8;
+  int kv_kind;      // fa_kv_dtype: bf16, fp8 e4m3, int4
   int path;
   int tile_tokens;  // T
   int stages;       // K tile slots

@@ -334,6 +334,18 @@ def _c5():
                     name="fp8_gqa8_L131072")
 
 
+def _c5_int4():
+    """The long-context GQA-8 decode with an INT4 KV cache (half the bytes of
+    FP8; "Beyond the Memory Wall", section "2. FlashInfer")."""
+    return generate(1, 64, 8, 128, [131072], kv_dtype="int4", seed=5, name="int4_gqa8_L131072")
+
+
+def _c4_int4():
+    """The batch-64 paged decode with an INT4 KV cache."""
+    return generate(64, 32, 8, 128, c4_lengths(), paged=True, page_size=16, seed=4,
+                    kv_dtype="int4", name="int4_paged_b64_gqa4_L512-16384")
+
+
 WORKLOADS = {
     "gqa4_d64_L512": _c1,
     "gemma3_1b_global_L8192": _c2_global,
@@ -345,6 +357,8 @@ WORKLOADS = {
     "paged_b64_gqa4_L512-16384": _c4,
     "paged_b16_gqa4_L512-16384": _c4_small,
     "fp8_gqa8_L131072": _c5,
+    "int4_gqa8_L131072": _c5_int4,
+    "int4_paged_b64_gqa4_L512-16384": _c4_int4,
     "paged_b64_gqa4_q2_L512-16384": _c4_q2,
     "paged_b64_gqa4_q4_L512-16384": _c4_q(4),
     "paged_b64_gqa4_q8_L512-16384": _c4_q(8),

@@ -34,7 +34,11 @@
  *  - Errors are returned as fa_status; nothing aborts or traps.  Argument
  *    errors are detected on the host before any work is enqueued.
  *  - bf16 tensors are raw IEEE bfloat16 bit patterns (uint16); fp8 tensors
- *    are e4m3 "fn" codes (uint8: bias 7, no infinities).
+ *    are e4m3 "fn" codes (uint8: bias 7, no infinities); int4 tensors are
+ *    two's-complement 4-bit codes in [-8, 7], two per byte, the even element
+ *    of a row in the low nibble (a row of head_dim codes is head_dim / 2
+ *    bytes).  INT4 KV quantisation is named on "Beyond the Memory Wall",
+ *    section "2. FlashInfer", without a layout; this is the plainest one.
  */
 #ifndef FADECODE_H_
 #define FADECODE_H_
@@ -62,7 +66,9 @@ typedef enum {
   FA_ERR_DEVICE_CHECK = 6         /* a kernel recorded a device-side check  */
 } fa_status;
 
-typedef enum { FA_KV_BF16 = 0, FA_KV_FP8_E4M3 = 1 } fa_kv_dtype;
+/* K/V element type.  FP8 and INT4 codes carry one fp32 scale per kv head
+ * for K and one for V (k_scale, v_scale): element = code * scale. */
+typedef enum { FA_KV_BF16 = 0, FA_KV_FP8_E4M3 = 1, FA_KV_INT4 = 2 } fa_kv_dtype;
 
 /* Dataflow for the KV-tile math.  SIMT computes q.k with per-lane fp32 FMAs
  * and warp-shuffle reductions (a GEMV per head); MMA runs the two skinny
@@ -83,7 +89,7 @@ typedef struct {
   int32_t batch;      /* requests, >= 1                                       */
   int32_t qo_heads;   /* query heads per request                              */
   int32_t kv_heads;   /* kv heads; qo_heads % kv_heads == 0                   */
-  int32_t head_dim;   /* 64, 128 or 256 (fp8: 128 or 256)                     */
+  int32_t head_dim;   /* 64, 128 or 256 (fp8, int4: 128 or 256)               */
   int32_t kv_dtype;   /* fa_kv_dtype                                          */
   int32_t paged;      /* 0: contiguous (ragged) rows, 1: paged pool           */
   int32_t page_size;  /* paged only: tokens per page, a power of two <= 256  */
@@ -103,7 +109,8 @@ typedef struct {
                       /* itself, or the last `window` of them.  The rows of  */
                       /* a (request, kv head) segment, (qo_heads / kv_heads) */
                       /* * q_len, must be <= 32 on the MMA dataflow (SIMT:   */
-                      /* exactly 1, 2, 4 or 8; 1, 2 or 4 for fp8).           */
+                      /* exactly 1, 2, 4 or 8; 1, 2 or 4 for fp8; int4 runs  */
+                      /* on the MMA dataflow only).                          */
   float logit_cap;    /* 0: none.  c > 0: logit soft-capping, each scaled    */
                       /* score s becomes c * tanh(s / c) before the softmax  */
                       /* (Gemma 2's soft-cap, named on "FlashInfer x JAX via */
@@ -215,7 +222,8 @@ FA_API fa_status fa_get_tuning(fa_tuning_entry* out, int32_t cap, int32_t* n);
  *              [kv_indptr[b], kv_indptr[b+1]) (batch 1: rows 0..kv_len-1).
  *              paged: pools [kv_rows, page_size, kv_heads, head_dim] where
  *              kv_rows is the number of pages.  Element type per desc
- *              (bf16 or e4m3), 16-byte aligned.
+ *              (bf16, e4m3, or int4 with head_dim / 2 bytes per row),
+ *              16-byte aligned.
  *  kv_rows     contiguous: number of rows of k and v; paged: number of pages
  *              in each pool.  Reads never leave [0, kv_rows).
  *  page_table  paged only (else NULL): int32 [batch, page_table_stride];
@@ -224,8 +232,9 @@ FA_API fa_status fa_get_tuning(fa_tuning_entry* out, int32_t cap, int32_t* n);
  *              tokens are read.  An entry outside [0, kv_rows) reads zeros
  *              and sets FA_DEVICE_BAD_PAGE.
  *  kv_indptr   int32 [batch + 1], device copy of the plan's indptr.
- *  k_scale,    fp8 only (else NULL): fp32 [kv_heads]; a stored code c of kv
- *  v_scale     head g means e4m3(c) * scale[g].
+ *  k_scale,    fp8 and int4 only (else NULL): fp32 [kv_heads]; a stored
+ *  v_scale     code c of kv head g means e4m3(c) * scale[g] (fp8) or
+ *              c * scale[g] (int4).
  *  out         bf16 [batch, q_len, qo_heads, head_dim], 16-byte aligned.
  *  lse         fp32 [batch, q_len, qo_heads], natural log; NULL = do not
  *              write.  A query token with no visible key (a request shorter

@@ -22,7 +22,7 @@ class DeviceInputs:
         self.x = x
         bits = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device)
         self.q = bits(x.q)
-        if x.kv_dtype == "fp8_e4m3":
+        if x.kv_dtype != "bf16":  # fp8 / int4 codes (bytes) with per-head scales
             self.k = torch.from_numpy(np.ascontiguousarray(x.k)).to(device)
             self.v = torch.from_numpy(np.ascontiguousarray(x.v)).to(device)
             self.k_scale = torch.from_numpy(x.k_scale).to(device)

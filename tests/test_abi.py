@@ -318,7 +318,7 @@ def test_tuning_table_drives_the_auto_choice(lib):
 
 @pytest.mark.parametrize("bad", [dict(rows_min=0), dict(rows_min=5, rows_max=4),
                                  dict(bytes_min=10, bytes_max=9), dict(bytes_min=-1),
-                                 dict(path=0), dict(path=3), dict(kv_dtype=2),
+                                 dict(path=0), dict(path=3), dict(kv_dtype=3),
                                  dict(max_pieces=-1), dict(max_pieces=1025), dict(head_dim=0)])
 def test_tuning_table_rejects_bad_rows(lib, bad):
     before = binding.get_tuning()
@@ -358,3 +358,28 @@ def test_builtin_tuning_rows_take_effect(lib):
         if r["max_pieces"]:
             assert inf.num_ctas <= r["max_pieces"] * 8, r
         lib.fa_plan_destroy(h)
+
+
+def test_int4_plans(lib):
+    """INT4 KV runs on the MMA dataflow (head_dim 128 and 256, up to 32
+    rows); SIMT has no INT4 kernel, head_dim 64 has none, an odd head_dim is
+    not a whole number of bytes."""
+    st, h, _ = _plan(lib, _desc(kv_dtype=binding.KV_INT4), [0, 1000])
+    assert st == 0
+    inf = _info(lib, h)
+    assert inf.path == binding.PATH_MMA and inf.tile_tokens == 64  # 64-byte rows, 4 KB tiles
+    lib.fa_plan_destroy(h)
+    st, h, _ = _plan(lib, _desc(kv_dtype=binding.KV_INT4, head_dim=256, qo_heads=32, kv_heads=1),
+                     [0, 1000])
+    assert st == 0 and _info(lib, h).path == binding.PATH_MMA
+    lib.fa_plan_destroy(h)
+    # one-token pages of 64-byte rows: a copy would land off a 128-byte boundary
+    for kw, code in ((dict(path=binding.PATH_SIMT), 2), (dict(head_dim=64), 2),
+                     (dict(head_dim=127), 1), (dict(paged=1, page_size=1), 2)):
+        st, h, _ = _plan(lib, _desc(kv_dtype=binding.KV_INT4, **kw), [0, 1000])
+        assert st == code and not h.value, kw
+    for ps in (2, 16):
+        st, h, _ = _plan(lib, _desc(kv_dtype=binding.KV_INT4, paged=1, page_size=ps), [0, 1000])
+        assert st == 0
+        lib.fa_plan_destroy(h)
+

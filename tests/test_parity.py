@@ -17,10 +17,13 @@ PATHS = ["simt", "mma"]
 
 
 def _has_path(x, path):
-    g = x.group
+    """Whether a kernel exists: rows per segment (group x query tokens) of
+    1, 2, 4 or 8 on SIMT (fp8: up to 4; no int4), up to 32 on MMA."""
+    rows = x.group * x.q_len
     if path == "simt":
-        return g in (1, 2, 4, 8) and not (x.kv_dtype == "fp8_e4m3" and g == 8)
-    return g <= 8
+        return (x.kv_dtype != "int4" and rows in (1, 2, 4, 8)
+                and not (x.kv_dtype == "fp8_e4m3" and rows == 8))
+    return rows <= 32
 
 
 def _check(x, path="auto", num_ctas=0, what=""):
@@ -51,6 +54,16 @@ SMALL = [
                                                  "kv_dtype": "fp8_e4m3"}),
     ("paged8_fp8_win", 3, 8, 8, 128, [90, 8, 150], {"paged": True, "page_size": 8,
                                                      "kv_dtype": "fp8_e4m3", "window": 17}),
+    # INT4 KV (64-byte rows at head_dim 128, 128-byte rows at 256)
+    ("int4_gqa8", 1, 16, 2, 128, [1111], {"kv_dtype": "int4"}),
+    ("int4_gqa4_d256", 2, 8, 2, 256, [333, 64], {"kv_dtype": "int4"}),
+    ("int4_mha_win", 1, 4, 4, 128, [257], {"kv_dtype": "int4", "window": 100}),
+    ("int4_gqa3", 2, 6, 2, 128, [129, 300], {"kv_dtype": "int4"}),
+    ("paged16_int4", 4, 8, 2, 128, [40, 16, 1, 300], {"paged": True, "page_size": 16,
+                                                      "kv_dtype": "int4"}),
+    ("paged2_int4", 2, 8, 2, 128, [70, 9], {"paged": True, "page_size": 2, "kv_dtype": "int4"}),
+    ("paged64_int4_d256_win", 2, 4, 1, 256, [200, 65], {"paged": True, "page_size": 64,
+                                                        "kv_dtype": "int4", "window": 70}),
 ]
 
 
@@ -273,6 +286,11 @@ MULTI = [
     ("gqa16_d128_rows16", 1, 16, 1, 128, [2000], {}),
     ("gqa32_d256_rows32", 1, 32, 1, 256, [900], {}),
     ("q4_gqa8_d256_fp8_rows32", 1, 16, 2, 256, [530], {"q_len": 4, "kv_dtype": "fp8_e4m3"}),
+    ("q2_gqa4_int4_paged", 3, 8, 2, 128, [300, 2, 65], {"q_len": 2, "paged": True,
+                                                        "page_size": 16, "kv_dtype": "int4"}),
+    ("q8_gqa4_int4_win_rows32", 2, 8, 2, 128, [700, 50], {"q_len": 8, "kv_dtype": "int4",
+                                                          "window": 200}),
+    ("q4_gqa4_int4_d256_rows16", 1, 8, 2, 256, [530], {"q_len": 4, "kv_dtype": "int4"}),
 ]
 
 
@@ -281,9 +299,8 @@ MULTI = [
 def test_several_query_tokens(case, path):
     name, B, Hq, Hk, d, lens, kw = case
     x = synth.generate(B, Hq, Hk, d, lens, seed=zlib.crc32(name.encode()) & 0xFFFF, name=name, **kw)
-    rows = x.group * x.q_len
-    if path == "simt" and (rows not in (1, 2, 4, 8) or (x.kv_dtype == "fp8_e4m3" and rows > 4)):
-        pytest.skip("no SIMT kernel for this many rows")
+    if not _has_path(x, path):
+        pytest.skip("no kernel for these rows on this path")
     _check(x, path=path)
 
 
@@ -340,6 +357,8 @@ CAPPED = [
                                                      "page_size": 16, "q_len": 2}),
     ("cap30_gqa16_q2_rows32", 1, 32, 2, 128, [1200], {"logit_cap": 30.0, "sm_scale": 0.5,
                                                        "q_len": 2}),
+    ("cap15_int4", 2, 8, 2, 128, [700, 33], {"logit_cap": 15.0, "sm_scale": 0.5,
+                                             "kv_dtype": "int4"}),
 ]
 
 
@@ -348,9 +367,8 @@ CAPPED = [
 def test_logit_softcap(case, path):
     name, B, Hq, Hk, d, lens, kw = case
     x = synth.generate(B, Hq, Hk, d, lens, seed=zlib.crc32(name.encode()) & 0xFFFF, name=name, **kw)
-    rows = x.group * x.q_len
-    if path == "simt" and (rows not in (1, 2, 4, 8) or (x.kv_dtype == "fp8_e4m3" and rows > 4)):
-        pytest.skip("no SIMT kernel for this many rows")
+    if not _has_path(x, path):
+        pytest.skip("no kernel for these rows on this path")
     out, lse, _ = _check(x, path=path)
     # the cap must matter here: the uncapped result is different
     plain = synth.DecodeInputs(**{**x.__dict__, "logit_cap": 0.0})
@@ -382,3 +400,18 @@ def test_tuned_choices_match_the_oracle():
                            name=f"tuned_d{d}_r{rows_per}_L{L}")
         out, lse, info = _check(x, path="auto")
         assert info["path"] == r["path"]
+
+
+# ------------------------------------------------------------------ INT4 KV
+def test_int4_forced_splits_agree():
+    """INT4 KV: every split of the tiles over blocks merges to the oracle's
+    result (one block, a few, one tile each)."""
+    x = synth.generate(2, 16, 2, 128, [2500, 203], kv_dtype="int4", seed=33)
+    _forced_splits_agree(x, "mma")
+
+
+def test_full_size_int4_long_context():
+    """The long-context GQA-8 decode with an INT4 cache at full size
+    (131072 keys), sampled rows against the oracle."""
+    _check_full(synth.workload("int4_gqa8_L131072"), path="mma", nrows=24, seed=3)
+
