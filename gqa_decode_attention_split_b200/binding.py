@@ -43,7 +43,8 @@ class DecodeDesc(ctypes.Structure):
                 ("page_size", ctypes.c_int32), ("window", ctypes.c_int32),
                 ("sm_scale", ctypes.c_float), ("path", ctypes.c_int32),
                 ("num_ctas", ctypes.c_int32), ("q_len", ctypes.c_int32),
-                ("logit_cap", ctypes.c_float)]
+                ("logit_cap", ctypes.c_float), ("unified_max", ctypes.c_int32),
+                ("softmax_phi", ctypes.c_float)]
 
 
 class PlanInfo(ctypes.Structure):
@@ -163,7 +164,10 @@ class DecodePlan:
 def plan(batch: int, qo_heads: int, kv_heads: int, head_dim: int, kv_indptr_host, *,
          kv_dtype: str = "bf16", paged: bool = False, page_size: int = 0, window: int = -1,
          sm_scale: Optional[float] = None, path: str = "auto", num_ctas: int = 0,
-         num_sms: int = 0, q_len: int = 1, logit_cap: float = 0.0) -> DecodePlan:
+         num_sms: int = 0, q_len: int = 1, logit_cap: float = 0.0,
+         softmax_phi: Optional[float] = None) -> DecodePlan:
+    """softmax_phi: None for the plain running max; a value turns on the
+    unified max with that phi (natural-log units of the scaled score)."""
     lib = load_library()
     ind = np.ascontiguousarray(np.asarray(
         kv_indptr_host.cpu().numpy() if hasattr(kv_indptr_host, "cpu") else kv_indptr_host,
@@ -174,7 +178,9 @@ def plan(batch: int, qo_heads: int, kv_heads: int, head_dim: int, kv_indptr_host
                       kv_dtype=_KV_DTYPES[kv_dtype],
                       paged=int(bool(paged)), page_size=int(page_size), window=int(window),
                       sm_scale=float(sm_scale), path=_PATH_NAMES[path], num_ctas=int(num_ctas),
-                      q_len=int(q_len), logit_cap=float(logit_cap))
+                      q_len=int(q_len), logit_cap=float(logit_cap),
+                      unified_max=0 if softmax_phi is None else 1,
+                      softmax_phi=0.0 if softmax_phi is None else float(softmax_phi))
     handle = ctypes.c_void_p()
     ws = ctypes.c_size_t()
     _check(lib.fa_decode_plan(ctypes.byref(desc), ind.ctypes.data, int(num_sms),

@@ -128,6 +128,8 @@ fa_status validate_desc(const fa_decode_desc* d) {
   if (d->num_ctas < 0) return FA_ERR_INVALID_ARG;
   if (d->q_len < 0 || d->q_len > 64) return FA_ERR_INVALID_ARG;
   if (!(d->logit_cap >= 0.f) || !isfinite(d->logit_cap)) return FA_ERR_INVALID_ARG;
+  if (d->unified_max != 0 && d->unified_max != 1) return FA_ERR_INVALID_ARG;
+  if (d->unified_max && !isfinite(d->softmax_phi)) return FA_ERR_INVALID_ARG;
   if (static_cast<int64_t>(d->batch) * d->kv_heads > (1 << 30)) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
@@ -506,6 +508,7 @@ extern "C" fa_status fa_decode_run(const fa_plan* plan, const void* q, const voi
   a.swz = plan->swz;
   a.score_scale = d.sm_scale * 1.4426950408889634f;
   a.cap_l2 = d.logit_cap > 0.f ? d.logit_cap * 1.4426950408889634f : 0.f;
+  a.m_init = d.unified_max ? d.softmax_phi * 1.4426950408889634f : -INFINITY;
 
   cudaError_t e = plan->kernel->launch(a, plan->num_ctas, plan->smem,
                                        static_cast<cudaStream_t>(stream));

@@ -73,6 +73,13 @@ namespace fa {
 #endif
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait, then give up
 constexpr float kRescaleSlack = 8.0f;               // log2 units
+// Unified max: a row whose first finite scores sit more than this far (log2
+// units) below phi starts from its own maximum instead; nothing has
+// accumulated yet, so the switch is exact.  With the slack above, a row's
+// largest weight stays in [2^-8, 2^8], inside the range of the f16
+// probabilities of the fp8 / int4 tensor-core products (a weight of 2^-43
+// against a phi far above the scores flushed to zero there).
+constexpr float kPhiDrop = kRescaleSlack;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -105,6 +112,7 @@ struct KernelArgs {
   int seg_parts;      // 0: equal runs of all tiles; k > 0: k runs per segment
   float score_scale;  // sm_scale * log2(e)
   float cap_l2;       // > 0: logit soft-cap in log2 units (cap * log2(e)); 0: none
+  float m_init;       // start of every running max: -inf, or the unified max phi (log2 units)
 };
 
 constexpr int kSmemPerBlock = 232448;  // 227 KB of shared memory per block (sm_100)
@@ -357,6 +365,7 @@ struct SimtConsumer {
   float q[G][E];
   float acc[G][E];
   float m[G], l[G];
+  uint32_t fresh;  // unified max: bit h set while row h has seen no finite score
   int slot, j;
 
   __device__ __forceinline__ int chunk_plane(int k) const { return (j + LPT * k) / NCP; }
@@ -418,9 +427,10 @@ struct SimtConsumer {
 #pragma unroll
         for (int e = 0; e < EPC; ++e) acc[h][k * EPC + e] = 0.f;
       }
-      m[h] = -CUDART_INF_F;
+      m[h] = a.m_init;
       l[h] = 0.f;
     }
+    fresh = a.m_init > -CUDART_INF_F ? (1u << G) - 1u : 0u;
   }
 
   // A tile is processed in sub-steps of TPSC tokens per slot (bounded
@@ -502,8 +512,17 @@ struct SimtConsumer {
         tmax[h] = s[0][h];
 #pragma unroll
         for (int tt = 1; tt < TPSC; ++tt) tmax[h] = fmaxf(tmax[h], s[tt][h]);
-        need |= tmax[h] > m[h] + kRescaleSlack;
       }
+      if (fresh != 0u) {  // unified max: a row's first finite scores
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+          if (((fresh >> h) & 1u) && tmax[h] > -CUDART_INF_F) {
+            if (tmax[h] < m[h] - kPhiDrop) m[h] = tmax[h];
+            fresh &= ~(1u << h);
+          }
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) need |= tmax[h] > m[h] + kRescaleSlack;
       if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
         for (int h = 0; h < G; ++h) {
@@ -549,10 +568,13 @@ struct SimtConsumer {
                                             int lane, int /*group*/) {
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      float M = m[h];
+      // a state that saw no finite score holds nothing: its max is -inf (with
+      // the unified max it would otherwise report phi)
+      const float mh = ((fresh >> h) & 1u) ? -CUDART_INF_F : m[h];
+      float M = mh;
 #pragma unroll
       for (int off = LPT; off < 32; off <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-      const float sc = (m[h] == -CUDART_INF_F) ? 0.f : exp2_approx(m[h] - M);
+      const float sc = (mh == -CUDART_INF_F) ? 0.f : exp2_approx(mh - M);
       float lh = l[h] * sc;
 #pragma unroll
       for (int off = LPT; off < 32; off <<= 1) lh += __shfl_xor_sync(0xffffffffu, lh, off);
@@ -630,6 +652,7 @@ struct MmaConsumer {
   uint32_t qb8[kQSplit ? KS32 : 1][3][2];  // e4m3 q parts (hi, mid, lo) per k-step
   float o[KS][4];
   float m[2], l[2];
+  uint32_t fresh;  // unified max: bit j set while row 2t + j has seen no finite score
   float sscale[2];
   int g, t;
   int rbase;  // first segment row of this warp's team
@@ -735,8 +758,9 @@ struct MmaConsumer {
     for (int mt = 0; mt < KS; ++mt)
 #pragma unroll
       for (int i = 0; i < 4; ++i) o[mt][i] = 0.f;
-    m[0] = m[1] = -CUDART_INF_F;
+    m[0] = m[1] = a.m_init;
     l[0] = l[1] = 0.f;
+    fresh = a.m_init > -CUDART_INF_F ? 3u : 0u;
   }
 
   __device__ __forceinline__ uint32_t chunk_addr(uint32_t tile, int row, int chunk, int swz) const {
@@ -871,6 +895,16 @@ struct MmaConsumer {
     for (int off = 4; off < 32; off <<= 1) {
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    if (fresh != 0u) {  // unified max: the rows' first finite scores (row-uniform: mx is reduced)
+      if ((fresh & 1u) && mx0 > -CUDART_INF_F) {
+        if (mx0 < m[0] - kPhiDrop) m[0] = mx0;
+        fresh &= ~1u;
+      }
+      if ((fresh & 2u) && mx1 > -CUDART_INF_F) {
+        if (mx1 < m[1] - kPhiDrop) m[1] = mx1;
+        fresh &= ~2u;
+      }
     }
     const bool up0 = mx0 > m[0] + kRescaleSlack, up1 = mx1 > m[1] + kRescaleSlack;
     if (__any_sync(0xffffffffu, up0 || up1)) {
@@ -1047,9 +1081,9 @@ struct MmaConsumer {
     }
     const int h0 = rbase + 2 * t, h1 = h0 + 1;
     const bool r0 = h0 < G, r1 = h1 < G;
-    if (g == 0) {
-      if (r0) m_area[w * G + h0] = m[0];
-      if (r1) m_area[w * G + h1] = m[1];
+    if (g == 0) {  // a row that saw no finite score holds nothing: max -inf (not phi)
+      if (r0) m_area[w * G + h0] = (fresh & 1u) ? -CUDART_INF_F : m[0];
+      if (r1) m_area[w * G + h1] = (fresh & 2u) ? -CUDART_INF_F : m[1];
       if (r0) l_area[w * G + h0] = l0;
       if (r1) l_area[w * G + h1] = l1;
     }

@@ -116,6 +116,18 @@ typedef struct {
                       /* (Gemma 2's soft-cap, named on "FlashInfer x JAX via */
                       /* jax-tvm-ffi", section "Applying it to Gemma 3").    */
                       /* Must be finite and >= 0.                            */
+  int32_t unified_max; /* 0: off.  1: unified max ("FlashDecoding++"         */
+                      /* explainer, section "Asynchronous softmax and        */
+                      /* unified max value"): every running max starts at   */
+                      /* softmax_phi instead of -inf, so partial states     */
+                      /* share one max and are not rescaled while the       */
+                      /* scores stay below it.  Exact for any phi: a score  */
+                      /* more than 8 log2-units above phi falls back to the */
+                      /* exact rescale, and a row whose first scores sit     */
+                      /* more than 8 log2-units below phi starts from its   */
+                      /* own maximum instead.                               */
+  float softmax_phi;  /* unified_max only: phi, in natural-log units of the */
+                      /* scaled (and soft-capped) score; must be finite.    */
 } fa_decode_desc;
 
 typedef struct fa_plan fa_plan;

@@ -383,3 +383,16 @@ def test_int4_plans(lib):
         assert st == 0
         lib.fa_plan_destroy(h)
 
+
+
+def test_unified_max_fields_are_validated(lib):
+    """unified_max is 0 or 1; with it on, softmax_phi must be finite (a
+    zero-filled descriptor keeps the plain running max)."""
+    for kw, code in ((dict(unified_max=1, softmax_phi=3.0), 0), (dict(unified_max=1, softmax_phi=-1e30), 0),
+                     (dict(unified_max=2), 1), (dict(unified_max=1, softmax_phi=float("nan")), 1),
+                     (dict(unified_max=1, softmax_phi=float("inf")), 1),
+                     (dict(unified_max=0, softmax_phi=float("nan")), 0)):
+        st, h, _ = _plan(lib, _desc(**kw), [0, 100])
+        assert st == code, kw
+        if h.value:
+            lib.fa_plan_destroy(h)

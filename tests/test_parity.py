@@ -415,3 +415,42 @@ def test_full_size_int4_long_context():
     (131072 keys), sampled rows against the oracle."""
     _check_full(synth.workload("int4_gqa8_L131072"), path="mma", nrows=24, seed=3)
 
+
+
+# ------------------------------------------------------------ unified max
+UNIFIED = [
+    # (name, batch, qo, kv, d, lens, kw)
+    ("gqa4_paged", 3, 8, 2, 128, [900, 33, 260], {"paged": True, "page_size": 16}),
+    ("fp8_gqa8", 1, 16, 2, 128, [1500], {"kv_dtype": "fp8_e4m3"}),
+    ("int4_gqa4", 2, 8, 2, 128, [700, 90], {"kv_dtype": "int4"}),
+    ("q4_rows16_win", 2, 8, 2, 128, [800, 40], {"q_len": 4, "window": 300}),
+    ("cap20_d256", 1, 8, 4, 256, [1000], {"logit_cap": 20.0, "sm_scale": 0.5}),
+]
+
+
+@pytest.mark.parametrize("phi", [2.0, 30.0, 500.0, -500.0])
+@pytest.mark.parametrize("case", UNIFIED, ids=[c[0] for c in UNIFIED])
+@pytest.mark.parametrize("path", PATHS)
+def test_unified_max_matches_the_oracle(case, path, phi):
+    """The unified max ("FlashDecoding++", "Asynchronous softmax and unified
+    max value") changes where the running max starts, not the result: with
+    phi near the scores (2), above them (30: no rescale ever), far above
+    (500: every row restarts from its own maximum) and far below (-500:
+    the exact rescale takes over at the first tile) the pass equals the
+    plain definition."""
+    name, B, Hq, Hk, d, lens, kw = case
+    x = synth.generate(B, Hq, Hk, d, lens, seed=zlib.crc32(name.encode()) & 0xFFFF, name=name, **kw)
+    if not _has_path(x, path):
+        pytest.skip("no kernel for these rows on this path")
+    ref_out, ref_lse = oracle.decode_all(x)
+    dev = DeviceInputs(x)
+    for n in (0, 7):
+        p = binding.plan(x.batch, x.qo_heads, x.kv_heads, x.head_dim, x.kv_indptr,
+                         kv_dtype=x.kv_dtype, paged=x.paged, page_size=x.page_size,
+                         window=x.window, sm_scale=x.sm_scale, path=path, num_ctas=n,
+                         q_len=x.q_len, logit_cap=x.logit_cap, softmax_phi=phi)
+        ws = p.new_workspace()
+        out, lse = dev.run(p, workspace=ws)
+        assert binding.decode_status(ws) == 0
+        o, l = to_numpy(out, lse)
+        assert_matches(o, l, ref_out, ref_lse, what=f"{name} {path} phi={phi} ctas={n}")
