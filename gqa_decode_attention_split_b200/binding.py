@@ -52,7 +52,7 @@ class PlanInfo(ctypes.Structure):
                 ("tile_tokens", ctypes.c_int32), ("stages", ctypes.c_int32),
                 ("total_tiles", ctypes.c_int32), ("max_partials", ctypes.c_int32),
                 ("workspace_bytes", ctypes.c_size_t), ("smem_bytes", ctypes.c_size_t),
-                ("v_stages", ctypes.c_int32)]
+                ("v_stages", ctypes.c_int32), ("heads_per_tile", ctypes.c_int32)]
 
 
 class TuningEntry(ctypes.Structure):

@@ -39,8 +39,21 @@ const KernelEntry* find_entry(int head_dim, int group, int kv_kind, int path) {
   std::call_once(g_registry_once, build_registry);
   for (int i = 0; i < g_num_entries; ++i) {
     const KernelEntry& e = g_entries[i];
-    if (e.head_dim != head_dim || e.kv_kind != kv_kind || e.path != path) continue;
+    if (e.head_dim != head_dim || e.kv_kind != kv_kind || e.path != path || e.heads_per_tile != 1)
+      continue;
     if (e.group != 0 ? e.group == group : group <= e.max_group) return &e;
+  }
+  return nullptr;
+}
+
+// The tensor-core variant whose tiles hold `ht` adjacent kv heads.
+const KernelEntry* find_head_entry(int head_dim, int kv_kind, int ht) {
+  std::call_once(g_registry_once, build_registry);
+  for (int i = 0; i < g_num_entries; ++i) {
+    const KernelEntry& e = g_entries[i];
+    if (e.head_dim == head_dim && e.kv_kind == kv_kind && e.path == fa::kPathMma &&
+        e.heads_per_tile == ht)
+      return &e;
   }
   return nullptr;
 }
@@ -86,7 +99,8 @@ EncodeTiledFn encode_fn() {
 struct fa_plan {
   fa_decode_desc desc;
   const KernelEntry* kernel;
-  int32_t group;
+  int32_t group;           // rows of a segment (group * q_len * heads_per_tile)
+  int32_t heads_per_tile;  // kv heads of a segment (> 1: head-team variant)
   int32_t num_ctas;
   int32_t box_t;
   int32_t swz;
@@ -260,6 +274,30 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   }
   if (k == nullptr) return FA_ERR_UNSUPPORTED;
 
+  // INT4 on the tensor-core dataflow: a tile of 256 / row-bytes adjacent kv
+  // heads per token, one row team per head.  A one-head int4 tile of 64
+  // tokens is 4 KB, so the per-tile work around the math (waits, releases,
+  // the softmax bookkeeping) outweighed its bytes: measured 2x faster on the
+  // batch-64 paged shape, 7% on the long-context one.  (The same tiles for
+  // fp8 and bf16 with 128-byte rows measured slower or equal: those passes
+  // stream at full rate and lose only a fixed start-up and merge time.)
+  // One query token, at most 8 rows per head.
+  int32_t ht = 1;
+  {
+    const int64_t rb = row_bytes_of(desc);
+    if (desc->kv_dtype == FA_KV_INT4 && k->path == fa::kPathMma && k->heads_per_tile == 1 &&
+        q_len_of(desc) == 1 && group <= 8 &&
+        rb < 256 && 256 % rb == 0 && desc->kv_heads % (256 / rb) == 0) {
+      const KernelEntry* kh = find_head_entry(desc->head_dim, kind, static_cast<int>(256 / rb));
+      if (kh != nullptr) {
+        k = kh;
+        ht = static_cast<int32_t>(256 / rb);
+      }
+    }
+  }
+  const int64_t seg_heads = desc->kv_heads / ht;  // segments per request
+  const int seg_rows = group * ht;                // rows of a segment
+
   const int T = k->tile_tokens;
   int64_t tiles = 0;
   int64_t seg_tiles = -1;  // tiles of every segment when all are equal, else -1
@@ -268,7 +306,7 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
     tiles += n;
     seg_tiles = b == 0 ? n : (seg_tiles == n ? n : -1);
   }
-  tiles *= desc->kv_heads;
+  tiles *= seg_heads;
 
   int64_t P;
   int32_t seg_parts = 0;
@@ -282,7 +320,7 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
     // average so that the last block's merge of the partial states stays
     // short (32 unless the measured table says otherwise).
     int64_t want = tiles;
-    const int64_t seg_cap = max_pieces * desc->batch * desc->kv_heads;
+    const int64_t seg_cap = max_pieces * desc->batch * desc->kv_heads;  // per kv head
     if (want > seg_cap) want = seg_cap;
     P = want < num_sms ? want : num_sms;
     if (P < 1) P = 1;
@@ -294,7 +332,7 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
     // open, instead of once per head at different times.  Measured on fp8
     // head_dim 128 (8 segments): 10% faster than equal runs over all tiles;
     // with 256-byte rows it made no difference.
-    const int64_t segs = static_cast<int64_t>(desc->batch) * desc->kv_heads;
+    const int64_t segs = static_cast<int64_t>(desc->batch) * seg_heads;
     if (seg_tiles > 0 && k->row_bytes <= 128 && P == num_sms && segs <= num_sms) {
       int64_t parts = num_sms / segs;
       if (parts > seg_tiles) parts = seg_tiles;  // every run gets a tile
@@ -310,11 +348,12 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   if (p == nullptr) return FA_ERR_INVALID_ARG;
   p->desc = *desc;
   p->kernel = k;
-  p->group = group;
+  p->group = seg_rows;
+  p->heads_per_tile = ht;
   p->num_ctas = static_cast<int32_t>(P);
   p->seg_parts = seg_parts;
   p->total_tiles = tiles;
-  const int segs = desc->batch * desc->kv_heads;
+  const int segs = desc->batch * static_cast<int>(seg_heads);
   p->max_partials = P + segs;
   p->page_shift = desc->paged ? ilog2_exact(desc->page_size) : 0;
   p->box_t = desc->paged ? (desc->page_size < T ? desc->page_size : T) : T;
@@ -322,26 +361,27 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   // than a tile) and a bulk tensor copy must land on a 128-byte boundary of
   // shared memory: rows narrower than 128 bytes (int4 at head_dim 128) need
   // pages of at least 128 / row-bytes tokens.
-  if ((static_cast<int64_t>(p->box_t) * k->row_bytes) % 128 != 0) {
+  if ((static_cast<int64_t>(p->box_t) * k->row_bytes * ht) % 128 != 0) {
     delete p;
     return FA_ERR_UNSUPPORTED;
   }
   // 128B swizzle needs every copy to start on a 1024-byte boundary of the
   // tile: whole 8-line groups of 128-byte lines per copy.
   {
-    const int lines_per_copy = k->token_major ? p->box_t * (k->row_bytes / k->plane_bytes) : p->box_t;
+    const int lines_per_copy =
+        k->token_major ? p->box_t * (k->row_bytes / k->plane_bytes) * ht : p->box_t;
     p->swz = (k->plane_bytes == 128 && lines_per_copy % 8 == 0) ? 1 : 0;
   }
   size_t off = 256;  // header: device-check word, timeout record
   p->off_records = off;
   off = align_up(off + sizeof(int32_t) * 4 * static_cast<size_t>(P), 256);
   p->off_part_o = off;
-  off = align_up(off + sizeof(float) * static_cast<size_t>(p->max_partials) * group * desc->head_dim,
+  off = align_up(off + sizeof(float) * static_cast<size_t>(p->max_partials) * seg_rows * desc->head_dim,
                  256);
   p->off_part_lse = off;
-  off = align_up(off + sizeof(float) * static_cast<size_t>(p->max_partials) * group, 256);
+  off = align_up(off + sizeof(float) * static_cast<size_t>(p->max_partials) * seg_rows, 256);
   p->ws_bytes = off;
-  p->smem = k->smem_bytes(desc->batch, group);
+  p->smem = k->smem_bytes(desc->batch, seg_rows);
   if (p->smem > 232448) {
     delete p;
     return FA_ERR_UNSUPPORTED;  // batch too large for the per-block schedule arrays
@@ -362,6 +402,7 @@ extern "C" fa_status fa_plan_get_info(const fa_plan* plan, fa_plan_info_t* info)
   info->max_partials = static_cast<int32_t>(plan->max_partials);
   info->workspace_bytes = plan->ws_bytes;
   info->smem_bytes = plan->smem;
+  info->heads_per_tile = plan->heads_per_tile;
   return FA_OK;
 }
 
@@ -397,9 +438,10 @@ fa_status make_kv_map(const fa_plan* p, const void* base, int64_t kv_rows, CUten
   // L2 fills no wider than a token row: a 256-byte fill of a 128-byte row
   // would pull in the next kv head's row, which another block reads much
   // later (measured 1.48x DRAM traffic on 128-byte fp8 rows).
-  const CUtensorMapL2promotion promo = row >= 256   ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B
-                                      : row >= 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
-                                                   : CU_TENSOR_MAP_L2_PROMOTION_NONE;
+  const cuuint64_t span = row * static_cast<cuuint64_t>(p->heads_per_tile);  // contiguous bytes a token
+  const CUtensorMapL2promotion promo = span >= 256   ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+                                      : span >= 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
+                                                    : CU_TENSOR_MAP_L2_PROMOTION_NONE;
   CUresult r;
   if (k->token_major) {
     // [.. rows][kv_heads][planes][plane elements]: one copy carries whole rows
@@ -407,7 +449,8 @@ fa_status make_kv_map(const fa_plan* p, const void* base, int64_t kv_rows, CUten
       const cuuint64_t dims[4] = {inner, np, static_cast<cuuint64_t>(d.kv_heads),
                                   static_cast<cuuint64_t>(kv_rows)};
       const cuuint64_t strides[3] = {cb, row, row * d.kv_heads};
-      const cuuint32_t box[4] = {inner, static_cast<cuuint32_t>(np), 1,
+      const cuuint32_t box[4] = {inner, static_cast<cuuint32_t>(np),
+                                 static_cast<cuuint32_t>(p->heads_per_tile),
                                  static_cast<cuuint32_t>(k->tile_tokens)};
       r = enc(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, promo,
@@ -417,7 +460,8 @@ fa_status make_kv_map(const fa_plan* p, const void* base, int64_t kv_rows, CUten
                                   static_cast<cuuint64_t>(d.page_size),
                                   static_cast<cuuint64_t>(kv_rows)};
       const cuuint64_t strides[4] = {cb, row, row * d.kv_heads, row * d.kv_heads * d.page_size};
-      const cuuint32_t box[5] = {inner, static_cast<cuuint32_t>(np), 1,
+      const cuuint32_t box[5] = {inner, static_cast<cuuint32_t>(np),
+                                 static_cast<cuuint32_t>(p->heads_per_tile),
                                  static_cast<cuuint32_t>(p->box_t), 1};
       r = enc(map, dt, 5, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, promo,
@@ -495,8 +539,10 @@ extern "C" fa_status fa_decode_run(const fa_plan* plan, const void* q, const voi
   a.max_partials = static_cast<int>(plan->max_partials);
   a.batch = d.batch;
   a.qo_heads = d.qo_heads;
-  a.kv_heads = d.kv_heads;
-  a.group = d.qo_heads / d.kv_heads;
+  // a segment covers heads_per_tile kv heads: seen by the kernel as one kv
+  // head whose group holds all their query heads
+  a.kv_heads = d.kv_heads / plan->heads_per_tile;
+  a.group = d.qo_heads / d.kv_heads * plan->heads_per_tile;
   a.q_len = q_len_of(&d);
   a.window_u = d.window > 0 ? union_window(&d) : -1;
   a.window = d.window > 0 ? d.window : -1;
@@ -521,9 +567,9 @@ extern "C" fa_status fa_decode_run(const fa_plan* plan, const void* q, const voi
   m.lse = a.lse;
   m.num_records = plan->num_ctas;
   m.group = plan->group;
-  m.kv_group = d.qo_heads / d.kv_heads;
+  m.kv_group = d.qo_heads / d.kv_heads * plan->heads_per_tile;
   m.q_len = q_len_of(&d);
-  m.kv_heads = d.kv_heads;
+  m.kv_heads = d.kv_heads / plan->heads_per_tile;
   m.qo_heads = d.qo_heads;
   m.batch = d.batch;
   m.max_partials = plan->max_partials;

@@ -64,6 +64,7 @@ KernelEntry make_entry(int path, int group, int max_group, int kv_kind) {
   e.row_bytes = C::ROWB;
   e.plane_bytes = C::CB;
   e.token_major = C::TOKEN_MAJOR ? 1 : 0;
+  e.heads_per_tile = C::HT;
   e.smem_bytes = &smem_bytes_for<Cons>;
   e.launch = &launch_decode<Cons>;
   return e;
@@ -96,6 +97,12 @@ int register_variants(KernelEntry* out, int cap, bool with_quant) {
       add(make_entry<MmaConsumer<D, kKvInt4, 1>>(kPathMma, 0, 8, kKvInt4));
       add(make_entry<MmaConsumer<D, kKvInt4, 2>>(kPathMma, 0, 16, kKvInt4));
       add(make_entry<MmaConsumer<D, kKvInt4, 4>>(kPathMma, 0, 32, kKvInt4));
+      // int4: tiles of 256 / row-bytes adjacent kv heads (one row team per
+      // head), so one tile's bookkeeping serves several heads' 4 KB
+      if constexpr (D == 128)
+        add(make_entry<MmaConsumer<D, kKvInt4, 4, true>>(kPathMma, 0, 8, kKvInt4));
+      else
+        add(make_entry<MmaConsumer<D, kKvInt4, 2, true>>(kPathMma, 0, 8, kKvInt4));
     }
   }
   return n;

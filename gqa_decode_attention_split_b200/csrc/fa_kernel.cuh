@@ -144,17 +144,23 @@ constexpr int kScaleCap = 128;         // fp8 per-kv-head scales kept in shared 
 // KV element kinds: bf16, fp8 e4m3, int4 (two codes per byte).
 enum : int { kKvBf16 = 0, kKvFp8 = 1, kKvInt4 = 2 };
 
-template <int D, int KIND, int GW, int R, int TILE_BYTES_TARGET, int NWARPS, bool EARLY_K>
+template <int D, int KIND, int GW, int R, int TILE_BYTES_TARGET, int NWARPS, bool EARLY_K,
+          int HT_ = 1>
 struct TileCfg {
   static constexpr int DIM = D;
+  // kv heads per tile: a tile holds the rows of HT adjacent kv heads for each
+  // of its tokens ([T][HT][row], one box), so a copy moves HT * ROWB
+  // contiguous bytes per token
+  static constexpr int HT = HT_;
   static constexpr bool QUANT = KIND != kKvBf16;  // codes with per-kv-head scales
   static constexpr int ES = KIND == kKvBf16 ? 2 : 1;  // bytes per tensor-map element
   static constexpr int ROWB = KIND == kKvBf16 ? 2 * D : (KIND == kKvFp8 ? D : D / 2);
   static constexpr int CB = ROWB < 128 ? ROWB : 128;
   static constexpr int NP = ROWB / CB;
-  static constexpr int T_RAW = TILE_BYTES_TARGET / ROWB;
+  static constexpr int TOKB = HT * ROWB;  // tile bytes per token
+  static constexpr int T_RAW = TILE_BYTES_TARGET / TOKB;
   static constexpr int T = T_RAW < 16 ? 16 : (T_RAW > 128 ? 128 : T_RAW);
-  static constexpr int TILE_BYTES = T * ROWB;
+  static constexpr int TILE_BYTES = T * TOKB;
   static constexpr int NW = NWARPS;
   static constexpr int TEAMS = R;       // row teams
   static constexpr int NT = NW / R;     // tile lanes (warps per team)
@@ -189,6 +195,7 @@ struct TileCfg {
   static constexpr int THREADS = (NW + 1) * 32;
   static constexpr bool TOKEN_MAJOR = FA_PLANE_COPIES == 0;
   static_assert(ROWB % 16 == 0, "rows must be whole 16-byte chunks");
+  static_assert(HT == 1 || TOKEN_MAJOR, "tiles of several heads are token-major");
 };
 
 __device__ __forceinline__ uint32_t swz_off(int row, int chunk, int swz) {
@@ -276,6 +283,15 @@ __device__ __forceinline__ uint2 lds64_in(uint32_t* status, uint32_t addr, uint3
 }
 
 // ------------------------------------------------------------ schedule
+// a / b for non-negative a, positive b: 32-bit division when both
+// fit (the schedule's tile counts do, short of 2^31 tiles), else 64-bit.  A
+// 64-bit division is a long software routine, and a block's schedule takes
+// several before its first copy goes out.
+__device__ __forceinline__ long long div_fast(long long a, long long b) {
+  if (((a | b) >> 31) == 0) return static_cast<long long>(static_cast<uint32_t>(a) / static_cast<uint32_t>(b));
+  return a / b;
+}
+
 struct Piece {
   int b, h;          // request, kv head
   int t0, t1;        // request-local tile indices [t0, t1)
@@ -317,8 +333,8 @@ __device__ __forceinline__ bool next_piece(PieceIter& it, Piece& pc, const int* 
   const int n = s_pre[b + 1] - s_pre[b];
   const long long base = static_cast<long long>(H) * s_pre[b];
   const long long off = it.u - base;
-  const int h = static_cast<int>(off / n);
-  const int tin = static_cast<int>(off % n);
+  const int h = static_cast<int>(div_fast(off, n));
+  const int tin = static_cast<int>(off - static_cast<long long>(h) * n);
   long long len = n - tin;
   if (it.u1 - it.u < len) len = it.u1 - it.u;
   const int ft = first_tile(s_len[b], window, T);
@@ -333,8 +349,8 @@ __device__ __forceinline__ bool next_piece(PieceIter& it, Piece& pc, const int* 
     pc.c_first = pc.seg * it.parts;
     pc.n_pieces = it.parts;
   } else {
-    pc.c_first = static_cast<int>(pc.seg_start / it.per);
-    pc.n_pieces = static_cast<int>((seg_end - 1) / it.per) - pc.c_first + 1;
+    pc.c_first = static_cast<int>(div_fast(pc.seg_start, it.per));
+    pc.n_pieces = static_cast<int>(div_fast(seg_end - 1, it.per)) - pc.c_first + 1;
   }
   it.u += len;
   return true;
@@ -349,6 +365,7 @@ __device__ __forceinline__ bool next_piece(PieceIter& it, Piece& pc, const int* 
 template <int D, int G, bool FP8>
 struct SimtConsumer {
   using C = TileCfg<D, FP8 ? kKvFp8 : kKvBf16, G, 1, FA_SIMT_TILE_BYTES, FA_SIMT_CONSUMER_WARPS, false>;
+  __host__ __device__ static constexpr int team_head(int) { return 0; }  // one kv head per tile
   static constexpr int EPC = 16 / C::ES;
   static constexpr int NCH = C::ROWB / 16;
   static constexpr int E_TARGET = 64 / G;
@@ -617,12 +634,17 @@ struct SimtConsumer {
 // 32 tokens, so that the fewer tile lanes still keep a deep ring.
 // KIND: bf16 (tiles through ldmatrix), fp8 e4m3 or int4 (bytes loaded per
 // lane and widened to f16; the query is held as f16 times a power of two).
-template <int D, int KIND, int R = 1>
+// HEADS: the R teams are R adjacent kv heads of one segment instead of R
+// blocks of 8 rows of one kv head: team t computes the (at most 8) query
+// rows of kv head t of the tile, whose rows sit at token * R + t.
+template <int D, int KIND, int R = 1, bool HEADS = false>
 struct MmaConsumer {
+  static constexpr int HT = HEADS ? R : 1;  // kv heads per tile
   static constexpr bool FP8 = KIND == kKvFp8;
   static constexpr bool I4 = KIND == kKvInt4;
   static constexpr bool BF16 = KIND == kKvBf16;
-  static constexpr int kTileBytes = FP8 ? FA_FP8_MMA_TILE_BYTES
+  static constexpr int kTileBytes = HEADS ? 16384
+                                    : FP8 ? FA_FP8_MMA_TILE_BYTES
                                     : I4  ? FA_FP8_MMA_TILE_BYTES / 2
                                           : (R == 1 ? FA_MMA_TILE_BYTES : FA_MMA_TILE_BYTES / 2);
   // Consumer warps: two teams of 3, or four of 2 (a 9-warp block, whose
@@ -634,7 +656,7 @@ struct MmaConsumer {
   // V held longer than K (EARLY_K: one K slot per two V slots) pays where
   // the V half of a tile is the longer one, fp8 with one team; elsewhere
   // equal rings keep the most tiles in flight.
-  using C = TileCfg<D, KIND, 8, R, kTileBytes, kWarps, !BF16 && R == 1>;
+  using C = TileCfg<D, KIND, 8, R, kTileBytes, kWarps, !BF16 && R == 1, HT>;
   static constexpr int KS = D / 16;     // k-steps of the score product = m-tiles of O^T
   static constexpr int SUB = C::T / 16;  // 16-token subtiles per tile
   static constexpr int BPT = D / 4;      // fp8 / int4 K: elements of a row owned by one lane
@@ -656,6 +678,13 @@ struct MmaConsumer {
   float sscale[2];
   int g, t;
   int rbase;  // first segment row of this warp's team
+  int tr;     // rows of the team (8; with HEADS the group of one kv head)
+  int hrow;   // with HEADS: the team's kv head within the tile, else 0
+
+  // Tile row (in units of one head's row) of token r for this team.
+  __device__ __forceinline__ int srow(int r) const { return r * HT + hrow; }
+  // First kv head of a team relative to its segment's first kv head.
+  __host__ __device__ static constexpr int team_head(int team) { return HEADS ? team : 0; }
 
   // qs: the piece's query rows (staged in shared memory, or in global
   // memory where the tile geometry leaves no room): row r (token r / group,
@@ -666,9 +695,11 @@ struct MmaConsumer {
                                               float kscale, int lane, int team) {
     g = lane >> 2;
     t = lane & 3;
-    rbase = 8 * team;
     const int G = a.group * a.q_len;
-    const bool real = rbase + g < G;
+    tr = HEADS ? a.group / HT : 8;  // with HEADS: one query token, group rows per head
+    rbase = tr * team;
+    hrow = HEADS ? team : 0;
+    const bool real = g < tr && rbase + g < G;
     const int r = real ? rbase + g : 0;
     const uint16_t* qrow = qs + (r / a.group) * qstride + (r % a.group) * D;
     if constexpr (BF16) {
@@ -766,8 +797,9 @@ struct MmaConsumer {
   __device__ __forceinline__ uint32_t chunk_addr(uint32_t tile, int row, int chunk, int swz) const {
     return tile_addr<C>(tile, row, chunk >> 3, chunk & 7, swz);
   }
-  // Shared address of byte `off` of a tile row: swizzled 128-byte planes, or
-  // one unswizzled plane for rows narrower than 128 bytes.
+  // Shared address of byte `off` of tile row `row` (a srow() index):
+  // swizzled 128-byte planes, or one unswizzled plane for rows narrower than
+  // 128 bytes.
   __device__ __forceinline__ uint32_t byte_addr(uint32_t tile, int row, int off, int swz) const {
     if constexpr (C::CB == 128)
       return chunk_addr(tile, row, off >> 4, swz) + (off & 15);
@@ -788,9 +820,9 @@ struct MmaConsumer {
         uint32_t af[4];
         const int ch = kk * 2 + (lane >> 4);
         if constexpr (C::CB == 128)
-          ldsm_x4(ldsm_addr_in(a.status, chunk_addr(kt, row, ch, swz), kt, C::TILE_BYTES, 201), af);
+          ldsm_x4(ldsm_addr_in(a.status, chunk_addr(kt, srow(row), ch, swz), kt, C::TILE_BYTES, 201), af);
         else  // 64-element rows: one plane of CB bytes, no swizzle
-          ldsm_x4(ldsm_addr_in(a.status, kt + row * C::CB + ch * 16, kt, C::TILE_BYTES, 202), af);
+          ldsm_x4(ldsm_addr_in(a.status, kt + srow(row) * C::CB + ch * 16, kt, C::TILE_BYTES, 202), af);
         if (kk & 1)
           mma_bf16(c2, af, qb[kk][0], qb[kk][1]);
         else
@@ -802,8 +834,8 @@ struct MmaConsumer {
 #pragma unroll
       for (int i = 0; i < KB / 16; ++i) {
         const int off = KB * t + 16 * i;
-        const uint4 x0 = lds128_in(a.status, byte_addr(kt, r0, off, swz), kt, C::TILE_BYTES, 203);
-        const uint4 x1 = lds128_in(a.status, byte_addr(kt, r1, off, swz), kt, C::TILE_BYTES, 204);
+        const uint4 x0 = lds128_in(a.status, byte_addr(kt, srow(r0), off, swz), kt, C::TILE_BYTES, 203);
+        const uint4 x1 = lds128_in(a.status, byte_addr(kt, srow(r1), off, swz), kt, C::TILE_BYTES, 204);
         w0[4 * i] = x0.x; w0[4 * i + 1] = x0.y; w0[4 * i + 2] = x0.z; w0[4 * i + 3] = x0.w;
         w1[4 * i] = x1.x; w1[4 * i + 1] = x1.y; w1[4 * i + 2] = x1.z; w1[4 * i + 3] = x1.w;
       }
@@ -968,9 +1000,9 @@ struct MmaConsumer {
           uint32_t af[4];
           const int ch = mt * 2 + ((lane >> 3) & 1);
           if constexpr (C::CB == 128)
-            ldsm_x4_trans(ldsm_addr_in(a.status, chunk_addr(vt, vrow, ch, a.swz), vt, C::TILE_BYTES, 205), af);
+            ldsm_x4_trans(ldsm_addr_in(a.status, chunk_addr(vt, srow(vrow), ch, a.swz), vt, C::TILE_BYTES, 205), af);
           else
-            ldsm_x4_trans(ldsm_addr_in(a.status, vt + vrow * C::CB + ch * 16, vt, C::TILE_BYTES, 206), af);
+            ldsm_x4_trans(ldsm_addr_in(a.status, vt + srow(vrow) * C::CB + ch * 16, vt, C::TILE_BYTES, 206), af);
           if (edge) {
             af[0] &= mk01;
             af[1] &= mk01;
@@ -993,11 +1025,11 @@ struct MmaConsumer {
 #pragma unroll
         for (int rr = 0; rr < 4; ++rr) {
           if constexpr (VB == 8) {
-            const uint2 x = lds64_in(a.status, byte_addr(vt, rows[rr], VB * g, a.swz), vt, C::TILE_BYTES, 208);
+            const uint2 x = lds64_in(a.status, byte_addr(vt, srow(rows[rr]), VB * g, a.swz), vt, C::TILE_BYTES, 208);
             vw[rr][0] = x.x;
             vw[rr][1] = x.y;
           } else {
-            const uint4 x = lds128_in(a.status, byte_addr(vt, rows[rr], VB * g, a.swz), vt, C::TILE_BYTES, 209);
+            const uint4 x = lds128_in(a.status, byte_addr(vt, srow(rows[rr]), VB * g, a.swz), vt, C::TILE_BYTES, 209);
             vw[rr][0] = x.x;
             vw[rr][1] = x.y;
             vw[rr][2] = x.z;
@@ -1033,7 +1065,7 @@ struct MmaConsumer {
         for (int rr = 0; rr < 4; ++rr)
 #pragma unroll
           for (int i = 0; i < VBT / 16; ++i) {
-            const uint4 x = lds128_in(a.status, chunk_addr(vt, rows[rr], (VBT * g) / 16 + i, a.swz), vt,
+            const uint4 x = lds128_in(a.status, chunk_addr(vt, srow(rows[rr]), (VBT * g) / 16 + i, a.swz), vt,
                                       C::TILE_BYTES, 207);
             vw[rr][4 * i] = x.x;
             vw[rr][4 * i + 1] = x.y;
@@ -1080,7 +1112,7 @@ struct MmaConsumer {
       l1 += __shfl_xor_sync(0xffffffffu, l1, off);
     }
     const int h0 = rbase + 2 * t, h1 = h0 + 1;
-    const bool r0 = h0 < G, r1 = h1 < G;
+    const bool r0 = 2 * t < tr && h0 < G, r1 = 2 * t + 1 < tr && h1 < G;
     if (g == 0) {  // a row that saw no finite score holds nothing: max -inf (not phi)
       if (r0) m_area[w * G + h0] = (fresh & 1u) ? -CUDART_INF_F : m[0];
       if (r1) m_area[w * G + h1] = (fresh & 2u) ? -CUDART_INF_F : m[1];
@@ -1209,9 +1241,10 @@ __global__ void __maxnreg__(max_regs<Cons>())
     s_len[b] = L;
     if (bad) atomicOr(a.status, kFlagBadIndptr);
   }
-  const bool scales_in_smem = H <= kScaleCap;
+  const int HK = H * C::HT;  // kv heads (a segment covers HT of them)
+  const bool scales_in_smem = HK <= kScaleCap;
   if (C::QUANT && scales_in_smem) {
-    for (int i = tid; i < H; i += blockDim.x) {
+    for (int i = tid; i < HK; i += blockDim.x) {
       s_kscale[i] = __ldg(a.k_scale + i);
       s_vscale[i] = __ldg(a.v_scale + i);
     }
@@ -1256,7 +1289,7 @@ __global__ void __maxnreg__(max_regs<Cons>())
   const long long N = static_cast<long long>(H) * s_pre[B];
   const int P = gridDim.x, c = blockIdx.x;
   PieceIter it;
-  it.per = N > 0 ? (N + P - 1) / P : 1;
+  it.per = N > 0 ? div_fast(N + P - 1, P) : 1;
   it.parts = 0;
   it.u = static_cast<long long>(c) * it.per;
   it.u1 = it.u + it.per < N ? it.u + it.per : N;
@@ -1271,8 +1304,8 @@ __global__ void __maxnreg__(max_regs<Cons>())
       const int b = seg / H, h = seg - b * H;
       const long long n = s_pre[b + 1] - s_pre[b];
       const long long base = static_cast<long long>(H) * s_pre[b] + static_cast<long long>(h) * n;
-      it.u = base + part * n / k;
-      it.u1 = base + (part + 1) * n / k;
+      it.u = base + div_fast(part * n, k);
+      it.u1 = base + div_fast((part + 1) * n, k);
     }
   }
 
@@ -1283,7 +1316,7 @@ __global__ void __maxnreg__(max_regs<Cons>())
   // inside a segment that began in block c - 1's run, it is the segment's
   // first cut and block c names the segment for the merge kernel; every
   // other block writes "none", so no record survives from an earlier pass.
-  if (tid == 0 && c > 0) {
+  if (tid == 32 && c > 0) {  // a consumer thread: the producer lane goes straight to its copies
     PieceIter i0 = it;
     Piece p0;
     int4 rec = make_int4(-1, 0, 0, 0);
@@ -1417,8 +1450,8 @@ __global__ void __maxnreg__(max_regs<Cons>())
           if (!a.paged) {
             const int row = s_start[pc.b] + tt * T;
             if constexpr (C::TOKEN_MAJOR) {
-              tma_load_4d(kdst, &a.kmap, kfb, 0, 0, pc.h, row, pol);
-              tma_load_4d(vdst, &a.vmap, vfb, 0, 0, pc.h, row, pol);
+              tma_load_4d(kdst, &a.kmap, kfb, 0, 0, pc.h * C::HT, row, pol);
+              tma_load_4d(vdst, &a.vmap, vfb, 0, 0, pc.h * C::HT, row, pol);
             } else {
 #pragma unroll
               for (int p = 0; p < C::NP; ++p) {
@@ -1435,12 +1468,12 @@ __global__ void __maxnreg__(max_regs<Cons>())
               const int pidx = tok >> a.page_shift;
               const int page = (pidx < npages && pidx - pbase < 64) ? s_pages[pidx - pbase] : -1;
               const int slot0 = tok & (ps - 1);
-              const uint32_t off = jb * a.box_t * C::ROWB;
-              if (FA_CHECK(a.status, off + a.box_t * C::ROWB <= C::TILE_BYTES && (off & 127u) == 0 &&
+              const uint32_t off = jb * a.box_t * C::TOKB;
+              if (FA_CHECK(a.status, off + a.box_t * C::TOKB <= C::TILE_BYTES && (off & 127u) == 0 &&
                                          pidx - pbase >= 0 && pidx - pbase < 64,
                            303, off)) {
-                tma_load_5d(kdst + off, &a.kmap, kfb, 0, 0, pc.h, slot0, page, pol);
-                tma_load_5d(vdst + off, &a.vmap, vfb, 0, 0, pc.h, slot0, page, pol);
+                tma_load_5d(kdst + off, &a.kmap, kfb, 0, 0, pc.h * C::HT, slot0, page, pol);
+                tma_load_5d(vdst + off, &a.vmap, vfb, 0, 0, pc.h * C::HT, slot0, page, pol);
               }
             }
           } else {
@@ -1571,12 +1604,14 @@ __global__ void __maxnreg__(max_regs<Cons>())
           alive = false;
         }
       }
-      const float ks = C::QUANT ? (scales_in_smem ? s_kscale[pc.h] : __ldg(a.k_scale + pc.h)) : 1.f;
+      const int kh = pc.h * C::HT + Cons::team_head(team);  // this team's kv head
+      const float ks = C::QUANT ? (scales_in_smem ? s_kscale[kh] : __ldg(a.k_scale + kh)) : 1.f;
       cons.begin_piece(a, q_slots + qs * (C::QSLOT_BYTES / 2), GK * D, ks, lane, team);
       __syncwarp();
       if (lane == 0) mbar_arrive(qempty0 + 8 * qs);
     } else {
-      const float ks = C::QUANT ? (scales_in_smem ? s_kscale[pc.h] : __ldg(a.k_scale + pc.h)) : 1.f;
+      const int kh = pc.h * C::HT + Cons::team_head(team);  // this team's kv head
+      const float ks = C::QUANT ? (scales_in_smem ? s_kscale[kh] : __ldg(a.k_scale + kh)) : 1.f;
       cons.begin_piece(a,
                        a.q + (static_cast<size_t>(pc.b) * Q * a.qo_heads + static_cast<size_t>(pc.h) * GK) * D,
                        a.qo_heads * D, ks, lane, team);
@@ -1628,7 +1663,11 @@ __global__ void __maxnreg__(max_regs<Cons>())
     // of the next piece; the last warp to park merges the NW states, writes
     // the result (or the partial) and frees the area.  A warp waits only if
     // it finishes its share of the next piece before that merge is done.
-    const float vs = C::QUANT ? (scales_in_smem ? s_vscale[pc.h] : __ldg(a.v_scale + pc.h)) : 1.f;
+    // V scale of row h's kv head (tiles of several heads: GK / HT rows per head)
+    auto vscale_of = [&](int h) {
+      const int vh = pc.h * C::HT + (C::HT > 1 ? h / (GK / C::HT) : 0);
+      return C::QUANT ? (scales_in_smem ? s_vscale[vh] : __ldg(a.v_scale + vh)) : 1.f;
+    };
     if (piece > 0 && alive) {
       const bool ok = __all_sync(0xffffffffu, mbar_wait(mfree, (piece - 1) & 1, kWaitLimitNs));
       if (!ok) {
@@ -1668,7 +1707,7 @@ __global__ void __maxnreg__(max_regs<Cons>())
           Ls = fmaf(l_area[ww * G + h], scw[ww], Ls);
         }
         const bool empty = !(Ls > 0.f);
-        const float f = empty ? 0.f : vs / Ls;
+        const float f = empty ? 0.f : vscale_of(h) / Ls;
 #pragma unroll
         for (int ww = 0; ww < NT; ++ww) m_area[ww * G + h] = scw[ww] * f;
         const float lv = empty ? -CUDART_INF_F : (M + __log2f(Ls)) * kLn2;

@@ -24,6 +24,7 @@ struct KernelEntry {
   int row_bytes;    // head_dim * element size
   int plane_bytes;  // min(128, row_bytes)
   int token_major;  // 1: one copy per box with planes as a tensor-map dimension
+  int heads_per_tile;  // kv heads per tile (> 1: head teams, one segment per head block)
   size_t (*smem_bytes)(int batch, int group);
   cudaError_t (*launch)(const KernelArgs& args, int grid, size_t smem, cudaStream_t stream);
 };

@@ -143,6 +143,8 @@ typedef struct {
   size_t workspace_bytes;   /* minimum workspace size for fa_decode_run       */
   size_t smem_bytes;        /* dynamic shared memory per thread block         */
   int32_t v_stages;         /* V tile slots (at least stages: V is held longer) */
+  int32_t heads_per_tile;   /* kv heads whose rows one tile holds per token:   */
+                            /* > 1 for int4 (256 contiguous bytes a token)     */
 } fa_plan_info_t;
 
 /*

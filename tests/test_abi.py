@@ -87,7 +87,9 @@ def test_plans_for_named_workloads(lib, name):
     T = inf.tile_tokens
     L = lens[0]
     lo = max(0, L - w) if w > 0 else 0
-    assert inf.total_tiles == Hk * ((L + T - 1) // T - lo // T)
+    # tiles count (request, block of heads_per_tile kv heads) segments
+    assert Hk % inf.heads_per_tile == 0
+    assert inf.total_tiles == Hk // inf.heads_per_tile * ((L + T - 1) // T - lo // T)
     lib.fa_plan_destroy(h)
 
 
@@ -104,7 +106,13 @@ def test_plan_paged_and_fp8(lib):
     assert st == 0 and _info(lib, h).path == binding.PATH_MMA
     # 8 equal segments of 128-byte rows: 18 whole runs per segment, so no run
     # crosses a segment boundary (144 of the 148 SMs)
-    assert _info(lib, h).num_ctas == 144
+    inf = _info(lib, h)
+    assert inf.heads_per_tile == 1 and inf.num_ctas == 144
+    lib.fa_plan_destroy(h)
+    # int4 at head_dim 128: tiles of 4 kv heads, 2 equal segments x 74 runs
+    st, h, ws = _plan(lib, _desc(qo_heads=64, kv_heads=8, kv_dtype=2), [0, 131072])
+    inf = _info(lib, h)
+    assert st == 0 and inf.heads_per_tile == 4 and inf.num_ctas == 2 * 74
     lib.fa_plan_destroy(h)
     # the same shape in bf16 (256-byte rows) keeps equal runs over every SM
     st, h, ws = _plan(lib, _desc(qo_heads=64, kv_heads=8), [0, 131072])
@@ -396,3 +404,21 @@ def test_unified_max_fields_are_validated(lib):
         assert st == code, kw
         if h.value:
             lib.fa_plan_destroy(h)
+
+
+def test_head_tile_choice(lib):
+    """INT4 on the MMA dataflow, one query token, at most 8 rows per head and
+    a kv-head count the block divides: tiles of 256 / row-bytes heads;
+    otherwise (and for bf16 / fp8) one head per tile."""
+    cases = [(dict(kv_dtype=2), 4), (dict(kv_dtype=2, head_dim=256), 2),
+             (dict(kv_dtype=1), 1), (dict(head_dim=64), 1), (dict(), 1),
+             (dict(kv_dtype=2, q_len=2), 1), (dict(kv_dtype=2, kv_heads=1, qo_heads=4), 1),
+             (dict(kv_dtype=2, kv_heads=2, qo_heads=8), 1),                # 2 heads, int4 wants 4
+             (dict(kv_dtype=2, qo_heads=64), 1)]                           # 16 rows per head
+    for kw, ht in cases:
+        kw = {"qo_heads": 16, "kv_heads": 4, **kw}
+        st, h, _ = _plan(lib, _desc(**kw), [0, 3000])
+        assert st == 0, kw
+        assert _info(lib, h).heads_per_tile == ht, kw
+        lib.fa_plan_destroy(h)
+

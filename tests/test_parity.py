@@ -117,6 +117,11 @@ def test_segment_aligned_split(window):
     out, lse, info = _check(x, path="mma")
     if window < 0:
         assert info["num_ctas"] == 8 * 18
+    # int4 with tiles of 4 kv heads: 2 segments (81 tiles each) x 74 runs
+    y = synth.generate(1, 64, 8, 128, [5141], kv_dtype="int4", window=window * 2, seed=28)
+    out, lse, info = _check(y, path="mma")
+    if window < 0:
+        assert info["heads_per_tile"] == 4 and info["num_ctas"] == 2 * 74
 
 
 def test_paged_equals_contiguous_on_gpu():
