@@ -628,22 +628,28 @@ struct SimtConsumer {
 // 2^-12 of the bf16 value) and the three products are summed in fp32.  e4m3
 // V is widened exactly to f16 for the P.V product.  The q scale is undone on
 // the fp32 scores.
-// R row teams of 8 query rows each (a segment of up to 8R rows: the query
-// heads of a kv head times the query tokens).  A team's warp computes its 8
-// rows of every tile it takes; with more than one team the bf16 tiles are
-// 32 tokens, so that the fewer tile lanes still keep a deep ring.
+// R row teams of 8 * NB query rows each (a segment of up to 8 * NB * R rows:
+// the query heads of a kv head times the query tokens).  A team's warp
+// computes its rows of every tile it takes, in NB blocks of 8 that share
+// each K / V fragment (one shared-memory read or conversion feeds NB
+// products).  Multi-row variants use 32-token tiles, so that the tile lanes
+// keep a deep ring.
 // KIND: bf16 (tiles through ldmatrix), fp8 e4m3 or int4 (bytes loaded per
 // lane and widened to f16; the query is held as f16 times a power of two).
 // HEADS: the R teams are R adjacent kv heads of one segment instead of R
-// blocks of 8 rows of one kv head: team t computes the (at most 8) query
-// rows of kv head t of the tile, whose rows sit at token * R + t.
-template <int D, int KIND, int R = 1, bool HEADS = false>
+// blocks of rows of one kv head: team t computes the (at most 8) query rows
+// of kv head t of the tile, whose rows sit at token * R + t.
+template <int D, int KIND, int R = 1, bool HEADS = false, int NB = 1>
 struct MmaConsumer {
   static constexpr int HT = HEADS ? R : 1;  // kv heads per tile
   static constexpr bool FP8 = KIND == kKvFp8;
   static constexpr bool I4 = KIND == kKvInt4;
   static constexpr bool BF16 = KIND == kKvBf16;
+  static_assert(NB == 1 || NB == 2, "one or two row blocks per warp");
+  static_assert(!HEADS || NB == 1, "head teams hold one row block");
+  static constexpr int ROWB_K = BF16 ? 2 * D : (FP8 ? D : D / 2);  // bytes of one head's row
   static constexpr int kTileBytes = HEADS ? 16384
+                                    : NB > 1 ? 32 * ROWB_K
                                     : FP8 ? FA_FP8_MMA_TILE_BYTES
                                     : I4  ? FA_FP8_MMA_TILE_BYTES / 2
                                           : (R == 1 ? FA_MMA_TILE_BYTES : FA_MMA_TILE_BYTES / 2);
@@ -654,13 +660,13 @@ struct MmaConsumer {
                                 : R == 2 ? 6
                                          : (!BF16 && D >= 256 ? 4 : 8);
   // V held longer than K (EARLY_K: one K slot per two V slots) pays where
-  // the V half of a tile is the longer one, fp8 with one team; elsewhere
-  // equal rings keep the most tiles in flight.
-  using C = TileCfg<D, KIND, 8, R, kTileBytes, kWarps, !BF16 && R == 1, HT>;
+  // the V half of a tile is the longer one, fp8 with one team of 8 rows;
+  // elsewhere equal rings keep the most tiles in flight.
+  using C = TileCfg<D, KIND, 8 * NB, R, kTileBytes, kWarps, !BF16 && R == 1 && NB == 1, HT>;
   static constexpr int KS = D / 16;     // k-steps of the score product = m-tiles of O^T
   static constexpr int SUB = C::T / 16;  // 16-token subtiles per tile
   static constexpr int BPT = D / 4;      // fp8 / int4 K: elements of a row owned by one lane
-  static constexpr bool kQSplit = FP8 && FA_FP8_QSPLIT;
+  static constexpr bool kQSplit = FP8 && FA_FP8_QSPLIT && NB == 1;
   static constexpr int KS32 = D / 32;    // k-steps of the e4m3 score product
   static constexpr int VBT = D / 8;      // fp8 / int4 V: elements of a row owned by one lane
   static constexpr int KB = I4 ? BPT / 2 : BPT;  // their bytes
@@ -670,15 +676,15 @@ struct MmaConsumer {
   static_assert(!I4 || ((D == 128 || D == 256) && KB % 16 == 0 && (VB == 8 || VB == 16)),
                 "int4 mma path: 64- or 128-byte rows");
 
-  uint32_t qb[KS][2];
+  uint32_t qb[NB][KS][2];
   uint32_t qb8[kQSplit ? KS32 : 1][3][2];  // e4m3 q parts (hi, mid, lo) per k-step
-  float o[KS][4];
-  float m[2], l[2];
-  uint32_t fresh;  // unified max: bit j set while row 2t + j has seen no finite score
-  float sscale[2];
+  float o[NB][KS][4];
+  float m[NB][2], l[NB][2];
+  uint32_t fresh;  // unified max: bit 2 nb + j set while row 8 nb + 2t + j has seen no finite score
+  float sscale[NB][2];
   int g, t;
   int rbase;  // first segment row of this warp's team
-  int tr;     // rows of the team (8; with HEADS the group of one kv head)
+  int tr;     // rows of the team (8 NB; with HEADS the group of one kv head)
   int hrow;   // with HEADS: the team's kv head within the tile, else 0
 
   // Tile row (in units of one head's row) of token r for this team.
@@ -690,108 +696,111 @@ struct MmaConsumer {
   // memory where the tile geometry leaves no room): row r (token r / group,
   // head r % group) at qs + (r / group) * qstride + (r % group) * D; kscale:
   // the fp8 K scale of the piece's kv head (1 for bf16); team: this warp's
-  // row team (rows 8 * team .. 8 * team + 7).
+  // row team (rows 8 NB team .. 8 NB team + 8 NB - 1).
   __device__ __forceinline__ void begin_piece(const KernelArgs& a, const uint16_t* qs, int qstride,
                                               float kscale, int lane, int team) {
     g = lane >> 2;
     t = lane & 3;
     const int G = a.group * a.q_len;
-    tr = HEADS ? a.group / HT : 8;  // with HEADS: one query token, group rows per head
+    tr = HEADS ? a.group / HT : 8 * NB;  // with HEADS: one query token, group rows per head
     rbase = tr * team;
     hrow = HEADS ? team : 0;
-    const bool real = g < tr && rbase + g < G;
-    const int r = real ? rbase + g : 0;
-    const uint16_t* qrow = qs + (r / a.group) * qstride + (r % a.group) * D;
-    if constexpr (BF16) {
 #pragma unroll
-      for (int kk = 0; kk < KS; ++kk) {
-        qb[kk][0] = real ? *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * t) : 0u;
-        qb[kk][1] = real ? *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * t + 8) : 0u;
-      }
-      sscale[0] = sscale[1] = a.score_scale;
-    } else {
-      // this lane's q elements: [BPT*t, BPT*t + BPT)
-      float mx = 0.f;
-      uint32_t qw[BPT / 2];
+    for (int nb = 0; nb < NB; ++nb) {
+      const bool real = 8 * nb + g < tr && rbase + 8 * nb + g < G;
+      const int r = real ? rbase + 8 * nb + g : 0;
+      const uint16_t* qrow = qs + (r / a.group) * qstride + (r % a.group) * D;
+      if constexpr (BF16) {
 #pragma unroll
-      for (int i = 0; i < BPT / 8; ++i) {
-        const uint4 w = real ? *reinterpret_cast<const uint4*>(qrow + BPT * t + 8 * i)
-                             : make_uint4(0, 0, 0, 0);
-        qw[4 * i] = w.x;
-        qw[4 * i + 1] = w.y;
-        qw[4 * i + 2] = w.z;
-        qw[4 * i + 3] = w.w;
-      }
+        for (int kk = 0; kk < KS; ++kk) {
+          qb[nb][kk][0] = real ? *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * t) : 0u;
+          qb[nb][kk][1] = real ? *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * t + 8) : 0u;
+        }
+        sscale[nb][0] = sscale[nb][1] = a.score_scale;
+      } else {
+        // this lane's q elements: [BPT*t, BPT*t + BPT)
+        float mx = 0.f;
+        uint32_t qw[BPT / 2];
 #pragma unroll
-      for (int i = 0; i < BPT / 2; ++i)
-        mx = fmaxf(mx, fmaxf(fabsf(bf16lo(qw[i])), fabsf(bf16hi(qw[i]))));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      int ex = 0;
-      frexpf(mx, &ex);
-      int sh = 0;
-      if constexpr (kQSplit) {
-        sh = (mx > 0.f && isfinite(mx)) ? 8 - ex : 0;  // max |q| * 2^sh in [128, 256)
-        const float mul = ldexpf(1.f, sh);
+        for (int i = 0; i < BPT / 8; ++i) {
+          const uint4 w = real ? *reinterpret_cast<const uint4*>(qrow + BPT * t + 8 * i)
+                               : make_uint4(0, 0, 0, 0);
+          qw[4 * i] = w.x;
+          qw[4 * i + 1] = w.y;
+          qw[4 * i + 2] = w.z;
+          qw[4 * i + 3] = w.w;
+        }
 #pragma unroll
-        for (int kk = 0; kk < KS32; ++kk) {
+        for (int i = 0; i < BPT / 2; ++i)
+          mx = fmaxf(mx, fmaxf(fabsf(bf16lo(qw[i])), fabsf(bf16hi(qw[i]))));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        int ex = 0;
+        frexpf(mx, &ex);
+        int sh = 0;
+        if constexpr (kQSplit) {
+          sh = (mx > 0.f && isfinite(mx)) ? 8 - ex : 0;  // max |q| * 2^sh in [128, 256)
+          const float mul = ldexpf(1.f, sh);
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            // logical k-columns 4t..4t+3 (half 0) / 16+4t..16+4t+3 (half 1) of
-            // step kk <-> dims BPT*t + 8kk + 4*half + 0..3
-            const uint32_t wa = qw[4 * kk + 2 * half], wb = qw[4 * kk + 2 * half + 1];
-            float x0 = bf16lo(wa) * mul, x1 = bf16hi(wa) * mul;
-            float x2 = bf16lo(wb) * mul, x3 = bf16hi(wb) * mul;
+          for (int kk = 0; kk < KS32; ++kk) {
 #pragma unroll
-            for (int part = 0; part < 3; ++part) {
-              const uint16_t e01 = float2_to_e4m3x2(x0, x1), e23 = float2_to_e4m3x2(x2, x3);
-              qb8[kk][part][half] = static_cast<uint32_t>(e01) | (static_cast<uint32_t>(e23) << 16);
-              if (part < 2) {  // the next part carries what this one missed
-                const float2 d01 = f16x2_to_float2(e4m3x2_to_f16x2(e01));
-                const float2 d23 = f16x2_to_float2(e4m3x2_to_f16x2(e23));
-                x0 -= d01.x;
-                x1 -= d01.y;
-                x2 -= d23.x;
-                x3 -= d23.y;
+            for (int half = 0; half < 2; ++half) {
+              // logical k-columns 4t..4t+3 (half 0) / 16+4t..16+4t+3 (half 1) of
+              // step kk <-> dims BPT*t + 8kk + 4*half + 0..3
+              const uint32_t wa = qw[4 * kk + 2 * half], wb = qw[4 * kk + 2 * half + 1];
+              float x0 = bf16lo(wa) * mul, x1 = bf16hi(wa) * mul;
+              float x2 = bf16lo(wb) * mul, x3 = bf16hi(wb) * mul;
+#pragma unroll
+              for (int part = 0; part < 3; ++part) {
+                const uint16_t e01 = float2_to_e4m3x2(x0, x1), e23 = float2_to_e4m3x2(x2, x3);
+                qb8[kk][part][half] = static_cast<uint32_t>(e01) | (static_cast<uint32_t>(e23) << 16);
+                if (part < 2) {  // the next part carries what this one missed
+                  const float2 d01 = f16x2_to_float2(e4m3x2_to_f16x2(e01));
+                  const float2 d23 = f16x2_to_float2(e4m3x2_to_f16x2(e23));
+                  x0 -= d01.x;
+                  x1 -= d01.y;
+                  x2 -= d23.x;
+                  x3 -= d23.y;
+                }
               }
             }
           }
-        }
-      } else {
-        sh = (mx > 0.f && isfinite(mx)) ? 15 - ex : 0;  // |q| * 2^sh < 2^15
-        const float mul = ldexpf(1.f, sh);
+        } else {
+          sh = (mx > 0.f && isfinite(mx)) ? 15 - ex : 0;  // |q| * 2^sh < 2^15
+          const float mul = ldexpf(1.f, sh);
 #pragma unroll
-        for (int kk = 0; kk < KS; ++kk) {
-          if constexpr (FP8) {
-            // logical k-columns 2t,2t+1 / 2t+8,2t+9 of step kk <-> bytes BPT*t + 4kk + {0,1} / {2,3}
-            const uint32_t w0 = qw[2 * kk], w1 = qw[2 * kk + 1];
-            qb[kk][0] = pack_f16x2(bf16lo(w0) * mul, bf16hi(w0) * mul);
-            qb[kk][1] = pack_f16x2(bf16lo(w1) * mul, bf16hi(w1) * mul);
-          } else {
-            // int4: logical k-columns 2t,2t+1 / 2t+8,2t+9 of step kk <-> the
-            // lane's elements (8j + 2c, 8j + 2c + 4) / (8j + 2c + 1, 8j + 2c + 5),
-            // j = kk / 2, c = kk % 2: the nibble pairs one shift and one mask
-            // take out of K's 32-bit word j
-            const int e = 8 * (kk >> 1) + 2 * (kk & 1);
-            auto qe = [&](int i) { return (i & 1) ? bf16hi(qw[i >> 1]) : bf16lo(qw[i >> 1]); };
-            qb[kk][0] = pack_f16x2(qe(e) * mul, qe(e + 4) * mul);
-            qb[kk][1] = pack_f16x2(qe(e + 1) * mul, qe(e + 5) * mul);
+          for (int kk = 0; kk < KS; ++kk) {
+            if constexpr (FP8) {
+              // logical k-columns 2t,2t+1 / 2t+8,2t+9 of step kk <-> bytes BPT*t + 4kk + {0,1} / {2,3}
+              const uint32_t w0 = qw[2 * kk], w1 = qw[2 * kk + 1];
+              qb[nb][kk][0] = pack_f16x2(bf16lo(w0) * mul, bf16hi(w0) * mul);
+              qb[nb][kk][1] = pack_f16x2(bf16lo(w1) * mul, bf16hi(w1) * mul);
+            } else {
+              // int4: logical k-columns 2t,2t+1 / 2t+8,2t+9 of step kk <-> the
+              // lane's elements (8j + 2c, 8j + 2c + 4) / (8j + 2c + 1, 8j + 2c + 5),
+              // j = kk / 2, c = kk % 2: the nibble pairs one shift and one mask
+              // take out of K's 32-bit word j
+              const int e = 8 * (kk >> 1) + 2 * (kk & 1);
+              auto qe = [&](int i) { return (i & 1) ? bf16hi(qw[i >> 1]) : bf16lo(qw[i >> 1]); };
+              qb[nb][kk][0] = pack_f16x2(qe(e) * mul, qe(e + 4) * mul);
+              qb[nb][kk][1] = pack_f16x2(qe(e + 1) * mul, qe(e + 5) * mul);
+            }
           }
         }
+        const int sh0 = __shfl_sync(0xffffffffu, sh, (2 * t) * 4);
+        const int sh1 = __shfl_sync(0xffffffffu, sh, (2 * t + 1) * 4);
+        const float base = a.score_scale * kscale;
+        sscale[nb][0] = base * ldexpf(1.f, -sh0);
+        sscale[nb][1] = base * ldexpf(1.f, -sh1);
       }
-      const int sh0 = __shfl_sync(0xffffffffu, sh, (2 * t) * 4);
-      const int sh1 = __shfl_sync(0xffffffffu, sh, (2 * t + 1) * 4);
-      const float base = a.score_scale * kscale;
-      sscale[0] = base * ldexpf(1.f, -sh0);
-      sscale[1] = base * ldexpf(1.f, -sh1);
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[nb][mt][i] = 0.f;
+      m[nb][0] = m[nb][1] = a.m_init;
+      l[nb][0] = l[nb][1] = 0.f;
     }
-#pragma unroll
-    for (int mt = 0; mt < KS; ++mt)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) o[mt][i] = 0.f;
-    m[0] = m[1] = a.m_init;
-    l[0] = l[1] = 0.f;
-    fresh = a.m_init > -CUDART_INF_F ? 3u : 0u;
+    fresh = a.m_init > -CUDART_INF_F ? (1u << (2 * NB)) - 1u : 0u;
   }
 
   __device__ __forceinline__ uint32_t chunk_addr(uint32_t tile, int row, int chunk, int swz) const {
@@ -807,12 +816,17 @@ struct MmaConsumer {
       return tile + row * C::ROWB + off;
   }
 
-  // Two accumulators (even / odd k-steps) halve the dependent chain of mma.
+  // One subtile's scores for every row block: each K fragment is read (or
+  // widened) once and feeds NB products.  Two accumulators per block (even /
+  // odd k-steps) halve the dependent chain of mma.
   __device__ __forceinline__ void scores(const KernelArgs& a, uint32_t kt, int sub, int lane,
-                                         float (&c)[4]) const {
+                                         float (&c)[NB][4]) const {
     const int swz = a.swz;
-    float c2[4] = {0.f, 0.f, 0.f, 0.f};
-    c[0] = c[1] = c[2] = c[3] = 0.f;
+    float c2[NB][4];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) c[nb][i] = c2[nb][i] = 0.f;
     if constexpr (BF16) {
       const int row = sub * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
@@ -823,10 +837,13 @@ struct MmaConsumer {
           ldsm_x4(ldsm_addr_in(a.status, chunk_addr(kt, srow(row), ch, swz), kt, C::TILE_BYTES, 201), af);
         else  // 64-element rows: one plane of CB bytes, no swizzle
           ldsm_x4(ldsm_addr_in(a.status, kt + srow(row) * C::CB + ch * 16, kt, C::TILE_BYTES, 202), af);
-        if (kk & 1)
-          mma_bf16(c2, af, qb[kk][0], qb[kk][1]);
-        else
-          mma_bf16(c, af, qb[kk][0], qb[kk][1]);
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+          if (kk & 1)
+            mma_bf16(c2[nb], af, qb[nb][kk][0], qb[nb][kk][1]);
+          else
+            mma_bf16(c[nb], af, qb[nb][kk][0], qb[nb][kk][1]);
+        }
       }
     } else {
       const int r0 = sub * 16 + g, r1 = r0 + 8;
@@ -846,45 +863,44 @@ struct MmaConsumer {
           // A (16 tokens x 32 dims, e4m3): rows g / g+8, logical k 4t..4t+3
           // and 16+4t..16+4t+3 <-> words 2kk and 2kk+1 of the lane's bytes
           const uint32_t af[4] = {w0[2 * kk], w1[2 * kk], w0[2 * kk + 1], w1[2 * kk + 1]};
-          mma_e4m3(c, af, qb8[kk][0][0], qb8[kk][0][1]);
-          mma_e4m3(c2, af, qb8[kk][1][0], qb8[kk][1][1]);
+          mma_e4m3(c[0], af, qb8[kk][0][0], qb8[kk][0][1]);
+          mma_e4m3(c2[0], af, qb8[kk][1][0], qb8[kk][1][1]);
           mma_e4m3(c3, af, qb8[kk][2][0], qb8[kk][2][1]);
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) c2[i] += c3[i];
-      } else if constexpr (I4) {
-#pragma unroll
-        for (int kk = 0; kk < KS; ++kk) {
-          // word kk / 2 of each row; pairs (8c, 8c + 4) bits up: the nibble
-          // pairs of the lane's elements listed in begin_piece
-          const int sh = 8 * (kk & 1);
-          uint32_t af[4];
-          af[0] = int4x2_to_f16x2(w0[kk >> 1] >> sh);
-          af[1] = int4x2_to_f16x2(w1[kk >> 1] >> sh);
-          af[2] = int4x2_to_f16x2(w0[kk >> 1] >> (sh + 4));
-          af[3] = int4x2_to_f16x2(w1[kk >> 1] >> (sh + 4));
-          if (kk & 1)
-            mma_f16(c2, af, qb[kk][0], qb[kk][1]);
-          else
-            mma_f16(c, af, qb[kk][0], qb[kk][1]);
-        }
+        for (int i = 0; i < 4; ++i) c2[0][i] += c3[i];
       } else {
 #pragma unroll
         for (int kk = 0; kk < KS; ++kk) {
           uint32_t af[4];
-          af[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(w0[kk] & 0xFFFFu));
-          af[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[kk] & 0xFFFFu));
-          af[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(w0[kk] >> 16));
-          af[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[kk] >> 16));
-          if (kk & 1)
-            mma_f16(c2, af, qb[kk][0], qb[kk][1]);
-          else
-            mma_f16(c, af, qb[kk][0], qb[kk][1]);
+          if constexpr (I4) {
+            // word kk / 2 of each row; pairs (8c, 8c + 4) bits up: the nibble
+            // pairs of the lane's elements listed in begin_piece
+            const int sh = 8 * (kk & 1);
+            af[0] = int4x2_to_f16x2(w0[kk >> 1] >> sh);
+            af[1] = int4x2_to_f16x2(w1[kk >> 1] >> sh);
+            af[2] = int4x2_to_f16x2(w0[kk >> 1] >> (sh + 4));
+            af[3] = int4x2_to_f16x2(w1[kk >> 1] >> (sh + 4));
+          } else {
+            af[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(w0[kk] & 0xFFFFu));
+            af[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[kk] & 0xFFFFu));
+            af[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(w0[kk] >> 16));
+            af[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[kk] >> 16));
+          }
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) {
+            if (kk & 1)
+              mma_f16(c2[nb], af, qb[nb][kk][0], qb[nb][kk][1]);
+            else
+              mma_f16(c[nb], af, qb[nb][kk][0], qb[nb][kk][1]);
+          }
         }
       }
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) c[i] += c2[i];
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) c[nb][i] += c2[nb][i];
   }
 
   // One tile: the scores of all SUB subtiles first (independent mma chains),
@@ -893,96 +909,115 @@ struct MmaConsumer {
   template <class ReleaseK>
   __device__ __forceinline__ void tile(const KernelArgs& a, uint32_t kt, uint32_t vt, int pos0,
                                        int lo, int hi, int lane, ReleaseK&& release_k) {
-    float sc[SUB][4];
+    float sc[SUB][NB][4];
 #pragma unroll
     for (int sub = 0; sub < SUB; ++sub) scores(a, kt, sub, lane, sc[sub]);
     release_k();
-    // key range of this lane's two columns (rows 2t, 2t + 1: query token
-    // row / group sees one key fewer per token before the last, within its
-    // own window); [lo, hi) is the union, and padding columns keep it
-    int chi0 = hi - (a.q_len - 1 - (rbase + 2 * t) / a.group);
-    int chi1 = hi - (a.q_len - 1 - (rbase + 2 * t + 1) / a.group);
-    chi0 = chi0 < hi ? chi0 : hi;
-    chi1 = chi1 < hi ? chi1 : hi;
-    const int clo0 = (a.window > 0 && chi0 > a.window) ? chi0 - a.window : 0;
-    const int clo1 = (a.window > 0 && chi1 > a.window) ? chi1 - a.window : 0;
-    float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F;
+    float mx[NB][2];
+    bool up = false;
 #pragma unroll
-    for (int sub = 0; sub < SUB; ++sub) {
-      const int pr = pos0 + sub * 16 + g;
-      const bool v00 = pr >= clo0 && pr < chi0, v01 = pr >= clo1 && pr < chi1;
-      const bool v80 = pr + 8 >= clo0 && pr + 8 < chi0, v81 = pr + 8 >= clo1 && pr + 8 < chi1;
-      sc[sub][0] = v00 ? sc[sub][0] * sscale[0] : -CUDART_INF_F;
-      sc[sub][1] = v01 ? sc[sub][1] * sscale[1] : -CUDART_INF_F;
-      sc[sub][2] = v80 ? sc[sub][2] * sscale[0] : -CUDART_INF_F;
-      sc[sub][3] = v81 ? sc[sub][3] * sscale[1] : -CUDART_INF_F;
-      if (a.cap_l2 > 0.f) {  // soft-cap: c tanh(s / c) (log2 units; -inf stays -inf)
+    for (int nb = 0; nb < NB; ++nb) {
+      // key range of this lane's two columns (rows 8 nb + 2t, + 1: query
+      // token row / group sees one key fewer per token before the last,
+      // within its own window); [lo, hi) is the union, and padding columns
+      // keep it
+      const int rr = rbase + 8 * nb + 2 * t;
+      int chi0 = hi - (a.q_len - 1 - rr / a.group);
+      int chi1 = hi - (a.q_len - 1 - (rr + 1) / a.group);
+      chi0 = chi0 < hi ? chi0 : hi;
+      chi1 = chi1 < hi ? chi1 : hi;
+      const int clo0 = (a.window > 0 && chi0 > a.window) ? chi0 - a.window : 0;
+      const int clo1 = (a.window > 0 && chi1 > a.window) ? chi1 - a.window : 0;
+      float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) sc[sub][e] = a.cap_l2 * tanhf(sc[sub][e] / a.cap_l2);
-      }
-      mx0 = fmaxf(mx0, fmaxf(sc[sub][0], sc[sub][2]));
-      mx1 = fmaxf(mx1, fmaxf(sc[sub][1], sc[sub][3]));
-    }
+      for (int sub = 0; sub < SUB; ++sub) {
+        float* s = sc[sub][nb];
+        const int pr = pos0 + sub * 16 + g;
+        const bool v00 = pr >= clo0 && pr < chi0, v01 = pr >= clo1 && pr < chi1;
+        const bool v80 = pr + 8 >= clo0 && pr + 8 < chi0, v81 = pr + 8 >= clo1 && pr + 8 < chi1;
+        s[0] = v00 ? s[0] * sscale[nb][0] : -CUDART_INF_F;
+        s[1] = v01 ? s[1] * sscale[nb][1] : -CUDART_INF_F;
+        s[2] = v80 ? s[2] * sscale[nb][0] : -CUDART_INF_F;
+        s[3] = v81 ? s[3] * sscale[nb][1] : -CUDART_INF_F;
+        if (a.cap_l2 > 0.f) {  // soft-cap: c tanh(s / c) (log2 units; -inf stays -inf)
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-    }
-    if (fresh != 0u) {  // unified max: the rows' first finite scores (row-uniform: mx is reduced)
-      if ((fresh & 1u) && mx0 > -CUDART_INF_F) {
-        if (mx0 < m[0] - kPhiDrop) m[0] = mx0;
-        fresh &= ~1u;
+          for (int e = 0; e < 4; ++e) s[e] = a.cap_l2 * tanhf(s[e] / a.cap_l2);
+        }
+        mx0 = fmaxf(mx0, fmaxf(s[0], s[2]));
+        mx1 = fmaxf(mx1, fmaxf(s[1], s[3]));
       }
-      if ((fresh & 2u) && mx1 > -CUDART_INF_F) {
-        if (mx1 < m[1] - kPhiDrop) m[1] = mx1;
-        fresh &= ~2u;
-      }
-    }
-    const bool up0 = mx0 > m[0] + kRescaleSlack, up1 = mx1 > m[1] + kRescaleSlack;
-    if (__any_sync(0xffffffffu, up0 || up1)) {
-      const float a0 = up0 ? exp2_approx(m[0] - mx0) : 1.f;
-      const float a1 = up1 ? exp2_approx(m[1] - mx1) : 1.f;
-      if (up0) m[0] = mx0;
-      if (up1) m[1] = mx1;
-      l[0] *= a0;
-      l[1] *= a1;
 #pragma unroll
-      for (int mt = 0; mt < KS; ++mt) {
-        o[mt][0] *= a0;
-        o[mt][1] *= a1;
-        o[mt][2] *= a0;
-        o[mt][3] *= a1;
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+      }
+      if (fresh != 0u) {  // unified max: the rows' first finite scores (row-uniform: mx is reduced)
+        const uint32_t b0 = 1u << (2 * nb), b1 = b0 << 1;
+        if ((fresh & b0) && mx0 > -CUDART_INF_F) {
+          if (mx0 < m[nb][0] - kPhiDrop) m[nb][0] = mx0;
+          fresh &= ~b0;
+        }
+        if ((fresh & b1) && mx1 > -CUDART_INF_F) {
+          if (mx1 < m[nb][1] - kPhiDrop) m[nb][1] = mx1;
+          fresh &= ~b1;
+        }
+      }
+      mx[nb][0] = mx0;
+      mx[nb][1] = mx1;
+      up |= mx0 > m[nb][0] + kRescaleSlack || mx1 > m[nb][1] + kRescaleSlack;
+    }
+    if (__any_sync(0xffffffffu, up)) {
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        const bool up0 = mx[nb][0] > m[nb][0] + kRescaleSlack, up1 = mx[nb][1] > m[nb][1] + kRescaleSlack;
+        const float a0 = up0 ? exp2_approx(m[nb][0] - mx[nb][0]) : 1.f;
+        const float a1 = up1 ? exp2_approx(m[nb][1] - mx[nb][1]) : 1.f;
+        if (up0) m[nb][0] = mx[nb][0];
+        if (up1) m[nb][1] = mx[nb][1];
+        l[nb][0] *= a0;
+        l[nb][1] *= a1;
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+          o[nb][mt][0] *= a0;
+          o[nb][mt][1] *= a1;
+          o[nb][mt][2] *= a0;
+          o[nb][mt][3] *= a1;
+        }
       }
     }
-    const bool dead0 = m[0] == -CUDART_INF_F, dead1 = m[1] == -CUDART_INF_F;
     // P enters the tensor core as hi + lo 16-bit parts (two products), so the
     // weights keep ~16 significant bits instead of 8 (bf16) or 11 (f16).
-    uint32_t pb[SUB][4];
+    uint32_t pb[SUB][NB][4];
 #pragma unroll
-    for (int sub = 0; sub < SUB; ++sub) {
-      const float p0 = dead0 ? 0.f : exp2_approx(sc[sub][0] - m[0]);
-      const float p1 = dead1 ? 0.f : exp2_approx(sc[sub][1] - m[1]);
-      const float p2 = dead0 ? 0.f : exp2_approx(sc[sub][2] - m[0]);
-      const float p3 = dead1 ? 0.f : exp2_approx(sc[sub][3] - m[1]);
-      l[0] += p0 + p2;
-      l[1] += p1 + p3;
-      uint32_t x0, x1, y0, y1;
-      if constexpr (!BF16) {  // the f16 product of the fp8 / int4 dataflow
-        x0 = pack_f16x2(p0, p1);
-        x1 = pack_f16x2(p2, p3);
-        const float2 h0 = f16x2_to_float2(x0), h1 = f16x2_to_float2(x1);
-        y0 = pack_f16x2(p0 - h0.x, p1 - h0.y);
-        y1 = pack_f16x2(p2 - h1.x, p3 - h1.y);
-      } else {
-        x0 = pack_bf16x2(p0, p1);
-        x1 = pack_bf16x2(p2, p3);
-        y0 = pack_bf16x2(p0 - bf16lo(x0), p1 - bf16hi(x0));
-        y1 = pack_bf16x2(p2 - bf16lo(x1), p3 - bf16hi(x1));
+    for (int nb = 0; nb < NB; ++nb) {
+      const bool dead0 = m[nb][0] == -CUDART_INF_F, dead1 = m[nb][1] == -CUDART_INF_F;
+#pragma unroll
+      for (int sub = 0; sub < SUB; ++sub) {
+        const float* s = sc[sub][nb];
+        const float p0 = dead0 ? 0.f : exp2_approx(s[0] - m[nb][0]);
+        const float p1 = dead1 ? 0.f : exp2_approx(s[1] - m[nb][1]);
+        const float p2 = dead0 ? 0.f : exp2_approx(s[2] - m[nb][0]);
+        const float p3 = dead1 ? 0.f : exp2_approx(s[3] - m[nb][1]);
+        l[nb][0] += p0 + p2;
+        l[nb][1] += p1 + p3;
+        uint32_t x0, x1, y0, y1;
+        if constexpr (!BF16) {  // the f16 product of the fp8 / int4 dataflow
+          x0 = pack_f16x2(p0, p1);
+          x1 = pack_f16x2(p2, p3);
+          const float2 h0 = f16x2_to_float2(x0), h1 = f16x2_to_float2(x1);
+          y0 = pack_f16x2(p0 - h0.x, p1 - h0.y);
+          y1 = pack_f16x2(p2 - h1.x, p3 - h1.y);
+        } else {
+          x0 = pack_bf16x2(p0, p1);
+          x1 = pack_bf16x2(p2, p3);
+          y0 = pack_bf16x2(p0 - bf16lo(x0), p1 - bf16hi(x0));
+          y1 = pack_bf16x2(p2 - bf16lo(x1), p3 - bf16hi(x1));
+        }
+        pb[sub][nb][0] = movmatrix_trans(x0);  // P[row g][tokens 2t, 2t+1]
+        pb[sub][nb][1] = movmatrix_trans(x1);  // P[row g][tokens 2t+8, 2t+9]
+        pb[sub][nb][2] = movmatrix_trans(y0);
+        pb[sub][nb][3] = movmatrix_trans(y1);
       }
-      pb[sub][0] = movmatrix_trans(x0);  // P[head g][tokens 2t, 2t+1]
-      pb[sub][1] = movmatrix_trans(x1);  // P[head g][tokens 2t+8, 2t+9]
-      pb[sub][2] = movmatrix_trans(y0);
-      pb[sub][3] = movmatrix_trans(y1);
     }
 #pragma unroll
     for (int sub = 0; sub < SUB; ++sub) {
@@ -1009,8 +1044,11 @@ struct MmaConsumer {
             af[2] &= mk89;
             af[3] &= mk89;
           }
-          mma_bf16(o[mt], af, pb[sub][0], pb[sub][1]);
-          mma_bf16(o[mt], af, pb[sub][2], pb[sub][3]);
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) {
+            mma_bf16(o[nb][mt], af, pb[sub][nb][0], pb[sub][nb][1]);
+            mma_bf16(o[nb][mt], af, pb[sub][nb][2], pb[sub][nb][3]);
+          }
         }
       } else if constexpr (I4) {
         // lane owns dims [VBT*g, VBT*g + VBT) (VB bytes) of tokens 2t, 2t+1,
@@ -1053,8 +1091,11 @@ struct MmaConsumer {
             af[2] &= mk89;
             af[3] &= mk89;
           }
-          mma_f16(o[mt], af, pb[sub][0], pb[sub][1]);
-          mma_f16(o[mt], af, pb[sub][2], pb[sub][3]);
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) {
+            mma_f16(o[nb][mt], af, pb[sub][nb][0], pb[sub][nb][1]);
+            mma_f16(o[nb][mt], af, pb[sub][nb][2], pb[sub][nb][3]);
+          }
         }
       } else {
         // lane owns dims [VBT*g, VBT*g + VBT) of tokens 2t, 2t+1, 2t+8, 2t+9
@@ -1088,8 +1129,11 @@ struct MmaConsumer {
             af[2] &= mk89;
             af[3] &= mk89;
           }
-          mma_f16(o[mt], af, pb[sub][0], pb[sub][1]);
-          mma_f16(o[mt], af, pb[sub][2], pb[sub][3]);
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) {
+            mma_f16(o[nb][mt], af, pb[sub][nb][0], pb[sub][nb][1]);
+            mma_f16(o[nb][mt], af, pb[sub][nb][2], pb[sub][nb][3]);
+          }
         }
       }
     }
@@ -1105,29 +1149,34 @@ struct MmaConsumer {
   // Park this warp's state for its team's rows as tile lane w's state.
   __device__ __forceinline__ void end_piece(float* m_area, float* l_area, float* acc_area, int w,
                                             int lane, int G) {
-    float l0 = l[0], l1 = l[1];
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-    }
-    const int h0 = rbase + 2 * t, h1 = h0 + 1;
-    const bool r0 = 2 * t < tr && h0 < G, r1 = 2 * t + 1 < tr && h1 < G;
-    if (g == 0) {  // a row that saw no finite score holds nothing: max -inf (not phi)
-      if (r0) m_area[w * G + h0] = (fresh & 1u) ? -CUDART_INF_F : m[0];
-      if (r1) m_area[w * G + h1] = (fresh & 2u) ? -CUDART_INF_F : m[1];
-      if (r0) l_area[w * G + h0] = l0;
-      if (r1) l_area[w * G + h1] = l1;
-    }
+    for (int nb = 0; nb < NB; ++nb) {
+      float l0 = l[nb][0], l1 = l[nb][1];
 #pragma unroll
-    for (int mt = 0; mt < KS; ++mt) {
-      if (r0) {
-        acc_area[(w * G + h0) * D + out_dim(mt, 0)] = o[mt][0];
-        acc_area[(w * G + h0) * D + out_dim(mt, 1)] = o[mt][2];
+      for (int off = 4; off < 32; off <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, off);
       }
-      if (r1) {
-        acc_area[(w * G + h1) * D + out_dim(mt, 0)] = o[mt][1];
-        acc_area[(w * G + h1) * D + out_dim(mt, 1)] = o[mt][3];
+      const int lr = 8 * nb + 2 * t;  // team-local row of column 0
+      const int h0 = rbase + lr, h1 = h0 + 1;
+      const bool r0 = lr < tr && h0 < G, r1 = lr + 1 < tr && h1 < G;
+      const uint32_t b0 = 1u << (2 * nb), b1 = b0 << 1;
+      if (g == 0) {  // a row that saw no finite score holds nothing: max -inf (not phi)
+        if (r0) m_area[w * G + h0] = (fresh & b0) ? -CUDART_INF_F : m[nb][0];
+        if (r1) m_area[w * G + h1] = (fresh & b1) ? -CUDART_INF_F : m[nb][1];
+        if (r0) l_area[w * G + h0] = l0;
+        if (r1) l_area[w * G + h1] = l1;
+      }
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        if (r0) {
+          acc_area[(w * G + h0) * D + out_dim(mt, 0)] = o[nb][mt][0];
+          acc_area[(w * G + h0) * D + out_dim(mt, 1)] = o[nb][mt][2];
+        }
+        if (r1) {
+          acc_area[(w * G + h1) * D + out_dim(mt, 0)] = o[nb][mt][1];
+          acc_area[(w * G + h1) * D + out_dim(mt, 1)] = o[nb][mt][3];
+        }
       }
     }
   }
