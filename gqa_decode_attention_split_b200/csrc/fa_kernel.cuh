@@ -632,8 +632,8 @@ struct SimtConsumer {
 // the query heads of a kv head times the query tokens).  A team's warp
 // computes its rows of every tile it takes, in NB blocks of 8 that share
 // each K / V fragment (one shared-memory read or conversion feeds NB
-// products).  Multi-row variants use 32-token tiles, so that the tile lanes
-// keep a deep ring.
+// products).  Several teams use 32-token tiles, so that the fewer tile
+// lanes keep a deep ring.
 // KIND: bf16 (tiles through ldmatrix), fp8 e4m3 or int4 (bytes loaded per
 // lane and widened to f16; the query is held as f16 times a power of two).
 // HEADS: the R teams are R adjacent kv heads of one segment instead of R
@@ -648,8 +648,11 @@ struct MmaConsumer {
   static_assert(NB == 1 || NB == 2, "one or two row blocks per warp");
   static_assert(!HEADS || NB == 1, "head teams hold one row block");
   static constexpr int ROWB_K = BF16 ? 2 * D : (FP8 ? D : D / 2);  // bytes of one head's row
+  // Two row blocks: 64-token tiles with one team (a few spilled registers,
+  // measured 5% faster than 32 tokens at 16 rows), 32 with two teams (64
+  // would leave 3 ring slots: 7% slower at 32 rows).
   static constexpr int kTileBytes = HEADS ? 16384
-                                    : NB > 1 ? 32 * ROWB_K
+                                    : NB > 1 ? (R == 1 ? 64 : 32) * ROWB_K
                                     : FP8 ? FA_FP8_MMA_TILE_BYTES
                                     : I4  ? FA_FP8_MMA_TILE_BYTES / 2
                                           : (R == 1 ? FA_MMA_TILE_BYTES : FA_MMA_TILE_BYTES / 2);

@@ -255,11 +255,12 @@ def test_plan_with_several_query_tokens(lib):
 
 
 def test_row_team_variants(lib):
-    """Segments of 9..32 rows take the MMA variants with two or four row
-    teams: bf16 tiles of 32 tokens, equal K and V rings, a larger grid of
-    threads; 8 rows or fewer keep the single-team variant."""
-    cases = [(dict(qo_heads=8, kv_heads=8), 1, 64), (dict(qo_heads=16, kv_heads=1), 2, 32),
-             (dict(qo_heads=32, kv_heads=8, q_len=3), 2, 32),
+    """Segments of 9..32 rows take the MMA variants whose warps hold two row
+    blocks of 8 (head_dim 128): one team with 64-token tiles up to 16 rows,
+    two teams with 32-token tiles up to 32, equal K and V rings; 8 rows or
+    fewer keep the one-block variant."""
+    cases = [(dict(qo_heads=8, kv_heads=8), 1, 64), (dict(qo_heads=16, kv_heads=1), 2, 64),
+             (dict(qo_heads=32, kv_heads=8, q_len=3), 2, 64),
              (dict(qo_heads=32, kv_heads=8, q_len=8), 4, 32),
              (dict(qo_heads=32, kv_heads=1), 4, 32)]
     for kw, teams, T in cases:
