@@ -423,3 +423,35 @@ def test_head_tile_choice(lib):
         assert _info(lib, h).heads_per_tile == ht, kw
         lib.fa_plan_destroy(h)
 
+
+
+def _largest_plannable_batch(lib, **kw):
+    def ok(batch):
+        lens = np.full(batch, 20)
+        st, h, _ = _plan(lib, _desc(batch=batch, paged=1, page_size=16, **kw),
+                         np.concatenate([[0], np.cumsum(lens)]))
+        if h.value:
+            lib.fa_plan_destroy(h)
+        assert st in (0, 2)
+        return st == 0
+    lo, hi = 1, 1 << 17
+    assert ok(lo) and not ok(hi)
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        lo, hi = (mid, hi) if ok(mid) else (lo, mid)
+    return lo
+
+
+def test_plan_batch_limit(lib):
+    """A block keeps every request's start, length and tile prefix in shared
+    memory next to its tile ring: the planner accepts every batch whose
+    block fits the 227 KB of shared memory and refuses larger ones as
+    unsupported (never a device fault); at least 682 requests always fit."""
+    for kw in (dict(), dict(kv_dtype=1), dict(path=binding.PATH_SIMT)):
+        top = _largest_plannable_batch(lib, **kw)
+        assert top >= 682, kw
+        lens = np.full(top, 20)
+        st, h, _ = _plan(lib, _desc(batch=top, paged=1, page_size=16, **kw),
+                         np.concatenate([[0], np.cumsum(lens)]))
+        assert st == 0 and _info(lib, h).smem_bytes <= 232448
+        lib.fa_plan_destroy(h)

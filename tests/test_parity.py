@@ -459,3 +459,39 @@ def test_unified_max_matches_the_oracle(case, path, phi):
         assert binding.decode_status(ws) == 0
         o, l = to_numpy(out, lse)
         assert_matches(o, l, ref_out, ref_lse, what=f"{name} {path} phi={phi} ctas={n}")
+
+
+# ------------------------------------------------------------------ limits
+def test_largest_batch():
+    """The largest batch the planner accepts for this shape (its block's
+    schedule arrays fill the shared memory the tile ring leaves), short and
+    ragged requests, paged: every row against the oracle."""
+    import ctypes
+    lib = binding.load_library()
+
+    def ok(batch):
+        d = binding.DecodeDesc(batch=batch, qo_heads=8, kv_heads=2, head_dim=128, kv_dtype=0,
+                               paged=1, page_size=16, window=-1, sm_scale=0.1, path=0,
+                               num_ctas=0)
+        ind = np.arange(batch + 1, dtype=np.int32) * 20
+        h, ws = ctypes.c_void_p(), ctypes.c_size_t()
+        st = lib.fa_decode_plan(ctypes.byref(d), ind.ctypes.data, 0, ctypes.byref(h),
+                                ctypes.byref(ws))
+        if h.value:
+            lib.fa_plan_destroy(h)
+        return st == 0
+    lo, hi = 682, 1 << 17
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        lo, hi = (mid, hi) if ok(mid) else (lo, mid)
+    rng = np.random.default_rng(50)
+    lens = rng.integers(0, 70, size=lo)
+    x = synth.generate(lo, 8, 2, 128, list(lens), paged=True, page_size=16, seed=51)
+    _check(x)
+
+
+def test_one_million_keys():
+    """One request of 2^20 keys (fp8, GQA 8 on one kv head): sampled rows
+    against the oracle."""
+    x = synth.generate(1, 8, 1, 128, [1 << 20], kv_dtype="fp8_e4m3", seed=52)
+    _check_full(x, path="mma", nrows=4, seed=5)
