@@ -35,12 +35,23 @@ void build_registry() {
   g_num_entries = n;
 }
 
-const KernelEntry* find_entry(int head_dim, int group, int kv_kind, int path) {
+// A paged tile is filled one page per box (pages shorter than the tile) or
+// from one page (pages at least as long): the page size and the tile length
+// must divide one another, or a tile would get too few copies, or a box
+// would run past its page into an unrelated one.
+bool tile_fits_pages(int tile_tokens, int page_size) {
+  if (page_size <= 0) return true;  // contiguous
+  return page_size < tile_tokens ? tile_tokens % page_size == 0 : page_size % tile_tokens == 0;
+}
+
+// The first variant (registry order) for the shape whose tiles fit the pages.
+const KernelEntry* find_entry(int head_dim, int group, int kv_kind, int path, int page_size) {
   std::call_once(g_registry_once, build_registry);
   for (int i = 0; i < g_num_entries; ++i) {
     const KernelEntry& e = g_entries[i];
     if (e.head_dim != head_dim || e.kv_kind != kv_kind || e.path != path || e.heads_per_tile != 1)
       continue;
+    if (!tile_fits_pages(e.tile_tokens, page_size)) continue;
     if (e.group != 0 ? e.group == group : group <= e.max_group) return &e;
   }
   return nullptr;
@@ -245,6 +256,7 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   // rows of a segment: the group's query heads for every query token
   const int group = desc->qo_heads / desc->kv_heads * q_len_of(desc);
   const int kind = desc->kv_dtype;  // registry kinds follow fa_kv_dtype
+  const int pages = desc->paged ? desc->page_size : 0;
 
   // Dataflow choice.  Asked for: that dataflow.  Otherwise the first row of
   // the measured table that covers the shape (when the grid is not forced),
@@ -253,9 +265,9 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   const KernelEntry* k = nullptr;
   int64_t max_pieces = 32;  // average blocks per segment, at most
   if (desc->path == FA_PATH_SIMT) {
-    k = find_entry(desc->head_dim, group, kind, fa::kPathSimt);
+    k = find_entry(desc->head_dim, group, kind, fa::kPathSimt, pages);
   } else if (desc->path == FA_PATH_MMA) {
-    k = find_entry(desc->head_dim, group, kind, fa::kPathMma);
+    k = find_entry(desc->head_dim, group, kind, fa::kPathMma, pages);
   } else {
     if (desc->num_ctas == 0) {
       const int64_t bytes = visible_kv_bytes(desc, kv_indptr_host);
@@ -263,14 +275,15 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
         if (e.head_dim != desc->head_dim || e.kv_dtype != desc->kv_dtype || group < e.rows_min ||
             group > e.rows_max || bytes < e.bytes_min || bytes > e.bytes_max)
           continue;
-        k = find_entry(desc->head_dim, group, kind, e.path == FA_PATH_SIMT ? fa::kPathSimt : fa::kPathMma);
+        k = find_entry(desc->head_dim, group, kind, e.path == FA_PATH_SIMT ? fa::kPathSimt : fa::kPathMma,
+                       pages);
         if (k == nullptr) continue;
         if (e.max_pieces > 0) max_pieces = e.max_pieces;
         break;
       }
     }
-    if (k == nullptr) k = find_entry(desc->head_dim, group, kind, fa::kPathMma);
-    if (k == nullptr) k = find_entry(desc->head_dim, group, kind, fa::kPathSimt);
+    if (k == nullptr) k = find_entry(desc->head_dim, group, kind, fa::kPathMma, pages);
+    if (k == nullptr) k = find_entry(desc->head_dim, group, kind, fa::kPathSimt, pages);
   }
   if (k == nullptr) return FA_ERR_UNSUPPORTED;
 
@@ -289,12 +302,13 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
         q_len_of(desc) == 1 && group <= 8 &&
         rb < 256 && 256 % rb == 0 && desc->kv_heads % (256 / rb) == 0) {
       const KernelEntry* kh = find_head_entry(desc->head_dim, kind, static_cast<int>(256 / rb));
-      if (kh != nullptr) {
+      if (kh != nullptr && tile_fits_pages(kh->tile_tokens, pages)) {
         k = kh;
         ht = static_cast<int32_t>(256 / rb);
       }
     }
   }
+  if (!tile_fits_pages(k->tile_tokens, pages)) return FA_ERR_UNSUPPORTED;
   const int64_t seg_heads = desc->kv_heads / ht;  // segments per request
   const int seg_rows = group * ht;                // rows of a segment
 

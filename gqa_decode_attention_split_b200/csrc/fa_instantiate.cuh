@@ -85,6 +85,7 @@ int register_variants(KernelEntry* out, int cap, bool with_quant) {
   add(make_entry<MmaConsumer<D, kKvBf16, 1>>(kPathMma, 0, 8, kKvBf16));
   if constexpr (D <= 128) {
     add(make_entry<MmaConsumer<D, kKvBf16, 1, false, 2>>(kPathMma, 0, 16, kKvBf16));
+    add(make_entry<MmaConsumer<D, kKvBf16, 2, false, 2, 48>>(kPathMma, 0, 32, kKvBf16));
     add(make_entry<MmaConsumer<D, kKvBf16, 2, false, 2>>(kPathMma, 0, 32, kKvBf16));
   } else {
     add(make_entry<MmaConsumer<D, kKvBf16, 2>>(kPathMma, 0, 16, kKvBf16));
@@ -99,6 +100,7 @@ int register_variants(KernelEntry* out, int cap, bool with_quant) {
       add(make_entry<MmaConsumer<D, kKvFp8, 1>>(kPathMma, 0, 8, kKvFp8));
       if constexpr (D <= 128) {
         add(make_entry<MmaConsumer<D, kKvFp8, 1, false, 2>>(kPathMma, 0, 16, kKvFp8));
+        add(make_entry<MmaConsumer<D, kKvFp8, 2, false, 2, 48>>(kPathMma, 0, 32, kKvFp8));
         add(make_entry<MmaConsumer<D, kKvFp8, 2, false, 2>>(kPathMma, 0, 32, kKvFp8));
       } else {
         add(make_entry<MmaConsumer<D, kKvFp8, 2>>(kPathMma, 0, 16, kKvFp8));
@@ -111,6 +113,7 @@ int register_variants(KernelEntry* out, int cap, bool with_quant) {
       add(make_entry<MmaConsumer<D, kKvInt4, 1>>(kPathMma, 0, 8, kKvInt4));
       if constexpr (D <= 128) {
         add(make_entry<MmaConsumer<D, kKvInt4, 1, false, 2>>(kPathMma, 0, 16, kKvInt4));
+        add(make_entry<MmaConsumer<D, kKvInt4, 2, false, 2, 48>>(kPathMma, 0, 32, kKvInt4));
         add(make_entry<MmaConsumer<D, kKvInt4, 2, false, 2>>(kPathMma, 0, 32, kKvInt4));
       } else {
         add(make_entry<MmaConsumer<D, kKvInt4, 2>>(kPathMma, 0, 16, kKvInt4));

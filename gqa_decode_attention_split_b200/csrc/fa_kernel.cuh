@@ -639,7 +639,7 @@ struct SimtConsumer {
 // HEADS: the R teams are R adjacent kv heads of one segment instead of R
 // blocks of rows of one kv head: team t computes the (at most 8) query rows
 // of kv head t of the tile, whose rows sit at token * R + t.
-template <int D, int KIND, int R = 1, bool HEADS = false, int NB = 1>
+template <int D, int KIND, int R = 1, bool HEADS = false, int NB = 1, int TOK = 0>
 struct MmaConsumer {
   static constexpr int HT = HEADS ? R : 1;  // kv heads per tile
   static constexpr bool FP8 = KIND == kKvFp8;
@@ -649,9 +649,12 @@ struct MmaConsumer {
   static_assert(!HEADS || NB == 1, "head teams hold one row block");
   static constexpr int ROWB_K = BF16 ? 2 * D : (FP8 ? D : D / 2);  // bytes of one head's row
   // Two row blocks: 64-token tiles with one team (a few spilled registers,
-  // measured 5% faster than 32 tokens at 16 rows), 32 with two teams (64
-  // would leave 3 ring slots: 7% slower at 32 rows).
+  // measured 5% faster than 32 tokens at 16 rows); with two teams TOK
+  // tokens (48 leaves two K and two V slots per tile lane: 7.5% faster than
+  // 32 at 32 rows; 32 serves pages that 48 does not divide).
+  static_assert(TOK == 0 || TOK % 16 == 0, "tiles are whole 16-token subtiles");
   static constexpr int kTileBytes = HEADS ? 16384
+                                    : TOK > 0 ? TOK * ROWB_K
                                     : NB > 1 ? (R == 1 ? 64 : 32) * ROWB_K
                                     : FP8 ? FA_FP8_MMA_TILE_BYTES
                                     : I4  ? FA_FP8_MMA_TILE_BYTES / 2

@@ -257,12 +257,12 @@ def test_plan_with_several_query_tokens(lib):
 def test_row_team_variants(lib):
     """Segments of 9..32 rows take the MMA variants whose warps hold two row
     blocks of 8 (head_dim 128): one team with 64-token tiles up to 16 rows,
-    two teams with 32-token tiles up to 32, equal K and V rings; 8 rows or
+    two teams with 48-token tiles up to 32, equal K and V rings; 8 rows or
     fewer keep the one-block variant."""
     cases = [(dict(qo_heads=8, kv_heads=8), 1, 64), (dict(qo_heads=16, kv_heads=1), 2, 64),
              (dict(qo_heads=32, kv_heads=8, q_len=3), 2, 64),
-             (dict(qo_heads=32, kv_heads=8, q_len=8), 4, 32),
-             (dict(qo_heads=32, kv_heads=1), 4, 32)]
+             (dict(qo_heads=32, kv_heads=8, q_len=8), 4, 48),
+             (dict(qo_heads=32, kv_heads=1), 4, 48)]
     for kw, teams, T in cases:
         st, h, ws = _plan(lib, _desc(path=2, **kw), [0, 5000])
         assert st == 0, kw
@@ -455,3 +455,18 @@ def test_plan_batch_limit(lib):
                          np.concatenate([[0], np.cumsum(lens)]))
         assert st == 0 and _info(lib, h).smem_bytes <= 232448
         lib.fa_plan_destroy(h)
+
+
+def test_tiles_fit_the_pages(lib):
+    """A paged tile is one page per box or a slice of one page, so tile and
+    page lengths must divide one another: 32 rows take 48-token tiles with
+    pages of 16 tokens or fewer, and the 32-token variant with 32- or
+    64-token pages."""
+    for ps, T in ((1, 48), (16, 48), (32, 32), (64, 32), (256, 32)):
+        st, h, _ = _plan(lib, _desc(qo_heads=32, kv_heads=1, paged=1, page_size=ps), [0, 3000])
+        assert st == 0, ps
+        inf = _info(lib, h)
+        assert inf.tile_tokens == T, (ps, inf.tile_tokens)
+        assert (ps % T == 0) if ps >= T else (T % ps == 0)
+        lib.fa_plan_destroy(h)
+

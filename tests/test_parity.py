@@ -284,6 +284,9 @@ MULTI = [
     ("q4_gqa4_paged_rows16", 3, 8, 2, 128, [300, 2, 65], {"q_len": 4, "paged": True, "page_size": 16}),
     ("q8_gqa4_paged_rows32", 3, 8, 2, 128, [411, 17, 96], {"q_len": 8, "paged": True,
                                                            "page_size": 16}),
+    ("q8_gqa4_paged32_rows32", 3, 8, 2, 128, [411, 17, 96], {"q_len": 8, "paged": True,
+                                                             "page_size": 32}),
+    ("gqa32_paged64_rows32", 2, 32, 1, 128, [700, 130], {"paged": True, "page_size": 64}),
     ("q8_gqa4_fp8_win_rows32", 2, 8, 2, 128, [700, 50], {"q_len": 8, "kv_dtype": "fp8_e4m3",
                                                          "window": 200}),
     ("q2_gqa8_fp8_paged_rows16", 2, 16, 2, 128, [333, 70], {"q_len": 2, "kv_dtype": "fp8_e4m3",
