@@ -617,17 +617,16 @@ struct SimtConsumer {
 };
 
 // ------------------------------------------------------- MMA dataflow
-// Scores S^T = K . Q^T on mma.m16n8k16 (16 tokens x 8 query heads x 16 dims
+// Scores S^T = K . Q^T on mma.m16n8k16 (16 tokens x 8 query rows x 16 dims
 // per instruction, fp32 accumulate); probabilities are transposed in
 // registers (movmatrix) into the B operand of O^T += V^T . P^T, with O^T
-// (dims x heads) accumulated in fp32 registers.  Up to 8 query heads per kv
-// head; missing heads are zero columns.  bf16 K/V use bf16 operands.  For
-// e4m3 K the scores run on the e4m3 product (m16n8k32) straight from the
-// stored codes: q, scaled by a power of two per head, is split into three
-// e4m3 parts hi + mid + lo (about 12 significant bits, the part sum is within
-// 2^-12 of the bf16 value) and the three products are summed in fp32.  e4m3
-// V is widened exactly to f16 for the P.V product.  The q scale is undone on
-// the fp32 scores.
+// (dims x rows) accumulated in fp32 registers.  A block of 8 query rows per
+// product; missing rows are zero columns.  bf16 K/V use bf16 operands.  fp8
+// and int4 K/V are widened exactly to f16, and q is held in f16 times a
+// power of two per row, undone on the fp32 scores.  (With FA_FP8_QSPLIT the
+// fp8 scores run on the e4m3 product (m16n8k32) straight from the stored
+// codes, q split into three e4m3 parts hi + mid + lo, about 12 significant
+// bits; measured slower than widening, so off by default.)
 // R row teams of 8 * NB query rows each (a segment of up to 8 * NB * R rows:
 // the query heads of a kv head times the query tokens).  A team's warp
 // computes its rows of every tile it takes, in NB blocks of 8 that share
