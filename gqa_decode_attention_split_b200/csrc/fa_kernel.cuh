@@ -682,6 +682,14 @@ struct MmaConsumer {
   static constexpr int VBT = D / 8;      // fp8 / int4 V: elements of a row owned by one lane
   static constexpr int KB = I4 ? BPT / 2 : BPT;  // their bytes
   static constexpr int VB = I4 ? VBT / 2 : VBT;
+  // Unified max: how far below phi a row's first scores may sit and keep
+  // phi.  The fp8 / int4 products carry the probabilities in f16, whose
+  // subnormals (below 2^-14) hold them to 2^-24 absolute: with the row's
+  // largest weight below 1 that costs up to 2^-8 of relative precision
+  // (measured: 1.6% error on a small output), so there a row keeps phi
+  // only when its first scores reach it; bf16 probabilities keep 8 exponent
+  // bits and allow the full drop.
+  static constexpr float kDrop = BF16 ? kPhiDrop : 0.f;
   static_assert(D % 16 == 0 && C::T % 16 == 0, "mma tiling");
   static_assert(!FP8 || C::CB == 128, "fp8 mma path needs 128-byte planes");
   static_assert(!I4 || ((D == 128 || D == 256) && KB % 16 == 0 && (VB == 8 || VB == 16)),
@@ -965,11 +973,11 @@ struct MmaConsumer {
       if (fresh != 0u) {  // unified max: the rows' first finite scores (row-uniform: mx is reduced)
         const uint32_t b0 = 1u << (2 * nb), b1 = b0 << 1;
         if ((fresh & b0) && mx0 > -CUDART_INF_F) {
-          if (mx0 < m[nb][0] - kPhiDrop) m[nb][0] = mx0;
+          if (mx0 < m[nb][0] - kDrop) m[nb][0] = mx0;
           fresh &= ~b0;
         }
         if ((fresh & b1) && mx1 > -CUDART_INF_F) {
-          if (mx1 < m[nb][1] - kPhiDrop) m[nb][1] = mx1;
+          if (mx1 < m[nb][1] - kDrop) m[nb][1] = mx1;
           fresh &= ~b1;
         }
       }

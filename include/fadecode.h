@@ -124,8 +124,9 @@ typedef struct {
                       /* scores stay below it.  Exact for any phi: a score  */
                       /* more than 8 log2-units above phi falls back to the */
                       /* exact rescale, and a row whose first scores sit     */
-                      /* more than 8 log2-units below phi starts from its   */
-                      /* own maximum instead.                               */
+                      /* more than 8 log2-units below phi (for fp8 / int4   */
+                      /* K/V on the MMA dataflow: below phi at all) starts  */
+                      /* from its own maximum instead.                      */
   float softmax_phi;  /* unified_max only: phi, in natural-log units of the */
                       /* scaled (and soft-capped) score; must be finite.    */
 } fa_decode_desc;

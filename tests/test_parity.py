@@ -498,3 +498,63 @@ def test_one_million_keys():
     against the oracle."""
     x = synth.generate(1, 8, 1, 128, [1 << 20], kv_dtype="fp8_e4m3", seed=52)
     _check_full(x, path="mma", nrows=4, seed=5)
+
+
+# ------------------------------------------------------ random shape sweep
+def _random_cases(n, seed):
+    rng = np.random.default_rng(seed)
+    cases = []
+    while len(cases) < n:
+        dtype = ["bf16", "fp8_e4m3", "int4"][rng.integers(3)]
+        d = int(rng.choice([64, 128, 256] if dtype == "bf16" else [128, 256]))
+        kv = int(rng.choice([1, 2, 4, 8]))
+        q_len = int(rng.choice([1, 1, 1, 2, 3, 4, 8]))
+        group = int(rng.choice([1, 2, 3, 4, 5, 8, 16]))
+        if group * q_len > 32:
+            continue
+        batch = int(rng.integers(1, 6))
+        lens = [int(x) for x in rng.integers(0, 700, size=batch)]
+        kw = {"q_len": q_len, "kv_dtype": dtype}
+        if rng.random() < 0.5:
+            kw.update(paged=True, page_size=int(rng.choice([1, 2, 4, 8, 16, 32, 64, 128, 256])),
+                      unused_slot_fill="nan")
+        if rng.random() < 0.3:
+            kw["window"] = int(rng.integers(1, 400))
+        if rng.random() < 0.2:
+            kw.update(logit_cap=float(rng.uniform(5, 50)), sm_scale=0.3)
+        path = ["auto", "mma", "simt"][rng.integers(3)]
+        ctas = int(rng.choice([0, 0, 1, 3, 17]))
+        phi = float(rng.uniform(-20, 20)) if rng.random() < 0.2 else None
+        cases.append((len(cases), batch, group * kv, kv, d, lens, kw, path, ctas, phi))
+    return cases
+
+
+@pytest.mark.parametrize("case", _random_cases(120, 2026), ids=lambda c: f"r{c[0]}")
+def test_random_shapes_match_the_oracle(case):
+    """Seeded random decodes over the options' cross product (dtype, head
+    size, group, query tokens, paging, window, soft-cap, unified max,
+    dataflow, forced split): every supported one matches the oracle; a
+    refused one is one the documented limits refuse."""
+    idx, B, Hq, Hk, d, lens, kw, path, ctas, phi = case
+    if kw.get("paged") and kw["kv_dtype"] == "int4" and d == 128 and kw["page_size"] == 1:
+        kw = {**kw, "page_size": 2}  # a one-token int4 page is refused (128-byte copy rule)
+    x = synth.generate(B, Hq, Hk, d, lens, seed=1000 + idx, name=f"random{idx}", **kw)
+    rows = x.group * x.q_len
+    try:
+        p = binding.plan(x.batch, x.qo_heads, x.kv_heads, x.head_dim, x.kv_indptr,
+                         kv_dtype=x.kv_dtype, paged=x.paged, page_size=x.page_size,
+                         window=x.window, sm_scale=x.sm_scale, path=path, num_ctas=ctas,
+                         q_len=x.q_len, logit_cap=x.logit_cap, softmax_phi=phi)
+    except binding.FadecodeError as e:
+        assert e.status == 2, str(e)
+        simt_ok = (x.kv_dtype != "int4" and rows in (1, 2, 4, 8)
+                   and not (x.kv_dtype == "fp8_e4m3" and rows == 8))
+        assert path == "simt" and not simt_ok, f"unexpected refusal: {e}"
+        return
+    ref_out, ref_lse = oracle.decode_all(x)
+    dev = DeviceInputs(x)
+    ws = p.new_workspace()
+    out, lse = dev.run(p, workspace=ws)
+    assert binding.decode_status(ws) == 0
+    o, l = to_numpy(out, lse)
+    assert_matches(o, l, ref_out, ref_lse, what=f"random{idx} {path} ctas={ctas} phi={phi} {kw}")
