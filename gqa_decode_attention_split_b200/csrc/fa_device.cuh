@@ -202,16 +202,34 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
-// Two int4 codes -> f16x2, exact: bits 0-3 of x give the low half, bits
-// 16-19 the high half, each a two's-complement nibble c.  The f16 with bit
-// pattern 0x6400 | u is 1024 + u for u < 1024 (the unit in the last place
-// of 1024 is 1), so (nibble ^ 8) = c + 8 placed under 0x6400 reads 1032 + c;
-// one f16x2 subtraction of 1032 leaves c.
-__device__ __forceinline__ uint32_t int4x2_to_f16x2(uint32_t x) {
-  const uint32_t biased = (x & 0x000F000Fu) ^ 0x64086408u;
-  uint32_t r;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(biased), "r"(0x64086408u));
+// Int4 codes -> f16x2, exact, each 16-bit half of x on its own; a code c
+// is a two's-complement nibble.  The f16 with bit pattern 0x6400 | u is
+// 1024 + u for u < 1024 (the unit in the last place of 1024 is 1).  With
+// B = 0x6488 in each half (1160):
+//  - lo: the nibble of bits 0-3, xor-ed into B, turns B's bits 0-3 into
+//    c ^ 8 = c + 8, which reads 1024 + 128 + c + 8 = B + c;
+//  - hi: the nibble of bits 4-7, xor-ed into B, turns B's bits 4-7 into
+//    c + 8, which reads 1024 + 16 (c + 8) + 8 = B + 16 c.
+// One f16x2 subtraction of B leaves c, or 16 c, exactly (every value on the
+// way is an integer below 2048).  Mask and xor are one three-input logic op
+// (table 0x6A = (a & b) ^ c) whose second constant is the subtrahend's
+// register, so a nibble pair costs two instructions, and the high nibble
+// of a byte needs no shift.
+constexpr uint32_t kInt4Bias = 0x64886488u;
+template <uint32_t MASK>
+__device__ __forceinline__ uint32_t int4_widen(uint32_t x, uint32_t bias) {
+  uint32_t b, r;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(b) : "r"(x), "n"(MASK), "r"(bias));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(b), "r"(bias));
   return r;
+}
+// codes in bits 0-3 and 16-19 -> (c0, c1)
+__device__ __forceinline__ uint32_t int4_lo_to_f16x2(uint32_t x, uint32_t bias) {
+  return int4_widen<0x000F000Fu>(x, bias);
+}
+// codes in bits 4-7 and 20-23 -> (16 c0, 16 c1)
+__device__ __forceinline__ uint32_t int4_hi_to_f16x2(uint32_t x, uint32_t bias) {
+  return int4_widen<0x00F000F0u>(x, bias);
 }
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t r;

@@ -798,11 +798,14 @@ struct MmaConsumer {
               // int4: logical k-columns 2t,2t+1 / 2t+8,2t+9 of step kk <-> the
               // lane's elements (8j + 2c, 8j + 2c + 4) / (8j + 2c + 1, 8j + 2c + 5),
               // j = kk / 2, c = kk % 2: the nibble pairs one shift and one mask
-              // take out of K's 32-bit word j
+              // take out of K's 32-bit word j.  The second pair is widened to
+              // 16 times its codes, so its q values carry 1/16 (exact: a power
+              // of two, with max |q| scaled to [2^10, 2^11) here)
               const int e = 8 * (kk >> 1) + 2 * (kk & 1);
+              const float mul16 = mul * 0.0625f;
               auto qe = [&](int i) { return (i & 1) ? bf16hi(qw[i >> 1]) : bf16lo(qw[i >> 1]); };
               qb[nb][kk][0] = pack_f16x2(qe(e) * mul, qe(e + 4) * mul);
-              qb[nb][kk][1] = pack_f16x2(qe(e + 1) * mul, qe(e + 5) * mul);
+              qb[nb][kk][1] = pack_f16x2(qe(e + 1) * mul16, qe(e + 5) * mul16);
             }
           }
         }
@@ -893,13 +896,17 @@ struct MmaConsumer {
         for (int kk = 0; kk < KS; ++kk) {
           uint32_t af[4];
           if constexpr (I4) {
-            // word kk / 2 of each row; pairs (8c, 8c + 4) bits up: the nibble
-            // pairs of the lane's elements listed in begin_piece
+            // word kk / 2 of each row, shifted down by 8c bits (c = kk % 2):
+            // its bits 0-3 / 16-19 and 4-7 / 20-23 are the nibble pairs of
+            // the lane's elements listed in begin_piece; the second pair
+            // widens to 16 times its codes, and begin_piece gives the q
+            // values it meets a factor 1/16
             const int sh = 8 * (kk & 1);
-            af[0] = int4x2_to_f16x2(w0[kk >> 1] >> sh);
-            af[1] = int4x2_to_f16x2(w1[kk >> 1] >> sh);
-            af[2] = int4x2_to_f16x2(w0[kk >> 1] >> (sh + 4));
-            af[3] = int4x2_to_f16x2(w1[kk >> 1] >> (sh + 4));
+            const uint32_t x0 = w0[kk >> 1] >> sh, x1 = w1[kk >> 1] >> sh;
+            af[0] = int4_lo_to_f16x2(x0, kInt4Bias);
+            af[1] = int4_lo_to_f16x2(x1, kInt4Bias);
+            af[2] = int4_hi_to_f16x2(x0, kInt4Bias);
+            af[3] = int4_hi_to_f16x2(x1, kInt4Bias);
           } else {
             af[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(w0[kk] & 0xFFFFu));
             af[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[kk] & 0xFFFFu));
@@ -1071,11 +1078,12 @@ struct MmaConsumer {
         }
       } else if constexpr (I4) {
         // lane owns dims [VBT*g, VBT*g + VBT) (VB bytes) of tokens 2t, 2t+1,
-        // 2t+8, 2t+9.  Bytes 2u, 2u+1 of two tokens' chunks, permuted into
-        // one word [tok0 byte 2u, tok0 byte 2u+1, tok1 byte 2u, tok1 byte
-        // 2u+1], give per shift of 0, 4, 8, 12 bits the f16 pair (tok0, tok1)
-        // of dims 4u, 4u+1, 4u+2, 4u+3: m-tile 2u + s takes dims 4u + 2s
-        // (row g) and 4u + 2s + 1 (row g + 8), as out_dim states.
+        // 2t+8, 2t+9.  Byte b = 2u + s of two tokens' chunks, permuted into
+        // bytes 0 and 2 of one word, holds the f16 pairs (tok0, tok1) of
+        // dims 2b (low nibbles) and 2b + 1 (high nibbles, widened to 16
+        // times their codes): m-tile b takes dims 4u + 2s (row g) and
+        // 4u + 2s + 1 (row g + 8), as out_dim states, and end_piece takes
+        // the factor 16 off the row g + 8 accumulators.
         const int rb = sub * 16 + 2 * t;
         const int rows[4] = {rb, rb + 1, rb + 8, rb + 9};
         uint32_t vw[4][VB / 4];
@@ -1095,15 +1103,16 @@ struct MmaConsumer {
         }
 #pragma unroll
         for (int mt = 0; mt < KS; ++mt) {
-          const int u = mt >> 1, sh = 8 * (mt & 1);
-          const uint32_t sel = (u & 1) ? 0x7632u : 0x5410u;
+          const int u = mt >> 1;
+          const uint32_t byt = mt & 3;  // byte of the tokens' word u / 2
+          const uint32_t sel = byt | ((4u + byt) << 8);  // -> bytes 0 and 2
           const uint32_t z01 = prmt(vw[0][u >> 1], vw[1][u >> 1], sel);
           const uint32_t z89 = prmt(vw[2][u >> 1], vw[3][u >> 1], sel);
           uint32_t af[4];
-          af[0] = int4x2_to_f16x2(z01 >> sh);
-          af[1] = int4x2_to_f16x2(z01 >> (sh + 4));
-          af[2] = int4x2_to_f16x2(z89 >> sh);
-          af[3] = int4x2_to_f16x2(z89 >> (sh + 4));
+          af[0] = int4_lo_to_f16x2(z01, kInt4Bias);
+          af[1] = int4_hi_to_f16x2(z01, kInt4Bias);
+          af[2] = int4_lo_to_f16x2(z89, kInt4Bias);
+          af[3] = int4_hi_to_f16x2(z89, kInt4Bias);
           if (edge) {
             af[0] &= mk01;
             af[1] &= mk01;
@@ -1186,15 +1195,17 @@ struct MmaConsumer {
         if (r0) l_area[w * G + h0] = l0;
         if (r1) l_area[w * G + h1] = l1;
       }
+      // int4: the odd dims were summed from values 16 times the codes
+      constexpr float kOdd = I4 ? 0.0625f : 1.f;
 #pragma unroll
       for (int mt = 0; mt < KS; ++mt) {
         if (r0) {
           acc_area[(w * G + h0) * D + out_dim(mt, 0)] = o[nb][mt][0];
-          acc_area[(w * G + h0) * D + out_dim(mt, 1)] = o[nb][mt][2];
+          acc_area[(w * G + h0) * D + out_dim(mt, 1)] = o[nb][mt][2] * kOdd;
         }
         if (r1) {
           acc_area[(w * G + h1) * D + out_dim(mt, 0)] = o[nb][mt][1];
-          acc_area[(w * G + h1) * D + out_dim(mt, 1)] = o[nb][mt][3];
+          acc_area[(w * G + h1) * D + out_dim(mt, 1)] = o[nb][mt][3] * kOdd;
         }
       }
     }
