@@ -44,7 +44,7 @@ class DecodeDesc(ctypes.Structure):
                 ("sm_scale", ctypes.c_float), ("path", ctypes.c_int32),
                 ("num_ctas", ctypes.c_int32), ("q_len", ctypes.c_int32),
                 ("logit_cap", ctypes.c_float), ("unified_max", ctypes.c_int32),
-                ("softmax_phi", ctypes.c_float)]
+                ("softmax_phi", ctypes.c_float), ("piece_cost", ctypes.c_int32)]
 
 
 class PlanInfo(ctypes.Structure):
@@ -52,7 +52,8 @@ class PlanInfo(ctypes.Structure):
                 ("tile_tokens", ctypes.c_int32), ("stages", ctypes.c_int32),
                 ("total_tiles", ctypes.c_int32), ("max_partials", ctypes.c_int32),
                 ("workspace_bytes", ctypes.c_size_t), ("smem_bytes", ctypes.c_size_t),
-                ("v_stages", ctypes.c_int32), ("heads_per_tile", ctypes.c_int32)]
+                ("v_stages", ctypes.c_int32), ("heads_per_tile", ctypes.c_int32),
+                ("piece_cost", ctypes.c_int32)]
 
 
 class TuningEntry(ctypes.Structure):
@@ -165,9 +166,11 @@ def plan(batch: int, qo_heads: int, kv_heads: int, head_dim: int, kv_indptr_host
          kv_dtype: str = "bf16", paged: bool = False, page_size: int = 0, window: int = -1,
          sm_scale: Optional[float] = None, path: str = "auto", num_ctas: int = 0,
          num_sms: int = 0, q_len: int = 1, logit_cap: float = 0.0,
-         softmax_phi: Optional[float] = None) -> DecodePlan:
+         softmax_phi: Optional[float] = None, piece_cost: int = 0) -> DecodePlan:
     """softmax_phi: None for the plain running max; a value turns on the
-    unified max with that phi (natural-log units of the scaled score)."""
+    unified max with that phi (natural-log units of the scaled score).
+    piece_cost: tiles charged per segment when the runs are cut (0: the
+    planner's choice, < 0: equal tiles)."""
     lib = load_library()
     ind = np.ascontiguousarray(np.asarray(
         kv_indptr_host.cpu().numpy() if hasattr(kv_indptr_host, "cpu") else kv_indptr_host,
@@ -180,7 +183,8 @@ def plan(batch: int, qo_heads: int, kv_heads: int, head_dim: int, kv_indptr_host
                       sm_scale=float(sm_scale), path=_PATH_NAMES[path], num_ctas=int(num_ctas),
                       q_len=int(q_len), logit_cap=float(logit_cap),
                       unified_max=0 if softmax_phi is None else 1,
-                      softmax_phi=0.0 if softmax_phi is None else float(softmax_phi))
+                      softmax_phi=0.0 if softmax_phi is None else float(softmax_phi),
+                      piece_cost=int(piece_cost))
     handle = ctypes.c_void_p()
     ws = ctypes.c_size_t()
     _check(lib.fa_decode_plan(ctypes.byref(desc), ind.ctypes.data, int(num_sms),

@@ -59,6 +59,12 @@ namespace fa {
 #ifndef FA_FP8_QSPLIT
 #define FA_FP8_QSPLIT 0              // 1: fp8 scores on the e4m3 product (measured slower)
 #endif
+#ifndef FA_NB2_TOKENS
+#define FA_NB2_TOKENS 64     // tile tokens, bf16 MMA with one team of two row blocks
+#endif
+#ifndef FA_NB2_WARPS
+#define FA_NB2_WARPS 3       // its consumer warps
+#endif
 #ifndef FA_SIMT_TILE_BYTES
 #define FA_SIMT_TILE_BYTES 8192
 #endif
@@ -110,6 +116,7 @@ struct KernelArgs {
   int window;
   int paged, page_shift, pt_stride, box_t, swz;
   int seg_parts;      // 0: equal runs of all tiles; k > 0: k runs per segment
+  int piece_cost;     // equal runs: tile units charged to every segment ahead of its tiles
   float score_scale;  // sm_scale * log2(e)
   float cap_l2;       // > 0: logit soft-cap in log2 units (cap * log2(e)); 0: none
   float m_init;       // start of every running max: -inf, or the unified max phi (log2 units)
@@ -298,15 +305,20 @@ struct Piece {
   int seg;           // b * kv_heads + h
   int n_pieces;      // blocks sharing this segment
   int c_first;       // first block of the segment
-  long long seg_start;
 };
 
-// The block's run is tiles [u, u1) of the segments laid end to end.  Either
-// all runs have `per` tiles (parts == 0), or every segment is cut into
-// `parts` runs, block c taking run c % parts of segment c / parts.
+// The block's run is units [u, u1) of the segments laid end to end.  Either
+// all runs have `per` units (parts == 0), or every segment is cut into
+// `parts` runs, block c taking run c % parts of segment c / parts (units are
+// tiles).  With equal runs every segment spans `cost` units ahead of its
+// tiles: the fixed cost of a piece (parking and merging its state, its
+// ragged last tile) in tile units, so a block whose run starts more
+// segments gets fewer tiles.  A run may end inside those units; units that
+// hold no tile are skipped.
 struct PieceIter {
   long long u, u1, per;
   int parts;
+  int cost;
 };
 
 __device__ __forceinline__ int first_tile(int L, int window, int T) {
@@ -320,40 +332,50 @@ __device__ __forceinline__ int num_tiles(int L, int window, int T) {
 
 __device__ __forceinline__ bool next_piece(PieceIter& it, Piece& pc, const int* s_pre,
                                            const int* s_len, int B, int H, int window, int T) {
-  if (it.u >= it.u1) return false;
-  int lo = 0, hi = B;  // H*pre[lo] <= u < H*pre[hi]
-  while (hi - lo > 1) {
-    int mid = (lo + hi) >> 1;
-    if (static_cast<long long>(H) * s_pre[mid] <= it.u)
-      lo = mid;
-    else
-      hi = mid;
+  const long long K = it.cost;
+  while (it.u < it.u1) {
+    // request b: H*(pre[b] + K*b) <= u < H*(pre[b+1] + K*(b+1))
+    int lo = 0, hi = B;
+    while (hi - lo > 1) {
+      int mid = (lo + hi) >> 1;
+      if (static_cast<long long>(H) * (s_pre[mid] + K * mid) <= it.u)
+        lo = mid;
+      else
+        hi = mid;
+    }
+    const int b = lo;
+    const int n = s_pre[b + 1] - s_pre[b];
+    const long long span = n + K;  // units of each of the request's segments
+    const long long base = static_cast<long long>(H) * (s_pre[b] + K * b);
+    const int h = static_cast<int>(div_fast(it.u - base, span));
+    const long long first = base + static_cast<long long>(h) * span + K;  // unit of tile 0
+    const long long seg_end = first + n;
+    if (n == 0) {  // no tile: skip the segment (reached only with K > 0)
+      it.u = seg_end;
+      continue;
+    }
+    if (it.u < first) it.u = first;
+    if (it.u >= it.u1) return false;  // the run ends among the segment's charge
+    const int tin = static_cast<int>(it.u - first);
+    long long len = n - tin;
+    if (it.u1 - it.u < len) len = it.u1 - it.u;
+    const int ft = first_tile(s_len[b], window, T);
+    pc.b = b;
+    pc.h = h;
+    pc.t0 = ft + tin;
+    pc.t1 = pc.t0 + static_cast<int>(len);
+    pc.seg = b * H + h;
+    if (it.parts > 0) {
+      pc.c_first = pc.seg * it.parts;
+      pc.n_pieces = it.parts;
+    } else {
+      pc.c_first = static_cast<int>(div_fast(first, it.per));
+      pc.n_pieces = static_cast<int>(div_fast(seg_end - 1, it.per)) - pc.c_first + 1;
+    }
+    it.u += len;
+    return true;
   }
-  const int b = lo;
-  const int n = s_pre[b + 1] - s_pre[b];
-  const long long base = static_cast<long long>(H) * s_pre[b];
-  const long long off = it.u - base;
-  const int h = static_cast<int>(div_fast(off, n));
-  const int tin = static_cast<int>(off - static_cast<long long>(h) * n);
-  long long len = n - tin;
-  if (it.u1 - it.u < len) len = it.u1 - it.u;
-  const int ft = first_tile(s_len[b], window, T);
-  pc.b = b;
-  pc.h = h;
-  pc.t0 = ft + tin;
-  pc.t1 = pc.t0 + static_cast<int>(len);
-  pc.seg = b * H + h;
-  pc.seg_start = base + static_cast<long long>(h) * n;
-  const long long seg_end = pc.seg_start + n;
-  if (it.parts > 0) {
-    pc.c_first = pc.seg * it.parts;
-    pc.n_pieces = it.parts;
-  } else {
-    pc.c_first = static_cast<int>(div_fast(pc.seg_start, it.per));
-    pc.n_pieces = static_cast<int>(div_fast(seg_end - 1, it.per)) - pc.c_first + 1;
-  }
-  it.u += len;
-  return true;
+  return false;
 }
 
 // ------------------------------------------------------ SIMT dataflow
@@ -654,7 +676,7 @@ struct MmaConsumer {
   static_assert(TOK == 0 || TOK % 16 == 0, "tiles are whole 16-token subtiles");
   static constexpr int kTileBytes = HEADS ? 16384
                                     : TOK > 0 ? TOK * ROWB_K
-                                    : NB > 1 ? (R == 1 ? 64 : 32) * ROWB_K
+                                    : NB > 1 ? (R == 1 ? (BF16 ? FA_NB2_TOKENS : 64) : 32) * ROWB_K
                                     : FP8 ? FA_FP8_MMA_TILE_BYTES
                                     : I4  ? FA_FP8_MMA_TILE_BYTES / 2
                                           : (R == 1 ? FA_MMA_TILE_BYTES : FA_MMA_TILE_BYTES / 2);
@@ -666,7 +688,7 @@ struct MmaConsumer {
   // computed; measured 5% faster than 5 warps with one slot each, while the
   // compute-bound fp8 / int4 variants keep their 7 warps: int4 was 75%
   // slower with 3).
-  static constexpr int kWarps = (R == 1 && NB == 2 && BF16) ? 3
+  static constexpr int kWarps = (R == 1 && NB == 2 && BF16) ? FA_NB2_WARPS
                                 : R == 1   ? (!BF16 ? FA_FP8_MMA_CONSUMER_WARPS : FA_MMA_CONSUMER_WARPS)
                                 : R == 2 ? 6
                                          : (!BF16 && D >= 256 ? 4 : 8);
@@ -1365,9 +1387,10 @@ __global__ void __maxnreg__(max_regs<Cons>())
   }
   __syncthreads();
 
-  const long long N = static_cast<long long>(H) * s_pre[B];
   const int P = gridDim.x, c = blockIdx.x;
   PieceIter it;
+  it.cost = a.seg_parts > 0 ? 0 : a.piece_cost;
+  const long long N = static_cast<long long>(H) * (s_pre[B] + static_cast<long long>(it.cost) * B);
   it.per = N > 0 ? div_fast(N + P - 1, P) : 1;
   it.parts = 0;
   it.u = static_cast<long long>(c) * it.per;

@@ -129,6 +129,15 @@ typedef struct {
                       /* from its own maximum instead.                      */
   float softmax_phi;  /* unified_max only: phi, in natural-log units of the */
                       /* scaled (and soft-capped) score; must be finite.    */
+  int32_t piece_cost; /* Cost model of the split.  A thread block pays a    */
+                      /* fixed cost per segment piece it takes (parking and */
+                      /* merging the piece's softmax state, its ragged last */
+                      /* tile).  With piece_cost c > 0 every segment is     */
+                      /* charged c tiles ahead of its own when the segments */
+                      /* are cut into equal runs, so a block that starts    */
+                      /* more segments gets fewer tiles.  0: planner's      */
+                      /* choice; c < 0: equal tiles, no charge; at most    */
+                      /* 4096.                                              */
 } fa_decode_desc;
 
 typedef struct fa_plan fa_plan;
@@ -146,6 +155,7 @@ typedef struct {
   int32_t v_stages;         /* V tile slots (at least stages: V is held longer) */
   int32_t heads_per_tile;   /* kv heads whose rows one tile holds per token:   */
                             /* > 1 for int4 (256 contiguous bytes a token)     */
+  int32_t piece_cost;       /* tiles charged per segment in the split (0: none) */
 } fa_plan_info_t;
 
 /*

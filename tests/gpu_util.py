@@ -33,12 +33,13 @@ class DeviceInputs:
         self.kv_indptr = torch.from_numpy(x.kv_indptr).to(device)
         self.page_table = (torch.from_numpy(x.page_table).to(device) if x.paged else None)
 
-    def plan(self, path="auto", num_ctas=0):
+    def plan(self, path="auto", num_ctas=0, piece_cost=0):
         x = self.x
         return binding.plan(x.batch, x.qo_heads, x.kv_heads, x.head_dim, x.kv_indptr,
                             kv_dtype=x.kv_dtype, paged=x.paged, page_size=x.page_size,
                             window=x.window, sm_scale=x.sm_scale, path=path, num_ctas=num_ctas,
-                            q_len=getattr(x, "q_len", 1), logit_cap=getattr(x, "logit_cap", 0.0))
+                            q_len=getattr(x, "q_len", 1), logit_cap=getattr(x, "logit_cap", 0.0),
+                            piece_cost=piece_cost)
 
     def run(self, p, workspace=None, out=None, lse=None, want_lse=True):
         return binding.run(p, self.q, self.k, self.v, self.kv_indptr, page_table=self.page_table,
@@ -53,10 +54,10 @@ def to_numpy(out, lse):
     return o, l
 
 
-def run_gpu(x, path="auto", num_ctas=0, dev=None):
+def run_gpu(x, path="auto", num_ctas=0, dev=None, piece_cost=0):
     """Returns (out float64, lse float64, device flags, plan info)."""
     dev = dev or DeviceInputs(x)
-    p = dev.plan(path=path, num_ctas=num_ctas)
+    p = dev.plan(path=path, num_ctas=num_ctas, piece_cost=piece_cost)
     ws = p.new_workspace()
     out, lse = dev.run(p, workspace=ws)
     flags = binding.decode_status(ws)

@@ -425,6 +425,34 @@ def test_head_tile_choice(lib):
 
 
 
+def test_piece_cost_choice(lib):
+    """The split's charge per segment: the caller's value when positive,
+    none when negative; otherwise 2 tiles up to 8 rows, 4 with int4 head
+    tiles, 8 with 16 or 32 rows.  Never on the segment-aligned split nor
+    when blocks get a tile each; a charge above 4096 is rejected."""
+    lens = np.concatenate([[0], np.cumsum([3000, 100, 9000, 40] * 16)])
+    B = len(lens) - 1
+    cases = [(dict(), 2), (dict(q_len=2), 2), (dict(qo_heads=32), 8), (dict(q_len=4), 8),
+             (dict(qo_heads=16, kv_heads=4, kv_dtype=2), 4), (dict(piece_cost=5), 5),
+             (dict(piece_cost=-1), 0), (dict(q_len=4, piece_cost=-7), 0),
+             (dict(piece_cost=4096), 4096), (dict(path=1), 2)]
+    for kw, want in cases:
+        st, h, _ = _plan(lib, _desc(batch=B, **kw), lens)
+        assert st == 0, kw
+        assert _info(lib, h).piece_cost == want, kw
+        lib.fa_plan_destroy(h)
+    st, h, _ = _plan(lib, _desc(batch=B, piece_cost=4097), lens)
+    assert st == 1 and not h.value
+    # one block per tile: nothing to balance
+    st, h, _ = _plan(lib, _desc(), [0, 300])
+    assert st == 0 and _info(lib, h).piece_cost == 0
+    lib.fa_plan_destroy(h)
+    # equal fp8 segments of 128-byte rows: segment-aligned runs, no charge
+    st, h, _ = _plan(lib, _desc(qo_heads=64, kv_heads=8, kv_dtype=1), [0, 131072])
+    assert st == 0 and _info(lib, h).piece_cost == 0
+    lib.fa_plan_destroy(h)
+
+
 def _largest_plannable_batch(lib, **kw):
     def ok(batch):
         lens = np.full(batch, 20)

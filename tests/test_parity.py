@@ -26,11 +26,12 @@ def _has_path(x, path):
     return rows <= 32
 
 
-def _check(x, path="auto", num_ctas=0, what=""):
-    ref_out, ref_lse = oracle.decode_all(x)
-    out, lse, flags, info = run_gpu(x, path=path, num_ctas=num_ctas)
+def _check(x, path="auto", num_ctas=0, what="", piece_cost=0, ref=None):
+    ref_out, ref_lse = ref if ref is not None else oracle.decode_all(x)
+    out, lse, flags, info = run_gpu(x, path=path, num_ctas=num_ctas, piece_cost=piece_cost)
     assert flags == 0, f"{what}: device flags {flags}"
-    assert_matches(out, lse, ref_out, ref_lse, what=f"{x.name} {path} ctas={num_ctas} {what}")
+    assert_matches(out, lse, ref_out, ref_lse,
+                   what=f"{x.name} {path} ctas={num_ctas} cost={piece_cost} {what}")
     return out, lse, info
 
 
@@ -107,6 +108,44 @@ def test_forced_splits_agree(path):
     for o, l in results[1:]:
         assert np.abs(l - results[0][1]).max() <= 2e-5
         assert np.abs(o - results[0][0]).max() <= 4e-3
+
+
+# Lengths that put cuts inside segments' charges: empty requests, one-key
+# requests and lengths around tile edges among long ones.
+COST_LENS = [1500, 0, 40, 1, 0, 700, 63, 64, 65, 0, 2000, 17]
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_piece_cost_splits_agree(path):
+    """A split that charges every segment a fixed cost in tile units ahead of
+    its tiles moves the cuts (a block that starts more segments takes fewer
+    tiles; a run may end inside a segment's charge, and empty requests carry
+    a charge but no tile) and gives the oracle's result at every charge and
+    grid, up to a charge so large that most blocks hold no tile."""
+    x = synth.generate(len(COST_LENS), 8, 2, 128, COST_LENS, seed=31)
+    ref = oracle.decode_all(x)
+    for cost in (-1, 1, 3, 17, 4096):
+        for n in (0, 5, 37):
+            _, _, info = _check(x, path=path, num_ctas=n, piece_cost=cost, ref=ref)
+            if cost > 0 and n > 0:
+                assert info["piece_cost"] == cost
+
+
+@pytest.mark.parametrize("kw", [
+    {"q_len": 4},
+    {"q_len": 2, "window": 50, "paged": True, "page_size": 16},
+    {"kv_dtype": "fp8_e4m3", "paged": True, "page_size": 32},
+    {"kv_dtype": "int4"},
+], ids=["q4_rows16", "q2_win_paged", "fp8_paged", "int4_head_tiles"])
+def test_piece_cost_variants(kw):
+    """The charged split on the row-team, paged, fp8 and int4 head-tile
+    variants, with the planner's own charge and with forced ones."""
+    kv = 4 if kw.get("kv_dtype") == "int4" else 2
+    x = synth.generate(len(COST_LENS), 4 * kv, kv, 128, COST_LENS, seed=32, **kw)
+    ref = oracle.decode_all(x)
+    for cost in (0, 2, 9):
+        for n in (0, 11):
+            _check(x, path="mma", num_ctas=n, piece_cost=cost, ref=ref)
 
 
 @pytest.mark.parametrize("window", [-1, 1500])
