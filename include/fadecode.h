@@ -165,9 +165,12 @@ typedef struct {
  * thread blocks ("FlashDecoding++", section "Hardware-aware heuristic
  * dataflow": the dataflow is chosen from batch, lengths and the GPU).
  * Every (request, kv head) is a segment of KV tiles; the segments are laid
- * end to end and cut into num_ctas equal runs, so every SM streams the same
- * number of bytes whatever the length mix.  A segment cut into several runs
- * yields partial softmax states that fa_decode_run merges exactly.
+ * end to end and cut into num_ctas equal runs, so every SM streams about the
+ * same number of bytes whatever the length mix.  Each segment is counted as
+ * its tiles plus piece_cost tiles for the fixed cost of a segment piece, so
+ * a block that starts more segments takes fewer tiles (see
+ * fa_decode_desc.piece_cost).  A segment cut into several runs yields
+ * partial softmax states that fa_decode_run merges exactly.
  *
  *  desc            shapes and options (copied into the plan).
  *  kv_indptr_host  int32[batch + 1], host memory: cumulative token counts;
