@@ -17,8 +17,9 @@ e2e         = the same metric through the C ABI with host buffers: every step
               memory and reads out and lse back.
 roofline    = algorithmic bytes per pass / the pass's average duration in the
               timed region (events on the launching stream), against the
-              measured HBM copy bandwidth; isolated_launch_us is the mean of
-              single launches each bracketed by its own events.
+              measured HBM copy bandwidth; isolated_launch_us is the mean
+              (isolated_launch_us_median the median) of single launches each
+              bracketed by its own events.
 cpu_baseline= the fp64 oracle on the host cores on a bounded sample.
 
 --impl reference times the oracle (this tier's reference arm) on the same
@@ -465,6 +466,7 @@ def main():
     launch_ms = per_launch_ms(runner.step, min(args.steps, 100), stream,
                               flush=None if kv_bytes > 256e6 else l2_flusher())
     mean_launch = max_over_ranks(statistics.mean(launch_ms), world, "cuda")
+    median_launch = max_over_ranks(statistics.median(launch_ms), world, "cuda")
     traffic = ncu_traffic(x.name)
     runner.check_status()
 
@@ -536,6 +538,7 @@ def main():
                              "traffic": traffic, "peak_source": peak_kind,
                              "launch_us": round(ms_step * 1e3, 2),
                              "isolated_launch_us": round(mean_launch * 1e3, 2),
+                             "isolated_launch_us_median": round(median_launch * 1e3, 2),
                              "algorithmic_bytes_per_launch": kv_bytes},
                 # per step: the decode kernel, plus the split-merge kernel when
                 # the pass runs on more than one block
