@@ -282,6 +282,12 @@ FA_API fa_status fa_get_tuning(fa_tuning_entry* out, int32_t cap, int32_t* n);
  * FA_ERR_INVALID_ARG, FA_ERR_MISALIGNED, FA_ERR_WORKSPACE_TOO_SMALL,
  * FA_ERR_CUDA (launch failure).  Device-side checks are reported later by
  * fa_decode_status.
+ * CUDA graphs: a pass can be recorded by stream capture, once the plan's
+ * kernel has run on the device outside a capture (its first launch sets the
+ * kernel's shared-memory limit).  A replay reads q, K/V, page_table and
+ * kv_indptr where they were at capture.  Their contents may change between
+ * replays, requests' lengths included, as long as the extents passed at
+ * capture (kv_rows, page_table_stride) still hold.
  */
 FA_API fa_status fa_decode_run(const fa_plan* plan, const void* q, const void* k, const void* v,
                         int64_t kv_rows, const int32_t* page_table, int32_t page_table_stride,

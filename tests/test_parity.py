@@ -627,3 +627,67 @@ def test_repeated_passes_are_bit_identical(kw):
         assert binding.decode_status(ws) == 0
         for o, l in outs[1:]:
             assert torch.equal(o, outs[0][0]) and torch.equal(l, outs[0][1]), f"ctas={n}"
+
+
+@pytest.mark.parametrize("kw", [
+    {"lens": [1500, 0, 40, 700, 2000, 17], "paged": True, "page_size": 16},
+    {"lens": [3000, 900], "kv_dtype": "fp8_e4m3"},
+    {"lens": [1200, 5, 333], "q_len": 4},
+], ids=["bf16_paged_split", "fp8", "q4_rows16"])
+def test_pass_captured_in_a_cuda_graph(kw):
+    """fa_decode_run enqueues kernel launches only (every argument by value,
+    no allocation, no synchronisation), so a decode loop can capture it in a
+    CUDA graph: the decode kernel and, for split segments, the merge kernel
+    as its programmatic dependent.  Replays give the oracle's result, the
+    same bits each time, also after the inputs change in place."""
+    import torch
+    kw = dict(kw)
+    lens = kw.pop("lens")
+    x = synth.generate(len(lens), 8, 2, 128, lens, seed=43, **kw)
+    dev = DeviceInputs(x)
+    p = dev.plan(num_ctas=0)
+    ws = p.new_workspace()
+    out, lse = dev.run(p, workspace=ws)  # warm-up outside the capture
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        dev.run(p, workspace=ws, out=out, lse=lse)
+    ref_out, ref_lse = oracle.decode_all(x)
+    first = None
+    for rep in range(3):
+        out.zero_()
+        lse.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        o, l = to_numpy(out, lse)
+        assert_matches(o, l, ref_out, ref_lse, what=f"graph replay {rep}")
+        bits = (out.view(torch.int16).cpu().clone(), lse.view(torch.int32).cpu().clone())
+        if first is None:
+            first = bits
+        else:
+            assert torch.equal(bits[0], first[0]) and torch.equal(bits[1], first[1])
+    assert binding.decode_status(ws) == 0
+    # the graph reads the inputs where they live: new q values, same buffers
+    y = synth.generate(len(lens), 8, 2, 128, lens, seed=44, **kw)
+    dev.q.copy_(torch.from_numpy(np.ascontiguousarray(y.q).view(np.int16)).to(dev.q.device))
+    x.q = y.q
+    g.replay()
+    torch.cuda.synchronize()
+    ref_out, ref_lse = oracle.decode_all(x)
+    o, l = to_numpy(out, lse)
+    assert_matches(o, l, ref_out, ref_lse, what="graph replay, new q")
+    # and new lengths: the kernels split the device copy of kv_indptr, so a
+    # replay follows requests that shrank (the extents given at capture hold)
+    q_len = kw.get("q_len", 1)
+    new_lens = [max(q_len, (3 * n) // 4) if n > 0 else 0 for n in lens]
+    ind = np.concatenate([[0], np.cumsum(new_lens)]).astype(np.int32)
+    dev.kv_indptr.copy_(torch.from_numpy(ind).to(dev.kv_indptr.device))
+    x.kv_indptr = ind
+    g.replay()
+    torch.cuda.synchronize()
+    ref_out, ref_lse = oracle.decode_all(x)
+    o, l = to_numpy(out, lse)
+    assert_matches(o, l, ref_out, ref_lse, what="graph replay, shorter requests")
+    assert binding.decode_status(ws) == 0
