@@ -36,6 +36,10 @@ class FadecodeError(RuntimeError):
         super().__init__(f"{where}: {name}{(' - ' + detail) if detail else ''}")
 
 
+# fadecode.h's FA_VERSION: the layouts of the structures below
+ABI_VERSION = 200
+
+
 class DecodeDesc(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("qo_heads", ctypes.c_int32),
                 ("kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
@@ -107,6 +111,9 @@ def load_library():
     lib.fa_get_tuning.restype = ctypes.c_int
     lib.fa_version.argtypes = []
     lib.fa_version.restype = i32
+    if lib.fa_version() // 100 != ABI_VERSION // 100:
+        raise RuntimeError(f"{path}: library version {lib.fa_version()}, this binding's structures "
+                           f"are those of {ABI_VERSION}; rebuild the library")
     _lib = lib
     return lib
 

@@ -711,6 +711,6 @@ extern "C" const char* fa_status_string(fa_status s) {
   return "unknown status";
 }
 
-extern "C" int32_t fa_version(void) { return 100; }
+extern "C" int32_t fa_version(void) { return FA_VERSION; }
 
 extern "C" const char* fa_last_error(void) { return g_last_error; }

@@ -364,7 +364,11 @@ FA_API const char* fa_status_string(fa_status status);
  * overwritten by the next failure. */
 FA_API const char* fa_last_error(void);
 
-/* Library version, major * 10000 + minor * 100 + patch. */
+/* Library version, major * 10000 + minor * 100 + patch.  The structures of
+ * this header are those of FA_VERSION (0.2.0 added fa_decode_desc.piece_cost
+ * and fa_plan_info_t.piece_cost); a caller built against it should check
+ * that fa_version() / 100 == FA_VERSION / 100. */
+#define FA_VERSION 200
 FA_API int32_t fa_version(void);
 
 #ifdef __cplusplus
