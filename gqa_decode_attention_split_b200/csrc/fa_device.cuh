@@ -156,15 +156,6 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], u
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-// D(16x8, fp32) += A(16x32, row) * B(32x8, col), e4m3 inputs.
-__device__ __forceinline__ void mma_e4m3(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 "
-      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
 // Transpose of an 8x8 matrix of 16-bit values held in the m8n8 fragment
 // layout (thread i holds row i/4, columns 2(i%4), 2(i%4)+1).
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
@@ -181,13 +172,6 @@ __device__ __forceinline__ float bf16hi(uint32_t x) { return __uint_as_float(x &
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t x) {
   uint32_t r;
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(x));
-  return r;
-}
-// Two floats -> two e4m3 codes (round to nearest even, saturating at +-448);
-// `lo` lands in the low byte.
-__device__ __forceinline__ uint16_t float2_to_e4m3x2(float lo, float hi) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
 }
 __device__ __forceinline__ float2 f16x2_to_float2(uint32_t x) {

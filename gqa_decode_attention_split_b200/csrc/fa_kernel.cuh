@@ -56,9 +56,6 @@ namespace fa {
 #ifndef FA_FP8_MMA_CONSUMER_WARPS
 #define FA_FP8_MMA_CONSUMER_WARPS 7
 #endif
-#ifndef FA_FP8_QSPLIT
-#define FA_FP8_QSPLIT 0              // 1: fp8 scores on the e4m3 product (measured slower)
-#endif
 #ifndef FA_NB2_TOKENS
 #define FA_NB2_TOKENS 64     // tile tokens, bf16 MMA with one team of two row blocks
 #endif
@@ -645,10 +642,7 @@ struct SimtConsumer {
 // (dims x rows) accumulated in fp32 registers.  A block of 8 query rows per
 // product; missing rows are zero columns.  bf16 K/V use bf16 operands.  fp8
 // and int4 K/V are widened exactly to f16, and q is held in f16 times a
-// power of two per row, undone on the fp32 scores.  (With FA_FP8_QSPLIT the
-// fp8 scores run on the e4m3 product (m16n8k32) straight from the stored
-// codes, q split into three e4m3 parts hi + mid + lo, about 12 significant
-// bits; measured slower than widening, so off by default.)
+// power of two per row, undone on the fp32 scores.
 // R row teams of 8 * NB query rows each (a segment of up to 8 * NB * R rows:
 // the query heads of a kv head times the query tokens).  A team's warp
 // computes its rows of every tile it takes, in NB blocks of 8 that share
@@ -699,8 +693,6 @@ struct MmaConsumer {
   static constexpr int KS = D / 16;     // k-steps of the score product = m-tiles of O^T
   static constexpr int SUB = C::T / 16;  // 16-token subtiles per tile
   static constexpr int BPT = D / 4;      // fp8 / int4 K: elements of a row owned by one lane
-  static constexpr bool kQSplit = FP8 && FA_FP8_QSPLIT && NB == 1;
-  static constexpr int KS32 = D / 32;    // k-steps of the e4m3 score product
   static constexpr int VBT = D / 8;      // fp8 / int4 V: elements of a row owned by one lane
   static constexpr int KB = I4 ? BPT / 2 : BPT;  // their bytes
   static constexpr int VB = I4 ? VBT / 2 : VBT;
@@ -718,7 +710,6 @@ struct MmaConsumer {
                 "int4 mma path: 64- or 128-byte rows");
 
   uint32_t qb[NB][KS][2];
-  uint32_t qb8[kQSplit ? KS32 : 1][3][2];  // e4m3 q parts (hi, mid, lo) per k-step
   float o[NB][KS][4];
   float m[NB][2], l[NB][2];
   uint32_t fresh;  // unified max: bit 2 nb + j set while row 8 nb + 2t + j has seen no finite score
@@ -778,57 +769,27 @@ struct MmaConsumer {
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
         int ex = 0;
         frexpf(mx, &ex);
-        int sh = 0;
-        if constexpr (kQSplit) {
-          sh = (mx > 0.f && isfinite(mx)) ? 8 - ex : 0;  // max |q| * 2^sh in [128, 256)
-          const float mul = ldexpf(1.f, sh);
+        const int sh = (mx > 0.f && isfinite(mx)) ? 15 - ex : 0;  // |q| * 2^sh < 2^15
+        const float mul = ldexpf(1.f, sh);
 #pragma unroll
-          for (int kk = 0; kk < KS32; ++kk) {
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              // logical k-columns 4t..4t+3 (half 0) / 16+4t..16+4t+3 (half 1) of
-              // step kk <-> dims BPT*t + 8kk + 4*half + 0..3
-              const uint32_t wa = qw[4 * kk + 2 * half], wb = qw[4 * kk + 2 * half + 1];
-              float x0 = bf16lo(wa) * mul, x1 = bf16hi(wa) * mul;
-              float x2 = bf16lo(wb) * mul, x3 = bf16hi(wb) * mul;
-#pragma unroll
-              for (int part = 0; part < 3; ++part) {
-                const uint16_t e01 = float2_to_e4m3x2(x0, x1), e23 = float2_to_e4m3x2(x2, x3);
-                qb8[kk][part][half] = static_cast<uint32_t>(e01) | (static_cast<uint32_t>(e23) << 16);
-                if (part < 2) {  // the next part carries what this one missed
-                  const float2 d01 = f16x2_to_float2(e4m3x2_to_f16x2(e01));
-                  const float2 d23 = f16x2_to_float2(e4m3x2_to_f16x2(e23));
-                  x0 -= d01.x;
-                  x1 -= d01.y;
-                  x2 -= d23.x;
-                  x3 -= d23.y;
-                }
-              }
-            }
-          }
-        } else {
-          sh = (mx > 0.f && isfinite(mx)) ? 15 - ex : 0;  // |q| * 2^sh < 2^15
-          const float mul = ldexpf(1.f, sh);
-#pragma unroll
-          for (int kk = 0; kk < KS; ++kk) {
-            if constexpr (FP8) {
-              // logical k-columns 2t,2t+1 / 2t+8,2t+9 of step kk <-> bytes BPT*t + 4kk + {0,1} / {2,3}
-              const uint32_t w0 = qw[2 * kk], w1 = qw[2 * kk + 1];
-              qb[nb][kk][0] = pack_f16x2(bf16lo(w0) * mul, bf16hi(w0) * mul);
-              qb[nb][kk][1] = pack_f16x2(bf16lo(w1) * mul, bf16hi(w1) * mul);
-            } else {
-              // int4: logical k-columns 2t,2t+1 / 2t+8,2t+9 of step kk <-> the
-              // lane's elements (8j + 2c, 8j + 2c + 4) / (8j + 2c + 1, 8j + 2c + 5),
-              // j = kk / 2, c = kk % 2: the nibble pairs one shift and one mask
-              // take out of K's 32-bit word j.  The second pair is widened to
-              // 16 times its codes, so its q values carry 1/16 (exact: a power
-              // of two, with max |q| scaled to [2^10, 2^11) here)
-              const int e = 8 * (kk >> 1) + 2 * (kk & 1);
-              const float mul16 = mul * 0.0625f;
-              auto qe = [&](int i) { return (i & 1) ? bf16hi(qw[i >> 1]) : bf16lo(qw[i >> 1]); };
-              qb[nb][kk][0] = pack_f16x2(qe(e) * mul, qe(e + 4) * mul);
-              qb[nb][kk][1] = pack_f16x2(qe(e + 1) * mul16, qe(e + 5) * mul16);
-            }
+        for (int kk = 0; kk < KS; ++kk) {
+          if constexpr (FP8) {
+            // logical k-columns 2t,2t+1 / 2t+8,2t+9 of step kk <-> bytes BPT*t + 4kk + {0,1} / {2,3}
+            const uint32_t w0 = qw[2 * kk], w1 = qw[2 * kk + 1];
+            qb[nb][kk][0] = pack_f16x2(bf16lo(w0) * mul, bf16hi(w0) * mul);
+            qb[nb][kk][1] = pack_f16x2(bf16lo(w1) * mul, bf16hi(w1) * mul);
+          } else {
+            // int4: logical k-columns 2t,2t+1 / 2t+8,2t+9 of step kk <-> the
+            // lane's elements (8j + 2c, 8j + 2c + 4) / (8j + 2c + 1, 8j + 2c + 5),
+            // j = kk / 2, c = kk % 2: the nibble pairs one shift and one mask
+            // take out of K's 32-bit word j.  The second pair is widened to
+            // 16 times its codes, so its q values carry 1/16 (exact: a power
+            // of two, with max |q| scaled to [2^10, 2^11) here)
+            const int e = 8 * (kk >> 1) + 2 * (kk & 1);
+            const float mul16 = mul * 0.0625f;
+            auto qe = [&](int i) { return (i & 1) ? bf16hi(qw[i >> 1]) : bf16lo(qw[i >> 1]); };
+            qb[nb][kk][0] = pack_f16x2(qe(e) * mul, qe(e + 4) * mul);
+            qb[nb][kk][1] = pack_f16x2(qe(e + 1) * mul16, qe(e + 5) * mul16);
           }
         }
         const int sh0 = __shfl_sync(0xffffffffu, sh, (2 * t) * 4);
@@ -900,48 +861,33 @@ struct MmaConsumer {
         w0[4 * i] = x0.x; w0[4 * i + 1] = x0.y; w0[4 * i + 2] = x0.z; w0[4 * i + 3] = x0.w;
         w1[4 * i] = x1.x; w1[4 * i + 1] = x1.y; w1[4 * i + 2] = x1.z; w1[4 * i + 3] = x1.w;
       }
-      if constexpr (kQSplit) {
-        float c3[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int kk = 0; kk < KS32; ++kk) {
-          // A (16 tokens x 32 dims, e4m3): rows g / g+8, logical k 4t..4t+3
-          // and 16+4t..16+4t+3 <-> words 2kk and 2kk+1 of the lane's bytes
-          const uint32_t af[4] = {w0[2 * kk], w1[2 * kk], w0[2 * kk + 1], w1[2 * kk + 1]};
-          mma_e4m3(c[0], af, qb8[kk][0][0], qb8[kk][0][1]);
-          mma_e4m3(c2[0], af, qb8[kk][1][0], qb8[kk][1][1]);
-          mma_e4m3(c3, af, qb8[kk][2][0], qb8[kk][2][1]);
+      for (int kk = 0; kk < KS; ++kk) {
+        uint32_t af[4];
+        if constexpr (I4) {
+          // word kk / 2 of each row, shifted down by 8c bits (c = kk % 2):
+          // its bits 0-3 / 16-19 and 4-7 / 20-23 are the nibble pairs of
+          // the lane's elements listed in begin_piece; the second pair
+          // widens to 16 times its codes, and begin_piece gives the q
+          // values it meets a factor 1/16
+          const int sh = 8 * (kk & 1);
+          const uint32_t x0 = w0[kk >> 1] >> sh, x1 = w1[kk >> 1] >> sh;
+          af[0] = int4_lo_to_f16x2(x0, kInt4Bias);
+          af[1] = int4_lo_to_f16x2(x1, kInt4Bias);
+          af[2] = int4_hi_to_f16x2(x0, kInt4Bias);
+          af[3] = int4_hi_to_f16x2(x1, kInt4Bias);
+        } else {
+          af[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(w0[kk] & 0xFFFFu));
+          af[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[kk] & 0xFFFFu));
+          af[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(w0[kk] >> 16));
+          af[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[kk] >> 16));
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) c2[0][i] += c3[i];
-      } else {
-#pragma unroll
-        for (int kk = 0; kk < KS; ++kk) {
-          uint32_t af[4];
-          if constexpr (I4) {
-            // word kk / 2 of each row, shifted down by 8c bits (c = kk % 2):
-            // its bits 0-3 / 16-19 and 4-7 / 20-23 are the nibble pairs of
-            // the lane's elements listed in begin_piece; the second pair
-            // widens to 16 times its codes, and begin_piece gives the q
-            // values it meets a factor 1/16
-            const int sh = 8 * (kk & 1);
-            const uint32_t x0 = w0[kk >> 1] >> sh, x1 = w1[kk >> 1] >> sh;
-            af[0] = int4_lo_to_f16x2(x0, kInt4Bias);
-            af[1] = int4_lo_to_f16x2(x1, kInt4Bias);
-            af[2] = int4_hi_to_f16x2(x0, kInt4Bias);
-            af[3] = int4_hi_to_f16x2(x1, kInt4Bias);
-          } else {
-            af[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(w0[kk] & 0xFFFFu));
-            af[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[kk] & 0xFFFFu));
-            af[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(w0[kk] >> 16));
-            af[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[kk] >> 16));
-          }
-#pragma unroll
-          for (int nb = 0; nb < NB; ++nb) {
-            if (kk & 1)
-              mma_f16(c2[nb], af, qb[nb][kk][0], qb[nb][kk][1]);
-            else
-              mma_f16(c[nb], af, qb[nb][kk][0], qb[nb][kk][1]);
-          }
+        for (int nb = 0; nb < NB; ++nb) {
+          if (kk & 1)
+            mma_f16(c2[nb], af, qb[nb][kk][0], qb[nb][kk][1]);
+          else
+            mma_f16(c[nb], af, qb[nb][kk][0], qb[nb][kk][1]);
         }
       }
     }

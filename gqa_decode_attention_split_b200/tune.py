@@ -9,8 +9,10 @@ for every shape the fastest configuration (the fixed rule unless another is
 at least MARGIN faster), merges neighbouring byte ranges with the same
 choice, and writes
 
-  csrc/fa_tuning_b200.inc   rows of the built-in table (rebuild the library)
-  tuning_b200.json          every measurement behind them
+  csrc/fa_tuning_b200.inc   rows of the built-in table (rebuild the library),
+                            under --inc-dir (default: this package)
+  tuning_b200.json          every measurement behind them, under --record-dir
+                            (default: the working directory, outside the package)
 
 Usage (one GPU):  python -m gqa_decode_attention_split_b200.tune [--quick]
 The table can also be installed at run time with binding.set_tuning(rows).
@@ -159,7 +161,10 @@ def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--quick", action="store_true", help="head_dim 128 bf16 only (a smoke run)")
     ap.add_argument("--reps", type=int, default=40)
-    ap.add_argument("--out-dir", default=_PKG, help="where tuning_b200.json and csrc/ are written")
+    ap.add_argument("--inc-dir", default=_PKG,
+                    help="where csrc/fa_tuning_b200.inc is written (default: this package)")
+    ap.add_argument("--record-dir", default=".",
+                    help="where the raw measurements (tuning_b200.json) are written")
     args = ap.parse_args()
     import torch
     flush = torch.empty(FLUSH_BELOW, dtype=torch.uint8, device="cuda")
@@ -194,12 +199,13 @@ def main():
                 torch.cuda.empty_cache()
             results[(d, dtype, r)] = per
     rows = table_rows(results)
-    with open(os.path.join(args.out_dir, "tuning_b200.json"), "w") as f:
+    os.makedirs(args.record_dir, exist_ok=True)
+    with open(os.path.join(args.record_dir, "tuning_b200.json"), "w") as f:
         json.dump({"margin": MARGIN, "margin_us": MARGIN_US, "kv_heads": KV_HEADS, "flush_below_bytes": FLUSH_BELOW,
                    "gpu": torch.cuda.get_device_name(), "measurements": record, "table": rows}, f,
                   indent=1)
-    os.makedirs(os.path.join(args.out_dir, "csrc"), exist_ok=True)
-    write_inc(rows, os.path.join(args.out_dir, "csrc", "fa_tuning_b200.inc"))
+    os.makedirs(os.path.join(args.inc_dir, "csrc"), exist_ok=True)
+    write_inc(rows, os.path.join(args.inc_dir, "csrc", "fa_tuning_b200.inc"))
     print(f"{len(rows)} table rows written", flush=True)
 
 

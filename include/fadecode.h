@@ -243,6 +243,18 @@ FA_API fa_status fa_get_tuning(fa_tuning_entry* out, int32_t cap, int32_t* n);
 /*
  * fa_decode_run -- enqueue one decode-attention pass on `stream`.
  *
+ * What it computes is the formula at the top of this header ("Forcing Flash
+ * Attention onto a TPU", section "Standard causal attention"), reached as the
+ * pages describe: the KV sequence is cut into tiles, each run of tiles is
+ * reduced to a partial softmax state (running max, running sum,
+ * accumulator; same page, section "Flash Attention in JAX"), and the states
+ * of a split request are merged exactly through log-sum-exp
+ * ("FlashDecoding++" explainer, section "Asynchronous softmax and unified max
+ * value").  The call shape is the single-request GQA decode with a scratch
+ * buffer of "FlashInfer x JAX via jax-tvm-ffi" (section on single_decode),
+ * extended to a batch over contiguous or paged KV ("Beyond the Memory Wall",
+ * section "2. FlashInfer").
+ *
  * Layouts (row-major, all device memory):
  *  q           bf16 [batch, q_len, qo_heads, head_dim] (q_len = 1:
  *              [batch, qo_heads, head_dim]), 16-byte aligned.
