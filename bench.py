@@ -60,7 +60,31 @@ SWEEP = ["gqa4_d64_L512", "gemma3_1b_global_L8192", "gemma3_1b_local_w512_L8192"
          # logit soft-capping
          "gemma2_2b_softcap50_L8192"]
 FALLBACK_HBM_GBS = 6650.0
+# unified max at phi = 4: the scaled scores of these inputs are N(0, 1), whose
+# maximum over 10^4..10^5 keys is about 4.4
 UNIFIED_PHI = 4.0
+
+
+def sweep_jobs(headline=HEADLINE):
+    """Every (workload, mode) the sweep times; mode is the planner's choice
+    ("auto"), a forced dataflow ("simt", "mma") or the unified max at
+    UNIFIED_PHI ("unified_max").  The parity tests run the same list."""
+    jobs = [(name, "auto") for name in SWEEP]
+    jobs += [(headline, "simt"), (headline, "mma"), ("fp8_gqa8_L131072", "mma"),
+             ("llama2_7b_mha_L32768", "simt"), ("llama2_7b_mha_L32768", "mma"),
+             (headline, "unified_max"), ("fp8_gqa8_L131072", "unified_max")]
+    return jobs
+
+
+def sweep_key(name, mode):
+    return name if mode == "auto" else f"{name}[{mode}]"
+
+
+def make_runner(x, mode, device="cuda"):
+    """The launch configuration the sweep times for (workload, mode)."""
+    if mode == "unified_max":
+        return Runner(x, device=device, softmax_phi=UNIFIED_PHI)
+    return Runner(x, path=mode, device=device)
 
 
 def hbm_peak():
@@ -208,6 +232,21 @@ class Runner:
         self._handle = ctypes.c_void_p()
         self._wsb = ctypes.c_size_t()
 
+    def run_only(self, plan_handle):
+        """One pass with a plan made beforehand (no host planning)."""
+        st = self.lib.fa_decode_run(plan_handle, *self.args)
+        if st != 0:
+            raise RuntimeError(f"fa_decode_run failed: {st}")
+
+    def make_plan(self):
+        h = ctypes.c_void_p()
+        wsb = ctypes.c_size_t()
+        st = self.lib.fa_decode_plan(ctypes.byref(self.desc), self.ind_host.ctypes.data, 0,
+                                     ctypes.byref(h), ctypes.byref(wsb))
+        if st != 0:
+            raise RuntimeError(f"fa_decode_plan failed: {st}")
+        return h
+
     def step(self):
         """plan + run (the whole hot path for one batch)."""
         lib = self.lib
@@ -250,6 +289,31 @@ def per_launch_ms(fn, reps, stream, flush=None):
         b.record(stream)
     torch.cuda.synchronize()
     return [a.elapsed_time(b) for a, b in evs]
+
+
+def device_launch_ms(runner, reps, flush=None):
+    """Device time of single passes: the plan is made once, outside the
+    timed region, and each pass is queued behind GPU work (the L2 flush, or
+    a short device-side delay when there is nothing to flush), so the start
+    event fires only once the host has already enqueued the pass: host
+    planning and launch overhead stay outside the bracket."""
+    import torch
+    h = runner.make_plan()
+    try:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        for a, b in evs:
+            if flush is not None:
+                flush()
+            else:
+                torch.cuda._sleep(40000)  # about 20 us at the B200's clocks
+            a.record(runner.stream)
+            runner.run_only(h)
+            b.record(runner.stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in evs]
+    finally:
+        runner.lib.fa_plan_destroy(h)
 
 
 def l2_flusher(device="cuda"):
@@ -342,7 +406,7 @@ def oracle_sample(x, budget_s, max_requests=None):
 def cpu_baseline(x, budget_s=12.0):
     t, nbytes, nreq, threads = oracle_sample(x, budget_s)
     return {"value": round(nbytes / t / 1e9, 4), "unit": "GB/s", "cores": threads,
-            "kind": "oracle", "tokens_per_s": round(nreq / t, 3),
+            "kind": "oracle", "tokens_per_s": round(nreq * x.q_len / t, 3),
             "sample": f"fp64 oracle over {nreq} whole request(s) of {x.name} "
                       f"({nbytes / 1e9:.3f} GB of K/V) in {t:.2f} s"}
 
@@ -406,6 +470,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--sweep-cpu-s", type=float, default=1.5,
+                    help="seconds of oracle time per sweep workload (its cpu_baseline)")
     ap.add_argument("--profile", type=int, default=0,
                     help="profiler driver: run --warmup steps, then N steps, print nothing")
     args = ap.parse_args()
@@ -483,39 +549,46 @@ def main():
     if rank == 0 and world == 1 and not args.no_sweep:
         sweep = {}
         flush = l2_flusher()
-        jobs = [(name, "auto") for name in SWEEP]
-        jobs += [(x.name, "simt"), (x.name, "mma"), ("fp8_gqa8_L131072", "mma"),
-                 ("llama2_7b_mha_L32768", "simt"), ("llama2_7b_mha_L32768", "mma"),
-                 # unified max at phi = 4: the scaled scores of these inputs are
-                 # N(0, 1), whose maximum over 10^4..10^5 keys is about 4.4
-                 (x.name, "unified_max"), ("fp8_gqa8_L131072", "unified_max")]
         cache = {x.name: x}
-        for name, path in jobs:
-            key = name if path == "auto" else f"{name}[{path}]"
+        cpu_cache = {}
+        for name, mode in sweep_jobs(x.name):
+            key = sweep_key(name, mode)
             try:
                 y = cache.get(name) or synth.workload(name)
                 cache = {x.name: x, name: y}
-                r = (Runner(y, softmax_phi=UNIFIED_PHI) if path == "unified_max"
-                     else Runner(y, path=path))
+                r = make_runner(y, mode)
                 for _ in range(5):
                     r.step()
                 big = y.kv_bytes() > 256e6
                 ms = per_launch_ms(r.step, 30, r.stream, flush=None if big else flush)
                 med = statistics.median(ms)
+                dev_ms = device_launch_ms(r, 30, flush=None if big else flush)
+                dmed = statistics.median(dev_ms)
                 loop_us = None
                 if big:  # back to back, as in the timed region (inputs exceed L2)
                     loop_us = 1e3 * time_steps(r.step, 50, r.stream) / 50
                 r.check_status()
                 gbps = y.kv_bytes() / (med * 1e-3) / 1e9
-                sweep[key] = {"us": round(med * 1e3, 2), "gbps": round(gbps, 1),
-                              "frac": round(gbps / peak, 4),
-                              "back_to_back_us": None if loop_us is None else round(loop_us, 2),
-                              "back_to_back_frac": None if loop_us is None else
-                              round(y.kv_bytes() / (loop_us * 1e-6) / 1e9 / peak, 4),
-                              "tokens_per_s": round(y.batch * y.q_len / (med * 1e-3), 1),
-                              "path": "mma" if r.info["path"] == 2 else "simt",
-                              "ctas": r.info["num_ctas"], "kv_bytes": y.kv_bytes()}
+                dgbps = y.kv_bytes() / (dmed * 1e-3) / 1e9
+                entry = {"us": round(med * 1e3, 2), "gbps": round(gbps, 1),
+                         "frac": round(gbps / peak, 4),
+                         "device_us": round(dmed * 1e3, 2),
+                         "device_frac": round(dgbps / peak, 4),
+                         "back_to_back_us": None if loop_us is None else round(loop_us, 2),
+                         "back_to_back_frac": None if loop_us is None else
+                         round(y.kv_bytes() / (loop_us * 1e-6) / 1e9 / peak, 4),
+                         "tokens_per_s": round(y.batch * y.q_len / (med * 1e-3), 1),
+                         "path": {1: "simt", 2: "mma"}.get(r.info["path"], str(r.info["path"])),
+                         "ctas": r.info["num_ctas"], "kv_bytes": y.kv_bytes()}
                 del r
+                torch.cuda.empty_cache()
+                # the oracle on a bounded sample of the same workload (the
+                # definition is the same with or without the unified max)
+                if not args.no_cpu_baseline:
+                    if name not in cpu_cache:
+                        cpu_cache[name] = cpu_baseline(y, budget_s=args.sweep_cpu_s)
+                    entry["cpu_baseline"] = cpu_cache[name]
+                sweep[key] = entry
             except Exception as e:  # keep the headline line even if a sweep entry fails
                 sweep[key] = {"error": str(e)[:300]}
             torch.cuda.empty_cache()

@@ -99,6 +99,8 @@ def load_library():
     lib.fa_decode_run_static.restype = ctypes.c_int
     lib.fa_decode_status.argtypes = [vp, sz, ctypes.POINTER(ctypes.c_uint32), vp]
     lib.fa_decode_status.restype = ctypes.c_int
+    lib.fa_decode_status_static.argtypes = [ctypes.POINTER(ctypes.c_uint32), vp]
+    lib.fa_decode_status_static.restype = ctypes.c_int
     lib.fa_merge_states.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp]
     lib.fa_merge_states.restype = ctypes.c_int
     lib.fa_status_string.argtypes = [ctypes.c_int]
@@ -256,6 +258,17 @@ def decode_status(workspace, stream=None) -> int:
                               ctypes.byref(flags), _stream_handle(stream))
     if st not in (FA_OK, 6):
         _check(st, "fa_decode_status")
+    return int(flags.value)
+
+
+def decode_status_static(stream=None) -> int:
+    """Synchronise and return (then clear) the device-side check bits of the
+    fixed scratch used by run_static (fa_decode_status_static)."""
+    lib = load_library()
+    flags = ctypes.c_uint32(0)
+    st = lib.fa_decode_status_static(ctypes.byref(flags), _stream_handle(stream))
+    if st not in (FA_OK, 6):
+        _check(st, "fa_decode_status_static")
     return int(flags.value)
 
 

@@ -617,7 +617,10 @@ extern "C" fa_status fa_decode_status(void* workspace, size_t workspace_bytes, u
   if (e != cudaSuccess) return cuda_failure("fa_decode_status: read", e);
   *flags = h;
   if (h != 0) {
-    e = cudaMemsetAsync(workspace, 0, sizeof(uint32_t), s);
+    // the whole header: the check word and the records of the first failed
+    // check and the first wait that gave up (a record is written only into
+    // a cleared slot, so a stale one would hide the next failure)
+    e = cudaMemsetAsync(workspace, 0, 256, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_failure("fa_decode_status: clear", e);
     return FA_ERR_DEVICE_CHECK;

@@ -41,7 +41,9 @@ fa_status cuda_error(const char* what, cudaError_t e) {
 }
 
 // Device address of the scratch on the current device, looked up once per
-// device (the first call on a device does this set-up).
+// device (the first call on a device does this set-up).  The address is kept
+// for the life of the process: after cudaDeviceReset the module may be loaded
+// again elsewhere, so the static entry points are not supported after a reset.
 fa_status scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -94,4 +96,29 @@ extern "C" fa_status fa_decode_run_static(const fa_plan* plan, const void* q, co
   if (e != cudaSuccess) return cuda_error("clearing the static scratch", e);
   return fa_decode_run(plan, q, k, v, kv_rows, page_table, page_table_stride, kv_indptr, k_scale,
                        v_scale, out, lse, scratch, FA_STATIC_WORKSPACE_BYTES, stream);
+}
+
+// Size of the scratch header that holds the device-check word (word 0), the
+// first failed check (words 1..5) and the first wait that gave up (words
+// 8..15); the same 256-byte header as a caller's workspace.
+constexpr size_t kHeaderBytes = 256;
+
+extern "C" fa_status fa_decode_status_static(uint32_t* flags, void* stream) {
+  if (flags == nullptr) return FA_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  fa_status st = scratch_address(&scratch);
+  if (st != FA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, scratch, sizeof(h), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_error("fa_decode_status_static: read", e);
+  *flags = h;
+  if (h != 0) {
+    e = cudaMemsetAsync(scratch, 0, kHeaderBytes, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_error("fa_decode_status_static: clear", e);
+    return FA_ERR_DEVICE_CHECK;
+  }
+  return FA_OK;
 }

@@ -315,6 +315,13 @@ def _c4_small_q4():
                     name="paged_b16_gqa4_q4_L512-16384")
 
 
+def _c4_small_q8():
+    """The first 16 requests of the batch-64 paged workload with 8 query
+    tokens (32 rows per segment): a profiler-sized case of two row teams."""
+    return generate(16, 32, 8, 128, c4_lengths()[:16], paged=True, page_size=16, seed=4, q_len=8,
+                    name="paged_b16_gqa4_q8_L512-16384")
+
+
 def _gqa16():
     """A Llama-3.1-405B-shaped layer on one of eight tensor-parallel GPUs
     (128 query / 8 kv heads in all: 16 query heads on one kv head per GPU),
@@ -370,6 +377,7 @@ WORKLOADS = {
     "paged_b64_gqa4_q4_L512-16384": _c4_q(4),
     "paged_b64_gqa4_q8_L512-16384": _c4_q(8),
     "paged_b16_gqa4_q4_L512-16384": _c4_small_q4,
+    "paged_b16_gqa4_q8_L512-16384": _c4_small_q8,
     "llama3_405b_tp8_gqa16_paged_b64_L512-16384": _gqa16,
     "llama2_7b_mha_q8_L32768": _c3_q8,
     "gemma2_2b_softcap50_L8192": _gemma2_softcap,

@@ -333,6 +333,11 @@ FA_API fa_status fa_decode_run(const fa_plan* plan, const void* q, const void* k
  *  - A plan whose workspace_bytes exceeds FA_STATIC_WORKSPACE_BYTES is
  *    rejected with FA_ERR_WORKSPACE_TOO_SMALL (fa_last_error says how much
  *    it needed).  Other errors as fa_decode_run.
+ *  - Device-side checks (bad page ids, a bad kv_indptr, a wait that gave
+ *    up) land in the scratch's check word; read them with
+ *    fa_decode_status_static before the next static call clears it.
+ *  - The scratch address is kept for the life of the process, so the
+ *    static entry points are not supported after cudaDeviceReset.
  */
 FA_API fa_status fa_decode_run_static(const fa_plan* plan, const void* q, const void* k,
                                       const void* v, int64_t kv_rows, const int32_t* page_table,
@@ -341,10 +346,31 @@ FA_API fa_status fa_decode_run_static(const fa_plan* plan, const void* q, const 
                                       float* lse, void* stream);
 
 /*
+ * fa_decode_status_static -- fa_decode_status for the fixed scratch behind
+ * fa_decode_run_static.  (An addition of this library; the pages have no
+ * counterpart.)
+ *
+ * A caller without a workspace has no address to pass to fa_decode_status,
+ * so this call reads the static scratch of the current device instead: it
+ * SYNCHRONISES `stream`, copies the device-check word into *flags
+ * (FA_DEVICE_* bits: a page id outside the pool, a kv_indptr that decreases
+ * or runs past the extent, a wait that gave up) and, when a bit was set,
+ * clears the 256-byte header (word and records).  Every fa_decode_run_static
+ * call clears the word before its kernel, so read the status of a call
+ * before the next static call is enqueued.  Like every static call, it
+ * allocates nothing; it needs one small device-to-host copy.
+ * Returns FA_ERR_DEVICE_CHECK when any bit was set, FA_ERR_INVALID_ARG for
+ * a NULL flags, FA_ERR_CUDA when the copy failed, else FA_OK.
+ */
+FA_API fa_status fa_decode_status_static(uint32_t* flags, void* stream);
+
+/*
  * fa_decode_status -- SYNCHRONISES `stream`, then reads the device-side check
- * word of `workspace` into *flags (FA_DEVICE_* bits, 0 = clean) and clears
- * it.  Returns FA_ERR_DEVICE_CHECK when any bit was set, FA_ERR_CUDA when the
- * copy failed, else FA_OK.
+ * word of `workspace` into *flags (FA_DEVICE_* bits, 0 = clean).  When a bit
+ * was set it clears the workspace's 256-byte header: the word and the records
+ * of the first failed check and the first wait that gave up.  Returns
+ * FA_ERR_DEVICE_CHECK when any bit was set, FA_ERR_CUDA when the copy failed,
+ * else FA_OK.
  */
 FA_API fa_status fa_decode_status(void* workspace, size_t workspace_bytes, uint32_t* flags,
                            void* stream);

@@ -214,7 +214,12 @@ def test_status_word_is_reported_and_cleared():
     hdr = ws[:64].view(torch.int32)
     hdr[0] = 2       # FA_DEVICE_TIMEOUT
     hdr[8] = 3       # timeout site: a consumer's wait on a full stage
+    hdr[9] = 7       # its block
     assert binding.decode_status(ws) == 2
+    torch.cuda.synchronize()
+    # the whole header is cleared: a record left behind would keep the next
+    # timeout from being recorded (a record is written only into a clear slot)
+    assert int(hdr.abs().sum()) == 0
     assert binding.decode_status(ws) == 0   # cleared by the first read
     out, lse = dev.run(p, workspace=ws)
     o, l = to_numpy(out, lse)
