@@ -211,7 +211,7 @@ class Runner:
             kv_dtype={"bf16": 0, "fp8_e4m3": 1, "int4": 2}[x.kv_dtype], paged=int(x.paged),
             page_size=int(x.page_size),
             window=int(x.window), sm_scale=float(x.sm_scale),
-            path={"auto": 0, "simt": 1, "mma": 2}[path], num_ctas=0, q_len=int(x.q_len),
+            path={"auto": 0, "simt": 1, "mma": 2, "tc": 3}[path], num_ctas=0, q_len=int(x.q_len),
             logit_cap=float(x.logit_cap), unified_max=0 if softmax_phi is None else 1,
             softmax_phi=0.0 if softmax_phi is None else float(softmax_phi))
         p = binding.plan(x.batch, x.qo_heads, x.kv_heads, x.head_dim, x.kv_indptr,
@@ -465,7 +465,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=HEADLINE)
-    ap.add_argument("--path", default="auto", choices=["auto", "simt", "mma"])
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "mma", "tc"])
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -578,7 +578,7 @@ def main():
                          "back_to_back_frac": None if loop_us is None else
                          round(y.kv_bytes() / (loop_us * 1e-6) / 1e9 / peak, 4),
                          "tokens_per_s": round(y.batch * y.q_len / (med * 1e-3), 1),
-                         "path": {1: "simt", 2: "mma"}.get(r.info["path"], str(r.info["path"])),
+                         "path": {1: "simt", 2: "mma", 3: "tc"}.get(r.info["path"], str(r.info["path"])),
                          "ctas": r.info["num_ctas"], "kv_bytes": y.kv_bytes()}
                 del r
                 torch.cuda.empty_cache()
@@ -604,7 +604,7 @@ def main():
                 "dtype": x.kv_dtype,
                 "data": "synthetic", "config": workload_config(x, world),
                 "tokens_per_s": round(tokens, 1), "frac_of_peak": round(value / world / peak, 4),
-                "path": "mma" if runner.info["path"] == 2 else "simt",
+                "path": {1: "simt", 2: "mma", 3: "tc"}[runner.info["path"]],
                 "num_ctas": runner.info["num_ctas"],
                 "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                              "unit": "GB/s", "frac": round(achieved / peak, 4),

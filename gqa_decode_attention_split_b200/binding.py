@@ -20,8 +20,8 @@ _LIB_NAME = "libfadecode.so"
 
 KV_BF16, KV_FP8_E4M3, KV_INT4 = 0, 1, 2
 _KV_DTYPES = {"bf16": KV_BF16, "fp8_e4m3": KV_FP8_E4M3, "int4": KV_INT4}
-PATH_AUTO, PATH_SIMT, PATH_MMA = 0, 1, 2
-_PATH_NAMES = {"auto": PATH_AUTO, "simt": PATH_SIMT, "mma": PATH_MMA}
+PATH_AUTO, PATH_SIMT, PATH_MMA, PATH_TC = 0, 1, 2, 3
+_PATH_NAMES = {"auto": PATH_AUTO, "simt": PATH_SIMT, "mma": PATH_MMA, "tc": PATH_TC}
 
 FA_OK = 0
 _STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",

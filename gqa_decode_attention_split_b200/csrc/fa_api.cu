@@ -32,6 +32,7 @@ void build_registry() {
   n += fa::register_d64(g_entries + n, kMaxEntries - n);
   n += fa::register_d128(g_entries + n, kMaxEntries - n);
   n += fa::register_d256(g_entries + n, kMaxEntries - n);
+  n += fa::register_tc(g_entries + n, kMaxEntries - n);
   g_num_entries = n;
 }
 
@@ -150,7 +151,7 @@ fa_status validate_desc(const fa_decode_desc* d) {
   if (d->paged && (d->page_size < 1 || d->page_size > 256 || ilog2_exact(d->page_size) < 0))
     return FA_ERR_INVALID_ARG;
   if (!isfinite(d->sm_scale)) return FA_ERR_INVALID_ARG;
-  if (d->path < FA_PATH_AUTO || d->path > FA_PATH_MMA) return FA_ERR_INVALID_ARG;
+  if (d->path < FA_PATH_AUTO || d->path > FA_PATH_TC) return FA_ERR_INVALID_ARG;
   if (d->num_ctas < 0) return FA_ERR_INVALID_ARG;
   if (d->q_len < 0 || d->q_len > 64) return FA_ERR_INVALID_ARG;
   if (!(d->logit_cap >= 0.f) || !isfinite(d->logit_cap)) return FA_ERR_INVALID_ARG;
@@ -201,7 +202,8 @@ bool valid_tuning_row(const fa_tuning_entry& e) {
   return e.head_dim > 0 &&
          (e.kv_dtype == FA_KV_BF16 || e.kv_dtype == FA_KV_FP8_E4M3 || e.kv_dtype == FA_KV_INT4) &&
          e.rows_min >= 1 && e.rows_min <= e.rows_max && e.bytes_min >= 0 &&
-         e.bytes_min <= e.bytes_max && (e.path == FA_PATH_SIMT || e.path == FA_PATH_MMA) &&
+         e.bytes_min <= e.bytes_max &&
+         (e.path == FA_PATH_SIMT || e.path == FA_PATH_MMA || e.path == FA_PATH_TC) &&
          e.max_pieces >= 0 && e.max_pieces <= 1024;
 }
 
@@ -266,10 +268,19 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   // for the shape, the SIMT path otherwise.
   const KernelEntry* k = nullptr;
   int64_t max_pieces = 32;  // average blocks per segment, at most
-  if (desc->path == FA_PATH_SIMT) {
-    k = find_entry(desc->head_dim, group, kind, fa::kPathSimt, pages);
-  } else if (desc->path == FA_PATH_MMA) {
-    k = find_entry(desc->head_dim, group, kind, fa::kPathMma, pages);
+  // the tcgen05 dataflow: bf16 K/V, head_dim 128, 9 to 32 rows, copies of
+  // 8 tokens (pages of at least 8), the plain running max
+  auto tc_entry = [&]() -> const KernelEntry* {
+    if (desc->unified_max || group <= 8 || (pages != 0 && pages < 8)) return nullptr;
+    return find_entry(desc->head_dim, group, kind, fa::kPathTc, pages);
+  };
+  auto path_entry = [&](int path) -> const KernelEntry* {
+    return path == FA_PATH_SIMT ? find_entry(desc->head_dim, group, kind, fa::kPathSimt, pages)
+           : path == FA_PATH_TC ? tc_entry()
+                                : find_entry(desc->head_dim, group, kind, fa::kPathMma, pages);
+  };
+  if (desc->path != FA_PATH_AUTO) {
+    k = path_entry(desc->path);
   } else {
     if (desc->num_ctas == 0) {
       const int64_t bytes = visible_kv_bytes(desc, kv_indptr_host);
@@ -277,13 +288,15 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
         if (e.head_dim != desc->head_dim || e.kv_dtype != desc->kv_dtype || group < e.rows_min ||
             group > e.rows_max || bytes < e.bytes_min || bytes > e.bytes_max)
           continue;
-        k = find_entry(desc->head_dim, group, kind, e.path == FA_PATH_SIMT ? fa::kPathSimt : fa::kPathMma,
-                       pages);
+        k = path_entry(e.path);
         if (k == nullptr) continue;
         if (e.max_pieces > 0) max_pieces = e.max_pieces;
         break;
       }
     }
+    // fixed rule: the tcgen05 dataflow where it applies, then the
+    // warp-level tensor-core one, then CUDA cores
+    if (k == nullptr) k = tc_entry();
     if (k == nullptr) k = find_entry(desc->head_dim, group, kind, fa::kPathMma, pages);
     if (k == nullptr) k = find_entry(desc->head_dim, group, kind, fa::kPathSimt, pages);
   }
@@ -378,7 +391,9 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   // by cost.
   p->piece_cost = 0;
   if (seg_parts == 0 && P > 1 && tiles > P && desc->piece_cost >= 0)
-    p->piece_cost = desc->piece_cost > 0 ? desc->piece_cost : (ht > 1 ? 4 : seg_rows <= 8 ? 2 : 8);
+    p->piece_cost = desc->piece_cost > 0 ? desc->piece_cost
+                    : k->path == fa::kPathTc ? 2
+                    : (ht > 1 ? 4 : seg_rows <= 8 ? 2 : 8);
   p->total_tiles = tiles;
   const int segs = desc->batch * static_cast<int>(seg_heads);
   p->max_partials = P + segs;
@@ -420,7 +435,9 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
 
 extern "C" fa_status fa_plan_get_info(const fa_plan* plan, fa_plan_info_t* info) {
   if (plan == nullptr || info == nullptr) return FA_ERR_INVALID_ARG;
-  info->path = plan->kernel->path == fa::kPathMma ? FA_PATH_MMA : FA_PATH_SIMT;
+  info->path = plan->kernel->path == fa::kPathMma ? FA_PATH_MMA
+               : plan->kernel->path == fa::kPathTc ? FA_PATH_TC
+                                                  : FA_PATH_SIMT;
   info->num_ctas = plan->num_ctas;
   info->tile_tokens = plan->kernel->tile_tokens;
   info->stages = plan->kernel->stages;
@@ -471,7 +488,19 @@ fa_status make_kv_map(const fa_plan* p, const void* base, int64_t kv_rows, CUten
                                       : span >= 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
                                                     : CU_TENSOR_MAP_L2_PROMOTION_NONE;
   CUresult r;
-  if (k->token_major) {
+  if (k->tc_copies) {
+    // tcgen05 dataflow: copies of 8 token rows of one kv head, landing as
+    // [plane][8 rows][128 bytes] (the 8-row groups the tensor core reads with
+    // the 128-byte swizzle).  Paged pools are read as token rows too: a page
+    // holds page_size consecutive rows of [kv_heads][head_dim].
+    const cuuint64_t rows = static_cast<cuuint64_t>(kv_rows) * (d.paged ? d.page_size : 1);
+    const cuuint64_t dims[4] = {inner, rows, np, static_cast<cuuint64_t>(d.kv_heads)};
+    const cuuint64_t strides[3] = {row * d.kv_heads, cb, row};
+    const cuuint32_t box[4] = {inner, 8, static_cast<cuuint32_t>(np), 1};
+    r = enc(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, promo,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else if (k->token_major) {
     // [.. rows][kv_heads][planes][plane elements]: one copy carries whole rows
     if (!d.paged) {
       const cuuint64_t dims[4] = {inner, np, static_cast<cuuint64_t>(d.kv_heads),
@@ -523,6 +552,32 @@ fa_status make_kv_map(const fa_plan* p, const void* base, int64_t kv_rows, CUten
   return FA_OK;
 }
 
+// The query rows of the tcgen05 dataflow: [batch * q_len * qo_heads rows]
+// of head_dim bf16, copied as (group) rows x one 128-byte plane with the
+// 128-byte swizzle.
+fa_status make_q_map(const fa_plan* p, const void* q, CUtensorMap* map) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) {
+    snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled unavailable");
+    return FA_ERR_CUDA;
+  }
+  const fa_decode_desc& d = p->desc;
+  const cuuint64_t rows = static_cast<cuuint64_t>(d.batch) * q_len_of(&d) * d.qo_heads;
+  const cuuint64_t dims[3] = {64, rows, static_cast<cuuint64_t>(d.head_dim / 64)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d.head_dim) * 2, 128};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(d.qo_heads / d.kv_heads), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(q), dims, strides,
+                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled (q) failed (%d)",
+             static_cast<int>(r));
+    return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
 }  // namespace
 
 extern "C" fa_status fa_decode_run(const fa_plan* plan, const void* q, const void* k,
@@ -546,10 +601,15 @@ extern "C" fa_status fa_decode_run(const fa_plan* plan, const void* q, const voi
     return FA_ERR_MISALIGNED;
   if (workspace_bytes < plan->ws_bytes) return FA_ERR_WORKSPACE_TOO_SMALL;
 
+  const bool tc = plan->kernel->tc_copies != 0;
+  // the tcgen05 dataflow addresses paged pools by token row (an int32)
+  if (tc && d.paged && kv_rows * d.page_size > INT32_MAX) return FA_ERR_UNSUPPORTED;
+
   fa::KernelArgs a;
   memset(&a, 0, sizeof(a));
   fa_status st = make_kv_map(plan, k, kv_rows, &a.kmap);
   if (st == FA_OK) st = make_kv_map(plan, v, kv_rows, &a.vmap);
+  if (st == FA_OK && tc) st = make_q_map(plan, q, &a.qmap);
   if (st != FA_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.q = static_cast<const uint16_t*>(q);

@@ -65,6 +65,7 @@ KernelEntry make_entry(int path, int group, int max_group, int kv_kind) {
   e.plane_bytes = C::CB;
   e.token_major = C::TOKEN_MAJOR ? 1 : 0;
   e.heads_per_tile = C::HT;
+  e.tc_copies = 0;
   e.smem_bytes = &smem_bytes_for<Cons>;
   e.launch = &launch_decode<Cons>;
   return e;
@@ -109,6 +110,7 @@ int register_variants(KernelEntry* out, int cap, bool with_quant) {
       add(make_entry<SimtConsumer<D, 1, true>>(kPathSimt, 1, 1, kKvFp8));
       add(make_entry<SimtConsumer<D, 2, true>>(kPathSimt, 2, 2, kKvFp8));
       add(make_entry<SimtConsumer<D, 4, true>>(kPathSimt, 4, 4, kKvFp8));
+      add(make_entry<SimtConsumer<D, 8, true>>(kPathSimt, 8, 8, kKvFp8));
       // int4 KV: tensor-core dataflow only
       add(make_entry<MmaConsumer<D, kKvInt4, 1>>(kPathMma, 0, 8, kKvInt4));
       if constexpr (D <= 128) {

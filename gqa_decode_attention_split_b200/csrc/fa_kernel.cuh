@@ -94,6 +94,7 @@ constexpr uint32_t kFlagBadIndptr = 4u;
 struct KernelArgs {
   CUtensorMap kmap;
   CUtensorMap vmap;
+  CUtensorMap qmap;   // tcgen05 dataflow only: the query rows, 128-byte swizzled planes
   const uint16_t* q;
   const int32_t* kv_indptr;
   const int32_t* page_table;
@@ -375,6 +376,126 @@ __device__ __forceinline__ bool next_piece(PieceIter& it, Piece& pc, const int* 
   return false;
 }
 
+// ------------------------------------------------------ pass set-up
+// Every kernel of a pass starts the same way: validated request lengths,
+// the tile prefix over requests, and the block's run of the schedule.
+
+// s_start[b], s_len[b] from the device kv_indptr (all threads of the block).
+// A decreasing indptr or one past the K/V extent (or the page table) sets
+// FA_DEVICE_BAD_INDPTR; such a request is read as empty or clipped.
+__device__ __forceinline__ void load_lengths(const KernelArgs& a, int* s_start, int* s_len) {
+  const int ps = a.paged ? (1 << a.page_shift) : 0;
+  for (int b = threadIdx.x; b < a.batch; b += blockDim.x) {
+    const int st = __ldg(a.kv_indptr + b), en = __ldg(a.kv_indptr + b + 1);
+    int L = en - st;
+    bool bad = false;
+    if (st < 0 || L < 0) {
+      L = 0;
+      bad = true;
+    } else if (!a.paged && static_cast<long long>(en) > a.kv_rows) {
+      bad = true;  // rows past the extent read as zeros
+    } else if (a.paged && L > 0 && ((L + ps - 1) >> a.page_shift) > a.pt_stride) {
+      L = a.pt_stride << a.page_shift;
+      bad = true;
+    }
+    s_start[b] = st;
+    s_len[b] = L;
+    if (bad) atomicOr(a.status, kFlagBadIndptr);
+  }
+}
+
+// s_pre[b] = tiles of requests before b, s_pre[batch] = all tiles (one warp).
+__device__ __forceinline__ void tile_prefix(const KernelArgs& a, const int* s_len, int* s_pre, int T,
+                                            int lane) {
+  const int B = a.batch;
+  int carry = 0;
+  for (int b0 = 0; b0 < B; b0 += 32) {
+    const int b = b0 + lane;
+    const int n = b < B ? num_tiles(s_len[b], a.window_u, T) : 0;
+    int incl = n;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    if (b < B) s_pre[b] = carry + incl - n;
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) s_pre[B] = carry;
+}
+
+// Block c's run of the schedule: equal runs of all segments' tiles (plus the
+// per-segment charge), or run c % k of segment c / k.
+__device__ __forceinline__ PieceIter block_run(const KernelArgs& a, const int* s_pre, int P, int c) {
+  const int B = a.batch, H = a.kv_heads;
+  PieceIter it;
+  it.cost = a.seg_parts > 0 ? 0 : a.piece_cost;
+  const long long N = static_cast<long long>(H) * (s_pre[B] + static_cast<long long>(it.cost) * B);
+  it.per = N > 0 ? div_fast(N + P - 1, P) : 1;
+  it.parts = 0;
+  it.u = static_cast<long long>(c) * it.per;
+  it.u1 = it.u + it.per < N ? it.u + it.per : N;
+  if (a.seg_parts > 0) {
+    // run c % k of segment c / k (runs differ by at most one tile; the
+    // planner gives every run at least one tile)
+    const int k = a.seg_parts;
+    const int seg = c / k, part = c - seg * k;
+    it.parts = k;
+    it.u = it.u1 = 0;
+    if (seg < B * H) {
+      const int b = seg / H, h = seg - b * H;
+      const long long n = s_pre[b + 1] - s_pre[b];
+      const long long base = static_cast<long long>(H) * s_pre[b] + static_cast<long long>(h) * n;
+      it.u = base + div_fast(part * n, k);
+      it.u1 = base + div_fast((part + 1) * n, k);
+    }
+  }
+  return it;
+}
+
+// Boundary record (one thread): block c's run starts at tile c * per.  If
+// that cut lies inside a segment that began in block c - 1's run, it is the
+// segment's first cut and block c names the segment for the merge kernel;
+// every other block writes "none", so no record survives from an earlier
+// pass.
+__device__ __forceinline__ void write_boundary_record(const KernelArgs& a, const PieceIter& it,
+                                                      const int* s_pre, const int* s_len, int T,
+                                                      int c) {
+  if (c == 0) return;
+  PieceIter i0 = it;
+  Piece p0;
+  int4 rec = make_int4(-1, 0, 0, 0);
+  if (next_piece(i0, p0, s_pre, s_len, a.batch, a.kv_heads, a.window_u, T) && p0.c_first == c - 1)
+    rec = make_int4(p0.seg, p0.c_first, p0.n_pieces, 0);
+  a.records[c] = rec;
+}
+
+// Results no piece writes (threads ctid < nct of the block): a run of a split
+// segment that holds no tile (only if the device indptr is not the plan's)
+// gets an empty partial state, so the merge gives it no weight; requests
+// without keys get out = 0, lse = -inf (spread over blocks).
+__device__ __forceinline__ void write_empty_results(const KernelArgs& a, const PieceIter& it,
+                                                    const int* s_len, int G, int D, int c, int P,
+                                                    int ctid, int nct) {
+  const int B = a.batch, H = a.kv_heads, Q = a.q_len;
+  if (it.parts > 1 && it.u >= it.u1 && c / it.parts < B * H) {
+    const size_t slot = static_cast<size_t>(c) + c / it.parts;
+    for (int x = ctid; x < G * D; x += nct) {
+      a.part_o[slot * G * D + x] = 0.f;
+      if (x < G) a.part_lse[slot * G + x] = -CUDART_INF_F;
+    }
+  }
+  for (int b = c; b < B; b += P) {
+    if (s_len[b] != 0) continue;
+    const int nq = Q * a.qo_heads * D;  // every query token's rows
+    for (int x = ctid; x < nq; x += nct) {
+      a.out[static_cast<size_t>(b) * nq + x] = 0;
+      if (a.lse != nullptr && (x % D) == 0)
+        a.lse[static_cast<size_t>(b) * Q * a.qo_heads + x / D] = -CUDART_INF_F;
+    }
+  }
+}
+
 // ------------------------------------------------------ SIMT dataflow
 // Lanes are grouped LPT per token; a lane owns CPL 16-byte chunks of every
 // row (E elements), holds q for those elements for all G heads and an fp32
@@ -385,8 +506,11 @@ template <int D, int G, bool FP8>
 struct SimtConsumer {
   using C = TileCfg<D, FP8 ? kKvFp8 : kKvBf16, G, 1, FA_SIMT_TILE_BYTES, FA_SIMT_CONSUMER_WARPS, false>;
   __host__ __device__ static constexpr int team_head(int) { return 0; }  // one kv head per tile
-  static constexpr int EPC = 16 / C::ES;
-  static constexpr int NCH = C::ROWB / 16;
+  // bytes of a lane's chunk: 16, or 8 for fp8 with 8 rows, whose 16-element
+  // chunks would hold q and acc for 8 x 16 elements per lane (256 registers)
+  static constexpr int CHB = (FP8 && G >= 8) ? 8 : 16;
+  static constexpr int EPC = CHB / C::ES;
+  static constexpr int NCH = C::ROWB / CHB;
   static constexpr int E_TARGET = 64 / G;
   static constexpr int CPL_RAW = E_TARGET / EPC;
   static constexpr int CPL = CPL_RAW < 1 ? 1 : (CPL_RAW > NCH ? NCH : CPL_RAW);
@@ -394,7 +518,7 @@ struct SimtConsumer {
   static constexpr int LPT = NCH / CPL;
   static constexpr int SLOTS = 32 / LPT;
   static constexpr int TPS = C::T / SLOTS;
-  static constexpr int NCP = C::CB / 16;
+  static constexpr int NCP = C::CB / CHB;
   static_assert(LPT >= 1 && LPT <= 32 && (NCH % CPL) == 0, "lane mapping");
   static_assert(TPS >= 1 && (C::T % SLOTS) == 0, "tokens per slot");
 
@@ -410,29 +534,48 @@ struct SimtConsumer {
     return chunk_plane(k) * (C::CB / C::ES) + chunk_in_plane(k) * EPC + e;
   }
 
-  __device__ __forceinline__ void convert(const uint4& w, float (&x)[EPC]) const {
-    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+  // The lane's chunk k of tile row r, widened to fp32 (site: the debug
+  // build's check code).
+  __device__ __forceinline__ void load(const KernelArgs& a, uint32_t tile, int r, int k,
+                                       uint32_t site, float (&x)[EPC]) const {
+    constexpr int W = CHB / 4;
+    uint32_t u[W];
+    const uint32_t ad = addr(tile, r, k, a.swz);
+    if constexpr (CHB == 16) {
+      const uint4 w = lds128_in(a.status, ad, tile, C::TILE_BYTES, site);
+      u[0] = w.x;
+      u[1] = w.y;
+      u[2] = w.z;
+      u[3] = w.w;
+    } else {
+      const uint2 w = lds64_in(a.status, ad, tile, C::TILE_BYTES, site);
+      u[0] = w.x;
+      u[1] = w.y;
+    }
     if constexpr (!FP8) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < W; ++i) {
         x[2 * i] = bf16lo(u[i]);
         x[2 * i + 1] = bf16hi(u[i]);
       }
     } else {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float2 a = f16x2_to_float2(e4m3x2_to_f16x2(static_cast<uint16_t>(u[i] & 0xFFFFu)));
-        float2 b = f16x2_to_float2(e4m3x2_to_f16x2(static_cast<uint16_t>(u[i] >> 16)));
-        x[4 * i] = a.x;
-        x[4 * i + 1] = a.y;
-        x[4 * i + 2] = b.x;
-        x[4 * i + 3] = b.y;
+      for (int i = 0; i < W; ++i) {
+        float2 lo2 = f16x2_to_float2(e4m3x2_to_f16x2(static_cast<uint16_t>(u[i] & 0xFFFFu)));
+        float2 hi2 = f16x2_to_float2(e4m3x2_to_f16x2(static_cast<uint16_t>(u[i] >> 16)));
+        x[4 * i] = lo2.x;
+        x[4 * i + 1] = lo2.y;
+        x[4 * i + 2] = hi2.x;
+        x[4 * i + 3] = hi2.y;
       }
     }
   }
 
+  // Shared address of the lane's chunk k of tile row r (8-byte chunks: the
+  // 16-byte chunk that holds it, plus the half).
   __device__ __forceinline__ uint32_t addr(uint32_t tile, int r, int k, int swz) const {
-    return tile_addr<C>(tile, r, chunk_plane(k), chunk_in_plane(k), swz);
+    const int cip = chunk_in_plane(k);
+    return tile_addr<C>(tile, r, chunk_plane(k), cip * CHB / 16, swz) + (cip * CHB) % 16;
   }
 
   // qs: the piece's query rows (staged in shared memory, or in global
@@ -501,7 +644,7 @@ struct SimtConsumer {
 #pragma unroll
         for (int k = 0; k < CPL; ++k) {
           float x[EPC];
-          convert(lds128_in(a.status, addr(kt, r, k, a.swz), kt, C::TILE_BYTES, 101), x);
+          load(a, kt, r, k, 101, x);
 #pragma unroll
           for (int h = 0; h < G; ++h)
 #pragma unroll
@@ -586,7 +729,7 @@ struct SimtConsumer {
 #pragma unroll
           for (int k = 0; k < CPL; ++k) {
             float x[EPC];
-            convert(lds128_in(a.status, addr(vt, r, k, a.swz), vt, C::TILE_BYTES, 102), x);
+            load(a, vt, r, k, 102, x);
 #pragma unroll
             for (int h = 0; h < G; ++h)
 #pragma unroll
@@ -929,14 +1072,19 @@ struct MmaConsumer {
         const int pr = pos0 + sub * 16 + g;
         const bool v00 = pr >= clo0 && pr < chi0, v01 = pr >= clo1 && pr < chi1;
         const bool v80 = pr + 8 >= clo0 && pr + 8 < chi0, v81 = pr + 8 >= clo1 && pr + 8 < chi1;
-        s[0] = v00 ? s[0] * sscale[nb][0] : -CUDART_INF_F;
-        s[1] = v01 ? s[1] * sscale[nb][1] : -CUDART_INF_F;
-        s[2] = v80 ? s[2] * sscale[nb][0] : -CUDART_INF_F;
-        s[3] = v81 ? s[3] * sscale[nb][1] : -CUDART_INF_F;
-        if (a.cap_l2 > 0.f) {  // soft-cap: c tanh(s / c) (log2 units; -inf stays -inf)
+        s[0] *= sscale[nb][0];
+        s[1] *= sscale[nb][1];
+        s[2] *= sscale[nb][0];
+        s[3] *= sscale[nb][1];
+        if (a.cap_l2 > 0.f) {  // soft-cap: c tanh(s / c) (log2 units), before the masks
 #pragma unroll
           for (int e = 0; e < 4; ++e) s[e] = a.cap_l2 * tanhf(s[e] / a.cap_l2);
         }
+        // a masked key has weight zero: -inf, never the cap's floor -c
+        s[0] = v00 ? s[0] : -CUDART_INF_F;
+        s[1] = v01 ? s[1] : -CUDART_INF_F;
+        s[2] = v80 ? s[2] : -CUDART_INF_F;
+        s[3] = v81 ? s[3] : -CUDART_INF_F;
         mx0 = fmaxf(mx0, fmaxf(s[0], s[2]));
         mx1 = fmaxf(mx1, fmaxf(s[1], s[3]));
       }
@@ -1271,23 +1419,7 @@ __global__ void __maxnreg__(max_regs<Cons>())
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // ---- setup: request lengths (validated), barriers, tile prefix sums
-  for (int b = tid; b < B; b += blockDim.x) {
-    const int st = __ldg(a.kv_indptr + b), en = __ldg(a.kv_indptr + b + 1);
-    int L = en - st;
-    bool bad = false;
-    if (st < 0 || L < 0) {
-      L = 0;
-      bad = true;
-    } else if (!a.paged && static_cast<long long>(en) > a.kv_rows) {
-      bad = true;  // rows past the extent read as zeros
-    } else if (a.paged && L > 0 && ((L + ps - 1) >> a.page_shift) > a.pt_stride) {
-      L = a.pt_stride << a.page_shift;
-      bad = true;
-    }
-    s_start[b] = st;
-    s_len[b] = L;
-    if (bad) atomicOr(a.status, kFlagBadIndptr);
-  }
+  load_lengths(a, s_start, s_len);
   const int HK = H * C::HT;  // kv heads (a segment covers HT of them)
   const bool scales_in_smem = HK <= kScaleCap;
   if (C::QUANT && scales_in_smem) {
@@ -1315,63 +1447,17 @@ __global__ void __maxnreg__(max_regs<Cons>())
     fence_mbar_init();
   }
   __syncthreads();
-  if (warp == 0) {
-    int carry = 0;
-    for (int b0 = 0; b0 < B; b0 += 32) {
-      const int b = b0 + lane;
-      const int n = b < B ? num_tiles(s_len[b], a.window_u, T) : 0;
-      int incl = n;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += y;
-      }
-      if (b < B) s_pre[b] = carry + incl - n;
-      carry += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) s_pre[B] = carry;
-  }
+  if (warp == 0) tile_prefix(a, s_len, s_pre, T, lane);
   __syncthreads();
 
   const int P = gridDim.x, c = blockIdx.x;
-  PieceIter it;
-  it.cost = a.seg_parts > 0 ? 0 : a.piece_cost;
-  const long long N = static_cast<long long>(H) * (s_pre[B] + static_cast<long long>(it.cost) * B);
-  it.per = N > 0 ? div_fast(N + P - 1, P) : 1;
-  it.parts = 0;
-  it.u = static_cast<long long>(c) * it.per;
-  it.u1 = it.u + it.per < N ? it.u + it.per : N;
-  if (a.seg_parts > 0) {
-    // run c % k of segment c / k (runs differ by at most one tile; the
-    // planner gives every run at least one tile)
-    const int k = a.seg_parts;
-    const int seg = c / k, part = c - seg * k;
-    it.parts = k;
-    it.u = it.u1 = 0;
-    if (seg < B * H) {
-      const int b = seg / H, h = seg - b * H;
-      const long long n = s_pre[b + 1] - s_pre[b];
-      const long long base = static_cast<long long>(H) * s_pre[b] + static_cast<long long>(h) * n;
-      it.u = base + div_fast(part * n, k);
-      it.u1 = base + div_fast((part + 1) * n, k);
-    }
-  }
+  PieceIter it = block_run(a, s_pre, P, c);
 
   // The merge kernel may be scheduled now (it waits for this grid to finish
   // before it reads anything this grid writes).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  // Boundary record: block c's run starts at tile c * per.  If that cut lies
-  // inside a segment that began in block c - 1's run, it is the segment's
-  // first cut and block c names the segment for the merge kernel; every
-  // other block writes "none", so no record survives from an earlier pass.
-  if (tid == 32 && c > 0) {  // a consumer thread: the producer lane goes straight to its copies
-    PieceIter i0 = it;
-    Piece p0;
-    int4 rec = make_int4(-1, 0, 0, 0);
-    if (next_piece(i0, p0, s_pre, s_len, B, H, a.window_u, T) && p0.c_first == c - 1)
-      rec = make_int4(p0.seg, p0.c_first, p0.n_pieces, 0);
-    a.records[c] = rec;
-  }
+  // a consumer thread: the producer lane goes straight to its copies
+  if (tid == 32) write_boundary_record(a, it, s_pre, s_len, T, c);
 
   if (warp == 0) {
     // ================= producer
@@ -1600,27 +1686,7 @@ __global__ void __maxnreg__(max_regs<Cons>())
   const int ctid = tid - 32;
   constexpr int NCT = NW * 32;
 
-  // a run of a split segment that holds no tile (only if the device indptr
-  // is not the plan's): an empty partial state, so the merge gives it no
-  // weight
-  if (it.parts > 1 && it.u >= it.u1 && c / it.parts < B * H) {
-    const size_t slot = static_cast<size_t>(c) + c / it.parts;
-    for (int x = ctid; x < G * D; x += NCT) {
-      a.part_o[slot * G * D + x] = 0.f;
-      if (x < G) a.part_lse[slot * G + x] = -CUDART_INF_F;
-    }
-  }
-
-  // requests without keys: out = 0, lse = -inf (spread over blocks)
-  for (int b = c; b < B; b += P) {
-    if (s_len[b] != 0) continue;
-    const int nq = Q * a.qo_heads * D;  // every query token's rows
-    for (int x = ctid; x < nq; x += NCT) {
-      a.out[static_cast<size_t>(b) * nq + x] = 0;
-      if (a.lse != nullptr && (x % D) == 0)
-        a.lse[static_cast<size_t>(b) * Q * a.qo_heads + x / D] = -CUDART_INF_F;
-    }
-  }
+  write_empty_results(a, it, s_len, G, D, c, P, ctid, NCT);
 
   // Tile i of the block's sequence lives in K slot i % KSTAGES and V slot
   // i % VSTAGES and is consumed by tile lane i % NT, one warp per row team

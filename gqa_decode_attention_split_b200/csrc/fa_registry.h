@@ -9,7 +9,7 @@ namespace fa {
 
 struct KernelArgs;
 
-enum : int { kPathSimt = 1, kPathMma = 2 };
+enum : int { kPathSimt = 1, kPathMma = 2, kPathTc = 3 };
 
 struct KernelEntry {
   int head_dim;
@@ -25,6 +25,7 @@ struct KernelEntry {
   int plane_bytes;  // min(128, row_bytes)
   int token_major;  // 1: one copy per box with planes as a tensor-map dimension
   int heads_per_tile;  // kv heads per tile (> 1: head teams, one segment per head block)
+  int tc_copies;    // tcgen05 dataflow: 8-token copies landing as [group][plane][8][128]
   size_t (*smem_bytes)(int batch, int group);
   cudaError_t (*launch)(const KernelArgs& args, int grid, size_t smem, cudaStream_t stream);
 };
@@ -51,5 +52,6 @@ cudaError_t launch_split_merge(const SplitMergeArgs& args, int head_dim, cudaStr
 int register_d64(KernelEntry* out, int cap);
 int register_d128(KernelEntry* out, int cap);
 int register_d256(KernelEntry* out, int cap);
+int register_tc(KernelEntry* out, int cap);
 
 }  // namespace fa

@@ -1,0 +1,672 @@
+// fa_tc.cuh -- the tcgen05 dataflow: decode attention with the two skinny
+// products on the 5th-generation tensor cores (bf16 K/V, head_dim 128,
+// segments of 9 to 32 query rows: several query tokens per request, or GQA
+// groups wider than 8).
+//
+// "FlashDecoding++" explainer, section "Flat GEMM optimization": with few
+// query rows per kv head the products are flat (small M); padding them to a
+// large tile wastes the tensor core.  Here the KV tile supplies the large
+// dimension instead: tokens are M = 128 of the score product and head
+// dimensions are M = 128 of the output product, while the 16 or 32 query
+// rows are N.
+//
+//   S^T[token][row] = K[token][:] . Q[row][:]        (TMEM, fp32)
+//   P = exp2(S^T * scale - m_row)                     (softmax warps, fp32)
+//   O^T[dim][row]   = V^T[dim][:] . P^T[:][row]       (TMEM, fp32; P as bf16
+//                                                      hi + lo parts)
+//
+// Warp roles of a block (one per SM):
+//   warp 0  producer: bulk tensor copies of K and V tiles (128 tokens, 16
+//           copies of 8 tokens each, landing as [8-token group][plane][8][128
+//           bytes], 128-byte swizzle) and of each piece's query rows;
+//   warp 1  allocates tensor memory; one lane issues every tcgen05.mma and
+//           commits its completion to mbarriers;
+//   warps 2-5  the softmax group (128 threads): thread t reads token t's
+//           scores from TMEM, keeps the running max per row (uniform over
+//           the group, rescaled only past an 8 log2-unit slack), writes P to
+//           shared memory, and reads back dimension t of each tile's O^T,
+//           accumulating it in fp32 registers.
+// The scores of tile i + 1 are computed while the softmax group works on tile
+// i; the output product of tile i runs while the scores of tile i + 1 are
+// read.  Every wait is bounded (2 s, then the block records the wait and
+// unwinds); tensor memory is freed on every exit path.
+#pragma once
+
+#include "fa_kernel.cuh"
+
+namespace fa {
+
+template <int NR>
+struct TcCfg {
+  static_assert(NR == 16 || NR == 32, "16 or 32 query rows per segment (padded)");
+  static constexpr int D = 128;
+  static constexpr int N = NR;
+  static constexpr int T = 128;            // tokens per tile: M of the score product
+  static constexpr int ROWB = 2 * D;       // bf16 row bytes
+  static constexpr int NP = ROWB / 128;    // 128-byte planes per row
+  static constexpr int BOX_T = 8;          // tokens per copy
+  static constexpr int GROUP_BYTES = BOX_T * ROWB;  // one copy: [NP][8][128]
+  static constexpr int BOXES = T / BOX_T;
+  static constexpr int TILE_BYTES = T * ROWB;
+  static constexpr int KSTAGES = 3;
+  static constexpr int VSTAGES = NR <= 16 ? 3 : 2;
+  static constexpr int QSLOT_BYTES = NP * N * 128;  // [NP][N rows][128]
+  static constexpr int P_BYTES = T * N * 2;         // P hi (or lo): [T][N] bf16
+  static constexpr int THREADS = 192;
+  static constexpr uint32_t TMEM_COLS = 128;        // S[2] and O[2], N columns each
+  static constexpr uint32_t P_LAYOUT = N == 32 ? tc::kSwizzle64 : tc::kSwizzle32;
+  // shared memory, from a 1024-aligned base
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + KSTAGES * TILE_BYTES;
+  static constexpr int OFF_Q = OFF_V + VSTAGES * TILE_BYTES;
+  static constexpr int OFF_P = OFF_Q + 2 * QSLOT_BYTES;
+  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+  static constexpr int NBARS = 2 * KSTAGES + 2 * VSTAGES + 14;
+  static constexpr int OFF_TMEM = OFF_BAR + 8 * NBARS;
+  static constexpr int OFF_RED = OFF_TMEM + 16;    // [4][N] floats
+  static constexpr int OFF_ALPHA = OFF_RED + 4 * N * 4;  // [2][N] floats
+  static constexpr int OFF_PAGES = OFF_ALPHA + 2 * N * 4;  // 64 page ids
+  static constexpr int OFF_SCHED = OFF_PAGES + 256;
+  static constexpr size_t bytes(int batch) {
+    return 1024 + static_cast<size_t>(OFF_SCHED) + static_cast<size_t>(3 * batch + 1) * 4;
+  }
+  static_assert(OFF_Q % 1024 == 0 && OFF_P % 1024 == 0 && P_BYTES % 1024 == 0, "operand alignment");
+};
+
+// Warp-wide reduction of N values per lane, one row per value: afterwards
+// lane l holds the reduction of row l % N over the warp (N <= 32).  Each
+// step halves the values a lane keeps, so the warp spends N - 1 shuffles
+// plus one per remaining lane bit, instead of 5 N.
+template <int N, bool MAX>
+__device__ __forceinline__ float warp_rows_reduce(float (&v)[N], int lane) {
+#pragma unroll
+  for (int k = N / 2; k >= 1; k >>= 1) {
+    const bool up = (lane & k) != 0;
+#pragma unroll
+    for (int j = 0; j < k; ++j) {
+      const float send = up ? v[j] : v[j + k];
+      const float keep = up ? v[j + k] : v[j];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, k);
+      v[j] = MAX ? fmaxf(keep, recv) : keep + recv;
+    }
+  }
+  float r = v[0];
+#pragma unroll
+  for (int k = N; k < 32; k <<= 1) {
+    const float o = __shfl_xor_sync(0xffffffffu, r, k);
+    r = MAX ? fmaxf(r, o) : r + o;
+  }
+  return r;
+}
+
+template <int NR>
+__global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
+    fa_decode_tc_kernel(const __grid_constant__ KernelArgs a) {
+  using C = TcCfg<NR>;
+  constexpr int D = C::D, T = C::T, N = C::N, NP = C::NP;
+  constexpr int KS = C::KSTAGES, VS = C::VSTAGES;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (sbase - raw);
+  const uint32_t kring = sbase + C::OFF_K, vring = sbase + C::OFF_V, qslots = sbase + C::OFF_Q;
+  const uint32_t p_hi = sbase + C::OFF_P, p_lo = p_hi + C::P_BYTES;
+  const uint32_t kfull0 = sbase + C::OFF_BAR, kempty0 = kfull0 + 8 * KS;
+  const uint32_t vfull0 = kempty0 + 8 * KS, vempty0 = vfull0 + 8 * VS;
+  const uint32_t qfull0 = vempty0 + 8 * VS, qempty0 = qfull0 + 16;
+  const uint32_t sfull0 = qempty0 + 16, sfree0 = sfull0 + 16;
+  const uint32_t pfull = sfree0 + 16, ofull0 = pfull + 8, ofree0 = ofull0 + 16;
+  const uint32_t done_bar = ofree0 + 16;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base + C::OFF_TMEM);
+  float* s_red = reinterpret_cast<float*>(base + C::OFF_RED);
+  float* s_alpha = reinterpret_cast<float*>(base + C::OFF_ALPHA);
+  int* s_pages = reinterpret_cast<int*>(base + C::OFF_PAGES);
+  int* s_start = reinterpret_cast<int*>(base + C::OFF_SCHED);
+  const int B = a.batch, H = a.kv_heads;
+  int* s_len = s_start + B;
+  int* s_pre = s_len + B;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {  // kernel parameters: safe to touch before the wait below
+    prefetch_tensormap(&a.kmap);
+    prefetch_tensormap(&a.vmap);
+    prefetch_tensormap(&a.qmap);
+  }
+  // nothing in global memory is touched before the preceding work is done
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  load_lengths(a, s_start, s_len);
+  if (warp == 1) {  // the whole warp allocates; the address lands in s_tmem
+    tc::tmem_alloc(smem_addr(s_tmem), C::TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  if (tid == 32) {
+    for (int s = 0; s < KS; ++s) {
+      mbar_init(kfull0 + 8 * s, 1);
+      mbar_init(kempty0 + 8 * s, 1);   // the commit of the tile's score product
+    }
+    for (int s = 0; s < VS; ++s) {
+      mbar_init(vfull0 + 8 * s, 1);
+      mbar_init(vempty0 + 8 * s, 1);   // the commit of the tile's output product
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(qfull0 + 8 * s, 1);
+      mbar_init(qempty0 + 8 * s, 1);   // the commit of the piece's last score product
+      mbar_init(sfull0 + 8 * s, 1);
+      mbar_init(sfree0 + 8 * s, 4);    // one arrival per softmax warp
+      mbar_init(ofull0 + 8 * s, 1);
+      mbar_init(ofree0 + 8 * s, 4);
+    }
+    mbar_init(pfull, 4);
+    mbar_init(done_bar, 1);
+    fence_mbar_init();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *s_tmem;
+  if (warp == 0) tile_prefix(a, s_len, s_pre, T, lane);
+  __syncthreads();
+
+  const int P = gridDim.x, c = blockIdx.x;
+  const PieceIter it = block_run(a, s_pre, P, c);
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (tid == 32) write_boundary_record(a, it, s_pre, s_len, T, c);
+
+  const int GK = a.group, Q = a.q_len;
+  const int G = GK * Q;  // rows of a segment (<= N)
+
+  if (warp == 0) {
+    // ================= producer
+    const uint64_t pol = l2_evict_first_policy();
+    const int ps = a.paged ? (1 << a.page_shift) : 0;
+    const int win_paged = !a.paged ? 1 : (ps >= T ? 63 * (ps / T) : (64 * ps) / T);
+    int ks = 0, vs = 0;
+    uint32_t kph = 0, vph = 0;
+    int kissued = 0, vissued = 0, pq = 0;  // tiles whose K / V copies went out
+    bool ok = true;
+    auto load_ids = [&](const Piece& p, int w, int (&v)[2], bool (&in)[2]) {
+      const int np = (s_len[p.b] + ps - 1) >> a.page_shift;
+      const int pb = (w * T) >> a.page_shift;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int e = pb + half * 32 + lane;
+        in[half] = e < np;
+        v[half] = in[half] ? __ldg(a.page_table + static_cast<long long>(p.b) * a.pt_stride + e) : -1;
+      }
+    };
+    auto store_ids = [&](const int (&v)[2], const bool (&in)[2]) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        int x = v[half];
+        if (in[half] && (x < 0 || static_cast<long long>(x) >= a.kv_rows)) {
+          atomicOr(a.status, kFlagBadPage);
+          x = -1;  // its copies read out of range: zeros, no memory access
+        }
+        s_pages[half * 32 + lane] = in[half] ? x : -1;
+      }
+    };
+    PieceIter itp = it;
+    Piece pc;
+    bool have = next_piece(itp, pc, s_pre, s_len, B, H, a.window_u, T);
+    int w0 = have ? pc.t0 : 0;
+    if (have && a.paged) {
+      int v[2];
+      bool in[2];
+      load_ids(pc, w0, v, in);
+      store_ids(v, in);
+      __syncwarp();
+    }
+    while (ok && have) {
+      const int L = s_len[pc.b];
+      if (w0 == pc.t0 && lane == 0) {
+        // the piece's query rows, plane by plane and token by token, into
+        // q slot pq % 2 as [plane][row][128 bytes] (128-byte swizzle)
+        const int qs = pq & 1;
+        const uint32_t qpar = ((pq >> 1) & 1) ^ 1u;
+        if (!mbar_wait(qempty0 + 8 * qs, qpar, kWaitLimitNs)) {
+          record_timeout(a.status, 5, pq, qs, qpar, qempty0 + 8 * qs);
+          ok = false;
+        } else {
+          mbar_arrive_expect_tx(qfull0 + 8 * qs, static_cast<uint32_t>(G * C::ROWB));
+          for (int i = 0; i < Q; ++i) {
+            const int row = (pc.b * Q + i) * a.qo_heads + pc.h * GK;
+#pragma unroll
+            for (int p = 0; p < NP; ++p)
+              tma_load_3d(qslots + qs * C::QSLOT_BYTES + p * (N * 128) + i * GK * 128, &a.qmap,
+                          qfull0 + 8 * qs, 0, row, p, pol);
+          }
+        }
+      }
+      if (w0 == pc.t0) {
+        ++pq;
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+      }
+      const int w1 = a.paged && w0 + win_paged < pc.t1 ? w0 + win_paged : pc.t1;
+      PieceIter itn = itp;
+      Piece pn = pc;
+      int nw0 = w1;
+      bool nhave = true;
+      if (w1 >= pc.t1) {
+        nhave = next_piece(itn, pn, s_pre, s_len, B, H, a.window_u, T);
+        nw0 = nhave ? pn.t0 : 0;
+      }
+      int nv[2] = {-1, -1};
+      bool nin[2] = {false, false};
+      if (a.paged && nhave) load_ids(pn, nw0, nv, nin);  // in flight during the issue loop
+      const int npages = a.paged ? (L + ps - 1) >> a.page_shift : 0;
+      const int pbase = a.paged ? (w0 * T) >> a.page_shift : 0;
+      if (lane == 0) {
+        // token row of box j of tile tt: contiguous rows, or the pool's rows
+        // (pages hold ps consecutive token rows; a missing page reads zeros)
+        auto box_row = [&](int tt, int j) {
+          const int tok = tt * T + j * C::BOX_T;
+          if (!a.paged) return s_start[pc.b] + tok;
+          const int pidx = tok >> a.page_shift;
+          const int page = (pidx < npages && pidx - pbase < 64) ? s_pages[pidx - pbase] : -1;
+          return page * ps + (tok & (ps - 1));  // page -1: rows -ps.. -1, all outside
+        };
+        for (int tt = w0; tt < w1; ++tt) {
+          if (!mbar_wait(kempty0 + 8 * ks, kph ^ 1u, kWaitLimitNs)) {
+            record_timeout(a.status, 1, kissued, ks, kph ^ 1u, kempty0 + 8 * ks);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(kfull0 + 8 * ks, C::TILE_BYTES);
+          for (int j = 0; j < C::BOXES; ++j)
+            tma_load_4d(kring + ks * C::TILE_BYTES + j * C::GROUP_BYTES, &a.kmap, kfull0 + 8 * ks, 0,
+                        box_row(tt, j), 0, pc.h, pol);
+          ++kissued;
+          if (!mbar_wait(vempty0 + 8 * vs, vph ^ 1u, kWaitLimitNs)) {
+            record_timeout(a.status, 8, vissued, vs, vph ^ 1u, vempty0 + 8 * vs);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(vfull0 + 8 * vs, C::TILE_BYTES);
+          for (int j = 0; j < C::BOXES; ++j)
+            tma_load_4d(vring + vs * C::TILE_BYTES + j * C::GROUP_BYTES, &a.vmap, vfull0 + 8 * vs, 0,
+                        box_row(tt, j), 0, pc.h, pol);
+          ++vissued;
+          if (++ks == KS) {
+            ks = 0;
+            kph ^= 1u;
+          }
+          if (++vs == VS) {
+            vs = 0;
+            vph ^= 1u;
+          }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      __syncwarp();
+      if (a.paged && nhave) store_ids(nv, nin);
+      __syncwarp();
+      if (w1 >= pc.t1) {
+        have = nhave;
+        pc = pn;
+        itp = itn;
+        w0 = nw0;
+      } else {
+        w0 = w1;
+      }
+    }
+    // drain: every issued copy has landed before the block may exit
+    if (lane == 0) {
+      for (int j = kissued - KS < 0 ? 0 : kissued - KS; j < kissued; ++j) {
+        const int st = j % KS;
+        const uint32_t par = (j / KS) & 1;
+        if (!mbar_wait(kfull0 + 8 * st, par, kWaitLimitNs)) {
+          record_timeout(a.status, 2, j, st, par, kfull0 + 8 * st);
+          break;
+        }
+      }
+      for (int j = vissued - VS < 0 ? 0 : vissued - VS; j < vissued; ++j) {
+        const int st = j % VS;
+        const uint32_t par = (j / VS) & 1;
+        if (!mbar_wait(vfull0 + 8 * st, par, kWaitLimitNs)) {
+          record_timeout(a.status, 9, j, st, par, vfull0 + 8 * st);
+          break;
+        }
+      }
+      for (int k = pq - 2 < 0 ? 0 : pq - 2; k < pq; ++k) {
+        if (!mbar_wait(qfull0 + 8 * (k & 1), (k >> 1) & 1, kWaitLimitNs)) {
+          record_timeout(a.status, 7, k, k & 1, (k >> 1) & 1, qfull0 + 8 * (k & 1));
+          break;
+        }
+      }
+    }
+    return;
+  }
+
+  constexpr uint32_t kIdescS = tc::idesc_bf16(128, N, false, false);
+  constexpr uint32_t kIdescO = tc::idesc_bf16(128, N, true, true);
+  const uint32_t tS = tmem, tO = tmem + 2 * N;  // column offsets of S[2] and O[2]
+
+  if (warp == 1) {
+    // ================= tcgen05.mma issue (one lane)
+    if (lane == 0) {
+      bool ok = true;
+      int i = 0, prev = -1, pcount = 0;
+      // output product of tile j: O^T[j % 2] = V_j^T . (P_hi + P_lo)^T
+      auto product_o = [&](int j) {
+        const int vsl = j % VS;
+        if (ok && !mbar_wait(vfull0 + 8 * vsl, (j / VS) & 1, kWaitLimitNs)) {
+          record_timeout(a.status, 11, j, vsl, (j / VS) & 1, vfull0 + 8 * vsl);
+          ok = false;
+        }
+        if (ok && !mbar_wait(pfull, j & 1, kWaitLimitNs)) {
+          record_timeout(a.status, 12, j, 0, j & 1, pfull);
+          ok = false;
+        }
+        if (ok && j >= 2 && !mbar_wait(ofree0 + 8 * (j & 1), ((j - 2) >> 1) & 1, kWaitLimitNs)) {
+          record_timeout(a.status, 13, j, j & 1, ((j - 2) >> 1) & 1, ofree0 + 8 * (j & 1));
+          ok = false;
+        }
+        if (!ok) return;
+        tc::fence_after_sync();
+        const uint32_t vt = vring + vsl * C::TILE_BYTES;
+        const uint32_t d = tO + (j & 1) * N;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          const uint32_t pb = part == 0 ? p_hi : p_lo;
+#pragma unroll
+          for (int k = 0; k < T / 16; ++k) {
+            // V^T: dims as M (64-dim atoms one plane = 1024 bytes apart),
+            // tokens as K (8-token groups GROUP_BYTES apart); P^T: rows as N
+            // (2N bytes a token), tokens as K (8-token groups 16 N apart)
+            const uint64_t ad = tc::smem_desc(vt + k * 2 * C::GROUP_BYTES, 1024, C::GROUP_BYTES,
+                                              tc::kSwizzle128);
+            const uint64_t bd = tc::smem_desc(pb + k * 16 * 2 * N, T * 2 * N, 8 * 2 * N, C::P_LAYOUT);
+            tc::mma_bf16_ss(d, ad, bd, kIdescO, part > 0 || k > 0);
+          }
+        }
+        tc::commit(ofull0 + 8 * (j & 1));
+        tc::commit(vempty0 + 8 * vsl);
+      };
+      PieceIter itm = it;
+      Piece pc;
+      while (ok && next_piece(itm, pc, s_pre, s_len, B, H, a.window_u, T)) {
+        const int qs = pcount & 1;
+        if (!mbar_wait(qfull0 + 8 * qs, (pcount >> 1) & 1, kWaitLimitNs)) {
+          record_timeout(a.status, 14, pcount, qs, (pcount >> 1) & 1, qfull0 + 8 * qs);
+          ok = false;
+          break;
+        }
+        const int n = pc.t1 - pc.t0;
+        for (int t = 0; t < n && ok; ++t, ++i) {
+          const int ksl = i % KS;
+          if (!mbar_wait(kfull0 + 8 * ksl, (i / KS) & 1, kWaitLimitNs)) {
+            record_timeout(a.status, 15, i, ksl, (i / KS) & 1, kfull0 + 8 * ksl);
+            ok = false;
+            break;
+          }
+          if (i >= 2 && !mbar_wait(sfree0 + 8 * (i & 1), ((i - 2) >> 1) & 1, kWaitLimitNs)) {
+            record_timeout(a.status, 16, i, i & 1, ((i - 2) >> 1) & 1, sfree0 + 8 * (i & 1));
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          // scores S^T[i % 2] = K_i . Q^T: tokens as M (8-token groups
+          // GROUP_BYTES apart), query rows as N (8-row groups 1024 bytes
+          // apart); a k-step of 16 dims is 32 bytes into a 128-byte plane
+          const uint32_t kt = kring + ksl * C::TILE_BYTES;
+          const uint32_t qt = qslots + qs * C::QSLOT_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 1024 + (kk & 3) * 32;
+            const uint32_t qoff = (kk >> 2) * (N * 128) + (kk & 3) * 32;
+            const uint64_t ad = tc::smem_desc(kt + off, 16, C::GROUP_BYTES, tc::kSwizzle128);
+            const uint64_t bd = tc::smem_desc(qt + qoff, 16, 1024, tc::kSwizzle128);
+            tc::mma_bf16_ss(tS + (i & 1) * N, ad, bd, kIdescS, kk > 0);
+          }
+          tc::commit(sfull0 + 8 * (i & 1));
+          tc::commit(kempty0 + 8 * ksl);
+          if (t == n - 1) tc::commit(qempty0 + 8 * qs);
+          if (prev >= 0) product_o(prev);
+          prev = i;
+        }
+        ++pcount;
+      }
+      if (prev >= 0) product_o(prev);
+      // every product issued has completed before tensor memory is freed
+      tc::commit(done_bar);
+      if (!mbar_wait(done_bar, 0, kWaitLimitNs)) record_timeout(a.status, 17, i, 0, 0, done_bar);
+    }
+    named_barrier_sync(2, 160);
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, C::TMEM_COLS);
+    return;
+  }
+
+  // ================= softmax group (warps 2..5)
+  const int quarter = warp & 3;              // this warp's quarter of TMEM lanes
+  const int tok = quarter * 32 + lane;       // token of a tile; dim of an output row
+  const uint32_t lanes = static_cast<uint32_t>(quarter * 32) << 16;
+  const int sw = warp - 2;                   // 0..3
+  write_empty_results(a, it, s_len, G, D, c, P, tid - 64, 128);
+
+  float acc[N], l[N], m[N];
+  bool alive = true;     // this warp's waits have all succeeded
+  int i = 0;             // tile of the block's sequence
+  int pending = -1;      // tile whose output product is not yet accumulated
+  uint32_t resc = 0;     // bit j % 2: tile j rescaled the running max (alpha in s_alpha[j % 2])
+  PieceIter its = it;
+  Piece pc;
+
+  // Accumulates O^T of tile j (this thread's dimension, every row).  A
+  // failed wait only stops this warp's work: the group agrees to stop at its
+  // next barrier (bar_any on !alive), so every named barrier below is
+  // reached by all 128 threads or by none.
+  auto take_o = [&](int j) {
+    if (!alive) return;
+    bool ok = mbar_wait(ofull0 + 8 * (j & 1), (j >> 1) & 1, kWaitLimitNs);
+    if (!ok && lane == 0) record_timeout(a.status, 18, j, j & 1, (j >> 1) & 1, ofull0 + 8 * (j & 1));
+    if (!__all_sync(0xffffffffu, ok)) {  // tcgen05.ld is warp-collective
+      alive = false;
+      return;
+    }
+    float o[N];
+    tc::ld_32x32b<N>(tO + lanes + (j & 1) * N, o);
+    tc::wait_ld();
+    tc::fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(ofree0 + 8 * (j & 1));
+    if (resc & (1u << (j & 1))) {
+      const float* al = s_alpha + (j & 1) * N;
+#pragma unroll
+      for (int r = 0; r < N; ++r) acc[r] = fmaf(acc[r], al[r], o[r]);
+    } else {
+#pragma unroll
+      for (int r = 0; r < N; ++r) acc[r] += o[r];
+    }
+  };
+  // A bounded wait of the whole warp: false (and the wait recorded) if any
+  // lane gave up.
+  auto warp_wait = [&](uint32_t bar, uint32_t parity, uint32_t site, int idx, int stage) {
+    const bool ok = mbar_wait(bar, parity, kWaitLimitNs);
+    if (!ok && lane == 0) record_timeout(a.status, site, idx, stage, parity, bar);
+    return __all_sync(0xffffffffu, ok);
+  };
+
+  bool stop = false;
+  while (!stop && next_piece(its, pc, s_pre, s_len, B, H, a.window_u, T)) {
+    const int L = s_len[pc.b];
+    const int lo = (a.window_u > 0 && L > a.window_u) ? L - a.window_u : 0;  // union of the rows' ranges
+    const int hi_min = L - (Q - 1);                                          // every row sees below this
+    const int lo_max = (a.window > 0 && L > a.window) ? L - a.window : 0;    // and from this on
+#pragma unroll
+    for (int r = 0; r < N; ++r) {
+      acc[r] = 0.f;
+      l[r] = 0.f;
+      m[r] = -CUDART_INF_F;
+    }
+    const int n = pc.t1 - pc.t0;
+    for (int t = 0; t < n; ++t, ++i) {
+      __syncwarp();
+      if (bar_any(1, 128, !alive)) {  // the group stops together
+        stop = true;
+        break;
+      }
+      const int pos0 = (pc.t0 + t) * T;
+      const int pos = pos0 + tok;
+      float x[N];
+      if (warp_wait(sfull0 + 8 * (i & 1), (i >> 1) & 1, 19, i, i & 1)) {
+        tc::ld_32x32b<N>(tS + lanes + (i & 1) * N, x);
+        tc::wait_ld();
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sfree0 + 8 * (i & 1));
+      } else {
+        alive = false;
+#pragma unroll
+        for (int r = 0; r < N; ++r) x[r] = 0.f;
+      }
+
+      // scale (log2 units), soft-cap, then the masks: rows past the
+      // segment's G, and keys outside a row's range (tiles at a request's
+      // start, end or window edge only)
+      const bool inner = pos0 >= lo_max && pos0 + T <= hi_min;
+#pragma unroll
+      for (int r = 0; r < N; ++r) {
+        float v = x[r] * a.score_scale;
+        if (a.cap_l2 > 0.f) v = a.cap_l2 * tanhf(v / a.cap_l2);
+        bool vis = r < G;
+        if (!inner) {
+          int chi = L - (Q - 1 - r / GK);
+          chi = chi < L ? chi : L;
+          const int clo = (a.window > 0 && chi > a.window) ? chi - a.window : 0;
+          vis = vis && pos >= clo && pos < chi;
+        }
+        x[r] = vis ? v : -CUDART_INF_F;
+      }
+      bool need = false;
+#pragma unroll
+      for (int r = 0; r < N; ++r) need |= x[r] > m[r] + kRescaleSlack;
+      __syncwarp();
+      const bool slow = bar_any(1, 128, need);
+      resc &= ~(1u << (i & 1));
+      if (slow) {
+        // the tile's maximum of every row over the 128 tokens
+        float v[N];
+#pragma unroll
+        for (int r = 0; r < N; ++r) v[r] = x[r];
+        const float wmax = warp_rows_reduce<N, true>(v, lane);
+        if (lane < N) s_red[sw * N + lane] = wmax;
+        named_barrier_sync(1, 128);
+#pragma unroll
+        for (int r = 0; r < N; ++r) {
+          const float tm = fmaxf(fmaxf(s_red[r], s_red[N + r]), fmaxf(s_red[2 * N + r], s_red[3 * N + r]));
+          float al = 1.f;
+          if (tm > m[r] + kRescaleSlack) {
+            al = exp2_approx(m[r] - tm);  // m = -inf: 0
+            m[r] = tm;
+          }
+          l[r] *= al;
+          if (tok == r) s_alpha[(i & 1) * N + r] = al;
+        }
+        resc |= 1u << (i & 1);
+        named_barrier_sync(1, 128);  // s_alpha written; s_red read by all
+      }
+      // P = exp2(x - m), its row sums, and the bf16 hi / lo parts
+      uint32_t ph[N / 2], pl[N / 2];
+#pragma unroll
+      for (int r = 0; r < N; r += 2) {
+        const float p0 = x[r] == -CUDART_INF_F ? 0.f : exp2_approx(x[r] - m[r]);
+        const float p1 = x[r + 1] == -CUDART_INF_F ? 0.f : exp2_approx(x[r + 1] - m[r + 1]);
+        l[r] += p0;
+        l[r + 1] += p1;
+        const uint32_t h = pack_bf16x2(p0, p1);
+        ph[r / 2] = h;
+        pl[r / 2] = pack_bf16x2(p0 - bf16lo(h), p1 - bf16hi(h));
+      }
+      if (!alive) continue;
+      // V rows of keys outside [lo, L) may hold anything (NaN included) and
+      // meet P = 0 in the product: zero them once the tile has landed
+      if (pos0 < lo || pos0 + T > L) {
+        const bool out = pos < lo || pos >= L;
+        if (__any_sync(0xffffffffu, out)) {
+          const int vsl = i % VS;
+          if (!warp_wait(vfull0 + 8 * vsl, (i / VS) & 1, 20, i, vsl)) {
+            alive = false;
+            continue;
+          }
+          if (out) {
+            const uint32_t row = vring + vsl * C::TILE_BYTES + (tok >> 3) * C::GROUP_BYTES + (tok & 7) * 128;
+#pragma unroll
+            for (int p = 0; p < NP; ++p)
+#pragma unroll
+              for (int ch = 0; ch < 8; ++ch) sts128(row + p * 1024 + ch * 16, make_uint4(0, 0, 0, 0));
+          }
+        }
+      }
+      // the P buffer is free once the previous tile's output product is done
+      if (pending >= 0 &&
+          !warp_wait(ofull0 + 8 * (pending & 1), (pending >> 1) & 1, 21, pending, pending & 1)) {
+        alive = false;
+        continue;
+      }
+      // P^T, N rows of a token contiguous (2N bytes), 16-byte chunks
+      // swizzled by the address bits above them (64- or 32-byte swizzle)
+      {
+        constexpr int CH = N / 8;  // 16-byte chunks a token
+        const int sel = N == 32 ? ((tok >> 1) & 3) : ((tok >> 2) & 1);
+#pragma unroll
+        for (int ch = 0; ch < CH; ++ch) {
+          const uint32_t off = tok * (2 * N) + ((ch ^ sel) * 16);
+          sts128(p_hi + off, make_uint4(ph[4 * ch], ph[4 * ch + 1], ph[4 * ch + 2], ph[4 * ch + 3]));
+          sts128(p_lo + off, make_uint4(pl[4 * ch], pl[4 * ch + 1], pl[4 * ch + 2], pl[4 * ch + 3]));
+        }
+      }
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pfull);
+      if (pending >= 0) take_o(pending);
+      pending = i;
+    }
+    if (stop) break;
+    // ---- piece end: the last tile's output, the row sums, the results
+    if (pending >= 0) take_o(pending);
+    pending = -1;
+    __syncwarp();
+    if (bar_any(1, 128, !alive)) break;  // also: every reader of s_red is done
+    float lsum[N];
+    {
+      float v[N];
+#pragma unroll
+      for (int r = 0; r < N; ++r) v[r] = l[r];
+      const float wsum = warp_rows_reduce<N, false>(v, lane);
+      if (lane < N) s_red[sw * N + lane] = wsum;
+      named_barrier_sync(1, 128);
+#pragma unroll
+      for (int r = 0; r < N; ++r) lsum[r] = (s_red[r] + s_red[N + r]) + (s_red[2 * N + r] + s_red[3 * N + r]);
+    }
+    const bool whole = pc.n_pieces == 1;
+    const int slot_idx = c + pc.seg;
+#pragma unroll
+    for (int r = 0; r < N; ++r) {
+      if (r >= G) break;
+      const bool empty = !(lsum[r] > 0.f);
+      const float val = empty ? 0.f : acc[r] / lsum[r];
+      const size_t row = (static_cast<size_t>(pc.b) * Q + r / GK) * a.qo_heads +
+                         static_cast<size_t>(pc.h) * GK + r % GK;
+      if (whole) {
+        a.out[row * D + tok] = bf16_bits(val);
+      } else if (FA_CHECK(a.status, slot_idx < a.max_partials, 402, slot_idx)) {
+        a.part_o[(static_cast<size_t>(slot_idx) * G + r) * D + tok] = val;
+      }
+      if (tok == r) {
+        const float lv = empty ? -CUDART_INF_F : (m[r] + __log2f(lsum[r])) * kLn2;
+        if (whole) {
+          if (a.lse != nullptr) a.lse[row] = lv;
+        } else if (slot_idx < a.max_partials) {
+          a.part_lse[static_cast<size_t>(slot_idx) * G + r] = lv;
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  named_barrier_sync(2, 160);
+}
+
+}  // namespace fa

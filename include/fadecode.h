@@ -74,9 +74,15 @@ typedef enum { FA_KV_BF16 = 0, FA_KV_FP8_E4M3 = 1, FA_KV_INT4 = 2 } fa_kv_dtype;
  * and warp-shuffle reductions (a GEMV per head); MMA runs the two skinny
  * products (scores and probabilities times V) on the warp-level tensor-core
  * instruction with fp32 accumulation, which keeps the instruction count per
- * KV byte low when several query heads share a kv head.  AUTO lets the
- * planner choose from the shape (see fa_plan_info). */
-typedef enum { FA_PATH_AUTO = 0, FA_PATH_SIMT = 1, FA_PATH_MMA = 2 } fa_path;
+ * KV byte low when several query heads share a kv head.  TC runs the same
+ * two products on the 5th-generation tensor cores (tcgen05, accumulators in
+ * tensor memory) with 128-token tiles as the large dimension; it covers bf16
+ * K/V with head_dim 128, 9 to 32 rows per segment (query heads per kv head
+ * times query tokens), contiguous K/V or pages of at least 8 tokens, and the
+ * plain running max (not unified_max).  AUTO lets the planner choose from the
+ * shape (see fa_plan_info): TC where it applies, else MMA, else SIMT, unless
+ * the measured table (fa_set_tuning) says otherwise. */
+typedef enum { FA_PATH_AUTO = 0, FA_PATH_SIMT = 1, FA_PATH_MMA = 2, FA_PATH_TC = 3 } fa_path;
 
 /* Device-side check bits, reported by fa_decode_status. */
 enum {
@@ -109,8 +115,8 @@ typedef struct {
                       /* itself, or the last `window` of them.  The rows of  */
                       /* a (request, kv head) segment, (qo_heads / kv_heads) */
                       /* * q_len, must be <= 32 on the MMA dataflow (SIMT:   */
-                      /* exactly 1, 2, 4 or 8; 1, 2 or 4 for fp8; int4 runs  */
-                      /* on the MMA dataflow only).                          */
+                      /* exactly 1, 2, 4 or 8; int4 runs on the tensor-core  */
+                      /* dataflows only; TC: 9 to 32, see fa_path).          */
   float logit_cap;    /* 0: none.  c > 0: logit soft-capping, each scaled    */
                       /* score s becomes c * tanh(s / c) before the softmax  */
                       /* (Gemma 2's soft-cap, named on "FlashInfer x JAX via */

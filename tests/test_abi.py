@@ -233,12 +233,20 @@ def test_plan_with_several_query_tokens(lib):
     inf = _info(lib, h)
     assert inf.path == binding.PATH_MMA
     lib.fa_plan_destroy(h)
-    # rows 4 * 4 = 16 and 4 * 8 = 32: row teams on the MMA dataflow
+    # rows 4 * 4 = 16 and 4 * 8 = 32: the tcgen05 dataflow (bf16, head_dim
+    # 128), or row teams on the MMA dataflow when that one is asked for or
+    # the unified max is on
     for q_len in (4, 8):
         st, h, ws = _plan(lib, _desc(qo_heads=8, kv_heads=2, q_len=q_len), [0, 1000])
         assert st == 0
-        assert _info(lib, h).path == binding.PATH_MMA
+        inf = _info(lib, h)
+        assert inf.path == binding.PATH_TC and inf.tile_tokens == 128
         lib.fa_plan_destroy(h)
+        for kw in (dict(path=binding.PATH_MMA), dict(unified_max=1, softmax_phi=2.0)):
+            st, h, ws = _plan(lib, _desc(qo_heads=8, kv_heads=2, q_len=q_len, **kw), [0, 1000])
+            assert st == 0
+            assert _info(lib, h).path == binding.PATH_MMA
+            lib.fa_plan_destroy(h)
     # rows 8 * 8 = 64 exceed every kernel
     st, h, ws = _plan(lib, _desc(qo_heads=16, kv_heads=2, q_len=8), [0, 1000])
     assert st == 2 and not h  # FA_ERR_UNSUPPORTED
@@ -312,8 +320,14 @@ def test_tuning_table_drives_the_auto_choice(lib):
             st, h, _ = _plan(lib, _desc(**kw), [0, 1000])
             assert _info(lib, h).path == binding.PATH_MMA
             lib.fa_plan_destroy(h)
-        # a SIMT row for 16 rows has no kernel: passed over, MMA row teams run it
+        # a SIMT row for 16 rows has no kernel: passed over, the fixed rule
+        # (the tcgen05 dataflow for bf16 head_dim 128) runs it
         binding.set_tuning([_row(rows_min=16, rows_max=16)])
+        st, h, _ = _plan(lib, _desc(qo_heads=16, kv_heads=1), [0, 1000])
+        assert st == 0 and _info(lib, h).path == binding.PATH_TC
+        lib.fa_plan_destroy(h)
+        # a measured MMA row for 16 rows takes precedence over it
+        binding.set_tuning([_row(rows_min=16, rows_max=16, path=binding.PATH_MMA)])
         st, h, _ = _plan(lib, _desc(qo_heads=16, kv_heads=1), [0, 1000])
         assert st == 0 and _info(lib, h).path == binding.PATH_MMA
         lib.fa_plan_destroy(h)
@@ -327,7 +341,7 @@ def test_tuning_table_drives_the_auto_choice(lib):
 
 @pytest.mark.parametrize("bad", [dict(rows_min=0), dict(rows_min=5, rows_max=4),
                                  dict(bytes_min=10, bytes_max=9), dict(bytes_min=-1),
-                                 dict(path=0), dict(path=3), dict(kv_dtype=3),
+                                 dict(path=0), dict(path=4), dict(kv_dtype=3),
                                  dict(max_pieces=-1), dict(max_pieces=1025), dict(head_dim=0)])
 def test_tuning_table_rejects_bad_rows(lib, bad):
     before = binding.get_tuning()
@@ -428,11 +442,13 @@ def test_head_tile_choice(lib):
 def test_piece_cost_choice(lib):
     """The split's charge per segment: the caller's value when positive,
     none when negative; otherwise 2 tiles up to 8 rows, 4 with int4 head
-    tiles, 8 with 16 or 32 rows.  Never on the segment-aligned split nor
-    when blocks get a tile each; a charge above 4096 is rejected."""
+    tiles, 8 with 16 or 32 rows on the MMA dataflow, 2 (128-token) tiles on
+    the tcgen05 one.  Never on the segment-aligned split nor when blocks get
+    a tile each; a charge above 4096 is rejected."""
     lens = np.concatenate([[0], np.cumsum([3000, 100, 9000, 40] * 16)])
     B = len(lens) - 1
-    cases = [(dict(), 2), (dict(q_len=2), 2), (dict(qo_heads=32), 8), (dict(q_len=4), 8),
+    cases = [(dict(), 2), (dict(q_len=2), 2), (dict(qo_heads=32), 2), (dict(q_len=4), 2),
+             (dict(qo_heads=32, path=2), 8), (dict(q_len=4, path=2), 8),
              (dict(qo_heads=16, kv_heads=4, kv_dtype=2), 4), (dict(piece_cost=5), 5),
              (dict(piece_cost=-1), 0), (dict(q_len=4, piece_cost=-7), 0),
              (dict(piece_cost=4096), 4096), (dict(path=1), 2)]
@@ -489,12 +505,24 @@ def test_tiles_fit_the_pages(lib):
     """A paged tile is one page per box or a slice of one page, so tile and
     page lengths must divide one another: 32 rows take 48-token tiles with
     pages of 16 tokens or fewer, and the 32-token variant with 32- or
-    64-token pages."""
+    64-token pages.  The tcgen05 dataflow copies 8 tokens at a time into
+    128-token tiles: pages of 8 tokens or more; shorter pages take the MMA
+    dataflow."""
     for ps, T in ((1, 48), (16, 48), (32, 32), (64, 32), (256, 32)):
-        st, h, _ = _plan(lib, _desc(qo_heads=32, kv_heads=1, paged=1, page_size=ps), [0, 3000])
+        st, h, _ = _plan(lib, _desc(qo_heads=32, kv_heads=1, paged=1, page_size=ps,
+                                    path=binding.PATH_MMA), [0, 3000])
         assert st == 0, ps
         inf = _info(lib, h)
         assert inf.tile_tokens == T, (ps, inf.tile_tokens)
         assert (ps % T == 0) if ps >= T else (T % ps == 0)
         lib.fa_plan_destroy(h)
+    for ps, path in ((1, binding.PATH_MMA), (4, binding.PATH_MMA), (8, binding.PATH_TC),
+                     (16, binding.PATH_TC), (256, binding.PATH_TC)):
+        st, h, _ = _plan(lib, _desc(qo_heads=32, kv_heads=1, paged=1, page_size=ps), [0, 3000])
+        assert st == 0, ps
+        assert _info(lib, h).path == path, ps
+        lib.fa_plan_destroy(h)
+    st, h, _ = _plan(lib, _desc(qo_heads=32, kv_heads=1, paged=1, page_size=4,
+                                path=binding.PATH_TC), [0, 3000])
+    assert st == 2 and not h.value  # no tcgen05 kernel for 4-token pages
 

@@ -18,11 +18,10 @@ PATHS = ["simt", "mma"]
 
 def _has_path(x, path):
     """Whether a kernel exists: rows per segment (group x query tokens) of
-    1, 2, 4 or 8 on SIMT (fp8: up to 4; no int4), up to 32 on MMA."""
+    1, 2, 4 or 8 on SIMT (no int4), up to 32 on MMA."""
     rows = x.group * x.q_len
     if path == "simt":
-        return (x.kv_dtype != "int4" and rows in (1, 2, 4, 8)
-                and not (x.kv_dtype == "fp8_e4m3" and rows == 8))
+        return x.kv_dtype != "int4" and rows in (1, 2, 4, 8)
     return rows <= 32
 
 
@@ -411,6 +410,15 @@ CAPPED = [
                                                        "q_len": 2}),
     ("cap15_int4", 2, 8, 2, 128, [700, 33], {"logit_cap": 15.0, "sm_scale": 0.5,
                                              "kv_dtype": "int4"}),
+    # small caps: the capped scores sit within [-c, c], so a masked key (window
+    # start, ragged tail, causal edge) given the cap's floor -c instead of -inf
+    # would carry a visible weight
+    ("cap1_window_q2_gqa2", 2, 4, 2, 128, [700, 45], {"logit_cap": 1.0, "sm_scale": 0.05,
+                                                       "window": 150, "q_len": 2}),
+    ("cap1_fp8_window", 2, 8, 2, 128, [500, 70], {"logit_cap": 1.0, "sm_scale": 0.05,
+                                                  "kv_dtype": "fp8_e4m3", "window": 100}),
+    ("cap2_int4_tail", 2, 8, 2, 128, [130, 33], {"logit_cap": 2.0, "sm_scale": 0.1,
+                                                 "kv_dtype": "int4"}),
 ]
 
 
@@ -591,8 +599,7 @@ def test_random_shapes_match_the_oracle(case):
                          q_len=x.q_len, logit_cap=x.logit_cap, softmax_phi=phi)
     except binding.FadecodeError as e:
         assert e.status == 2, str(e)
-        simt_ok = (x.kv_dtype != "int4" and rows in (1, 2, 4, 8)
-                   and not (x.kv_dtype == "fp8_e4m3" and rows == 8))
+        simt_ok = x.kv_dtype != "int4" and rows in (1, 2, 4, 8)
         assert path == "simt" and not simt_ok, f"unexpected refusal: {e}"
         return
     ref_out, ref_lse = oracle.decode_all(x)
