@@ -522,9 +522,15 @@ struct SimtConsumer {
   static_assert(LPT >= 1 && LPT <= 32 && (NCH % CPL) == 0, "lane mapping");
   static_assert(TPS >= 1 && (C::T % SLOTS) == 0, "tokens per slot");
 
-  float q[G][E];
-  float acc[G][E];
+  // q and the accumulators in element pairs: both products run on the
+  // packed fp32 FMA (two lanes of fp32 per instruction on sm_100)
+  float2 q[G][E / 2];
+  float2 acc[G][E / 2];
   float m[G], l[G];
+  // the lane's chunk offsets within a tile row, when the swizzle phase of a
+  // row depends only on the lane's slot (rows of one lane step by SLOTS)
+  static constexpr bool kFixedSwizzle = C::TOKEN_MAJOR && (SLOTS * C::NP) % 8 == 0;
+  uint32_t koff[CPL];
   uint32_t fresh;  // unified max: bit h set while row h has seen no finite score
   int slot, j;
 
@@ -574,8 +580,12 @@ struct SimtConsumer {
   // Shared address of the lane's chunk k of tile row r (8-byte chunks: the
   // 16-byte chunk that holds it, plus the half).
   __device__ __forceinline__ uint32_t addr(uint32_t tile, int r, int k, int swz) const {
-    const int cip = chunk_in_plane(k);
-    return tile_addr<C>(tile, r, chunk_plane(k), cip * CHB / 16, swz) + (cip * CHB) % 16;
+    if constexpr (kFixedSwizzle) {
+      return tile + static_cast<uint32_t>(r * C::NP * C::CB) + koff[k];
+    } else {
+      const int cip = chunk_in_plane(k);
+      return tile_addr<C>(tile, r, chunk_plane(k), cip * CHB / 16, swz) + (cip * CHB) % 16;
+    }
   }
 
   // qs: the piece's query rows (staged in shared memory, or in global
@@ -586,6 +596,14 @@ struct SimtConsumer {
                                               float kscale, int lane, int /*team: one team*/) {
     slot = lane / LPT;
     j = lane % LPT;
+    if constexpr (kFixedSwizzle) {
+#pragma unroll
+      for (int k = 0; k < CPL; ++k) {
+        const int cip = chunk_in_plane(k), p = chunk_plane(k);
+        koff[k] = tile_addr<C>(0u, slot, p, cip * CHB / 16, a.swz) - slot * C::NP * C::CB +
+                  (cip * CHB) % 16;
+      }
+    }
     float scale = a.score_scale;
     if constexpr (FP8) scale *= kscale;
 #pragma unroll
@@ -599,12 +617,11 @@ struct SimtConsumer {
           const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            q[h][k * EPC + e + 2 * i] = bf16lo(u[i]) * scale;
-            q[h][k * EPC + e + 2 * i + 1] = bf16hi(u[i]) * scale;
+            q[h][(k * EPC + e) / 2 + i] = make_float2(bf16lo(u[i]) * scale, bf16hi(u[i]) * scale);
           }
         }
 #pragma unroll
-        for (int e = 0; e < EPC; ++e) acc[h][k * EPC + e] = 0.f;
+        for (int e = 0; e < EPC / 2; ++e) acc[h][k * EPC / 2 + e] = make_float2(0.f, 0.f);
       }
       m[h] = a.m_init;
       l[h] = 0.f;
@@ -638,9 +655,9 @@ struct SimtConsumer {
 #pragma unroll
       for (int tt = 0; tt < TPSC; ++tt) {
         const int r = (si * TPSC + tt) * SLOTS + slot;
-        float part[G];
+        float2 part2[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) part[h] = 0.f;
+        for (int h = 0; h < G; ++h) part2[h] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int k = 0; k < CPL; ++k) {
           float x[EPC];
@@ -648,8 +665,12 @@ struct SimtConsumer {
 #pragma unroll
           for (int h = 0; h < G; ++h)
 #pragma unroll
-            for (int e = 0; e < EPC; ++e) part[h] = fmaf(q[h][k * EPC + e], x[e], part[h]);
+            for (int e = 0; e < EPC; e += 2)
+              part2[h] = __ffma2_rn(q[h][(k * EPC + e) / 2], make_float2(x[e], x[e + 1]), part2[h]);
         }
+        float part[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) part[h] = part2[h].x + part2[h].y;
 #pragma unroll
         for (int off = 1; off < LPT; off <<= 1)
 #pragma unroll
@@ -709,7 +730,10 @@ struct SimtConsumer {
             const float alpha = exp2_approx(m[h] - tmax[h]);  // m = -inf -> 0
             l[h] *= alpha;
 #pragma unroll
-            for (int e = 0; e < E; ++e) acc[h][e] *= alpha;
+            for (int e = 0; e < E / 2; ++e) {
+              acc[h][e].x *= alpha;
+              acc[h][e].y *= alpha;
+            }
             m[h] = tmax[h];
           }
         }
@@ -734,7 +758,9 @@ struct SimtConsumer {
             for (int h = 0; h < G; ++h)
 #pragma unroll
               for (int e = 0; e < EPC; ++e)
-                acc[h][k * EPC + e] = fmaf(s[tt][h], x[e], acc[h][k * EPC + e]);
+                acc[h][(k * EPC) / 2 + e / 2] = __ffma2_rn(make_float2(s[tt][h], s[tt][h]),
+                                                           make_float2(x[e], x[e + 1]),
+                                                           acc[h][(k * EPC) / 2 + e / 2]);
           }
         }
       }
@@ -758,11 +784,14 @@ struct SimtConsumer {
 #pragma unroll
       for (int off = LPT; off < 32; off <<= 1) lh += __shfl_xor_sync(0xffffffffu, lh, off);
 #pragma unroll
-      for (int e = 0; e < E; ++e) {
-        float v = acc[h][e] * sc;
+      for (int e = 0; e < E / 2; ++e) {
+        float v0 = acc[h][e].x * sc, v1 = acc[h][e].y * sc;
 #pragma unroll
-        for (int off = LPT; off < 32; off <<= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        acc[h][e] = v;
+        for (int off = LPT; off < 32; off <<= 1) {
+          v0 += __shfl_xor_sync(0xffffffffu, v0, off);
+          v1 += __shfl_xor_sync(0xffffffffu, v1, off);
+        }
+        acc[h][e] = make_float2(v0, v1);
       }
       if (lane == 0) {
         m_area[w * G + h] = M;
@@ -772,7 +801,11 @@ struct SimtConsumer {
 #pragma unroll
         for (int k = 0; k < CPL; ++k)
 #pragma unroll
-          for (int e = 0; e < EPC; ++e) acc_area[(w * G + h) * D + dim_of(k, e)] = acc[h][k * EPC + e];
+          for (int e = 0; e < EPC; e += 2) {
+            const float2 v = acc[h][(k * EPC + e) / 2];
+            acc_area[(w * G + h) * D + dim_of(k, e)] = v.x;
+            acc_area[(w * G + h) * D + dim_of(k, e + 1)] = v.y;
+          }
       }
     }
   }
