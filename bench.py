@@ -614,8 +614,8 @@ def main():
                              "isolated_launch_us_median": round(median_launch * 1e3, 2),
                              "algorithmic_bytes_per_launch": kv_bytes},
                 # per step: the decode kernel, plus the split-merge kernel when
-                # the pass runs on more than one block
-                "gpu_launches": args.steps * (2 if runner.info["num_ctas"] > 1 else 1),
+                # some segment is split over blocks
+                "gpu_launches": args.steps * runner.info["launches"],
                 "clocks": clocks, "e2e": e2e,
                 "cpu_baseline": cpu, "sweep": sweep}
         print(json.dumps(line), flush=True)

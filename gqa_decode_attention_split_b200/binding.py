@@ -37,7 +37,7 @@ class FadecodeError(RuntimeError):
 
 
 # fadecode.h's FA_VERSION: the layouts of the structures below
-ABI_VERSION = 200
+ABI_VERSION = 300
 
 
 class DecodeDesc(ctypes.Structure):
@@ -57,7 +57,7 @@ class PlanInfo(ctypes.Structure):
                 ("total_tiles", ctypes.c_int32), ("max_partials", ctypes.c_int32),
                 ("workspace_bytes", ctypes.c_size_t), ("smem_bytes", ctypes.c_size_t),
                 ("v_stages", ctypes.c_int32), ("heads_per_tile", ctypes.c_int32),
-                ("piece_cost", ctypes.c_int32)]
+                ("piece_cost", ctypes.c_int32), ("launches", ctypes.c_int32)]
 
 
 class TuningEntry(ctypes.Structure):

@@ -370,6 +370,14 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
         seg_parts = static_cast<int32_t>(parts);
       }
     }
+    // A cap of one block per segment (measured faster for passes of a few
+    // hundred KB): every block takes one whole segment, whatever the lengths
+    // on the device, so no segment is ever split and the merge launch is
+    // not needed.
+    if (max_pieces == 1 && segs <= (1 << 20)) {
+      P = segs;
+      seg_parts = 1;
+    }
   }
   if (P > (1 << 20)) return FA_ERR_UNSUPPORTED;
 
@@ -448,6 +456,7 @@ extern "C" fa_status fa_plan_get_info(const fa_plan* plan, fa_plan_info_t* info)
   info->smem_bytes = plan->smem;
   info->heads_per_tile = plan->heads_per_tile;
   info->piece_cost = plan->piece_cost;
+  info->launches = (plan->num_ctas > 1 && plan->seg_parts != 1) ? 2 : 1;
   return FA_OK;
 }
 
@@ -662,6 +671,8 @@ extern "C" fa_status fa_decode_run(const fa_plan* plan, const void* q, const voi
   m.qo_heads = d.qo_heads;
   m.batch = d.batch;
   m.max_partials = plan->max_partials;
+  // one whole segment per block: nothing is split, nothing to merge
+  if (plan->seg_parts == 1) return FA_OK;
   e = fa::launch_split_merge(m, d.head_dim, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_failure("fa_decode_run: merge launch", e);
   return FA_OK;

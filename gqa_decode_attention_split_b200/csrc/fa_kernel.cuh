@@ -757,7 +757,7 @@ struct SimtConsumer {
 #pragma unroll
             for (int h = 0; h < G; ++h)
 #pragma unroll
-              for (int e = 0; e < EPC; ++e)
+              for (int e = 0; e < EPC; e += 2)
                 acc[h][(k * EPC) / 2 + e / 2] = __ffma2_rn(make_float2(s[tt][h], s[tt][h]),
                                                            make_float2(x[e], x[e + 1]),
                                                            acc[h][(k * EPC) / 2 + e / 2]);

@@ -150,7 +150,7 @@ typedef struct fa_plan fa_plan;
 
 /* What the planner chose (read-only view of a plan). */
 typedef struct {
-  int32_t path;             /* FA_PATH_SIMT or FA_PATH_MMA                    */
+  int32_t path;             /* FA_PATH_SIMT, FA_PATH_MMA or FA_PATH_TC        */
   int32_t num_ctas;         /* thread blocks launched by fa_decode_run        */
   int32_t tile_tokens;      /* tokens per KV tile moved by one TMA transaction */
   int32_t stages;           /* K tile slots of the shared-memory ring         */
@@ -162,6 +162,9 @@ typedef struct {
   int32_t heads_per_tile;   /* kv heads whose rows one tile holds per token:   */
                             /* > 1 for int4 (256 contiguous bytes a token)     */
   int32_t piece_cost;       /* tiles charged per segment in the split (0: none) */
+  int32_t launches;         /* kernel launches of one fa_decode_run: 1 (no     */
+                            /* segment is ever split: one block, or one whole  */
+                            /* segment per block) or 2 (with the split merge)  */
 } fa_plan_info_t;
 
 /*
@@ -410,9 +413,10 @@ FA_API const char* fa_last_error(void);
 
 /* Library version, major * 10000 + minor * 100 + patch.  The structures of
  * this header are those of FA_VERSION (0.2.0 added fa_decode_desc.piece_cost
- * and fa_plan_info_t.piece_cost); a caller built against it should check
- * that fa_version() / 100 == FA_VERSION / 100. */
-#define FA_VERSION 200
+ * and fa_plan_info_t.piece_cost; 0.3.0 added FA_PATH_TC and
+ * fa_plan_info_t.launches); a caller built against it should check that
+ * fa_version() / 100 == FA_VERSION / 100. */
+#define FA_VERSION 300
 FA_API int32_t fa_version(void);
 
 #ifdef __cplusplus

@@ -526,3 +526,27 @@ def test_tiles_fit_the_pages(lib):
                                 path=binding.PATH_TC), [0, 3000])
     assert st == 2 and not h.value  # no tcgen05 kernel for 4-token pages
 
+
+
+def test_one_block_per_segment_needs_no_merge(lib):
+    """A measured cap of one block per segment gives every (request, kv head)
+    segment one block and one launch per pass (no segment is ever split, so
+    no merge kernel), whatever the lengths."""
+    try:
+        binding.set_tuning([_row(rows_min=4, rows_max=4, path=binding.PATH_MMA, max_pieces=1)])
+        st, h, _ = _plan(lib, _desc(batch=3, qo_heads=8, kv_heads=2), [0, 5000, 5001, 9000])
+        assert st == 0
+        inf = _info(lib, h)
+        assert inf.num_ctas == 3 * 2 and inf.launches == 1 and inf.piece_cost == 0
+        lib.fa_plan_destroy(h)
+    finally:
+        binding.set_tuning(None)
+    # the default cut splits segments: two launches
+    st, h, _ = _plan(lib, _desc(batch=3, qo_heads=8, kv_heads=2), [0, 5000, 5001, 9000])
+    inf = _info(lib, h)
+    assert inf.num_ctas > 6 and inf.launches == 2
+    lib.fa_plan_destroy(h)
+    # one block: one launch
+    st, h, _ = _plan(lib, _desc(num_ctas=1), [0, 5000])
+    assert _info(lib, h).launches == 1
+    lib.fa_plan_destroy(h)

@@ -188,6 +188,38 @@ def test_paged_equals_contiguous_on_gpu():
         np.testing.assert_array_equal(l1, l2)
 
 
+@pytest.mark.parametrize("path", PATHS)
+def test_one_block_per_segment(path):
+    """With a measured cap of one block per segment the pass is one launch
+    and every segment is computed whole by one block: the oracle's result,
+    also when the device lengths are not the plan's (shorter requests)."""
+    x = synth.generate(4, 8, 2, 128, [700, 1, 0, 2300], seed=37, paged=True, page_size=16)
+    try:
+        binding.set_tuning([dict(head_dim=128, kv_dtype=0, rows_min=4, rows_max=4, bytes_min=0,
+                                 bytes_max=1 << 40, path=binding.PATH_SIMT if path == "simt"
+                                 else binding.PATH_MMA, max_pieces=1)])
+        dev = DeviceInputs(x)
+        p = dev.plan()
+        info = p.info()
+        assert info["launches"] == 1 and info["num_ctas"] == 8
+        ws = p.new_workspace()
+        o, l = to_numpy(*dev.run(p, workspace=ws))
+        assert binding.decode_status(ws) == 0
+        ref_out, ref_lse = oracle.decode_all(x)
+        assert_matches(o, l, ref_out, ref_lse, what=f"one block per segment {path}")
+        # shorter requests on the device than at planning time
+        import torch
+        short = np.array([0, 300, 301, 301, 1001], dtype=np.int32)
+        dev.kv_indptr.copy_(torch.from_numpy(short))
+        y = synth.DecodeInputs(**{**x.__dict__, "kv_indptr": short})
+        o, l = to_numpy(*dev.run(p, workspace=ws))
+        assert binding.decode_status(ws) == 0
+        ref_out, ref_lse = oracle.decode_all(y)
+        assert_matches(o, l, ref_out, ref_lse, what=f"one block per segment, shorter {path}")
+    finally:
+        binding.set_tuning(None)
+
+
 def test_bad_page_id_is_flagged_not_read():
     x = synth.generate(2, 8, 2, 128, [64, 64], paged=True, page_size=16, seed=25)
     x.page_table[1, 2] = x.k.shape[0] + 5  # outside the pool

@@ -72,7 +72,7 @@ def test_tc_matches_the_oracle(case):
     assert info["path"] == binding.PATH_TC and flags == 0
 
 
-@pytest.mark.parametrize("q_len", [2, 4, 8])
+@pytest.mark.parametrize("q_len", [3, 4, 8])
 def test_tc_forced_splits_agree(q_len):
     """Splitting over more blocks, then merging, gives the oracle's result at
     every granularity (one block up to one tile per block)."""
