@@ -268,6 +268,7 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   // for the shape, the SIMT path otherwise.
   const KernelEntry* k = nullptr;
   int64_t max_pieces = 32;  // average blocks per segment, at most
+  bool table_cap = false;   // max_pieces came from the measured table
   // the tcgen05 dataflow: bf16 K/V, head_dim 128, 9 to 32 rows, copies of
   // 8 tokens (pages of at least 8), the plain running max
   auto tc_entry = [&]() -> const KernelEntry* {
@@ -290,7 +291,10 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
           continue;
         k = path_entry(e.path);
         if (k == nullptr) continue;
-        if (e.max_pieces > 0) max_pieces = e.max_pieces;
+        if (e.max_pieces > 0) {
+          max_pieces = e.max_pieces;
+          table_cap = true;
+        }
         break;
       }
     }
@@ -330,10 +334,16 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   const int T = k->tile_tokens;
   int64_t tiles = 0;
   int64_t seg_tiles = -1;  // tiles of every segment when all are equal, else -1
+  int64_t max_seg_bytes = 0;  // visible K/V bytes of the largest segment
   for (int b = 0; b < desc->batch; ++b) {
-    const int64_t n = host_num_tiles(kv_indptr_host[b + 1] - kv_indptr_host[b], union_window(desc), T);
+    const int32_t L = kv_indptr_host[b + 1] - kv_indptr_host[b];
+    const int64_t n = host_num_tiles(L, union_window(desc), T);
     tiles += n;
     seg_tiles = b == 0 ? n : (seg_tiles == n ? n : -1);
+    const int32_t wu = union_window(desc);
+    const int64_t vis = (wu > 0 && L > wu) ? wu : L;
+    const int64_t sb = vis * 2 * row_bytes_of(desc) * ht;
+    if (sb > max_seg_bytes) max_seg_bytes = sb;
   }
   tiles *= seg_heads;
 
@@ -370,11 +380,16 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
         seg_parts = static_cast<int32_t>(parts);
       }
     }
-    // A cap of one block per segment (measured faster for passes of a few
-    // hundred KB): every block takes one whole segment, whatever the lengths
-    // on the device, so no segment is ever split and the merge launch is
-    // not needed.
-    if (max_pieces == 1 && segs <= (1 << 20)) {
+    // One whole segment per block: no segment is ever split, whatever the
+    // lengths on the device, so the merge launch is not needed.  Taken when
+    // the measured table caps the blocks per segment at one, and by default
+    // when every segment is small enough that splitting it cannot pay for
+    // the merge launch: a block streams a 128 KB segment in about the time
+    // the second launch costs (measured on B200: 2 segments of 128 KB,
+    // 15.4 us split over 8 blocks, 12.3 us whole; one 512 KB segment, 15.4
+    // us split, 22.7 us whole), and as long as the segments fit one wave.
+    const bool small_segs = max_seg_bytes <= (128 << 10) && segs <= num_sms;
+    if ((max_pieces == 1 || (small_segs && !table_cap)) && P > 1 && segs <= (1 << 20)) {
       P = segs;
       seg_parts = 1;
     }
