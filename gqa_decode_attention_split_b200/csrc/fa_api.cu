@@ -273,7 +273,10 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   // 8 tokens (pages of at least 8), the plain running max
   auto tc_entry = [&]() -> const KernelEntry* {
     if (desc->unified_max || group <= 8 || (pages != 0 && pages < 8)) return nullptr;
-    return find_entry(desc->head_dim, group, kind, fa::kPathTc, pages);
+    const KernelEntry* e = find_entry(desc->head_dim, group, kind, fa::kPathTc, pages);
+    // its rings leave room for the schedule arrays of a few hundred requests
+    if (e != nullptr && e->smem_bytes(desc->batch, group) > 232448) return nullptr;
+    return e;
   };
   auto path_entry = [&](int path) -> const KernelEntry* {
     return path == FA_PATH_SIMT ? find_entry(desc->head_dim, group, kind, fa::kPathSimt, pages)

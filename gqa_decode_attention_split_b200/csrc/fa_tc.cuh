@@ -51,7 +51,7 @@ struct TcCfg {
   static constexpr int KSTAGES = 3;
   static constexpr int VSTAGES = NR <= 16 ? 3 : 2;
   static constexpr int QSLOT_BYTES = NP * N * 128;  // [NP][N rows][128]
-  static constexpr int P_BYTES = T * N * 2;         // P hi (or lo): [T][N] bf16
+  static constexpr int P_BYTES = T * N * 2;         // P hi (or lo) of a tile: [T][N] bf16
   static constexpr int THREADS = 192;
   static constexpr uint32_t TMEM_COLS = 128;        // S[2] and O[2], N columns each
   static constexpr uint32_t P_LAYOUT = N == 32 ? tc::kSwizzle64 : tc::kSwizzle32;
@@ -60,8 +60,8 @@ struct TcCfg {
   static constexpr int OFF_V = OFF_K + KSTAGES * TILE_BYTES;
   static constexpr int OFF_Q = OFF_V + VSTAGES * TILE_BYTES;
   static constexpr int OFF_P = OFF_Q + 2 * QSLOT_BYTES;
-  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
-  static constexpr int NBARS = 2 * KSTAGES + 2 * VSTAGES + 14;
+  static constexpr int OFF_BAR = OFF_P + 4 * P_BYTES;  // P[2], hi + lo each
+  static constexpr int NBARS = 2 * KSTAGES + 2 * VSTAGES + 15;
   static constexpr int OFF_TMEM = OFF_BAR + 8 * NBARS;
   static constexpr int OFF_RED = OFF_TMEM + 16;    // [4][N] floats
   static constexpr int OFF_ALPHA = OFF_RED + 4 * N * 4;  // [2][N] floats
@@ -110,12 +110,12 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (sbase - raw);
   const uint32_t kring = sbase + C::OFF_K, vring = sbase + C::OFF_V, qslots = sbase + C::OFF_Q;
-  const uint32_t p_hi = sbase + C::OFF_P, p_lo = p_hi + C::P_BYTES;
+  const uint32_t p_buf = sbase + C::OFF_P;  // tile j: hi at p_buf + (j % 2) * 2 P_BYTES, lo after it
   const uint32_t kfull0 = sbase + C::OFF_BAR, kempty0 = kfull0 + 8 * KS;
   const uint32_t vfull0 = kempty0 + 8 * KS, vempty0 = vfull0 + 8 * VS;
   const uint32_t qfull0 = vempty0 + 8 * VS, qempty0 = qfull0 + 16;
   const uint32_t sfull0 = qempty0 + 16, sfree0 = sfull0 + 16;
-  const uint32_t pfull = sfree0 + 16, ofull0 = pfull + 8, ofree0 = ofull0 + 16;
+  const uint32_t pfull0 = sfree0 + 16, ofull0 = pfull0 + 16, ofree0 = ofull0 + 16;
   const uint32_t done_bar = ofree0 + 16;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base + C::OFF_TMEM);
   float* s_red = reinterpret_cast<float*>(base + C::OFF_RED);
@@ -156,8 +156,8 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
       mbar_init(sfree0 + 8 * s, 4);    // one arrival per softmax warp
       mbar_init(ofull0 + 8 * s, 1);
       mbar_init(ofree0 + 8 * s, 4);
+      mbar_init(pfull0 + 8 * s, 4);
     }
-    mbar_init(pfull, 4);
     mbar_init(done_bar, 1);
     fence_mbar_init();
   }
@@ -355,8 +355,8 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
           record_timeout(a.status, 11, j, vsl, (j / VS) & 1, vfull0 + 8 * vsl);
           ok = false;
         }
-        if (ok && !mbar_wait(pfull, j & 1, kWaitLimitNs)) {
-          record_timeout(a.status, 12, j, 0, j & 1, pfull);
+        if (ok && !mbar_wait(pfull0 + 8 * (j & 1), (j >> 1) & 1, kWaitLimitNs)) {
+          record_timeout(a.status, 12, j, j & 1, (j >> 1) & 1, pfull0 + 8 * (j & 1));
           ok = false;
         }
         if (ok && j >= 2 && !mbar_wait(ofree0 + 8 * (j & 1), ((j - 2) >> 1) & 1, kWaitLimitNs)) {
@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
         const uint32_t d = tO + (j & 1) * N;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
-          const uint32_t pb = part == 0 ? p_hi : p_lo;
+          const uint32_t pb = p_buf + (j & 1) * 2 * C::P_BYTES + part * C::P_BYTES;
 #pragma unroll
           for (int k = 0; k < T / 16; ++k) {
             // V^T: dims as M (64-dim atoms one plane = 1024 bytes apart),
@@ -445,6 +445,13 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
   const uint32_t lanes = static_cast<uint32_t>(quarter * 32) << 16;
   const int sw = warp - 2;                   // 0..3
   write_empty_results(a, it, s_len, G, D, c, P, tid - 64, 128);
+  // parameters in registers for the tile loop
+  const float sscale = a.score_scale, cap = a.cap_l2;
+  const int W = a.window, WU = a.window_u;
+  // a finite start for the running max: exp2(x - m) is then 0 for a masked
+  // score (x = -inf) without a select, and the first finite score of a row
+  // always passes the slack test (which rescales by exp2(-1e30 - x) = 0)
+  constexpr float kMStart = -1e30f;
 
   float acc[N], l[N], m[N];
   bool alive = true;     // this warp's waits have all succeeded
@@ -460,7 +467,7 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
   // reached by all 128 threads or by none.
   auto take_o = [&](int j) {
     if (!alive) return;
-    bool ok = mbar_wait(ofull0 + 8 * (j & 1), (j >> 1) & 1, kWaitLimitNs);
+    const bool ok = mbar_wait(ofull0 + 8 * (j & 1), (j >> 1) & 1, kWaitLimitNs);
     if (!ok && lane == 0) record_timeout(a.status, 18, j, j & 1, (j >> 1) & 1, ofull0 + 8 * (j & 1));
     if (!__all_sync(0xffffffffu, ok)) {  // tcgen05.ld is warp-collective
       alive = false;
@@ -492,14 +499,12 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
   bool stop = false;
   while (!stop && next_piece(its, pc, s_pre, s_len, B, H, a.window_u, T)) {
     const int L = s_len[pc.b];
-    const int lo = (a.window_u > 0 && L > a.window_u) ? L - a.window_u : 0;  // union of the rows' ranges
-    const int hi_min = L - (Q - 1);                                          // every row sees below this
-    const int lo_max = (a.window > 0 && L > a.window) ? L - a.window : 0;    // and from this on
+    const int lo = (WU > 0 && L > WU) ? L - WU : 0;  // keys some row sees: [lo, L)
 #pragma unroll
     for (int r = 0; r < N; ++r) {
       acc[r] = 0.f;
       l[r] = 0.f;
-      m[r] = -CUDART_INF_F;
+      m[r] = kMStart;
     }
     const int n = pc.t1 - pc.t0;
     for (int t = 0; t < n; ++t, ++i) {
@@ -522,27 +527,27 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
 #pragma unroll
         for (int r = 0; r < N; ++r) x[r] = 0.f;
       }
-
-      // scale (log2 units), soft-cap, then the masks: rows past the
-      // segment's G, and keys outside a row's range (tiles at a request's
-      // start, end or window edge only)
-      const bool inner = pos0 >= lo_max && pos0 + T <= hi_min;
+      // The rows that see this thread's key: query token q (rows q GK ..
+      // q GK + GK - 1) sees keys below L - Q + 1 + q and, with a window, from
+      // L - Q + 1 + q - W on, so the rows form one range [rlo, rhi).
+      const int base = pos - L + Q;
+      const int qlo = base > 0 ? base : 0;
+      const int qhi = W > 0 ? (base + W < Q ? base + W : Q) : Q;
+      const int rlo = qlo * GK;
+      const uint32_t rspan = qhi > qlo ? static_cast<uint32_t>((qhi - qlo) * GK) : 0u;
+      // scale (log2 units), soft-cap, then the masks
 #pragma unroll
-      for (int r = 0; r < N; ++r) {
-        float v = x[r] * a.score_scale;
-        if (a.cap_l2 > 0.f) v = a.cap_l2 * tanhf(v / a.cap_l2);
-        bool vis = r < G;
-        if (!inner) {
-          int chi = L - (Q - 1 - r / GK);
-          chi = chi < L ? chi : L;
-          const int clo = (a.window > 0 && chi > a.window) ? chi - a.window : 0;
-          vis = vis && pos >= clo && pos < chi;
-        }
-        x[r] = vis ? v : -CUDART_INF_F;
+      for (int r = 0; r < N; ++r) x[r] *= sscale;
+      if (cap > 0.f) {
+#pragma unroll
+        for (int r = 0; r < N; ++r) x[r] = cap * tanhf(x[r] / cap);
       }
       bool need = false;
 #pragma unroll
-      for (int r = 0; r < N; ++r) need |= x[r] > m[r] + kRescaleSlack;
+      for (int r = 0; r < N; ++r) {
+        x[r] = static_cast<uint32_t>(r - rlo) < rspan ? x[r] : -CUDART_INF_F;
+        need |= x[r] - m[r] > kRescaleSlack;
+      }
       __syncwarp();
       const bool slow = bar_any(1, 128, need);
       resc &= ~(1u << (i & 1));
@@ -558,8 +563,8 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
         for (int r = 0; r < N; ++r) {
           const float tm = fmaxf(fmaxf(s_red[r], s_red[N + r]), fmaxf(s_red[2 * N + r], s_red[3 * N + r]));
           float al = 1.f;
-          if (tm > m[r] + kRescaleSlack) {
-            al = exp2_approx(m[r] - tm);  // m = -inf: 0
+          if (tm - m[r] > kRescaleSlack) {
+            al = exp2_approx(m[r] - tm);  // from the start value: 0
             m[r] = tm;
           }
           l[r] *= al;
@@ -568,12 +573,13 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
         resc |= 1u << (i & 1);
         named_barrier_sync(1, 128);  // s_alpha written; s_red read by all
       }
-      // P = exp2(x - m), its row sums, and the bf16 hi / lo parts
+      // P = exp2(x - m) (0 for a masked key), its row sums, and the bf16
+      // hi / lo parts
       uint32_t ph[N / 2], pl[N / 2];
 #pragma unroll
       for (int r = 0; r < N; r += 2) {
-        const float p0 = x[r] == -CUDART_INF_F ? 0.f : exp2_approx(x[r] - m[r]);
-        const float p1 = x[r + 1] == -CUDART_INF_F ? 0.f : exp2_approx(x[r + 1] - m[r + 1]);
+        const float p0 = exp2_approx(x[r] - m[r]);
+        const float p1 = exp2_approx(x[r + 1] - m[r + 1]);
         l[r] += p0;
         l[r + 1] += p1;
         const uint32_t h = pack_bf16x2(p0, p1);
@@ -600,27 +606,25 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
           }
         }
       }
-      // the P buffer is free once the previous tile's output product is done
-      if (pending >= 0 &&
-          !warp_wait(ofull0 + 8 * (pending & 1), (pending >> 1) & 1, 21, pending, pending & 1)) {
-        alive = false;
-        continue;
-      }
-      // P^T, N rows of a token contiguous (2N bytes), 16-byte chunks
-      // swizzled by the address bits above them (64- or 32-byte swizzle)
+      // P^T of tile i into buffer i % 2 (free: the output product of tile
+      // i - 2 was waited for when its O was read), N rows of a token
+      // contiguous (2N bytes), 16-byte chunks swizzled by the address bits
+      // above them (64- or 32-byte swizzle)
       {
         constexpr int CH = N / 8;  // 16-byte chunks a token
         const int sel = N == 32 ? ((tok >> 1) & 3) : ((tok >> 2) & 1);
+        const uint32_t hi_buf = p_buf + (i & 1) * 2 * C::P_BYTES;
 #pragma unroll
         for (int ch = 0; ch < CH; ++ch) {
           const uint32_t off = tok * (2 * N) + ((ch ^ sel) * 16);
-          sts128(p_hi + off, make_uint4(ph[4 * ch], ph[4 * ch + 1], ph[4 * ch + 2], ph[4 * ch + 3]));
-          sts128(p_lo + off, make_uint4(pl[4 * ch], pl[4 * ch + 1], pl[4 * ch + 2], pl[4 * ch + 3]));
+          sts128(hi_buf + off, make_uint4(ph[4 * ch], ph[4 * ch + 1], ph[4 * ch + 2], ph[4 * ch + 3]));
+          sts128(hi_buf + C::P_BYTES + off,
+                 make_uint4(pl[4 * ch], pl[4 * ch + 1], pl[4 * ch + 2], pl[4 * ch + 3]));
         }
       }
       tc::fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(pfull);
+      if (lane == 0) mbar_arrive(pfull0 + 8 * (i & 1));
       if (pending >= 0) take_o(pending);
       pending = i;
     }
