@@ -515,16 +515,29 @@ fa_status make_kv_map(const fa_plan* p, const void* base, int64_t kv_rows, CUten
                                       : span >= 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
                                                     : CU_TENSOR_MAP_L2_PROMOTION_NONE;
   CUresult r;
-  if (k->tc_copies) {
-    // tcgen05 dataflow: copies of 8 token rows of one kv head, landing as
-    // [plane][8 rows][128 bytes] (the 8-row groups the tensor core reads with
-    // the 128-byte swizzle).  Paged pools are read as token rows too: a page
-    // holds page_size consecutive rows of [kv_heads][head_dim].
-    const cuuint64_t rows = static_cast<cuuint64_t>(kv_rows) * (d.paged ? d.page_size : 1);
-    const cuuint64_t dims[4] = {inner, rows, np, static_cast<cuuint64_t>(d.kv_heads)};
+  if (k->tc_copies && !d.paged) {
+    // tcgen05 dataflow, contiguous rows: copies of 8 token rows of one kv
+    // head, landing as [plane][8 rows][128 bytes] (the 8-row groups the
+    // tensor core reads with the 128-byte swizzle)
+    const cuuint64_t dims[4] = {inner, static_cast<cuuint64_t>(kv_rows), np,
+                                static_cast<cuuint64_t>(d.kv_heads)};
     const cuuint64_t strides[3] = {row * d.kv_heads, cb, row};
     const cuuint32_t box[4] = {inner, 8, static_cast<cuuint32_t>(np), 1};
     r = enc(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, promo,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else if (k->tc_copies) {
+    // tcgen05 dataflow, paged pool: the pool's token rows (a page holds
+    // page_size consecutive rows of [kv_heads][head_dim]) as groups of 8, so
+    // one copy moves a whole page (or a 128-token slice of a longer one) and
+    // lands as [group][plane][8 rows][128 bytes]
+    const cuuint64_t groups = static_cast<cuuint64_t>(kv_rows) * d.page_size / 8;
+    const cuuint64_t dims[5] = {inner, 8, np, static_cast<cuuint64_t>(d.kv_heads), groups};
+    const cuuint64_t strides[4] = {row * d.kv_heads, cb, row, 8 * row * d.kv_heads};
+    const int per_copy = d.page_size < k->tile_tokens ? d.page_size : k->tile_tokens;
+    const cuuint32_t box[5] = {inner, 8, static_cast<cuuint32_t>(np), 1,
+                               static_cast<cuuint32_t>(per_copy / 8)};
+    r = enc(map, dt, 5, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, promo,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   } else if (k->token_major) {

@@ -16,9 +16,10 @@
 //                                                      hi + lo parts)
 //
 // Warp roles of a block (one per SM):
-//   warp 0  producer: bulk tensor copies of K and V tiles (128 tokens, 16
-//           copies of 8 tokens each, landing as [8-token group][plane][8][128
-//           bytes], 128-byte swizzle) and of each piece's query rows;
+//   warp 0  producer: bulk tensor copies of K and V tiles (128 tokens,
+//           landing as [8-token group][plane][8][128 bytes], 128-byte
+//           swizzle: one copy per page of a paged pool, 16 copies of 8 rows
+//           of contiguous K/V) and of each piece's query rows;
 //   warp 1  allocates tensor memory; one lane issues every tcgen05.mma and
 //           commits its completion to mbarriers;
 //   warps 2-5  the softmax group (128 threads): thread t reads token t's
@@ -258,25 +259,45 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
       const int npages = a.paged ? (L + ps - 1) >> a.page_shift : 0;
       const int pbase = a.paged ? (w0 * T) >> a.page_shift : 0;
       if (lane == 0) {
-        // token row of box j of tile tt: contiguous rows, or the pool's rows
-        // (pages hold ps consecutive token rows; a missing page reads zeros)
-        auto box_row = [&](int tt, int j) {
-          const int tok = tt * T + j * C::BOX_T;
-          if (!a.paged) return s_start[pc.b] + tok;
-          const int pidx = tok >> a.page_shift;
-          const int page = (pidx < npages && pidx - pbase < 64) ? s_pages[pidx - pbase] : -1;
-          return page * ps + (tok & (ps - 1));  // page -1: rows -ps.. -1, all outside
-        };
+        // Copies of a tile: contiguous rows, 16 copies of 8 rows (row
+        // s_start + token); paged, one copy per page of up to 128 tokens,
+        // addressed by 8-row group of the pool (a page holds page_size
+        // consecutive rows; a missing page reads zeros from a negative
+        // group).  The page ids of a tile are read before its copies go out.
+        const int cp = a.paged ? (ps < T ? ps : T) : C::BOX_T;  // tokens per copy
+        const int ncp = T / cp;
         for (int tt = w0; tt < w1; ++tt) {
+          int crd[C::BOXES];  // contiguous: first row; paged: first 8-row group
+#pragma unroll
+          for (int j = 0; j < C::BOXES; ++j) {
+            if (j < ncp) {
+              const int tok = tt * T + j * cp;
+              if (!a.paged) {
+                crd[j] = s_start[pc.b] + tok;
+              } else {
+                const int pidx = tok >> a.page_shift;
+                const int page = (pidx < npages && pidx - pbase < 64) ? s_pages[pidx - pbase] : -1;
+                crd[j] = (page * ps + (tok & (ps - 1))) >> 3;
+              }
+            }
+          }
           if (!mbar_wait(kempty0 + 8 * ks, kph ^ 1u, kWaitLimitNs)) {
             record_timeout(a.status, 1, kissued, ks, kph ^ 1u, kempty0 + 8 * ks);
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(kfull0 + 8 * ks, C::TILE_BYTES);
-          for (int j = 0; j < C::BOXES; ++j)
-            tma_load_4d(kring + ks * C::TILE_BYTES + j * C::GROUP_BYTES, &a.kmap, kfull0 + 8 * ks, 0,
-                        box_row(tt, j), 0, pc.h, pol);
+          const uint32_t kd = kring + ks * C::TILE_BYTES;
+#pragma unroll
+          for (int j = 0; j < C::BOXES; ++j) {
+            if (j < ncp) {
+              const uint32_t dst = kd + j * (cp / 8) * C::GROUP_BYTES;
+              if (a.paged)
+                tma_load_5d(dst, &a.kmap, kfull0 + 8 * ks, 0, 0, 0, pc.h, crd[j], pol);
+              else
+                tma_load_4d(dst, &a.kmap, kfull0 + 8 * ks, 0, crd[j], 0, pc.h, pol);
+            }
+          }
           ++kissued;
           if (!mbar_wait(vempty0 + 8 * vs, vph ^ 1u, kWaitLimitNs)) {
             record_timeout(a.status, 8, vissued, vs, vph ^ 1u, vempty0 + 8 * vs);
@@ -284,9 +305,17 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
             break;
           }
           mbar_arrive_expect_tx(vfull0 + 8 * vs, C::TILE_BYTES);
-          for (int j = 0; j < C::BOXES; ++j)
-            tma_load_4d(vring + vs * C::TILE_BYTES + j * C::GROUP_BYTES, &a.vmap, vfull0 + 8 * vs, 0,
-                        box_row(tt, j), 0, pc.h, pol);
+          const uint32_t vd = vring + vs * C::TILE_BYTES;
+#pragma unroll
+          for (int j = 0; j < C::BOXES; ++j) {
+            if (j < ncp) {
+              const uint32_t dst = vd + j * (cp / 8) * C::GROUP_BYTES;
+              if (a.paged)
+                tma_load_5d(dst, &a.vmap, vfull0 + 8 * vs, 0, 0, 0, pc.h, crd[j], pol);
+              else
+                tma_load_4d(dst, &a.vmap, vfull0 + 8 * vs, 0, crd[j], 0, pc.h, pol);
+            }
+          }
           ++vissued;
           if (++ks == KS) {
             ks = 0;
