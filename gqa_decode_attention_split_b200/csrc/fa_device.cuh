@@ -312,6 +312,16 @@ __device__ __forceinline__ void commit(uint32_t bar) {
 template <int N>
 __device__ __forceinline__ void ld_32x32b(uint32_t taddr, float (&v)[N]);
 template <>
+__device__ __forceinline__ void ld_32x32b<8>(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                 "=r"(r[7])
+               : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+template <>
 __device__ __forceinline__ void ld_32x32b<16>(uint32_t taddr, float (&v)[16]) {
   uint32_t r[16];
   asm volatile(

@@ -22,10 +22,12 @@
 //           of contiguous K/V) and of each piece's query rows;
 //   warp 1  allocates tensor memory; one lane issues every tcgen05.mma and
 //           commits its completion to mbarriers;
-//   warps 2-5  the softmax group (128 threads): thread t reads token t's
-//           scores from TMEM, keeps the running max per row (uniform over
-//           the group, rescaled only past an 8 log2-unit slack), writes P to
-//           shared memory, and reads back dimension t of each tile's O^T,
+//   warps 2-9  the softmax group: two row halves of four warps, each half
+//           covering the four TMEM lane quarters.  Thread (half, t) reads
+//           token t's scores of its half of the rows from TMEM, keeps their
+//           running max (uniform over the group, rescaled only past an 8
+//           log2-unit slack), writes its part of P to shared memory, and
+//           reads back dimension t of each tile's O^T for the same rows,
 //           accumulating it in fp32 registers.
 // The scores of tile i + 1 are computed while the softmax group works on tile
 // i; the output product of tile i runs while the scores of tile i + 1 are
@@ -53,7 +55,8 @@ struct TcCfg {
   static constexpr int VSTAGES = NR <= 16 ? 3 : 2;
   static constexpr int QSLOT_BYTES = NP * N * 128;  // [NP][N rows][128]
   static constexpr int P_BYTES = T * N * 2;         // P hi (or lo) of a tile: [T][N] bf16
-  static constexpr int THREADS = 192;
+  static constexpr int SG_WARPS = 8;   // softmax group: two row halves x 4 TMEM lane quarters
+  static constexpr int THREADS = 64 + 32 * SG_WARPS;
   static constexpr uint32_t TMEM_COLS = 128;        // S[2] and O[2], N columns each
   static constexpr uint32_t P_LAYOUT = N == 32 ? tc::kSwizzle64 : tc::kSwizzle32;
   // shared memory, from a 1024-aligned base
@@ -154,10 +157,10 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
       mbar_init(qfull0 + 8 * s, 1);
       mbar_init(qempty0 + 8 * s, 1);   // the commit of the piece's last score product
       mbar_init(sfull0 + 8 * s, 1);
-      mbar_init(sfree0 + 8 * s, 4);    // one arrival per softmax warp
+      mbar_init(sfree0 + 8 * s, C::SG_WARPS);  // one arrival per softmax warp
       mbar_init(ofull0 + 8 * s, 1);
-      mbar_init(ofree0 + 8 * s, 4);
-      mbar_init(pfull0 + 8 * s, 4);
+      mbar_init(ofree0 + 8 * s, C::SG_WARPS);
+      mbar_init(pfull0 + 8 * s, C::SG_WARPS);
     }
     mbar_init(done_bar, 1);
     fence_mbar_init();
@@ -258,63 +261,63 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
       if (a.paged && nhave) load_ids(pn, nw0, nv, nin);  // in flight during the issue loop
       const int npages = a.paged ? (L + ps - 1) >> a.page_shift : 0;
       const int pbase = a.paged ? (w0 * T) >> a.page_shift : 0;
-      if (lane == 0) {
+      {
         // Copies of a tile: contiguous rows, 16 copies of 8 rows (row
         // s_start + token); paged, one copy per page of up to 128 tokens,
         // addressed by 8-row group of the pool (a page holds page_size
         // consecutive rows; a missing page reads zeros from a negative
-        // group).  The page ids of a tile are read before its copies go out.
+        // group).  Lane j of the warp issues copy j, so one instruction sends
+        // all of a tile's copies; lane 0 waits for the slot and arms its
+        // barrier first.
         const int cp = a.paged ? (ps < T ? ps : T) : C::BOX_T;  // tokens per copy
         const int ncp = T / cp;
-        for (int tt = w0; tt < w1; ++tt) {
-          int crd[C::BOXES];  // contiguous: first row; paged: first 8-row group
-#pragma unroll
-          for (int j = 0; j < C::BOXES; ++j) {
-            if (j < ncp) {
-              const int tok = tt * T + j * cp;
-              if (!a.paged) {
-                crd[j] = s_start[pc.b] + tok;
-              } else {
-                const int pidx = tok >> a.page_shift;
-                const int page = (pidx < npages && pidx - pbase < 64) ? s_pages[pidx - pbase] : -1;
-                crd[j] = (page * ps + (tok & (ps - 1))) >> 3;
-              }
+        for (int tt = w0; tt < w1 && ok; ++tt) {
+          int crd = 0;  // this lane's copy: contiguous, first row; paged, first 8-row group
+          if (lane < ncp) {
+            const int tok = tt * T + lane * cp;
+            if (!a.paged) {
+              crd = s_start[pc.b] + tok;
+            } else {
+              const int pidx = tok >> a.page_shift;
+              const int page = (pidx < npages && pidx - pbase < 64) ? s_pages[pidx - pbase] : -1;
+              crd = (page * ps + (tok & (ps - 1))) >> 3;
             }
           }
-          if (!mbar_wait(kempty0 + 8 * ks, kph ^ 1u, kWaitLimitNs)) {
-            record_timeout(a.status, 1, kissued, ks, kph ^ 1u, kempty0 + 8 * ks);
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(kfull0 + 8 * ks, C::TILE_BYTES);
-          const uint32_t kd = kring + ks * C::TILE_BYTES;
-#pragma unroll
-          for (int j = 0; j < C::BOXES; ++j) {
-            if (j < ncp) {
-              const uint32_t dst = kd + j * (cp / 8) * C::GROUP_BYTES;
-              if (a.paged)
-                tma_load_5d(dst, &a.kmap, kfull0 + 8 * ks, 0, 0, 0, pc.h, crd[j], pol);
-              else
-                tma_load_4d(dst, &a.kmap, kfull0 + 8 * ks, 0, crd[j], 0, pc.h, pol);
+          const uint32_t dst_off = static_cast<uint32_t>(lane * (cp / 8) * C::GROUP_BYTES);
+          if (lane == 0) {
+            if (!mbar_wait(kempty0 + 8 * ks, kph ^ 1u, kWaitLimitNs)) {
+              record_timeout(a.status, 1, kissued, ks, kph ^ 1u, kempty0 + 8 * ks);
+              ok = false;
+            } else {
+              mbar_arrive_expect_tx(kfull0 + 8 * ks, C::TILE_BYTES);
             }
+          }
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+          if (lane < ncp) {
+            const uint32_t dst = kring + ks * C::TILE_BYTES + dst_off;
+            if (a.paged)
+              tma_load_5d(dst, &a.kmap, kfull0 + 8 * ks, 0, 0, 0, pc.h, crd, pol);
+            else
+              tma_load_4d(dst, &a.kmap, kfull0 + 8 * ks, 0, crd, 0, pc.h, pol);
           }
           ++kissued;
-          if (!mbar_wait(vempty0 + 8 * vs, vph ^ 1u, kWaitLimitNs)) {
-            record_timeout(a.status, 8, vissued, vs, vph ^ 1u, vempty0 + 8 * vs);
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(vfull0 + 8 * vs, C::TILE_BYTES);
-          const uint32_t vd = vring + vs * C::TILE_BYTES;
-#pragma unroll
-          for (int j = 0; j < C::BOXES; ++j) {
-            if (j < ncp) {
-              const uint32_t dst = vd + j * (cp / 8) * C::GROUP_BYTES;
-              if (a.paged)
-                tma_load_5d(dst, &a.vmap, vfull0 + 8 * vs, 0, 0, 0, pc.h, crd[j], pol);
-              else
-                tma_load_4d(dst, &a.vmap, vfull0 + 8 * vs, 0, crd[j], 0, pc.h, pol);
+          if (lane == 0) {
+            if (!mbar_wait(vempty0 + 8 * vs, vph ^ 1u, kWaitLimitNs)) {
+              record_timeout(a.status, 8, vissued, vs, vph ^ 1u, vempty0 + 8 * vs);
+              ok = false;
+            } else {
+              mbar_arrive_expect_tx(vfull0 + 8 * vs, C::TILE_BYTES);
             }
+          }
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+          if (lane < ncp) {
+            const uint32_t dst = vring + vs * C::TILE_BYTES + dst_off;
+            if (a.paged)
+              tma_load_5d(dst, &a.vmap, vfull0 + 8 * vs, 0, 0, 0, pc.h, crd, pol);
+            else
+              tma_load_4d(dst, &a.vmap, vfull0 + 8 * vs, 0, crd, 0, pc.h, pol);
           }
           ++vissued;
           if (++ks == KS) {
@@ -462,18 +465,26 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
       tc::commit(done_bar);
       if (!mbar_wait(done_bar, 0, kWaitLimitNs)) record_timeout(a.status, 17, i, 0, 0, done_bar);
     }
-    named_barrier_sync(2, 160);
+    named_barrier_sync(2, 32 + 32 * C::SG_WARPS);
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, C::TMEM_COLS);
     return;
   }
 
-  // ================= softmax group (warps 2..5)
+  // ================= softmax group (warps 2..9)
+  // Two row halves of 4 warps each: the warps of a half cover the four TMEM
+  // lane quarters (a warp reads the lanes of quarter warp % 4), so thread
+  // (half, tok) handles token tok of a tile for rows [r0, r0 + NH), and
+  // dimension tok of the output for the same rows.
+  constexpr int NH = N / 2;
+  constexpr int SGT = 32 * C::SG_WARPS;       // softmax-group threads
   const int quarter = warp & 3;              // this warp's quarter of TMEM lanes
   const int tok = quarter * 32 + lane;       // token of a tile; dim of an output row
+  const int half = (warp - 2) >> 2;          // 0 or 1
+  const int r0 = half * NH;                  // first row of this half
   const uint32_t lanes = static_cast<uint32_t>(quarter * 32) << 16;
-  const int sw = warp - 2;                   // 0..3
-  write_empty_results(a, it, s_len, G, D, c, P, tid - 64, 128);
+  float* red = s_red + half * 4 * NH;        // this half's [quarter][NH] scratch
+  write_empty_results(a, it, s_len, G, D, c, P, tid - 64, SGT);
   // parameters in registers for the tile loop
   const float sscale = a.score_scale, cap = a.cap_l2;
   const int W = a.window, WU = a.window_u;
@@ -482,7 +493,7 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
   // always passes the slack test (which rescales by exp2(-1e30 - x) = 0)
   constexpr float kMStart = -1e30f;
 
-  float acc[N], l[N], m[N];
+  float acc[NH], l[NH], m[NH];
   bool alive = true;     // this warp's waits have all succeeded
   int i = 0;             // tile of the block's sequence
   int pending = -1;      // tile whose output product is not yet accumulated
@@ -490,10 +501,10 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
   PieceIter its = it;
   Piece pc;
 
-  // Accumulates O^T of tile j (this thread's dimension, every row).  A
+  // Accumulates O^T of tile j (this thread's dimension, its rows).  A
   // failed wait only stops this warp's work: the group agrees to stop at its
   // next barrier (bar_any on !alive), so every named barrier below is
-  // reached by all 128 threads or by none.
+  // reached by all the group's threads or by none.
   auto take_o = [&](int j) {
     if (!alive) return;
     const bool ok = mbar_wait(ofull0 + 8 * (j & 1), (j >> 1) & 1, kWaitLimitNs);
@@ -502,19 +513,19 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
       alive = false;
       return;
     }
-    float o[N];
-    tc::ld_32x32b<N>(tO + lanes + (j & 1) * N, o);
+    float o[NH];
+    tc::ld_32x32b<NH>(tO + lanes + (j & 1) * N + r0, o);
     tc::wait_ld();
     tc::fence_before_sync();
     __syncwarp();
     if (lane == 0) mbar_arrive(ofree0 + 8 * (j & 1));
     if (resc & (1u << (j & 1))) {
-      const float* al = s_alpha + (j & 1) * N;
+      const float* al = s_alpha + (j & 1) * N + r0;
 #pragma unroll
-      for (int r = 0; r < N; ++r) acc[r] = fmaf(acc[r], al[r], o[r]);
+      for (int r = 0; r < NH; ++r) acc[r] = fmaf(acc[r], al[r], o[r]);
     } else {
 #pragma unroll
-      for (int r = 0; r < N; ++r) acc[r] += o[r];
+      for (int r = 0; r < NH; ++r) acc[r] += o[r];
     }
   };
   // A bounded wait of the whole warp: false (and the wait recorded) if any
@@ -530,7 +541,7 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
     const int L = s_len[pc.b];
     const int lo = (WU > 0 && L > WU) ? L - WU : 0;  // keys some row sees: [lo, L)
 #pragma unroll
-    for (int r = 0; r < N; ++r) {
+    for (int r = 0; r < NH; ++r) {
       acc[r] = 0.f;
       l[r] = 0.f;
       m[r] = kMStart;
@@ -538,15 +549,15 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
     const int n = pc.t1 - pc.t0;
     for (int t = 0; t < n; ++t, ++i) {
       __syncwarp();
-      if (bar_any(1, 128, !alive)) {  // the group stops together
+      if (bar_any(1, SGT, !alive)) {  // the group stops together
         stop = true;
         break;
       }
       const int pos0 = (pc.t0 + t) * T;
       const int pos = pos0 + tok;
-      float x[N];
+      float x[NH];
       if (warp_wait(sfull0 + 8 * (i & 1), (i >> 1) & 1, 19, i, i & 1)) {
-        tc::ld_32x32b<N>(tS + lanes + (i & 1) * N, x);
+        tc::ld_32x32b<NH>(tS + lanes + (i & 1) * N + r0, x);
         tc::wait_ld();
         tc::fence_before_sync();
         __syncwarp();
@@ -554,59 +565,59 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
       } else {
         alive = false;
 #pragma unroll
-        for (int r = 0; r < N; ++r) x[r] = 0.f;
+        for (int r = 0; r < NH; ++r) x[r] = 0.f;
       }
       // The rows that see this thread's key: query token q (rows q GK ..
       // q GK + GK - 1) sees keys below L - Q + 1 + q and, with a window, from
-      // L - Q + 1 + q - W on, so the rows form one range [rlo, rhi).
+      // L - Q + 1 + q - W on, so the rows form one range [rlo, rlo + rspan).
       const int base = pos - L + Q;
       const int qlo = base > 0 ? base : 0;
       const int qhi = W > 0 ? (base + W < Q ? base + W : Q) : Q;
-      const int rlo = qlo * GK;
+      const int rlo = qlo * GK - r0;  // relative to this half's first row
       const uint32_t rspan = qhi > qlo ? static_cast<uint32_t>((qhi - qlo) * GK) : 0u;
       // scale (log2 units), soft-cap, then the masks
 #pragma unroll
-      for (int r = 0; r < N; ++r) x[r] *= sscale;
+      for (int r = 0; r < NH; ++r) x[r] *= sscale;
       if (cap > 0.f) {
 #pragma unroll
-        for (int r = 0; r < N; ++r) x[r] = cap * tanhf(x[r] / cap);
+        for (int r = 0; r < NH; ++r) x[r] = cap * tanhf(x[r] / cap);
       }
       bool need = false;
 #pragma unroll
-      for (int r = 0; r < N; ++r) {
+      for (int r = 0; r < NH; ++r) {
         x[r] = static_cast<uint32_t>(r - rlo) < rspan ? x[r] : -CUDART_INF_F;
         need |= x[r] - m[r] > kRescaleSlack;
       }
       __syncwarp();
-      const bool slow = bar_any(1, 128, need);
+      const bool slow = bar_any(1, SGT, need);
       resc &= ~(1u << (i & 1));
       if (slow) {
-        // the tile's maximum of every row over the 128 tokens
-        float v[N];
+        // the tile's maximum of each of this half's rows over the 128 tokens
+        float v[NH];
 #pragma unroll
-        for (int r = 0; r < N; ++r) v[r] = x[r];
-        const float wmax = warp_rows_reduce<N, true>(v, lane);
-        if (lane < N) s_red[sw * N + lane] = wmax;
-        named_barrier_sync(1, 128);
+        for (int r = 0; r < NH; ++r) v[r] = x[r];
+        const float wmax = warp_rows_reduce<NH, true>(v, lane);
+        if (lane < NH) red[quarter * NH + lane] = wmax;
+        named_barrier_sync(1, SGT);
 #pragma unroll
-        for (int r = 0; r < N; ++r) {
-          const float tm = fmaxf(fmaxf(s_red[r], s_red[N + r]), fmaxf(s_red[2 * N + r], s_red[3 * N + r]));
+        for (int r = 0; r < NH; ++r) {
+          const float tm = fmaxf(fmaxf(red[r], red[NH + r]), fmaxf(red[2 * NH + r], red[3 * NH + r]));
           float al = 1.f;
           if (tm - m[r] > kRescaleSlack) {
             al = exp2_approx(m[r] - tm);  // from the start value: 0
             m[r] = tm;
           }
           l[r] *= al;
-          if (tok == r) s_alpha[(i & 1) * N + r] = al;
+          if (tok == r) s_alpha[(i & 1) * N + r0 + r] = al;
         }
         resc |= 1u << (i & 1);
-        named_barrier_sync(1, 128);  // s_alpha written; s_red read by all
+        named_barrier_sync(1, SGT);  // s_alpha written; the scratch read by all
       }
       // P = exp2(x - m) (0 for a masked key), its row sums, and the bf16
       // hi / lo parts
-      uint32_t ph[N / 2], pl[N / 2];
+      uint32_t ph[NH / 2], pl[NH / 2];
 #pragma unroll
-      for (int r = 0; r < N; r += 2) {
+      for (int r = 0; r < NH; r += 2) {
         const float p0 = exp2_approx(x[r] - m[r]);
         const float p1 = exp2_approx(x[r + 1] - m[r + 1]);
         l[r] += p0;
@@ -617,8 +628,9 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
       }
       if (!alive) continue;
       // V rows of keys outside [lo, L) may hold anything (NaN included) and
-      // meet P = 0 in the product: zero them once the tile has landed
-      if (pos0 < lo || pos0 + T > L) {
+      // meet P = 0 in the product: zeroed once the tile has landed (by the
+      // first half; every half's P arrival precedes the product)
+      if (half == 0 && (pos0 < lo || pos0 + T > L)) {
         const bool out = pos < lo || pos >= L;
         if (__any_sync(0xffffffffu, out)) {
           const int vsl = i % VS;
@@ -637,15 +649,16 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
       }
       // P^T of tile i into buffer i % 2 (free: the output product of tile
       // i - 2 was waited for when its O was read), N rows of a token
-      // contiguous (2N bytes), 16-byte chunks swizzled by the address bits
-      // above them (64- or 32-byte swizzle)
+      // contiguous (2N bytes), 16-byte chunks of 8 rows swizzled by the
+      // address bits above them (64- or 32-byte swizzle); this half writes
+      // its chunks
       {
-        constexpr int CH = N / 8;  // 16-byte chunks a token
+        constexpr int CH = NH / 8;  // 16-byte chunks of this half's rows
         const int sel = N == 32 ? ((tok >> 1) & 3) : ((tok >> 2) & 1);
         const uint32_t hi_buf = p_buf + (i & 1) * 2 * C::P_BYTES;
 #pragma unroll
         for (int ch = 0; ch < CH; ++ch) {
-          const uint32_t off = tok * (2 * N) + ((ch ^ sel) * 16);
+          const uint32_t off = tok * (2 * N) + (((half * CH + ch) ^ sel) * 16);
           sts128(hi_buf + off, make_uint4(ph[4 * ch], ph[4 * ch + 1], ph[4 * ch + 2], ph[4 * ch + 3]));
           sts128(hi_buf + C::P_BYTES + off,
                  make_uint4(pl[4 * ch], pl[4 * ch + 1], pl[4 * ch + 2], pl[4 * ch + 3]));
@@ -662,44 +675,45 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
     if (pending >= 0) take_o(pending);
     pending = -1;
     __syncwarp();
-    if (bar_any(1, 128, !alive)) break;  // also: every reader of s_red is done
-    float lsum[N];
+    if (bar_any(1, SGT, !alive)) break;  // also: every reader of the scratch is done
+    float lsum[NH];
     {
-      float v[N];
+      float v[NH];
 #pragma unroll
-      for (int r = 0; r < N; ++r) v[r] = l[r];
-      const float wsum = warp_rows_reduce<N, false>(v, lane);
-      if (lane < N) s_red[sw * N + lane] = wsum;
-      named_barrier_sync(1, 128);
+      for (int r = 0; r < NH; ++r) v[r] = l[r];
+      const float wsum = warp_rows_reduce<NH, false>(v, lane);
+      if (lane < NH) red[quarter * NH + lane] = wsum;
+      named_barrier_sync(1, SGT);
 #pragma unroll
-      for (int r = 0; r < N; ++r) lsum[r] = (s_red[r] + s_red[N + r]) + (s_red[2 * N + r] + s_red[3 * N + r]);
+      for (int r = 0; r < NH; ++r) lsum[r] = (red[r] + red[NH + r]) + (red[2 * NH + r] + red[3 * NH + r]);
     }
     const bool whole = pc.n_pieces == 1;
     const int slot_idx = c + pc.seg;
 #pragma unroll
-    for (int r = 0; r < N; ++r) {
-      if (r >= G) break;
+    for (int r = 0; r < NH; ++r) {
+      const int rr = r0 + r;  // segment row
+      if (rr >= G) break;
       const bool empty = !(lsum[r] > 0.f);
       const float val = empty ? 0.f : acc[r] / lsum[r];
-      const size_t row = (static_cast<size_t>(pc.b) * Q + r / GK) * a.qo_heads +
-                         static_cast<size_t>(pc.h) * GK + r % GK;
+      const size_t row = (static_cast<size_t>(pc.b) * Q + rr / GK) * a.qo_heads +
+                         static_cast<size_t>(pc.h) * GK + rr % GK;
       if (whole) {
         a.out[row * D + tok] = bf16_bits(val);
       } else if (FA_CHECK(a.status, slot_idx < a.max_partials, 402, slot_idx)) {
-        a.part_o[(static_cast<size_t>(slot_idx) * G + r) * D + tok] = val;
+        a.part_o[(static_cast<size_t>(slot_idx) * G + rr) * D + tok] = val;
       }
       if (tok == r) {
         const float lv = empty ? -CUDART_INF_F : (m[r] + __log2f(lsum[r])) * kLn2;
         if (whole) {
           if (a.lse != nullptr) a.lse[row] = lv;
         } else if (slot_idx < a.max_partials) {
-          a.part_lse[static_cast<size_t>(slot_idx) * G + r] = lv;
+          a.part_lse[static_cast<size_t>(slot_idx) * G + rr] = lv;
         }
       }
     }
   }
   tc::fence_before_sync();
-  named_barrier_sync(2, 160);
+  named_barrier_sync(2, 32 + SGT);
 }
 
 }  // namespace fa
