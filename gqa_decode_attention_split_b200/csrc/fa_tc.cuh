@@ -51,12 +51,16 @@ struct TcCfg {
   static constexpr int GROUP_BYTES = BOX_T * ROWB;  // one copy: [NP][8][128]
   static constexpr int BOXES = T / BOX_T;
   static constexpr int TILE_BYTES = T * ROWB;
-  static constexpr int KSTAGES = 3;
-  static constexpr int VSTAGES = NR <= 16 ? 3 : 2;
+  // V slots are held until the output product (after the softmax of the
+  // tile), K slots only until the score product: 32 rows keep 2 K slots to
+  // afford a third V slot
+  static constexpr int KSTAGES = NR <= 16 ? 3 : 2;
+  static constexpr int VSTAGES = 3;
   static constexpr int QSLOT_BYTES = NP * N * 128;  // [NP][N rows][128]
   static constexpr int P_BYTES = T * N * 2;         // P hi (or lo) of a tile: [T][N] bf16
   static constexpr int SG_WARPS = 8;   // softmax group: two row halves x 4 TMEM lane quarters
-  static constexpr int THREADS = 64 + 32 * SG_WARPS;
+  static constexpr int PV_WARP = 2 + SG_WARPS;  // issues the output products
+  static constexpr int THREADS = 32 * (PV_WARP + 1);
   static constexpr uint32_t TMEM_COLS = 128;        // S[2] and O[2], N columns each
   static constexpr uint32_t P_LAYOUT = N == 32 ? tc::kSwizzle64 : tc::kSwizzle32;
   // shared memory, from a 1024-aligned base
@@ -65,7 +69,7 @@ struct TcCfg {
   static constexpr int OFF_Q = OFF_V + VSTAGES * TILE_BYTES;
   static constexpr int OFF_P = OFF_Q + 2 * QSLOT_BYTES;
   static constexpr int OFF_BAR = OFF_P + 4 * P_BYTES;  // P[2], hi + lo each
-  static constexpr int NBARS = 2 * KSTAGES + 2 * VSTAGES + 15;
+  static constexpr int NBARS = 2 * KSTAGES + 2 * VSTAGES + 16;
   static constexpr int OFF_TMEM = OFF_BAR + 8 * NBARS;
   static constexpr int OFF_RED = OFF_TMEM + 16;    // [4][N] floats
   static constexpr int OFF_ALPHA = OFF_RED + 4 * N * 4;  // [2][N] floats
@@ -120,7 +124,7 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
   const uint32_t qfull0 = vempty0 + 8 * VS, qempty0 = qfull0 + 16;
   const uint32_t sfull0 = qempty0 + 16, sfree0 = sfull0 + 16;
   const uint32_t pfull0 = sfree0 + 16, ofull0 = pfull0 + 16, ofree0 = ofull0 + 16;
-  const uint32_t done_bar = ofree0 + 16;
+  const uint32_t done_bar = ofree0 + 16, done_o = done_bar + 8;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base + C::OFF_TMEM);
   float* s_red = reinterpret_cast<float*>(base + C::OFF_RED);
   float* s_alpha = reinterpret_cast<float*>(base + C::OFF_ALPHA);
@@ -163,6 +167,7 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
       mbar_init(pfull0 + 8 * s, C::SG_WARPS);
     }
     mbar_init(done_bar, 1);
+    mbar_init(done_o, 1);
     fence_mbar_init();
   }
   tc::fence_before_sync();
@@ -375,47 +380,64 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
   constexpr uint32_t kIdescO = tc::idesc_bf16(128, N, true, true);
   const uint32_t tS = tmem, tO = tmem + 2 * N;  // column offsets of S[2] and O[2]
 
-  if (warp == 1) {
-    // ================= tcgen05.mma issue (one lane)
-    if (lane == 0) {
+  if (warp == 1 || warp == C::PV_WARP) {
+    // ================= tcgen05.mma issue: lane 0 of warp 1 the score
+    // products, lane 0 of PV_WARP the output products, so that a tile's
+    // output product (and the release of its V slot) never waits behind the
+    // next tile's K copy
+    if (lane == 0 && warp == C::PV_WARP) {
       bool ok = true;
-      int i = 0, prev = -1, pcount = 0;
-      // output product of tile j: O^T[j % 2] = V_j^T . (P_hi + P_lo)^T
-      auto product_o = [&](int j) {
-        const int vsl = j % VS;
-        if (ok && !mbar_wait(vfull0 + 8 * vsl, (j / VS) & 1, kWaitLimitNs)) {
-          record_timeout(a.status, 11, j, vsl, (j / VS) & 1, vfull0 + 8 * vsl);
-          ok = false;
-        }
-        if (ok && !mbar_wait(pfull0 + 8 * (j & 1), (j >> 1) & 1, kWaitLimitNs)) {
-          record_timeout(a.status, 12, j, j & 1, (j >> 1) & 1, pfull0 + 8 * (j & 1));
-          ok = false;
-        }
-        if (ok && j >= 2 && !mbar_wait(ofree0 + 8 * (j & 1), ((j - 2) >> 1) & 1, kWaitLimitNs)) {
-          record_timeout(a.status, 13, j, j & 1, ((j - 2) >> 1) & 1, ofree0 + 8 * (j & 1));
-          ok = false;
-        }
-        if (!ok) return;
-        tc::fence_after_sync();
-        const uint32_t vt = vring + vsl * C::TILE_BYTES;
-        const uint32_t d = tO + (j & 1) * N;
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          const uint32_t pb = p_buf + (j & 1) * 2 * C::P_BYTES + part * C::P_BYTES;
-#pragma unroll
-          for (int k = 0; k < T / 16; ++k) {
-            // V^T: dims as M (64-dim atoms one plane = 1024 bytes apart),
-            // tokens as K (8-token groups GROUP_BYTES apart); P^T: rows as N
-            // (2N bytes a token), tokens as K (8-token groups 16 N apart)
-            const uint64_t ad = tc::smem_desc(vt + k * 2 * C::GROUP_BYTES, 1024, C::GROUP_BYTES,
-                                              tc::kSwizzle128);
-            const uint64_t bd = tc::smem_desc(pb + k * 16 * 2 * N, T * 2 * N, 8 * 2 * N, C::P_LAYOUT);
-            tc::mma_bf16_ss(d, ad, bd, kIdescO, part > 0 || k > 0);
+      PieceIter itv = it;
+      Piece pc;
+      int j = 0;
+      while (ok && next_piece(itv, pc, s_pre, s_len, B, H, a.window_u, T)) {
+        const int n = pc.t1 - pc.t0;
+        for (int t = 0; t < n && ok; ++t, ++j) {
+          // output product of tile j: O^T[j % 2] = V_j^T . (P_hi + P_lo)^T
+          const int vsl = j % VS;
+          if (!mbar_wait(vfull0 + 8 * vsl, (j / VS) & 1, kWaitLimitNs)) {
+            record_timeout(a.status, 11, j, vsl, (j / VS) & 1, vfull0 + 8 * vsl);
+            ok = false;
+            break;
           }
+          if (!mbar_wait(pfull0 + 8 * (j & 1), (j >> 1) & 1, kWaitLimitNs)) {
+            record_timeout(a.status, 12, j, j & 1, (j >> 1) & 1, pfull0 + 8 * (j & 1));
+            ok = false;
+            break;
+          }
+          if (j >= 2 && !mbar_wait(ofree0 + 8 * (j & 1), ((j - 2) >> 1) & 1, kWaitLimitNs)) {
+            record_timeout(a.status, 13, j, j & 1, ((j - 2) >> 1) & 1, ofree0 + 8 * (j & 1));
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t vt = vring + vsl * C::TILE_BYTES;
+          const uint32_t d = tO + (j & 1) * N;
+#pragma unroll
+          for (int part = 0; part < 2; ++part) {
+            const uint32_t pb = p_buf + (j & 1) * 2 * C::P_BYTES + part * C::P_BYTES;
+#pragma unroll
+            for (int k = 0; k < T / 16; ++k) {
+              // V^T: dims as M (64-dim atoms one plane = 1024 bytes apart),
+              // tokens as K (8-token groups GROUP_BYTES apart); P^T: rows as N
+              // (2N bytes a token), tokens as K (8-token groups 16 N apart)
+              const uint64_t ad = tc::smem_desc(vt + k * 2 * C::GROUP_BYTES, 1024, C::GROUP_BYTES,
+                                                tc::kSwizzle128);
+              const uint64_t bd = tc::smem_desc(pb + k * 16 * 2 * N, T * 2 * N, 8 * 2 * N, C::P_LAYOUT);
+              tc::mma_bf16_ss(d, ad, bd, kIdescO, part > 0 || k > 0);
+            }
+          }
+          tc::commit(ofull0 + 8 * (j & 1));
+          tc::commit(vempty0 + 8 * vsl);
         }
-        tc::commit(ofull0 + 8 * (j & 1));
-        tc::commit(vempty0 + 8 * vsl);
-      };
+      }
+      // every product issued has completed before tensor memory is freed
+      tc::commit(done_o);
+      if (!mbar_wait(done_o, 0, kWaitLimitNs)) record_timeout(a.status, 17, j, 1, 0, done_o);
+    }
+    if (lane == 0 && warp == 1) {
+      bool ok = true;
+      int i = 0, pcount = 0;
       PieceIter itm = it;
       Piece pc;
       while (ok && next_piece(itm, pc, s_pre, s_len, B, H, a.window_u, T)) {
@@ -455,19 +477,18 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
           tc::commit(sfull0 + 8 * (i & 1));
           tc::commit(kempty0 + 8 * ksl);
           if (t == n - 1) tc::commit(qempty0 + 8 * qs);
-          if (prev >= 0) product_o(prev);
-          prev = i;
         }
         ++pcount;
       }
-      if (prev >= 0) product_o(prev);
       // every product issued has completed before tensor memory is freed
       tc::commit(done_bar);
       if (!mbar_wait(done_bar, 0, kWaitLimitNs)) record_timeout(a.status, 17, i, 0, 0, done_bar);
     }
-    named_barrier_sync(2, 32 + 32 * C::SG_WARPS);
-    tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, C::TMEM_COLS);
+    named_barrier_sync(2, 64 + 32 * C::SG_WARPS);
+    if (warp == 1) {
+      tc::fence_after_sync();
+      tc::tmem_dealloc(tmem, C::TMEM_COLS);
+    }
     return;
   }
 
@@ -713,7 +734,7 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
     }
   }
   tc::fence_before_sync();
-  named_barrier_sync(2, 32 + SGT);
+  named_barrier_sync(2, 64 + SGT);
 }
 
 }  // namespace fa
