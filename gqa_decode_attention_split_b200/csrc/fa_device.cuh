@@ -233,6 +233,13 @@ __device__ __forceinline__ float exp2_approx(float x) {
   return y;
 }
 
+// 1/x with the hardware approximation (relative error below 2^-22).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Barrier over `nthreads` threads (a multiple of 32) of the block.  The
 // non-aligned form is used, and the warp is reconverged first, because
 // callers reach it after per-lane branches (the .aligned form, which

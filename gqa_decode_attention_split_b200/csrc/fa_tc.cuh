@@ -710,27 +710,47 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
     }
     const bool whole = pc.n_pieces == 1;
     const int slot_idx = c + pc.seg;
+    // O = acc / l and the row's lse (natural log).  Straight-line code with
+    // one pointer stepped row by row: this runs once per piece, so its
+    // instructions are cold, and each cache line of them fetched while the
+    // copies saturate memory stalls the whole group.
+    float val[NH];
+    float my_lse = -CUDART_INF_F;  // row r0 + tok (tok < NH)
 #pragma unroll
     for (int r = 0; r < NH; ++r) {
-      const int rr = r0 + r;  // segment row
-      if (rr >= G) break;
       const bool empty = !(lsum[r] > 0.f);
-      const float val = empty ? 0.f : acc[r] / lsum[r];
-      const size_t row = (static_cast<size_t>(pc.b) * Q + rr / GK) * a.qo_heads +
-                         static_cast<size_t>(pc.h) * GK + rr % GK;
-      if (whole) {
-        a.out[row * D + tok] = bf16_bits(val);
-      } else if (FA_CHECK(a.status, slot_idx < a.max_partials, 402, slot_idx)) {
-        a.part_o[(static_cast<size_t>(slot_idx) * G + rr) * D + tok] = val;
-      }
-      if (tok == r) {
-        const float lv = empty ? -CUDART_INF_F : (m[r] + __log2f(lsum[r])) * kLn2;
-        if (whole) {
-          if (a.lse != nullptr) a.lse[row] = lv;
-        } else if (slot_idx < a.max_partials) {
-          a.part_lse[static_cast<size_t>(slot_idx) * G + rr] = lv;
+      val[r] = empty ? 0.f : acc[r] * rcp_approx(lsum[r]);
+      const float lv = empty ? -CUDART_INF_F : (m[r] + __log2f(lsum[r])) * kLn2;
+      my_lse = tok == r ? lv : my_lse;
+    }
+    const int nrows = G - r0 < NH ? G - r0 : NH;  // rows of this half that exist
+    if (whole) {
+      // segment row rr is query token rr / GK, head rr % GK of the group
+      int hd = r0 % GK;
+      const size_t row0 = (static_cast<size_t>(pc.b) * Q + r0 / GK) * a.qo_heads +
+                          static_cast<size_t>(pc.h) * GK + hd;
+      uint16_t* po = a.out + row0 * D + tok;
+      const int jump = (a.qo_heads - GK) * D;  // last head of a token -> first of the next
+#pragma unroll
+      for (int r = 0; r < NH; ++r) {
+        if (r < nrows) *po = bf16_bits(val[r]);
+        po += D;
+        if (++hd == GK) {
+          hd = 0;
+          po += jump;
         }
       }
+      if (tok < nrows && a.lse != nullptr) {
+        const int rr = r0 + tok;
+        a.lse[(static_cast<size_t>(pc.b) * Q + rr / GK) * a.qo_heads +
+              static_cast<size_t>(pc.h) * GK + rr % GK] = my_lse;
+      }
+    } else if (FA_CHECK(a.status, slot_idx < a.max_partials, 402, slot_idx)) {
+      float* po = a.part_o + (static_cast<size_t>(slot_idx) * G + r0) * D + tok;
+#pragma unroll
+      for (int r = 0; r < NH; ++r)
+        if (r < nrows) po[r * D] = val[r];
+      if (tok < nrows) a.part_lse[static_cast<size_t>(slot_idx) * G + r0 + tok] = my_lse;
     }
   }
   tc::fence_before_sync();
