@@ -70,8 +70,12 @@ def sweep_jobs(headline=HEADLINE):
     ("auto"), a forced dataflow ("simt", "mma") or the unified max at
     UNIFIED_PHI ("unified_max").  The parity tests run the same list."""
     jobs = [(name, "auto") for name in SWEEP]
-    jobs += [(headline, "simt"), (headline, "mma"), ("fp8_gqa8_L131072", "mma"),
+    jobs += [(headline, "simt"), (headline, "mma"),
+             ("fp8_gqa8_L131072", "simt"), ("fp8_gqa8_L131072", "mma"),
              ("llama2_7b_mha_L32768", "simt"), ("llama2_7b_mha_L32768", "mma"),
+             # 16 and 32 rows: the warp-level products beside the tcgen05 ones
+             ("paged_b64_gqa4_q4_L512-16384", "mma"), ("paged_b64_gqa4_q8_L512-16384", "mma"),
+             ("llama3_405b_tp8_gqa16_paged_b64_L512-16384", "mma"),
              (headline, "unified_max"), ("fp8_gqa8_L131072", "unified_max")]
     return jobs
 

@@ -8,7 +8,7 @@ import numpy as np
 import pytest
 
 from gqa_decode_attention_split_b200 import binding, synth
-from gpu_util import DeviceInputs, assert_matches, run_gpu, to_numpy
+from gpu_util import LSE_ABS, DeviceInputs, assert_matches, run_gpu, to_numpy
 from oracle import oracle
 
 pytestmark = pytest.mark.gpu
@@ -463,10 +463,11 @@ def test_logit_softcap(case, path):
     if not _has_path(x, path):
         pytest.skip("no kernel for these rows on this path")
     out, lse, _ = _check(x, path=path)
-    # the cap must matter here: the uncapped result is different
+    # the cap must matter here: the uncapped lse differs by far more than
+    # the lse tolerance (the small-cap cases move it by about 0.1)
     plain = synth.DecodeInputs(**{**x.__dict__, "logit_cap": 0.0})
     po, pl = oracle.decode_all(plain)
-    assert np.abs(pl - lse).max() > 0.1
+    assert np.abs(pl - lse).max() > 20 * LSE_ABS
 
 
 def test_logit_softcap_forced_splits():
