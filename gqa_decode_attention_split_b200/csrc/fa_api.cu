@@ -267,7 +267,7 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   // else the fixed rule: the tensor-core (MMA) path whenever a kernel exists
   // for the shape, the SIMT path otherwise.
   const KernelEntry* k = nullptr;
-  int64_t max_pieces = 32;  // average blocks per segment, at most
+  int64_t max_pieces = 64;  // average blocks per segment, at most
   bool table_cap = false;   // max_pieces came from the measured table
   // the tcgen05 dataflow: bf16 K/V, head_dim 128, 9 to 32 rows, copies of
   // 8 tokens (pages of at least 8), the plain running max
@@ -358,12 +358,19 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
     // One block per SM (each holds a ~170 KB tile ring).  A problem with
     // fewer tiles than SMs gets one tile per block (the fixed cost of a
     // block is small next to a KV tile's load latency, and the tiles load in
-    // parallel); a segment is cut into at most max_pieces runs on
-    // average so that the last block's merge of the partial states stays
-    // short (32 unless the measured table says otherwise).
+    // parallel); a segment is cut into at most max_pieces runs on average,
+    // so that merging its partial states stays short (64 unless the
+    // measured table says otherwise), except where the K/V give every SM at
+    // least 256 KB: then the streaming outweighs the merge.  Measured on B200
+    // (one segment, device time per pass, 32 / 64 / 148 blocks): 8.4 MB
+    // 21.5 / 19.5 / 21.5 us, 16.8 MB 23.5 / 19.5 / 21.5 us, 67 MB
+    // 44.1 / 31.7 / 29.7 us; passes of 4 or more segments reach all SMs
+    // either way.
     int64_t want = tiles;
     const int64_t seg_cap = max_pieces * desc->batch * desc->kv_heads;  // per kv head
-    if (want > seg_cap) want = seg_cap;
+    const bool wide = !table_cap && visible_kv_bytes(desc, kv_indptr_host) >=
+                                        static_cast<int64_t>(num_sms) * (256 << 10);
+    if (want > seg_cap && !wide) want = seg_cap;
     P = want < num_sms ? want : num_sms;
     if (P < 1) P = 1;
     // Segments of equal length and rows of at most 128 bytes: cut every

@@ -35,7 +35,7 @@ from gqa_decode_attention_split_b200 import binding  # noqa: E402
 
 MARGIN = 0.03                    # an alternative must be this much faster,
 MARGIN_US = 1.0                  # and by at least this many microseconds
-PIECES = (0, 8, 2)               # 0: the planner's default (32)
+PIECES = (0, 8, 2)               # 0: the planner's default (64)
 BYTES = [1 << 18, 1 << 21, 1 << 24, 1 << 27, 1 << 30]
 SHAPES = [(64, "bf16"), (128, "bf16"), (256, "bf16"), (128, "fp8_e4m3"), (256, "fp8_e4m3")]
 KV_HEADS = 8
@@ -189,9 +189,9 @@ def main():
                 base = configs.get((binding.PATH_MMA, 0)) or configs[(binding.PATH_SIMT, 0)]
                 rec = {"head_dim": d, "kv_dtype": dtype, "rows": r, "bytes": x[6] * KV_HEADS * 2 * d *
                        (1 if dtype == "fp8_e4m3" else 2), "configs": {
-                           f"{'mma' if p == binding.PATH_MMA else 'simt'}/pieces={k or 32}": v
+                           f"{'mma' if p == binding.PATH_MMA else 'simt'}/pieces={k or 64}": v
                            for (p, k), v in configs.items()},
-                       "choice": f"{'mma' if ch[0] == binding.PATH_MMA else 'simt'}/pieces={ch[1] or 32}",
+                       "choice": f"{'mma' if ch[0] == binding.PATH_MMA else 'simt'}/pieces={ch[1] or 64}",
                        "speedup_vs_fixed_rule": round(base["us"] / configs[ch]["us"], 3)}
                 record.append(rec)
                 print(json.dumps(rec), flush=True)
