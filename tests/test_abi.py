@@ -93,6 +93,32 @@ def test_plans_for_named_workloads(lib, name):
     lib.fa_plan_destroy(h)
 
 
+@pytest.mark.parametrize("L,d,ctas", [
+    (8192, 256, 64),      # 8.4 MB in one segment: 64 runs (the per-segment cap)
+    (16384, 128, 64),     # 8.4 MB: capped at 64 as well
+    (131072, 128, 148),   # 67 MB: every SM gets over 256 KB, so all take part
+    (1024, 128, 64),      # 0.5 MB: fewer tiles than the cap, one per block
+])
+def test_blocks_per_segment(lib, L, d, ctas):
+    """One segment is cut into at most 64 runs (its merge stays short) unless
+    its K/V give every SM at least 256 KB; a measured-table cap overrides."""
+    st, h, _ = _plan(lib, _desc(qo_heads=4, kv_heads=1, head_dim=d), [0, L])
+    assert st == 0
+    inf = _info(lib, h)
+    assert inf.path == binding.PATH_MMA
+    tiles = inf.total_tiles
+    assert inf.num_ctas == min(ctas, tiles), (inf.num_ctas, tiles)
+    lib.fa_plan_destroy(h)
+    try:
+        binding.set_tuning([_row(head_dim=d, rows_min=4, rows_max=4, bytes_max=1 << 40,
+                                 path=binding.PATH_MMA, max_pieces=8)])
+        st, h, _ = _plan(lib, _desc(qo_heads=4, kv_heads=1, head_dim=d), [0, L])
+        assert st == 0 and _info(lib, h).num_ctas == min(8, tiles)
+        lib.fa_plan_destroy(h)
+    finally:
+        binding.set_tuning(None)
+
+
 def test_plan_paged_and_fp8(lib):
     lens = synth.c4_lengths()
     ind = np.concatenate([[0], np.cumsum(lens)])
