@@ -20,15 +20,18 @@
 //           landing as [8-token group][plane][8][128 bytes], 128-byte
 //           swizzle: one copy per page of a paged pool, 16 copies of 8 rows
 //           of contiguous K/V) and of each piece's query rows;
-//   warp 1  allocates tensor memory; one lane issues every tcgen05.mma and
-//           commits its completion to mbarriers;
+//   warp 1  allocates tensor memory; one lane issues every score product
+//           and commits its completion to mbarriers;
 //   warps 2-9  the softmax group: two row halves of four warps, each half
 //           covering the four TMEM lane quarters.  Thread (half, t) reads
 //           token t's scores of its half of the rows from TMEM, keeps their
 //           running max (uniform over the group, rescaled only past an 8
 //           log2-unit slack), writes its part of P to shared memory, and
 //           reads back dimension t of each tile's O^T for the same rows,
-//           accumulating it in fp32 registers.
+//           accumulating it in fp32 registers;
+//   warp 10 one lane issues every output product (so that a tile's output
+//           product, and the release of its V slot, never waits behind the
+//           next tile's K copy).
 // The scores of tile i + 1 are computed while the softmax group works on tile
 // i; the output product of tile i runs while the scores of tile i + 1 are
 // read.  Every wait is bounded (2 s, then the block records the wait and
