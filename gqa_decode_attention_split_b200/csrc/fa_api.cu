@@ -420,12 +420,15 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   // states); a sweep of the charge then measured the best values: 2 tiles
   // up to 8 rows (batch-64 paged, 1%; MHA 32k, 2%), 8 with 16 or 32 rows
   // (batch-16 paged with 4 query tokens, 22%; GQA-16, 8%), 4 for int4
-  // head tiles (5%).  Only equal runs of several tiles per block are cut
+  // head tiles (5%), 3 of the 128-token tiles of the tcgen05 dataflow (a
+  // device timeline put a piece boundary near 3.5 us against 1.25 us a
+  // tile; against 2 tiles, 32 rows 392.2 -> 390.0 us, GQA-16 60.3 -> 59.7
+  // us back to back).  Only equal runs of several tiles per block are cut
   // by cost.
   p->piece_cost = 0;
   if (seg_parts == 0 && P > 1 && tiles > P && desc->piece_cost >= 0)
     p->piece_cost = desc->piece_cost > 0 ? desc->piece_cost
-                    : k->path == fa::kPathTc ? 2
+                    : k->path == fa::kPathTc ? 3
                     : (ht > 1 ? 4 : seg_rows <= 8 ? 2 : 8);
   p->total_tiles = tiles;
   const int segs = desc->batch * static_cast<int>(seg_heads);

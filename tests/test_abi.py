@@ -468,12 +468,12 @@ def test_head_tile_choice(lib):
 def test_piece_cost_choice(lib):
     """The split's charge per segment: the caller's value when positive,
     none when negative; otherwise 2 tiles up to 8 rows, 4 with int4 head
-    tiles, 8 with 16 or 32 rows on the MMA dataflow, 2 (128-token) tiles on
+    tiles, 8 with 16 or 32 rows on the MMA dataflow, 3 (128-token) tiles on
     the tcgen05 one.  Never on the segment-aligned split nor when blocks get
     a tile each; a charge above 4096 is rejected."""
     lens = np.concatenate([[0], np.cumsum([3000, 100, 9000, 40] * 16)])
     B = len(lens) - 1
-    cases = [(dict(), 2), (dict(q_len=2), 2), (dict(qo_heads=32), 2), (dict(q_len=4), 2),
+    cases = [(dict(), 2), (dict(q_len=2), 2), (dict(qo_heads=32), 3), (dict(q_len=4), 3),
              (dict(qo_heads=32, path=2), 8), (dict(q_len=4, path=2), 8),
              (dict(qo_heads=16, kv_heads=4, kv_dtype=2), 4), (dict(piece_cost=5), 5),
              (dict(piece_cost=-1), 0), (dict(q_len=4, piece_cost=-7), 0),
