@@ -289,6 +289,19 @@ __host__ __device__ constexpr uint64_t smem_desc(uint32_t addr, uint32_t lbo, ui
          (static_cast<uint64_t>(layout & 7u) << 61);
 }
 constexpr uint32_t kSwizzle128 = 2, kSwizzle64 = 4, kSwizzle32 = 6;
+// The two halves of the same descriptor.  The start address sits in the low
+// 14 bits of the low word as addr / 16, so for shared addresses below 256 KB
+// the descriptor of addr + d (d a multiple of 16) is the low word plus d / 16:
+// an issue loop steps through a tile with one add per product.
+__host__ __device__ constexpr uint32_t smem_desc_lo(uint32_t addr, uint32_t lbo) {
+  return ((addr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+__host__ __device__ constexpr uint32_t smem_desc_hi(uint32_t sbo, uint32_t layout) {
+  return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | ((layout & 7u) << 29);
+}
+__device__ __forceinline__ uint64_t desc_of(uint32_t lo, uint32_t hi) {
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
 
 // Instruction descriptor of kind::f16 with bf16 A and B, fp32 D, M x N;
 // a_mn / b_mn: the operand is MN-major (else K-major).

@@ -414,19 +414,21 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
             break;
           }
           tc::fence_after_sync();
-          const uint32_t vt = vring + vsl * C::TILE_BYTES;
           const uint32_t d = tO + (j & 1) * N;
+          // V^T: dims as M (64-dim atoms one plane = 1024 bytes apart),
+          // tokens as K (8-token groups GROUP_BYTES apart); P^T: rows as N
+          // (2N bytes a token), tokens as K (8-token groups 16 N apart).
+          // Descriptors of step k: the first one plus the step's offset / 16.
+          const uint32_t a_lo = tc::smem_desc_lo(vring + vsl * C::TILE_BYTES, 1024);
+          const uint32_t b_lo = tc::smem_desc_lo(p_buf + (j & 1) * 2 * C::P_BYTES, T * 2 * N);
+          constexpr uint32_t a_hi = tc::smem_desc_hi(C::GROUP_BYTES, tc::kSwizzle128);
+          constexpr uint32_t b_hi = tc::smem_desc_hi(8 * 2 * N, C::P_LAYOUT);
 #pragma unroll
           for (int part = 0; part < 2; ++part) {
-            const uint32_t pb = p_buf + (j & 1) * 2 * C::P_BYTES + part * C::P_BYTES;
 #pragma unroll
             for (int k = 0; k < T / 16; ++k) {
-              // V^T: dims as M (64-dim atoms one plane = 1024 bytes apart),
-              // tokens as K (8-token groups GROUP_BYTES apart); P^T: rows as N
-              // (2N bytes a token), tokens as K (8-token groups 16 N apart)
-              const uint64_t ad = tc::smem_desc(vt + k * 2 * C::GROUP_BYTES, 1024, C::GROUP_BYTES,
-                                                tc::kSwizzle128);
-              const uint64_t bd = tc::smem_desc(pb + k * 16 * 2 * N, T * 2 * N, 8 * 2 * N, C::P_LAYOUT);
+              const uint64_t ad = tc::desc_of(a_lo + k * (2 * C::GROUP_BYTES / 16), a_hi);
+              const uint64_t bd = tc::desc_of(b_lo + part * (C::P_BYTES / 16) + k * (16 * 2 * N / 16), b_hi);
               tc::mma_bf16_ss(d, ad, bd, kIdescO, part > 0 || k > 0);
             }
           }
@@ -467,14 +469,16 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
           // scores S^T[i % 2] = K_i . Q^T: tokens as M (8-token groups
           // GROUP_BYTES apart), query rows as N (8-row groups 1024 bytes
           // apart); a k-step of 16 dims is 32 bytes into a 128-byte plane
-          const uint32_t kt = kring + ksl * C::TILE_BYTES;
-          const uint32_t qt = qslots + qs * C::QSLOT_BYTES;
+          const uint32_t a_lo = tc::smem_desc_lo(kring + ksl * C::TILE_BYTES, 16);
+          const uint32_t b_lo = tc::smem_desc_lo(qslots + qs * C::QSLOT_BYTES, 16);
+          constexpr uint32_t a_hi = tc::smem_desc_hi(C::GROUP_BYTES, tc::kSwizzle128);
+          constexpr uint32_t b_hi = tc::smem_desc_hi(1024, tc::kSwizzle128);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 1024 + (kk & 3) * 32;
             const uint32_t qoff = (kk >> 2) * (N * 128) + (kk & 3) * 32;
-            const uint64_t ad = tc::smem_desc(kt + off, 16, C::GROUP_BYTES, tc::kSwizzle128);
-            const uint64_t bd = tc::smem_desc(qt + qoff, 16, 1024, tc::kSwizzle128);
+            const uint64_t ad = tc::desc_of(a_lo + off / 16, a_hi);
+            const uint64_t bd = tc::desc_of(b_lo + qoff / 16, b_hi);
             tc::mma_bf16_ss(tS + (i & 1) * N, ad, bd, kIdescS, kk > 0);
           }
           tc::commit(sfull0 + 8 * (i & 1));
