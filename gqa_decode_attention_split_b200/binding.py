@@ -101,6 +101,8 @@ def load_library():
     lib.fa_decode_status.restype = ctypes.c_int
     lib.fa_decode_status_static.argtypes = [ctypes.POINTER(ctypes.c_uint32), vp]
     lib.fa_decode_status_static.restype = ctypes.c_int
+    lib.fa_selftest_wait.argtypes = [vp, sz, i64, i32, vp]
+    lib.fa_selftest_wait.restype = ctypes.c_int
     lib.fa_merge_states.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp]
     lib.fa_merge_states.restype = ctypes.c_int
     lib.fa_status_string.argtypes = [ctypes.c_int]
@@ -259,6 +261,16 @@ def decode_status(workspace, stream=None) -> int:
     if st not in (FA_OK, 6):
         _check(st, "fa_decode_status")
     return int(flags.value)
+
+
+def selftest_wait(workspace, limit_ns: int, arrive: bool, stream=None) -> None:
+    """fa_selftest_wait: one bounded wait on the device, ended by an arrival
+    (arrive=True) or by its time limit, which it then records in the
+    workspace header as a pipeline wait that gave up."""
+    lib = load_library()
+    _check(lib.fa_selftest_wait(_ptr(workspace), int(workspace.numel() * workspace.element_size()),
+                                int(limit_ns), 1 if arrive else 0, _stream_handle(stream)),
+           "fa_selftest_wait")
 
 
 def decode_status_static(stream=None) -> int:

@@ -740,6 +740,40 @@ extern "C" fa_status fa_decode_status(void* workspace, size_t workspace_bytes, u
   return FA_OK;
 }
 
+// ------------------------------------------------------- bounded-wait test
+namespace {
+
+// One thread waits on a fresh mbarrier with the kernels' bounded wait.  With
+// `arrive` the thread arrives first, so the wait succeeds at once; without
+// it nothing ever arrives, the wait gives up after limit_ns and records the
+// timeout (site kSelftestSite, block 0, warp 0) as a pipeline wait would.
+constexpr uint32_t kSelftestSite = 99;
+
+__global__ void fa_wait_selftest_kernel(uint32_t* status, unsigned long long limit_ns, int arrive) {
+  __shared__ alignas(8) unsigned long long bar;
+  const uint32_t b = fa::smem_addr(&bar);
+  if (threadIdx.x == 0) {
+    fa::mbar_init(b, 1);
+    fa::fence_mbar_init();
+    if (arrive) fa::mbar_arrive(b);
+    if (!fa::mbar_wait(b, 0, limit_ns)) fa::record_timeout(status, kSelftestSite, 0, 0, 0, b);
+  }
+}
+
+}  // namespace
+
+extern "C" fa_status fa_selftest_wait(void* workspace, size_t workspace_bytes, int64_t limit_ns,
+                                      int32_t arrive, void* stream) {
+  if (workspace == nullptr || workspace_bytes < 256 || limit_ns < 1 || limit_ns > 1000000000LL)
+    return FA_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256)) return FA_ERR_MISALIGNED;
+  fa_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint32_t*>(workspace), static_cast<unsigned long long>(limit_ns), arrive ? 1 : 0);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_failure("fa_selftest_wait: launch", e);
+  return FA_OK;
+}
+
 // ------------------------------------------------------------ merge states
 namespace {
 

@@ -736,11 +736,11 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
       int hd = r0 % GK;
       const size_t row0 = (static_cast<size_t>(pc.b) * Q + r0 / GK) * a.qo_heads +
                           static_cast<size_t>(pc.h) * GK + hd;
-      uint16_t* po = a.out + row0 * D + tok;
-      const int jump = (a.qo_heads - GK) * D;  // last head of a token -> first of the next
+      size_t po = row0 * D + tok;  // element of out for row r0 + r
+      const size_t jump = static_cast<size_t>(a.qo_heads - GK) * D;  // last head of a token -> first of the next
 #pragma unroll
       for (int r = 0; r < NH; ++r) {
-        if (r < nrows) *po = bf16_bits(val[r]);
+        if (r < nrows) a.out[po] = bf16_bits(val[r]);
         po += D;
         if (++hd == GK) {
           hd = 0;

@@ -385,6 +385,22 @@ FA_API fa_status fa_decode_status(void* workspace, size_t workspace_bytes, uint3
                            void* stream);
 
 /*
+ * fa_selftest_wait -- a check of the failure path, not part of a pass.
+ * Enqueues on `stream` a one-thread kernel that waits on an mbarrier with
+ * the same bounded wait every pipeline wait of the decode kernels uses.
+ * With arrive != 0 the thread arrives first and the wait succeeds at once;
+ * with arrive == 0 nothing arrives, so the wait gives up after limit_ns
+ * (1 .. 10^9 ns) and records itself as a pipeline wait that timed out:
+ * FA_DEVICE_TIMEOUT in the check word of `workspace` and the wait's record
+ * (site 99, block 0, warp 0) in its header, which fa_decode_status then
+ * reports and clears.  The GPU context stays usable.  workspace: >= 256
+ * bytes, 256-byte aligned, its header zero-filled.  Returns
+ * FA_ERR_INVALID_ARG, FA_ERR_MISALIGNED, FA_ERR_CUDA (launch) or FA_OK.
+ */
+FA_API fa_status fa_selftest_wait(void* workspace, size_t workspace_bytes, int64_t limit_ns,
+                                  int32_t arrive, void* stream);
+
+/*
  * fa_merge_states -- exact merge of n partial attention states per
  * (row, head) ("FlashDecoding++" explainer, partial softmax per tile combined
  * afterwards; "Flashlight", section "Method": exp(x - y) = exp(x) / exp(y)

@@ -40,6 +40,17 @@ def test_library_exports_every_declared_symbol(lib):
     assert lib.fa_version() >= 100
 
 
+def test_selftest_wait_checks_its_arguments(lib):
+    """fa_selftest_wait rejects a missing or short workspace, a limit outside
+    1 ns .. 1 s and a misaligned workspace before it launches anything."""
+    vp = ctypes.c_void_p
+    assert lib.fa_selftest_wait(None, 256, 1000, 0, None) == 1
+    assert lib.fa_selftest_wait(vp(0x1000), 255, 1000, 0, None) == 1
+    assert lib.fa_selftest_wait(vp(0x1000), 256, 0, 0, None) == 1
+    assert lib.fa_selftest_wait(vp(0x1000), 256, 1_000_000_001, 0, None) == 1
+    assert lib.fa_selftest_wait(vp(0x1010), 256, 1000, 0, None) == 4  # FA_ERR_MISALIGNED
+
+
 def test_status_strings(lib):
     for code in range(7):
         s = lib.fa_status_string(code)

@@ -259,6 +259,34 @@ def test_status_word_is_reported_and_cleared():
     assert binding.decode_status(ws) == 0
 
 
+def test_bounded_wait_gives_up_and_is_reported():
+    """The failure path on the device: a wait that nothing ends gives up after
+    its limit (the kernels' own bounded wait, 50 ms here), records itself in
+    the workspace header as a pipeline wait that timed out, and
+    fa_decode_status reports and clears it; the context stays usable.  No
+    fault is provoked: the wait is bounded by the global timer."""
+    import time
+    import torch
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    binding.selftest_wait(ws, 50_000_000, arrive=True)  # ended by an arrival
+    assert binding.decode_status(ws) == 0
+    t0 = time.perf_counter()
+    binding.selftest_wait(ws, 50_000_000, arrive=False)
+    torch.cuda.synchronize()
+    waited = time.perf_counter() - t0
+    hdr = ws[:64].view(torch.int32).cpu().numpy()
+    assert hdr[0] == 2 and hdr[8] == 99 and hdr[9] == 0 and hdr[10] == 0  # FA_DEVICE_TIMEOUT, site, block, warp
+    assert waited >= 0.045, waited
+    assert binding.decode_status(ws) == 2
+    assert int(ws.sum()) == 0 and binding.decode_status(ws) == 0
+    # a pass after it computes the right result
+    x = synth.generate(2, 8, 2, 128, [500, 70], seed=29)
+    out, lse, flags, _ = run_gpu(x)
+    ref_out, ref_lse = oracle.decode_all(x)
+    assert flags == 0
+    assert_matches(out, lse, ref_out, ref_lse, what="after a timed-out wait")
+
+
 def test_lse_optional_and_workspace_reuse():
     x = synth.generate(2, 8, 2, 128, [700, 900], seed=26)
     dev = DeviceInputs(x)
