@@ -430,9 +430,10 @@ FA_API const char* fa_last_error(void);
 /* Library version, major * 10000 + minor * 100 + patch.  The structures of
  * this header are those of FA_VERSION (0.2.0 added fa_decode_desc.piece_cost
  * and fa_plan_info_t.piece_cost; 0.3.0 added FA_PATH_TC and
- * fa_plan_info_t.launches); a caller built against it should check that
+ * fa_plan_info_t.launches; 0.3.1 added fa_selftest_wait, no structure
+ * changed); a caller built against it should check that
  * fa_version() / 100 == FA_VERSION / 100. */
-#define FA_VERSION 300
+#define FA_VERSION 301
 FA_API int32_t fa_version(void);
 
 #ifdef __cplusplus
