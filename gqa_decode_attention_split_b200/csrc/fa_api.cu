@@ -272,7 +272,9 @@ extern "C" fa_status fa_decode_plan(const fa_decode_desc* desc, const int32_t* k
   // the tcgen05 dataflow: bf16 K/V, head_dim 128, 9 to 32 rows, copies of
   // 8 tokens (pages of at least 8), the plain running max
   auto tc_entry = [&]() -> const KernelEntry* {
-    if (desc->unified_max || group <= 8 || (pages != 0 && pages < 8)) return nullptr;
+    // 9-32 rows by default; fewer (padded to 16) only when asked for
+    if (desc->unified_max || (group <= 8 && desc->path != FA_PATH_TC) || (pages != 0 && pages < 8))
+      return nullptr;
     const KernelEntry* e = find_entry(desc->head_dim, group, kind, fa::kPathTc, pages);
     // its rings leave room for the schedule arrays of a few hundred requests
     if (e != nullptr && e->smem_bytes(desc->batch, group) > 232448) return nullptr;

@@ -78,10 +78,11 @@ typedef enum { FA_KV_BF16 = 0, FA_KV_FP8_E4M3 = 1, FA_KV_INT4 = 2 } fa_kv_dtype;
  * two products on the 5th-generation tensor cores (tcgen05, accumulators in
  * tensor memory) with 128-token tiles as the large dimension; it covers bf16
  * K/V with head_dim 128, 9 to 32 rows per segment (query heads per kv head
- * times query tokens), contiguous K/V or pages of at least 8 tokens, and the
- * plain running max (not unified_max).  AUTO lets the planner choose from the
- * shape (see fa_plan_info): TC where it applies, else MMA, else SIMT, unless
- * the measured table (fa_set_tuning) says otherwise. */
+ * times query tokens; 1 to 8 rows too when TC is asked for, padded to 16,
+ * where MMA measured faster), contiguous K/V or pages of at least 8 tokens,
+ * and the plain running max (not unified_max).  AUTO lets the planner choose
+ * from the shape (see fa_plan_info): TC where it applies, else MMA, else
+ * SIMT, unless the measured table (fa_set_tuning) says otherwise. */
 typedef enum { FA_PATH_AUTO = 0, FA_PATH_SIMT = 1, FA_PATH_MMA = 2, FA_PATH_TC = 3 } fa_path;
 
 /* Device-side check bits, reported by fa_decode_status. */

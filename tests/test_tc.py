@@ -72,6 +72,32 @@ def test_tc_matches_the_oracle(case):
     assert info["path"] == binding.PATH_TC and flags == 0
 
 
+SMALL_ROWS = [
+    # (batch, qo, kv, lens, kw): 1 to 8 rows, padded to 16 on this dataflow
+    (3, 8, 2, [700, 129, 1], {}),
+    (2, 8, 2, [500, 70], {"q_len": 2, "paged": True, "page_size": 16}),
+    (2, 4, 4, [900, 33], {"q_len": 8}),
+    (2, 16, 2, [300, 2000], {"window": 200}),
+    (2, 2, 2, [129, 64], {"logit_cap": 10.0}),
+]
+
+
+@pytest.mark.parametrize("case", SMALL_ROWS, ids=["gqa4", "gqa4_q2_paged", "mha_q8", "gqa8_win",
+                                                  "mha_cap"])
+def test_tc_asked_for_eight_rows_or_fewer(case):
+    """Asked for, the dataflow also takes 1 to 8 rows (padded to 16, the
+    padding rows' results discarded); the planner does not choose it there
+    (the warp-level products measured faster)."""
+    B, Hq, Hk, lens, kw = case
+    x = synth.generate(B, Hq, Hk, 128, lens, seed=51,
+                       unused_slot_fill="nan" if kw.get("paged") else None, **kw)
+    ref = oracle.decode_all(x)
+    _check(x, ref=ref)
+    _check(x, num_ctas=7, ref=ref)
+    _, _, _, info = run_gpu(x)
+    assert info["path"] != binding.PATH_TC
+
+
 @pytest.mark.parametrize("q_len", [3, 4, 8])
 def test_tc_forced_splits_agree(q_len):
     """Splitting over more blocks, then merging, gives the oracle's result at
