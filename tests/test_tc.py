@@ -154,3 +154,37 @@ def test_tc_bad_page_is_flagged_not_read():
                                 "kv_indptr": x.kv_indptr[:2], "page_table": x.page_table[:1]})
     ro, rl = oracle.decode_all(one)
     assert_matches(out[:1], lse[:1], ro, rl, what="unaffected request")
+
+
+def _random_tc_cases(n, seed):
+    rng = np.random.default_rng(seed)
+    cases = []
+    while len(cases) < n:
+        kv = int(rng.choice([1, 2, 4]))
+        q_len = int(rng.choice([1, 2, 3, 4, 8]))
+        group = int(rng.choice([1, 2, 3, 4, 5, 8, 16]))
+        if group * q_len > 32:
+            continue
+        batch = int(rng.integers(1, 6))
+        lens = [int(v) for v in rng.integers(0, 1500, size=batch)]
+        kw = {"q_len": q_len}
+        if rng.random() < 0.5:
+            kw.update(paged=True, page_size=int(rng.choice([8, 16, 32, 64, 128, 256])),
+                      unused_slot_fill="nan")
+        if rng.random() < 0.3:
+            kw["window"] = int(rng.integers(1, 600))
+        if rng.random() < 0.2:
+            kw.update(logit_cap=float(rng.uniform(2, 50)), sm_scale=0.3)
+        ctas = int(rng.choice([0, 0, 1, 3, 17]))
+        cases.append((len(cases), batch, group * kv, kv, lens, kw, ctas))
+    return cases
+
+
+@pytest.mark.parametrize("case", _random_tc_cases(40, 2027), ids=lambda c: f"r{c[0]}")
+def test_tc_random_shapes_match_the_oracle(case):
+    """Seeded random decodes on this dataflow over its options' cross
+    product (1-32 rows, query tokens, paging, window, soft-cap, forced
+    split), each against the oracle."""
+    idx, B, Hq, Hk, lens, kw, ctas = case
+    x = synth.generate(B, Hq, Hk, 128, lens, seed=3000 + idx, name=f"tc_random{idx}", **kw)
+    _check(x, num_ctas=ctas, what=f"random{idx} {kw}")
