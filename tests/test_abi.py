@@ -538,6 +538,36 @@ def test_plan_batch_limit(lib):
         lib.fa_plan_destroy(h)
 
 
+@pytest.mark.parametrize("q_len", [4, 8])
+def test_tc_batch_limit(lib, q_len):
+    """The tcgen05 dataflow keeps the schedule arrays next to its rings: it is
+    chosen up to the largest batch whose block fits 227 KB of shared memory
+    (at least 682 requests), and beyond it the plan is refused as
+    unsupported, by both tensor-core dataflows alike (never a launch that
+    cannot fit)."""
+    def plan(batch, **kw):
+        lens = np.concatenate([[0], np.cumsum(np.full(batch, 300))])
+        return _plan(lib, _desc(batch=batch, q_len=q_len, paged=1, page_size=16, **kw), lens)
+    lo, hi = 10, 20000
+    while hi - lo > 1:  # the largest batch the tcgen05 dataflow takes
+        mid = (lo + hi) // 2
+        st, h, _ = plan(mid, path=binding.PATH_TC)
+        if st == 0:
+            lib.fa_plan_destroy(h)
+            lo = mid
+        else:
+            assert st == 2 and not h.value
+            hi = mid
+    assert lo >= 682
+    st, h, _ = plan(lo)
+    inf = _info(lib, h)
+    assert st == 0 and inf.path == binding.PATH_TC and inf.smem_bytes <= 232448
+    lib.fa_plan_destroy(h)
+    for kw in (dict(), dict(path=binding.PATH_MMA), dict(path=binding.PATH_TC)):
+        st, h, _ = plan(lo + 2, **kw)
+        assert st == 2 and not h.value, kw
+
+
 def test_tiles_fit_the_pages(lib):
     """A paged tile is one page per box or a slice of one page, so tile and
     page lengths must divide one another: 32 rows take 48-token tiles with
