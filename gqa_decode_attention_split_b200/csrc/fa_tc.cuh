@@ -565,7 +565,8 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
   };
 
   bool stop = false;
-  while (!stop && next_piece(its, pc, s_pre, s_len, B, H, a.window_u, T)) {
+  bool have = next_piece(its, pc, s_pre, s_len, B, H, a.window_u, T);
+  while (!stop && have) {
     const int L = s_len[pc.b];
     const int lo = (WU > 0 && L > WU) ? L - WU : 0;  // keys some row sees: [lo, L)
 #pragma unroll
@@ -699,7 +700,11 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
       pending = i;
     }
     if (stop) break;
-    // ---- piece end: the last tile's output, the row sums, the results
+    // ---- piece end: the next piece's schedule (looked up while the last
+    // tile's output product runs), the last tile's output, the row sums,
+    // the results
+    Piece pn;
+    const bool have_next = next_piece(its, pn, s_pre, s_len, B, H, a.window_u, T);
     if (pending >= 0) take_o(pending);
     pending = -1;
     __syncwarp();
@@ -759,6 +764,8 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
         if (r < nrows) po[r * D] = val[r];
       if (tok < nrows) a.part_lse[static_cast<size_t>(slot_idx) * G + r0 + tok] = my_lse;
     }
+    pc = pn;
+    have = have_next;
   }
   tc::fence_before_sync();
   named_barrier_sync(2, 64 + SGT);
