@@ -727,14 +727,14 @@ __global__ void __launch_bounds__(TcCfg<NR>::THREADS, 1)
     // instructions are cold, and each cache line of them fetched while the
     // copies saturate memory stalls the whole group.
     float val[NH];
-    float my_lse = -CUDART_INF_F;  // row r0 + tok (tok < NH)
+    float my_l = 0.f, my_m = 0.f;  // row r0 + tok's sum and max (tok < NH): its lse
 #pragma unroll
     for (int r = 0; r < NH; ++r) {
-      const bool empty = !(lsum[r] > 0.f);
-      val[r] = empty ? 0.f : acc[r] * rcp_approx(lsum[r]);
-      const float lv = empty ? -CUDART_INF_F : (m[r] + __log2f(lsum[r])) * kLn2;
-      my_lse = tok == r ? lv : my_lse;
+      val[r] = lsum[r] > 0.f ? acc[r] * rcp_approx(lsum[r]) : 0.f;
+      my_l = tok == r ? lsum[r] : my_l;
+      my_m = tok == r ? m[r] : my_m;
     }
+    const float my_lse = my_l > 0.f ? (my_m + __log2f(my_l)) * kLn2 : -CUDART_INF_F;
     const int nrows = G - r0 < NH ? G - r0 : NH;  // rows of this half that exist
     if (whole) {
       // segment row rr is query token rr / GK, head rr % GK of the group
