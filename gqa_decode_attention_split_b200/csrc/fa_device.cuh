@@ -278,21 +278,15 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Shared-memory matrix descriptor: start address, leading- and stride-
-// dimension byte offsets (16-byte units), descriptor version 1 and the
-// swizzle layout (2: 128-byte, 4: 64-byte, 6: 32-byte swizzle).
-__host__ __device__ constexpr uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
-                                                 uint32_t layout) {
-  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) |
-         (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
-         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) |
-         (static_cast<uint64_t>(layout & 7u) << 61);
-}
+// Shared-memory matrix descriptor, as two 32-bit halves: the low word holds
+// the start address and the leading-dimension byte offset, the high word the
+// stride-dimension byte offset, descriptor version 1 and the swizzle layout
+// (2: 128-byte, 4: 64-byte, 6: 32-byte swizzle), all offsets in 16-byte
+// units.  The start address sits in the low 14 bits as addr / 16, so for
+// shared addresses below 256 KB the descriptor of addr + d (d a multiple of
+// 16) is the low word plus d / 16: an issue loop steps through a tile with
+// one add per product.
 constexpr uint32_t kSwizzle128 = 2, kSwizzle64 = 4, kSwizzle32 = 6;
-// The two halves of the same descriptor.  The start address sits in the low
-// 14 bits of the low word as addr / 16, so for shared addresses below 256 KB
-// the descriptor of addr + d (d a multiple of 16) is the low word plus d / 16:
-// an issue loop steps through a tile with one add per product.
 __host__ __device__ constexpr uint32_t smem_desc_lo(uint32_t addr, uint32_t lbo) {
   return ((addr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
 }
